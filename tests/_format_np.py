@@ -1,0 +1,68 @@
+"""Independent numpy decoder of the slot bit layout (test helper).
+
+Written from the layout description (blocks of 128 inputs, 4 units of 32
+codes, pair (even, odd) in the low/high 16-bit halves of a word), in a
+vectorised style unrelated to the oracle's per-bit C loop, so that an index
+mistake in either one shows up as a mismatch.
+"""
+import numpy as np
+
+
+def ceil128(k):
+    return (k + 127) // 128 * 128
+
+
+def _bit_positions(K, b):
+    """For every input k < Kp and code bit j: (word index in row, bit in word)."""
+    Kp = ceil128(K)
+    k = np.arange(Kp)
+    blk, kk = k // 128, k % 128
+    s, r16 = kk // 16, kk % 16
+    h = r16 // 8
+    p = (r16 % 8) // 2
+    odd = k & 1
+    i = 2 * s + h
+    unit = 4 * blk + p
+    W = np.zeros((Kp, b), np.int64)
+    B = np.zeros((Kp, b), np.int64)
+    for j in range(b):
+        if b == 4:
+            wi, bi = i // 4, 4 * (i % 4) + j
+        elif b == 3:
+            wi = np.where(i < 15, i // 5, j)
+            bi = np.where(i < 15, 3 * (i % 5) + j, 15)
+        elif b == 6:
+            m = i - 12
+            if j < 4:
+                wi = np.where(i < 12, i // 2, m)
+                bi = np.where(i < 12, 6 * (i % 2) + j, 12 + j)
+            else:
+                wi = np.where(i < 12, i // 2, 4 + m // 2)
+                bi = np.where(i < 12, 6 * (i % 2) + j, 12 + 2 * (m % 2) + (j - 4))
+        else:
+            raise ValueError(b)
+        W[:, j] = unit * b + wi
+        B[:, j] = bi + 16 * odd
+    return W, B
+
+
+def decode_rows(q, K, b):
+    """q uint8 [rows, Kp*b/8] -> codes int64 [rows, K]."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    words = q.view("<u4").astype(np.int64)
+    W, B = _bit_positions(K, b)
+    codes = np.zeros((q.shape[0], W.shape[0]), np.int64)
+    for j in range(b):
+        codes |= ((words[:, W[:, j]] >> B[:, j]) & 1) << j
+    return codes[:, :K]
+
+
+def dequant_rows(q, sb, K, g, b):
+    """Closed form of fma(scale, q, bias) in fp32: the exact product-sum in
+    float64 (exact for bf16 scale/bias and q < 64), rounded once to fp32."""
+    codes = decode_rows(q, K, b).astype(np.float64)
+    sb = np.ascontiguousarray(sb, dtype=np.uint32)
+    s = ((sb & 0xFFFF).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    bb = ((sb >> 16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    gi = np.arange(K) // g
+    return (s[:, gi] * codes + bb[:, gi]).astype(np.float32)
