@@ -1,0 +1,257 @@
+/*
+ * moe.h -- C ABI of libmoe: the routed-expert FFN run out of a bounded,
+ * slot-indexed device expert cache, for NVIDIA B200 (sm_100a).
+ *
+ * The path, in five stages, follows web pages on streaming MoE experts:
+ *   1. moe_route        router softmax -> top-k -> renormalise, with optional
+ *                       cache-aware substitution (BigMoeOnEdge, commit note on
+ *                       cache-aware substitution)
+ *   2. moe_sort         tokens grouped by expert; prefill runs at most 64
+ *                       experts per pass (transformers PR #50717 "POC:
+ *                       Experts offload" notes; RFC "stream MoE experts from
+ *                       disk in from_pretrained", section "How the prototype
+ *                       works", item "Prefill")
+ *   3. moe_slot_lookup  per-layer expert -> slot table over one preallocated
+ *                       pool, with a miss list (RFC, "How the prototype
+ *                       works", items "Cache" and "Reads")
+ *      moe_install_slots  one host-to-device copy per missed expert from
+ *                       pinned host rows (RFC, items "Reads" and "Host tier")
+ *   4+5. moe_expert_ffn fused group-wise affine dequant (w = scale*q + bias)
+ *                       feeding the SwiGLU gate/up/down projections straight
+ *                       from the slot pool (RFC: quantized experts through
+ *                       gather_qmm on the pool; experts "gated, concatenated,
+ *                       untransposed, no bias"), then the weighted combine of
+ *                       the k expert outputs per token.
+ *   Size classes: layers whose experts need the same bytes share one pool
+ *   with its own slots (1bit-MONSTER engine PR #137 "expert slots in size
+ *   classes"); the host side of that is the moe_cache_* functions.
+ *
+ * Conventions for every call:
+ *   - Device pointers are raw CUDA device addresses; "host" pointers are
+ *     ordinary (or pinned, where stated) host memory.  bf16 tensors are passed
+ *     as uint16_t bit patterns.  All arrays are dense, row-major.
+ *   - The library allocates no device memory and keeps no state between
+ *     calls (the host slot cache object is the one exception, and it lives in
+ *     host memory).  The caller owns every buffer, stream and event.
+ *   - Every device call is asynchronous on the given stream and does not
+ *     synchronise with the host.
+ *   - Argument errors are found before anything is launched and return
+ *     MOE_ERR_INVALID or MOE_ERR_UNSUPPORTED; launch failures return
+ *     MOE_ERR_CUDA.  Data errors found on the device (a slot id of -1 or past
+ *     the pool reaching the FFN, a wait that ran out) are OR-ed into the
+ *     caller's int32 *dev_err word (MOE_DEV_ERR_* bits); the offending work
+ *     item is skipped, nothing traps.  The caller reads dev_err after its
+ *     next synchronisation.
+ *
+ * Slot format (one expert = one slot; the pages name "MLX's affine format,
+ * one contiguous row per expert" but give no bit layout -- this one is
+ * chosen so that the GPU unpacks two codes per logic operation):
+ *   A weight row of K inputs is padded to Kp = K rounded up to 128 (padded
+ *   groups have scale = bias = 0).  Each block of 128 inputs is 4 units of 32
+ *   codes; unit p holds, for s = 0..7, the input pairs (128B+16s+2p, +1) and
+ *   (128B+16s+2p+8, +1) as pair indices 2s and 2s+1, the even input in the
+ *   low 16-bit half of a 32-bit word and the odd input at the same offset in
+ *   the high half.  A unit is b little-endian words:
+ *     b=4: pair i in word i/4, bits 4*(i%4)..+3
+ *     b=3: pair i<15 in word i/5, bits 3*(i%5)..+2; pair 15: bit j of the
+ *          code is bit 15 of word j
+ *     b=6: pair i<12 in word i/2, bits 6*(i%2)..+5; pair 12+m: code bits 0..3
+ *          at bits 12..15 of word m, bits 4..5 at bits 12+2*(m%2)+{0,1} of
+ *          word 4+m/2
+ *   Per group of g inputs, one 32-bit word: bf16 scale (low half), bf16 bias
+ *   (high half).  A slot is four sections, each 256-byte aligned:
+ *     q_gate_up [2I rows][Kp(H)*b_gu/8]   rows 0..I-1 gate, I..2I-1 up
+ *     q_down    [H rows][Kp(I)*b_d/8]
+ *     sb_gate_up[2I rows][Kp(H)/g] words
+ *     sb_down   [H rows][Kp(I)/g] words
+ *   slot_bytes = end of the last section rounded to 256.  Dequantised weight
+ *   = fmaf(scale, q, bias) in fp32 (one rounding).
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID = 1,      /* bad argument (null pointer, size, alignment) */
+  MOE_ERR_CUDA = 2,         /* a CUDA runtime call or launch failed */
+  MOE_ERR_UNSUPPORTED = 3,  /* valid request outside what is built (bits, group, sizes) */
+  MOE_ERR_NOT_RESIDENT = 4, /* an expert needed by the call has no slot */
+  MOE_ERR_CAPACITY = 5,     /* no free slot / buffer too small */
+  MOE_ERR_TIMEOUT = 6       /* a bounded device wait ran out */
+} moe_status;
+
+/* Bits OR-ed into the caller's device int32 *dev_err. */
+#define MOE_DEV_ERR_NOT_RESIDENT 1 /* slot id -1 reached the FFN: pair skipped */
+#define MOE_DEV_ERR_SLOT_RANGE 2   /* slot id >= n_slots: pair skipped */
+#define MOE_DEV_ERR_TIMEOUT 4      /* bounded wait on a copy barrier ran out */
+#define MOE_DEV_ERR_BAD_EXPERT 8   /* an expert id outside [0, E) */
+
+/* Shapes of one MoE layer.  Limits: 1 <= k <= E <= 1024; H and I multiples of
+ * group; group in {32, 64, 128}; bits in {3, 4, 6}. */
+typedef struct {
+  int32_t E;         /* experts in the layer */
+  int32_t k;         /* experts per token (top-k) */
+  int32_t H;         /* hidden size: input of gate/up, output of down */
+  int32_t I;         /* expert intermediate size */
+  int32_t group;     /* inputs per (scale, bias) group */
+  int32_t bits_gu;   /* code width of the gate/up projection */
+  int32_t bits_down; /* code width of the down projection */
+} moe_layer_desc;
+
+/* Byte offsets of the four slot sections and the slot size (the size-class
+ * key of 1bit-MONSTER PR #137: "the sum of its aligned read windows"). */
+typedef struct {
+  uint64_t q_gate_up, q_down, sb_gate_up, sb_down, slot_bytes;
+} moe_slot_layout_t;
+
+/* Slot byte size for d, or 0 if d is invalid. */
+size_t moe_slot_bytes(const moe_layer_desc* d);
+
+/* Section offsets for d.  Returns MOE_ERR_INVALID/UNSUPPORTED for a bad d. */
+moe_status moe_slot_layout(const moe_layer_desc* d, moe_slot_layout_t* out);
+
+/* Device workspace needed by moe_sort and moe_expert_ffn for up to
+ * max_tokens tokens (0 if d is invalid).  One buffer of this size may be
+ * shared by the two calls when they run in stream order. */
+size_t moe_workspace_bytes(const moe_layer_desc* d, int32_t max_tokens);
+
+/* Stage 1.  Cache-aware top-k (BigMoeOnEdge note: every expert already in
+ * the cache gets its score raised by L times the token's score range, then
+ * the top-k is taken again; the same number of experts runs).
+ *   logits     device fp32 [T, E], finite
+ *   L          substitution strength; 0 = plain top-k.  Meant for decode.
+ *   slot_table device int32 [E], this layer's expert -> slot (-1 = absent),
+ *              read before this step's installs; may be NULL when L == 0.
+ *   ids        device int32 [T, k], experts in rank order
+ *   w          device fp32 [T, k], u_e / sum over the chosen u (unboosted)
+ * Per token: u_e = exp(l_e - max l) with a fixed fp32 exp (range reduction by
+ * ln2 + degree-7 Taylor) so that ids match a CPU evaluation bit for bit;
+ * u'_e = u_e + L*(1 - min u) for resident e; key (u' desc, l desc, e asc).
+ * T = 0 is a no-op. */
+moe_status moe_route(const float* logits, int32_t T, const moe_layer_desc* d, float L,
+                     const int32_t* slot_table, int32_t* ids, float* w, cudaStream_t stream);
+
+/* Stage 2.  Stable counting sort of the T*k (token, rank) pairs by expert.
+ *   ids      device int32 [T, k]
+ *   x        device bf16 [T, H] or NULL; when given, x_sorted is written
+ *   offsets  device int32 [E+1]: pairs of expert e are offsets[e]..offsets[e+1]
+ *   pairs    device int32 [T*k]: flat index t*k+j, by expert then flat index
+ *   active   device int32 [E]: experts with >= 1 pair, ascending
+ *   n_active device int32 [1]
+ *   x_sorted device bf16 [T*k, H]: x_sorted[i] = x[pairs[i] / k] (if x)
+ *   ws       device workspace of ws_bytes >= moe_workspace_bytes(d, T)
+ * Prefill pass p covers active[64p .. 64p+64). */
+moe_status moe_sort(const int32_t* ids, const uint16_t* x, int32_t T, const moe_layer_desc* d,
+                    int32_t* offsets, int32_t* pairs, int32_t* active, int32_t* n_active,
+                    uint16_t* x_sorted, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Stage 3.  Slots of one pass of the active list.
+ *   slot_table device int32 [E]
+ *   active, n_active  from moe_sort (device)
+ *   pass_begin, pass_len  host ints: the pass is active[pass_begin ..
+ *              min(pass_begin+pass_len, *n_active))
+ *   n_slots    slots in the pool (ids >= n_slots are flagged in dev_err)
+ *   slots      device int32 [pass_len]: table[active[i]]
+ *   miss       device int32 [pass_len]: experts of the pass with slot -1,
+ *              ascending
+ *   n_miss     device int32 [1]
+ *   dev_err    device int32 [1] (MOE_DEV_ERR_SLOT_RANGE) or NULL */
+moe_status moe_slot_lookup(const int32_t* slot_table, const int32_t* active, const int32_t* n_active,
+                           int32_t pass_begin, int32_t pass_len, int32_t n_slots, int32_t* slots,
+                           int32_t* miss, int32_t* n_miss, int32_t* dev_err, cudaStream_t stream);
+
+/* Stage 3'.  Install n experts: cudaMemcpyAsync of slot_bytes from pinned
+ * host_rows[i] to pool + slots[i]*slot_bytes, on the side stream, then
+ * records done (if not NULL) on it.  host_rows (pinned) must not change until
+ * done has fired (RFC, "Host tier": rows stay reserved until the copy that
+ * reads them has run).  slots is a host array; each id must be < n_slots. */
+moe_status moe_install_slots(void* pool, size_t slot_bytes, int32_t n_slots, const void* const* host_rows,
+                             const int32_t* slots, int32_t n, cudaStream_t side, cudaEvent_t done);
+
+/* Stages 4 + 5 for one pass.
+ *   x          device bf16 [T, H]
+ *   pool       device base of this layer's size-class pool (slot_bytes stride)
+ *   n_slots    slots in the pool
+ *   slot_table device int32 [E]
+ *   ids, w     from moe_route; offsets, pairs, active, n_active from moe_sort
+ *   x_sorted   from moe_sort, or NULL (needed by the tensor-core prefill path
+ *              when T >= 256; else unused)
+ *   pass_begin, pass_len  which active experts this call runs
+ *   y_accum    device fp32 [T, H]; the pass's expert outputs are ADDED:
+ *              y_t += sum over the pass's pairs (t, j) of w[t,j] * o_{t,j}.
+ *              Zero it before the first pass.  Summation order is fixed
+ *              (deterministic run to run).
+ *   ws         device workspace, ws_bytes >= moe_workspace_bytes(d, T)
+ *   dev_err    device int32 [1]: MOE_DEV_ERR_NOT_RESIDENT / SLOT_RANGE /
+ *              TIMEOUT; affected experts are skipped */
+moe_status moe_expert_ffn(const uint16_t* x, int32_t T, const moe_layer_desc* d, const void* pool,
+                          int32_t n_slots, const int32_t* slot_table, const int32_t* ids, const float* w,
+                          const int32_t* offsets, const int32_t* pairs, const int32_t* active,
+                          const int32_t* n_active, const uint16_t* x_sorted, int32_t pass_begin,
+                          int32_t pass_len, float* y_accum, void* ws, size_t ws_bytes, int32_t* dev_err,
+                          cudaStream_t stream);
+
+/* Test/inspection: dequantise slot `slot` of pool through the same code
+ * extraction the FFN kernels use.  out_fp32 (device, may be NULL):
+ * gate_up [2I, H] then down [H, I], fp32 = fmaf(scale, q, bias); out_bf16
+ * (device, may be NULL): the same values rounded to bf16 (RNE). */
+moe_status moe_dequant_slot(const void* pool, int32_t slot, const moe_layer_desc* d, float* out_fp32,
+                            uint16_t* out_bf16, cudaStream_t stream);
+
+/* Input preparation (the RFC's one-time quantize_experts, on the GPU):
+ * quantise rows of fp32 weights w [rows, K] into the slot row format:
+ * per group scale = bf16((max-min)/(2^b-1)), bias = bf16(min),
+ * q = clamp(rint((w - bias)/scale), 0, 2^b-1) (q = 0 if scale = 0).
+ *   q  device [rows][Kp*bits/8] bytes;  sb device uint32 [rows][Kp/group] */
+moe_status moe_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t group, int32_t bits, uint8_t* q,
+                             uint32_t* sb, cudaStream_t stream);
+
+/* Test: the fp32 exp used by moe_route, elementwise on n device floats. */
+moe_status moe_exp_portable(const float* x, int64_t n, float* out, cudaStream_t stream);
+
+const char* moe_status_string(moe_status s);
+
+/* ------------------------------------------------------------------------
+ * Host slot cache (1bit-MONSTER PR #137: per size class, one LRU per layer,
+ * every layer keeps the same share of its experts, empty slots taken first).
+ * Host memory only.  Layer l of class c owns slots [base, base + S) of the
+ * class pool, base = (index of l among the layers of class c) * S.
+ * ---------------------------------------------------------------------- */
+typedef struct moe_cache moe_cache;
+
+/* layer_class: host int32 [n_layers] class of each layer (NULL: all 0);
+ * slots_per_layer S.  *out receives the object. */
+moe_status moe_cache_create(int32_t E, int32_t n_layers, const int32_t* layer_class, int32_t slots_per_layer,
+                            moe_cache** out);
+void moe_cache_destroy(moe_cache* c);
+/* Host expert -> slot table of a layer ([E], -1 = absent), owned by c. */
+const int32_t* moe_cache_table(const moe_cache* c, int32_t layer);
+int32_t moe_cache_layer_base(const moe_cache* c, int32_t layer);
+/* Slots in the pool of class cls (layers of the class * S). */
+int32_t moe_cache_class_slots(const moe_cache* c, int32_t cls);
+/* Initial residency: experts[i] into slot slots[i] (absolute pool ids inside
+ * the layer's range); later entries are more recent. */
+moe_status moe_cache_place(moe_cache* c, int32_t layer, const int32_t* experts, const int32_t* slots, int32_t n);
+/* One pass: pass_experts (ascending, host) are the experts the pass runs.
+ * Hits are touched in order; each miss (ascending) takes the least recently
+ * used slot of the layer not used by this pass (never-used slots first),
+ * evicting its owner.  Writes the n_out misses and their slots.  Returns
+ * MOE_ERR_CAPACITY if a miss found no slot (its out_slot is -1). */
+moe_status moe_cache_step(moe_cache* c, int32_t layer, const int32_t* pass_experts, int32_t n_pass,
+                          int32_t* out_experts, int32_t* out_slots, int32_t* n_out);
+/* Counters since creation: hits, misses, evictions (of a resident expert). */
+void moe_cache_stats(const moe_cache* c, int64_t* hits, int64_t* misses, int64_t* evictions);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

@@ -467,17 +467,26 @@ void orc_dequant_slot(const uint8_t* slot, int32_t H, int32_t I, int32_t g, int3
 void orc_expert_ffn(const uint16_t* x, int32_t H, int32_t I, int32_t g, int32_t b_gu, int32_t b_d,
                     int32_t k, const uint8_t* const* expert_slot, const int32_t* ids, const double* w,
                     const int32_t* tok, int32_t n_tok, double* y) {
+  /* Each expert's weights are dequantised once per distinct slot and reused
+   * for every (token, rank) it serves; o_{t,j} is kept per (t, j) and y_t is
+   * summed over j in rank order at the end. */
+  int64_t npair = (int64_t)n_tok * k;
   float* wgu = (float*)malloc(sizeof(float) * (size_t)2 * I * H);
   float* wd = (float*)malloc(sizeof(float) * (size_t)H * I);
   double* xd = (double*)malloc(sizeof(double) * (size_t)H);
   double* h = (double*)malloc(sizeof(double) * (size_t)I);
-  memset(y, 0, sizeof(double) * (size_t)n_tok * H);
-  for (int32_t ti = 0; ti < n_tok; ++ti) {
-    int32_t t = tok[ti];
-    for (int32_t c = 0; c < H; ++c) xd[c] = (double)orc_bf16_to_f32(x[(int64_t)t * H + c]);
-    for (int32_t j = 0; j < k; ++j) {
-      int32_t e = ids[(int64_t)t * k + j];
-      orc_dequant_slot(expert_slot[e], H, I, g, b_gu, b_d, wgu, wd);
+  double* o = (double*)malloc(sizeof(double) * (size_t)(npair > 0 ? npair : 1) * H);
+  unsigned char* done = (unsigned char*)calloc((size_t)(npair > 0 ? npair : 1), 1);
+  for (int64_t p = 0; p < npair; ++p) {
+    if (done[p]) continue;
+    int32_t tp = tok[p / k];
+    const uint8_t* slot = expert_slot[ids[(int64_t)tp * k + p % k]];
+    orc_dequant_slot(slot, H, I, g, b_gu, b_d, wgu, wd);
+    for (int64_t q = p; q < npair; ++q) {
+      int32_t t = tok[q / k];
+      if (done[q] || expert_slot[ids[(int64_t)t * k + q % k]] != slot) continue;
+      done[q] = 1;
+      for (int32_t c = 0; c < H; ++c) xd[c] = (double)orc_bf16_to_f32(x[(int64_t)t * H + c]);
       for (int32_t r = 0; r < I; ++r) {
         double a = 0.0, u = 0.0;
         for (int32_t c = 0; c < H; ++c) {
@@ -486,18 +495,27 @@ void orc_expert_ffn(const uint16_t* x, int32_t H, int32_t I, int32_t g, int32_t 
         }
         h[r] = a / (1.0 + exp(-a)) * u;
       }
-      double wj = w[(int64_t)t * k + j];
       for (int32_t r = 0; r < H; ++r) {
-        double o = 0.0;
-        for (int32_t c = 0; c < I; ++c) o += (double)wd[(int64_t)r * I + c] * h[c];
-        y[(int64_t)ti * H + r] += wj * o;
+        double acc = 0.0;
+        for (int32_t c = 0; c < I; ++c) acc += (double)wd[(int64_t)r * I + c] * h[c];
+        o[q * H + r] = acc;
       }
+    }
+  }
+  for (int32_t ti = 0; ti < n_tok; ++ti) {
+    int32_t t = tok[ti];
+    for (int32_t r = 0; r < H; ++r) {
+      double acc = 0.0;
+      for (int32_t j = 0; j < k; ++j) acc += w[(int64_t)t * k + j] * o[((int64_t)ti * k + j) * H + r];
+      y[(int64_t)ti * H + r] = acc;
     }
   }
   free(wgu);
   free(wd);
   free(xd);
   free(h);
+  free(o);
+  free(done);
 }
 
 /* ------------------------------------------------------------------ */

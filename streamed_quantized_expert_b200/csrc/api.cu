@@ -1,0 +1,215 @@
+// libmoe C ABI: argument checks, workspace carving and launches.  Every
+// entry point validates before launching anything and returns a moe_status;
+// see include/moe.h for the contract of each call.
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "moe.h"
+
+using namespace moe;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status check_desc(const moe_layer_desc* d) {
+  if (!d) return MOE_ERR_INVALID;
+  if (d->E < 1 || d->k < 1 || d->k > d->E || d->H < 1 || d->I < 1) return MOE_ERR_INVALID;
+  if (d->group != 32 && d->group != 64 && d->group != 128) return MOE_ERR_UNSUPPORTED;
+  auto bits_ok = [](int b) { return b == 3 || b == 4 || b == 6; };
+  if (!bits_ok(d->bits_gu) || !bits_ok(d->bits_down)) return MOE_ERR_UNSUPPORTED;
+  if (d->H % d->group || d->I % d->group) return MOE_ERR_INVALID;
+  if (d->E > 1024 || d->k > 32) return MOE_ERR_UNSUPPORTED;
+  if (d->H > 1 << 16 || d->I > 1 << 16) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+int device_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+struct WsCarve {
+  size_t sort, h, o, total;
+};
+
+WsCarve carve(const moe_layer_desc& d, int T) {
+  WsCarve c{};
+  const int64_t np = (int64_t)T * d.k;
+  c.sort = (size_t)round_up((int64_t)sort_ws_bytes((int)np, d.E), 256);
+  c.h = (size_t)round_up(np * d.I * 2, 256);
+  c.o = T > kFusedMaxTokens ? (size_t)round_up(np * d.H * 4, 256) : 0;
+  // sort scratch and FFN scratch are used by different calls: overlap them
+  const size_t ffn = c.h + c.o;
+  c.total = c.sort > ffn ? c.sort : ffn;
+  if (c.total == 0) c.total = 256;
+  return c;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID: return "invalid argument";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_NOT_RESIDENT: return "expert not resident";
+    case MOE_ERR_CAPACITY: return "capacity exceeded";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t moe_slot_bytes(const moe_layer_desc* d) {
+  if (check_desc(d) != MOE_OK) return 0;
+  return (size_t)make_layout(*d).slot_bytes;
+}
+
+moe_status moe_slot_layout(const moe_layer_desc* d, moe_slot_layout_t* out) {
+  moe_status s = check_desc(d);
+  if (s != MOE_OK) return s;
+  if (!out) return MOE_ERR_INVALID;
+  const Layout L = make_layout(*d);
+  out->q_gate_up = (uint64_t)L.q_gu;
+  out->q_down = (uint64_t)L.q_d;
+  out->sb_gate_up = (uint64_t)L.sb_gu;
+  out->sb_down = (uint64_t)L.sb_d;
+  out->slot_bytes = (uint64_t)L.slot_bytes;
+  return MOE_OK;
+}
+
+size_t moe_workspace_bytes(const moe_layer_desc* d, int32_t max_tokens) {
+  if (check_desc(d) != MOE_OK || max_tokens < 0) return 0;
+  return carve(*d, max_tokens).total;
+}
+
+moe_status moe_route(const float* logits, int32_t T, const moe_layer_desc* d, float L, const int32_t* slot_table,
+                     int32_t* ids, float* w, cudaStream_t stream) {
+  moe_status s = check_desc(d);
+  if (s != MOE_OK) return s;
+  if (T < 0 || !(L >= 0.0f) || L > 1e30f) return MOE_ERR_INVALID;
+  if (T == 0) return MOE_OK;
+  if (!logits || !ids || !w) return MOE_ERR_INVALID;
+  if (L > 0.0f && !slot_table) return MOE_ERR_INVALID;
+  return cuda_status(launch_route(logits, T, d->E, d->k, L, slot_table, ids, w, stream));
+}
+
+moe_status moe_sort(const int32_t* ids, const uint16_t* x, int32_t T, const moe_layer_desc* d, int32_t* offsets,
+                    int32_t* pairs, int32_t* active, int32_t* n_active, uint16_t* x_sorted, void* ws,
+                    size_t ws_bytes, cudaStream_t stream) {
+  moe_status s = check_desc(d);
+  if (s != MOE_OK) return s;
+  if (T < 0 || (int64_t)T * d->k > (1 << 24)) return MOE_ERR_INVALID;
+  if (!offsets || !active || !n_active) return MOE_ERR_INVALID;
+  if (T > 0 && (!ids || !pairs)) return MOE_ERR_INVALID;
+  if (x && (!x_sorted || !aligned(x, 16) || !aligned(x_sorted, 16) || d->H % 8)) return MOE_ERR_INVALID;
+  const WsCarve c = carve(*d, T);
+  if (c.sort > 0 && (!ws || ws_bytes < c.total)) return MOE_ERR_CAPACITY;
+  return cuda_status(launch_sort(ids, x, T, d->k, d->E, d->H, offsets, pairs, active, n_active, x_sorted, ws,
+                                 stream));
+}
+
+moe_status moe_slot_lookup(const int32_t* slot_table, const int32_t* active, const int32_t* n_active,
+                           int32_t pass_begin, int32_t pass_len, int32_t n_slots, int32_t* slots, int32_t* miss,
+                           int32_t* n_miss, int32_t* dev_err, cudaStream_t stream) {
+  if (!slot_table || !active || !n_active || !slots || !miss || !n_miss) return MOE_ERR_INVALID;
+  if (pass_begin < 0 || pass_len < 0 || n_slots < 0) return MOE_ERR_INVALID;
+  return cuda_status(launch_lookup(slot_table, active, n_active, pass_begin, pass_len, n_slots, slots, miss, n_miss,
+                                   dev_err, stream));
+}
+
+moe_status moe_install_slots(void* pool, size_t slot_bytes, int32_t n_slots, const void* const* host_rows,
+                             const int32_t* slots, int32_t n, cudaStream_t side, cudaEvent_t done) {
+  if (n < 0) return MOE_ERR_INVALID;
+  if (n > 0 && (!pool || !host_rows || !slots || slot_bytes == 0)) return MOE_ERR_INVALID;
+  for (int32_t i = 0; i < n; ++i)
+    if (slots[i] < 0 || slots[i] >= n_slots || !host_rows[i]) return MOE_ERR_INVALID;
+  for (int32_t i = 0; i < n; ++i) {
+    char* dst = static_cast<char*>(pool) + (size_t)slots[i] * slot_bytes;
+    cudaError_t e = cudaMemcpyAsync(dst, host_rows[i], slot_bytes, cudaMemcpyHostToDevice, side);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  if (done && cudaEventRecord(done, side) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_expert_ffn(const uint16_t* x, int32_t T, const moe_layer_desc* d, const void* pool, int32_t n_slots,
+                          const int32_t* slot_table, const int32_t* ids, const float* w, const int32_t* offsets,
+                          const int32_t* pairs, const int32_t* active, const int32_t* n_active,
+                          const uint16_t* x_sorted, int32_t pass_begin, int32_t pass_len, float* y_accum, void* ws,
+                          size_t ws_bytes, int32_t* dev_err, cudaStream_t stream) {
+  moe_status s = check_desc(d);
+  if (s != MOE_OK) return s;
+  if (T < 0 || pass_begin < 0 || pass_len < 0 || n_slots < 0) return MOE_ERR_INVALID;
+  if (T == 0 || pass_len == 0) return MOE_OK;
+  if (!x || !pool || !slot_table || !ids || !w || !offsets || !pairs || !active || !n_active || !y_accum)
+    return MOE_ERR_INVALID;
+  if (!aligned(pool, 256) || !aligned(x, 16) || !aligned(ws, 256)) return MOE_ERR_INVALID;
+  if ((int64_t)T * d->k > (1 << 24)) return MOE_ERR_UNSUPPORTED;
+  if (!ffn_decode_supported(*d)) return MOE_ERR_UNSUPPORTED;
+  const WsCarve c = carve(*d, T);
+  if (!ws || ws_bytes < c.total) return MOE_ERR_CAPACITY;
+  FfnArgs a{};
+  a.x = x;
+  a.T = T;
+  a.E = d->E;
+  a.k = d->k;
+  a.H = d->H;
+  a.I = d->I;
+  a.g = d->group;
+  a.pool = static_cast<const uint8_t*>(pool);
+  a.L = make_layout(*d);
+  a.slot_bytes = a.L.slot_bytes;
+  a.n_slots = n_slots;
+  a.table = slot_table;
+  a.ids = ids;
+  a.w = w;
+  a.offsets = offsets;
+  a.pairs = pairs;
+  a.active = active;
+  a.n_active = n_active;
+  a.x_sorted = x_sorted;
+  a.pass_begin = pass_begin;
+  a.pass_len = pass_len;
+  a.y = y_accum;
+  a.h = static_cast<uint16_t*>(ws);
+  a.o = c.o ? reinterpret_cast<float*>(static_cast<char*>(ws) + c.h) : nullptr;
+  a.dev_err = dev_err;
+  return cuda_status(launch_ffn_decode(a, *d, device_sms(), stream));
+}
+
+moe_status moe_dequant_slot(const void* pool, int32_t slot, const moe_layer_desc* d, float* out_fp32,
+                            uint16_t* out_bf16, cudaStream_t stream) {
+  moe_status s = check_desc(d);
+  if (s != MOE_OK) return s;
+  if (!pool || slot < 0 || (!out_fp32 && !out_bf16)) return MOE_ERR_INVALID;
+  const Layout L = make_layout(*d);
+  const uint8_t* base = static_cast<const uint8_t*>(pool) + (int64_t)slot * L.slot_bytes;
+  return cuda_status(launch_dequant_slot(base, *d, L, out_fp32, out_bf16, stream));
+}
+
+moe_status moe_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t group, int32_t bits, uint8_t* q,
+                             uint32_t* sb, cudaStream_t stream) {
+  if (rows < 0 || K < 1) return MOE_ERR_INVALID;
+  if (group != 32 && group != 64 && group != 128) return MOE_ERR_UNSUPPORTED;
+  if (bits != 3 && bits != 4 && bits != 6) return MOE_ERR_UNSUPPORTED;
+  if (K % group) return MOE_ERR_INVALID;
+  if (rows == 0) return MOE_OK;
+  if (!w || !q || !sb || !aligned(q, 4) || !aligned(sb, 4)) return MOE_ERR_INVALID;
+  return cuda_status(launch_quantize(w, rows, K, group, bits, q, sb, stream));
+}
+
+moe_status moe_exp_portable(const float* x, int64_t n, float* out, cudaStream_t stream) {
+  if (n < 0 || (n > 0 && (!x || !out))) return MOE_ERR_INVALID;
+  return cuda_status(launch_exp(x, n, out, stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,80 @@
+// Internal launcher declarations shared by the libmoe translation units.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "moe.h"
+
+namespace moe {
+
+constexpr int kFusedMaxTokens = 64;  // decode down kernel combines in shared memory up to this T
+
+struct FfnArgs {
+  const uint16_t* x;
+  int T;
+  int E, k, H, I, g;
+  const uint8_t* pool;
+  int64_t slot_bytes;
+  int n_slots;
+  const int32_t* table;
+  const int32_t* ids;
+  const float* w;
+  const int32_t* offsets;
+  const int32_t* pairs;
+  const int32_t* active;
+  const int32_t* n_active;
+  const uint16_t* x_sorted;
+  int pass_begin, pass_len;
+  float* y;
+  uint16_t* h;  // workspace: [T*k][I] bf16, by sorted position
+  float* o;     // workspace: [T*k][H] fp32, by flat pair index (T > kFusedMaxTokens)
+  int32_t* dev_err;
+  Layout L;
+  // filled by the launcher
+  int64_t q_gu, q_d, sb_gu, sb_d, rb_gu, rb_d;
+  int ng_gu, ng_d, nblk_gu, nblk_d;
+  int sr_gu, sr_d;
+  int gu_stage_bytes, d_stage_bytes, gu_nstage;
+};
+
+// Launch with programmatic stream serialization, so the kernel's CTAs can be
+// scheduled while the previous kernel in the stream drains; every kernel
+// calls griddepcontrol.wait before reading what earlier kernels wrote.
+template <typename... Args>
+inline cudaError_t launch_pdl(const void* func, int grid, int block, size_t smem, cudaStream_t st,
+                              const Args&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void* argv[] = {const_cast<void*>(static_cast<const void*>(&args))...};
+  return cudaLaunchKernelExC(&cfg, func, argv);
+}
+
+cudaError_t launch_route(const float* logits, int T, int E, int k, float L, const int32_t* table, int32_t* ids,
+                         float* w, cudaStream_t st);
+size_t sort_ws_bytes(int n, int E);
+cudaError_t launch_sort(const int32_t* ids, const uint16_t* x, int T, int k, int E, int H, int32_t* offsets,
+                        int32_t* pairs, int32_t* active, int32_t* n_active, uint16_t* x_sorted, void* ws,
+                        cudaStream_t st);
+cudaError_t launch_lookup(const int32_t* table, const int32_t* active, const int32_t* n_active, int pass_begin,
+                          int pass_len, int n_slots, int32_t* slots, int32_t* miss, int32_t* n_miss,
+                          int32_t* dev_err, cudaStream_t st);
+cudaError_t launch_exp(const float* x, int64_t n, float* out, cudaStream_t st);
+cudaError_t launch_quantize(const float* w, int rows, int K, int g, int b, uint8_t* q, uint32_t* sb,
+                            cudaStream_t st);
+cudaError_t launch_dequant_slot(const uint8_t* slot, const moe_layer_desc& d, const Layout& L, float* out32,
+                                uint16_t* out16, cudaStream_t st);
+size_t ffn_ws_bytes(const moe_layer_desc& d, int T);
+bool ffn_decode_supported(const moe_layer_desc& d);
+cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st);
+
+}  // namespace moe

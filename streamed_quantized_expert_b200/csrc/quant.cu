@@ -1,0 +1,168 @@
+// Quantization into the slot row format (input preparation: the RFC's
+// one-time quantize_experts, which writes experts in MLX's affine format) and
+// the test-only dequantisation of a slot through the FFN's code unpackers.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+// Word index (within a 128-input block) and bit of code bit j of input kk.
+__device__ __forceinline__ void block_bit(int kk, int b, int j, int& word, int& bit) {
+  const int s = kk >> 4, r16 = kk & 15;
+  const int h = r16 >> 3, p = (r16 & 7) >> 1;
+  const int i = 2 * s + h;
+  int wi, bi;
+  if (b == 4) {
+    wi = i >> 2;
+    bi = 4 * (i & 3) + j;
+  } else if (b == 3) {
+    if (i < 15) {
+      wi = i / 5;
+      bi = 3 * (i % 5) + j;
+    } else {
+      wi = j;
+      bi = 15;
+    }
+  } else {
+    if (i < 12) {
+      wi = i >> 1;
+      bi = 6 * (i & 1) + j;
+    } else if (j < 4) {
+      wi = i - 12;
+      bi = 12 + j;
+    } else {
+      wi = 4 + ((i - 12) >> 1);
+      bi = 12 + 2 * ((i - 12) & 1) + (j - 4);
+    }
+  }
+  word = p * b + wi;
+  bit = bi + ((kk & 1) ? 16 : 0);
+}
+
+// One warp per (row, 128-block); lane owns inputs 4*lane .. 4*lane+3.
+__global__ void __launch_bounds__(256) quantize_kernel(const float* __restrict__ w, int rows, int K, int g, int b,
+                                                       uint8_t* __restrict__ q, uint32_t* __restrict__ sb) {
+  __shared__ uint32_t s_words[8][24];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nblk = (int)(padded_k(K) / 128);
+  const int64_t task = (int64_t)blockIdx.x * 8 + warp;
+  if (task >= (int64_t)rows * nblk) return;
+  const int r = (int)(task / nblk), blk = (int)(task % nblk);
+  const int k0 = blk * 128 + 4 * lane;
+  float v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = (k0 + i < K) ? w[(int64_t)r * K + k0 + i] : 0.0f;
+  // group min / max over the g/4 lanes of the group
+  float mn = fminf(fminf(v[0], v[1]), fminf(v[2], v[3]));
+  float mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+  const int lanes_per_group = g / 4;
+  for (int o = 1; o < lanes_per_group; o <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const int qmax = (1 << b) - 1;
+  const bool group_padded = (blk * 128 + (lane / lanes_per_group) * g) >= K;
+  uint16_t sh = 0, bh = 0;
+  if (!group_padded) {
+    sh = f32_to_bf16_rne(__fdiv_rn(__fsub_rn(mx, mn), (float)qmax));
+    bh = f32_to_bf16_rne(mn);
+  }
+  const float sf = __uint_as_float((uint32_t)sh << 16), bf = __uint_as_float((uint32_t)bh << 16);
+  if (lane < 4 * b) s_words[warp][lane] = 0u;
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int code = 0;
+    if (!group_padded && k0 + i < K && sf != 0.0f) {
+      float t = rintf(__fdiv_rn(__fsub_rn(v[i], bf), sf));
+      t = fminf(fmaxf(t, 0.0f), (float)qmax);
+      code = (int)t;
+    }
+    for (int j = 0; j < b; ++j) {
+      if ((code >> j) & 1) {
+        int word, bit;
+        block_bit(4 * lane + i, b, j, word, bit);
+        atomicOr(&s_words[warp][word], 1u << bit);
+      }
+    }
+  }
+  __syncwarp();
+  const int64_t rb = row_bytes(K, b);
+  if (lane < 4 * b)
+    reinterpret_cast<uint32_t*>(q + (int64_t)r * rb + (int64_t)blk * 16 * b)[lane] = s_words[warp][lane];
+  if (lane % lanes_per_group == 0) {
+    const int gi = (blk * 128 + 4 * lane) / g;
+    sb[(int64_t)r * row_groups(K, g) + gi] = (uint32_t)sh | ((uint32_t)bh << 16);
+  }
+}
+
+// Dequantise rows of one projection: one thread per (row, unit), through the
+// same unpack_unit<B> the FFN kernels use.  out[r][k] = fmaf(s, q, b).
+template <int B>
+__global__ void dequant_kernel(const uint8_t* __restrict__ qbase, const uint32_t* __restrict__ sbbase, int rows,
+                               int K, int g, float* __restrict__ out32, uint16_t* __restrict__ out16) {
+  const int nunit = (int)(padded_k(K) / 32);
+  const int64_t task = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (task >= (int64_t)rows * nunit) return;
+  const int r = (int)(task / nunit), u = (int)(task % nunit);
+  const int blk = u >> 2, t = u & 3;
+  const uint32_t* wp = reinterpret_cast<const uint32_t*>(qbase + (int64_t)r * row_bytes(K, B)) + (int64_t)u * B;
+  uint32_t wv[B];
+#pragma unroll
+  for (int i = 0; i < B; ++i) wv[i] = wp[i];
+  uint32_t p[16];
+  unpack_unit<B>(wv, p);
+  const uint32_t* sbr = sbbase + (int64_t)r * row_groups(K, g);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int a = PairShift<B>::a(i);
+    const int k = blk * 128 + pair_input(i, t);
+    if (k >= K) continue;  // K is a multiple of 32, so k+1 < K too
+    const uint32_t sbw = sbr[k / g];
+    const float s = bf16_lo(sbw), bb = bf16_hi(sbw);
+    const float v0 = __fmaf_rn(s, pair_lo_q(p[i], a), bb);
+    const float v1 = __fmaf_rn(s, pair_hi_q(p[i], a), bb);
+    if (out32) {
+      out32[(int64_t)r * K + k] = v0;
+      out32[(int64_t)r * K + k + 1] = v1;
+    }
+    if (out16) {
+      out16[(int64_t)r * K + k] = f32_to_bf16_rne(v0);
+      out16[(int64_t)r * K + k + 1] = f32_to_bf16_rne(v1);
+    }
+  }
+}
+
+template <int B>
+static void launch_dq(const uint8_t* q, const uint32_t* sb, int rows, int K, int g, float* o32, uint16_t* o16,
+                      cudaStream_t st) {
+  const int64_t n = (int64_t)rows * (padded_k(K) / 32);
+  dequant_kernel<B><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(q, sb, rows, K, g, o32, o16);
+}
+
+static void dq_dispatch(int b, const uint8_t* q, const uint32_t* sb, int rows, int K, int g, float* o32,
+                        uint16_t* o16, cudaStream_t st) {
+  if (b == 3) launch_dq<3>(q, sb, rows, K, g, o32, o16, st);
+  else if (b == 4) launch_dq<4>(q, sb, rows, K, g, o32, o16, st);
+  else launch_dq<6>(q, sb, rows, K, g, o32, o16, st);
+}
+
+cudaError_t launch_dequant_slot(const uint8_t* slot, const moe_layer_desc& d, const Layout& L, float* out32,
+                                uint16_t* out16, cudaStream_t st) {
+  const int64_t n_gu = (int64_t)2 * d.I * d.H;
+  dq_dispatch(d.bits_gu, slot + L.q_gu, reinterpret_cast<const uint32_t*>(slot + L.sb_gu), 2 * d.I, d.H, d.group,
+              out32, out16, st);
+  dq_dispatch(d.bits_down, slot + L.q_d, reinterpret_cast<const uint32_t*>(slot + L.sb_d), d.H, d.I, d.group,
+              out32 ? out32 + n_gu : nullptr, out16 ? out16 + n_gu : nullptr, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const float* w, int rows, int K, int g, int b, uint8_t* q, uint32_t* sb,
+                            cudaStream_t st) {
+  const int64_t tasks = (int64_t)rows * (padded_k(K) / 128);
+  if (tasks == 0) return cudaSuccess;
+  quantize_kernel<<<(unsigned)((tasks + 7) / 8), 256, 0, st>>>(w, rows, K, g, b, q, sb);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,244 @@
+"""ctypes binding of libmoe (include/moe.h): the same names, argument
+marshalling only.  Device buffers are torch CUDA tensors (or raw device
+addresses); every step of the path runs in the library's CUDA kernels.
+
+The library is loaded from this package directory.  If it is missing the
+first call raises: there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID, MOE_ERR_CUDA, MOE_ERR_UNSUPPORTED, MOE_ERR_NOT_RESIDENT, MOE_ERR_CAPACITY, \
+    MOE_ERR_TIMEOUT = range(7)
+DEV_ERR_NOT_RESIDENT, DEV_ERR_SLOT_RANGE, DEV_ERR_TIMEOUT, DEV_ERR_BAD_EXPERT = 1, 2, 4, 8
+
+# every entry point declared in include/moe.h
+ABI_SYMBOLS = [
+    "moe_slot_bytes", "moe_slot_layout", "moe_workspace_bytes", "moe_route", "moe_sort", "moe_slot_lookup",
+    "moe_install_slots", "moe_expert_ffn", "moe_dequant_slot", "moe_quantize_rows", "moe_exp_portable",
+    "moe_status_string", "moe_cache_create", "moe_cache_destroy", "moe_cache_table", "moe_cache_layer_base",
+    "moe_cache_class_slots", "moe_cache_place", "moe_cache_step", "moe_cache_stats",
+]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class LayerDesc(C.Structure):
+    _fields_ = [("E", C.c_int32), ("k", C.c_int32), ("H", C.c_int32), ("I", C.c_int32), ("group", C.c_int32),
+                ("bits_gu", C.c_int32), ("bits_down", C.c_int32)]
+
+    def __repr__(self):
+        return (f"LayerDesc(E={self.E}, k={self.k}, H={self.H}, I={self.I}, group={self.group}, "
+                f"bits_gu={self.bits_gu}, bits_down={self.bits_down})")
+
+
+class SlotLayout(C.Structure):
+    _fields_ = [("q_gate_up", C.c_uint64), ("q_down", C.c_uint64), ("sb_gate_up", C.c_uint64),
+                ("sb_down", C.c_uint64), ("slot_bytes", C.c_uint64)]
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmoe.so not built ({LIB_PATH}); run streamed_quantized_expert_b200.build.build()")
+        L = C.CDLL(LIB_PATH)
+        P, i32, i64, f32, sz = C.c_void_p, C.c_int32, C.c_int64, C.c_float, C.c_size_t
+        D = C.POINTER(LayerDesc)
+        sig = {
+            "moe_slot_bytes": (sz, [D]),
+            "moe_slot_layout": (C.c_int, [D, C.POINTER(SlotLayout)]),
+            "moe_workspace_bytes": (sz, [D, i32]),
+            "moe_route": (C.c_int, [P, i32, D, f32, P, P, P, P]),
+            "moe_sort": (C.c_int, [P, P, i32, D, P, P, P, P, P, P, sz, P]),
+            "moe_slot_lookup": (C.c_int, [P, P, P, i32, i32, i32, P, P, P, P, P]),
+            "moe_install_slots": (C.c_int, [P, sz, i32, P, P, i32, P, P]),
+            "moe_expert_ffn": (C.c_int, [P, i32, D, P, i32, P, P, P, P, P, P, P, P, i32, i32, P, P, sz, P, P]),
+            "moe_dequant_slot": (C.c_int, [P, i32, D, P, P, P]),
+            "moe_quantize_rows": (C.c_int, [P, i32, i32, i32, i32, P, P, P]),
+            "moe_exp_portable": (C.c_int, [P, i64, P, P]),
+            "moe_status_string": (C.c_char_p, [C.c_int]),
+            "moe_cache_create": (C.c_int, [i32, i32, P, i32, C.POINTER(P)]),
+            "moe_cache_destroy": (None, [P]),
+            "moe_cache_table": (C.POINTER(i32), [P, i32]),
+            "moe_cache_layer_base": (i32, [P, i32]),
+            "moe_cache_class_slots": (i32, [P, i32]),
+            "moe_cache_place": (C.c_int, [P, i32, P, P, i32]),
+            "moe_cache_step": (C.c_int, [P, i32, P, i32, P, P, P]),
+            "moe_cache_stats": (None, [P, P, P, P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().moe_status_string(int(s)).decode()
+
+
+def _ck(status: int, where: str) -> None:
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def _ptr(t) -> int | None:
+    """Device (or host) address of a tensor / int / None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream  # torch.cuda.Stream
+
+
+def desc(E, k, H, I, group, bits_gu, bits_down=None) -> LayerDesc:
+    return LayerDesc(E, k, H, I, group, bits_gu, bits_gu if bits_down is None else bits_down)
+
+
+# ---------------------------------------------------------------------------
+# sizes
+# ---------------------------------------------------------------------------
+def moe_slot_bytes(d: LayerDesc) -> int:
+    return int(lib().moe_slot_bytes(C.byref(d)))
+
+
+def moe_slot_layout(d: LayerDesc) -> SlotLayout:
+    out = SlotLayout()
+    _ck(lib().moe_slot_layout(C.byref(d), C.byref(out)), "moe_slot_layout")
+    return out
+
+
+def moe_workspace_bytes(d: LayerDesc, max_tokens: int) -> int:
+    return int(lib().moe_workspace_bytes(C.byref(d), int(max_tokens)))
+
+
+# ---------------------------------------------------------------------------
+# stages
+# ---------------------------------------------------------------------------
+def moe_route(logits, T, d, L, slot_table, ids, w, stream=None) -> None:
+    _ck(lib().moe_route(_ptr(logits), int(T), C.byref(d), float(L), _ptr(slot_table), _ptr(ids), _ptr(w),
+                        _stream(stream)), "moe_route")
+
+
+def moe_sort(ids, x, T, d, offsets, pairs, active, n_active, x_sorted, ws, ws_bytes, stream=None) -> None:
+    _ck(lib().moe_sort(_ptr(ids), _ptr(x), int(T), C.byref(d), _ptr(offsets), _ptr(pairs), _ptr(active),
+                       _ptr(n_active), _ptr(x_sorted), _ptr(ws), int(ws_bytes), _stream(stream)), "moe_sort")
+
+
+def moe_slot_lookup(slot_table, active, n_active, pass_begin, pass_len, n_slots, slots, miss, n_miss, dev_err,
+                    stream=None) -> None:
+    _ck(lib().moe_slot_lookup(_ptr(slot_table), _ptr(active), _ptr(n_active), int(pass_begin), int(pass_len),
+                              int(n_slots), _ptr(slots), _ptr(miss), _ptr(n_miss), _ptr(dev_err), _stream(stream)),
+        "moe_slot_lookup")
+
+
+def moe_install_slots(pool, slot_bytes, n_slots, host_rows, slots, side=None, done=None) -> None:
+    """host_rows: sequence of pinned host addresses (ints); slots: host ints."""
+    n = len(slots)
+    rows = (C.c_void_p * max(n, 1))(*host_rows)
+    sl = (C.c_int32 * max(n, 1))(*[int(s) for s in slots])
+    ev = None if done is None else (done if isinstance(done, int) else done.cuda_event)
+    _ck(lib().moe_install_slots(_ptr(pool), int(slot_bytes), int(n_slots), rows, sl, n, _stream(side), ev),
+        "moe_install_slots")
+
+
+def moe_expert_ffn(x, T, d, pool, n_slots, slot_table, ids, w, offsets, pairs, active, n_active, x_sorted,
+                   pass_begin, pass_len, y_accum, ws, ws_bytes, dev_err, stream=None) -> None:
+    _ck(lib().moe_expert_ffn(_ptr(x), int(T), C.byref(d), _ptr(pool), int(n_slots), _ptr(slot_table), _ptr(ids),
+                             _ptr(w), _ptr(offsets), _ptr(pairs), _ptr(active), _ptr(n_active), _ptr(x_sorted),
+                             int(pass_begin), int(pass_len), _ptr(y_accum), _ptr(ws), int(ws_bytes), _ptr(dev_err),
+                             _stream(stream)), "moe_expert_ffn")
+
+
+def moe_dequant_slot(pool, slot, d, out_fp32, out_bf16, stream=None) -> None:
+    _ck(lib().moe_dequant_slot(_ptr(pool), int(slot), C.byref(d), _ptr(out_fp32), _ptr(out_bf16),
+                               _stream(stream)), "moe_dequant_slot")
+
+
+def moe_quantize_rows(w, rows, K, group, bits, q, sb, stream=None) -> None:
+    _ck(lib().moe_quantize_rows(_ptr(w), int(rows), int(K), int(group), int(bits), _ptr(q), _ptr(sb),
+                                _stream(stream)), "moe_quantize_rows")
+
+
+def moe_exp_portable(x, n, out, stream=None) -> None:
+    _ck(lib().moe_exp_portable(_ptr(x), int(n), _ptr(out), _stream(stream)), "moe_exp_portable")
+
+
+# ---------------------------------------------------------------------------
+# host slot cache
+# ---------------------------------------------------------------------------
+class SlotCache:
+    """moe_cache_*: one LRU per (size class, layer), host memory."""
+
+    def __init__(self, E: int, n_layers: int, slots_per_layer: int, layer_class=None):
+        self.E, self.n_layers, self.S = E, n_layers, slots_per_layer
+        h = C.c_void_p()
+        lc = None if layer_class is None else (C.c_int32 * n_layers)(*[int(c) for c in layer_class])
+        _ck(lib().moe_cache_create(E, n_layers, lc, slots_per_layer, C.byref(h)), "moe_cache_create")
+        self._h = h
+        self._out_e = (C.c_int32 * E)()
+        self._out_s = (C.c_int32 * E)()
+
+    def close(self):
+        if self._h:
+            lib().moe_cache_destroy(self._h)
+            self._h = None
+
+    __del__ = close
+
+    def table(self, layer: int):
+        """Host expert -> slot table of the layer (a live ctypes view, length E)."""
+        p = lib().moe_cache_table(self._h, layer)
+        return (C.c_int32 * self.E).from_address(C.addressof(p.contents))
+
+    def table_address(self, layer: int) -> int:
+        return C.addressof(lib().moe_cache_table(self._h, layer).contents)
+
+    def layer_base(self, layer: int) -> int:
+        return int(lib().moe_cache_layer_base(self._h, layer))
+
+    def class_slots(self, cls: int) -> int:
+        return int(lib().moe_cache_class_slots(self._h, cls))
+
+    def place(self, layer: int, experts, slots) -> None:
+        n = len(experts)
+        ea = (C.c_int32 * max(n, 1))(*[int(e) for e in experts])
+        sa = (C.c_int32 * max(n, 1))(*[int(s) for s in slots])
+        _ck(lib().moe_cache_place(self._h, layer, ea, sa, n), "moe_cache_place")
+
+    def step(self, layer: int, pass_experts):
+        """Returns (status, [(expert, slot), ...]) for the misses, ascending."""
+        n = len(pass_experts)
+        pa = (C.c_int32 * max(n, 1))(*[int(e) for e in pass_experts])
+        nout = C.c_int32(0)
+        st = lib().moe_cache_step(self._h, layer, pa, n, self._out_e, self._out_s, C.byref(nout))
+        if st not in (MOE_OK, MOE_ERR_CAPACITY):
+            _ck(st, "moe_cache_step")
+        return st, [(self._out_e[i], self._out_s[i]) for i in range(nout.value)]
+
+    def stats(self):
+        h, m, e = C.c_int64(), C.c_int64(), C.c_int64()
+        lib().moe_cache_stats(self._h, C.byref(h), C.byref(m), C.byref(e))
+        return h.value, m.value, e.value

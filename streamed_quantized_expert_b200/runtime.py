@@ -1,0 +1,215 @@
+"""Per-layer driver of the streamed expert FFN over the C ABI.
+
+Sequencing only: every step below is one libmoe call (or a plain copy).
+  decode layer:  route -> sort -> slot lookup -> (misses to host, LRU step,
+                 pinned installs on a side stream, table upload) -> FFN
+  prefill layer: route (L = 0) -> sort -> for each pass of <= 64 active
+                 experts: lookup -> installs -> FFN   (RFC "How the prototype
+                 works", items "Reads" and "Prefill")
+When every expert of a layer is resident the layer never synchronises with
+the host (RFC: "When every expert is resident, layers never synchronize with
+the host").  Layers are grouped into size classes by slot byte size, one
+device pool and one LRU range per (class, layer) (1bit-MONSTER PR #137).
+"""
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+
+import torch
+
+from . import ops
+
+PASS_EXPERTS = 64  # RFC / PR #50717: sorted prefill runs 64 experts at a time
+
+
+@dataclass
+class LayerSpec:
+    desc: ops.LayerDesc
+    bank: torch.Tensor            # pinned uint8 [rows, slot_bytes] of this layer's class
+    bank_row: list                # expert e -> row of `bank`
+
+
+class Streamer:
+    def __init__(self, layers: list[LayerSpec], slots_per_layer: int, max_tokens: int, device="cuda",
+                 stream: torch.cuda.Stream | None = None):
+        self.layers = layers
+        self.n_layers = len(layers)
+        self.device = torch.device(device)
+        self.E = layers[0].desc.E
+        self.k = layers[0].desc.k
+        self.H = layers[0].desc.H
+        assert all(l.desc.E == self.E and l.desc.H == self.H for l in layers)
+        self.S = slots_per_layer
+        self.max_tokens = max_tokens
+        self.stream = stream or torch.cuda.current_stream(self.device)
+        self.side = torch.cuda.Stream(self.device)
+        self.installed = torch.cuda.Event()
+        # size classes
+        sizes = []
+        self.layer_class = []
+        for l in layers:
+            sb = ops.moe_slot_bytes(l.desc)
+            if sb not in sizes:
+                sizes.append(sb)
+            self.layer_class.append(sizes.index(sb))
+        self.class_bytes = sizes
+        self.cache = ops.SlotCache(self.E, self.n_layers, self.S, self.layer_class)
+        self.pools = []
+        for c, sb in enumerate(sizes):
+            n = self.cache.class_slots(c)
+            self.pools.append(torch.empty(n * sb, dtype=torch.uint8, device=self.device))
+        self.class_n_slots = [self.cache.class_slots(c) for c in range(len(sizes))]
+        # device tables + pinned mirrors
+        self.table_dev = torch.full((self.n_layers, self.E), -1, dtype=torch.int32, device=self.device)
+        self.table_pin = torch.full((self.n_layers, self.E), -1, dtype=torch.int32).pin_memory()
+        # per-call buffers
+        T, E, k = max_tokens, self.E, self.k
+        self.ids = torch.empty((T, k), dtype=torch.int32, device=self.device)
+        self.w = torch.empty((T, k), dtype=torch.float32, device=self.device)
+        self.offsets = torch.empty(E + 1, dtype=torch.int32, device=self.device)
+        self.pairs = torch.empty(max(T * k, 1), dtype=torch.int32, device=self.device)
+        # meta: [n_active, n_miss, active[E], miss[E]] -> one small D2H per layer
+        self.meta = torch.zeros(2 + 2 * E, dtype=torch.int32, device=self.device)
+        self.meta_pin = torch.zeros(2 + 2 * E, dtype=torch.int32).pin_memory()
+        self.slots = torch.empty(E, dtype=torch.int32, device=self.device)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=self.device)
+        ws = max(ops.moe_workspace_bytes(l.desc, T) for l in layers)
+        self.ws_bytes = ws
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=self.device)
+        self.x_sorted = None
+        self.y = torch.zeros((T, self.H), dtype=torch.float32, device=self.device)
+        self.installed_bytes = 0
+        self.installs = 0
+
+    # -- views into meta --------------------------------------------------
+    def _n_active(self):
+        return self.meta[0:1]
+
+    def _n_miss(self):
+        return self.meta[1:2]
+
+    def _active(self):
+        return self.meta[2: 2 + self.E]
+
+    def _miss(self):
+        return self.meta[2 + self.E: 2 + 2 * self.E]
+
+    # -- residency ----------------------------------------------------------
+    def pool_of(self, layer: int) -> torch.Tensor:
+        return self.pools[self.layer_class[layer]]
+
+    def n_slots_of(self, layer: int) -> int:
+        return self.class_n_slots[self.layer_class[layer]]
+
+    def _row_addr(self, layer: int, e: int) -> int:
+        spec = self.layers[layer]
+        row = spec.bank_row[e]
+        return spec.bank.data_ptr() + row * spec.bank.shape[1]
+
+    def _upload_table(self, layer: int, stream) -> None:
+        tab = self.cache.table(layer)
+        C.memmove(self.table_pin[layer].data_ptr(), C.addressof(tab), 4 * self.E)
+        with torch.cuda.stream(stream):
+            self.table_dev[layer].copy_(self.table_pin[layer], non_blocking=True)
+
+    def place(self, layer: int, experts, slots_rel=None) -> None:
+        """Make `experts` resident in layer `layer` (slots relative to the
+        layer's range; default 0, 1, ...), copying their rows synchronously."""
+        base = self.cache.layer_base(layer)
+        rel = list(range(len(experts))) if slots_rel is None else list(slots_rel)
+        self.cache.place(layer, experts, [base + s for s in rel])
+        sb = self.class_bytes[self.layer_class[layer]]
+        ops.moe_install_slots(self.pool_of(layer), sb, self.n_slots_of(layer),
+                              [self._row_addr(layer, e) for e in experts], [base + s for s in rel],
+                              self.side, None)
+        self._upload_table(layer, self.side)
+        self.side.synchronize()
+
+    def fully_resident(self, layer: int) -> bool:
+        return all(v >= 0 for v in self.cache.table(layer))
+
+    def _install_pass(self, layer: int, pass_experts) -> int:
+        st, inst = self.cache.step(layer, pass_experts)
+        if st != ops.MOE_OK:
+            raise ops.MoeError(st, f"slot cache step (layer {layer})")
+        if inst:
+            sb = self.class_bytes[self.layer_class[layer]]
+            ops.moe_install_slots(self.pool_of(layer), sb, self.n_slots_of(layer),
+                                  [self._row_addr(layer, e) for e, _ in inst], [s for _, s in inst], self.side, None)
+            self._upload_table(layer, self.side)
+            self.installed.record(self.side)
+            self.stream.wait_event(self.installed)
+            self.installed_bytes += sb * len(inst)
+            self.installs += len(inst)
+        return len(inst)
+
+    # -- stages -------------------------------------------------------------
+    def route_sort(self, layer: int, x, logits, T: int, L: float = 0.0, want_sorted_x: bool = False):
+        d = self.layers[layer].desc
+        s = self.stream
+        ops.moe_route(logits, T, d, L, self.table_dev[layer], self.ids, self.w, s)
+        xs = None
+        if want_sorted_x:
+            if self.x_sorted is None or self.x_sorted.numel() < T * self.k * self.H:
+                self.x_sorted = torch.empty((self.max_tokens * self.k, self.H), dtype=torch.uint16,
+                                            device=self.device)
+            xs = self.x_sorted
+        ops.moe_sort(self.ids, x if want_sorted_x else None, T, d, self.offsets, self.pairs, self._active(),
+                     self._n_active(), xs, self.ws, self.ws_bytes, s)
+
+    def ffn(self, layer: int, x, T: int, pass_begin: int, pass_len: int, y) -> None:
+        d = self.layers[layer].desc
+        ops.moe_expert_ffn(x, T, d, self.pool_of(layer), self.n_slots_of(layer), self.table_dev[layer], self.ids,
+                           self.w, self.offsets, self.pairs, self._active(), self._n_active(),
+                           self.x_sorted if T >= 256 else None, pass_begin, pass_len, y, self.ws, self.ws_bytes,
+                           self.dev_err, self.stream)
+
+    def decode_layer(self, layer: int, x, logits, T: int, L: float = 0.0, y=None):
+        """One decode layer (T <= 64 tokens); returns y fp32 [T, H] (device)."""
+        y = self.y[:T] if y is None else y
+        s = self.stream
+        self.route_sort(layer, x, logits, T, L)
+        if not self.fully_resident(layer):
+            d = self.layers[layer].desc
+            ops.moe_slot_lookup(self.table_dev[layer], self._active(), self._n_active(), 0, self.E,
+                                self.n_slots_of(layer), self.slots, self._miss(), self._n_miss(), self.dev_err, s)
+            with torch.cuda.stream(s):
+                self.meta_pin.copy_(self.meta, non_blocking=True)
+            s.synchronize()
+            na = int(self.meta_pin[0])
+            act = self.meta_pin[2: 2 + na].tolist()
+            self._install_pass(layer, act)
+            del d
+        with torch.cuda.stream(s):
+            y.zero_()
+        self.ffn(layer, x, T, 0, self.E, y)
+        return y
+
+    def prefill_layer(self, layer: int, x, logits, T: int, y=None):
+        """One prefill chunk: passes of <= 64 active experts; returns y."""
+        y = self.y[:T] if y is None else y
+        s = self.stream
+        self.route_sort(layer, x, logits, T, 0.0, want_sorted_x=T >= 256)
+        with torch.cuda.stream(s):
+            y.zero_()
+            self.meta_pin.copy_(self.meta, non_blocking=True)
+        s.synchronize()
+        na = int(self.meta_pin[0])
+        active = self.meta_pin[2: 2 + na].tolist()
+        resident = self.fully_resident(layer)
+        for p in range(0, na, PASS_EXPERTS):
+            pe = active[p: p + PASS_EXPERTS]
+            if not resident:
+                # every pass synchronises: its slots come from the host LRU
+                ops.moe_slot_lookup(self.table_dev[layer], self._active(), self._n_active(), p, PASS_EXPERTS,
+                                    self.n_slots_of(layer), self.slots, self._miss(), self._n_miss(), self.dev_err,
+                                    s)
+                s.synchronize()  # previous pass's FFN done before its slots can be reused
+                self._install_pass(layer, pe)
+            self.ffn(layer, x, T, p, PASS_EXPERTS, y)
+        return y
+
+    def check_dev_err(self) -> int:
+        v = int(self.dev_err.item())
+        return v
