@@ -39,22 +39,25 @@ def make(orc, n_layers, E, k, H, I, g, bits, S, R, seed=0):
 
 
 def initial_fill(st, seed, S):
+    placed = []
     for l in range(st.n_layers):
         rank = synth.popularity_rank(seed, l, st.E)
         hot = np.argsort(rank)[:S]  # most popular experts first
         rel = synth.slot_permutation(seed, l, S)
         st.place(l, hot.tolist(), rel.tolist())
+        placed.append((hot.astype(np.int32), rel.astype(np.int32) + st.cache.layer_base(l)))
+    return placed
 
 
 def test_decode_with_installs(orc):
     E, k, H, I, g, S = 512, 10, 2048, 512, 64, 192
     specs, host_slots = make(orc, 2, E, k, H, I, g, [(3, 3), (3, 3)], S, R=12)
     st = Streamer(specs, S, max_tokens=1)
-    initial_fill(st, 0, S)
+    placed = initial_fill(st, 0, S)
     models = []
     for l in range(2):
         m = orc.LruModel(E, S, slot_base=st.cache.layer_base(l))
-        m.table[:] = np.frombuffer(st.cache.table(l), dtype=np.int32)
+        m.place(*placed[l])
         models.append(m)
     total_inst = 0
     for step in range(6):
