@@ -30,6 +30,25 @@ class LayerSpec:
     bank_row: list                # expert e -> row of `bank`
 
 
+def quantize_bank_gpu(E: int, desc: ops.LayerDesc, seed: int, device="cuda", std: float = 0.02) -> torch.Tensor:
+    """Pinned uint8 [E, slot_bytes]: expert e = N(0, std) weights (seeded torch
+    generator) quantised on the GPU by moe_quantize_rows into the slot format."""
+    from . import synth
+
+    lay = ops.moe_slot_layout(desc)
+    sb = int(lay.slot_bytes)
+    H, I, g = desc.H, desc.I, desc.group
+    bank = torch.empty((E, sb), dtype=torch.uint8).pin_memory()
+    slot = torch.zeros(sb, dtype=torch.uint8, device=device)
+    for e in range(E):
+        w_gu, w_d = synth.expert_weights_torch(seed, e, H, I, device, std)
+        base = slot.data_ptr()
+        ops.moe_quantize_rows(w_gu, 2 * I, H, g, desc.bits_gu, base + lay.q_gate_up, base + lay.sb_gate_up)
+        ops.moe_quantize_rows(w_d, H, I, g, desc.bits_down, base + lay.q_down, base + lay.sb_down)
+        bank[e].copy_(slot, non_blocking=False)
+    return bank
+
+
 class Streamer:
     def __init__(self, layers: list[LayerSpec], slots_per_layer: int, max_tokens: int, device="cuda",
                  stream: torch.cuda.Stream | None = None):
@@ -81,6 +100,9 @@ class Streamer:
         self.y = torch.zeros((T, self.H), dtype=torch.float32, device=self.device)
         self.installed_bytes = 0
         self.installs = 0
+        self.launches = 0          # libmoe kernel launches issued (for reporting)
+        self._full = [False] * self.n_layers
+        self.ffn_events = None     # list to collect (start, end) CUDA events around FFN calls
 
     # -- views into meta --------------------------------------------------
     def _n_active(self):
@@ -125,9 +147,10 @@ class Streamer:
                               self.side, None)
         self._upload_table(layer, self.side)
         self.side.synchronize()
+        self._full[layer] = self.S >= self.E and all(v >= 0 for v in self.cache.table(layer))
 
     def fully_resident(self, layer: int) -> bool:
-        return all(v >= 0 for v in self.cache.table(layer))
+        return self._full[layer]
 
     def _install_pass(self, layer: int, pass_experts) -> int:
         st, inst = self.cache.step(layer, pass_experts)
@@ -149,6 +172,7 @@ class Streamer:
         d = self.layers[layer].desc
         s = self.stream
         ops.moe_route(logits, T, d, L, self.table_dev[layer], self.ids, self.w, s)
+        self.launches += 1
         xs = None
         if want_sorted_x:
             if self.x_sorted is None or self.x_sorted.numel() < T * self.k * self.H:
@@ -157,13 +181,22 @@ class Streamer:
             xs = self.x_sorted
         ops.moe_sort(self.ids, x if want_sorted_x else None, T, d, self.offsets, self.pairs, self._active(),
                      self._n_active(), xs, self.ws, self.ws_bytes, s)
+        self.launches += (1 if T * self.k <= 1024 else 3) + (1 if want_sorted_x else 0)
 
     def ffn(self, layer: int, x, T: int, pass_begin: int, pass_len: int, y) -> None:
         d = self.layers[layer].desc
+        ev = None
+        if self.ffn_events is not None:
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            ev[0].record(self.stream)
+        self.launches += 2 if T <= 64 else 3
         ops.moe_expert_ffn(x, T, d, self.pool_of(layer), self.n_slots_of(layer), self.table_dev[layer], self.ids,
                            self.w, self.offsets, self.pairs, self._active(), self._n_active(),
                            self.x_sorted if T >= 256 else None, pass_begin, pass_len, y, self.ws, self.ws_bytes,
                            self.dev_err, self.stream)
+        if ev is not None:
+            ev[1].record(self.stream)
+            self.ffn_events.append(ev)
 
     def decode_layer(self, layer: int, x, logits, T: int, L: float = 0.0, y=None):
         """One decode layer (T <= 64 tokens); returns y fp32 [T, H] (device)."""
@@ -174,6 +207,7 @@ class Streamer:
             d = self.layers[layer].desc
             ops.moe_slot_lookup(self.table_dev[layer], self._active(), self._n_active(), 0, self.E,
                                 self.n_slots_of(layer), self.slots, self._miss(), self._n_miss(), self.dev_err, s)
+            self.launches += 1
             with torch.cuda.stream(s):
                 self.meta_pin.copy_(self.meta, non_blocking=True)
             s.synchronize()
@@ -205,6 +239,7 @@ class Streamer:
                 ops.moe_slot_lookup(self.table_dev[layer], self._active(), self._n_active(), p, PASS_EXPERTS,
                                     self.n_slots_of(layer), self.slots, self._miss(), self._n_miss(), self.dev_err,
                                     s)
+                self.launches += 1
                 s.synchronize()  # previous pass's FFN done before its slots can be reused
                 self._install_pass(layer, pe)
             self.ffn(layer, x, T, p, PASS_EXPERTS, y)
