@@ -31,8 +31,9 @@
  *     ordinary (or pinned, where stated) host memory.  bf16 tensors are passed
  *     as uint16_t bit patterns.  All arrays are dense, row-major.
  *   - The library allocates no device memory and keeps no state between
- *     calls (the host slot cache object is the one exception, and it lives in
- *     host memory).  The caller owns every buffer, stream and event.
+ *     calls (the host slot cache object lives in host memory; the one fixed
+ *     device array is the scratch of moe_expert_ffn_noalloc).  The caller owns
+ *     every buffer, stream and event.
  *   - Every device call is asynchronous on the given stream and does not
  *     synchronise with the host.
  *   - Argument errors are found before anything is launched and return
@@ -199,6 +200,32 @@ moe_status moe_expert_ffn(const uint16_t* x, int32_t T, const moe_layer_desc* d,
                           const int32_t* n_active, const uint16_t* x_sorted, int32_t pass_begin,
                           int32_t pass_len, float* y_accum, void* ws, size_t ws_bytes, int32_t* dev_err,
                           cudaStream_t stream);
+
+/* moe_expert_ffn without a caller-supplied workspace.  (The pages have no
+ * counterpart; this is an interface convenience.)  For callers that cannot
+ * allocate device memory themselves -- e.g. a plugin whose host process owns
+ * all device memory through its own allocator, or a serving loop that must
+ * not call cudaMalloc (which can synchronise the device) once it is running.
+ * The scratch is one fixed device array of moe_noalloc_scratch_bytes() bytes
+ * (1 MiB) inside the library, held by every GPU that loads it until the
+ * process exits.  Same arguments and results as moe_expert_ffn, except:
+ *   - T must be <= 64 and moe_workspace_bytes(d, T) <= 1 MiB, else
+ *     MOE_ERR_CAPACITY is returned and nothing is launched;
+ *   - x_sorted is not taken (the decode kernels do not use it);
+ *   - the first call on a device looks up the array's device address (with
+ *     that device current); make that first call outside any stream capture;
+ *   - every call shares the one array and leaves its contents behind; nothing
+ *     in it has to start at zero, but calls whose kernels overlap on the GPU
+ *     (e.g. on two streams at once) race on it.
+ * Allocates nothing. */
+moe_status moe_expert_ffn_noalloc(const uint16_t* x, int32_t T, const moe_layer_desc* d, const void* pool,
+                                  int32_t n_slots, const int32_t* slot_table, const int32_t* ids, const float* w,
+                                  const int32_t* offsets, const int32_t* pairs, const int32_t* active,
+                                  const int32_t* n_active, int32_t pass_begin, int32_t pass_len, float* y_accum,
+                                  int32_t* dev_err, cudaStream_t stream);
+
+/* Size of the fixed scratch array used by moe_expert_ffn_noalloc. */
+size_t moe_noalloc_scratch_bytes(void);
 
 /* Test/inspection: dequantise slot `slot` of pool through the same code
  * extraction the FFN kernels use.  out_fp32 (device, may be NULL):

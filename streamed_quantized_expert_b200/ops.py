@@ -23,6 +23,7 @@ ABI_SYMBOLS = [
     "moe_install_slots", "moe_expert_ffn", "moe_dequant_slot", "moe_quantize_rows", "moe_exp_portable",
     "moe_status_string", "moe_cache_create", "moe_cache_destroy", "moe_cache_table", "moe_cache_layer_base",
     "moe_cache_class_slots", "moe_cache_place", "moe_cache_step", "moe_cache_stats",
+    "moe_expert_ffn_noalloc", "moe_noalloc_scratch_bytes",
 ]
 
 
@@ -66,6 +67,8 @@ def lib():
             "moe_slot_lookup": (C.c_int, [P, P, P, i32, i32, i32, P, P, P, P, P]),
             "moe_install_slots": (C.c_int, [P, sz, i32, P, P, i32, P, P]),
             "moe_expert_ffn": (C.c_int, [P, i32, D, P, i32, P, P, P, P, P, P, P, P, i32, i32, P, P, sz, P, P]),
+            "moe_expert_ffn_noalloc": (C.c_int, [P, i32, D, P, i32, P, P, P, P, P, P, P, i32, i32, P, P, P]),
+            "moe_noalloc_scratch_bytes": (sz, []),
             "moe_dequant_slot": (C.c_int, [P, i32, D, P, P, P]),
             "moe_quantize_rows": (C.c_int, [P, i32, i32, i32, i32, P, P, P]),
             "moe_exp_portable": (C.c_int, [P, i64, P, P]),
@@ -170,6 +173,20 @@ def moe_expert_ffn(x, T, d, pool, n_slots, slot_table, ids, w, offsets, pairs, a
                              _ptr(w), _ptr(offsets), _ptr(pairs), _ptr(active), _ptr(n_active), _ptr(x_sorted),
                              int(pass_begin), int(pass_len), _ptr(y_accum), _ptr(ws), int(ws_bytes), _ptr(dev_err),
                              _stream(stream)), "moe_expert_ffn")
+
+
+def moe_expert_ffn_noalloc(x, T, d, pool, n_slots, slot_table, ids, w, offsets, pairs, active, n_active,
+                           pass_begin, pass_len, y_accum, dev_err, stream=None) -> None:
+    """moe_expert_ffn with the library's own fixed scratch array (no workspace
+    argument): for callers that cannot allocate device memory."""
+    _ck(lib().moe_expert_ffn_noalloc(_ptr(x), int(T), C.byref(d), _ptr(pool), int(n_slots), _ptr(slot_table),
+                                     _ptr(ids), _ptr(w), _ptr(offsets), _ptr(pairs), _ptr(active), _ptr(n_active),
+                                     int(pass_begin), int(pass_len), _ptr(y_accum), _ptr(dev_err),
+                                     _stream(stream)), "moe_expert_ffn_noalloc")
+
+
+def moe_noalloc_scratch_bytes() -> int:
+    return int(lib().moe_noalloc_scratch_bytes())
 
 
 def moe_dequant_slot(pool, slot, d, out_fp32, out_bf16, stream=None) -> None:
