@@ -69,7 +69,7 @@ class ClockSampler:
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -132,16 +132,16 @@ def build_streamer(cfg, seed, device):
     return st
 
 
-def make_inputs(cfg, seed, n_steps, device, pinned=False):
+def make_inputs(cfg, seed, n_steps, device, pinned=False, step0=0):
     import numpy as np
     import torch
 
     from streamed_quantized_expert_b200 import synth
 
     n_layers, E, k, H, I, g, bg, bd, T, S, _ = cfg
-    xs = np.stack([np.stack([synth.activations(seed, l, T, H, step=s) for l in range(n_layers)])
+    xs = np.stack([np.stack([synth.activations(seed, l, T, H, step=step0 + s) for l in range(n_layers)])
                    for s in range(n_steps)])
-    lg = np.stack([np.stack([synth.router_logits(seed, l, T, E, step=s) for l in range(n_layers)])
+    lg = np.stack([np.stack([synth.router_logits(seed, l, T, E, step=step0 + s) for l in range(n_layers)])
                    for s in range(n_steps)])
     x = torch.from_numpy(xs.view(np.int16))
     logits = torch.from_numpy(lg)
@@ -150,16 +150,42 @@ def make_inputs(cfg, seed, n_steps, device, pinned=False):
     return x.to(device), logits.to(device)
 
 
-def algorithmic_bytes_per_ffn(cfg, n_unique):
+def ffn_graph_time(st, cfg, snaps, reps, device):
+    """Time the FFN alone: a CUDA graph of the 48 layers' moe_expert_ffn calls
+    (each with its layer's routing from one decode step), replayed `reps`
+    times; returns microseconds per layer."""
+    import torch
+
     from streamed_quantized_expert_b200 import ops
 
     n_layers, E, k, H, I, g, bg, bd, T, S, _ = cfg
-    sb = ops.moe_slot_bytes(ops.desc(E, k, H, I, g, bg, bd))
-    return n_unique * sb + T * H * 2 + T * H * 4  # unique experts' slots + x in (bf16) + y out (fp32)
+    y = torch.zeros((T, H), dtype=torch.float32, device=device)
+    g_ = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(device)
+    torch.cuda.synchronize(device)
+    with torch.cuda.graph(g_, stream=cap):
+        cs = torch.cuda.current_stream(device)
+        for l in range(n_layers):
+            sn = snaps[l]
+            ops.moe_expert_ffn(sn["x"], T, st.layers[l].desc, st.pool_of(l), st.n_slots_of(l), st.table_dev[l],
+                               sn["ids"], sn["w"], sn["offsets"], sn["pairs"], sn["meta"][2:], sn["meta"][0:1], None,
+                               0, E, y, st.ws, st.ws_bytes, st.dev_err, cs)
+    for _ in range(3):
+        g_.replay()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s = torch.cuda.current_stream(device)
+    e0.record(s)
+    for _ in range(reps):
+        g_.replay()
+    e1.record(s)
+    torch.cuda.synchronize(device)
+    us = 1e3 * e0.elapsed_time(e1) / (reps * n_layers)
+    del g_
+    return us
 
 
 def run_ours(args, rank, world, local_rank):
-    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -175,25 +201,22 @@ def run_ours(args, rank, world, local_rank):
     seed = 1000 * rank
     st = build_streamer(cfg, seed, device)
     steps_total = args.warmup + args.steps
-    x, logits = make_inputs(cfg, seed + 1, steps_total, device)
+    # the popularity bias of the logits and the initially resident experts come from the same seed
+    x, logits = make_inputs(cfg, seed, steps_total + 1, device)
     s = st.stream
 
     def step(i, x_src, lg_src):
         for l in range(n_layers):
             st.decode_layer(l, x_src[i, l], lg_src[i, l], T)
 
-    # warm-up
     for i in range(args.warmup):
         step(i, x, logits)
     torch.cuda.synchronize(device)
     if world > 1:
         dist.barrier()
 
-    # timed: K steps, events around every FFN call for the kernel roofline
-    st.ffn_events = []
     inst0, bytes0, l0 = st.installs, st.installed_bytes, st.launches
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    uniq = []
     with ClockSampler(local_rank) as clk:
         torch.cuda.synchronize(device)
         e0.record(s)
@@ -201,16 +224,19 @@ def run_ours(args, rank, world, local_rank):
             step(i, x, logits)
         e1.record(s)
         torch.cuda.synchronize(device)
-    ms = e0.elapsed_time(e1)
-    ffn_ms = [a.elapsed_time(b) for a, b in st.ffn_events]
-    st.ffn_events = None
-    launches = st.launches - l0
-    installs, inst_bytes = st.installs - inst0, st.installed_bytes - bytes0
-    # unique experts per FFN call (T tokens x k, distinct): recompute from the oracle-free routing of the
-    # library itself is not needed for T = 1 (k distinct experts); for T > 1 count on the host from ids
-    n_unique = k if T == 1 else None
-    if n_unique is None:
-        n_unique = int(torch.unique(st.ids[:T]).numel())
+        ms = e0.elapsed_time(e1)
+        launches = st.launches - l0
+        installs, inst_bytes = st.installs - inst0, st.installed_bytes - bytes0
+
+        # one more (untimed) step whose per-layer routing is kept for the FFN-only replay
+        snaps = []
+        for l in range(n_layers):
+            st.decode_layer(l, x[steps_total, l], logits[steps_total, l], T)
+            snaps.append({"x": x[steps_total, l], "ids": st.ids.clone(), "w": st.w.clone(),
+                          "offsets": st.offsets.clone(), "pairs": st.pairs.clone(), "meta": st.meta.clone()})
+        torch.cuda.synchronize(device)
+        n_unique = sum(int(sn["meta"][0].item()) for sn in snaps) / n_layers
+        ffn_us = ffn_graph_time(st, cfg, snaps, args.ffn_reps, device)
     t = torch.tensor([ms], dtype=torch.float64, device=device)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -218,7 +244,7 @@ def run_ours(args, rank, world, local_rank):
     err = st.check_dev_err()
 
     # e2e: inputs from pinned host memory copied in, y of every layer read back, same K steps
-    xh, lgh = make_inputs(cfg, seed + 2, args.steps, device, pinned=True)
+    xh, lgh = make_inputs(cfg, seed, args.steps, device, pinned=True, step0=steps_total + 1)
     yh = torch.empty((args.steps, n_layers, T, H), dtype=torch.float32).pin_memory()
     xd = torch.empty((n_layers, T, H), dtype=torch.int16, device=device)
     lgd = torch.empty((n_layers, T, E), dtype=torch.float32, device=device)
@@ -247,16 +273,16 @@ def run_ours(args, rank, world, local_rank):
         return None
     hbm_peak, tf_peak, peak_kind = peaks()
     tokens = args.steps * T * world
-    ffn_bytes = algorithmic_bytes_per_ffn(cfg, n_unique)
-    ffn_avg_us = 1e3 * sum(ffn_ms) / len(ffn_ms)
-    achieved = ffn_bytes / (ffn_avg_us * 1e-6) / 1e9
-    ffn_total_s = sum(ffn_ms) / 1e3
+    from streamed_quantized_expert_b200 import ops as _ops
+
+    slot_b = _ops.moe_slot_bytes(_ops.desc(E, k, H, I, g, bg, bd))
+    ffn_bytes = n_unique * slot_b + T * H * 2 + T * H * 4
+    achieved = ffn_bytes / (ffn_us * 1e-6) / 1e9
     flops_per_ffn = 2.0 * T * k * 3 * H * I
     out = {
         "metric": METRIC,
         "value": round(tokens / (ms_max / 1e3), 3),
-        "unit": "tok/s (whole path: route+sort+lookup+installs+FFN+combine, 48 layers)"
-        if n_layers == 48 else "tok/s (whole path)",
+        "unit": "tok/s (whole path: route+sort+lookup+installs+FFN+combine, %d layers)" % n_layers,
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
@@ -271,17 +297,19 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "inputs larger than L2: each step reads ~%.0f MB of distinct expert slots" %
                          (n_layers * ffn_bytes / 1e6),
                    "parallelism": f"replicas x{world} (independent token streams)"},
-        "ffn": {"tok_s_equiv": round(args.steps * T / ffn_total_s, 1),
-                "us_per_layer": round(ffn_avg_us, 3),
+        "ffn": {"tok_s_equiv": round(T / (n_layers * ffn_us * 1e-6), 1),
+                "us_per_layer": round(ffn_us, 3),
                 "hbm_gbs": round(achieved, 1),
-                "tflops": round(flops_per_ffn / (ffn_avg_us * 1e-6) / 1e12, 3)},
-        "installs": {"experts": installs, "per_token": round(installs / max(args.steps, 1), 2),
+                "tflops": round(flops_per_ffn / (ffn_us * 1e-6) / 1e12, 3),
+                "how": "CUDA graph of the %d layers' moe_expert_ffn calls, replayed %d times, CUDA events" %
+                       (n_layers, args.ffn_reps)},
+        "installs": {"experts": installs, "per_token": round(installs / max(args.steps * T, 1), 2),
                      "miss_rate": round(installs / max(args.steps * n_layers * T * k, 1), 4),
                      "bytes": inst_bytes},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "traffic": None,
-                     "kernel": "moe_expert_ffn (gate/up+SwiGLU kernel + down+combine kernel)",
-                     "peak_kind": peak_kind},
+                     "kernel": "moe_expert_ffn (gate/up+SwiGLU kernel + down+combine kernel), per layer",
+                     "bytes_per_launch": int(ffn_bytes), "peak_kind": peak_kind},
         "gpu_launches": launches,
         "dev_err": err,
         "clocks": clk.summary(),
@@ -361,12 +389,19 @@ def main():
     ap.add_argument("--config", choices=sorted(CONFIGS), default="decode")
     ap.add_argument("--cpu-layers", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ffn-reps", type=int, default=20)
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (small profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.layers:
+        c = list(CONFIGS[args.config])
+        c[0] = args.layers
+        c[-1] = c[-1] + f" [layers overridden to {args.layers}]"
+        CONFIGS[args.config] = tuple(c)
     if args.impl == "reference":
         out = run_reference(args, rank)
         if out is not None:

@@ -247,6 +247,10 @@ moe_status moe_exp_portable(const float* x, int64_t n, float* out, cudaStream_t 
 
 const char* moe_status_string(moe_status s);
 
+/* Name of the last CUDA error that made a call of this thread return
+ * MOE_ERR_CUDA ("no error" if none). */
+const char* moe_last_cuda_error(void);
+
 /* ------------------------------------------------------------------------
  * Host slot cache (1bit-MONSTER PR #137: per size class, one LRU per layer,
  * every layer keeps the same share of its experts, empty slots taken first).
@@ -277,6 +281,53 @@ moe_status moe_cache_step(moe_cache* c, int32_t layer, const int32_t* pass_exper
                           int32_t* out_experts, int32_t* out_slots, int32_t* n_out);
 /* Counters since creation: hits, misses, evictions (of a resident expert). */
 void moe_cache_stats(const moe_cache* c, int64_t* hits, int64_t* misses, int64_t* evictions);
+
+/* Experts of `layer` that currently have a slot (E means fully resident). */
+int32_t moe_cache_resident(const moe_cache* c, int32_t layer);
+
+/* ------------------------------------------------------------------------
+ * Native driver of one decode layer (the sequence of the calls above).
+ * ---------------------------------------------------------------------- */
+
+/* Per-call device buffers, caller-owned, sized for max_tokens tokens. */
+typedef struct {
+  int32_t* ids;        /* device int32 [max_tokens, k] */
+  float* w;            /* device fp32 [max_tokens, k] */
+  int32_t* offsets;    /* device int32 [E+1] */
+  int32_t* pairs;      /* device int32 [max_tokens*k] */
+  int32_t* meta;       /* device int32 [2+2E]: n_active, n_miss, active[E], miss[E] */
+  int32_t* meta_host;  /* pinned host int32 [2+2E] */
+  int32_t* slots;      /* device int32 [E] */
+  int32_t* dev_err;    /* device int32 [1] */
+  void* ws;            /* device workspace */
+  size_t ws_bytes;     /* >= moe_workspace_bytes(desc, max_tokens) */
+  int32_t max_tokens;
+} moe_step_buffers;
+
+/* One layer's slot pool and tables. */
+typedef struct {
+  const moe_layer_desc* desc;
+  void* pool;                   /* device base of the layer's size-class pool */
+  int32_t n_slots;              /* slots in that pool */
+  size_t slot_bytes;            /* moe_slot_bytes(desc) */
+  int32_t* table_dev;           /* device int32 [E]: this layer's expert -> slot */
+  int32_t* table_stage;         /* pinned host int32 [E]: staging for table uploads */
+  const void* const* bank_rows; /* host [E]: pinned host address of each expert's slot bytes */
+} moe_layer_ctx;
+
+/* One decode layer, T <= 64 tokens (RFC "How the prototype works": each layer
+ * copies its routing to the host once; misses cost one host-to-device copy
+ * per expert; a fully resident layer never synchronises with the host):
+ *   moe_route (L) -> moe_sort -> if the layer is not fully resident in `cache`:
+ *   moe_slot_lookup, copy n_active/active to meta_host, synchronise `stream`,
+ *   moe_cache_step, moe_install_slots on `side`, upload the table, record
+ *   `installed` on `side` and make `stream` wait on it -> zero y -> one pass of
+ *   moe_expert_ffn over every active expert.
+ * y: device fp32 [T, H] (overwritten).  *n_installed (host, may be NULL): the
+ * number of experts installed.  Errors as the calls it makes. */
+moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc, const moe_step_buffers* b,
+                            const uint16_t* x, const float* logits, int32_t T, float L, float* y,
+                            cudaStream_t stream, cudaStream_t side, cudaEvent_t installed, int32_t* n_installed);
 
 #ifdef __cplusplus
 }

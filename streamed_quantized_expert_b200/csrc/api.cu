@@ -26,12 +26,23 @@ moe_status check_desc(const moe_layer_desc* d) {
   return MOE_OK;
 }
 
-moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+thread_local const char* g_last_cuda_error = "no error";
+
+moe_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  g_last_cuda_error = cudaGetErrorName(e);
+  return MOE_ERR_CUDA;
+}
 
 int device_sms() {
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms > 0 ? sms : 148;
+  static int cached[128] = {0};
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 128 && cached[dev] > 0) return cached[dev];
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms <= 0) sms = 148;
+  if (dev >= 0 && dev < 128) cached[dev] = sms;
+  return sms;
 }
 
 struct WsCarve {
@@ -54,6 +65,8 @@ WsCarve carve(const moe_layer_desc& d, int T) {
 }  // namespace
 
 extern "C" {
+
+const char* moe_last_cuda_error(void) { return g_last_cuda_error; }
 
 const char* moe_status_string(moe_status s) {
   switch (s) {

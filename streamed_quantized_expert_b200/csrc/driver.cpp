@@ -1,0 +1,69 @@
+// Host driver of one decode layer: the whole five-stage sequence in native
+// code, so the per-layer host cost is the launches and (when the layer is not
+// fully resident) one small device->host copy and its synchronisation.
+//
+//   route -> sort -> [lookup -> misses to host -> LRU step -> pinned installs on
+//   the side stream + table upload -> compute stream waits] -> y = 0 -> FFN
+//
+// RFC "How the prototype works": each layer copies its routing to the host
+// once; misses become one host-to-device copy per expert; when every expert
+// is resident the layer never synchronises with the host.
+#include <cstring>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "moe.h"
+
+extern "C" moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc,
+                                       const moe_step_buffers* b, const uint16_t* x, const float* logits,
+                                       int32_t T, float L, float* y, cudaStream_t stream, cudaStream_t side,
+                                       cudaEvent_t installed, int32_t* n_installed) {
+  if (!cache || !lc || !b || !lc->desc || !y || !x || !logits) return MOE_ERR_INVALID;
+  const moe_layer_desc* d = lc->desc;
+  if (T < 1 || T > b->max_tokens || T > 64) return MOE_ERR_INVALID;
+  const int32_t E = d->E;
+  if (n_installed) *n_installed = 0;
+  int32_t* n_active = b->meta;
+  int32_t* n_miss = b->meta + 1;
+  int32_t* active = b->meta + 2;
+  int32_t* miss = b->meta + 2 + E;
+  moe_status s = moe_route(logits, T, d, L, lc->table_dev, b->ids, b->w, stream);
+  if (s != MOE_OK) return s;
+  s = moe_sort(b->ids, nullptr, T, d, b->offsets, b->pairs, active, n_active, nullptr, b->ws, b->ws_bytes, stream);
+  if (s != MOE_OK) return s;
+  if (moe_cache_resident(cache, layer) < E) {
+    s = moe_slot_lookup(lc->table_dev, active, n_active, 0, E, lc->n_slots, b->slots, miss, n_miss, b->dev_err,
+                        stream);
+    if (s != MOE_OK) return s;
+    if (cudaMemcpyAsync(b->meta_host, b->meta, sizeof(int32_t) * (size_t)(2 + E), cudaMemcpyDeviceToHost,
+                        stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+    const int32_t na = b->meta_host[0];
+    if (na < 0 || na > E) return MOE_ERR_INVALID;
+    thread_local std::vector<int32_t> out_e, out_s;
+    thread_local std::vector<const void*> rows;
+    out_e.resize(E);
+    out_s.resize(E);
+    int32_t n = 0;
+    s = moe_cache_step(cache, layer, b->meta_host + 2, na, out_e.data(), out_s.data(), &n);
+    if (s != MOE_OK) return s;
+    if (n > 0) {
+      rows.resize(n);
+      for (int32_t i = 0; i < n; ++i) rows[i] = lc->bank_rows[out_e[i]];
+      s = moe_install_slots(lc->pool, lc->slot_bytes, lc->n_slots, rows.data(), out_s.data(), n, side, nullptr);
+      if (s != MOE_OK) return s;
+      std::memcpy(lc->table_stage, moe_cache_table(cache, layer), sizeof(int32_t) * (size_t)E);
+      if (cudaMemcpyAsync(lc->table_dev, lc->table_stage, sizeof(int32_t) * (size_t)E, cudaMemcpyHostToDevice,
+                          side) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (cudaEventRecord(installed, side) != cudaSuccess) return MOE_ERR_CUDA;
+      if (cudaStreamWaitEvent(stream, installed, 0) != cudaSuccess) return MOE_ERR_CUDA;
+      if (n_installed) *n_installed = n;
+    }
+  }
+  if (cudaMemsetAsync(y, 0, sizeof(float) * (size_t)T * d->H, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  return moe_expert_ffn(x, T, d, lc->pool, lc->n_slots, lc->table_dev, b->ids, b->w, b->offsets, b->pairs, active,
+                        n_active, nullptr, 0, E, y, b->ws, b->ws_bytes, b->dev_err, stream);
+}

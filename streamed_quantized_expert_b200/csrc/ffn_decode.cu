@@ -22,8 +22,6 @@
 
 namespace moe {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
 
 template <int B>
 __device__ __forceinline__ void load_unit(const uint8_t* p, uint32_t (&w)[B]) {
@@ -138,76 +136,139 @@ __device__ __forceinline__ void flag_slot(const FfnArgs& a, int slot) {
   if (a.dev_err) atomicOr(a.dev_err, slot < 0 ? MOE_DEV_ERR_NOT_RESIDENT : MOE_DEV_ERR_SLOT_RANGE);
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// Named barrier over the consumer warps only (the producer warp never joins).
+__device__ __forceinline__ void consumers_sync(int nthreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // gate/up + SwiGLU:  h[pos][j] = silu(gate_j . x_t) * (up_j . x_t)
-// Work item = (active expert of the pass, 8 consecutive j); warps split K.
+// Work item = (active expert of the pass, 8 consecutive j) = a 16-row MMA
+// tile (8 gate rows, 8 up rows).  Each CTA takes a contiguous range of items.
+// Warp 8 is the producer: it streams every item's rows into a ring of shared
+// memory stages (full/empty mbarriers).  Warps 0-7 split K (BPW 128-blocks
+// each, x fragments stay in registers while the token set is unchanged) and
+// run through all their items without CTA-wide barriers; partial sums are
+// reduced across warps once per batch of kRedBatch (item, token-tile) entries.
 // ---------------------------------------------------------------------------
+constexpr int kGuConsumers = 8;
+constexpr int kGuThreads = (kGuConsumers + 1) * 32;
+constexpr int kRedBatch = 8;
+
+struct RedMeta {
+  int pos;   // first sorted position of the token tile
+  int ntok;  // tokens in the tile
+  int jt;    // 8-row tile of the intermediate dimension
+  int pad;
+};
+
 template <int B, int BPW, int GS>
-__global__ void __launch_bounds__(kThreads, 1) ffn_gu_kernel(const FfnArgs a) {
+__global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, t4 = lane & 3, g8 = lane >> 2;
   const int NST = a.gu_nstage, SB = a.gu_stage_bytes, SR = a.sr_gu;
-  float* red = reinterpret_cast<float*>(smem + (size_t)NST * SB);  // [8 warps][32][4]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + kWarps * 32 * 4);
+  float* red = reinterpret_cast<float*>(smem + (size_t)NST * SB);  // [kRedBatch][8 warps][32][4]
+  RedMeta* meta = reinterpret_cast<RedMeta*>(red + kRedBatch * kGuConsumers * 32 * 4);
+  uint64_t* full = reinterpret_cast<uint64_t*>(meta + kRedBatch);
+  uint64_t* empty = full + NST;
 
   pdl_wait();
   const int n_act = pass_count(a);
   const int jt_n = a.I / 8;
   const int n_items = n_act * jt_n;
-  const int my_items = (int)blockIdx.x < n_items ? (n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-  if (my_items == 0) return;
+  const int i0 = (int)(((int64_t)n_items * blockIdx.x) / gridDim.x);
+  const int i1 = (int)(((int64_t)n_items * (blockIdx.x + 1)) / gridDim.x);
+  const int my_items = i1 - i0;
+  pdl_launch_dependents();
+  if (my_items <= 0) return;
   if (tid == 0) {
-    for (int s = 0; s < NST; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kGuConsumers);
+    }
     fence_barrier_init();
   }
   __syncthreads();
 
-  const uint32_t sbb = 8u * a.ng_gu * 4u;
-  auto issue = [&](int r) {
-    const int item = (int)blockIdx.x + r * (int)gridDim.x;
-    const int jt = item % jt_n;
-    const int e = a.active[a.pass_begin + item / jt_n];
-    const int slot = a.table[e];
-    uint8_t* st = smem + (size_t)(r % NST) * SB;
-    uint64_t* bar = &bars[r % NST];
-    if (!slot_ok(a, slot)) {
-      mbar_arrive_expect_tx(bar, 0);
-      return;
+  if (warp == kGuConsumers) {  // producer
+    if (lane == 0) {
+      const uint32_t sbb = 8u * a.ng_gu * 4u;
+      for (int r = 0; r < my_items; ++r) {
+        const int s = r % NST;
+        if (r >= NST && !mbar_wait_bounded(&empty[s], (uint32_t)(((r / NST) - 1) & 1))) {
+          if (a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
+          // the consumers will time out on full[s]; nothing more is issued
+          break;
+        }
+        const int item = i0 + r;
+        const int jt = item % jt_n;
+        const int slot = a.table[a.active[a.pass_begin + item / jt_n]];
+        uint8_t* st = smem + (size_t)s * SB;
+        if (!slot_ok(a, slot)) {
+          mbar_arrive_expect_tx(&full[s], 0);
+          continue;
+        }
+        const uint8_t* base = a.pool + (int64_t)slot * a.slot_bytes;
+        mbar_arrive_expect_tx(&full[s], 16u * (uint32_t)a.rb_gu + 2u * sbb);
+        for (int rr = 0; rr < 16; ++rr) {
+          const int grow = (rr < 8 ? 0 : a.I) + jt * 8 + (rr & 7);
+          bulk_g2s(st + rr * SR, base + a.q_gu + (int64_t)grow * a.rb_gu, (uint32_t)a.rb_gu, &full[s]);
+        }
+        uint8_t* sbd = st + 16 * SR;
+        bulk_g2s(sbd, base + a.sb_gu + (int64_t)jt * sbb, sbb, &full[s]);
+        bulk_g2s(sbd + sbb, base + a.sb_gu + (int64_t)(a.I + jt * 8) * a.ng_gu * 4, sbb, &full[s]);
+      }
     }
-    const uint8_t* base = a.pool + (int64_t)slot * a.slot_bytes;
-    mbar_arrive_expect_tx(bar, 16u * (uint32_t)a.rb_gu + 2u * sbb);
-    for (int rr = 0; rr < 16; ++rr) {
-      const int grow = (rr < 8 ? 0 : a.I) + jt * 8 + (rr & 7);
-      bulk_g2s(st + rr * SR, base + a.q_gu + (int64_t)grow * a.rb_gu, (uint32_t)a.rb_gu, bar);
-    }
-    uint8_t* sbd = st + 16 * SR;
-    bulk_g2s(sbd, base + a.sb_gu + (int64_t)jt * sbb, sbb, bar);
-    bulk_g2s(sbd + sbb, base + a.sb_gu + (int64_t)(a.I + jt * 8) * a.ng_gu * 4, sbb, bar);
-  };
-  if (tid == 0)
-    for (int r = 0; r < NST && r < my_items; ++r) issue(r);
+    return;
+  }
 
+  // consumers
   uint32_t bf[BPW][8][2];
   float xs[BPW][8 / GS][2], xo[BPW][8 / GS][2];
   int cached_tok = -2;
   bool timed_out = false;
+  int nent = 0;  // entries in the current reduction batch
+
+  auto flush = [&]() {
+    consumers_sync(kGuConsumers * 32);
+    for (int idx = tid; idx < nent * 64; idx += kGuConsumers * 32) {
+      const int en = idx >> 6, j = (idx >> 3) & 7, n = idx & 7;
+      const RedMeta m = meta[en];
+      if (n >= m.ntok) continue;
+      const int src = 4 * j + (n >> 1), c = n & 1;
+      const float* rp = red + (size_t)en * kGuConsumers * 32 * 4;
+      float gate = 0.f, up = 0.f;
+#pragma unroll
+      for (int w = 0; w < kGuConsumers; ++w) {
+        gate += rp[(w * 32 + src) * 4 + c];
+        up += rp[(w * 32 + src) * 4 + 2 + c];
+      }
+      const float hv = gate / (1.0f + expf(-gate)) * up;
+      a.h[(int64_t)(m.pos + n) * a.I + m.jt * 8 + j] = f32_to_bf16_rne(hv);
+    }
+    consumers_sync(kGuConsumers * 32);
+    nent = 0;
+  };
 
   for (int r = 0; r < my_items; ++r) {
-    const int item = (int)blockIdx.x + r * (int)gridDim.x;
+    const int s = r % NST;
+    const int item = i0 + r;
     const int jt = item % jt_n;
     const int e = a.active[a.pass_begin + item / jt_n];
     const int slot = a.table[e];
     const bool ok = slot_ok(a, slot);
-    if (!ok && tid == 0) flag_slot(a, slot);
-    const uint8_t* st = smem + (size_t)(r % NST) * SB;
-    const bool arrived = mbar_wait_bounded(&bars[r % NST], (uint32_t)((r / NST) & 1));
-    if (__syncthreads_or(!arrived)) {
-      timed_out = true;
-      break;
-    }
+    if (!ok && tid == 0 && jt == 0) flag_slot(a, slot);
+    // a wait that runs out marks the warp; it keeps walking the items (no
+    // waits, no math) so that every consumer reaches the same batch barriers
+    if (!timed_out && !mbar_wait_bounded(&full[s], (uint32_t)((r / NST) & 1))) timed_out = true;
+    const uint8_t* st = smem + (size_t)s * SB;
     const uint32_t* sbs = reinterpret_cast<const uint32_t*>(st + 16 * SR);
-    const int pos0 = a.offsets[e], cnt_e = a.offsets[e + 1] - pos0;
-    for (int tt = 0; ok && tt * 8 < cnt_e; ++tt) {
+    const int pos0 = a.offsets[e], cnt_e = ok ? a.offsets[e + 1] - pos0 : 0;
+    for (int tt = 0; tt * 8 < cnt_e; ++tt) {
       const int ntok = min(8, cnt_e - tt * 8);
       const int my_tok = g8 < ntok ? a.pairs[pos0 + tt * 8 + g8] / a.k : -1;
       if (!__all_sync(0xffffffffu, my_tok == cached_tok)) {
@@ -220,166 +281,166 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_gu_kernel(const FfnArgs a) {
 #pragma unroll
       for (int bi = 0; bi < BPW; ++bi) {
         const int kb = warp * BPW + bi;
-        if (kb < a.nblk_gu)
+        if (kb < a.nblk_gu && !timed_out)
           block_mma<B, GS>(st + g8 * SR, st + (8 + g8) * SR, sbs + g8 * a.ng_gu, sbs + (8 + g8) * a.ng_gu, kb, t4,
                            bf[bi], xs[bi], xo[bi], acc);
       }
-      *reinterpret_cast<float4*>(&red[(warp * 32 + lane) * 4]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      __syncthreads();
-      if (tid < 64) {
-        const int j = tid >> 3, n = tid & 7;
-        const int src = 4 * j + (n >> 1), c = n & 1;
-        float gate = 0.f, up = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-          gate += red[(w * 32 + src) * 4 + c];
-          up += red[(w * 32 + src) * 4 + 2 + c];
-        }
-        if (n < ntok) {
-          const float hv = gate / (1.0f + expf(-gate)) * up;
-          a.h[(int64_t)(pos0 + tt * 8 + n) * a.I + jt * 8 + j] = f32_to_bf16_rne(hv);
-        }
-      }
-      __syncthreads();
+      *reinterpret_cast<float4*>(&red[(((size_t)nent * kGuConsumers + warp) * 32 + lane) * 4]) =
+          make_float4(acc[0], acc[1], acc[2], acc[3]);
+      if (warp == 0 && lane == 0) meta[nent] = RedMeta{pos0 + tt * 8, ntok, jt, 0};
+      if (++nent == kRedBatch) flush();
     }
-    __syncthreads();
-    if (tid == 0 && r + NST < my_items) issue(r + NST);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
   }
-  if (timed_out) {
-    if (tid == 0) {
-      if (a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
-      // drain what is still in flight before the CTA's shared memory goes away
-      for (int s = 0; s < NST; ++s) {
-        mbar_wait_bounded(&bars[s], 0u, 100000000ull);
-        mbar_wait_bounded(&bars[s], 1u, 100000000ull);
-      }
-    }
-    __syncthreads();
-  }
+  // every consumer warp reaches here with the same nent (same items, same order)
+  if (nent > 0) flush();
+  if (timed_out && lane == 0 && a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
 }
 
 // ---------------------------------------------------------------------------
-// down (+ combine).  CTA owns 16 output rows; warp w runs the pass's experts
-// w, w+8, ...; partial sums per warp are added in warp order (deterministic).
-// FUSED: y[t][rows] += sum_j w[t,j] o_{t,j}   (T <= 64)
-// else : o[pair][rows] = o_{t,j}   (combined by combine_kernel)
+// down (+ combine).  CTA owns 16 output rows.  Warp 4 is the producer: it
+// streams the pass's experts' 16-row slices into a ring of stages as soon as
+// the CTA starts -- before waiting for the gate/up kernel, since the slots do
+// not depend on it.  Warps 0-3 split K (128-blocks round-robin) over every
+// expert of the pass.
+// FUSED (T <= 64): y[t][rows] += sum_j w[t,j] o_{t,j}   (deterministic order)
+// else           : o[pair][rows] = o_{t,j}   (combined by combine_kernel)
 // ---------------------------------------------------------------------------
-constexpr int kDownStages = 2;
+constexpr int kDnConsumers = 4;
+constexpr int kDnThreads = (kDnConsumers + 1) * 32;
 
 template <int B, int GS, bool FUSED>
-__global__ void __launch_bounds__(kThreads, 1) ffn_down_kernel(const FfnArgs a) {
+__global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, t4 = lane & 3, g8 = lane >> 2;
-  const int SB = a.d_stage_bytes, SR = a.sr_d;
-  uint8_t* my_stages = smem + (size_t)warp * kDownStages * SB;
-  float* ypart = reinterpret_cast<float*>(smem + (size_t)kWarps * kDownStages * SB);  // [8][T][16]
-  const int ypart_n = FUSED ? kWarps * a.T * 16 : 0;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ypart + ypart_n);  // [8][kDownStages]
-  uint64_t* my_bars = bars + warp * kDownStages;
+  const int NST = a.d_nstage, SB = a.d_stage_bytes, SR = a.sr_d;
+  float* ypart = reinterpret_cast<float*>(smem + (size_t)NST * SB);  // [4 warps][T][16]
+  const int ypart_n = FUSED ? kDnConsumers * a.T * 16 : 0;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ypart + ypart_n);
+  uint64_t* empty = full + NST;
 
-  pdl_wait();
-  const int n_act = pass_count(a);
+  // the pass's experts and their slots were written before the gate/up kernel
+  // started, so they can be read before waiting on it
+  int n_act = *a.n_active - a.pass_begin;
+  if (n_act > a.pass_len) n_act = a.pass_len;
   const int n_rt = a.H / 16;
-  if ((int)blockIdx.x >= n_rt || n_act == 0) return;
-  if (lane == 0) {
-    for (int s = 0; s < kDownStages; ++s) mbar_init(&my_bars[s], 1);
+  const int rt = blockIdx.x;
+  if (rt >= n_rt || n_act <= 0) {
+    pdl_wait();
+    return;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kDnConsumers);
+    }
     fence_barrier_init();
   }
-  __syncwarp();
-  const uint32_t sbb = 16u * a.ng_d * 4u;
-  const int my_n = n_act > warp ? (n_act - 1 - warp) / kWarps + 1 : 0;
-  int seq = 0;  // items consumed by this warp so far (all row tiles)
-  bool timed_out = false;
+  __syncthreads();
 
-  auto issue = [&](int rt, int r, int sq) {
-    const int e = a.active[a.pass_begin + warp + kWarps * r];
-    const int slot = a.table[e];
-    uint8_t* st = my_stages + (size_t)(sq % kDownStages) * SB;
-    uint64_t* bar = &my_bars[sq % kDownStages];
-    if (!slot_ok(a, slot)) {
-      mbar_arrive_expect_tx(bar, 0);
-      return;
-    }
-    const uint8_t* base = a.pool + (int64_t)slot * a.slot_bytes;
-    mbar_arrive_expect_tx(bar, 16u * (uint32_t)a.rb_d + sbb);
-    for (int rr = 0; rr < 16; ++rr)
-      bulk_g2s(st + rr * SR, base + a.q_d + (int64_t)(rt * 16 + rr) * a.rb_d, (uint32_t)a.rb_d, bar);
-    bulk_g2s(st + 16 * SR, base + a.sb_d + (int64_t)rt * sbb, sbb, bar);
-  };
-
-  for (int rt = blockIdx.x; rt < n_rt && !timed_out; rt += gridDim.x) {
-    if (FUSED)
-      for (int i = tid; i < ypart_n; i += kThreads) ypart[i] = 0.f;
-    __syncthreads();
-    if (lane == 0)
-      for (int r = 0; r < kDownStages && r < my_n; ++r) issue(rt, r, seq + r);
-    for (int r = 0; r < my_n; ++r) {
-      const int sq = seq + r;
-      const int e = a.active[a.pass_begin + warp + kWarps * r];
-      const int slot = a.table[e];
-      const bool ok = slot_ok(a, slot);
-      if (!ok && lane == 0 && rt == (int)blockIdx.x) flag_slot(a, slot);
-      if (!mbar_wait_bounded(&my_bars[sq % kDownStages], (uint32_t)((sq / kDownStages) & 1))) {
-        timed_out = true;
-        break;
-      }
-      const uint8_t* st = my_stages + (size_t)(sq % kDownStages) * SB;
-      const uint32_t* sbs = reinterpret_cast<const uint32_t*>(st + 16 * SR);
-      const int pos0 = a.offsets[e], cnt_e = a.offsets[e + 1] - pos0;
-      for (int tt = 0; ok && tt * 8 < cnt_e; ++tt) {
-        const int ntok = min(8, cnt_e - tt * 8);
-        const uint16_t* hrow = g8 < ntok ? a.h + (int64_t)(pos0 + tt * 8 + g8) * a.I : nullptr;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int kb = 0; kb < a.nblk_d; ++kb) {
-          uint32_t bf[8][2];
-          float xs[8 / GS][2], xo[8 / GS][2];
-          load_b_block<B, GS>(hrow, kb, a.I, t4, bf, xs, xo);
-          block_mma<B, GS>(st + g8 * SR, st + (8 + g8) * SR, sbs + g8 * a.ng_d, sbs + (8 + g8) * a.ng_d, kb, t4, bf,
-                           xs, xo, acc);
+  if (warp == kDnConsumers) {  // producer
+    if (lane == 0) {
+      const uint32_t sbb = 16u * a.ng_d * 4u;
+      for (int r = 0; r < n_act; ++r) {
+        const int s = r % NST;
+        if (r >= NST && !mbar_wait_bounded(&empty[s], (uint32_t)(((r / NST) - 1) & 1))) {
+          if (a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
+          break;
         }
+        const int slot = a.table[a.active[a.pass_begin + r]];
+        uint8_t* st = smem + (size_t)s * SB;
+        if (!slot_ok(a, slot)) {
+          mbar_arrive_expect_tx(&full[s], 0);
+          continue;
+        }
+        const uint8_t* base = a.pool + (int64_t)slot * a.slot_bytes;
+        mbar_arrive_expect_tx(&full[s], 16u * (uint32_t)a.rb_d + sbb);
+        for (int rr = 0; rr < 16; ++rr)
+          bulk_g2s(st + rr * SR, base + a.q_d + (int64_t)(rt * 16 + rr) * a.rb_d, (uint32_t)a.rb_d, &full[s]);
+        bulk_g2s(st + 16 * SR, base + a.sb_d + (int64_t)rt * sbb, sbb, &full[s]);
+      }
+    }
+    pdl_wait();
+    return;
+  }
+
+  pdl_wait();  // h (gate/up output) and y are ready
+  if (FUSED) {
+    for (int i = tid; i < ypart_n; i += kDnConsumers * 32) ypart[i] = 0.f;
+    consumers_sync(kDnConsumers * 32);
+  }
+  bool timed_out = false;
+  float acc1[4] = {0.f, 0.f, 0.f, 0.f};  // T == 1: every expert feeds the same token
+  const bool single = FUSED && a.T == 1;
+  // FUSED: the 4 warps split K of every expert.  Otherwise each warp owns
+  // whole experts (r % 4 == warp), so o is written once, without atomics.
+  const int kb0 = FUSED ? warp : 0, kbs = FUSED ? kDnConsumers : 1;
+  for (int r = 0; r < n_act; ++r) {
+    const int s = r % NST;
+    const int e = a.active[a.pass_begin + r];
+    const bool ok = slot_ok(a, a.table[e]);
+    // every warp waits on every stage before releasing it, which keeps the
+    // phases of the empty barriers in order
+    if (!timed_out && !mbar_wait_bounded(&full[s], (uint32_t)((r / NST) & 1))) timed_out = true;
+    const uint8_t* st = smem + (size_t)s * SB;
+    const uint32_t* sbs = reinterpret_cast<const uint32_t*>(st + 16 * SR);
+    const bool mine = FUSED || (r % kDnConsumers) == warp;
+    const int pos0 = a.offsets[e], cnt_e = (ok && mine && !timed_out) ? a.offsets[e + 1] - pos0 : 0;
+    for (int tt = 0; tt * 8 < cnt_e; ++tt) {
+      const int ntok = min(8, cnt_e - tt * 8);
+      const uint16_t* hrow = g8 < ntok ? a.h + (int64_t)(pos0 + tt * 8 + g8) * a.I : nullptr;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int kb = kb0; kb < a.nblk_d; kb += kbs) {
+        uint32_t bf[8][2];
+        float xs[8 / GS][2], xo[8 / GS][2];
+        load_b_block<B, GS>(hrow, kb, a.I, t4, bf, xs, xo);
+        block_mma<B, GS>(st + g8 * SR, st + (8 + g8) * SR, sbs + g8 * a.ng_d, sbs + (8 + g8) * a.ng_d, kb, t4, bf,
+                         xs, xo, acc);
+      }
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int n = 2 * t4 + c;
-          if (n < ntok) {
-            const int pf = a.pairs[pos0 + tt * 8 + n];
-            if (FUSED) {
-              const int tok = pf / a.k;
-              const float wg = a.w[pf];
-              float* yp = ypart + ((size_t)warp * a.T + tok) * 16;
+      for (int c = 0; c < 2; ++c) {
+        const int n = 2 * t4 + c;
+        if (n < ntok) {
+          const int pf = a.pairs[pos0 + tt * 8 + n];
+          if (FUSED) {
+            const float wg = a.w[pf];
+            if (single) {
+              acc1[c] += wg * acc[c];
+              acc1[2 + c] += wg * acc[2 + c];
+            } else {
+              float* yp = ypart + ((size_t)warp * a.T + pf / a.k) * 16;
               yp[g8] += wg * acc[c];
               yp[8 + g8] += wg * acc[2 + c];
-            } else {
-              float* op = a.o + (int64_t)pf * a.H + rt * 16;
-              op[g8] = acc[c];
-              op[8 + g8] = acc[2 + c];
             }
+          } else {
+            float* op = a.o + (int64_t)pf * a.H + rt * 16;
+            op[g8] = acc[c];
+            op[8 + g8] = acc[2 + c];
           }
         }
       }
-      __syncwarp();
-      if (lane == 0 && r + kDownStages < my_n) issue(rt, r + kDownStages, sq + kDownStages);
     }
-    seq += my_n;
-    if (__syncthreads_or(timed_out)) {
-      timed_out = true;
-      break;
-    }
-    if (FUSED) {
-      for (int i = tid; i < a.T * 16; i += kThreads) {
-        const int tok = i >> 4, row = i & 15;
-        float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) s += ypart[((size_t)w * a.T + tok) * 16 + row];
-        a.y[(int64_t)tok * a.H + rt * 16 + row] += s;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+  if (timed_out && lane == 0 && a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
+  if (FUSED) {
+    consumers_sync(kDnConsumers * 32);  // all ypart updates done before the single-token write
+    if (single) {
+      // only column 0 (t4 == 0, c == 0) carries token 0
+      if (t4 == 0) {
+        ypart[(size_t)warp * 16 + g8] = acc1[0];
+        ypart[(size_t)warp * 16 + 8 + g8] = acc1[2];
       }
     }
-    __syncthreads();
-  }
-  if (timed_out && lane == 0) {
-    if (a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
-    for (int s = 0; s < kDownStages; ++s) {
-      mbar_wait_bounded(&my_bars[s], 0u, 100000000ull);
-      mbar_wait_bounded(&my_bars[s], 1u, 100000000ull);
+    consumers_sync(kDnConsumers * 32);
+    for (int i = tid; i < a.T * 16; i += kDnConsumers * 32) {
+      const int tok = i >> 4, row = i & 15;
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDnConsumers; ++w) sum += ypart[((size_t)w * a.T + tok) * 16 + row];
+      a.y[(int64_t)tok * a.H + rt * 16 + row] += sum;
     }
   }
 }
@@ -422,20 +483,34 @@ size_t ffn_ws_bytes(const moe_layer_desc& d, int T) {
   return b;
 }
 
+// Opt a kernel into the large dynamic shared-memory carve-out once per
+// (kernel, device); the attribute call is not free on the launch path.  Each
+// caller passes its own flag word (one per kernel instantiation).
+static cudaError_t ensure_smem_attr(const void* kern, int (&done_mask)[4]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 128 && ((__atomic_load_n(&done_mask[dev >> 5], __ATOMIC_RELAXED) >> (dev & 31)) & 1)) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e == cudaSuccess && dev < 128) __atomic_fetch_or(&done_mask[dev >> 5], 1 << (dev & 31), __ATOMIC_RELAXED);
+  return e;
+}
+
 template <int B, int BPW, int GS>
 static cudaError_t launch_gu(const FfnArgs& a, int grid, size_t smem, cudaStream_t st) {
-  auto kern = ffn_gu_kernel<B, BPW, GS>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static int done[4] = {0, 0, 0, 0};
+  const void* kern = reinterpret_cast<const void*>(ffn_gu_kernel<B, BPW, GS>);
+  cudaError_t e = ensure_smem_attr(kern, done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(reinterpret_cast<const void*>(kern), grid, kThreads, smem, st, a);
+  return launch_pdl(kern, grid, kGuThreads, smem, st, a);
 }
 
 template <int B, int GS, bool F>
 static cudaError_t launch_dn(const FfnArgs& a, int grid, size_t smem, cudaStream_t st) {
-  auto kern = ffn_down_kernel<B, GS, F>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static int done[4] = {0, 0, 0, 0};
+  const void* kern = reinterpret_cast<const void*>(ffn_down_kernel<B, GS, F>);
+  cudaError_t e = ensure_smem_attr(kern, done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(reinterpret_cast<const void*>(kern), grid, kThreads, smem, st, a);
+  return launch_pdl(kern, grid, kDnThreads, smem, st, a);
 }
 
 template <int B, int BPW>
@@ -468,8 +543,14 @@ static cudaError_t dn_by_bits(const FfnArgs& a, int bits, int gs, int grid, size
 
 bool ffn_decode_supported(const moe_layer_desc& d) {
   const int nblk = (int)(padded_k(d.H) / 128);
-  return nblk <= kWarps * 4 && d.H % 16 == 0 && d.I % 8 == 0;
+  return nblk <= kGuConsumers * 4 && d.H % 16 == 0 && d.I % 8 == 0;
 }
+
+// Shared-memory budgets: the gate/up and down kernels of one layer are sized
+// to be resident on an SM together (the down kernel starts early and streams
+// its weights while gate/up finishes).
+constexpr size_t kGuSmemCap = 150 * 1024;
+constexpr size_t kDnSmemCap = 72 * 1024;
 
 cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st) {
   const Layout& L = a.L;
@@ -489,31 +570,40 @@ cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, c
   a.d_stage_bytes = (int)round_up(16 * a.sr_d + 16 * L.ng_d * 4, 128);
   const int gs = d.group / 16;
   const int nblk = L.nblk_gu;
-  const int bpw = nblk <= kWarps ? 1 : nblk <= 2 * kWarps ? 2 : 4;
-  const size_t smem_cap = 200 * 1024;
-  const size_t red_bytes = kWarps * 32 * 4 * sizeof(float);
-  int nst = (int)((smem_cap - red_bytes - 8 * 16) / a.gu_stage_bytes);
-  if (nst > 8) nst = 8;
-  if (nst < 1) return cudaErrorInvalidConfiguration;
-  a.gu_nstage = nst;
-  const size_t gu_smem = (size_t)nst * a.gu_stage_bytes + red_bytes + (size_t)nst * 8;
+  const int bpw = nblk <= kGuConsumers ? 1 : nblk <= 2 * kGuConsumers ? 2 : 4;
   const int max_pass = a.pass_len < d.E ? a.pass_len : d.E;
+
+  // gate/up: 148 CTAs (or fewer items), stages for every item of a CTA if they fit
   const int64_t items = (int64_t)max_pass * (d.I / 8);
   int grid = (int)(items < num_sms ? items : num_sms);
   if (grid < 1) grid = 1;
+  const size_t red_bytes = (size_t)kRedBatch * kGuConsumers * 32 * 4 * sizeof(float) + kRedBatch * sizeof(RedMeta);
+  const int64_t items_per_cta = (items + grid - 1) / grid;
+  int nst = (int)((kGuSmemCap - red_bytes) / (a.gu_stage_bytes + 16));
+  if (nst > items_per_cta) nst = (int)items_per_cta;
+  if (nst > 32) nst = 32;
+  if (nst < 1) return cudaErrorInvalidConfiguration;
+  a.gu_nstage = nst;
+  const size_t gu_smem = (size_t)nst * a.gu_stage_bytes + red_bytes + (size_t)nst * 16;
+
+  const bool fused = a.T <= kFusedMaxTokens;
+  const size_t ypart = fused ? (size_t)kDnConsumers * a.T * 16 * sizeof(float) : 0;
+  int dnst = (int)((kDnSmemCap - ypart) / (a.d_stage_bytes + 16));
+  if (dnst > max_pass) dnst = max_pass;
+  if (dnst > 32) dnst = 32;
+  if (dnst < 2) dnst = 2;
+  a.d_nstage = dnst;
+  const size_t dn_smem = (size_t)dnst * a.d_stage_bytes + ypart + (size_t)dnst * 16;
+
   cudaError_t e = cudaSuccess;
   if (d.bits_gu == 3) e = gu_by_bpw<3>(a, bpw, gs, grid, gu_smem, st);
   else if (d.bits_gu == 4) e = gu_by_bpw<4>(a, bpw, gs, grid, gu_smem, st);
   else e = gu_by_bpw<6>(a, bpw, gs, grid, gu_smem, st);
   if (e != cudaSuccess) return e;
 
-  const bool fused = a.T <= kFusedMaxTokens;
-  const size_t dn_smem = (size_t)kWarps * kDownStages * a.d_stage_bytes +
-                         (fused ? (size_t)kWarps * a.T * 16 * sizeof(float) : 0) + kWarps * kDownStages * 8;
   const int n_rt = d.H / 16;
-  const int dgrid = n_rt < num_sms ? n_rt : num_sms;
-  if (fused) e = dn_by_bits<true>(a, d.bits_down, gs, dgrid, dn_smem, st);
-  else e = dn_by_bits<false>(a, d.bits_down, gs, dgrid, dn_smem, st);
+  if (fused) e = dn_by_bits<true>(a, d.bits_down, gs, n_rt, dn_smem, st);
+  else e = dn_by_bits<false>(a, d.bits_down, gs, n_rt, dn_smem, st);
   if (e != cudaSuccess || fused) return e;
   const int64_t total = (int64_t)a.T * d.H;
   int cgrid = (int)((total + 255) / 256);

@@ -36,7 +36,7 @@ struct FfnArgs {
   int64_t q_gu, q_d, sb_gu, sb_d, rb_gu, rb_d;
   int ng_gu, ng_d, nblk_gu, nblk_d;
   int sr_gu, sr_d;
-  int gu_stage_bytes, d_stage_bytes, gu_nstage;
+  int gu_stage_bytes, d_stage_bytes, gu_nstage, d_nstage;
 };
 
 // Launch with programmatic stream serialization, so the kernel's CTAs can be

@@ -16,6 +16,7 @@ struct moe_cache {
   std::vector<std::vector<int32_t>> owner;  // [layer][S]: expert in slot base+i, or -1
   std::vector<std::vector<int64_t>> stamp;  // [layer][S]: last use, 0 = never used
   std::vector<uint8_t> used;                // scratch [S]
+  std::vector<int32_t> resident;            // [layer]: experts with a slot
   int64_t clock = 0, hits = 0, misses = 0, evictions = 0;
 };
 
@@ -49,6 +50,7 @@ moe_status moe_cache_create(int32_t E, int32_t n_layers, const int32_t* layer_cl
   c->owner.assign(n_layers, std::vector<int32_t>(slots_per_layer, -1));
   c->stamp.assign(n_layers, std::vector<int64_t>(slots_per_layer, 0));
   c->used.assign(slots_per_layer, 0);
+  c->resident.assign(n_layers, 0);
   *out = c;
   return MOE_OK;
 }
@@ -78,10 +80,17 @@ moe_status moe_cache_place(moe_cache* c, int32_t layer, const int32_t* experts, 
     if (e < 0 || e >= c->E || s < 0 || s >= c->S) return MOE_ERR_INVALID;
     auto& tab = c->table[layer];
     auto& own = c->owner[layer];
-    if (own[s] >= 0) tab[own[s]] = -1;
-    if (tab[e] >= 0) own[tab[e] - base] = -1;
+    if (own[s] >= 0) {
+      tab[own[s]] = -1;
+      --c->resident[layer];
+    }
+    if (tab[e] >= 0) {
+      own[tab[e] - base] = -1;
+      --c->resident[layer];
+    }
     own[s] = e;
     tab[e] = base + s;
+    ++c->resident[layer];
     c->stamp[layer][s] = ++c->clock;  // placed slots are more recent than empty ones
   }
   return MOE_OK;
@@ -125,15 +134,22 @@ moe_status moe_cache_step(moe_cache* c, int32_t layer, const int32_t* pass_exper
     if (own[best] >= 0) {
       tab[own[best]] = -1;
       ++c->evictions;
+      --c->resident[layer];
     }
     own[best] = e;
     tab[e] = base + best;
+    ++c->resident[layer];
     c->used[best] = 1;
     stp[best] = ++c->clock;
     out_slots[n++] = base + best;
   }
   *n_out = n;
   return st;
+}
+
+int32_t moe_cache_resident(const moe_cache* c, int32_t layer) {
+  if (!c || layer < 0 || layer >= c->n_layers) return -1;
+  return c->resident[layer];
 }
 
 void moe_cache_stats(const moe_cache* c, int64_t* hits, int64_t* misses, int64_t* evictions) {

@@ -23,13 +23,15 @@ ABI_SYMBOLS = [
     "moe_install_slots", "moe_expert_ffn", "moe_dequant_slot", "moe_quantize_rows", "moe_exp_portable",
     "moe_status_string", "moe_cache_create", "moe_cache_destroy", "moe_cache_table", "moe_cache_layer_base",
     "moe_cache_class_slots", "moe_cache_place", "moe_cache_step", "moe_cache_stats",
-    "moe_expert_ffn_noalloc", "moe_noalloc_scratch_bytes",
+    "moe_expert_ffn_noalloc", "moe_noalloc_scratch_bytes", "moe_cache_resident", "moe_decode_layer",
+    "moe_last_cuda_error",
 ]
 
 
 class MoeError(RuntimeError):
     def __init__(self, status: int, where: str):
-        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        extra = f" [{lib().moe_last_cuda_error().decode()}]" if status == MOE_ERR_CUDA else ""
+        super().__init__(f"{where}: {status_string(status)} (status {status}){extra}")
         self.status = status
 
 
@@ -40,6 +42,18 @@ class LayerDesc(C.Structure):
     def __repr__(self):
         return (f"LayerDesc(E={self.E}, k={self.k}, H={self.H}, I={self.I}, group={self.group}, "
                 f"bits_gu={self.bits_gu}, bits_down={self.bits_down})")
+
+
+class StepBuffers(C.Structure):
+    _fields_ = [("ids", C.c_void_p), ("w", C.c_void_p), ("offsets", C.c_void_p), ("pairs", C.c_void_p),
+                ("meta", C.c_void_p), ("meta_host", C.c_void_p), ("slots", C.c_void_p), ("dev_err", C.c_void_p),
+                ("ws", C.c_void_p), ("ws_bytes", C.c_size_t), ("max_tokens", C.c_int32)]
+
+
+class LayerCtx(C.Structure):
+    _fields_ = [("desc", C.POINTER(LayerDesc)), ("pool", C.c_void_p), ("n_slots", C.c_int32),
+                ("slot_bytes", C.c_size_t), ("table_dev", C.c_void_p), ("table_stage", C.c_void_p),
+                ("bank_rows", C.POINTER(C.c_void_p))]
 
 
 class SlotLayout(C.Structure):
@@ -73,6 +87,7 @@ def lib():
             "moe_quantize_rows": (C.c_int, [P, i32, i32, i32, i32, P, P, P]),
             "moe_exp_portable": (C.c_int, [P, i64, P, P]),
             "moe_status_string": (C.c_char_p, [C.c_int]),
+            "moe_last_cuda_error": (C.c_char_p, []),
             "moe_cache_create": (C.c_int, [i32, i32, P, i32, C.POINTER(P)]),
             "moe_cache_destroy": (None, [P]),
             "moe_cache_table": (C.POINTER(i32), [P, i32]),
@@ -81,6 +96,9 @@ def lib():
             "moe_cache_place": (C.c_int, [P, i32, P, P, i32]),
             "moe_cache_step": (C.c_int, [P, i32, P, i32, P, P, P]),
             "moe_cache_stats": (None, [P, P, P, P]),
+            "moe_cache_resident": (i32, [P, i32]),
+            "moe_decode_layer": (C.c_int, [P, i32, C.POINTER(LayerCtx), C.POINTER(StepBuffers), P, P, i32, f32, P,
+                                           P, P, P, C.POINTER(i32)]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -255,7 +273,21 @@ class SlotCache:
             _ck(st, "moe_cache_step")
         return st, [(self._out_e[i], self._out_s[i]) for i in range(nout.value)]
 
+    def resident(self, layer: int) -> int:
+        return int(lib().moe_cache_resident(self._h, layer))
+
     def stats(self):
         h, m, e = C.c_int64(), C.c_int64(), C.c_int64()
         lib().moe_cache_stats(self._h, C.byref(h), C.byref(m), C.byref(e))
         return h.value, m.value, e.value
+
+
+def moe_decode_layer(cache: "SlotCache", layer: int, ctx: LayerCtx, bufs: StepBuffers, x, logits, T: int, L: float,
+                     y, stream, side, installed) -> int:
+    """One decode layer through the native driver; returns experts installed."""
+    n = C.c_int32(0)
+    ev = installed if isinstance(installed, int) else installed.cuda_event
+    _ck(lib().moe_decode_layer(cache._h, int(layer), C.byref(ctx), C.byref(bufs), _ptr(x), _ptr(logits), int(T),
+                               float(L), _ptr(y), _stream(stream), _stream(side), ev, C.byref(n)),
+        "moe_decode_layer")
+    return n.value

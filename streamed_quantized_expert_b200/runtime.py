@@ -101,7 +101,21 @@ class Streamer:
         self.installed_bytes = 0
         self.installs = 0
         self.launches = 0          # libmoe kernel launches issued (for reporting)
-        self._full = [False] * self.n_layers
+        # native per-layer driver state
+        self.installed.record(self.side)  # materialise the event
+        self._bufs = ops.StepBuffers(self.ids.data_ptr(), self.w.data_ptr(), self.offsets.data_ptr(),
+                                     self.pairs.data_ptr(), self.meta.data_ptr(), self.meta_pin.data_ptr(),
+                                     self.slots.data_ptr(), self.dev_err.data_ptr(), self.ws.data_ptr(),
+                                     self.ws_bytes, max_tokens)
+        self._ctx = []
+        self._rows = []
+        for l, spec in enumerate(layers):
+            rows = (C.c_void_p * self.E)(*[self._row_addr(l, e) for e in range(self.E)])
+            self._rows.append(rows)
+            self._ctx.append(ops.LayerCtx(C.pointer(spec.desc), self.pools[self.layer_class[l]].data_ptr(),
+                                          self.class_n_slots[self.layer_class[l]],
+                                          self.class_bytes[self.layer_class[l]], self.table_dev[l].data_ptr(),
+                                          self.table_pin[l].data_ptr(), rows))
         self.ffn_events = None     # list to collect (start, end) CUDA events around FFN calls
 
     # -- views into meta --------------------------------------------------
@@ -147,10 +161,9 @@ class Streamer:
                               self.side, None)
         self._upload_table(layer, self.side)
         self.side.synchronize()
-        self._full[layer] = self.S >= self.E and all(v >= 0 for v in self.cache.table(layer))
 
     def fully_resident(self, layer: int) -> bool:
-        return self._full[layer]
+        return self.cache.resident(layer) >= self.E
 
     def _install_pass(self, layer: int, pass_experts) -> int:
         st, inst = self.cache.step(layer, pass_experts)
@@ -199,7 +212,20 @@ class Streamer:
             self.ffn_events.append(ev)
 
     def decode_layer(self, layer: int, x, logits, T: int, L: float = 0.0, y=None):
-        """One decode layer (T <= 64 tokens); returns y fp32 [T, H] (device)."""
+        """One decode layer (T <= 64 tokens) through the native driver
+        (moe_decode_layer); returns y fp32 [T, H] (device)."""
+        y = self.y[:T] if y is None else y
+        full = self.cache.resident(layer) >= self.E
+        n = ops.moe_decode_layer(self.cache, layer, self._ctx[layer], self._bufs, x, logits, T, L, y, self.stream,
+                                 self.side, self.installed)
+        if n:
+            self.installs += n
+            self.installed_bytes += n * self.class_bytes[self.layer_class[layer]]
+        self.launches += 4 + (0 if full else 1) + (0 if T * self.k <= 1024 else 2)
+        return y
+
+    def decode_layer_steps(self, layer: int, x, logits, T: int, L: float = 0.0, y=None):
+        """Same as decode_layer, one ABI call at a time from Python."""
         y = self.y[:T] if y is None else y
         s = self.stream
         self.route_sort(layer, x, logits, T, L)
