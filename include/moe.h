@@ -52,7 +52,13 @@
  *   codes; unit p holds, for s = 0..7, the input pairs (128B+16s+2p, +1) and
  *   (128B+16s+2p+8, +1) as pair indices 2s and 2s+1, the even input in the
  *   low 16-bit half of a 32-bit word and the odd input at the same offset in
- *   the high half.  A unit is b little-endian words:
+ *   the high half.  Rows are stored in groups of 8 consecutive rows
+ *   (8*Kp*b/8 bytes per group); inside a group, unit u = 4B+p of row r (0..7)
+ *   is at unit position 8u + sigma(u, r) (4b bytes per position), sigma = r
+ *   for b=3, (r + 2(u mod 4)) mod 8 for b=4, (r + 4((u/2) mod 2)) mod 8 for
+ *   b=6 -- so one tile of rows is one contiguous copy and the GEMV's
+ *   per-thread unit loads from shared memory are bank-conflict free.  A unit
+ *   is b little-endian words:
  *     b=4: pair i in word i/4, bits 4*(i%4)..+3
  *     b=3: pair i<15 in word i/5, bits 3*(i%5)..+2; pair 15: bit j of the
  *          code is bit 15 of word j
@@ -61,9 +67,10 @@
  *          word 4+m/2
  *   Per group of g inputs, one 32-bit word: bf16 scale (low half), bf16 bias
  *   (high half).  A slot is four sections, each 256-byte aligned:
- *     q_gate_up [2I rows][Kp(H)*b_gu/8]   rows 0..I-1 gate, I..2I-1 up
+ *     q_gate_up [2I rows][Kp(H)*b_gu/8]   storage row order: blocks of 16
+ *               rows, block m = gate rows 8m..8m+7 then up rows 8m..8m+7
  *     q_down    [H rows][Kp(I)*b_d/8]
- *     sb_gate_up[2I rows][Kp(H)/g] words
+ *     sb_gate_up[2I rows][Kp(H)/g] words (same row order as q_gate_up)
  *     sb_down   [H rows][Kp(I)/g] words
  *   slot_bytes = end of the last section rounded to 256.  Dequantised weight
  *   = fmaf(scale, q, bias) in fp32 (one rounding).
@@ -235,12 +242,17 @@ moe_status moe_dequant_slot(const void* pool, int32_t slot, const moe_layer_desc
                             uint16_t* out_bf16, cudaStream_t stream);
 
 /* Input preparation (the RFC's one-time quantize_experts, on the GPU):
- * quantise rows of fp32 weights w [rows, K] into the slot row format:
+ * quantise rows of fp32 weights w [rows, K] into the slot format:
  * per group scale = bf16((max-min)/(2^b-1)), bias = bf16(min),
  * q = clamp(rint((w - bias)/scale), 0, 2^b-1) (q = 0 if scale = 0).
- *   q  device [rows][Kp*bits/8] bytes;  sb device uint32 [rows][Kp/group] */
-moe_status moe_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t group, int32_t bits, uint8_t* q,
-                             uint32_t* sb, cudaStream_t stream);
+ *   rows       a multiple of 8
+ *   gate_up_I  0: row r of w is storage row r; I > 0: w is a gate/up matrix
+ *              [2I, K] (gate rows then up rows) and its rows go to their
+ *              storage rows (blocks of 8 gate + 8 up rows)
+ *   q  device [rows * Kp*bits/8] bytes (8-row groups, see the format above)
+ *   sb device uint32 [rows][Kp/group] (storage row order) */
+moe_status moe_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t group, int32_t bits,
+                             int32_t gate_up_I, uint8_t* q, uint32_t* sb, cudaStream_t stream);
 
 /* Test: the fp32 exp used by moe_route, elementwise on n device floats. */
 moe_status moe_exp_portable(const float* x, int64_t n, float* out, cudaStream_t stream);

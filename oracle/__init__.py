@@ -55,8 +55,9 @@ def lib():
             "orc_row_bytes": (i64, [i32, i32]),
             "orc_row_groups": (i64, [i32, i32]),
             "orc_slot_layout": (None, [i32, i32, i32, i32, i32, P]),
-            "orc_get_code": (i32, [P, i32, i32]),
-            "orc_set_code": (None, [P, i32, i32, i32]),
+            "orc_get_code": (i32, [P, i32, i32, i32, i32]),
+            "orc_set_code": (None, [P, i32, i32, i32, i32, i32]),
+            "orc_gate_up_row": (i32, [i32, i32]),
             "orc_quantize_rows": (None, [P, i32, i32, i32, i32, P, P]),
             "orc_dequant_rows": (None, [P, P, i32, i32, i32, i32, P]),
             "orc_dequant_slot": (None, [P, i32, i32, i32, i32, i32, P, P]),
@@ -162,20 +163,37 @@ def slot_bytes(H: int, I: int, g: int, b_gu: int, b_d: int) -> int:
     return slot_layout(H, I, g, b_gu, b_d)[1]
 
 
-def get_code(row: np.ndarray, k: int, b: int) -> int:
-    row = np.ascontiguousarray(row, dtype=np.uint8)
-    return int(lib().orc_get_code(_p(row), k, b))
+def get_code(proj: np.ndarray, K: int, row: int, k: int, b: int) -> int:
+    """Code of input k of row `row` of a projection (bytes of all its rows)."""
+    proj = np.ascontiguousarray(proj, dtype=np.uint8)
+    return int(lib().orc_get_code(_p(proj), K, row, k, b))
 
 
-def set_code(row: np.ndarray, k: int, b: int, q: int) -> None:
-    assert row.dtype == np.uint8 and row.flags["C_CONTIGUOUS"]
-    lib().orc_set_code(_p(row), k, b, q)
+def set_code(proj: np.ndarray, K: int, row: int, k: int, b: int, q: int) -> None:
+    assert proj.dtype == np.uint8 and proj.flags["C_CONTIGUOUS"]
+    lib().orc_set_code(_p(proj), K, row, k, b, q)
+
+
+def gate_up_row(R: int, I: int) -> int:
+    """Storage row of logical gate/up row R."""
+    return int(lib().orc_gate_up_row(R, I))
+
+
+def gate_up_order(I: int) -> np.ndarray:
+    """order[p] = logical gate/up row stored at storage row p."""
+    order = np.empty(2 * I, np.int64)
+    for R in range(2 * I):
+        order[gate_up_row(R, I)] = R
+    return order
 
 
 def quantize_rows(w: np.ndarray, g: int, b: int):
-    """w fp32 [rows, K] -> (q uint8 [rows, row_bytes], sb uint32 [rows, row_groups])."""
+    """w fp32 [rows, K] (storage order, rows a multiple of 8) -> (q uint8
+    [rows, row_bytes] -- rows interleaved in groups of 8, see oracle.c --,
+    sb uint32 [rows, row_groups])."""
     w = np.ascontiguousarray(w, dtype=np.float32)
     rows, K = w.shape
+    assert rows % 8 == 0, "rows come in groups of 8"
     q = np.zeros((rows, row_bytes(K, b)), np.uint8)
     sb = np.zeros((rows, row_groups(K, g)), np.uint32)
     lib().orc_quantize_rows(_p(w), rows, K, g, b, _p(q), _p(sb))
@@ -198,7 +216,7 @@ def build_slot(w_gu: np.ndarray, w_d: np.ndarray, g: int, b_gu: int, b_d: int) -
     assert w_d.shape == (H, I)
     off, nbytes = slot_layout(H, I, g, b_gu, b_d)
     slot = np.zeros(nbytes, np.uint8)
-    qg, sg = quantize_rows(w_gu, g, b_gu)
+    qg, sg = quantize_rows(np.ascontiguousarray(w_gu[gate_up_order(I)]), g, b_gu)
     qd, sd = quantize_rows(w_d, g, b_d)
     slot[off[0]: off[0] + qg.size] = qg.reshape(-1)
     slot[off[1]: off[1] + qd.size] = qd.reshape(-1)

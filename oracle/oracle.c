@@ -246,9 +246,9 @@ void orc_slot_lookup(const int32_t* table, const int32_t* active, int32_t n_acti
  *
  * A weight row of K inputs is padded to Kp = K rounded up to 128; padded
  * groups have scale = bias = 0 (so they dequantise to exactly 0).  The row is
- * cut into blocks of 128 inputs; block B is stored as 4 units, unit p in
- * 0..3, each unit 32 codes in b 32-bit little-endian words (4b bytes).
- * Unit p of block B holds, for s = 0..7, the two input pairs
+ * cut into blocks of 128 inputs; block B is 4 units, unit p in 0..3, each unit
+ * 32 codes in b 32-bit little-endian words (4b bytes).  Unit p of block B
+ * holds, for s = 0..7, the two input pairs
  *     (128B + 16s + 2p,     +1)      -> pair index i = 2s
  *     (128B + 16s + 2p + 8, +1)      -> pair index i = 2s + 1
  * The even input of a pair sits in the low 16-bit half of a word, the odd
@@ -259,15 +259,21 @@ void orc_slot_lookup(const int32_t* table, const int32_t* active, int32_t n_acti
  *   b = 6: pair i < 12 in word i/2 at bits 6*(i%2) .. +5;
  *          pair i >= 12, m = i - 12: code bits 0..3 at bits 12..15 of
  *          word m; code bits 4,5 at bits 12 + 2*(m%2) + {0,1} of word 4+m/2
- * Per group of g inputs (g in 32, 64, 128): a (scale, bias) pair of bf16,
- * stored as one 32-bit word, scale in the low half.
+ * Rows are stored in groups of 8 consecutive rows (8 * row_bytes bytes per
+ * group).  Inside a group, unit u (= 4B + p) of row r (0..7) sits at unit
+ * position 8u + sigma(u, r) (unit positions are 4b bytes apart), with
+ *   b = 3: sigma = r
+ *   b = 4: sigma = (r + 2 (u mod 4)) mod 8
+ *   b = 6: sigma = (r + 4 ((u / 2) mod 2)) mod 8
+ * Per group of g inputs: a (scale, bias) pair of bf16, stored as one 32-bit
+ * word, scale in the low half; row-major [rows][Kp/g].
  *
  * A slot (one expert) is four sections, each starting on a 256-byte
- * boundary:  q_gate_up [2I rows, Kp(H)*b_gu/8 bytes each] (rows 0..I-1 gate,
- * I..2I-1 up), q_down [H rows, Kp(I)*b_d/8 bytes], sb_gate_up [2I rows,
- * Kp(H)/g words], sb_down [H rows, Kp(I)/g words].  The slot's byte size is
- * the end of the last section rounded to 256 -- the "sum of its aligned read
- * windows" that keys its size class (1bit-MONSTER PR #137).
+ * boundary:  q_gate_up [2I rows] (row order: blocks of 16, block m = gate
+ * rows 8m..8m+7 then up rows 8m..8m+7), q_down [H rows], sb_gate_up [2I rows,
+ * same order], sb_down [H rows].  The slot's byte size is the end of the last
+ * section rounded to 256 -- the "sum of its aligned read windows" that keys
+ * its size class (1bit-MONSTER PR #137).
  */
 static int64_t orc_round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
@@ -294,16 +300,24 @@ void orc_slot_layout(int32_t H, int32_t I, int32_t g, int32_t b_gu, int32_t b_d,
   off[4] = o; /* slot bytes */
 }
 
-/* Bit position of code bit j of input k inside its row; word index + bit. */
-static void orc_code_bit(int32_t k, int32_t b, int32_t j, int64_t* word, int32_t* bit) {
+/* Position of code bit j of input k of row `row` of a projection whose rows
+ * are row_bytes long: byte offset of its 32-bit word from the projection's
+ * start, and the bit inside that word. */
+static void orc_code_bit(int32_t row, int64_t row_bytes, int32_t k, int32_t b, int32_t j, int64_t* word_byte,
+                         int32_t* bit) {
   int32_t blk = k / 128, kk = k % 128;
   int32_t s = kk / 16, r16 = kk % 16;
   int32_t h = r16 / 8;
   int32_t p = (r16 % 8) / 2;
   int32_t odd = k & 1;
   int32_t i = 2 * s + h;
-  int64_t unit = (int64_t)blk * 4 + p;
-  int64_t w0 = unit * b; /* first word of the unit */
+  int64_t u = (int64_t)blk * 4 + p;
+  int32_t r = row % 8;
+  int32_t sigma;
+  if (b == 3) sigma = r;
+  else if (b == 4) sigma = (r + 2 * (int32_t)(u % 4)) % 8;
+  else sigma = (r + 4 * (int32_t)((u / 2) % 2)) % 8;
+  int64_t pos = 8 * u + sigma; /* unit position inside the 8-row group */
   int32_t wi, bi;
   if (b == 4) {
     wi = i / 4;
@@ -331,44 +345,51 @@ static void orc_code_bit(int32_t k, int32_t b, int32_t j, int64_t* word, int32_t
       }
     }
   }
-  *word = w0 + wi;
+  *word_byte = (int64_t)(row / 8) * 8 * row_bytes + pos * 4 * b + 4 * wi;
   *bit = bi + (odd ? 16 : 0);
 }
 
-static uint32_t orc_load_word(const uint8_t* row, int64_t w) {
-  const uint8_t* p = row + 4 * w;
+static uint32_t orc_load_word(const uint8_t* p) {
   return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);
 }
 
-static void orc_store_word(uint8_t* row, int64_t w, uint32_t v) {
-  uint8_t* p = row + 4 * w;
+static void orc_store_word(uint8_t* p, uint32_t v) {
   p[0] = (uint8_t)v;
   p[1] = (uint8_t)(v >> 8);
   p[2] = (uint8_t)(v >> 16);
   p[3] = (uint8_t)(v >> 24);
 }
 
-int32_t orc_get_code(const uint8_t* row, int32_t k, int32_t b) {
+/* Code of input k of row `row` in a projection of K inputs per row. */
+int32_t orc_get_code(const uint8_t* proj, int32_t K, int32_t row, int32_t k, int32_t b) {
+  int64_t rb = orc_row_bytes(K, b);
   int32_t q = 0;
   for (int32_t j = 0; j < b; ++j) {
-    int64_t w;
+    int64_t wb;
     int32_t bit;
-    orc_code_bit(k, b, j, &w, &bit);
-    q |= (int32_t)((orc_load_word(row, w) >> bit) & 1u) << j;
+    orc_code_bit(row, rb, k, b, j, &wb, &bit);
+    q |= (int32_t)((orc_load_word(proj + wb) >> bit) & 1u) << j;
   }
   return q;
 }
 
-void orc_set_code(uint8_t* row, int32_t k, int32_t b, int32_t q) {
+void orc_set_code(uint8_t* proj, int32_t K, int32_t row, int32_t k, int32_t b, int32_t q) {
+  int64_t rb = orc_row_bytes(K, b);
   for (int32_t j = 0; j < b; ++j) {
-    int64_t w;
+    int64_t wb;
     int32_t bit;
-    orc_code_bit(k, b, j, &w, &bit);
-    uint32_t v = orc_load_word(row, w);
+    orc_code_bit(row, rb, k, b, j, &wb, &bit);
+    uint32_t v = orc_load_word(proj + wb);
     v &= ~(1u << bit);
     v |= (uint32_t)((q >> j) & 1) << bit;
-    orc_store_word(row, w, v);
+    orc_store_word(proj + wb, v);
   }
+}
+
+/* Storage row of logical gate/up row R (gate rows 0..I-1, up rows I..2I-1). */
+int32_t orc_gate_up_row(int32_t R, int32_t I) {
+  int32_t j = R < I ? R : R - I;
+  return 16 * (j / 8) + (R < I ? 0 : 8) + j % 8;
 }
 
 /* ------------------------------------------------------------------ */
@@ -382,8 +403,9 @@ void orc_set_code(uint8_t* row, int32_t k, int32_t b, int32_t q) {
  *   q = clamp(rint((w - bias) / scale), 0, 2^b - 1), using the rounded scale
  *   and bias; q = 0 when scale == 0.
  * All arithmetic in fp32, one rounding per operation.
- * w: [rows, K] fp32.  q_out: rows * row_bytes(K, b) bytes (zeroed here).
- * sb_out: rows * row_groups(K, g) words.
+ * w: [rows, K] fp32 in storage row order (rows a multiple of 8).  q_out: rows
+ * * row_bytes(K, b) bytes (zeroed here).  sb_out: rows * row_groups(K, g)
+ * words.
  */
 void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32_t b, uint8_t* q_out,
                        uint32_t* sb_out) {
@@ -393,7 +415,6 @@ void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32
   memset(q_out, 0, (size_t)(rb * rows));
   for (int32_t r = 0; r < rows; ++r) {
     const float* wr = w + (int64_t)r * K;
-    uint8_t* qr = q_out + (int64_t)r * rb;
     for (int64_t gi = 0; gi < ng; ++gi) {
       int32_t k0 = (int32_t)(gi * g);
       if (k0 >= K) {
@@ -416,7 +437,7 @@ void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32
           if (t > (float)qmax) t = (float)qmax;
           q = (int32_t)t;
         }
-        orc_set_code(qr, k, b, q);
+        orc_set_code(q_out, K, r, k, b, q);
       }
       sb_out[(int64_t)r * ng + gi] = (uint32_t)sh | ((uint32_t)bh << 16);
     }
@@ -426,28 +447,33 @@ void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32
 /* ------------------------------------------------------------------ */
 /* Dequantization (bit-exact target)                                     */
 /* ------------------------------------------------------------------ */
-/* deq = fma(scale, q, bias) in fp32: one rounding.  Rows of K (unpadded). */
+/* deq = fma(scale, q, bias) in fp32: one rounding.  Rows of K (unpadded), in
+ * storage order. */
 void orc_dequant_rows(const uint8_t* q, const uint32_t* sb, int32_t rows, int32_t K, int32_t g, int32_t b,
                       float* out) {
-  int64_t rb = orc_row_bytes(K, b);
   int64_t ng = orc_row_groups(K, g);
   for (int32_t r = 0; r < rows; ++r) {
     for (int32_t k = 0; k < K; ++k) {
       uint32_t sbw = sb[(int64_t)r * ng + k / g];
       float s = orc_bf16_to_f32((uint16_t)(sbw & 0xffffu));
       float bb = orc_bf16_to_f32((uint16_t)(sbw >> 16));
-      int32_t c = orc_get_code(q + (int64_t)r * rb, k, b);
+      int32_t c = orc_get_code(q, K, r, k, b);
       out[(int64_t)r * K + k] = fmaf(s, (float)c, bb);
     }
   }
 }
 
-/* Whole slot: gate_up [2I, H] and down [H, I], fp32. */
+/* Whole slot: gate_up [2I, H] (logical row order: gate then up) and down
+ * [H, I], fp32. */
 void orc_dequant_slot(const uint8_t* slot, int32_t H, int32_t I, int32_t g, int32_t b_gu, int32_t b_d,
                       float* gate_up, float* down) {
   int64_t off[5];
   orc_slot_layout(H, I, g, b_gu, b_d, off);
-  orc_dequant_rows(slot + off[0], (const uint32_t*)(slot + off[2]), 2 * I, H, g, b_gu, gate_up);
+  float* tmp = (float*)malloc(sizeof(float) * (size_t)2 * I * H);
+  orc_dequant_rows(slot + off[0], (const uint32_t*)(slot + off[2]), 2 * I, H, g, b_gu, tmp);
+  for (int32_t R = 0; R < 2 * I; ++R)
+    memcpy(gate_up + (int64_t)R * H, tmp + (int64_t)orc_gate_up_row(R, I) * H, sizeof(float) * (size_t)H);
+  free(tmp);
   orc_dequant_rows(slot + off[1], (const uint32_t*)(slot + off[3]), H, I, g, b_d, down);
 }
 

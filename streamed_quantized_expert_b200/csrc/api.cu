@@ -209,15 +209,16 @@ moe_status moe_dequant_slot(const void* pool, int32_t slot, const moe_layer_desc
   return cuda_status(launch_dequant_slot(base, *d, L, out_fp32, out_bf16, stream));
 }
 
-moe_status moe_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t group, int32_t bits, uint8_t* q,
-                             uint32_t* sb, cudaStream_t stream) {
-  if (rows < 0 || K < 1) return MOE_ERR_INVALID;
+moe_status moe_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t group, int32_t bits,
+                             int32_t gate_up_I, uint8_t* q, uint32_t* sb, cudaStream_t stream) {
+  if (rows < 0 || K < 1 || rows % 8) return MOE_ERR_INVALID;
+  if (gate_up_I < 0 || (gate_up_I > 0 && (rows != 2 * gate_up_I || gate_up_I % 8))) return MOE_ERR_INVALID;
   if (group != 32 && group != 64 && group != 128) return MOE_ERR_UNSUPPORTED;
   if (bits != 3 && bits != 4 && bits != 6) return MOE_ERR_UNSUPPORTED;
   if (K % group) return MOE_ERR_INVALID;
   if (rows == 0) return MOE_OK;
   if (!w || !q || !sb || !aligned(q, 4) || !aligned(sb, 4)) return MOE_ERR_INVALID;
-  return cuda_status(launch_quantize(w, rows, K, group, bits, q, sb, stream));
+  return cuda_status(launch_quantize(w, rows, K, group, bits, gate_up_I, q, sb, stream));
 }
 
 moe_status moe_exp_portable(const float* x, int64_t n, float* out, cudaStream_t stream) {

@@ -139,6 +139,25 @@ __device__ __forceinline__ float pair_hi_q(uint32_t p, int a) {
   return (__uint_as_float(p & 0xFFFF0000u) - 128.0f) * (a ? 0.125f : 1.0f);
 }
 
+// Rows are stored in groups of 8 (unit-major inside a group): unit u of row r
+// sits at unit position 8u + sigma(u, r), which keeps the per-thread unit
+// loads of the GEMV kernels free of shared-memory bank conflicts.
+template <int B>
+__host__ __device__ constexpr int unit_sigma(int u, int r) {
+  return B == 3 ? r : B == 4 ? (r + 2 * (u & 3)) & 7 : (r + 4 * ((u >> 1) & 1)) & 7;
+}
+
+// Byte offset of unit u of row `row` from the start of its projection.
+template <int B>
+__host__ __device__ constexpr int64_t unit_offset(int64_t row, int64_t u, int64_t row_bytes) {
+  return (row >> 3) * 8 * row_bytes + (8 * u + unit_sigma<B>((int)u, (int)(row & 7))) * 4 * B;
+}
+
+// Storage row of logical gate/up row R (blocks of 16: 8 gate rows, 8 up rows).
+__host__ __device__ constexpr int gate_up_row(int R, int I) {
+  return 16 * ((R < I ? R : R - I) >> 3) + (R < I ? 0 : 8) + ((R < I ? R : R - I) & 7);
+}
+
 // Logical input (within a 128-block) of register i's even member for unit t:
 // i = 2s + h  ->  16s + 2t + 8h.
 __host__ __device__ constexpr int pair_input(int i, int t) { return 16 * (i >> 1) + 2 * t + 8 * (i & 1); }
@@ -196,22 +215,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-
 // Bounded wait on a barrier phase: gives up (returns false) after about
-// `limit_ns` nanoseconds of device time, so a copy that never lands cannot
-// keep the GPU busy; the caller records MOE_DEV_ERR_TIMEOUT and returns.
+// `limit_cycles` SM clock cycles (default 4e9: about 2 s at the top clock), so
+// a copy that never lands cannot keep the GPU busy; the caller records
+// MOE_DEV_ERR_TIMEOUT and returns.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  uint64_t limit_ns = 2000000000ull) {
+                                                  long long limit_cycles = 4000000000ll) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
+  const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > limit_ns) return false;
+    if (clock64() - t0 > limit_cycles) return false;
   }
 }
 

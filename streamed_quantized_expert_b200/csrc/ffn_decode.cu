@@ -93,16 +93,24 @@ __device__ __forceinline__ void load_b_block(const uint16_t* row, int kb, int K,
   }
 }
 
-// One 128-block of a 16-row tile: rows ra (A rows 0-7) and rb (rows 8-15) in
-// shared memory, unit t4; accumulate the group epilogues into acc.
+// Offset of this thread's unit (unit t4 of block 0, row g8) inside an 8-row
+// group in shared memory; block kb adds kb * 32 units.
+template <int B>
+__device__ __forceinline__ int thread_unit_off(int t4, int g8) {
+  return (8 * t4 + unit_sigma<B>(t4, g8)) * 4 * B;
+}
+
+// One 128-block of a 16-row tile: 8-row groups ga (A rows 0-7) and gb (rows
+// 8-15) in shared memory; uoff = thread_unit_off; accumulate the group
+// epilogues into acc.
 template <int B, int GS>
-__device__ __forceinline__ void block_mma(const uint8_t* ra, const uint8_t* rbp, const uint32_t* sbA,
-                                          const uint32_t* sbB, int kb, int t4, const uint32_t (&bf)[8][2],
+__device__ __forceinline__ void block_mma(const uint8_t* ga, const uint8_t* gb, const uint32_t* sbA,
+                                          const uint32_t* sbB, int kb, int uoff, const uint32_t (&bf)[8][2],
                                           const float (&xs)[8 / GS][2], const float (&xo)[8 / GS][2],
                                           float (&acc)[4]) {
   uint32_t wa[B], wb[B], pa[16], pb[16];
-  load_unit<B>(ra + (kb * 4 + t4) * 4 * B, wa);
-  load_unit<B>(rbp + (kb * 4 + t4) * 4 * B, wb);
+  load_unit<B>(ga + kb * 128 * B + uoff, wa);
+  load_unit<B>(gb + kb * 128 * B + uoff, wb);
   unpack_unit<B>(wa, pa);
   unpack_unit<B>(wb, pb);
 #pragma unroll
@@ -146,34 +154,84 @@ __device__ __forceinline__ void consumers_sync(int nthreads) {
 }
 
 // ---------------------------------------------------------------------------
+// Per-CTA expert metadata, loaded once in a prologue (the loads for all of a
+// CTA's experts are independent, so they cost one or two L2 round trips in
+// total instead of a dependent chain per work item).
+// ---------------------------------------------------------------------------
+constexpr int kDenseMaxTokens = 8;  // T <= 8: every token gets its own MMA column
+constexpr int kMaxCtaExperts = 64;
+
+struct ExpMeta {
+  int e;     // expert id
+  int slot;  // slot in the pool (may be invalid: the expert is skipped)
+  int pos0;  // first sorted position of the expert's pairs
+  int cnt;   // pairs routed to the expert
+};
+
+// Thread i < n fills meta[i] for pass entry first + i; in dense mode also
+// tokpos[i][t] = sorted position of (expert, token t) or -1, and (if wtab)
+// wtab[i][t] = its routing weight (0 if absent).
+template <bool DENSE>
+__device__ __forceinline__ void load_expert_meta(const FfnArgs& a, int first, int n, ExpMeta* meta, int* tokpos,
+                                                 float* wtab) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int e = a.active[a.pass_begin + first + i];
+    ExpMeta m;
+    m.e = e;
+    m.slot = a.table[e];
+    m.pos0 = a.offsets[e];
+    m.cnt = a.offsets[e + 1] - m.pos0;
+    meta[i] = m;
+    if (DENSE) {
+      for (int t = 0; t < kDenseMaxTokens; ++t) {
+        tokpos[i * kDenseMaxTokens + t] = -1;
+        if (wtab) wtab[i * kDenseMaxTokens + t] = 0.f;
+      }
+      for (int p = m.pos0; p < m.pos0 + m.cnt; ++p) {
+        const int pf = a.pairs[p];
+        const int t = pf / a.k;
+        tokpos[i * kDenseMaxTokens + t] = p;
+        if (wtab) wtab[i * kDenseMaxTokens + t] = a.w[pf];
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // gate/up + SwiGLU:  h[pos][j] = silu(gate_j . x_t) * (up_j . x_t)
 // Work item = (active expert of the pass, 8 consecutive j) = a 16-row MMA
 // tile (8 gate rows, 8 up rows).  Each CTA takes a contiguous range of items.
 // Warp 8 is the producer: it streams every item's rows into a ring of shared
 // memory stages (full/empty mbarriers).  Warps 0-7 split K (BPW 128-blocks
-// each, x fragments stay in registers while the token set is unchanged) and
-// run through all their items without CTA-wide barriers; partial sums are
-// reduced across warps once per batch of kRedBatch (item, token-tile) entries.
+// each, x fragments in registers) and run through all their items without
+// CTA-wide barriers; partial sums are reduced across warps once per batch of
+// kRedBatch entries.  DENSE (T <= 8): MMA column n is token n for every
+// expert, so x is loaded once per kernel; otherwise columns are the expert's
+// own tokens, 8 at a time.
 // ---------------------------------------------------------------------------
 constexpr int kGuConsumers = 8;
 constexpr int kGuThreads = (kGuConsumers + 1) * 32;
 constexpr int kRedBatch = 8;
 
 struct RedMeta {
-  int pos;   // first sorted position of the token tile
-  int ntok;  // tokens in the tile
+  int ei;    // CTA-local expert index
+  int pos;   // first sorted position of the token tile (tile mode)
+  int ntok;  // tokens in the tile (tile mode)
   int jt;    // 8-row tile of the intermediate dimension
-  int pad;
 };
 
-template <int B, int BPW, int GS>
+template <int B, int BPW, int GS, bool DENSE>
 __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, t4 = lane & 3, g8 = lane >> 2;
-  const int NST = a.gu_nstage, SB = a.gu_stage_bytes, SR = a.sr_gu;
+  const int NST = a.gu_nstage, SB = a.gu_stage_bytes;
+  const int GRP = 8 * (int)a.rb_gu;  // bytes of an 8-row group
+  const int uoff = thread_unit_off<B>(t4, g8);
   float* red = reinterpret_cast<float*>(smem + (size_t)NST * SB);  // [kRedBatch][8 warps][32][4]
-  RedMeta* meta = reinterpret_cast<RedMeta*>(red + kRedBatch * kGuConsumers * 32 * 4);
-  uint64_t* full = reinterpret_cast<uint64_t*>(meta + kRedBatch);
+  RedMeta* rmeta = reinterpret_cast<RedMeta*>(red + kRedBatch * kGuConsumers * 32 * 4);
+  ExpMeta* emeta = reinterpret_cast<ExpMeta*>(rmeta + kRedBatch);
+  int* tokpos = reinterpret_cast<int*>(emeta + kMaxCtaExperts);  // [kMaxCtaExperts][8]
+  uint64_t* full = reinterpret_cast<uint64_t*>(tokpos + kMaxCtaExperts * kDenseMaxTokens);
   uint64_t* empty = full + NST;
 
   pdl_wait();
@@ -185,6 +243,9 @@ __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) 
   const int my_items = i1 - i0;
   pdl_launch_dependents();
   if (my_items <= 0) return;
+  const int e_first = i0 / jt_n;
+  const int n_exp = (i1 - 1) / jt_n - e_first + 1;  // <= kMaxCtaExperts (checked by the launcher)
+  load_expert_meta<DENSE>(a, e_first, n_exp, emeta, tokpos, nullptr);
   if (tid == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
@@ -196,31 +257,26 @@ __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) 
 
   if (warp == kGuConsumers) {  // producer
     if (lane == 0) {
-      const uint32_t sbb = 8u * a.ng_gu * 4u;
+      const uint32_t qb = 16u * (uint32_t)a.rb_gu, sbb = 16u * a.ng_gu * 4u;
       for (int r = 0; r < my_items; ++r) {
         const int s = r % NST;
         if (r >= NST && !mbar_wait_bounded(&empty[s], (uint32_t)(((r / NST) - 1) & 1))) {
           if (a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
-          // the consumers will time out on full[s]; nothing more is issued
-          break;
+          break;  // the consumers time out on full[s]; nothing more is issued
         }
         const int item = i0 + r;
         const int jt = item % jt_n;
-        const int slot = a.table[a.active[a.pass_begin + item / jt_n]];
+        const int slot = emeta[item / jt_n - e_first].slot;
         uint8_t* st = smem + (size_t)s * SB;
         if (!slot_ok(a, slot)) {
           mbar_arrive_expect_tx(&full[s], 0);
           continue;
         }
+        // storage rows 16 jt .. 16 jt + 15 = gate rows 8 jt.. then up rows 8 jt..
         const uint8_t* base = a.pool + (int64_t)slot * a.slot_bytes;
-        mbar_arrive_expect_tx(&full[s], 16u * (uint32_t)a.rb_gu + 2u * sbb);
-        for (int rr = 0; rr < 16; ++rr) {
-          const int grow = (rr < 8 ? 0 : a.I) + jt * 8 + (rr & 7);
-          bulk_g2s(st + rr * SR, base + a.q_gu + (int64_t)grow * a.rb_gu, (uint32_t)a.rb_gu, &full[s]);
-        }
-        uint8_t* sbd = st + 16 * SR;
-        bulk_g2s(sbd, base + a.sb_gu + (int64_t)jt * sbb, sbb, &full[s]);
-        bulk_g2s(sbd + sbb, base + a.sb_gu + (int64_t)(a.I + jt * 8) * a.ng_gu * 4, sbb, &full[s]);
+        mbar_arrive_expect_tx(&full[s], qb + sbb);
+        bulk_g2s(st, base + a.q_gu + (int64_t)jt * qb, qb, &full[s]);
+        bulk_g2s(st + qb, base + a.sb_gu + (int64_t)jt * sbb, sbb, &full[s]);
       }
     }
     return;
@@ -233,12 +289,24 @@ __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) 
   bool timed_out = false;
   int nent = 0;  // entries in the current reduction batch
 
+  if (DENSE) {  // column g8 = token g8 for every expert: load x once
+    const uint16_t* xrow = g8 < a.T ? a.x + (int64_t)g8 * a.H : nullptr;
+#pragma unroll
+    for (int bi = 0; bi < BPW; ++bi) load_b_block<B, GS>(xrow, warp * BPW + bi, a.H, t4, bf[bi], xs[bi], xo[bi]);
+  }
+
   auto flush = [&]() {
     consumers_sync(kGuConsumers * 32);
     for (int idx = tid; idx < nent * 64; idx += kGuConsumers * 32) {
       const int en = idx >> 6, j = (idx >> 3) & 7, n = idx & 7;
-      const RedMeta m = meta[en];
-      if (n >= m.ntok) continue;
+      const RedMeta m = rmeta[en];
+      int pos;
+      if (DENSE) {
+        pos = n < a.T ? tokpos[m.ei * kDenseMaxTokens + n] : -1;
+      } else {
+        pos = n < m.ntok ? m.pos + n : -1;
+      }
+      if (pos < 0) continue;
       const int src = 4 * j + (n >> 1), c = n & 1;
       const float* rp = red + (size_t)en * kGuConsumers * 32 * 4;
       float gate = 0.f, up = 0.f;
@@ -248,7 +316,7 @@ __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) 
         up += rp[(w * 32 + src) * 4 + 2 + c];
       }
       const float hv = gate / (1.0f + expf(-gate)) * up;
-      a.h[(int64_t)(m.pos + n) * a.I + m.jt * 8 + j] = f32_to_bf16_rne(hv);
+      a.h[(int64_t)pos * a.I + m.jt * 8 + j] = f32_to_bf16_rne(hv);
     }
     consumers_sync(kGuConsumers * 32);
     nent = 0;
@@ -258,36 +326,39 @@ __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) 
     const int s = r % NST;
     const int item = i0 + r;
     const int jt = item % jt_n;
-    const int e = a.active[a.pass_begin + item / jt_n];
-    const int slot = a.table[e];
-    const bool ok = slot_ok(a, slot);
-    if (!ok && tid == 0 && jt == 0) flag_slot(a, slot);
+    const int ei = item / jt_n - e_first;
+    const ExpMeta em = emeta[ei];
+    const bool ok = slot_ok(a, em.slot);
+    if (!ok && tid == 0 && jt == 0) flag_slot(a, em.slot);
     // a wait that runs out marks the warp; it keeps walking the items (no
     // waits, no math) so that every consumer reaches the same batch barriers
     if (!timed_out && !mbar_wait_bounded(&full[s], (uint32_t)((r / NST) & 1))) timed_out = true;
     const uint8_t* st = smem + (size_t)s * SB;
-    const uint32_t* sbs = reinterpret_cast<const uint32_t*>(st + 16 * SR);
-    const int pos0 = a.offsets[e], cnt_e = ok ? a.offsets[e + 1] - pos0 : 0;
-    for (int tt = 0; tt * 8 < cnt_e; ++tt) {
-      const int ntok = min(8, cnt_e - tt * 8);
-      const int my_tok = g8 < ntok ? a.pairs[pos0 + tt * 8 + g8] / a.k : -1;
-      if (!__all_sync(0xffffffffu, my_tok == cached_tok)) {
-        const uint16_t* xrow = my_tok >= 0 ? a.x + (int64_t)my_tok * a.H : nullptr;
+    const uint32_t* sbs = reinterpret_cast<const uint32_t*>(st + 2 * GRP);
+    const int n_tiles = !ok ? 0 : DENSE ? 1 : (em.cnt + 7) / 8;
+    for (int tt = 0; tt < n_tiles; ++tt) {
+      const int ntok = DENSE ? a.T : min(8, em.cnt - tt * 8);
+      if (!DENSE) {
+        const int my_tok = g8 < ntok ? a.pairs[em.pos0 + tt * 8 + g8] / a.k : -1;
+        if (!__all_sync(0xffffffffu, my_tok == cached_tok)) {
+          const uint16_t* xrow = my_tok >= 0 ? a.x + (int64_t)my_tok * a.H : nullptr;
 #pragma unroll
-        for (int bi = 0; bi < BPW; ++bi) load_b_block<B, GS>(xrow, warp * BPW + bi, a.H, t4, bf[bi], xs[bi], xo[bi]);
-        cached_tok = my_tok;
+          for (int bi = 0; bi < BPW; ++bi)
+            load_b_block<B, GS>(xrow, warp * BPW + bi, a.H, t4, bf[bi], xs[bi], xo[bi]);
+          cached_tok = my_tok;
+        }
       }
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int bi = 0; bi < BPW; ++bi) {
         const int kb = warp * BPW + bi;
         if (kb < a.nblk_gu && !timed_out)
-          block_mma<B, GS>(st + g8 * SR, st + (8 + g8) * SR, sbs + g8 * a.ng_gu, sbs + (8 + g8) * a.ng_gu, kb, t4,
-                           bf[bi], xs[bi], xo[bi], acc);
+          block_mma<B, GS>(st, st + GRP, sbs + g8 * a.ng_gu, sbs + (8 + g8) * a.ng_gu, kb, uoff, bf[bi], xs[bi],
+                           xo[bi], acc);
       }
       *reinterpret_cast<float4*>(&red[(((size_t)nent * kGuConsumers + warp) * 32 + lane) * 4]) =
           make_float4(acc[0], acc[1], acc[2], acc[3]);
-      if (warp == 0 && lane == 0) meta[nent] = RedMeta{pos0 + tt * 8, ntok, jt, 0};
+      if (warp == 0 && lane == 0) rmeta[nent] = RedMeta{ei, em.pos0 + tt * 8, ntok, jt};
       if (++nent == kRedBatch) flush();
     }
     __syncwarp();
@@ -302,26 +373,37 @@ __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) 
 // down (+ combine).  CTA owns 16 output rows.  Warp 4 is the producer: it
 // streams the pass's experts' 16-row slices into a ring of stages as soon as
 // the CTA starts -- before waiting for the gate/up kernel, since the slots do
-// not depend on it.  Warps 0-3 split K (128-blocks round-robin) over every
-// expert of the pass.
-// FUSED (T <= 64): y[t][rows] += sum_j w[t,j] o_{t,j}   (deterministic order)
-// else           : o[pair][rows] = o_{t,j}   (combined by combine_kernel)
+// not depend on it.  Warps 0-3 split K (128-blocks round-robin).
+// DENSE (T <= 8): column n = token n; h rows are staged in shared memory when
+//   they fit; y[t][rows] += sum over experts of w * o, summed in registers in
+//   expert order, then over the K-split warps in warp order.
+// FUSED (T <= 64): per-warp partial y in shared memory, summed in warp order.
+// else: o[pair][rows] = o_{t,j} (combined by combine_kernel); each warp owns
+//   whole experts.
 // ---------------------------------------------------------------------------
 constexpr int kDnConsumers = 4;
 constexpr int kDnThreads = (kDnConsumers + 1) * 32;
+constexpr int kHStageMax = 24 * 1024;
 
-template <int B, int GS, bool FUSED>
+template <int B, int GS, int MODE>  // MODE 0: dense, 1: fused token tiles, 2: per-pair output
 __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a) {
+  constexpr bool DENSE = MODE == 0, FUSED = MODE <= 1;
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, t4 = lane & 3, g8 = lane >> 2;
-  const int NST = a.d_nstage, SB = a.d_stage_bytes, SR = a.sr_d;
-  float* ypart = reinterpret_cast<float*>(smem + (size_t)NST * SB);  // [4 warps][T][16]
-  const int ypart_n = FUSED ? kDnConsumers * a.T * 16 : 0;
-  uint64_t* full = reinterpret_cast<uint64_t*>(ypart + ypart_n);
+  const int NST = a.d_nstage, SB = a.d_stage_bytes;
+  const int GRP = 8 * (int)a.rb_d;  // bytes of an 8-row group
+  const int uoff = thread_unit_off<B>(t4, g8);
+  uint8_t* hst = smem + (size_t)NST * SB;  // staged h (DENSE), kHStageMax bytes
+  float* ypart = reinterpret_cast<float*>(hst + (DENSE ? kHStageMax : 0));  // [4][T][16] or [4][32][4]
+  const int ypart_n = DENSE ? kDnConsumers * 32 * 4 : MODE == 1 ? kDnConsumers * a.T * 16 : 0;
+  ExpMeta* emeta = reinterpret_cast<ExpMeta*>(ypart + ypart_n);
+  int* tokpos = reinterpret_cast<int*>(emeta + kMaxCtaExperts);
+  float* wtab = reinterpret_cast<float*>(tokpos + kMaxCtaExperts * kDenseMaxTokens);
+  uint64_t* full = reinterpret_cast<uint64_t*>(wtab + kMaxCtaExperts * kDenseMaxTokens);
   uint64_t* empty = full + NST;
 
-  // the pass's experts and their slots were written before the gate/up kernel
-  // started, so they can be read before waiting on it
+  // the pass's experts, slots and routing were written before the gate/up
+  // kernel started, so they can be read before waiting on it
   int n_act = *a.n_active - a.pass_begin;
   if (n_act > a.pass_len) n_act = a.pass_len;
   const int n_rt = a.H / 16;
@@ -330,6 +412,8 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
     pdl_wait();
     return;
   }
+  const int n_meta = n_act < kMaxCtaExperts ? n_act : kMaxCtaExperts;
+  load_expert_meta<DENSE>(a, 0, n_meta, emeta, tokpos, wtab);
   if (tid == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
@@ -341,24 +425,23 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
 
   if (warp == kDnConsumers) {  // producer
     if (lane == 0) {
-      const uint32_t sbb = 16u * a.ng_d * 4u;
+      const uint32_t qb = 16u * (uint32_t)a.rb_d, sbb = 16u * a.ng_d * 4u;
       for (int r = 0; r < n_act; ++r) {
         const int s = r % NST;
         if (r >= NST && !mbar_wait_bounded(&empty[s], (uint32_t)(((r / NST) - 1) & 1))) {
           if (a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
           break;
         }
-        const int slot = a.table[a.active[a.pass_begin + r]];
+        const int slot = r < n_meta ? emeta[r].slot : a.table[a.active[a.pass_begin + r]];
         uint8_t* st = smem + (size_t)s * SB;
         if (!slot_ok(a, slot)) {
           mbar_arrive_expect_tx(&full[s], 0);
           continue;
         }
         const uint8_t* base = a.pool + (int64_t)slot * a.slot_bytes;
-        mbar_arrive_expect_tx(&full[s], 16u * (uint32_t)a.rb_d + sbb);
-        for (int rr = 0; rr < 16; ++rr)
-          bulk_g2s(st + rr * SR, base + a.q_d + (int64_t)(rt * 16 + rr) * a.rb_d, (uint32_t)a.rb_d, &full[s]);
-        bulk_g2s(st + 16 * SR, base + a.sb_d + (int64_t)rt * sbb, sbb, &full[s]);
+        mbar_arrive_expect_tx(&full[s], qb + sbb);
+        bulk_g2s(st, base + a.q_d + (int64_t)rt * qb, qb, &full[s]);
+        bulk_g2s(st + qb, base + a.sb_d + (int64_t)rt * sbb, sbb, &full[s]);
       }
     }
     pdl_wait();
@@ -366,57 +449,86 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
   }
 
   pdl_wait();  // h (gate/up output) and y are ready
-  if (FUSED) {
-    for (int i = tid; i < ypart_n; i += kDnConsumers * 32) ypart[i] = 0.f;
-    consumers_sync(kDnConsumers * 32);
+  const int np = a.T * a.k;
+  const bool h_staged = DENSE && (size_t)np * a.I * 2 <= (size_t)kHStageMax;
+  if (h_staged) {
+    // h is read by every CTA: plain coalesced copy into shared memory
+    const uint4* src = reinterpret_cast<const uint4*>(a.h);
+    uint4* dst = reinterpret_cast<uint4*>(hst);
+    for (int i = tid; i < np * a.I / 8; i += kDnConsumers * 32) dst[i] = src[i];
   }
+  if (MODE == 1)
+    for (int i = tid; i < ypart_n; i += kDnConsumers * 32) ypart[i] = 0.f;
+  consumers_sync(kDnConsumers * 32);
+
   bool timed_out = false;
-  float acc1[4] = {0.f, 0.f, 0.f, 0.f};  // T == 1: every expert feeds the same token
-  const bool single = FUSED && a.T == 1;
-  // FUSED: the 4 warps split K of every expert.  Otherwise each warp owns
-  // whole experts (r % 4 == warp), so o is written once, without atomics.
+  float yacc[4] = {0.f, 0.f, 0.f, 0.f};  // DENSE: (row g8 | g8+8) x (token 2t4 | 2t4+1)
   const int kb0 = FUSED ? warp : 0, kbs = FUSED ? kDnConsumers : 1;
   for (int r = 0; r < n_act; ++r) {
     const int s = r % NST;
-    const int e = a.active[a.pass_begin + r];
-    const bool ok = slot_ok(a, a.table[e]);
+    ExpMeta em;
+    if (r < n_meta) {
+      em = emeta[r];
+    } else {
+      em.e = a.active[a.pass_begin + r];
+      em.slot = a.table[em.e];
+      em.pos0 = a.offsets[em.e];
+      em.cnt = a.offsets[em.e + 1] - em.pos0;
+    }
+    const bool ok = slot_ok(a, em.slot);
     // every warp waits on every stage before releasing it, which keeps the
     // phases of the empty barriers in order
     if (!timed_out && !mbar_wait_bounded(&full[s], (uint32_t)((r / NST) & 1))) timed_out = true;
     const uint8_t* st = smem + (size_t)s * SB;
-    const uint32_t* sbs = reinterpret_cast<const uint32_t*>(st + 16 * SR);
+    const uint32_t* sbs = reinterpret_cast<const uint32_t*>(st + 2 * GRP);
     const bool mine = FUSED || (r % kDnConsumers) == warp;
-    const int pos0 = a.offsets[e], cnt_e = (ok && mine && !timed_out) ? a.offsets[e + 1] - pos0 : 0;
-    for (int tt = 0; tt * 8 < cnt_e; ++tt) {
-      const int ntok = min(8, cnt_e - tt * 8);
-      const uint16_t* hrow = g8 < ntok ? a.h + (int64_t)(pos0 + tt * 8 + g8) * a.I : nullptr;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int kb = kb0; kb < a.nblk_d; kb += kbs) {
-        uint32_t bf[8][2];
-        float xs[8 / GS][2], xo[8 / GS][2];
-        load_b_block<B, GS>(hrow, kb, a.I, t4, bf, xs, xo);
-        block_mma<B, GS>(st + g8 * SR, st + (8 + g8) * SR, sbs + g8 * a.ng_d, sbs + (8 + g8) * a.ng_d, kb, t4, bf,
-                         xs, xo, acc);
+    const bool run = ok && mine && !timed_out;
+    if (DENSE) {
+      if (run) {
+        const int pos = g8 < a.T ? tokpos[r * kDenseMaxTokens + g8] : -1;
+        const uint16_t* hrow = pos < 0 ? nullptr
+                               : h_staged ? reinterpret_cast<const uint16_t*>(hst) + (size_t)pos * a.I
+                                          : a.h + (int64_t)pos * a.I;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int kb = kb0; kb < a.nblk_d; kb += kbs) {
+          uint32_t bf[8][2];
+          float xs[8 / GS][2], xo[8 / GS][2];
+          load_b_block<B, GS>(hrow, kb, a.I, t4, bf, xs, xo);
+          block_mma<B, GS>(st, st + GRP, sbs + g8 * a.ng_d, sbs + (8 + g8) * a.ng_d, kb, uoff, bf, xs, xo, acc);
+        }
+        const float w0 = wtab[r * kDenseMaxTokens + 2 * t4], w1 = wtab[r * kDenseMaxTokens + 2 * t4 + 1];
+        yacc[0] += w0 * acc[0];
+        yacc[1] += w1 * acc[1];
+        yacc[2] += w0 * acc[2];
+        yacc[3] += w1 * acc[3];
       }
+    } else {
+      const int cnt_e = run ? em.cnt : 0;
+      for (int tt = 0; tt * 8 < cnt_e; ++tt) {
+        const int ntok = min(8, cnt_e - tt * 8);
+        const uint16_t* hrow = g8 < ntok ? a.h + (int64_t)(em.pos0 + tt * 8 + g8) * a.I : nullptr;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int kb = kb0; kb < a.nblk_d; kb += kbs) {
+          uint32_t bf[8][2];
+          float xs[8 / GS][2], xo[8 / GS][2];
+          load_b_block<B, GS>(hrow, kb, a.I, t4, bf, xs, xo);
+          block_mma<B, GS>(st, st + GRP, sbs + g8 * a.ng_d, sbs + (8 + g8) * a.ng_d, kb, uoff, bf, xs, xo, acc);
+        }
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int n = 2 * t4 + c;
-        if (n < ntok) {
-          const int pf = a.pairs[pos0 + tt * 8 + n];
-          if (FUSED) {
-            const float wg = a.w[pf];
-            if (single) {
-              acc1[c] += wg * acc[c];
-              acc1[2 + c] += wg * acc[2 + c];
-            } else {
+        for (int c = 0; c < 2; ++c) {
+          const int n = 2 * t4 + c;
+          if (n < ntok) {
+            const int pf = a.pairs[em.pos0 + tt * 8 + n];
+            if (FUSED) {
+              const float wg = a.w[pf];
               float* yp = ypart + ((size_t)warp * a.T + pf / a.k) * 16;
               yp[g8] += wg * acc[c];
               yp[8 + g8] += wg * acc[2 + c];
+            } else {
+              float* op = a.o + (int64_t)pf * a.H + rt * 16;
+              op[g8] = acc[c];
+              op[8 + g8] = acc[2 + c];
             }
-          } else {
-            float* op = a.o + (int64_t)pf * a.H + rt * 16;
-            op[g8] = acc[c];
-            op[8 + g8] = acc[2 + c];
           }
         }
       }
@@ -425,15 +537,19 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
     if (lane == 0) mbar_arrive(&empty[s]);
   }
   if (timed_out && lane == 0 && a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
-  if (FUSED) {
-    consumers_sync(kDnConsumers * 32);  // all ypart updates done before the single-token write
-    if (single) {
-      // only column 0 (t4 == 0, c == 0) carries token 0
-      if (t4 == 0) {
-        ypart[(size_t)warp * 16 + g8] = acc1[0];
-        ypart[(size_t)warp * 16 + 8 + g8] = acc1[2];
-      }
+  if (DENSE) {
+    *reinterpret_cast<float4*>(&ypart[(warp * 32 + lane) * 4]) = make_float4(yacc[0], yacc[1], yacc[2], yacc[3]);
+    consumers_sync(kDnConsumers * 32);
+    for (int i = tid; i < a.T * 16; i += kDnConsumers * 32) {
+      const int tok = i >> 4, row = i & 15;
+      // value of (row, token) sits at lane 4*(row&7) + tok/2, component (row>>3)*2 + (tok&1)
+      const int src = 4 * (row & 7) + (tok >> 1), c = (row >> 3) * 2 + (tok & 1);
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kDnConsumers; ++w) sum += ypart[(w * 32 + src) * 4 + c];
+      a.y[(int64_t)tok * a.H + rt * 16 + row] += sum;
     }
+  } else if (MODE == 1) {
     consumers_sync(kDnConsumers * 32);
     for (int i = tid; i < a.T * 16; i += kDnConsumers * 32) {
       const int tok = i >> 4, row = i & 15;
@@ -467,21 +583,16 @@ __global__ void combine_kernel(const FfnArgs a) {
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-static int smem_row_stride(int64_t rb, int bits) {
-  // words per row congruent to 12 (3-bit units), 16 (4-bit) or 24 (6-bit)
-  // mod 32: the per-thread unit loads of 8 rows x 4 units hit distinct banks
-  const int target = bits == 3 ? 12 : bits == 4 ? 16 : 24;
-  int sr = (int)round_up(rb, 16);
-  while (((sr / 4) & 31) != target) sr += 16;
-  return sr;
-}
-
 size_t ffn_ws_bytes(const moe_layer_desc& d, int T) {
   const int64_t np = (int64_t)T * d.k;
   size_t b = (size_t)round_up(np * d.I * 2, 256);  // h (bf16)
   if (T > kFusedMaxTokens) b += (size_t)round_up(np * d.H * 4, 256);  // o (fp32)
   return b;
 }
+
+// T <= 8 tokens with every routed pair fitting the per-CTA tables: one MMA
+// column per token for every expert.
+static bool dense_mode(const FfnArgs& a) { return a.T <= kDenseMaxTokens && a.T * a.k <= kMaxCtaExperts; }
 
 // Opt a kernel into the large dynamic shared-memory carve-out once per
 // (kernel, device); the attribute call is not free on the launch path.  Each
@@ -498,13 +609,16 @@ static cudaError_t ensure_smem_attr(const void* kern, int (&done_mask)[4]) {
 template <int B, int BPW, int GS>
 static cudaError_t launch_gu(const FfnArgs& a, int grid, size_t smem, cudaStream_t st) {
   static int done[4] = {0, 0, 0, 0};
-  const void* kern = reinterpret_cast<const void*>(ffn_gu_kernel<B, BPW, GS>);
-  cudaError_t e = ensure_smem_attr(kern, done);
+  static int done_d[4] = {0, 0, 0, 0};
+  const bool dense = dense_mode(a);
+  const void* kern = dense ? reinterpret_cast<const void*>(ffn_gu_kernel<B, BPW, GS, true>)
+                           : reinterpret_cast<const void*>(ffn_gu_kernel<B, BPW, GS, false>);
+  cudaError_t e = ensure_smem_attr(kern, dense ? done_d : done);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, grid, kGuThreads, smem, st, a);
 }
 
-template <int B, int GS, bool F>
+template <int B, int GS, int F>
 static cudaError_t launch_dn(const FfnArgs& a, int grid, size_t smem, cudaStream_t st) {
   static int done[4] = {0, 0, 0, 0};
   const void* kern = reinterpret_cast<const void*>(ffn_down_kernel<B, GS, F>);
@@ -527,14 +641,14 @@ static cudaError_t gu_by_bpw(const FfnArgs& a, int bpw, int gs, int grid, size_t
   return gu_by_gs<B, 4>(a, gs, grid, smem, st);
 }
 
-template <int B, bool F>
+template <int B, int F>
 static cudaError_t dn_by_gs(const FfnArgs& a, int gs, int grid, size_t smem, cudaStream_t st) {
   if (gs == 2) return launch_dn<B, 2, F>(a, grid, smem, st);
   if (gs == 4) return launch_dn<B, 4, F>(a, grid, smem, st);
   return launch_dn<B, 8, F>(a, grid, smem, st);
 }
 
-template <bool F>
+template <int F>
 static cudaError_t dn_by_bits(const FfnArgs& a, int bits, int gs, int grid, size_t smem, cudaStream_t st) {
   if (bits == 3) return dn_by_gs<3, F>(a, gs, grid, smem, st);
   if (bits == 4) return dn_by_gs<4, F>(a, gs, grid, smem, st);
@@ -564,10 +678,8 @@ cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, c
   a.ng_d = L.ng_d;
   a.nblk_gu = L.nblk_gu;
   a.nblk_d = L.nblk_d;
-  a.sr_gu = smem_row_stride(L.rb_gu, d.bits_gu);
-  a.sr_d = smem_row_stride(L.rb_d, d.bits_down);
-  a.gu_stage_bytes = (int)round_up(16 * a.sr_gu + 16 * L.ng_gu * 4, 128);
-  a.d_stage_bytes = (int)round_up(16 * a.sr_d + 16 * L.ng_d * 4, 128);
+  a.gu_stage_bytes = (int)round_up(16 * L.rb_gu + 16 * L.ng_gu * 4, 128);
+  a.d_stage_bytes = (int)round_up(16 * L.rb_d + 16 * L.ng_d * 4, 128);
   const int gs = d.group / 16;
   const int nblk = L.nblk_gu;
   const int bpw = nblk <= kGuConsumers ? 1 : nblk <= 2 * kGuConsumers ? 2 : 4;
@@ -577,23 +689,27 @@ cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, c
   const int64_t items = (int64_t)max_pass * (d.I / 8);
   int grid = (int)(items < num_sms ? items : num_sms);
   if (grid < 1) grid = 1;
+  const size_t meta_bytes = (size_t)kMaxCtaExperts * (sizeof(ExpMeta) + kDenseMaxTokens * 2 * sizeof(int));
   const size_t red_bytes = (size_t)kRedBatch * kGuConsumers * 32 * 4 * sizeof(float) + kRedBatch * sizeof(RedMeta);
   const int64_t items_per_cta = (items + grid - 1) / grid;
-  int nst = (int)((kGuSmemCap - red_bytes) / (a.gu_stage_bytes + 16));
+  if (items_per_cta / (d.I / 8) + 2 > kMaxCtaExperts) return cudaErrorInvalidConfiguration;
+  int nst = (int)((kGuSmemCap - red_bytes - meta_bytes) / (a.gu_stage_bytes + 16));
   if (nst > items_per_cta) nst = (int)items_per_cta;
   if (nst > 32) nst = 32;
   if (nst < 1) return cudaErrorInvalidConfiguration;
   a.gu_nstage = nst;
-  const size_t gu_smem = (size_t)nst * a.gu_stage_bytes + red_bytes + (size_t)nst * 16;
+  const size_t gu_smem = (size_t)nst * a.gu_stage_bytes + red_bytes + meta_bytes + (size_t)nst * 16;
 
-  const bool fused = a.T <= kFusedMaxTokens;
-  const size_t ypart = fused ? (size_t)kDnConsumers * a.T * 16 * sizeof(float) : 0;
-  int dnst = (int)((kDnSmemCap - ypart) / (a.d_stage_bytes + 16));
+  const bool dense = dense_mode(a);
+  const int mode = dense ? 0 : a.T <= kFusedMaxTokens ? 1 : 2;
+  const size_t ypart = mode == 0 ? (size_t)kDnConsumers * 32 * 4 * sizeof(float) + kHStageMax
+                       : mode == 1 ? (size_t)kDnConsumers * a.T * 16 * sizeof(float) : 0;
+  int dnst = (int)((kDnSmemCap - ypart - meta_bytes) / (a.d_stage_bytes + 16));
   if (dnst > max_pass) dnst = max_pass;
   if (dnst > 32) dnst = 32;
   if (dnst < 2) dnst = 2;
   a.d_nstage = dnst;
-  const size_t dn_smem = (size_t)dnst * a.d_stage_bytes + ypart + (size_t)dnst * 16;
+  const size_t dn_smem = (size_t)dnst * a.d_stage_bytes + ypart + meta_bytes + (size_t)dnst * 16;
 
   cudaError_t e = cudaSuccess;
   if (d.bits_gu == 3) e = gu_by_bpw<3>(a, bpw, gs, grid, gu_smem, st);
@@ -602,9 +718,10 @@ cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, c
   if (e != cudaSuccess) return e;
 
   const int n_rt = d.H / 16;
-  if (fused) e = dn_by_bits<true>(a, d.bits_down, gs, n_rt, dn_smem, st);
-  else e = dn_by_bits<false>(a, d.bits_down, gs, n_rt, dn_smem, st);
-  if (e != cudaSuccess || fused) return e;
+  if (mode == 0) e = dn_by_bits<0>(a, d.bits_down, gs, n_rt, dn_smem, st);
+  else if (mode == 1) e = dn_by_bits<1>(a, d.bits_down, gs, n_rt, dn_smem, st);
+  else e = dn_by_bits<2>(a, d.bits_down, gs, n_rt, dn_smem, st);
+  if (e != cudaSuccess || mode < 2) return e;
   const int64_t total = (int64_t)a.T * d.H;
   int cgrid = (int)((total + 255) / 256);
   if (cgrid > num_sms * 8) cgrid = num_sms * 8;

@@ -35,7 +35,6 @@ struct FfnArgs {
   // filled by the launcher
   int64_t q_gu, q_d, sb_gu, sb_d, rb_gu, rb_d;
   int ng_gu, ng_d, nblk_gu, nblk_d;
-  int sr_gu, sr_d;
   int gu_stage_bytes, d_stage_bytes, gu_nstage, d_nstage;
 };
 
@@ -69,7 +68,7 @@ cudaError_t launch_lookup(const int32_t* table, const int32_t* active, const int
                           int pass_len, int n_slots, int32_t* slots, int32_t* miss, int32_t* n_miss,
                           int32_t* dev_err, cudaStream_t st);
 cudaError_t launch_exp(const float* x, int64_t n, float* out, cudaStream_t st);
-cudaError_t launch_quantize(const float* w, int rows, int K, int g, int b, uint8_t* q, uint32_t* sb,
+cudaError_t launch_quantize(const float* w, int rows, int K, int g, int b, int gu_I, uint8_t* q, uint32_t* sb,
                             cudaStream_t st);
 cudaError_t launch_dequant_slot(const uint8_t* slot, const moe_layer_desc& d, const Layout& L, float* out32,
                                 uint16_t* out16, cudaStream_t st);

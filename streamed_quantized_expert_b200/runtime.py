@@ -43,7 +43,8 @@ def quantize_bank_gpu(E: int, desc: ops.LayerDesc, seed: int, device="cuda", std
     for e in range(E):
         w_gu, w_d = synth.expert_weights_torch(seed, e, H, I, device, std)
         base = slot.data_ptr()
-        ops.moe_quantize_rows(w_gu, 2 * I, H, g, desc.bits_gu, base + lay.q_gate_up, base + lay.sb_gate_up)
+        ops.moe_quantize_rows(w_gu, 2 * I, H, g, desc.bits_gu, base + lay.q_gate_up, base + lay.sb_gate_up,
+                              gate_up_I=I)
         ops.moe_quantize_rows(w_d, H, I, g, desc.bits_down, base + lay.q_down, base + lay.sb_down)
         bank[e].copy_(slot, non_blocking=False)
     return bank

@@ -1,9 +1,10 @@
 """Independent numpy decoder of the slot bit layout (test helper).
 
 Written from the layout description (blocks of 128 inputs, 4 units of 32
-codes, pair (even, odd) in the low/high 16-bit halves of a word), in a
-vectorised style unrelated to the oracle's per-bit C loop, so that an index
-mistake in either one shows up as a mismatch.
+codes, pair (even, odd) in the low/high 16-bit halves of a word; rows in
+groups of 8 stored unit-major with a per-width lane permutation; gate/up rows
+in blocks of 16), in a vectorised style unrelated to the oracle's per-bit C
+loop, so that an index mistake in either one shows up as a mismatch.
 """
 import numpy as np
 
@@ -12,8 +13,16 @@ def ceil128(k):
     return (k + 127) // 128 * 128
 
 
+def _sigma(u, r, b):
+    if b == 3:
+        return r
+    if b == 4:
+        return (r + 2 * (u % 4)) % 8
+    return (r + 4 * ((u // 2) % 2)) % 8
+
+
 def _bit_positions(K, b):
-    """For every input k < Kp and code bit j: (word index in row, bit in word)."""
+    """For every input k < Kp and code bit j: (unit index u, word in unit, bit in word)."""
     Kp = ceil128(K)
     k = np.arange(Kp)
     blk, kk = k // 128, k % 128
@@ -23,6 +32,7 @@ def _bit_positions(K, b):
     odd = k & 1
     i = 2 * s + h
     unit = 4 * blk + p
+    U = np.zeros((Kp, b), np.int64)
     W = np.zeros((Kp, b), np.int64)
     B = np.zeros((Kp, b), np.int64)
     for j in range(b):
@@ -41,19 +51,27 @@ def _bit_positions(K, b):
                 bi = np.where(i < 12, 6 * (i % 2) + j, 12 + 2 * (m % 2) + (j - 4))
         else:
             raise ValueError(b)
-        W[:, j] = unit * b + wi
+        U[:, j] = unit
+        W[:, j] = wi
         B[:, j] = bi + 16 * odd
-    return W, B
+    return U, W, B
 
 
 def decode_rows(q, K, b):
-    """q uint8 [rows, Kp*b/8] -> codes int64 [rows, K]."""
+    """q uint8 [rows, Kp*b/8] (a whole projection, rows in groups of 8) ->
+    codes int64 [rows, K]."""
     q = np.ascontiguousarray(q, dtype=np.uint8)
-    words = q.view("<u4").astype(np.int64)
-    W, B = _bit_positions(K, b)
-    codes = np.zeros((q.shape[0], W.shape[0]), np.int64)
-    for j in range(b):
-        codes |= ((words[:, W[:, j]] >> B[:, j]) & 1) << j
+    rows = q.shape[0]
+    rb = q.shape[1]
+    words = q.reshape(-1).view("<u4").astype(np.int64)
+    U, W, B = _bit_positions(K, b)
+    codes = np.zeros((rows, U.shape[0]), np.int64)
+    for r in range(rows):
+        grp_word = (r // 8) * 8 * rb // 4
+        for j in range(b):
+            pos = 8 * U[:, j] + _sigma(U[:, j], r % 8, b)
+            idx = grp_word + pos * b + W[:, j]
+            codes[r] |= ((words[idx] >> B[:, j]) & 1) << j
     return codes[:, :K]
 
 
@@ -66,3 +84,9 @@ def dequant_rows(q, sb, K, g, b):
     bb = ((sb >> 16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     gi = np.arange(K) // g
     return (s[:, gi] * codes + bb[:, gi]).astype(np.float32)
+
+
+def gate_up_storage_row(R, I):
+    """Storage row of logical gate/up row R: blocks of 16 = 8 gate + 8 up rows."""
+    j = R if R < I else R - I
+    return 16 * (j // 8) + (0 if R < I else 8) + j % 8

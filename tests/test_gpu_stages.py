@@ -41,8 +41,8 @@ def test_exp_bit_exact_on_every_float_in_domain(orc):
             pytest.fail(f"exp mismatch at bits {start + i:#x}: gpu {got[i]!r} cpu {ref[i]!r}")
 
 
-@pytest.mark.parametrize("rows,K,g,b", [(7, 64, 32, 4), (33, 2048, 64, 3), (16, 512, 64, 6), (5, 768, 128, 4),
-                                        (3, 32, 32, 3), (64, 2048, 64, 4)])
+@pytest.mark.parametrize("rows,K,g,b", [(8, 64, 32, 4), (40, 2048, 64, 3), (16, 512, 64, 6), (8, 768, 128, 4),
+                                        (8, 32, 32, 3), (64, 2048, 64, 4)])
 def test_quantize_bit_exact(orc, rows, K, g, b):
     w = (synth.rng(rows, K, g, b).standard_normal((rows, K), dtype=np.float32) * np.float32(0.02))
     w[0, :g] = np.float32(0.5)  # constant group
@@ -54,6 +54,21 @@ def test_quantize_bit_exact(orc, rows, K, g, b):
     torch.cuda.synchronize()
     assert np.array_equal(q.cpu().numpy(), qr)
     assert np.array_equal(sb.cpu().numpy().view(np.uint32), sbr)
+
+
+def test_quantize_gate_up_order_bit_exact(orc):
+    # a whole expert through moe_quantize_rows (gate/up row order) vs the oracle's slot builder
+    H, I, g, bg, bd = 256, 64, 64, 3, 4
+    w_gu, w_d = synth.expert_weights(4, 0, H, I)
+    ref = orc.build_slot(w_gu, w_d, g, bg, bd)
+    d = ops.desc(8, 2, H, I, g, bg, bd)
+    lay = ops.moe_slot_layout(d)
+    slot = torch.zeros(lay.slot_bytes, dtype=torch.uint8, device="cuda")
+    base = slot.data_ptr()
+    ops.moe_quantize_rows(dev(w_gu), 2 * I, H, g, bg, base + lay.q_gate_up, base + lay.sb_gate_up, gate_up_I=I)
+    ops.moe_quantize_rows(dev(w_d), H, I, g, bd, base + lay.q_down, base + lay.sb_down)
+    torch.cuda.synchronize()
+    assert np.array_equal(slot.cpu().numpy(), ref)
 
 
 @pytest.mark.parametrize("H,I,g,bg,bd", [(64, 32, 32, 4, 4), (2048, 512, 64, 3, 3), (256, 128, 64, 4, 6),

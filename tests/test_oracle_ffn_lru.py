@@ -24,7 +24,9 @@ def _bank(orc, E, H, I, g, b_gu, b_d, seed=0):
         sg = s[off[2]: off[2] + 2 * I * orc.row_groups(H, g) * 4].view(np.uint32).reshape(2 * I, -1)
         qd = s[off[1]: off[1] + H * orc.row_bytes(I, b_d)].reshape(H, -1)
         sd = s[off[3]: off[3] + H * orc.row_groups(I, g) * 4].view(np.uint32).reshape(H, -1)
-        dense.append((F.dequant_rows(qg, sg, H, g, b_gu).astype(np.float64),
+        gu_stored = F.dequant_rows(qg, sg, H, g, b_gu)
+        gu_logical = gu_stored[[F.gate_up_storage_row(R, I) for R in range(2 * I)]]
+        dense.append((gu_logical.astype(np.float64),
                       F.dequant_rows(qd, sd, I, g, b_d).astype(np.float64)))
     return slots, dense
 

@@ -13,34 +13,37 @@ from tests import _format_np as F
 @pytest.mark.parametrize("K", [32, 64, 128, 512, 768, 2048])
 def test_code_roundtrip_and_independent_decoder(orc, b, K):
     r = np.random.default_rng(b * 1000 + K)
-    rows = 3
+    rows = 16
     rb = orc.row_bytes(K, b)
     assert rb == F.ceil128(K) * b // 8
     q = np.zeros((rows, rb), np.uint8)
     codes = r.integers(0, 1 << b, size=(rows, K))
     for i in range(rows):
         for k in range(K):
-            orc.set_code(q[i], k, b, int(codes[i, k]))
+            orc.set_code(q, K, i, k, b, int(codes[i, k]))
     for i in range(rows):
-        assert [orc.get_code(q[i], k, b) for k in range(K)] == codes[i].tolist()
+        assert [orc.get_code(q, K, i, k, b) for k in range(K)] == codes[i].tolist()
     assert np.array_equal(F.decode_rows(q, K, b), codes)
 
 
 @pytest.mark.parametrize("b", [3, 4, 6])
 def test_layout_is_a_bijection(orc, b):
-    # every bit of a 128-input block belongs to exactly one (input, code bit)
-    W, B = F._bit_positions(128, b)
-    flat = (W * 32 + B).reshape(-1)
-    assert np.array_equal(np.sort(flat), np.arange(128 * b))
-    # all-ones codes fill every byte; one all-ones code sets exactly b bits
-    q = np.zeros((1, orc.row_bytes(128, b)), np.uint8)
-    for k in range(128):
-        orc.set_code(q[0], k, b, (1 << b) - 1)
+    # every bit of an 8-row group of 128-input blocks belongs to exactly one
+    # (row, input, code bit): setting the codes one by one to all-ones adds b
+    # new bits each time and ends with every byte 0xFF
+    q = np.zeros((8, orc.row_bytes(128, b)), np.uint8)
+    seen = 0
+    for row in range(8):
+        for k in range(128):
+            orc.set_code(q, 128, row, k, b, (1 << b) - 1)
+            n = int(np.unpackbits(q).sum())
+            assert n == seen + b
+            seen = n
     assert np.all(q == 0xFF)
-    for k in (0, 1, 9, 31, 62, 127):
-        q = np.zeros(orc.row_bytes(128, b), np.uint8)
-        orc.set_code(q, k, b, (1 << b) - 1)
-        assert int(np.unpackbits(q).sum()) == b
+    # the numpy description agrees: unit-word-bit triples cover a unit exactly once
+    U, W, B = F._bit_positions(128, b)
+    flat = ((U * b + W) * 32 + B).reshape(-1)
+    assert np.array_equal(np.sort(flat), np.arange(128 * b))
 
 
 def test_slot_sizes_for_the_workload_shapes(orc):
@@ -59,7 +62,7 @@ def test_slot_sizes_for_the_workload_shapes(orc):
 def test_quantizer_properties(orc, b, g):
     r = np.random.default_rng(b * 7 + g)
     K = 256
-    w = (r.standard_normal((20, K)) * 0.02).astype(np.float32)
+    w = (r.standard_normal((24, K)) * 0.02).astype(np.float32)
     w[3, :g] = np.float32(0.0123)  # constant group
     q, sb = orc.quantize_rows(w, g, b)
     codes = F.decode_rows(q, K, b)
@@ -68,7 +71,7 @@ def test_quantizer_properties(orc, b, g):
     s = ((sb & 0xFFFF).astype(np.uint32) << 16).view(np.float32)
     bias = ((sb >> 16).astype(np.uint32) << 16).view(np.float32)
     # scale = bf16 of (max-min)/(2^b-1); bias = bf16 of the group minimum
-    wg = w.reshape(20, K // g, g)
+    wg = w.reshape(24, K // g, g)
     assert np.all(np.abs(s[:, : K // g] - (wg.max(2) - wg.min(2)) / ((1 << b) - 1)) <= np.abs(s[:, : K // g]) * 2 ** -8 + 1e-30)
     assert np.all(np.abs(bias[:, : K // g] - wg.min(2)) <= np.abs(wg.min(2)) * 2 ** -8)
     # |w - deq| <= scale/2 + bf16 rounding of scale and bias over the whole code range
@@ -81,9 +84,9 @@ def test_quantizer_properties(orc, b, g):
 
 
 def test_padded_groups_are_zero(orc):
-    w = (np.random.default_rng(1).standard_normal((4, 32)) * 0.02).astype(np.float32)
+    w = (np.random.default_rng(1).standard_normal((8, 32)) * 0.02).astype(np.float32)
     q, sb = orc.quantize_rows(w, 32, 4)
-    assert q.shape == (4, 64) and sb.shape == (4, 4)
+    assert q.shape == (8, 64) and sb.shape == (8, 4)
     assert np.all(sb[:, 1:] == 0) and np.all(sb[:, 0] != 0)
 
 
@@ -108,7 +111,11 @@ def test_slot_sections_roundtrip(orc):
     gu, dn = orc.dequant_slot(slot, H, I, g, 4, 6)
     q = slot[off[0]: off[0] + 2 * I * orc.row_bytes(H, 4)].reshape(2 * I, -1)
     sb = slot[off[2]: off[2] + 2 * I * orc.row_groups(H, g) * 4].view(np.uint32).reshape(2 * I, -1)
-    assert np.array_equal(gu, F.dequant_rows(q, sb, H, g, 4))
+    stored = F.dequant_rows(q, sb, H, g, 4)
+    logical = stored[[F.gate_up_storage_row(R, I) for R in range(2 * I)]]
+    assert np.array_equal(gu, logical)
+    # gate rows first, then up rows: the quantised gate block reproduces w_gu[:I]
+    assert np.max(np.abs(gu - w_gu)) < 0.02
     qd = slot[off[1]: off[1] + H * orc.row_bytes(I, 6)].reshape(H, -1)
     sd = slot[off[3]: off[3] + H * orc.row_groups(I, g) * 4].view(np.uint32).reshape(H, -1)
     assert np.array_equal(dn, F.dequant_rows(qd, sd, I, g, 6))
