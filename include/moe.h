@@ -66,7 +66,9 @@
  *          at bits 12..15 of word m, bits 4..5 at bits 12+2*(m%2)+{0,1} of
  *          word 4+m/2
  *   Per group of g inputs, one 32-bit word: bf16 scale (low half), bf16 bias
- *   (high half).  A slot is four sections, each 256-byte aligned:
+ *   (high half); the words of 16 consecutive rows form a tile stored
+ *   group-major (word (r, gi) at (r/16)*16*(Kp/g) + gi*16 + r%16).  A slot is
+ *   four sections, each 256-byte aligned:
  *     q_gate_up [2I rows][Kp(H)*b_gu/8]   storage row order: blocks of 16
  *               rows, block m = gate rows 8m..8m+7 then up rows 8m..8m+7
  *     q_down    [H rows][Kp(I)*b_d/8]
@@ -245,12 +247,12 @@ moe_status moe_dequant_slot(const void* pool, int32_t slot, const moe_layer_desc
  * quantise rows of fp32 weights w [rows, K] into the slot format:
  * per group scale = bf16((max-min)/(2^b-1)), bias = bf16(min),
  * q = clamp(rint((w - bias)/scale), 0, 2^b-1) (q = 0 if scale = 0).
- *   rows       a multiple of 8
+ *   rows       a multiple of 16
  *   gate_up_I  0: row r of w is storage row r; I > 0: w is a gate/up matrix
  *              [2I, K] (gate rows then up rows) and its rows go to their
  *              storage rows (blocks of 8 gate + 8 up rows)
  *   q  device [rows * Kp*bits/8] bytes (8-row groups, see the format above)
- *   sb device uint32 [rows][Kp/group] (storage row order) */
+ *   sb device uint32 [rows * Kp/group] (16-row tiles, group-major) */
 moe_status moe_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t group, int32_t bits,
                              int32_t gate_up_I, uint8_t* q, uint32_t* sb, cudaStream_t stream);
 
@@ -333,8 +335,8 @@ typedef struct {
  *   moe_route (L) -> moe_sort -> if the layer is not fully resident in `cache`:
  *   moe_slot_lookup, copy n_active/active to meta_host, synchronise `stream`,
  *   moe_cache_step, moe_install_slots on `side`, upload the table, record
- *   `installed` on `side` and make `stream` wait on it -> zero y -> one pass of
- *   moe_expert_ffn over every active expert.
+ *   `installed` on `side` and make `stream` wait on it -> one pass of
+ *   moe_expert_ffn over every active expert, writing y.
  * y: device fp32 [T, H] (overwritten).  *n_installed (host, may be NULL): the
  * number of experts installed.  Errors as the calls it makes. */
 moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc, const moe_step_buffers* b,

@@ -188,12 +188,12 @@ def gate_up_order(I: int) -> np.ndarray:
 
 
 def quantize_rows(w: np.ndarray, g: int, b: int):
-    """w fp32 [rows, K] (storage order, rows a multiple of 8) -> (q uint8
+    """w fp32 [rows, K] (storage order, rows a multiple of 16) -> (q uint8
     [rows, row_bytes] -- rows interleaved in groups of 8, see oracle.c --,
-    sb uint32 [rows, row_groups])."""
+    sb uint32 [rows, row_groups] -- the flat words in the 16-row tile order)."""
     w = np.ascontiguousarray(w, dtype=np.float32)
     rows, K = w.shape
-    assert rows % 8 == 0, "rows come in groups of 8"
+    assert rows % 16 == 0, "rows come in tiles of 16"
     q = np.zeros((rows, row_bytes(K, b)), np.uint8)
     sb = np.zeros((rows, row_groups(K, g)), np.uint32)
     lib().orc_quantize_rows(_p(w), rows, K, g, b, _p(q), _p(sb))

@@ -266,7 +266,9 @@ void orc_slot_lookup(const int32_t* table, const int32_t* active, int32_t n_acti
  *   b = 4: sigma = (r + 2 (u mod 4)) mod 8
  *   b = 6: sigma = (r + 4 ((u / 2) mod 2)) mod 8
  * Per group of g inputs: a (scale, bias) pair of bf16, stored as one 32-bit
- * word, scale in the low half; row-major [rows][Kp/g].
+ * word, scale in the low half.  The words of 16 consecutive rows form a tile
+ * stored group-major: the word of (row r, group gi) is word
+ * (r/16)*16*(Kp/g) + gi*16 + r%16.
  *
  * A slot (one expert) is four sections, each starting on a 256-byte
  * boundary:  q_gate_up [2I rows] (row order: blocks of 16, block m = gate
@@ -386,6 +388,9 @@ void orc_set_code(uint8_t* proj, int32_t K, int32_t row, int32_t k, int32_t b, i
   }
 }
 
+/* Word index of the (scale, bias) word of (row, group gi), ng groups per row. */
+int64_t orc_sb_index(int32_t row, int64_t gi, int64_t ng) { return (int64_t)(row / 16) * 16 * ng + gi * 16 + row % 16; }
+
 /* Storage row of logical gate/up row R (gate rows 0..I-1, up rows I..2I-1). */
 int32_t orc_gate_up_row(int32_t R, int32_t I) {
   int32_t j = R < I ? R : R - I;
@@ -403,9 +408,9 @@ int32_t orc_gate_up_row(int32_t R, int32_t I) {
  *   q = clamp(rint((w - bias) / scale), 0, 2^b - 1), using the rounded scale
  *   and bias; q = 0 when scale == 0.
  * All arithmetic in fp32, one rounding per operation.
- * w: [rows, K] fp32 in storage row order (rows a multiple of 8).  q_out: rows
- * * row_bytes(K, b) bytes (zeroed here).  sb_out: rows * row_groups(K, g)
- * words.
+ * w: [rows, K] fp32 in storage row order (rows a multiple of 16).  q_out:
+ * rows * row_bytes(K, b) bytes (zeroed here).  sb_out: rows * row_groups(K, g)
+ * words (tile layout above).
  */
 void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32_t b, uint8_t* q_out,
                        uint32_t* sb_out) {
@@ -418,7 +423,7 @@ void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32
     for (int64_t gi = 0; gi < ng; ++gi) {
       int32_t k0 = (int32_t)(gi * g);
       if (k0 >= K) {
-        sb_out[(int64_t)r * ng + gi] = 0u;
+        sb_out[orc_sb_index(r, gi, ng)] = 0u;
         continue;
       }
       float mn = wr[k0], mx = wr[k0];
@@ -439,7 +444,7 @@ void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32
         }
         orc_set_code(q_out, K, r, k, b, q);
       }
-      sb_out[(int64_t)r * ng + gi] = (uint32_t)sh | ((uint32_t)bh << 16);
+      sb_out[orc_sb_index(r, gi, ng)] = (uint32_t)sh | ((uint32_t)bh << 16);
     }
   }
 }
@@ -454,7 +459,7 @@ void orc_dequant_rows(const uint8_t* q, const uint32_t* sb, int32_t rows, int32_
   int64_t ng = orc_row_groups(K, g);
   for (int32_t r = 0; r < rows; ++r) {
     for (int32_t k = 0; k < K; ++k) {
-      uint32_t sbw = sb[(int64_t)r * ng + k / g];
+      uint32_t sbw = sb[orc_sb_index(r, k / g, ng)];
       float s = orc_bf16_to_f32((uint16_t)(sbw & 0xffffu));
       float bb = orc_bf16_to_f32((uint16_t)(sbw >> 16));
       int32_t c = orc_get_code(q, K, r, k, b);

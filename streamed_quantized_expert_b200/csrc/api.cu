@@ -154,11 +154,14 @@ moe_status moe_install_slots(void* pool, size_t slot_bytes, int32_t n_slots, con
   return MOE_OK;
 }
 
-moe_status moe_expert_ffn(const uint16_t* x, int32_t T, const moe_layer_desc* d, const void* pool, int32_t n_slots,
-                          const int32_t* slot_table, const int32_t* ids, const float* w, const int32_t* offsets,
-                          const int32_t* pairs, const int32_t* active, const int32_t* n_active,
-                          const uint16_t* x_sorted, int32_t pass_begin, int32_t pass_len, float* y_accum, void* ws,
-                          size_t ws_bytes, int32_t* dev_err, cudaStream_t stream) {
+// moe_expert_ffn with a choice of y semantics: overwrite = 1 writes y = the
+// pass's result (used by the decode driver, whose single pass covers every
+// active expert, so that y needs no separate zeroing); 0 adds to y.
+__attribute__((visibility("hidden"))) moe_status moe_internal_expert_ffn(
+    const uint16_t* x, int32_t T, const moe_layer_desc* d, const void* pool, int32_t n_slots,
+    const int32_t* slot_table, const int32_t* ids, const float* w, const int32_t* offsets, const int32_t* pairs,
+    const int32_t* active, const int32_t* n_active, const uint16_t* x_sorted, int32_t pass_begin, int32_t pass_len,
+    float* y_accum, void* ws, size_t ws_bytes, int32_t* dev_err, cudaStream_t stream, int overwrite) {
   moe_status s = check_desc(d);
   if (s != MOE_OK) return s;
   if (T < 0 || pass_begin < 0 || pass_len < 0 || n_slots < 0) return MOE_ERR_INVALID;
@@ -196,7 +199,17 @@ moe_status moe_expert_ffn(const uint16_t* x, int32_t T, const moe_layer_desc* d,
   a.h = static_cast<uint16_t*>(ws);
   a.o = c.o ? reinterpret_cast<float*>(static_cast<char*>(ws) + c.h) : nullptr;
   a.dev_err = dev_err;
+  a.y_overwrite = overwrite ? 1 : 0;
   return cuda_status(launch_ffn_decode(a, *d, device_sms(), stream));
+}
+
+moe_status moe_expert_ffn(const uint16_t* x, int32_t T, const moe_layer_desc* d, const void* pool, int32_t n_slots,
+                          const int32_t* slot_table, const int32_t* ids, const float* w, const int32_t* offsets,
+                          const int32_t* pairs, const int32_t* active, const int32_t* n_active,
+                          const uint16_t* x_sorted, int32_t pass_begin, int32_t pass_len, float* y_accum, void* ws,
+                          size_t ws_bytes, int32_t* dev_err, cudaStream_t stream) {
+  return moe_internal_expert_ffn(x, T, d, pool, n_slots, slot_table, ids, w, offsets, pairs, active, n_active,
+                                 x_sorted, pass_begin, pass_len, y_accum, ws, ws_bytes, dev_err, stream, 0);
 }
 
 moe_status moe_dequant_slot(const void* pool, int32_t slot, const moe_layer_desc* d, float* out_fp32,
@@ -211,7 +224,7 @@ moe_status moe_dequant_slot(const void* pool, int32_t slot, const moe_layer_desc
 
 moe_status moe_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t group, int32_t bits,
                              int32_t gate_up_I, uint8_t* q, uint32_t* sb, cudaStream_t stream) {
-  if (rows < 0 || K < 1 || rows % 8) return MOE_ERR_INVALID;
+  if (rows < 0 || K < 1 || rows % 16) return MOE_ERR_INVALID;
   if (gate_up_I < 0 || (gate_up_I > 0 && (rows != 2 * gate_up_I || gate_up_I % 8))) return MOE_ERR_INVALID;
   if (group != 32 && group != 64 && group != 128) return MOE_ERR_UNSUPPORTED;
   if (bits != 3 && bits != 4 && bits != 6) return MOE_ERR_UNSUPPORTED;

@@ -153,6 +153,12 @@ __host__ __device__ constexpr int64_t unit_offset(int64_t row, int64_t u, int64_
   return (row >> 3) * 8 * row_bytes + (8 * u + unit_sigma<B>((int)u, (int)(row & 7))) * 4 * B;
 }
 
+// Word index of the (scale, bias) word of (row, group gi), ng groups per row:
+// tiles of 16 rows, group-major inside a tile.
+__host__ __device__ constexpr int64_t sb_index(int64_t row, int64_t gi, int64_t ng) {
+  return (row >> 4) * 16 * ng + gi * 16 + (row & 15);
+}
+
 // Storage row of logical gate/up row R (blocks of 16: 8 gate rows, 8 up rows).
 __host__ __device__ constexpr int gate_up_row(int R, int I) {
   return 16 * ((R < I ? R : R - I) >> 3) + (R < I ? 0 : 8) + ((R < I ? R : R - I) & 7);

@@ -3,7 +3,7 @@
 // fully resident) one small device->host copy and its synchronisation.
 //
 //   route -> sort -> [lookup -> misses to host -> LRU step -> pinned installs on
-//   the side stream + table upload -> compute stream waits] -> y = 0 -> FFN
+//   the side stream + table upload -> compute stream waits] -> FFN (writes y)
 //
 // RFC "How the prototype works": each layer copies its routing to the host
 // once; misses become one host-to-device copy per expert; when every expert
@@ -14,6 +14,14 @@
 #include <cuda_runtime.h>
 
 #include "moe.h"
+
+extern "C" moe_status moe_internal_expert_ffn(const uint16_t* x, int32_t T, const moe_layer_desc* d,
+                                              const void* pool, int32_t n_slots, const int32_t* slot_table,
+                                              const int32_t* ids, const float* w, const int32_t* offsets,
+                                              const int32_t* pairs, const int32_t* active, const int32_t* n_active,
+                                              const uint16_t* x_sorted, int32_t pass_begin, int32_t pass_len,
+                                              float* y_accum, void* ws, size_t ws_bytes, int32_t* dev_err,
+                                              cudaStream_t stream, int overwrite);
 
 extern "C" moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc,
                                        const moe_step_buffers* b, const uint16_t* x, const float* logits,
@@ -63,7 +71,7 @@ extern "C" moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const mo
       if (n_installed) *n_installed = n;
     }
   }
-  if (cudaMemsetAsync(y, 0, sizeof(float) * (size_t)T * d->H, stream) != cudaSuccess) return MOE_ERR_CUDA;
-  return moe_expert_ffn(x, T, d, lc->pool, lc->n_slots, lc->table_dev, b->ids, b->w, b->offsets, b->pairs, active,
-                        n_active, nullptr, 0, E, y, b->ws, b->ws_bytes, b->dev_err, stream);
+  // one pass over every active expert, writing y (no separate zeroing)
+  return moe_internal_expert_ffn(x, T, d, lc->pool, lc->n_slots, lc->table_dev, b->ids, b->w, b->offsets, b->pairs,
+                                 active, n_active, nullptr, 0, E, y, b->ws, b->ws_bytes, b->dev_err, stream, 1);
 }

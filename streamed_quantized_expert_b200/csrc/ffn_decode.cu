@@ -101,8 +101,9 @@ __device__ __forceinline__ int thread_unit_off(int t4, int g8) {
 }
 
 // One 128-block of a 16-row tile: 8-row groups ga (A rows 0-7) and gb (rows
-// 8-15) in shared memory; uoff = thread_unit_off; accumulate the group
-// epilogues into acc.
+// 8-15) in shared memory; uoff = thread_unit_off; sbA / sbB point at the
+// tile's (scale, bias) words of rows g8 / 8+g8 (group gi at [16 gi]);
+// accumulate the group epilogues into acc.
 template <int B, int GS>
 __device__ __forceinline__ void block_mma(const uint8_t* ga, const uint8_t* gb, const uint32_t* sbA,
                                           const uint32_t* sbB, int kb, int uoff, const uint32_t (&bf)[8][2],
@@ -123,7 +124,7 @@ __device__ __forceinline__ void block_mma(const uint8_t* ga, const uint8_t* gb, 
       mma_bf16(d, af, bf[s][0], bf[s][1]);
     }
     const int gi = kb * (8 / GS) + G;
-    const uint32_t wA = sbA[gi], wB = sbB[gi];
+    const uint32_t wA = sbA[gi * 16], wB = sbB[gi * 16];
     const float sA = bf16_lo(wA), bA = bf16_hi(wA), sB = bf16_lo(wB), bB = bf16_hi(wB);
     acc[0] += sA * (d[0] - xo[G][0]) + bA * xs[G][0];
     acc[1] += sA * (d[1] - xo[G][1]) + bA * xs[G][1];
@@ -173,8 +174,8 @@ struct ExpMeta {
 // wtab[i][t] = its routing weight (0 if absent).
 template <bool DENSE>
 __device__ __forceinline__ void load_expert_meta(const FfnArgs& a, int first, int n, ExpMeta* meta, int* tokpos,
-                                                 float* wtab) {
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+                                                 float* wtab, int nthreads) {
+  for (int i = threadIdx.x; i < n; i += nthreads) {
     const int e = a.active[a.pass_begin + first + i];
     ExpMeta m;
     m.e = e;
@@ -245,7 +246,6 @@ __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) 
   if (my_items <= 0) return;
   const int e_first = i0 / jt_n;
   const int n_exp = (i1 - 1) / jt_n - e_first + 1;  // <= kMaxCtaExperts (checked by the launcher)
-  load_expert_meta<DENSE>(a, e_first, n_exp, emeta, tokpos, nullptr);
   if (tid == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
@@ -255,9 +255,10 @@ __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) 
   }
   __syncthreads();
 
-  if (warp == kGuConsumers) {  // producer
+  if (warp == kGuConsumers) {  // producer: finds its experts' slots itself and starts the copies at once
     if (lane == 0) {
       const uint32_t qb = 16u * (uint32_t)a.rb_gu, sbb = 16u * a.ng_gu * 4u;
+      int cur_ai = -1, slot = -1;
       for (int r = 0; r < my_items; ++r) {
         const int s = r % NST;
         if (r >= NST && !mbar_wait_bounded(&empty[s], (uint32_t)(((r / NST) - 1) & 1))) {
@@ -266,7 +267,10 @@ __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) 
         }
         const int item = i0 + r;
         const int jt = item % jt_n;
-        const int slot = emeta[item / jt_n - e_first].slot;
+        if (item / jt_n != cur_ai) {
+          cur_ai = item / jt_n;
+          slot = a.table[a.active[a.pass_begin + cur_ai]];
+        }
         uint8_t* st = smem + (size_t)s * SB;
         if (!slot_ok(a, slot)) {
           mbar_arrive_expect_tx(&full[s], 0);
@@ -281,6 +285,10 @@ __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) 
     }
     return;
   }
+
+  // consumers: the experts' metadata (loaded while the first copies fly)
+  load_expert_meta<DENSE>(a, e_first, n_exp, emeta, tokpos, nullptr, kGuConsumers * 32);
+  consumers_sync(kGuConsumers * 32);
 
   // consumers
   uint32_t bf[BPW][8][2];
@@ -353,7 +361,7 @@ __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) 
       for (int bi = 0; bi < BPW; ++bi) {
         const int kb = warp * BPW + bi;
         if (kb < a.nblk_gu && !timed_out)
-          block_mma<B, GS>(st, st + GRP, sbs + g8 * a.ng_gu, sbs + (8 + g8) * a.ng_gu, kb, uoff, bf[bi], xs[bi],
+          block_mma<B, GS>(st, st + GRP, sbs + g8, sbs + 8 + g8, kb, uoff, bf[bi], xs[bi],
                            xo[bi], acc);
       }
       *reinterpret_cast<float4*>(&red[(((size_t)nent * kGuConsumers + warp) * 32 + lane) * 4]) =
@@ -381,7 +389,8 @@ __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) 
 // else: o[pair][rows] = o_{t,j} (combined by combine_kernel); each warp owns
 //   whole experts.
 // ---------------------------------------------------------------------------
-constexpr int kDnConsumers = 4;
+constexpr int kDnConsumers = 8;
+constexpr int kDnKSplit = 4;  // FUSED modes: warps w and w+4 split K the same way, experts alternate
 constexpr int kDnThreads = (kDnConsumers + 1) * 32;
 constexpr int kHStageMax = 24 * 1024;
 
@@ -396,6 +405,7 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
   uint8_t* hst = smem + (size_t)NST * SB;  // staged h (DENSE), kHStageMax bytes
   float* ypart = reinterpret_cast<float*>(hst + (DENSE ? kHStageMax : 0));  // [4][T][16] or [4][32][4]
   const int ypart_n = DENSE ? kDnConsumers * 32 * 4 : MODE == 1 ? kDnConsumers * a.T * 16 : 0;
+  const bool overwrite = a.y_overwrite != 0;
   ExpMeta* emeta = reinterpret_cast<ExpMeta*>(ypart + ypart_n);
   int* tokpos = reinterpret_cast<int*>(emeta + kMaxCtaExperts);
   float* wtab = reinterpret_cast<float*>(tokpos + kMaxCtaExperts * kDenseMaxTokens);
@@ -410,10 +420,12 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
   const int rt = blockIdx.x;
   if (rt >= n_rt || n_act <= 0) {
     pdl_wait();
+    if (rt < n_rt && a.y_overwrite)
+      for (int i = threadIdx.x; i < a.T * 16; i += blockDim.x) a.y[(int64_t)(i >> 4) * a.H + rt * 16 + (i & 15)] = 0.f;
     return;
   }
   const int n_meta = n_act < kMaxCtaExperts ? n_act : kMaxCtaExperts;
-  load_expert_meta<DENSE>(a, 0, n_meta, emeta, tokpos, wtab);
+  load_expert_meta<DENSE>(a, 0, n_meta, emeta, tokpos, wtab, kDnThreads);
   if (tid == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
@@ -463,7 +475,9 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
 
   bool timed_out = false;
   float yacc[4] = {0.f, 0.f, 0.f, 0.f};  // DENSE: (row g8 | g8+8) x (token 2t4 | 2t4+1)
-  const int kb0 = FUSED ? warp : 0, kbs = FUSED ? kDnConsumers : 1;
+  const int kb0 = FUSED ? (warp % kDnKSplit) : 0, kbs = FUSED ? kDnKSplit : 1;
+  const int egrp = FUSED ? kDnConsumers / kDnKSplit : kDnConsumers;  // warp groups taking experts in turn
+  const int my_grp = FUSED ? warp / kDnKSplit : warp;
   for (int r = 0; r < n_act; ++r) {
     const int s = r % NST;
     ExpMeta em;
@@ -481,7 +495,7 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
     if (!timed_out && !mbar_wait_bounded(&full[s], (uint32_t)((r / NST) & 1))) timed_out = true;
     const uint8_t* st = smem + (size_t)s * SB;
     const uint32_t* sbs = reinterpret_cast<const uint32_t*>(st + 2 * GRP);
-    const bool mine = FUSED || (r % kDnConsumers) == warp;
+    const bool mine = (r % egrp) == my_grp;
     const bool run = ok && mine && !timed_out;
     if (DENSE) {
       if (run) {
@@ -494,7 +508,7 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
           uint32_t bf[8][2];
           float xs[8 / GS][2], xo[8 / GS][2];
           load_b_block<B, GS>(hrow, kb, a.I, t4, bf, xs, xo);
-          block_mma<B, GS>(st, st + GRP, sbs + g8 * a.ng_d, sbs + (8 + g8) * a.ng_d, kb, uoff, bf, xs, xo, acc);
+          block_mma<B, GS>(st, st + GRP, sbs + g8, sbs + 8 + g8, kb, uoff, bf, xs, xo, acc);
         }
         const float w0 = wtab[r * kDenseMaxTokens + 2 * t4], w1 = wtab[r * kDenseMaxTokens + 2 * t4 + 1];
         yacc[0] += w0 * acc[0];
@@ -512,7 +526,7 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
           uint32_t bf[8][2];
           float xs[8 / GS][2], xo[8 / GS][2];
           load_b_block<B, GS>(hrow, kb, a.I, t4, bf, xs, xo);
-          block_mma<B, GS>(st, st + GRP, sbs + g8 * a.ng_d, sbs + (8 + g8) * a.ng_d, kb, uoff, bf, xs, xo, acc);
+          block_mma<B, GS>(st, st + GRP, sbs + g8, sbs + 8 + g8, kb, uoff, bf, xs, xo, acc);
         }
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -547,7 +561,8 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
       float sum = 0.f;
 #pragma unroll
       for (int w = 0; w < kDnConsumers; ++w) sum += ypart[(w * 32 + src) * 4 + c];
-      a.y[(int64_t)tok * a.H + rt * 16 + row] += sum;
+      float* yp = a.y + (int64_t)tok * a.H + rt * 16 + row;
+      *yp = overwrite ? sum : *yp + sum;
     }
   } else if (MODE == 1) {
     consumers_sync(kDnConsumers * 32);
@@ -556,7 +571,8 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
       float sum = 0.f;
 #pragma unroll
       for (int w = 0; w < kDnConsumers; ++w) sum += ypart[((size_t)w * a.T + tok) * 16 + row];
-      a.y[(int64_t)tok * a.H + rt * 16 + row] += sum;
+      float* yp = a.y + (int64_t)tok * a.H + rt * 16 + row;
+      *yp = overwrite ? sum : *yp + sum;
     }
   }
 }
@@ -565,7 +581,13 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
 __global__ void combine_kernel(const FfnArgs a) {
   pdl_wait();
   const int n_act = pass_count(a);
-  if (n_act == 0) return;
+  if (n_act == 0) {
+    if (a.y_overwrite)
+      for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)a.T * a.H;
+           i += (int64_t)gridDim.x * blockDim.x)
+        a.y[i] = 0.f;
+    return;
+  }
   const int e_lo = a.active[a.pass_begin], e_hi = a.active[a.pass_begin + n_act - 1];
   const int64_t total = (int64_t)a.T * a.H;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
@@ -576,7 +598,7 @@ __global__ void combine_kernel(const FfnArgs a) {
       const int e = a.ids[pf];
       if (e >= e_lo && e <= e_hi && slot_ok(a, a.table[e])) s += a.w[pf] * a.o[(int64_t)pf * a.H + r];
     }
-    a.y[i] += s;
+    a.y[i] = a.y_overwrite ? s : a.y[i] + s;
   }
 }
 
@@ -602,6 +624,9 @@ static cudaError_t ensure_smem_attr(const void* kern, int (&done_mask)[4]) {
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   if (dev < 128 && ((__atomic_load_n(&done_mask[dev >> 5], __ATOMIC_RELAXED) >> (dev & 31)) & 1)) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  // the whole carve-out as shared memory, so the gate/up and down kernels of
+  // one layer fit on an SM together
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e == cudaSuccess && dev < 128) __atomic_fetch_or(&done_mask[dev >> 5], 1 << (dev & 31), __ATOMIC_RELAXED);
   return e;
 }
@@ -683,7 +708,9 @@ cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, c
   const int gs = d.group / 16;
   const int nblk = L.nblk_gu;
   const int bpw = nblk <= kGuConsumers ? 1 : nblk <= 2 * kGuConsumers ? 2 : 4;
-  const int max_pass = a.pass_len < d.E ? a.pass_len : d.E;
+  // at most T*k experts are active, however long the pass
+  int max_pass = a.pass_len < d.E ? a.pass_len : d.E;
+  if ((int64_t)a.T * d.k < max_pass) max_pass = a.T * d.k;
 
   // gate/up: 148 CTAs (or fewer items), stages for every item of a CTA if they fit
   const int64_t items = (int64_t)max_pass * (d.I / 8);

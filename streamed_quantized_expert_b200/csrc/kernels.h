@@ -31,6 +31,7 @@ struct FfnArgs {
   uint16_t* h;  // workspace: [T*k][I] bf16, by sorted position
   float* o;     // workspace: [T*k][H] fp32, by flat pair index (T > kFusedMaxTokens)
   int32_t* dev_err;
+  int y_overwrite;  // 1: y = result (single pass over all experts); 0: y += result
   Layout L;
   // filled by the launcher
   int64_t q_gu, q_d, sb_gu, sb_d, rb_gu, rb_d;

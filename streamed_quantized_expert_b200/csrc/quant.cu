@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const float* __restrict__
   }
   if (lane % lanes_per_group == 0) {
     const int gi = (blk * 128 + 4 * lane) / g;
-    sb[(int64_t)srow * row_groups(K, g) + gi] = (uint32_t)sh | ((uint32_t)bh << 16);
+    sb[sb_index(srow, gi, row_groups(K, g))] = (uint32_t)sh | ((uint32_t)bh << 16);
   }
 }
 
@@ -129,13 +129,13 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ qbase, const uint32_t
   for (int i = 0; i < B; ++i) wv[i] = wp[i];
   uint32_t p[16];
   unpack_unit<B>(wv, p);
-  const uint32_t* sbr = sbbase + (int64_t)r * row_groups(K, g);
+  const int64_t ng = row_groups(K, g);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int a = PairShift<B>::a(i);
     const int k = blk * 128 + pair_input(i, t);
     if (k >= K) continue;  // K is a multiple of 32, so k+1 < K too
-    const uint32_t sbw = sbr[k / g];
+    const uint32_t sbw = sbbase[sb_index(r, k / g, ng)];
     const float s = bf16_lo(sbw), bb = bf16_hi(sbw);
     const float v0 = __fmaf_rn(s, pair_lo_q(p[i], a), bb);
     const float v1 = __fmaf_rn(s, pair_hi_q(p[i], a), bb);

@@ -59,6 +59,7 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
   const int lane = threadIdx.x & 31;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   pdl_wait();
+  pdl_launch_dependents();
   if (t >= T) return;
   const float* l = logits + (size_t)t * E;
   float lv[NPL], u[NPL], up[NPL];
@@ -191,6 +192,7 @@ __global__ void __launch_bounds__(1024) sort_small_kernel(const int32_t* __restr
   __shared__ int s_warp[32];
   const int tid = threadIdx.x;
   pdl_wait();
+  pdl_launch_dependents();
   s_hist[tid] = 0;
   __syncthreads();
   int e = -1;
@@ -214,6 +216,7 @@ __global__ void __launch_bounds__(1024) sort_hist_kernel(const int32_t* __restri
                                                          int32_t* __restrict__ chunk_hist) {
   __shared__ int s_hist[1024];
   pdl_wait();
+  pdl_launch_dependents();
   s_hist[threadIdx.x] = 0;
   __syncthreads();
   const int i = blockIdx.x * 1024 + threadIdx.x;
@@ -230,6 +233,7 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(int32_t* __restrict__ c
   __shared__ int s_warp[32];
   const int e = threadIdx.x;
   pdl_wait();
+  pdl_launch_dependents();
   int tot = 0;
   if (e < E)
     for (int c = 0; c < nchunk; ++c) tot += chunk_hist[(size_t)c * E + e];
@@ -251,6 +255,7 @@ __global__ void __launch_bounds__(1024) sort_scatter_kernel(const int32_t* __res
   __shared__ int s_ids[1024];
   __shared__ int s_base[1024];
   pdl_wait();
+  pdl_launch_dependents();
   const int i = blockIdx.x * 1024 + threadIdx.x;
   const int e = i < n ? ids[i] : -1;
   s_ids[threadIdx.x] = e;
@@ -285,6 +290,7 @@ __global__ void __launch_bounds__(1024) lookup_kernel(const int32_t* __restrict_
                                                       int32_t* __restrict__ dev_err) {
   __shared__ int s_warp[32];
   pdl_wait();
+  pdl_launch_dependents();
   const int na = *n_active;
   int end = pass_begin + pass_len;
   if (end > na) end = na;
@@ -310,11 +316,11 @@ __global__ void __launch_bounds__(1024) lookup_kernel(const int32_t* __restrict_
 cudaError_t launch_route(const float* logits, int T, int E, int k, float L, const int32_t* table, int32_t* ids,
                          float* w, cudaStream_t st) {
   const int blocks = (T + 7) / 8;
-  if (E <= 32) route_kernel<1><<<blocks, 256, 0, st>>>(logits, T, E, k, L, table, ids, w);
-  else if (E <= 128) route_kernel<4><<<blocks, 256, 0, st>>>(logits, T, E, k, L, table, ids, w);
-  else if (E <= 512) route_kernel<16><<<blocks, 256, 0, st>>>(logits, T, E, k, L, table, ids, w);
-  else route_kernel<32><<<blocks, 256, 0, st>>>(logits, T, E, k, L, table, ids, w);
-  return cudaGetLastError();
+  const void* kern = E <= 32    ? reinterpret_cast<const void*>(route_kernel<1>)
+                     : E <= 128 ? reinterpret_cast<const void*>(route_kernel<4>)
+                     : E <= 512 ? reinterpret_cast<const void*>(route_kernel<16>)
+                                : reinterpret_cast<const void*>(route_kernel<32>);
+  return launch_pdl(kern, blocks, 256, 0, st, logits, T, E, k, L, table, ids, w);
 }
 
 size_t sort_ws_bytes(int n, int E) { return n <= 1024 ? 0 : (size_t)((n + 1023) / 1024) * E * sizeof(int32_t); }
@@ -324,7 +330,9 @@ cudaError_t launch_sort(const int32_t* ids, const uint16_t* x, int T, int k, int
                         cudaStream_t st) {
   const int n = T * k;
   if (n <= 1024) {
-    sort_small_kernel<<<1, 1024, 0, st>>>(ids, n, E, offsets, pairs, active, n_active);
+    cudaError_t e = launch_pdl(reinterpret_cast<const void*>(sort_small_kernel), 1, 1024, 0, st, ids, n, E, offsets,
+                               pairs, active, n_active);
+    if (e != cudaSuccess) return e;
   } else {
     const int nchunk = (n + 1023) / 1024;
     int32_t* ch = static_cast<int32_t*>(ws);
@@ -344,9 +352,8 @@ cudaError_t launch_sort(const int32_t* ids, const uint16_t* x, int T, int k, int
 cudaError_t launch_lookup(const int32_t* table, const int32_t* active, const int32_t* n_active, int pass_begin,
                           int pass_len, int n_slots, int32_t* slots, int32_t* miss, int32_t* n_miss,
                           int32_t* dev_err, cudaStream_t st) {
-  lookup_kernel<<<1, 1024, 0, st>>>(table, active, n_active, pass_begin, pass_len, n_slots, slots, miss, n_miss,
-                                    dev_err);
-  return cudaGetLastError();
+  return launch_pdl(reinterpret_cast<const void*>(lookup_kernel), 1, 1024, 0, st, table, active, n_active, pass_begin,
+                    pass_len, n_slots, slots, miss, n_miss, dev_err);
 }
 
 cudaError_t launch_exp(const float* x, int64_t n, float* out, cudaStream_t st) {

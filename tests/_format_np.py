@@ -75,11 +75,19 @@ def decode_rows(q, K, b):
     return codes[:, :K]
 
 
+def sb_rows(sb_flat, rows, ng):
+    """Flat scale/bias words in the 16-row tile (group-major) order -> [rows, ng]."""
+    t = np.ascontiguousarray(sb_flat, dtype=np.uint32).reshape(rows // 16, ng, 16)
+    return t.transpose(0, 2, 1).reshape(rows, ng)
+
+
 def dequant_rows(q, sb, K, g, b):
     """Closed form of fma(scale, q, bias) in fp32: the exact product-sum in
-    float64 (exact for bf16 scale/bias and q < 64), rounded once to fp32."""
+    float64 (exact for bf16 scale/bias and q < 64), rounded once to fp32.
+    sb: the flat words as stored (16-row tiles, group-major)."""
     codes = decode_rows(q, K, b).astype(np.float64)
-    sb = np.ascontiguousarray(sb, dtype=np.uint32)
+    rows = q.shape[0]
+    sb = sb_rows(sb, rows, np.asarray(sb).size // rows)
     s = ((sb & 0xFFFF).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     bb = ((sb >> 16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     gi = np.arange(K) // g

@@ -58,7 +58,7 @@ def test_argument_checks(lib):
         ops.moe_install_slots(1 << 20, 256, 4, [1 << 21], [4])  # slot id past the pool
     assert ei.value.status == ops.MOE_ERR_INVALID
     with pytest.raises(ops.MoeError) as ei:
-        ops.moe_quantize_rows(1 << 20, 8, 64, 32, 5, 1 << 21, 1 << 22)
+        ops.moe_quantize_rows(1 << 20, 16, 64, 32, 5, 1 << 21, 1 << 22)
     assert ei.value.status == ops.MOE_ERR_UNSUPPORTED
     with pytest.raises(ops.MoeError) as ei:  # workspace too small
         ops.moe_expert_ffn(1 << 20, 4, d, 1 << 24, 8, 1 << 21, 1 << 21, 1 << 21, 1 << 21, 1 << 21, 1 << 21,

@@ -41,8 +41,8 @@ def test_exp_bit_exact_on_every_float_in_domain(orc):
             pytest.fail(f"exp mismatch at bits {start + i:#x}: gpu {got[i]!r} cpu {ref[i]!r}")
 
 
-@pytest.mark.parametrize("rows,K,g,b", [(8, 64, 32, 4), (40, 2048, 64, 3), (16, 512, 64, 6), (8, 768, 128, 4),
-                                        (8, 32, 32, 3), (64, 2048, 64, 4)])
+@pytest.mark.parametrize("rows,K,g,b", [(16, 64, 32, 4), (48, 2048, 64, 3), (16, 512, 64, 6), (16, 768, 128, 4),
+                                        (16, 32, 32, 3), (64, 2048, 64, 4)])
 def test_quantize_bit_exact(orc, rows, K, g, b):
     w = (synth.rng(rows, K, g, b).standard_normal((rows, K), dtype=np.float32) * np.float32(0.02))
     w[0, :g] = np.float32(0.5)  # constant group

@@ -62,16 +62,17 @@ def test_slot_sizes_for_the_workload_shapes(orc):
 def test_quantizer_properties(orc, b, g):
     r = np.random.default_rng(b * 7 + g)
     K = 256
-    w = (r.standard_normal((24, K)) * 0.02).astype(np.float32)
+    w = (r.standard_normal((32, K)) * 0.02).astype(np.float32)
     w[3, :g] = np.float32(0.0123)  # constant group
     q, sb = orc.quantize_rows(w, g, b)
     codes = F.decode_rows(q, K, b)
     assert codes.min() >= 0 and codes.max() <= (1 << b) - 1
     deq = orc.dequant_rows(q, sb, K, g, b)
-    s = ((sb & 0xFFFF).astype(np.uint32) << 16).view(np.float32)
-    bias = ((sb >> 16).astype(np.uint32) << 16).view(np.float32)
+    sbr = F.sb_rows(sb, 32, sb.size // 32)
+    s = ((sbr & 0xFFFF).astype(np.uint32) << 16).view(np.float32)
+    bias = ((sbr >> 16).astype(np.uint32) << 16).view(np.float32)
     # scale = bf16 of (max-min)/(2^b-1); bias = bf16 of the group minimum
-    wg = w.reshape(24, K // g, g)
+    wg = w.reshape(32, K // g, g)
     assert np.all(np.abs(s[:, : K // g] - (wg.max(2) - wg.min(2)) / ((1 << b) - 1)) <= np.abs(s[:, : K // g]) * 2 ** -8 + 1e-30)
     assert np.all(np.abs(bias[:, : K // g] - wg.min(2)) <= np.abs(wg.min(2)) * 2 ** -8)
     # |w - deq| <= scale/2 + bf16 rounding of scale and bias over the whole code range
@@ -84,10 +85,11 @@ def test_quantizer_properties(orc, b, g):
 
 
 def test_padded_groups_are_zero(orc):
-    w = (np.random.default_rng(1).standard_normal((8, 32)) * 0.02).astype(np.float32)
+    w = (np.random.default_rng(1).standard_normal((16, 32)) * 0.02).astype(np.float32)
     q, sb = orc.quantize_rows(w, 32, 4)
-    assert q.shape == (8, 64) and sb.shape == (8, 4)
-    assert np.all(sb[:, 1:] == 0) and np.all(sb[:, 0] != 0)
+    assert q.shape == (16, 64) and sb.shape == (16, 4)
+    sbr = F.sb_rows(sb, 16, 4)
+    assert np.all(sbr[:, 1:] == 0) and np.all(sbr[:, 0] != 0)
 
 
 @pytest.mark.parametrize("b", [3, 4, 6])
