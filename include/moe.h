@@ -52,13 +52,14 @@
  *   codes; unit p holds, for s = 0..7, the input pairs (128B+16s+2p, +1) and
  *   (128B+16s+2p+8, +1) as pair indices 2s and 2s+1, the even input in the
  *   low 16-bit half of a 32-bit word and the odd input at the same offset in
- *   the high half.  Rows are stored in groups of 8 consecutive rows
- *   (8*Kp*b/8 bytes per group); inside a group, unit u = 4B+p of row r (0..7)
- *   is at unit position 8u + sigma(u, r) (4b bytes per position), sigma = r
- *   for b=3, (r + 2(u mod 4)) mod 8 for b=4, (r + 4((u/2) mod 2)) mod 8 for
- *   b=6 -- so one tile of rows is one contiguous copy and the GEMV's
- *   per-thread unit loads from shared memory are bank-conflict free.  A unit
- *   is b little-endian words:
+ *   the high half.  Rows are stored in tiles of 16 consecutive rows; a tile
+ *   is the rows' codes (16*Kp*b/8 bytes) followed by their (scale, bias)
+ *   words, and consecutive tiles are adjacent.  The codes are two groups of
+ *   8 rows; inside a group, unit u = 4B+p of row r (0..7) is at unit position
+ *   8u + sigma(u, r) (4b bytes per position), sigma = r for b=3,
+ *   (r + 2(u mod 4)) mod 8 for b=4, (r + 4((u/2) mod 2)) mod 8 for b=6 -- so a
+ *   tile is one contiguous copy and the GEMV's per-thread unit loads from
+ *   shared memory are bank-conflict free.  A unit is b little-endian words:
  *     b=4: pair i in word i/4, bits 4*(i%4)..+3
  *     b=3: pair i<15 in word i/5, bits 3*(i%5)..+2; pair 15: bit j of the
  *          code is bit 15 of word j
@@ -66,15 +67,12 @@
  *          at bits 12..15 of word m, bits 4..5 at bits 12+2*(m%2)+{0,1} of
  *          word 4+m/2
  *   Per group of g inputs, one 32-bit word: bf16 scale (low half), bf16 bias
- *   (high half); the words of 16 consecutive rows form a tile stored
- *   group-major (word (r, gi) at (r/16)*16*(Kp/g) + gi*16 + r%16).  A slot is
- *   four sections, each 256-byte aligned:
- *     q_gate_up [2I rows][Kp(H)*b_gu/8]   storage row order: blocks of 16
- *               rows, block m = gate rows 8m..8m+7 then up rows 8m..8m+7
- *     q_down    [H rows][Kp(I)*b_d/8]
- *     sb_gate_up[2I rows][Kp(H)/g] words (same row order as q_gate_up)
- *     sb_down   [H rows][Kp(I)/g] words
- *   slot_bytes = end of the last section rounded to 256.  Dequantised weight
+ *   (high half); inside a tile the words are group-major (word (r, gi) at
+ *   gi*16 + r).  A slot is two projections, each 256-byte aligned:
+ *     gate_up [2I rows]  storage row order: blocks of 16 rows, block m =
+ *             gate rows 8m..8m+7 then up rows 8m..8m+7 (one tile per block)
+ *     down    [H rows]
+ *   slot_bytes = end of the down projection rounded to 256.  Dequantised weight
  *   = fmaf(scale, q, bias) in fp32 (one rounding).
  */
 #ifndef MOE_H
@@ -117,21 +115,26 @@ typedef struct {
   int32_t bits_down; /* code width of the down projection */
 } moe_layer_desc;
 
-/* Byte offsets of the four slot sections and the slot size (the size-class
- * key of 1bit-MONSTER PR #137: "the sum of its aligned read windows"). */
+/* Byte offsets of the two projections in a slot, their 16-row tile sizes, and
+ * the slot size (the size-class key of 1bit-MONSTER PR #137: "the sum of its
+ * aligned read windows"). */
 typedef struct {
-  uint64_t q_gate_up, q_down, sb_gate_up, sb_down, slot_bytes;
+  uint64_t gate_up, down, gate_up_tile_bytes, down_tile_bytes, slot_bytes;
 } moe_slot_layout_t;
 
 /* Slot byte size for d, or 0 if d is invalid. */
 size_t moe_slot_bytes(const moe_layer_desc* d);
 
-/* Section offsets for d.  Returns MOE_ERR_INVALID/UNSUPPORTED for a bad d. */
+/* Projection offsets and tile sizes for d.  Returns MOE_ERR_INVALID or
+ * MOE_ERR_UNSUPPORTED for a bad d. */
 moe_status moe_slot_layout(const moe_layer_desc* d, moe_slot_layout_t* out);
 
 /* Device workspace needed by moe_sort and moe_expert_ffn for up to
  * max_tokens tokens (0 if d is invalid).  One buffer of this size may be
- * shared by the two calls when they run in stream order. */
+ * shared by the two calls when they run in stream order.  Its first 256
+ * bytes are a control block (the grid barrier of the single-launch decode
+ * FFN): zero them once after allocating the workspace (e.g. cudaMemset);
+ * every call leaves them zero again.  The rest needs no initialisation. */
 size_t moe_workspace_bytes(const moe_layer_desc* d, int32_t max_tokens);
 
 /* Stage 1.  Cache-aware top-k (BigMoeOnEdge note: every expert already in
@@ -251,10 +254,10 @@ moe_status moe_dequant_slot(const void* pool, int32_t slot, const moe_layer_desc
  *   gate_up_I  0: row r of w is storage row r; I > 0: w is a gate/up matrix
  *              [2I, K] (gate rows then up rows) and its rows go to their
  *              storage rows (blocks of 8 gate + 8 up rows)
- *   q  device [rows * Kp*bits/8] bytes (8-row groups, see the format above)
- *   sb device uint32 [rows * Kp/group] (16-row tiles, group-major) */
+ *   proj       device, (rows/16) tiles (see the format above), 16-byte
+ *              aligned: a slot's gate_up or down projection */
 moe_status moe_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t group, int32_t bits,
-                             int32_t gate_up_I, uint8_t* q, uint32_t* sb, cudaStream_t stream);
+                             int32_t gate_up_I, uint8_t* proj, cudaStream_t stream);
 
 /* Test: the fp32 exp used by moe_route, elementwise on n device floats. */
 moe_status moe_exp_portable(const float* x, int64_t n, float* out, cudaStream_t stream);

@@ -55,11 +55,12 @@ def lib():
             "orc_row_bytes": (i64, [i32, i32]),
             "orc_row_groups": (i64, [i32, i32]),
             "orc_slot_layout": (None, [i32, i32, i32, i32, i32, P]),
-            "orc_get_code": (i32, [P, i32, i32, i32, i32]),
-            "orc_set_code": (None, [P, i32, i32, i32, i32, i32]),
+            "orc_get_code": (i32, [P, i32, i32, i32, i32, i32]),
+            "orc_set_code": (None, [P, i32, i32, i32, i32, i32, i32]),
+            "orc_tile_bytes": (i64, [i32, i32, i32]),
             "orc_gate_up_row": (i32, [i32, i32]),
-            "orc_quantize_rows": (None, [P, i32, i32, i32, i32, P, P]),
-            "orc_dequant_rows": (None, [P, P, i32, i32, i32, i32, P]),
+            "orc_quantize_rows": (None, [P, i32, i32, i32, i32, P]),
+            "orc_dequant_rows": (None, [P, i32, i32, i32, i32, P]),
             "orc_dequant_slot": (None, [P, i32, i32, i32, i32, i32, P, P]),
             "orc_expert_ffn": (None, [P, i32, i32, i32, i32, i32, i32, P, P, P, P, i32, P]),
             "orc_lru_step": (i32, [i32, i32, i32, P, P, P, P, P, i32, P, P]),
@@ -153,25 +154,29 @@ def row_groups(K: int, g: int) -> int:
 
 
 def slot_layout(H: int, I: int, g: int, b_gu: int, b_d: int):
-    """Section offsets (q_gu, q_d, sb_gu, sb_d) and the slot byte size."""
+    """([gate_up offset, down offset, gate_up tile bytes, down tile bytes], slot bytes)."""
     off = np.zeros(5, np.int64)
     lib().orc_slot_layout(H, I, g, b_gu, b_d, _p(off))
     return [int(v) for v in off[:4]], int(off[4])
+
+
+def tile_bytes(K: int, g: int, b: int) -> int:
+    return int(lib().orc_tile_bytes(K, g, b))
 
 
 def slot_bytes(H: int, I: int, g: int, b_gu: int, b_d: int) -> int:
     return slot_layout(H, I, g, b_gu, b_d)[1]
 
 
-def get_code(proj: np.ndarray, K: int, row: int, k: int, b: int) -> int:
-    """Code of input k of row `row` of a projection (bytes of all its rows)."""
+def get_code(proj: np.ndarray, K: int, g: int, row: int, k: int, b: int) -> int:
+    """Code of input k of row `row` of a projection (bytes of all its tiles)."""
     proj = np.ascontiguousarray(proj, dtype=np.uint8)
-    return int(lib().orc_get_code(_p(proj), K, row, k, b))
+    return int(lib().orc_get_code(_p(proj), K, g, row, k, b))
 
 
-def set_code(proj: np.ndarray, K: int, row: int, k: int, b: int, q: int) -> None:
+def set_code(proj: np.ndarray, K: int, g: int, row: int, k: int, b: int, q: int) -> None:
     assert proj.dtype == np.uint8 and proj.flags["C_CONTIGUOUS"]
-    lib().orc_set_code(_p(proj), K, row, k, b, q)
+    lib().orc_set_code(_p(proj), K, g, row, k, b, q)
 
 
 def gate_up_row(R: int, I: int) -> int:
@@ -187,25 +192,21 @@ def gate_up_order(I: int) -> np.ndarray:
     return order
 
 
-def quantize_rows(w: np.ndarray, g: int, b: int):
-    """w fp32 [rows, K] (storage order, rows a multiple of 16) -> (q uint8
-    [rows, row_bytes] -- rows interleaved in groups of 8, see oracle.c --,
-    sb uint32 [rows, row_groups] -- the flat words in the 16-row tile order)."""
+def quantize_rows(w: np.ndarray, g: int, b: int) -> np.ndarray:
+    """w fp32 [rows, K] (storage order, rows a multiple of 16) -> the
+    projection's bytes, uint8 [rows/16, tile_bytes] (see oracle.c)."""
     w = np.ascontiguousarray(w, dtype=np.float32)
     rows, K = w.shape
     assert rows % 16 == 0, "rows come in tiles of 16"
-    q = np.zeros((rows, row_bytes(K, b)), np.uint8)
-    sb = np.zeros((rows, row_groups(K, g)), np.uint32)
-    lib().orc_quantize_rows(_p(w), rows, K, g, b, _p(q), _p(sb))
-    return q, sb
+    proj = np.zeros((rows // 16, tile_bytes(K, g, b)), np.uint8)
+    lib().orc_quantize_rows(_p(w), rows, K, g, b, _p(proj))
+    return proj
 
 
-def dequant_rows(q: np.ndarray, sb: np.ndarray, K: int, g: int, b: int) -> np.ndarray:
-    q = np.ascontiguousarray(q, dtype=np.uint8)
-    sb = np.ascontiguousarray(sb, dtype=np.uint32)
-    rows = q.shape[0]
+def dequant_rows(proj: np.ndarray, rows: int, K: int, g: int, b: int) -> np.ndarray:
+    proj = np.ascontiguousarray(proj, dtype=np.uint8)
     out = np.empty((rows, K), np.float32)
-    lib().orc_dequant_rows(_p(q), _p(sb), rows, K, g, b, _p(out))
+    lib().orc_dequant_rows(_p(proj), rows, K, g, b, _p(out))
     return out
 
 
@@ -216,12 +217,10 @@ def build_slot(w_gu: np.ndarray, w_d: np.ndarray, g: int, b_gu: int, b_d: int) -
     assert w_d.shape == (H, I)
     off, nbytes = slot_layout(H, I, g, b_gu, b_d)
     slot = np.zeros(nbytes, np.uint8)
-    qg, sg = quantize_rows(np.ascontiguousarray(w_gu[gate_up_order(I)]), g, b_gu)
-    qd, sd = quantize_rows(w_d, g, b_d)
-    slot[off[0]: off[0] + qg.size] = qg.reshape(-1)
-    slot[off[1]: off[1] + qd.size] = qd.reshape(-1)
-    slot[off[2]: off[2] + sg.size * 4] = sg.reshape(-1).view(np.uint8)
-    slot[off[3]: off[3] + sd.size * 4] = sd.reshape(-1).view(np.uint8)
+    pg = quantize_rows(np.ascontiguousarray(w_gu[gate_up_order(I)]), g, b_gu)
+    pd = quantize_rows(w_d, g, b_d)
+    slot[off[0]: off[0] + pg.size] = pg.reshape(-1)
+    slot[off[1]: off[1] + pd.size] = pd.reshape(-1)
     return slot
 
 

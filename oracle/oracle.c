@@ -259,23 +259,24 @@ void orc_slot_lookup(const int32_t* table, const int32_t* active, int32_t n_acti
  *   b = 6: pair i < 12 in word i/2 at bits 6*(i%2) .. +5;
  *          pair i >= 12, m = i - 12: code bits 0..3 at bits 12..15 of
  *          word m; code bits 4,5 at bits 12 + 2*(m%2) + {0,1} of word 4+m/2
- * Rows are stored in groups of 8 consecutive rows (8 * row_bytes bytes per
- * group).  Inside a group, unit u (= 4B + p) of row r (0..7) sits at unit
- * position 8u + sigma(u, r) (unit positions are 4b bytes apart), with
+ * Rows are stored in tiles of 16 consecutive rows.  A tile is the rows'
+ * codes (16 * row_bytes bytes) followed by their (scale, bias) words (16 *
+ * Kp/g words); consecutive tiles are adjacent.  Codes: the tile's rows form
+ * two groups of 8 (rows 0-7, rows 8-15), each 8 * row_bytes bytes; inside a
+ * group, unit u (= 4B + p) of row r (0..7) sits at unit position
+ * 8u + sigma(u, r) (unit positions are 4b bytes apart), with
  *   b = 3: sigma = r
  *   b = 4: sigma = (r + 2 (u mod 4)) mod 8
  *   b = 6: sigma = (r + 4 ((u / 2) mod 2)) mod 8
- * Per group of g inputs: a (scale, bias) pair of bf16, stored as one 32-bit
- * word, scale in the low half.  The words of 16 consecutive rows form a tile
- * stored group-major: the word of (row r, group gi) is word
- * (r/16)*16*(Kp/g) + gi*16 + r%16.
+ * Scale/bias: per group of g inputs a (scale, bias) pair of bf16 in one
+ * 32-bit word, scale in the low half; inside a tile group-major: the word of
+ * (row r, group gi) is word gi*16 + r.
  *
- * A slot (one expert) is four sections, each starting on a 256-byte
- * boundary:  q_gate_up [2I rows] (row order: blocks of 16, block m = gate
- * rows 8m..8m+7 then up rows 8m..8m+7), q_down [H rows], sb_gate_up [2I rows,
- * same order], sb_down [H rows].  The slot's byte size is the end of the last
- * section rounded to 256 -- the "sum of its aligned read windows" that keys
- * its size class (1bit-MONSTER PR #137).
+ * A slot (one expert) is two projections, each starting on a 256-byte
+ * boundary: gate_up (2I rows; row order: blocks of 16, block m = gate rows
+ * 8m..8m+7 then up rows 8m..8m+7, so tile m is one block) then down (H rows).
+ * The slot's byte size is the end rounded to 256 -- the "sum of its aligned
+ * read windows" that keys its size class (1bit-MONSTER PR #137).
  */
 static int64_t orc_round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
@@ -285,28 +286,40 @@ int64_t orc_row_bytes(int32_t K, int32_t b) { return orc_round_up(K, 128) * b / 
 
 int64_t orc_row_groups(int32_t K, int32_t g) { return orc_round_up(K, 128) / g; }
 
-void orc_slot_layout(int32_t H, int32_t I, int32_t g, int32_t b_gu, int32_t b_d, int64_t* off /*[5]*/) {
+/* Bytes of one 16-row tile of a projection with K inputs per row. */
+int64_t orc_tile_bytes(int32_t K, int32_t g, int32_t b) { return 16 * orc_row_bytes(K, b) + 16 * orc_row_groups(K, g) * 4; }
+
+/* off[0] = gate_up projection, off[1] = down projection, off[2] = gate_up
+ * tile bytes, off[3] = down tile bytes, off[4] = slot bytes. */
+void orc_slot_layout(int32_t H, int32_t I, int32_t g, int32_t b_gu, int32_t b_d, int64_t* off) {
   int64_t o = 0;
   off[0] = 0;
-  o += (int64_t)2 * I * orc_row_bytes(H, b_gu);
+  o += (int64_t)(2 * I / 16) * orc_tile_bytes(H, g, b_gu);
   o = orc_round_up(o, 256);
   off[1] = o;
-  o += (int64_t)H * orc_row_bytes(I, b_d);
+  o += (int64_t)(H / 16) * orc_tile_bytes(I, g, b_d);
   o = orc_round_up(o, 256);
-  off[2] = o;
-  o += (int64_t)2 * I * orc_row_groups(H, g) * 4;
-  o = orc_round_up(o, 256);
-  off[3] = o;
-  o += (int64_t)H * orc_row_groups(I, g) * 4;
-  o = orc_round_up(o, 256);
+  off[2] = orc_tile_bytes(H, g, b_gu);
+  off[3] = orc_tile_bytes(I, g, b_d);
   off[4] = o; /* slot bytes */
 }
 
-/* Position of code bit j of input k of row `row` of a projection whose rows
- * are row_bytes long: byte offset of its 32-bit word from the projection's
- * start, and the bit inside that word. */
-static void orc_code_bit(int32_t row, int64_t row_bytes, int32_t k, int32_t b, int32_t j, int64_t* word_byte,
-                         int32_t* bit) {
+static uint32_t orc_load_word(const uint8_t* p) {
+  return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);
+}
+
+static void orc_store_word(uint8_t* p, uint32_t v) {
+  p[0] = (uint8_t)v;
+  p[1] = (uint8_t)(v >> 8);
+  p[2] = (uint8_t)(v >> 16);
+  p[3] = (uint8_t)(v >> 24);
+}
+
+/* Position of code bit j of input k of row `row` of a projection (rows of
+ * row_bytes code bytes, tiles of tile_bytes): byte offset of its 32-bit word
+ * from the projection's start, and the bit inside that word. */
+static void orc_code_bit(int32_t row, int64_t row_bytes, int64_t tile_bytes, int32_t k, int32_t b, int32_t j,
+                         int64_t* word_byte, int32_t* bit) {
   int32_t blk = k / 128, kk = k % 128;
   int32_t s = kk / 16, r16 = kk % 16;
   int32_t h = r16 / 8;
@@ -347,40 +360,29 @@ static void orc_code_bit(int32_t row, int64_t row_bytes, int32_t k, int32_t b, i
       }
     }
   }
-  *word_byte = (int64_t)(row / 8) * 8 * row_bytes + pos * 4 * b + 4 * wi;
+  *word_byte = (int64_t)(row / 16) * tile_bytes + (int64_t)((row % 16) / 8) * 8 * row_bytes + pos * 4 * b + 4 * wi;
   *bit = bi + (odd ? 16 : 0);
 }
 
-static uint32_t orc_load_word(const uint8_t* p) {
-  return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);
-}
-
-static void orc_store_word(uint8_t* p, uint32_t v) {
-  p[0] = (uint8_t)v;
-  p[1] = (uint8_t)(v >> 8);
-  p[2] = (uint8_t)(v >> 16);
-  p[3] = (uint8_t)(v >> 24);
-}
-
 /* Code of input k of row `row` in a projection of K inputs per row. */
-int32_t orc_get_code(const uint8_t* proj, int32_t K, int32_t row, int32_t k, int32_t b) {
-  int64_t rb = orc_row_bytes(K, b);
+int32_t orc_get_code(const uint8_t* proj, int32_t K, int32_t g, int32_t row, int32_t k, int32_t b) {
+  int64_t rb = orc_row_bytes(K, b), tb = orc_tile_bytes(K, g, b);
   int32_t q = 0;
   for (int32_t j = 0; j < b; ++j) {
     int64_t wb;
     int32_t bit;
-    orc_code_bit(row, rb, k, b, j, &wb, &bit);
+    orc_code_bit(row, rb, tb, k, b, j, &wb, &bit);
     q |= (int32_t)((orc_load_word(proj + wb) >> bit) & 1u) << j;
   }
   return q;
 }
 
-void orc_set_code(uint8_t* proj, int32_t K, int32_t row, int32_t k, int32_t b, int32_t q) {
-  int64_t rb = orc_row_bytes(K, b);
+void orc_set_code(uint8_t* proj, int32_t K, int32_t g, int32_t row, int32_t k, int32_t b, int32_t q) {
+  int64_t rb = orc_row_bytes(K, b), tb = orc_tile_bytes(K, g, b);
   for (int32_t j = 0; j < b; ++j) {
     int64_t wb;
     int32_t bit;
-    orc_code_bit(row, rb, k, b, j, &wb, &bit);
+    orc_code_bit(row, rb, tb, k, b, j, &wb, &bit);
     uint32_t v = orc_load_word(proj + wb);
     v &= ~(1u << bit);
     v |= (uint32_t)((q >> j) & 1) << bit;
@@ -388,8 +390,15 @@ void orc_set_code(uint8_t* proj, int32_t K, int32_t row, int32_t k, int32_t b, i
   }
 }
 
-/* Word index of the (scale, bias) word of (row, group gi), ng groups per row. */
-int64_t orc_sb_index(int32_t row, int64_t gi, int64_t ng) { return (int64_t)(row / 16) * 16 * ng + gi * 16 + row % 16; }
+/* Byte offset of the (scale, bias) word of (row, group gi) from the
+ * projection's start. */
+int64_t orc_sb_offset(int32_t row, int64_t gi, int32_t K, int32_t g, int32_t b) {
+  return (int64_t)(row / 16) * orc_tile_bytes(K, g, b) + 16 * orc_row_bytes(K, b) + 4 * (gi * 16 + row % 16);
+}
+
+static uint32_t orc_get_sb(const uint8_t* proj, int32_t row, int64_t gi, int32_t K, int32_t g, int32_t b) {
+  return orc_load_word(proj + orc_sb_offset(row, gi, K, g, b));
+}
 
 /* Storage row of logical gate/up row R (gate rows 0..I-1, up rows I..2I-1). */
 int32_t orc_gate_up_row(int32_t R, int32_t I) {
@@ -408,22 +417,19 @@ int32_t orc_gate_up_row(int32_t R, int32_t I) {
  *   q = clamp(rint((w - bias) / scale), 0, 2^b - 1), using the rounded scale
  *   and bias; q = 0 when scale == 0.
  * All arithmetic in fp32, one rounding per operation.
- * w: [rows, K] fp32 in storage row order (rows a multiple of 16).  q_out:
- * rows * row_bytes(K, b) bytes (zeroed here).  sb_out: rows * row_groups(K, g)
- * words (tile layout above).
+ * w: [rows, K] fp32 in storage row order (rows a multiple of 16).  proj:
+ * (rows/16) * tile_bytes(K, g, b) bytes, the tiles above (zeroed here).
  */
-void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32_t b, uint8_t* q_out,
-                       uint32_t* sb_out) {
-  int64_t rb = orc_row_bytes(K, b);
+void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32_t b, uint8_t* proj) {
   int64_t ng = orc_row_groups(K, g);
   int32_t qmax = (1 << b) - 1;
-  memset(q_out, 0, (size_t)(rb * rows));
+  memset(proj, 0, (size_t)((rows / 16) * orc_tile_bytes(K, g, b)));
   for (int32_t r = 0; r < rows; ++r) {
     const float* wr = w + (int64_t)r * K;
     for (int64_t gi = 0; gi < ng; ++gi) {
       int32_t k0 = (int32_t)(gi * g);
       if (k0 >= K) {
-        sb_out[orc_sb_index(r, gi, ng)] = 0u;
+        orc_store_word(proj + orc_sb_offset(r, gi, K, g, b), 0u);
         continue;
       }
       float mn = wr[k0], mx = wr[k0];
@@ -442,9 +448,9 @@ void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32
           if (t > (float)qmax) t = (float)qmax;
           q = (int32_t)t;
         }
-        orc_set_code(q_out, K, r, k, b, q);
+        orc_set_code(proj, K, g, r, k, b, q);
       }
-      sb_out[orc_sb_index(r, gi, ng)] = (uint32_t)sh | ((uint32_t)bh << 16);
+      orc_store_word(proj + orc_sb_offset(r, gi, K, g, b), (uint32_t)sh | ((uint32_t)bh << 16));
     }
   }
 }
@@ -454,15 +460,13 @@ void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32
 /* ------------------------------------------------------------------ */
 /* deq = fma(scale, q, bias) in fp32: one rounding.  Rows of K (unpadded), in
  * storage order. */
-void orc_dequant_rows(const uint8_t* q, const uint32_t* sb, int32_t rows, int32_t K, int32_t g, int32_t b,
-                      float* out) {
-  int64_t ng = orc_row_groups(K, g);
+void orc_dequant_rows(const uint8_t* proj, int32_t rows, int32_t K, int32_t g, int32_t b, float* out) {
   for (int32_t r = 0; r < rows; ++r) {
     for (int32_t k = 0; k < K; ++k) {
-      uint32_t sbw = sb[orc_sb_index(r, k / g, ng)];
+      uint32_t sbw = orc_get_sb(proj, r, k / g, K, g, b);
       float s = orc_bf16_to_f32((uint16_t)(sbw & 0xffffu));
       float bb = orc_bf16_to_f32((uint16_t)(sbw >> 16));
-      int32_t c = orc_get_code(q, K, r, k, b);
+      int32_t c = orc_get_code(proj, K, g, r, k, b);
       out[(int64_t)r * K + k] = fmaf(s, (float)c, bb);
     }
   }
@@ -475,11 +479,11 @@ void orc_dequant_slot(const uint8_t* slot, int32_t H, int32_t I, int32_t g, int3
   int64_t off[5];
   orc_slot_layout(H, I, g, b_gu, b_d, off);
   float* tmp = (float*)malloc(sizeof(float) * (size_t)2 * I * H);
-  orc_dequant_rows(slot + off[0], (const uint32_t*)(slot + off[2]), 2 * I, H, g, b_gu, tmp);
+  orc_dequant_rows(slot + off[0], 2 * I, H, g, b_gu, tmp);
   for (int32_t R = 0; R < 2 * I; ++R)
     memcpy(gate_up + (int64_t)R * H, tmp + (int64_t)orc_gate_up_row(R, I) * H, sizeof(float) * (size_t)H);
   free(tmp);
-  orc_dequant_rows(slot + off[1], (const uint32_t*)(slot + off[3]), H, I, g, b_d, down);
+  orc_dequant_rows(slot + off[1], H, I, g, b_d, down);
 }
 
 /* ------------------------------------------------------------------ */

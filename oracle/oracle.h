@@ -24,14 +24,13 @@ int orc_bits_supported(int32_t b);
 int64_t orc_row_bytes(int32_t K, int32_t b);
 int64_t orc_row_groups(int32_t K, int32_t g);
 void orc_slot_layout(int32_t H, int32_t I, int32_t g, int32_t b_gu, int32_t b_d, int64_t* off);
-int32_t orc_get_code(const uint8_t* proj, int32_t K, int32_t row, int32_t k, int32_t b);
-void orc_set_code(uint8_t* proj, int32_t K, int32_t row, int32_t k, int32_t b, int32_t q);
+int32_t orc_get_code(const uint8_t* proj, int32_t K, int32_t g, int32_t row, int32_t k, int32_t b);
+void orc_set_code(uint8_t* proj, int32_t K, int32_t g, int32_t row, int32_t k, int32_t b, int32_t q);
+int64_t orc_tile_bytes(int32_t K, int32_t g, int32_t b);
 int32_t orc_gate_up_row(int32_t R, int32_t I);
-int64_t orc_sb_index(int32_t row, int64_t gi, int64_t ng);
-void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32_t b, uint8_t* q_out,
-                       uint32_t* sb_out);
-void orc_dequant_rows(const uint8_t* q, const uint32_t* sb, int32_t rows, int32_t K, int32_t g, int32_t b,
-                      float* out);
+int64_t orc_sb_offset(int32_t row, int64_t gi, int32_t K, int32_t g, int32_t b);
+void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32_t b, uint8_t* proj);
+void orc_dequant_rows(const uint8_t* proj, int32_t rows, int32_t K, int32_t g, int32_t b, float* out);
 void orc_dequant_slot(const uint8_t* slot, int32_t H, int32_t I, int32_t g, int32_t b_gu, int32_t b_d,
                       float* gate_up, float* down);
 void orc_expert_ffn(const uint16_t* x, int32_t H, int32_t I, int32_t g, int32_t b_gu, int32_t b_d,

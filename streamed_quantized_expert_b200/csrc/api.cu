@@ -45,6 +45,10 @@ int device_sms() {
   return sms;
 }
 
+// Workspace: [control block (kWsControlBytes)][sort scratch | FFN scratch].
+// The control block must be zero before the first call with a workspace and
+// is left zero by every call; the sort and FFN scratch overlap (different
+// calls, stream-ordered).
 struct WsCarve {
   size_t sort, h, o, total;
 };
@@ -55,10 +59,8 @@ WsCarve carve(const moe_layer_desc& d, int T) {
   c.sort = (size_t)round_up((int64_t)sort_ws_bytes((int)np, d.E), 256);
   c.h = (size_t)round_up(np * d.I * 2, 256);
   c.o = T > kFusedMaxTokens ? (size_t)round_up(np * d.H * 4, 256) : 0;
-  // sort scratch and FFN scratch are used by different calls: overlap them
   const size_t ffn = c.h + c.o;
-  c.total = c.sort > ffn ? c.sort : ffn;
-  if (c.total == 0) c.total = 256;
+  c.total = kWsControlBytes + (c.sort > ffn ? c.sort : ffn);
   return c;
 }
 
@@ -91,10 +93,10 @@ moe_status moe_slot_layout(const moe_layer_desc* d, moe_slot_layout_t* out) {
   if (s != MOE_OK) return s;
   if (!out) return MOE_ERR_INVALID;
   const Layout L = make_layout(*d);
-  out->q_gate_up = (uint64_t)L.q_gu;
-  out->q_down = (uint64_t)L.q_d;
-  out->sb_gate_up = (uint64_t)L.sb_gu;
-  out->sb_down = (uint64_t)L.sb_d;
+  out->gate_up = (uint64_t)L.gu;
+  out->down = (uint64_t)L.d;
+  out->gate_up_tile_bytes = (uint64_t)L.tile_gu;
+  out->down_tile_bytes = (uint64_t)L.tile_d;
   out->slot_bytes = (uint64_t)L.slot_bytes;
   return MOE_OK;
 }
@@ -126,7 +128,8 @@ moe_status moe_sort(const int32_t* ids, const uint16_t* x, int32_t T, const moe_
   if (x && (!x_sorted || !aligned(x, 16) || !aligned(x_sorted, 16) || d->H % 8)) return MOE_ERR_INVALID;
   const WsCarve c = carve(*d, T);
   if (c.sort > 0 && (!ws || ws_bytes < c.total)) return MOE_ERR_CAPACITY;
-  return cuda_status(launch_sort(ids, x, T, d->k, d->E, d->H, offsets, pairs, active, n_active, x_sorted, ws,
+  void* scratch = c.sort > 0 ? static_cast<char*>(ws) + kWsControlBytes : nullptr;
+  return cuda_status(launch_sort(ids, x, T, d->k, d->E, d->H, offsets, pairs, active, n_active, x_sorted, scratch,
                                  stream));
 }
 
@@ -196,8 +199,9 @@ __attribute__((visibility("hidden"))) moe_status moe_internal_expert_ffn(
   a.pass_begin = pass_begin;
   a.pass_len = pass_len;
   a.y = y_accum;
-  a.h = static_cast<uint16_t*>(ws);
-  a.o = c.o ? reinterpret_cast<float*>(static_cast<char*>(ws) + c.h) : nullptr;
+  a.ctl = static_cast<unsigned*>(ws);
+  a.h = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + kWsControlBytes);
+  a.o = c.o ? reinterpret_cast<float*>(static_cast<char*>(ws) + kWsControlBytes + c.h) : nullptr;
   a.dev_err = dev_err;
   a.y_overwrite = overwrite ? 1 : 0;
   return cuda_status(launch_ffn_decode(a, *d, device_sms(), stream));
@@ -223,15 +227,15 @@ moe_status moe_dequant_slot(const void* pool, int32_t slot, const moe_layer_desc
 }
 
 moe_status moe_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t group, int32_t bits,
-                             int32_t gate_up_I, uint8_t* q, uint32_t* sb, cudaStream_t stream) {
+                             int32_t gate_up_I, uint8_t* proj, cudaStream_t stream) {
   if (rows < 0 || K < 1 || rows % 16) return MOE_ERR_INVALID;
   if (gate_up_I < 0 || (gate_up_I > 0 && (rows != 2 * gate_up_I || gate_up_I % 8))) return MOE_ERR_INVALID;
   if (group != 32 && group != 64 && group != 128) return MOE_ERR_UNSUPPORTED;
   if (bits != 3 && bits != 4 && bits != 6) return MOE_ERR_UNSUPPORTED;
   if (K % group) return MOE_ERR_INVALID;
   if (rows == 0) return MOE_OK;
-  if (!w || !q || !sb || !aligned(q, 4) || !aligned(sb, 4)) return MOE_ERR_INVALID;
-  return cuda_status(launch_quantize(w, rows, K, group, bits, gate_up_I, q, sb, stream));
+  if (!w || !proj || !aligned(proj, 16)) return MOE_ERR_INVALID;
+  return cuda_status(launch_quantize(w, rows, K, group, bits, gate_up_I, proj, stream));
 }
 
 moe_status moe_exp_portable(const float* x, int64_t n, float* out, cudaStream_t stream) {

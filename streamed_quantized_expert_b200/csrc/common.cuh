@@ -21,11 +21,17 @@ __host__ __device__ constexpr int64_t row_bytes(int64_t K, int bits) { return pa
 __host__ __device__ constexpr int64_t row_groups(int64_t K, int g) { return padded_k(K) / g; }
 
 struct Layout {
-  int64_t q_gu, q_d, sb_gu, sb_d, slot_bytes;
-  int64_t rb_gu, rb_d;  // row bytes
-  int ng_gu, ng_d;      // groups per (padded) row
-  int nblk_gu, nblk_d;  // 128-input blocks per row
+  int64_t gu, d;            // byte offsets of the gate_up and down projections in a slot
+  int64_t rb_gu, rb_d;      // code bytes of one row
+  int ng_gu, ng_d;          // (scale, bias) groups per (padded) row
+  int nblk_gu, nblk_d;      // 128-input blocks per row
+  int64_t tile_gu, tile_d;  // bytes of one 16-row tile: codes, then scale/bias words
+  int64_t slot_bytes;
 };
+
+__host__ __device__ constexpr int64_t tile_bytes(int64_t K, int g, int bits) {
+  return 16 * row_bytes(K, bits) + 16 * row_groups(K, g) * 4;
+}
 
 inline Layout make_layout(const moe_layer_desc& d) {
   Layout L{};
@@ -35,16 +41,11 @@ inline Layout make_layout(const moe_layer_desc& d) {
   L.ng_d = (int)row_groups(d.I, d.group);
   L.nblk_gu = (int)(padded_k(d.H) / 128);
   L.nblk_d = (int)(padded_k(d.I) / 128);
-  int64_t o = 0;
-  L.q_gu = o;
-  o = round_up(o + (int64_t)2 * d.I * L.rb_gu, 256);
-  L.q_d = o;
-  o = round_up(o + (int64_t)d.H * L.rb_d, 256);
-  L.sb_gu = o;
-  o = round_up(o + (int64_t)2 * d.I * L.ng_gu * 4, 256);
-  L.sb_d = o;
-  o = round_up(o + (int64_t)d.H * L.ng_d * 4, 256);
-  L.slot_bytes = o;
+  L.tile_gu = tile_bytes(d.H, d.group, d.bits_gu);
+  L.tile_d = tile_bytes(d.I, d.group, d.bits_down);
+  L.gu = 0;
+  L.d = round_up((int64_t)(2 * d.I / 16) * L.tile_gu, 256);
+  L.slot_bytes = round_up(L.d + (int64_t)(d.H / 16) * L.tile_d, 256);
   return L;
 }
 
@@ -139,9 +140,10 @@ __device__ __forceinline__ float pair_hi_q(uint32_t p, int a) {
   return (__uint_as_float(p & 0xFFFF0000u) - 128.0f) * (a ? 0.125f : 1.0f);
 }
 
-// Rows are stored in groups of 8 (unit-major inside a group): unit u of row r
-// sits at unit position 8u + sigma(u, r), which keeps the per-thread unit
-// loads of the GEMV kernels free of shared-memory bank conflicts.
+// Rows are stored in tiles of 16 (codes of two 8-row groups, then the tile's
+// scale/bias words).  Inside a group (unit-major) unit u of row r sits at unit
+// position 8u + sigma(u, r), which keeps the per-thread unit loads of the GEMV
+// kernels free of shared-memory bank conflicts.
 template <int B>
 __host__ __device__ constexpr int unit_sigma(int u, int r) {
   return B == 3 ? r : B == 4 ? (r + 2 * (u & 3)) & 7 : (r + 4 * ((u >> 1) & 1)) & 7;
@@ -149,14 +151,14 @@ __host__ __device__ constexpr int unit_sigma(int u, int r) {
 
 // Byte offset of unit u of row `row` from the start of its projection.
 template <int B>
-__host__ __device__ constexpr int64_t unit_offset(int64_t row, int64_t u, int64_t row_bytes) {
-  return (row >> 3) * 8 * row_bytes + (8 * u + unit_sigma<B>((int)u, (int)(row & 7))) * 4 * B;
+__host__ __device__ constexpr int64_t unit_offset(int64_t row, int64_t u, int64_t row_bytes, int64_t tile) {
+  return (row >> 4) * tile + ((row >> 3) & 1) * 8 * row_bytes + (8 * u + unit_sigma<B>((int)u, (int)(row & 7))) * 4 * B;
 }
 
-// Word index of the (scale, bias) word of (row, group gi), ng groups per row:
-// tiles of 16 rows, group-major inside a tile.
-__host__ __device__ constexpr int64_t sb_index(int64_t row, int64_t gi, int64_t ng) {
-  return (row >> 4) * 16 * ng + gi * 16 + (row & 15);
+// Byte offset of the (scale, bias) word of (row, group gi) from the start of
+// its projection: group-major inside the row's tile, after the tile's codes.
+__host__ __device__ constexpr int64_t sb_offset(int64_t row, int64_t gi, int64_t row_bytes, int64_t tile) {
+  return (row >> 4) * tile + 16 * row_bytes + 4 * (gi * 16 + (row & 15));
 }
 
 // Storage row of logical gate/up row R (blocks of 16: 8 gate rows, 8 up rows).

@@ -31,10 +31,11 @@ struct FfnArgs {
   uint16_t* h;  // workspace: [T*k][I] bf16, by sorted position
   float* o;     // workspace: [T*k][H] fp32, by flat pair index (T > kFusedMaxTokens)
   int32_t* dev_err;
+  unsigned* ctl;    // workspace control block (grid barrier of the fused kernel); zero between calls
   int y_overwrite;  // 1: y = result (single pass over all experts); 0: y += result
   Layout L;
   // filled by the launcher
-  int64_t q_gu, q_d, sb_gu, sb_d, rb_gu, rb_d;
+  int64_t q_gu, q_d, tile_gu, tile_d, rb_gu, rb_d;
   int ng_gu, ng_d, nblk_gu, nblk_d;
   int gu_stage_bytes, d_stage_bytes, gu_nstage, d_nstage;
 };
@@ -69,12 +70,13 @@ cudaError_t launch_lookup(const int32_t* table, const int32_t* active, const int
                           int pass_len, int n_slots, int32_t* slots, int32_t* miss, int32_t* n_miss,
                           int32_t* dev_err, cudaStream_t st);
 cudaError_t launch_exp(const float* x, int64_t n, float* out, cudaStream_t st);
-cudaError_t launch_quantize(const float* w, int rows, int K, int g, int b, int gu_I, uint8_t* q, uint32_t* sb,
-                            cudaStream_t st);
+cudaError_t launch_quantize(const float* w, int rows, int K, int g, int b, int gu_I, uint8_t* q, cudaStream_t st);
 cudaError_t launch_dequant_slot(const uint8_t* slot, const moe_layer_desc& d, const Layout& L, float* out32,
                                 uint16_t* out16, cudaStream_t st);
 size_t ffn_ws_bytes(const moe_layer_desc& d, int T);
 bool ffn_decode_supported(const moe_layer_desc& d);
 cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st);
+cudaError_t launch_ffn_fused(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st);
+constexpr size_t kWsControlBytes = 256;  // head of the workspace: grid-barrier words
 
 }  // namespace moe

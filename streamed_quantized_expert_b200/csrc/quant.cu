@@ -40,20 +40,16 @@ __device__ __forceinline__ void block_bit(int kk, int b, int j, int& word, int& 
   bit = bi + ((kk & 1) ? 16 : 0);
 }
 
-template <int B>
-__device__ __forceinline__ int64_t unit_off_b(int64_t row, int64_t u, int64_t rb) {
-  return unit_offset<B>(row, u, rb);
-}
-
-__device__ __forceinline__ int64_t unit_off(int b, int64_t row, int64_t u, int64_t rb) {
-  return b == 3 ? unit_off_b<3>(row, u, rb) : b == 4 ? unit_off_b<4>(row, u, rb) : unit_off_b<6>(row, u, rb);
+__device__ __forceinline__ int64_t unit_off(int b, int64_t row, int64_t u, int64_t rb, int64_t tile) {
+  return b == 3 ? unit_offset<3>(row, u, rb, tile) : b == 4 ? unit_offset<4>(row, u, rb, tile)
+                                                            : unit_offset<6>(row, u, rb, tile);
 }
 
 // One warp per (row, 128-block); lane owns inputs 4*lane .. 4*lane+3.
 // gu_I > 0: the rows are a gate/up matrix (gate rows 0..gu_I-1, then up
 // rows), written to their storage rows; else row r is storage row r.
 __global__ void __launch_bounds__(256) quantize_kernel(const float* __restrict__ w, int rows, int K, int g, int b,
-                                                       int gu_I, uint8_t* __restrict__ q, uint32_t* __restrict__ sb) {
+                                                       int gu_I, uint8_t* __restrict__ q) {
   __shared__ uint32_t s_words[8][24];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nblk = (int)(padded_k(K) / 128);
@@ -99,15 +95,15 @@ __global__ void __launch_bounds__(256) quantize_kernel(const float* __restrict__
     }
   }
   __syncwarp();
-  const int64_t rb = row_bytes(K, b);
+  const int64_t rb = row_bytes(K, b), tile = tile_bytes(K, g, b);
   const int srow = gu_I > 0 ? gate_up_row(r, gu_I) : r;
   if (lane < 4 * b) {
     const int p = lane / b, wi = lane % b;
-    reinterpret_cast<uint32_t*>(q + unit_off(b, srow, 4 * blk + p, rb))[wi] = s_words[warp][lane];
+    reinterpret_cast<uint32_t*>(q + unit_off(b, srow, 4 * blk + p, rb, tile))[wi] = s_words[warp][lane];
   }
   if (lane % lanes_per_group == 0) {
     const int gi = (blk * 128 + 4 * lane) / g;
-    sb[sb_index(srow, gi, row_groups(K, g))] = (uint32_t)sh | ((uint32_t)bh << 16);
+    *reinterpret_cast<uint32_t*>(q + sb_offset(srow, gi, rb, tile)) = (uint32_t)sh | ((uint32_t)bh << 16);
   }
 }
 
@@ -115,27 +111,27 @@ __global__ void __launch_bounds__(256) quantize_kernel(const float* __restrict__
 // through the same unpack_unit<B> the FFN kernels use.  out[r][k] = fmaf(s,
 // q, b), r the logical row (gu_I > 0: gate/up row order).
 template <int B>
-__global__ void dequant_kernel(const uint8_t* __restrict__ qbase, const uint32_t* __restrict__ sbbase, int rows,
-                               int K, int g, int gu_I, float* __restrict__ out32, uint16_t* __restrict__ out16) {
+__global__ void dequant_kernel(const uint8_t* __restrict__ qbase, int rows, int K, int g, int gu_I,
+                               float* __restrict__ out32, uint16_t* __restrict__ out16) {
   const int nunit = (int)(padded_k(K) / 32);
   const int64_t task = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (task >= (int64_t)rows * nunit) return;
   const int lr = (int)(task / nunit), u = (int)(task % nunit);
   const int r = gu_I > 0 ? gate_up_row(lr, gu_I) : lr;  // storage row
   const int blk = u >> 2, t = u & 3;
-  const uint32_t* wp = reinterpret_cast<const uint32_t*>(qbase + unit_offset<B>(r, u, row_bytes(K, B)));
+  const int64_t rb = row_bytes(K, B), tile = tile_bytes(K, g, B);
+  const uint32_t* wp = reinterpret_cast<const uint32_t*>(qbase + unit_offset<B>(r, u, rb, tile));
   uint32_t wv[B];
 #pragma unroll
   for (int i = 0; i < B; ++i) wv[i] = wp[i];
   uint32_t p[16];
   unpack_unit<B>(wv, p);
-  const int64_t ng = row_groups(K, g);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int a = PairShift<B>::a(i);
     const int k = blk * 128 + pair_input(i, t);
     if (k >= K) continue;  // K is a multiple of 32, so k+1 < K too
-    const uint32_t sbw = sbbase[sb_index(r, k / g, ng)];
+    const uint32_t sbw = *reinterpret_cast<const uint32_t*>(qbase + sb_offset(r, k / g, rb, tile));
     const float s = bf16_lo(sbw), bb = bf16_hi(sbw);
     const float v0 = __fmaf_rn(s, pair_lo_q(p[i], a), bb);
     const float v1 = __fmaf_rn(s, pair_hi_q(p[i], a), bb);
@@ -151,34 +147,32 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ qbase, const uint32_t
 }
 
 template <int B>
-static void launch_dq(const uint8_t* q, const uint32_t* sb, int rows, int K, int g, int gu_I, float* o32,
-                      uint16_t* o16, cudaStream_t st) {
+static void launch_dq(const uint8_t* q, int rows, int K, int g, int gu_I, float* o32, uint16_t* o16,
+                      cudaStream_t st) {
   const int64_t n = (int64_t)rows * (padded_k(K) / 32);
-  dequant_kernel<B><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(q, sb, rows, K, g, gu_I, o32, o16);
+  dequant_kernel<B><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(q, rows, K, g, gu_I, o32, o16);
 }
 
-static void dq_dispatch(int b, const uint8_t* q, const uint32_t* sb, int rows, int K, int g, int gu_I, float* o32,
-                        uint16_t* o16, cudaStream_t st) {
-  if (b == 3) launch_dq<3>(q, sb, rows, K, g, gu_I, o32, o16, st);
-  else if (b == 4) launch_dq<4>(q, sb, rows, K, g, gu_I, o32, o16, st);
-  else launch_dq<6>(q, sb, rows, K, g, gu_I, o32, o16, st);
+static void dq_dispatch(int b, const uint8_t* q, int rows, int K, int g, int gu_I, float* o32, uint16_t* o16,
+                        cudaStream_t st) {
+  if (b == 3) launch_dq<3>(q, rows, K, g, gu_I, o32, o16, st);
+  else if (b == 4) launch_dq<4>(q, rows, K, g, gu_I, o32, o16, st);
+  else launch_dq<6>(q, rows, K, g, gu_I, o32, o16, st);
 }
 
 cudaError_t launch_dequant_slot(const uint8_t* slot, const moe_layer_desc& d, const Layout& L, float* out32,
                                 uint16_t* out16, cudaStream_t st) {
   const int64_t n_gu = (int64_t)2 * d.I * d.H;
-  dq_dispatch(d.bits_gu, slot + L.q_gu, reinterpret_cast<const uint32_t*>(slot + L.sb_gu), 2 * d.I, d.H, d.group,
-              d.I, out32, out16, st);
-  dq_dispatch(d.bits_down, slot + L.q_d, reinterpret_cast<const uint32_t*>(slot + L.sb_d), d.H, d.I, d.group, 0,
-              out32 ? out32 + n_gu : nullptr, out16 ? out16 + n_gu : nullptr, st);
+  dq_dispatch(d.bits_gu, slot + L.gu, 2 * d.I, d.H, d.group, d.I, out32, out16, st);
+  dq_dispatch(d.bits_down, slot + L.d, d.H, d.I, d.group, 0, out32 ? out32 + n_gu : nullptr,
+              out16 ? out16 + n_gu : nullptr, st);
   return cudaGetLastError();
 }
 
-cudaError_t launch_quantize(const float* w, int rows, int K, int g, int b, int gu_I, uint8_t* q, uint32_t* sb,
-                            cudaStream_t st) {
+cudaError_t launch_quantize(const float* w, int rows, int K, int g, int b, int gu_I, uint8_t* q, cudaStream_t st) {
   const int64_t tasks = (int64_t)rows * (padded_k(K) / 128);
   if (tasks == 0) return cudaSuccess;
-  quantize_kernel<<<(unsigned)((tasks + 7) / 8), 256, 0, st>>>(w, rows, K, g, b, gu_I, q, sb);
+  quantize_kernel<<<(unsigned)((tasks + 7) / 8), 256, 0, st>>>(w, rows, K, g, b, gu_I, q);
   return cudaGetLastError();
 }
 

@@ -57,8 +57,8 @@ class LayerCtx(C.Structure):
 
 
 class SlotLayout(C.Structure):
-    _fields_ = [("q_gate_up", C.c_uint64), ("q_down", C.c_uint64), ("sb_gate_up", C.c_uint64),
-                ("sb_down", C.c_uint64), ("slot_bytes", C.c_uint64)]
+    _fields_ = [("gate_up", C.c_uint64), ("down", C.c_uint64), ("gate_up_tile_bytes", C.c_uint64),
+                ("down_tile_bytes", C.c_uint64), ("slot_bytes", C.c_uint64)]
 
 
 _lib = None
@@ -84,7 +84,7 @@ def lib():
             "moe_expert_ffn_noalloc": (C.c_int, [P, i32, D, P, i32, P, P, P, P, P, P, P, i32, i32, P, P, P]),
             "moe_noalloc_scratch_bytes": (sz, []),
             "moe_dequant_slot": (C.c_int, [P, i32, D, P, P, P]),
-            "moe_quantize_rows": (C.c_int, [P, i32, i32, i32, i32, i32, P, P, P]),
+            "moe_quantize_rows": (C.c_int, [P, i32, i32, i32, i32, i32, P, P]),
             "moe_exp_portable": (C.c_int, [P, i64, P, P]),
             "moe_status_string": (C.c_char_p, [C.c_int]),
             "moe_last_cuda_error": (C.c_char_p, []),
@@ -212,8 +212,8 @@ def moe_dequant_slot(pool, slot, d, out_fp32, out_bf16, stream=None) -> None:
                                _stream(stream)), "moe_dequant_slot")
 
 
-def moe_quantize_rows(w, rows, K, group, bits, q, sb, stream=None, gate_up_I=0) -> None:
-    _ck(lib().moe_quantize_rows(_ptr(w), int(rows), int(K), int(group), int(bits), int(gate_up_I), _ptr(q), _ptr(sb),
+def moe_quantize_rows(w, rows, K, group, bits, proj, stream=None, gate_up_I=0) -> None:
+    _ck(lib().moe_quantize_rows(_ptr(w), int(rows), int(K), int(group), int(bits), int(gate_up_I), _ptr(proj),
                                 _stream(stream)), "moe_quantize_rows")
 
 

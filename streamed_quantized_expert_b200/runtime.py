@@ -43,9 +43,8 @@ def quantize_bank_gpu(E: int, desc: ops.LayerDesc, seed: int, device="cuda", std
     for e in range(E):
         w_gu, w_d = synth.expert_weights_torch(seed, e, H, I, device, std)
         base = slot.data_ptr()
-        ops.moe_quantize_rows(w_gu, 2 * I, H, g, desc.bits_gu, base + lay.q_gate_up, base + lay.sb_gate_up,
-                              gate_up_I=I)
-        ops.moe_quantize_rows(w_d, H, I, g, desc.bits_down, base + lay.q_down, base + lay.sb_down)
+        ops.moe_quantize_rows(w_gu, 2 * I, H, g, desc.bits_gu, base + lay.gate_up, gate_up_I=I)
+        ops.moe_quantize_rows(w_d, H, I, g, desc.bits_down, base + lay.down)
         bank[e].copy_(slot, non_blocking=False)
     return bank
 
@@ -96,7 +95,7 @@ class Streamer:
         self.dev_err = torch.zeros(1, dtype=torch.int32, device=self.device)
         ws = max(ops.moe_workspace_bytes(l.desc, T) for l in layers)
         self.ws_bytes = ws
-        self.ws = torch.empty(ws, dtype=torch.uint8, device=self.device)
+        self.ws = torch.zeros(ws, dtype=torch.uint8, device=self.device)
         self.x_sorted = None
         self.y = torch.zeros((T, self.H), dtype=torch.float32, device=self.device)
         self.installed_bytes = 0

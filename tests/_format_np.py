@@ -57,17 +57,22 @@ def _bit_positions(K, b):
     return U, W, B
 
 
-def decode_rows(q, K, b):
-    """q uint8 [rows, Kp*b/8] (a whole projection, rows in groups of 8) ->
-    codes int64 [rows, K]."""
-    q = np.ascontiguousarray(q, dtype=np.uint8)
-    rows = q.shape[0]
-    rb = q.shape[1]
-    words = q.reshape(-1).view("<u4").astype(np.int64)
+def geometry(K, g, b):
+    """(row bytes of codes, groups per row, tile bytes)."""
+    rb = ceil128(K) * b // 8
+    ng = ceil128(K) // g
+    return rb, ng, 16 * rb + 16 * ng * 4
+
+
+def decode_rows(proj, rows, K, g, b):
+    """proj: a projection's bytes (tiles of 16 rows: codes, then scale/bias
+    words) -> codes int64 [rows, K]."""
+    rb, ng, tb = geometry(K, g, b)
+    words = np.ascontiguousarray(proj, dtype=np.uint8).reshape(-1).view("<u4").astype(np.int64)
     U, W, B = _bit_positions(K, b)
     codes = np.zeros((rows, U.shape[0]), np.int64)
     for r in range(rows):
-        grp_word = (r // 8) * 8 * rb // 4
+        grp_word = ((r // 16) * tb + ((r % 16) // 8) * 8 * rb) // 4
         for j in range(b):
             pos = 8 * U[:, j] + _sigma(U[:, j], r % 8, b)
             idx = grp_word + pos * b + W[:, j]
@@ -75,19 +80,19 @@ def decode_rows(q, K, b):
     return codes[:, :K]
 
 
-def sb_rows(sb_flat, rows, ng):
-    """Flat scale/bias words in the 16-row tile (group-major) order -> [rows, ng]."""
-    t = np.ascontiguousarray(sb_flat, dtype=np.uint32).reshape(rows // 16, ng, 16)
+def sb_rows(proj, rows, K, g, b):
+    """The (scale, bias) words of a projection as [rows, groups]."""
+    rb, ng, tb = geometry(K, g, b)
+    t = np.ascontiguousarray(proj, dtype=np.uint8).reshape(rows // 16, tb)[:, 16 * rb:]
+    t = np.ascontiguousarray(t).view("<u4").reshape(rows // 16, ng, 16)
     return t.transpose(0, 2, 1).reshape(rows, ng)
 
 
-def dequant_rows(q, sb, K, g, b):
+def dequant_rows(proj, rows, K, g, b):
     """Closed form of fma(scale, q, bias) in fp32: the exact product-sum in
-    float64 (exact for bf16 scale/bias and q < 64), rounded once to fp32.
-    sb: the flat words as stored (16-row tiles, group-major)."""
-    codes = decode_rows(q, K, b).astype(np.float64)
-    rows = q.shape[0]
-    sb = sb_rows(sb, rows, np.asarray(sb).size // rows)
+    float64 (exact for bf16 scale/bias and q < 64), rounded once to fp32."""
+    codes = decode_rows(proj, rows, K, g, b).astype(np.float64)
+    sb = sb_rows(proj, rows, K, g, b)
     s = ((sb & 0xFFFF).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     bb = ((sb >> 16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     gi = np.arange(K) // g

@@ -38,7 +38,7 @@ def test_sizes_match_oracle(lib, orc):
         off, n = orc.slot_layout(H, I, g, bg, bd)
         lay = ops.moe_slot_layout(d)
         assert ops.moe_slot_bytes(d) == n == lay.slot_bytes
-        assert [lay.q_gate_up, lay.q_down, lay.sb_gate_up, lay.sb_down] == off
+        assert [lay.gate_up, lay.down, lay.gate_up_tile_bytes, lay.down_tile_bytes] == off
 
 
 def test_argument_checks(lib):
@@ -58,7 +58,7 @@ def test_argument_checks(lib):
         ops.moe_install_slots(1 << 20, 256, 4, [1 << 21], [4])  # slot id past the pool
     assert ei.value.status == ops.MOE_ERR_INVALID
     with pytest.raises(ops.MoeError) as ei:
-        ops.moe_quantize_rows(1 << 20, 16, 64, 32, 5, 1 << 21, 1 << 22)
+        ops.moe_quantize_rows(1 << 20, 16, 64, 32, 5, 1 << 21)
     assert ei.value.status == ops.MOE_ERR_UNSUPPORTED
     with pytest.raises(ops.MoeError) as ei:  # workspace too small
         ops.moe_expert_ffn(1 << 20, 4, d, 1 << 24, 8, 1 << 21, 1 << 21, 1 << 21, 1 << 21, 1 << 21, 1 << 21,

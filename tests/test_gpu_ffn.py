@@ -44,7 +44,7 @@ class Setup:
     def gpu(self, x, ids, w, T, passes=None, table=None):
         E, k = self.E, self.k
         ws_b = ops.moe_workspace_bytes(self.d, T)
-        ws = torch.empty(ws_b, dtype=torch.uint8, device="cuda")
+        ws = torch.zeros(ws_b, dtype=torch.uint8, device="cuda")
         offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
         pairs = torch.empty(max(T * k, 1), dtype=torch.int32, device="cuda")
         active = torch.empty(E, dtype=torch.int32, device="cuda")

@@ -47,13 +47,11 @@ def test_quantize_bit_exact(orc, rows, K, g, b):
     w = (synth.rng(rows, K, g, b).standard_normal((rows, K), dtype=np.float32) * np.float32(0.02))
     w[0, :g] = np.float32(0.5)  # constant group
     w[1, :] = 0.0
-    qr, sbr = orc.quantize_rows(w, g, b)
-    q = torch.zeros(qr.shape, dtype=torch.uint8, device="cuda")
-    sb = torch.zeros(sbr.shape, dtype=torch.int32, device="cuda")
-    ops.moe_quantize_rows(dev(w), rows, K, g, b, q, sb)
+    ref = orc.quantize_rows(w, g, b)
+    proj = torch.zeros(ref.shape, dtype=torch.uint8, device="cuda")
+    ops.moe_quantize_rows(dev(w), rows, K, g, b, proj)
     torch.cuda.synchronize()
-    assert np.array_equal(q.cpu().numpy(), qr)
-    assert np.array_equal(sb.cpu().numpy().view(np.uint32), sbr)
+    assert np.array_equal(proj.cpu().numpy(), ref)
 
 
 def test_quantize_gate_up_order_bit_exact(orc):
@@ -65,8 +63,8 @@ def test_quantize_gate_up_order_bit_exact(orc):
     lay = ops.moe_slot_layout(d)
     slot = torch.zeros(lay.slot_bytes, dtype=torch.uint8, device="cuda")
     base = slot.data_ptr()
-    ops.moe_quantize_rows(dev(w_gu), 2 * I, H, g, bg, base + lay.q_gate_up, base + lay.sb_gate_up, gate_up_I=I)
-    ops.moe_quantize_rows(dev(w_d), H, I, g, bd, base + lay.q_down, base + lay.sb_down)
+    ops.moe_quantize_rows(dev(w_gu), 2 * I, H, g, bg, base + lay.gate_up, gate_up_I=I)
+    ops.moe_quantize_rows(dev(w_d), H, I, g, bd, base + lay.down)
     torch.cuda.synchronize()
     assert np.array_equal(slot.cpu().numpy(), ref)
 
@@ -124,7 +122,7 @@ def test_sort(orc, T, E, k):
     x_np = synth.activations(T, 0, T, H)
     d = ops.desc(E, k, H, 32, 32, 4)
     ws_b = ops.moe_workspace_bytes(d, T)
-    ws = torch.empty(ws_b, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(ws_b, dtype=torch.uint8, device="cuda")
     offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
     pairs = torch.empty(T * k, dtype=torch.int32, device="cuda")
     active = torch.full((E,), -1, dtype=torch.int32, device="cuda")

@@ -20,14 +20,12 @@ def _bank(orc, E, H, I, g, b_gu, b_d, seed=0):
         s = orc.build_slot(w_gu, w_d, g, b_gu, b_d)
         slots.append(s)
         # dequantise with the independent numpy decoder
-        qg = s[off[0]: off[0] + 2 * I * orc.row_bytes(H, b_gu)].reshape(2 * I, -1)
-        sg = s[off[2]: off[2] + 2 * I * orc.row_groups(H, g) * 4].view(np.uint32).reshape(2 * I, -1)
-        qd = s[off[1]: off[1] + H * orc.row_bytes(I, b_d)].reshape(H, -1)
-        sd = s[off[3]: off[3] + H * orc.row_groups(I, g) * 4].view(np.uint32).reshape(H, -1)
-        gu_stored = F.dequant_rows(qg, sg, H, g, b_gu)
+        pg = s[off[0]: off[0] + 2 * I // 16 * off[2]]
+        pd = s[off[1]: off[1] + H // 16 * off[3]]
+        gu_stored = F.dequant_rows(pg, 2 * I, H, g, b_gu)
         gu_logical = gu_stored[[F.gate_up_storage_row(R, I) for R in range(2 * I)]]
         dense.append((gu_logical.astype(np.float64),
-                      F.dequant_rows(qd, sd, I, g, b_d).astype(np.float64)))
+                      F.dequant_rows(pd, H, I, g, b_d).astype(np.float64)))
     return slots, dense
 
 

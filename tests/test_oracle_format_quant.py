@@ -13,17 +13,18 @@ from tests import _format_np as F
 @pytest.mark.parametrize("K", [32, 64, 128, 512, 768, 2048])
 def test_code_roundtrip_and_independent_decoder(orc, b, K):
     r = np.random.default_rng(b * 1000 + K)
-    rows = 16
+    rows, g = 32, 32
     rb = orc.row_bytes(K, b)
     assert rb == F.ceil128(K) * b // 8
-    q = np.zeros((rows, rb), np.uint8)
+    assert orc.tile_bytes(K, g, b) == F.geometry(K, g, b)[2]
+    proj = np.zeros(rows // 16 * orc.tile_bytes(K, g, b), np.uint8)
     codes = r.integers(0, 1 << b, size=(rows, K))
     for i in range(rows):
         for k in range(K):
-            orc.set_code(q, K, i, k, b, int(codes[i, k]))
+            orc.set_code(proj, K, g, i, k, b, int(codes[i, k]))
     for i in range(rows):
-        assert [orc.get_code(q, K, i, k, b) for k in range(K)] == codes[i].tolist()
-    assert np.array_equal(F.decode_rows(q, K, b), codes)
+        assert [orc.get_code(proj, K, g, i, k, b) for k in range(K)] == codes[i].tolist()
+    assert np.array_equal(F.decode_rows(proj, rows, K, g, b), codes)
 
 
 @pytest.mark.parametrize("b", [3, 4, 6])
@@ -31,15 +32,17 @@ def test_layout_is_a_bijection(orc, b):
     # every bit of an 8-row group of 128-input blocks belongs to exactly one
     # (row, input, code bit): setting the codes one by one to all-ones adds b
     # new bits each time and ends with every byte 0xFF
-    q = np.zeros((8, orc.row_bytes(128, b)), np.uint8)
+    g = 128
+    proj = np.zeros(orc.tile_bytes(128, g, b), np.uint8)
+    codes = proj[: 16 * orc.row_bytes(128, b)]  # the tile's code bytes (a view)
     seen = 0
-    for row in range(8):
+    for row in range(16):
         for k in range(128):
-            orc.set_code(q, 128, row, k, b, (1 << b) - 1)
-            n = int(np.unpackbits(q).sum())
+            orc.set_code(proj, 128, g, row, k, b, (1 << b) - 1)
+            n = int(np.unpackbits(proj).sum())
             assert n == seen + b
             seen = n
-    assert np.all(q == 0xFF)
+    assert np.all(codes == 0xFF) and np.all(proj[codes.size:] == 0)
     # the numpy description agrees: unit-word-bit triples cover a unit exactly once
     U, W, B = F._bit_positions(128, b)
     flat = ((U * b + W) * 32 + B).reshape(-1)
@@ -55,7 +58,8 @@ def test_slot_sizes_for_the_workload_shapes(orc):
     # H=2048, I=768, 4-bit g64
     assert orc.slot_bytes(2048, 768, 64, 4, 4) == 2_654_208
     off, n = orc.slot_layout(2048, 512, 64, 3, 3)
-    assert off == [0, 786_432, 1_179_648, 1_310_720] and all(o % 256 == 0 for o in off)
+    # 64 gate/up tiles of 16 x 768 B codes + 16 x 32 words; 128 down tiles of 16 x 192 B + 16 x 8 words
+    assert off == [0, 917_504, 14_336, 3_584] and n == 1_376_256
 
 
 @pytest.mark.parametrize("b,g", [(3, 64), (4, 32), (4, 64), (6, 64), (4, 128), (3, 32)])
@@ -64,11 +68,11 @@ def test_quantizer_properties(orc, b, g):
     K = 256
     w = (r.standard_normal((32, K)) * 0.02).astype(np.float32)
     w[3, :g] = np.float32(0.0123)  # constant group
-    q, sb = orc.quantize_rows(w, g, b)
-    codes = F.decode_rows(q, K, b)
+    proj = orc.quantize_rows(w, g, b)
+    codes = F.decode_rows(proj, 32, K, g, b)
     assert codes.min() >= 0 and codes.max() <= (1 << b) - 1
-    deq = orc.dequant_rows(q, sb, K, g, b)
-    sbr = F.sb_rows(sb, 32, sb.size // 32)
+    deq = orc.dequant_rows(proj, 32, K, g, b)
+    sbr = F.sb_rows(proj, 32, K, g, b)
     s = ((sbr & 0xFFFF).astype(np.uint32) << 16).view(np.float32)
     bias = ((sbr >> 16).astype(np.uint32) << 16).view(np.float32)
     # scale = bf16 of (max-min)/(2^b-1); bias = bf16 of the group minimum
@@ -86,9 +90,9 @@ def test_quantizer_properties(orc, b, g):
 
 def test_padded_groups_are_zero(orc):
     w = (np.random.default_rng(1).standard_normal((16, 32)) * 0.02).astype(np.float32)
-    q, sb = orc.quantize_rows(w, 32, 4)
-    assert q.shape == (16, 64) and sb.shape == (16, 4)
-    sbr = F.sb_rows(sb, 16, 4)
+    proj = orc.quantize_rows(w, 32, 4)
+    assert proj.shape == (1, 16 * 64 + 16 * 4 * 4)
+    sbr = F.sb_rows(proj, 16, 32, 32, 4)
     assert np.all(sbr[:, 1:] == 0) and np.all(sbr[:, 0] != 0)
 
 
@@ -97,9 +101,9 @@ def test_dequant_is_single_rounding_fma(orc, b):
     r = np.random.default_rng(b)
     K, g = 512, 64
     w = (r.standard_normal((16, K)) * 0.05).astype(np.float32)
-    q, sb = orc.quantize_rows(w, g, b)
-    assert np.array_equal(orc.dequant_rows(q, sb, K, g, b).view(np.uint32),
-                          F.dequant_rows(q, sb, K, g, b).view(np.uint32))
+    proj = orc.quantize_rows(w, g, b)
+    assert np.array_equal(orc.dequant_rows(proj, 16, K, g, b).view(np.uint32),
+                          F.dequant_rows(proj, 16, K, g, b).view(np.uint32))
 
 
 def test_slot_sections_roundtrip(orc):
@@ -111,13 +115,11 @@ def test_slot_sections_roundtrip(orc):
     off, n = orc.slot_layout(H, I, g, 4, 6)
     assert slot.size == n
     gu, dn = orc.dequant_slot(slot, H, I, g, 4, 6)
-    q = slot[off[0]: off[0] + 2 * I * orc.row_bytes(H, 4)].reshape(2 * I, -1)
-    sb = slot[off[2]: off[2] + 2 * I * orc.row_groups(H, g) * 4].view(np.uint32).reshape(2 * I, -1)
-    stored = F.dequant_rows(q, sb, H, g, 4)
+    pg = slot[off[0]: off[0] + 2 * I // 16 * off[2]]
+    stored = F.dequant_rows(pg, 2 * I, H, g, 4)
     logical = stored[[F.gate_up_storage_row(R, I) for R in range(2 * I)]]
     assert np.array_equal(gu, logical)
     # gate rows first, then up rows: the quantised gate block reproduces w_gu[:I]
     assert np.max(np.abs(gu - w_gu)) < 0.02
-    qd = slot[off[1]: off[1] + H * orc.row_bytes(I, 6)].reshape(H, -1)
-    sd = slot[off[3]: off[3] + H * orc.row_groups(I, g) * 4].view(np.uint32).reshape(H, -1)
-    assert np.array_equal(dn, F.dequant_rows(qd, sd, I, g, 6))
+    pd = slot[off[1]: off[1] + H // 16 * off[3]]
+    assert np.array_equal(dn, F.dequant_rows(pd, H, I, g, 6))

@@ -27,12 +27,12 @@ def test_noalloc_matches_workspace_entry_point():
     for e in range(E):
         w_gu, w_d = synth.expert_weights_torch(3, e, H, I, "cuda")
         base = pool[e].data_ptr()
-        ops.moe_quantize_rows(w_gu, 2 * I, H, g, b, base + lay.q_gate_up, base + lay.sb_gate_up, gate_up_I=I)
-        ops.moe_quantize_rows(w_d, H, I, g, b, base + lay.q_down, base + lay.sb_down)
+        ops.moe_quantize_rows(w_gu, 2 * I, H, g, b, base + lay.gate_up, gate_up_I=I)
+        ops.moe_quantize_rows(w_d, H, I, g, b, base + lay.down)
     table = torch.arange(E, dtype=torch.int32, device="cuda")
     ws_b = ops.moe_workspace_bytes(d, T)
     assert ws_b <= ops.moe_noalloc_scratch_bytes()
-    ws = torch.empty(ws_b, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(ws_b, dtype=torch.uint8, device="cuda")
     for call in range(2):
         x = dev(synth.activations(10 + call, 0, T, H).view(np.int16))
         ids_np, w_np = synth.random_routing(20 + call, T, E, k)
