@@ -284,8 +284,19 @@ static cudaError_t launch_fused_t(const FfnArgs& a, int grid, size_t smem, cudaS
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
   void* argv[] = {const_cast<void*>(static_cast<const void*>(&a))};
+  // co-residency of every CTA is required (grid barrier): always cooperative;
+  // early launch behind the previous kernel as well where the driver accepts
+  // the combination (remembered after the first refusal)
+  static int pdl_refused = 0;
+  if (!__atomic_load_n(&pdl_refused, __ATOMIC_RELAXED)) {
+    cfg.numAttrs = 2;
+    const cudaError_t e = cudaLaunchKernelExC(&cfg, kern, argv);
+    if (e != cudaErrorInvalidValue && e != cudaErrorNotSupported) return e;
+    (void)cudaGetLastError();  // a refused launch configuration is not sticky
+    __atomic_store_n(&pdl_refused, 1, __ATOMIC_RELAXED);
+  }
+  cfg.numAttrs = 1;
   return cudaLaunchKernelExC(&cfg, kern, argv);
 }
 
