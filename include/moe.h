@@ -133,8 +133,10 @@ moe_status moe_slot_layout(const moe_layer_desc* d, moe_slot_layout_t* out);
  * max_tokens tokens (0 if d is invalid).  One buffer of this size may be
  * shared by the two calls when they run in stream order.  Its first 256
  * bytes are a control block (the grid barrier of the single-launch decode
- * FFN): zero them once after allocating the workspace (e.g. cudaMemset);
- * every call leaves them zero again.  The rest needs no initialisation. */
+ * FFN, an arrival counter that every launch advances by its grid size): zero
+ * them once after allocating the workspace (e.g. cudaMemset), and again after
+ * a call that reported MOE_DEV_ERR_TIMEOUT.  The rest needs no
+ * initialisation. */
 size_t moe_workspace_bytes(const moe_layer_desc* d, int32_t max_tokens);
 
 /* Stage 1.  Cache-aware top-k (BigMoeOnEdge note: every expert already in

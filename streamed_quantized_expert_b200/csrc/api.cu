@@ -46,18 +46,20 @@ int device_sms() {
 }
 
 // Workspace: [control block (kWsControlBytes)][sort scratch | FFN scratch].
-// The control block must be zero before the first call with a workspace and
-// is left zero by every call; the sort and FFN scratch overlap (different
-// calls, stream-ordered).
+// The control block must be zero before the first call with a workspace
+// (every fused launch then advances its arrival counter by its grid size);
+// the sort and FFN scratch overlap (different calls, stream-ordered).
 struct WsCarve {
-  size_t sort, h, o, total;
+  size_t sort, hb, h, o, total;
 };
 
 WsCarve carve(const moe_layer_desc& d, int T) {
   WsCarve c{};
   const int64_t np = (int64_t)T * d.k;
   c.sort = (size_t)round_up((int64_t)sort_ws_bytes((int)np, d.E), 256);
-  c.h = (size_t)round_up(np * d.I * 2, 256);
+  // h (bf16, rows padded to 128-blocks) and its per-8-column partial sums
+  c.hb = (size_t)round_up(np * padded_k(d.I) * 2, 256);
+  c.h = c.hb + (size_t)round_up(np * padded_k(d.I), 256);
   c.o = T > kFusedMaxTokens ? (size_t)round_up(np * d.H * 4, 256) : 0;
   const size_t ffn = c.h + c.o;
   c.total = kWsControlBytes + (c.sort > ffn ? c.sort : ffn);
@@ -201,6 +203,7 @@ __attribute__((visibility("hidden"))) moe_status moe_internal_expert_ffn(
   a.y = y_accum;
   a.ctl = static_cast<unsigned*>(ws);
   a.h = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + kWsControlBytes);
+  a.hpart = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsControlBytes + c.hb);
   a.o = c.o ? reinterpret_cast<float*>(static_cast<char*>(ws) + kWsControlBytes + c.h) : nullptr;
   a.dev_err = dev_err;
   a.y_overwrite = overwrite ? 1 : 0;

@@ -69,14 +69,17 @@ __device__ __forceinline__ void load_b_block(const uint16_t* row, int kb, int K,
   float sx[8 / GS], so[8 / GS];
 #pragma unroll
   for (int G = 0; G < 8 / GS; ++G) sx[G] = so[G] = 0.0f;
+  // all sixteen loads first, so that they are in flight together
+  uint32_t vv[8][2];
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     const int klo = kb * 128 + 16 * s + 2 * t4, khi = klo + 8;
-    uint32_t v0 = 0u, v1 = 0u;
-    if (row) {
-      if (klo < K) v0 = ld_pair(row + klo);
-      if (khi < K) v1 = ld_pair(row + khi);
-    }
+    vv[s][0] = (row != nullptr && klo < K) ? ld_pair(row + klo) : 0u;
+    vv[s][1] = (row != nullptr && khi < K) ? ld_pair(row + khi) : 0u;
+  }
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    uint32_t v0 = vv[s][0], v1 = vv[s][1];
     const float x0 = bf16_lo(v0) + bf16_hi(v0), x1 = bf16_lo(v1) + bf16_hi(v1);
     if (PairShift<B>::a(2 * s) == 3) v0 = bf2_scale_eighth(v0);
     if (PairShift<B>::a(2 * s + 1) == 3) v1 = bf2_scale_eighth(v1);
@@ -201,9 +204,14 @@ inline cudaError_t ensure_smem_attr(const void* kern, int (&done_mask)[4]) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   if (dev < 128 && ((__atomic_load_n(&done_mask[dev >> 5], __ATOMIC_RELAXED) >> (dev & 31)) & 1)) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-  // the whole carve-out as shared memory, so the gate/up and down kernels of
-  // one layer fit on an SM together
+  // dynamic limit = the device's per-block opt-in maximum minus the kernel's static shared memory
+  int optin = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  cudaFuncAttributes fa;
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, kern);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes);
+  // the whole carve-out as shared memory
   if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e == cudaSuccess && dev < 128) __atomic_fetch_or(&done_mask[dev >> 5], 1 << (dev & 31), __ATOMIC_RELAXED);
   return e;

@@ -419,13 +419,6 @@ __global__ void combine_kernel(const FfnArgs a) {
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-size_t ffn_ws_bytes(const moe_layer_desc& d, int T) {
-  const int64_t np = (int64_t)T * d.k;
-  size_t b = (size_t)round_up(np * d.I * 2, 256);  // h (bf16)
-  if (T > kFusedMaxTokens) b += (size_t)round_up(np * d.H * 4, 256);  // o (fp32)
-  return b;
-}
-
 template <int B, int BPW, int GS>
 static cudaError_t launch_gu(const FfnArgs& a, int grid, size_t smem, cudaStream_t st) {
   static int done[4] = {0, 0, 0, 0};

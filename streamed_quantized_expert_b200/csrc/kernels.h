@@ -28,7 +28,9 @@ struct FfnArgs {
   const uint16_t* x_sorted;
   int pass_begin, pass_len;
   float* y;
-  uint16_t* h;  // workspace: [T*k][I] bf16, by sorted position
+  uint16_t* h;    // workspace: [T*k][I] bf16 by sorted position (two-kernel path); the fused kernel
+                  // uses [T*k][padded I] by flat pair, scaled by 2^-a of the down pair slot
+  float* hpart;   // workspace (fused kernel): [T*k][padded I / 8] (sum h, sum 128 h 2^-a) pairs
   float* o;     // workspace: [T*k][H] fp32, by flat pair index (T > kFusedMaxTokens)
   int32_t* dev_err;
   unsigned* ctl;    // workspace control block (grid barrier of the fused kernel); zero between calls
@@ -38,6 +40,7 @@ struct FfnArgs {
   int64_t q_gu, q_d, tile_gu, tile_d, rb_gu, rb_d;
   int ng_gu, ng_d, nblk_gu, nblk_d;
   int gu_stage_bytes, d_stage_bytes, gu_nstage, d_nstage;
+  int xh_stage_bytes;  // fused kernel: shared region for x (gate/up phase), then h (down phase)
 };
 
 // Launch with programmatic stream serialization, so the kernel's CTAs can be
@@ -73,7 +76,6 @@ cudaError_t launch_exp(const float* x, int64_t n, float* out, cudaStream_t st);
 cudaError_t launch_quantize(const float* w, int rows, int K, int g, int b, int gu_I, uint8_t* q, cudaStream_t st);
 cudaError_t launch_dequant_slot(const uint8_t* slot, const moe_layer_desc& d, const Layout& L, float* out32,
                                 uint16_t* out16, cudaStream_t st);
-size_t ffn_ws_bytes(const moe_layer_desc& d, int T);
 bool ffn_decode_supported(const moe_layer_desc& d);
 cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st);
 cudaError_t launch_ffn_fused(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st);
