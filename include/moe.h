@@ -266,6 +266,19 @@ moe_status moe_exp_portable(const float* x, int64_t n, float* out, cudaStream_t 
 
 const char* moe_status_string(moe_status s);
 
+/* Which kernels moe_expert_ffn runs on the current device for a call over
+ * all E experts of a layer of shape d with T tokens, with (has_x_sorted != 0)
+ * or without x_sorted:
+ *   MOE_PATH_FUSED_DECODE  one launch: gate/up + SwiGLU, grid barrier, down +
+ *                          combine (T <= 8, T*k <= 64, H/16 <= SM count)
+ *   MOE_PATH_GEMV          gate/up + SwiGLU kernel, down kernel (+ combine
+ *                          kernel for T > 64): tensor-core GEMV (mma.sync)
+ *   MOE_PATH_TC_PREFILL    tcgen05/TMEM grouped GEMM fed by TMA (T >= 256,
+ *                          x_sorted given, H and I multiples of 128)
+ * or -1 if d is invalid or T < 1.  Host only; no device work. */
+enum { MOE_PATH_FUSED_DECODE = 0, MOE_PATH_GEMV = 1, MOE_PATH_TC_PREFILL = 2 };
+int32_t moe_ffn_kernel_path(const moe_layer_desc* d, int32_t T, int32_t has_x_sorted);
+
 /* Name of the last CUDA error that made a call of this thread return
  * MOE_ERR_CUDA ("no error" if none). */
 const char* moe_last_cuda_error(void);

@@ -13,7 +13,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 SO = os.path.join(HERE, "libmoe.so")
-SOURCES = ["api.cu", "route_sort.cu", "quant.cu", "ffn_decode.cu", "ffn_fused.cu", "noalloc.cu", "slot_cache.cpp", "driver.cpp"]
+SOURCES = ["api.cu", "route_sort.cu", "quant.cu", "ffn_decode.cu", "ffn_fused.cu", "prefill_tc.cu", "noalloc.cu", "slot_cache.cpp", "driver.cpp"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

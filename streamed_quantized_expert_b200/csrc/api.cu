@@ -72,6 +72,11 @@ extern "C" {
 
 const char* moe_last_cuda_error(void) { return g_last_cuda_error; }
 
+int32_t moe_ffn_kernel_path(const moe_layer_desc* d, int32_t T, int32_t has_x_sorted) {
+  if (check_desc(d) != MOE_OK || T < 1 || !ffn_decode_supported(*d)) return -1;
+  return ffn_kernel_path(*d, T, has_x_sorted != 0, device_sms());
+}
+
 const char* moe_status_string(moe_status s) {
   switch (s) {
     case MOE_OK: return "ok";

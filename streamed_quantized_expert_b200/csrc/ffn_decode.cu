@@ -479,6 +479,22 @@ bool ffn_decode_supported(const moe_layer_desc& d) {
 constexpr size_t kGuSmemCap = 150 * 1024;
 constexpr size_t kDnSmemCap = 72 * 1024;
 
+// 0: fused single-launch decode; 1: gate/up + down GEMV kernels (mma.sync);
+// 2: tcgen05 grouped GEMM (prefill) -- the choice launch_ffn_decode makes
+// for a call covering every expert of the layer.
+int ffn_kernel_path(const moe_layer_desc& d, int T, bool has_x_sorted, int num_sms) {
+  FfnArgs a{};
+  a.T = T;
+  a.pass_len = d.E;
+  a.L = make_layout(d);
+  unsigned ctl_stub = 0;
+  a.ctl = &ctl_stub;  // the plan only checks that a control block exists
+  size_t smem = 0;
+  if (ffn_fused_plan(a, d, num_sms, smem)) return 0;
+  if (T >= kPrefillTcMinTokens && has_x_sorted && ffn_prefill_tc_shape_ok(d)) return 2;
+  return 1;
+}
+
 cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st) {
   const Layout& L = a.L;
   {
@@ -506,6 +522,10 @@ cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, c
   a.ng_d = L.ng_d;
   a.nblk_gu = L.nblk_gu;
   a.nblk_d = L.nblk_d;
+  if (a.T >= kPrefillTcMinTokens) {  // tensor-core grouped GEMM (needs x_sorted)
+    const cudaError_t e = launch_ffn_prefill_tc(a, d, num_sms, st);
+    if (e != cudaErrorNotSupported) return e;
+  }
   a.gu_stage_bytes = (int)round_up(L.tile_gu, 128);
   a.d_stage_bytes = (int)round_up(L.tile_d, 128);
   const int gs = d.group / 16;

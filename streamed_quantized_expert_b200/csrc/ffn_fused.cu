@@ -508,13 +508,12 @@ static cudaError_t fused_bd(const FfnArgs& a, int bd, int bpw, int gs, int grid,
 
 // Returns cudaErrorNotSupported when the fused path does not apply (the
 // caller then uses the two-kernel path).
-cudaError_t launch_ffn_fused(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st) {
-  if (!(a.T <= kDenseMaxTokens && a.T * d.k <= kMaxCtaExperts) || a.ctl == nullptr) return cudaErrorNotSupported;
-  const int nblk = a.L.nblk_gu;
-  if (nblk > 2 * kFuConsumers) return cudaErrorNotSupported;
-  const int bpw = nblk <= kFuConsumers ? 1 : 2;
-  const int n_rt = d.H / 16;
-  if (n_rt > num_sms) return cudaErrorNotSupported;
+// Stage sizes and counts of the fused kernel for this call (into a), its
+// shared memory; false when the fused path does not apply.
+bool ffn_fused_plan(FfnArgs& a, const moe_layer_desc& d, int num_sms, size_t& smem) {
+  if (!(a.T <= kDenseMaxTokens && a.T * d.k <= kMaxCtaExperts) || a.ctl == nullptr) return false;
+  if (a.L.nblk_gu > 2 * kFuConsumers) return false;
+  if (d.H / 16 > num_sms) return false;
   const int grid = num_sms;
   int max_pass = a.pass_len < d.E ? a.pass_len : d.E;
   if (a.T * d.k < max_pass) max_pass = a.T * d.k;
@@ -532,7 +531,7 @@ cudaError_t launch_ffn_fused(FfnArgs a, const moe_layer_desc& d, int num_sms, cu
                        (size_t)kFuConsumers * 32 * 4 * 4 + kRedBatch * sizeof(RedMeta) +
                        kFuTableBytes;
   const size_t cap = 220 * 1024;
-  if (fixed + a.gu_stage_bytes + a.d_stage_bytes + 64 > cap) return cudaErrorNotSupported;
+  if (fixed + a.gu_stage_bytes + a.d_stage_bytes + 64 > cap) return false;
   // down stages: every expert of the pass if possible, else half the room
   int nsd = max_pass;
   int nsg = (int)(items_per_cta < 1 ? 1 : items_per_cta);
@@ -540,11 +539,19 @@ cudaError_t launch_ffn_fused(FfnArgs a, const moe_layer_desc& d, int num_sms, cu
     if (nsg > nsd && nsg > 2) --nsg;
     else if (nsd > 2) --nsd;
     else if (nsg > 1) --nsg;
-    else return cudaErrorNotSupported;
+    else return false;
   }
   a.gu_nstage = nsg;
   a.d_nstage = nsd;
-  const size_t smem = (size_t)nsg * a.gu_stage_bytes + (size_t)nsd * a.d_stage_bytes + fixed + 16 * (nsd + nsg);
+  smem = (size_t)nsg * a.gu_stage_bytes + (size_t)nsd * a.d_stage_bytes + fixed + 16 * (nsd + nsg);
+  return true;
+}
+
+cudaError_t launch_ffn_fused(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st) {
+  size_t smem = 0;
+  if (!ffn_fused_plan(a, d, num_sms, smem)) return cudaErrorNotSupported;
+  const int grid = num_sms;
+  const int bpw = a.L.nblk_gu <= kFuConsumers ? 1 : 2;
   const int gs = d.group / 16;
   if (d.bits_gu == 3) return fused_bd<3>(a, d.bits_down, bpw, gs, grid, smem, st);
   if (d.bits_gu == 4) return fused_bd<4>(a, d.bits_down, bpw, gs, grid, smem, st);

@@ -10,6 +10,7 @@
 namespace moe {
 
 constexpr int kFusedMaxTokens = 64;  // decode down kernel combines in shared memory up to this T
+constexpr int kPrefillTcMinTokens = 256;  // from this T on, prefill runs on the tcgen05 grouped GEMM
 
 struct FfnArgs {
   const uint16_t* x;
@@ -79,6 +80,11 @@ cudaError_t launch_dequant_slot(const uint8_t* slot, const moe_layer_desc& d, co
 bool ffn_decode_supported(const moe_layer_desc& d);
 cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st);
 cudaError_t launch_ffn_fused(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st);
+cudaError_t launch_ffn_prefill_tc(const FfnArgs& a, const moe_layer_desc& d, int num_sms, cudaStream_t st);
+bool ffn_fused_plan(FfnArgs& a, const moe_layer_desc& d, int num_sms, size_t& smem);
+bool ffn_prefill_tc_shape_ok(const moe_layer_desc& d);
+int ffn_kernel_path(const moe_layer_desc& d, int T, bool has_x_sorted, int num_sms);
+__global__ void combine_kernel(const FfnArgs a);
 constexpr size_t kWsControlBytes = 256;  // head of the workspace: grid-barrier words
 
 }  // namespace moe

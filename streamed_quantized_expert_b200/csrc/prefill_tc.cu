@@ -1,0 +1,635 @@
+// Prefill expert FFN on the 5th-generation tensor cores (tcgen05 + TMEM),
+// fed by TMA: the grouped GEMM of a pass's experts over their sorted tokens.
+//
+// Two launches per pass, one persistent CTA per SM, each looping over tiles
+// of (expert, 128 weight rows, up to 128 tokens):
+//   gate/up: GU[rows, tokens] = deq(W_gu[e])[rows, H] . X_sorted[tokens, H]^T,
+//            then h[token][j] = silu(gate_j) * up_j (bf16), j = intermediate;
+//   down:    O[rows, tokens]  = deq(W_d[e])[rows, I] . h[tokens, I]^T,
+//            o[pair][row] = O (fp32), summed per token by the combine kernel.
+// The weight rows are the MMA's M side (the "swap AB" arrangement for grouped
+// expert GEMMs: a token count per expert of tens to hundreds fits N, which
+// steps by 16, where it would leave most of a 128-row M tile empty).
+//
+// Warp roles (320 threads):
+//   0-3  dequant: thread = weight row; unpack the packed codes of a 128-input
+//        block (landed by TMA), w = fma(scale, q, bias) in bf16x2 with one
+//        rounding, stored as the MMA's A operand in the 128-byte swizzled
+//        K-major layout;
+//   4-7  epilogue: TMEM -> registers (warp i reads TMEM lanes 32 (i % 4)..);
+//   8    producer: TMA loads of codes, (scale, bias) words and token rows;
+//   9    MMA issuer (one thread): tcgen05.mma kind::f16 (bf16 x bf16 -> fp32
+//        in TMEM), M = 128, N = tokens rounded up to 16, K = 16 per
+//        instruction; tcgen05.commit frees stages and publishes accumulators.
+// Accumulators are double-buffered in TMEM (2 x 128 columns), so the epilogue
+// of one tile overlaps the MMAs of the next.
+//
+// Every wait is bounded; a wait that runs out sets a CTA-wide abort flag and
+// MOE_DEV_ERR_TIMEOUT, the roles leave their loops, the producer waits for
+// the copies it issued, the MMA thread waits for its MMAs, and TMEM is freed.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "ffn_common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int kPfBM = 128;      // weight rows per tile (MMA M)
+constexpr int kPfBN = 128;      // tokens per tile (MMA N, at most)
+constexpr int kPfStages = 3;    // load stages (codes + scale/bias + token rows)
+constexpr int kPfABufs = 2;     // dequantised A buffers
+constexpr int kPfThreads = 320;
+constexpr int kPfTmemCols = 256;  // two accumulators of kPfBN fp32 columns
+constexpr int kPfXHalf = kPfBN * 128;   // one 64-input half of a token stage: 128 rows x 128 B
+constexpr int kPfAHalf = kPfBM * 128;   // one 64-input half of an A buffer
+
+struct PfEntry {
+  int slot;    // slot of the expert (tiles skipped when not resident)
+  int pos0;    // first sorted position of its tokens
+  int cnt;     // tokens
+  int tile0;   // first tile of the entry in the CTA-wide tile order
+};
+
+struct PfArgs {
+  int T, k, H, I, g, E;
+  int K;            // reduction length: H (gate/up) or I (down)
+  int nkb;          // 128-input blocks of K
+  int mtiles;       // 128-row tiles of the weight rows: 2I/128 or H/128
+  int n_slots;
+  const int32_t* table;
+  const int32_t* active;
+  const int32_t* n_active;
+  const int32_t* offsets;
+  const int32_t* pairs;
+  int pass_begin, pass_len;
+  uint16_t* h;      // [T*k][I] bf16 by sorted position (gate/up writes, down reads through its map)
+  float* o;         // [T*k][H] fp32 by flat pair (down writes)
+  int32_t* dev_err;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_addr(dst)),
+      "l"(tm), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* tm, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::
+          "r"(smem_addr(dst)),
+      "l"(tm), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* tm, int x, int y, int z, int w,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+      "[%6];" ::"r"(smem_addr(dst)),
+      "l"(tm), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tmap_prefetch(const CUtensorMap* tm) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(tm) : "memory");
+}
+
+// Shared-memory matrix descriptor of a 128-byte swizzled K-major operand
+// whose 8-row groups are 1024 bytes apart (rows of 64 bf16): start address
+// >> 4 in bits 0-13, leading byte offset 16 B (unused by swizzled K-major) in
+// bits 16-29, stride byte offset 1024 B in bits 32-45, descriptor version 1
+// in bits 46-47, swizzle mode 2 (128 B) in bits 61-63.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+         ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator (bits 4-5 = 1), A and
+// B bf16 (bits 7-9 = 1, bits 10-12 = 1), both K-major (bits 15, 16 = 0),
+// N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+__device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` once every tcgen05 operation this thread issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void proxy_fence_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// 32 TMEM lanes x 16 consecutive 32-bit columns: thread i of the warp gets
+// lane (base lane + i), columns col..col+15.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ bool slot_ok_pf(int n_slots, int slot) { return slot >= 0 && slot < n_slots; }
+
+// Bounded wait that also gives up once another role of the CTA has aborted.
+__device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_test(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_try_wait(bar, parity, 20000u)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > 4000000000ll) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// One 128-input block of weight row r (0..127 of the tile) -> bf16 A operand.
+// Codes: the tile's 16 8-row groups, each 4 units x 8 rows x B words (unit t
+// of row rr at word (8 t + sigma) B); scale/bias: per 16-row tile, GPB groups
+// of 16 words.  Input k = 16 s + 2 t + 8 h' (+1) of the block is pair 2 s + h'
+// of unit t, so the 16-byte chunk c = 2 (s % 4) + h' of 64-input half s / 4
+// holds pair (2 s + h') of units 0..3 in that order.
+template <int B, int GPB>
+__device__ __forceinline__ void pf_dequant_block(const uint32_t* cs, const uint32_t* sbs, uint8_t* abuf, int r) {
+  const int g8 = r >> 3, rr = r & 7;
+  uint32_t p[4][16];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    uint32_t w[B];
+    const uint32_t* up = cs + g8 * 32 * B + (8 * t + unit_sigma<B>(t, rr)) * B;
+#pragma unroll
+    for (int i = 0; i < B; ++i) w[i] = up[i];
+    unpack_unit<B>(w, p[t]);
+  }
+  __nv_bfloat162 sc[GPB], sc8[GPB], bi[GPB];
+#pragma unroll
+  for (int gi = 0; gi < GPB; ++gi) {
+    const uint32_t word = sbs[(r >> 4) * 16 * GPB + gi * 16 + (r & 15)];
+    const uint32_t s2 = (word & 0xFFFFu) * 0x10001u, b2 = (word >> 16) * 0x10001u;
+    sc[gi] = *reinterpret_cast<const __nv_bfloat162*>(&s2);
+    bi[gi] = *reinterpret_cast<const __nv_bfloat162*>(&b2);
+    sc8[gi] = __hmul2(sc[gi], __floats2bfloat162_rn(0.125f, 0.125f));
+  }
+  const uint32_t m = kMagic;
+  const __nv_bfloat162 m128 = *reinterpret_cast<const __nv_bfloat162*>(&m);
+  uint8_t* rowbase = abuf + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int s = i >> 1, hp = i & 1, hf = s >> 2, c = 2 * (s & 3) + hp;
+    const int gi = (s * GPB) >> 3;
+    const __nv_bfloat162 scale = PairShift<B>::a(i) == 3 ? sc8[gi] : sc[gi];
+    uint32_t o[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const __nv_bfloat162 q = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&p[t][i]), m128);
+      const __nv_bfloat162 v = __hfma2(scale, q, bi[gi]);
+      o[t] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    *reinterpret_cast<uint4*>(rowbase + hf * kPfAHalf + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+struct PfTile {
+  int ent, mt, nt, n;  // entry, 128-row tile, token tile, tokens in the tile
+  int slot, row0;      // slot; first sorted position of the tile's tokens
+};
+
+template <int B, int GPB, bool GU>
+__global__ void __launch_bounds__(kPfThreads, 1)
+    pf_gemm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_sb,
+                   const __grid_constant__ CUtensorMap tm_b, const PfArgs a) {
+  extern __shared__ uint8_t pf_smem_raw[];
+  constexpr int kCodesBytes = 2048 * B;   // 16 groups x 4 units x 8 rows x B words
+  constexpr int kSbBytes = 512 * GPB;     // 8 tiles x 16 GPB words
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* xst = base;                                           // [stage][2 halves][128 rows][128 B]
+  uint8_t* abuf = xst + kPfStages * 2 * kPfXHalf;                // [buf][2 halves][128 rows][128 B]
+  uint8_t* cst = abuf + kPfABufs * 2 * kPfAHalf;                 // [stage] codes
+  uint8_t* sbst = cst + kPfStages * kCodesBytes;                 // [stage] scale/bias words
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sbst + kPfStages * kSbBytes);
+  uint64_t* full = bars;                        // producer (expect_tx) -> dequant, MMA
+  uint64_t* empty = full + kPfStages;           // MMA commit -> producer
+  uint64_t* afull = empty + kPfStages;          // dequant threads (128) -> MMA
+  uint64_t* aempty = afull + kPfABufs;          // MMA commit -> dequant
+  uint64_t* accfull = aempty + kPfABufs;        // MMA commit -> epilogue
+  uint64_t* accempty = accfull + 2;             // epilogue threads (128) -> MMA
+  uint64_t* drain = accempty + 2;               // MMA commit at exit
+  __shared__ PfEntry s_ent[kMaxCtaExperts];
+  __shared__ int s_nent, s_ntiles;
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+
+  if (tid == 0) {
+    for (int s = 0; s < kPfStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < kPfABufs; ++b) {
+      mbar_init(&afull[b], 128);
+      mbar_init(&aempty[b], 1);
+    }
+    for (int c = 0; c < 2; ++c) {
+      mbar_init(&accfull[c], 1);
+      mbar_init(&accempty[c], 128);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+    s_abort = 0;
+  }
+  if (warp == 9) {  // TMEM: two accumulators of kPfBN columns
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
+                 "r"(kPfTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (warp == 8 && lane == 0) {
+    tmap_prefetch(&tm_q);
+    tmap_prefetch(&tm_sb);
+    tmap_prefetch(&tm_b);
+  }
+  pdl_wait();
+  // the pass's experts and their tiles (token tiles x row tiles, row tile fastest)
+  if (warp == 0) {
+    int n = *a.n_active - a.pass_begin;
+    if (n > a.pass_len) n = a.pass_len;
+    if (n > kMaxCtaExperts) n = kMaxCtaExperts;
+    if (n < 0) n = 0;
+    for (int i = lane; i < n; i += 32) {
+      const int e = a.active[a.pass_begin + i];
+      PfEntry en;
+      en.slot = (e >= 0 && e < a.E) ? a.table[e] : -1;
+      en.pos0 = (e >= 0 && e < a.E) ? a.offsets[e] : 0;
+      en.cnt = (e >= 0 && e < a.E) ? a.offsets[e + 1] - en.pos0 : 0;
+      en.tile0 = 0;
+      s_ent[i] = en;
+      if (blockIdx.x == 0 && !slot_ok_pf(a.n_slots, en.slot) && a.dev_err)
+        atomicOr(a.dev_err, en.slot < 0 ? MOE_DEV_ERR_NOT_RESIDENT : MOE_DEV_ERR_SLOT_RANGE);
+    }
+    __syncwarp();
+    if (lane == 0) {
+      int acc = 0;
+      for (int i = 0; i < n; ++i) {
+        s_ent[i].tile0 = acc;
+        if (slot_ok_pf(a.n_slots, s_ent[i].slot)) acc += ((s_ent[i].cnt + kPfBN - 1) / kPfBN) * a.mtiles;
+      }
+      s_nent = n;
+      s_ntiles = acc;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = s_tmem;
+  const int nent = s_nent, ntiles = s_ntiles;
+  auto tile_at = [&](int t) -> PfTile {
+    int i = 0;
+    while (i + 1 < nent && s_ent[i + 1].tile0 <= t) ++i;
+    const PfEntry en = s_ent[i];
+    const int local = t - en.tile0;
+    PfTile tl;
+    tl.ent = i;
+    tl.nt = local / a.mtiles;
+    tl.mt = local - tl.nt * a.mtiles;
+    tl.n = en.cnt - tl.nt * kPfBN < kPfBN ? en.cnt - tl.nt * kPfBN : kPfBN;
+    tl.slot = en.slot;
+    tl.row0 = en.pos0 + tl.nt * kPfBN;
+    return tl;
+  };
+
+  if (warp == 8) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, issued = 0, last_ph = 0;  // per-stage bit masks for the exit drain
+      for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
+        const PfTile tl = tile_at(t);
+        const int nbox = (tl.n + 31) >> 5;
+        const uint32_t bytes = kCodesBytes + kSbBytes + (uint32_t)nbox * 2 * 32 * 128;
+        bool ok = true;
+        for (int kb = 0; kb < a.nkb; ++kb) {
+          if (!pf_wait(&empty[s], ph ^ 1u, &s_abort)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], bytes);
+          tma_load_4d(cst + s * kCodesBytes, &tm_q, kb * 32 * B, 0, tl.mt * 8, tl.slot, &full[s]);
+          tma_load_3d(sbst + s * kSbBytes, &tm_sb, kb * 16 * GPB, tl.mt * 8, tl.slot, &full[s]);
+          for (int j = 0; j < nbox; ++j)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_2d(xst + (s * 2 + hf) * kPfXHalf + j * 4096, &tm_b, kb * 128 + hf * 64, tl.row0 + 32 * j,
+                          &full[s]);
+          issued |= 1u << s;
+          last_ph = (last_ph & ~(1u << s)) | (ph << s);
+          if (++s == kPfStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      // every copy issued lands before the CTA can exit
+      for (int q = 0; q < kPfStages; ++q)
+        if ((issued >> q) & 1u) mbar_wait_bounded(&full[q], (last_ph >> q) & 1u);
+    }
+  } else if (warp == 9) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int s = 0, ab = 0, c = 0;
+      uint32_t ph = 0, pa = 0, pc = 0;
+      bool issued_any = false;
+      for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
+        const PfTile tl = tile_at(t);
+        const int npad = (tl.n + 15) & ~15;
+        const uint32_t idesc = idesc_bf16(kPfBM, npad);
+        if (!pf_wait(&accempty[c], pc ^ 1u, &s_abort)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(c * kPfBN);
+        bool ok = true;
+        for (int kb = 0; kb < a.nkb; ++kb) {
+          if (!pf_wait(&full[s], ph, &s_abort) || !pf_wait(&afull[ab], pa, &s_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t abase = smem_addr(abuf + ab * 2 * kPfAHalf), xbase = smem_addr(xst + s * 2 * kPfXHalf);
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16) {
+            const uint32_t off = (uint32_t)((k16 >> 2) * kPfAHalf + (k16 & 3) * 32);
+            umma_bf16(d, sw128_desc(abase + off), sw128_desc(xbase + off), idesc, (kb | k16) != 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          umma_commit(&empty[s]);
+          umma_commit(&aempty[ab]);
+          if (++s == kPfStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+          if (++ab == kPfABufs) {
+            ab = 0;
+            pa ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&accfull[c]);
+        if (++c == 2) {
+          c = 0;
+          pc ^= 1u;
+        }
+      }
+      if (issued_any) {  // every MMA issued completes before TMEM is freed
+        umma_commit(drain);
+        mbar_wait_bounded(drain, 0);
+      }
+    }
+  } else if (warp < 4) {
+    // ---------------- dequant ----------------
+    int s = 0, ab = 0;
+    uint32_t ph = 0, pa = 0;
+    for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
+      bool ok = true;
+      for (int kb = 0; kb < a.nkb; ++kb) {
+        if (!pf_wait(&full[s], ph, &s_abort) || !pf_wait(&aempty[ab], pa ^ 1u, &s_abort)) {
+          ok = false;
+          break;
+        }
+        pf_dequant_block<B, GPB>(reinterpret_cast<const uint32_t*>(cst + s * kCodesBytes),
+                                 reinterpret_cast<const uint32_t*>(sbst + s * kSbBytes), abuf + ab * 2 * kPfAHalf,
+                                 tid);
+        proxy_fence_smem();
+        mbar_arrive(&afull[ab]);
+        if (++s == kPfStages) {
+          s = 0;
+          ph ^= 1u;
+        }
+        if (++ab == kPfABufs) {
+          ab = 0;
+          pa ^= 1u;
+        }
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ---------------- epilogue (warps 4-7: TMEM lanes 32 (warp % 4) ..) ----------------
+    const int q = warp & 3, r = 32 * q + lane;
+    int c = 0;
+    uint32_t pc = 0;
+    for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
+      const PfTile tl = tile_at(t);
+      if (!pf_wait(&accfull[c], pc, &s_abort)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * kPfBN);
+      for (int n0 = 0; n0 < tl.n; n0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(taddr + (uint32_t)n0, v);
+        tmem_ld_wait();
+        if (GU) {
+          // storage rows: 16-row blocks of 8 gate rows then 8 up rows
+          const bool gate = (r & 15) < 8;
+          const int j = tl.mt * (kPfBM / 2) + (r >> 4) * 8 + (r & 7);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float x = __uint_as_float(v[i]);
+            const float u = __shfl_xor_sync(0xffffffffu, x, 8);
+            if (gate && n0 + i < tl.n)
+              a.h[(int64_t)(tl.row0 + n0 + i) * a.I + j] = f32_to_bf16_rne(x / (1.0f + expf(-x)) * u);
+          }
+        } else {
+          const int row = tl.mt * kPfBM + r;
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (n0 + i < tl.n) a.o[(int64_t)a.pairs[tl.row0 + n0 + i] * a.H + row] = __uint_as_float(v[i]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&accempty[c]);
+      if (++c == 2) {
+        c = 0;
+        pc ^= 1u;
+      }
+    }
+  }
+  pdl_launch_dependents();
+  if (s_abort && tid == 0 && a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kPfTmemCols)
+                 : "memory");
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* addr, const cuuint64_t* dims,
+            const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle sw) {
+  const auto fn = tmap_encoder();
+  if (!fn) return false;
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return fn(m, dt, (cuuint32_t)rank, const_cast<void*>(addr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Maps of one projection of the pool: codes as 32-bit words (8-row group
+// words, half, 16-row tile, slot) and the (scale, bias) words (tile words,
+// tile, slot); a box is one 128-input block of a 128-row tile.
+bool encode_proj(CUtensorMap* q, CUtensorMap* sb, const uint8_t* proj, int64_t rb, int64_t tile, int ng, int rows,
+                 int bits, int gpb, int64_t slot_bytes, int n_slots) {
+  const cuuint64_t qd[4] = {(cuuint64_t)(2 * rb), 2, (cuuint64_t)(rows / 16), (cuuint64_t)n_slots};
+  const cuuint64_t qs[3] = {(cuuint64_t)(8 * rb), (cuuint64_t)tile, (cuuint64_t)slot_bytes};
+  const cuuint32_t qb[4] = {(cuuint32_t)(32 * bits), 2, 8, 1};
+  if (!encode(q, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, proj, qd, qs, qb, CU_TENSOR_MAP_SWIZZLE_NONE)) return false;
+  const cuuint64_t sd[3] = {(cuuint64_t)(16 * ng), (cuuint64_t)(rows / 16), (cuuint64_t)n_slots};
+  const cuuint64_t ss[2] = {(cuuint64_t)tile, (cuuint64_t)slot_bytes};
+  const cuuint32_t sbx[3] = {(cuuint32_t)(16 * gpb), 8, 1};
+  return encode(sb, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, proj + 16 * rb, sd, ss, sbx, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// Token rows (bf16 [rows][cols], row-major) for the MMA's B operand: boxes of
+// 64 columns (128 bytes, 128-byte swizzle) x 32 rows.
+bool encode_rows(CUtensorMap* m, const uint16_t* base, int64_t rows, int cols) {
+  const cuuint64_t d[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t s[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t b[2] = {64, 32};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, d, s, b, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+size_t pf_smem_bytes(int bits, int gpb) {
+  return 1024 + (size_t)kPfStages * 2 * kPfXHalf + (size_t)kPfABufs * 2 * kPfAHalf + (size_t)kPfStages * 2048 * bits +
+         (size_t)kPfStages * 512 * gpb + 16 * 8;
+}
+
+template <int B, int GPB, bool GU>
+cudaError_t launch_pf_t(const CUtensorMap& q, const CUtensorMap& sb, const CUtensorMap& bm, const PfArgs& pa,
+                        int grid, cudaStream_t st) {
+  static int done[4] = {0, 0, 0, 0};
+  const void* kern = reinterpret_cast<const void*>(pf_gemm_kernel<B, GPB, GU>);
+  const size_t smem = pf_smem_bytes(B, GPB);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev >= 128) return cudaErrorNotSupported;
+  if (!((__atomic_load_n(&done[dev >> 5], __ATOMIC_RELAXED) >> (dev & 31)) & 1)) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    __atomic_fetch_or(&done[dev >> 5], 1 << (dev & 31), __ATOMIC_RELAXED);
+  }
+  return launch_pdl(kern, grid, kPfThreads, smem, st, q, sb, bm, pa);
+}
+
+template <int B, bool GU>
+cudaError_t launch_pf_gpb(int gpb, const CUtensorMap& q, const CUtensorMap& sb, const CUtensorMap& bm,
+                          const PfArgs& pa, int grid, cudaStream_t st) {
+  if (gpb == 1) return launch_pf_t<B, 1, GU>(q, sb, bm, pa, grid, st);
+  if (gpb == 2) return launch_pf_t<B, 2, GU>(q, sb, bm, pa, grid, st);
+  return launch_pf_t<B, 4, GU>(q, sb, bm, pa, grid, st);
+}
+
+template <bool GU>
+cudaError_t launch_pf(int bits, int gpb, const CUtensorMap& q, const CUtensorMap& sb, const CUtensorMap& bm,
+                      const PfArgs& pa, int grid, cudaStream_t st) {
+  if (bits == 3) return launch_pf_gpb<3, GU>(gpb, q, sb, bm, pa, grid, st);
+  if (bits == 4) return launch_pf_gpb<4, GU>(gpb, q, sb, bm, pa, grid, st);
+  return launch_pf_gpb<6, GU>(gpb, q, sb, bm, pa, grid, st);
+}
+
+}  // namespace
+
+bool ffn_prefill_tc_shape_ok(const moe_layer_desc& d) {
+  return d.H % 128 == 0 && d.I % 128 == 0 && (d.group == 32 || d.group == 64 || d.group == 128) &&
+         tmap_encoder() != nullptr;
+}
+
+static bool ffn_prefill_tc_supported(const FfnArgs& a, const moe_layer_desc& d) {
+  return a.x_sorted != nullptr && a.o != nullptr && a.n_slots > 0 && ffn_prefill_tc_shape_ok(d);
+}
+
+// gate/up + SwiGLU -> h, down -> o (per pair), combine -> y; returns
+// cudaErrorNotSupported when the shapes or inputs do not fit this path.
+cudaError_t launch_ffn_prefill_tc(const FfnArgs& a, const moe_layer_desc& d, int num_sms, cudaStream_t st) {
+  if (!ffn_prefill_tc_supported(a, d)) return cudaErrorNotSupported;
+  const Layout& L = a.L;
+  const int gpb = 128 / d.group;
+  const int64_t np = (int64_t)a.T * d.k;
+  CUtensorMap q_gu, sb_gu, q_d, sb_d, xm, hm;
+  if (!encode_proj(&q_gu, &sb_gu, a.pool + L.gu, L.rb_gu, L.tile_gu, L.ng_gu, 2 * d.I, d.bits_gu, gpb, L.slot_bytes,
+                   a.n_slots) ||
+      !encode_proj(&q_d, &sb_d, a.pool + L.d, L.rb_d, L.tile_d, L.ng_d, d.H, d.bits_down, gpb, L.slot_bytes,
+                   a.n_slots) ||
+      !encode_rows(&xm, a.x_sorted, np, d.H) || !encode_rows(&hm, a.h, np, d.I))
+    return cudaErrorInvalidValue;
+  PfArgs pa{};
+  pa.T = a.T;
+  pa.k = d.k;
+  pa.H = d.H;
+  pa.I = d.I;
+  pa.g = d.group;
+  pa.E = d.E;
+  pa.n_slots = a.n_slots;
+  pa.table = a.table;
+  pa.active = a.active;
+  pa.n_active = a.n_active;
+  pa.offsets = a.offsets;
+  pa.pairs = a.pairs;
+  pa.pass_begin = a.pass_begin;
+  pa.pass_len = a.pass_len;
+  pa.h = a.h;
+  pa.o = a.o;
+  pa.dev_err = a.dev_err;
+  const int grid = num_sms;
+  pa.K = d.H;
+  pa.nkb = L.nblk_gu;
+  pa.mtiles = 2 * d.I / kPfBM;
+  cudaError_t e = launch_pf<true>(d.bits_gu, gpb, q_gu, sb_gu, xm, pa, grid, st);
+  if (e != cudaSuccess) return e;
+  pa.K = d.I;
+  pa.nkb = L.nblk_d;
+  pa.mtiles = d.H / kPfBM;
+  e = launch_pf<false>(d.bits_down, gpb, q_d, sb_d, hm, pa, grid, st);
+  if (e != cudaSuccess) return e;
+  const int64_t total = (int64_t)a.T * d.H;
+  int cgrid = (int)((total + 255) / 256);
+  if (cgrid > num_sms * 8) cgrid = num_sms * 8;
+  return launch_pdl(reinterpret_cast<const void*>(combine_kernel), cgrid, 256, 0, st, a);
+}
+
+}  // namespace moe

@@ -24,7 +24,7 @@ ABI_SYMBOLS = [
     "moe_status_string", "moe_cache_create", "moe_cache_destroy", "moe_cache_table", "moe_cache_layer_base",
     "moe_cache_class_slots", "moe_cache_place", "moe_cache_step", "moe_cache_stats",
     "moe_expert_ffn_noalloc", "moe_noalloc_scratch_bytes", "moe_cache_resident", "moe_decode_layer",
-    "moe_last_cuda_error",
+    "moe_last_cuda_error", "moe_ffn_kernel_path",
 ]
 
 
@@ -88,6 +88,7 @@ def lib():
             "moe_exp_portable": (C.c_int, [P, i64, P, P]),
             "moe_status_string": (C.c_char_p, [C.c_int]),
             "moe_last_cuda_error": (C.c_char_p, []),
+            "moe_ffn_kernel_path": (i32, [D, i32, i32]),
             "moe_cache_create": (C.c_int, [i32, i32, P, i32, C.POINTER(P)]),
             "moe_cache_destroy": (None, [P]),
             "moe_cache_table": (C.POINTER(i32), [P, i32]),
@@ -106,6 +107,14 @@ def lib():
             fn.argtypes = args
         _lib = L
     return _lib
+
+
+MOE_PATH_FUSED_DECODE, MOE_PATH_GEMV, MOE_PATH_TC_PREFILL = 0, 1, 2
+
+
+def moe_ffn_kernel_path(d: LayerDesc, T: int, has_x_sorted: bool) -> int:
+    """Kernels moe_expert_ffn runs for this layer shape and token count."""
+    return int(lib().moe_ffn_kernel_path(C.byref(d), int(T), 1 if has_x_sorted else 0))
 
 
 def status_string(s: int) -> str:

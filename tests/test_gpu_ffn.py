@@ -41,7 +41,7 @@ class Setup:
         self.table = dev(self.perm)
         self.slots_np = [self.bank[self.row[e]] for e in range(E)]
 
-    def gpu(self, x, ids, w, T, passes=None, table=None):
+    def gpu(self, x, ids, w, T, passes=None, table=None, sorted_x=False):
         E, k = self.E, self.k
         ws_b = ops.moe_workspace_bytes(self.d, T)
         ws = torch.zeros(ws_b, dtype=torch.uint8, device="cuda")
@@ -50,12 +50,13 @@ class Setup:
         active = torch.empty(E, dtype=torch.int32, device="cuda")
         na = torch.zeros(1, dtype=torch.int32, device="cuda")
         ids_d, w_d, x_d = dev(ids), dev(w), dev(x.view(np.int16))
-        ops.moe_sort(ids_d, None, T, self.d, offsets, pairs, active, na, None, ws, ws_b)
+        xs = torch.empty((max(T * k, 1), self.H), dtype=torch.int16, device="cuda") if sorted_x else None
+        ops.moe_sort(ids_d, x_d if sorted_x else None, T, self.d, offsets, pairs, active, na, xs, ws, ws_b)
         y = torch.zeros((T, self.H), dtype=torch.float32, device="cuda")
         err = torch.zeros(1, dtype=torch.int32, device="cuda")
         tab = self.table if table is None else table
         for pb, pl in passes or [(0, E)]:
-            ops.moe_expert_ffn(x_d, T, self.d, self.pool, E, tab, ids_d, w_d, offsets, pairs, active, na, None,
+            ops.moe_expert_ffn(x_d, T, self.d, self.pool, E, tab, ids_d, w_d, offsets, pairs, active, na, xs,
                                pb, pl, y, ws, ws_b, err)
         torch.cuda.synchronize()
         return y.cpu().numpy(), int(err.item())
