@@ -50,6 +50,18 @@ CONFIGS = {
     "tiny": (1, 8, 2, 64, 32, 32, 4, 4, 4, 8, "tiny MoE layer: 8 experts, top-2, H 64, I 32, 4-bit g32, 4 tokens"),
 }
 
+# Prefill chunks: every expert of every layer resident (the metric is the expert
+# FFN's tensor-core rate; installs are PCIe-bound and reported by decode).
+# name: (layers, E, k, H, I, g, bits(layer) -> (gate/up, down), T, description)
+PREFILL = {
+    "prefill": (48, 512, 10, 2048, 512, 64, lambda l: (3, 3), 1024,
+                "Flash-Next-like prefill: 48 layers x 512 experts, top-10, H 2048, I 512, SwiGLU, 3-bit g64, "
+                "1024-token chunk, passes of 64 active experts, tcgen05 grouped GEMM"),
+    "prefill_mixed": (48, 512, 10, 2048, 512, 64, lambda l: (4, 6) if l % 4 == 0 else (4, 4), 4096,
+                      "mixed size classes prefill: Flash-Next-like shapes, 4-bit gate/up, 6-bit down on layers "
+                      "l % 4 == 0 (2 slot size classes), 4096-token chunk, passes of 64 active experts"),
+}
+
 
 # ---------------------------------------------------------------------------
 # clocks
@@ -183,6 +195,166 @@ def ffn_graph_time(st, cfg, snaps, reps, device):
     us = 1e3 * e0.elapsed_time(e1) / (reps * n_layers)
     del g_
     return us
+
+
+def run_prefill(args, rank, world, local_rank):
+    """Prefill chunk through every layer: route + sort (with sorted x), then
+    passes of 64 active experts on the tensor-core grouped GEMM.  `value` is
+    the expert FFN's TFLOP/s from a CUDA graph of every pass of every layer."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from streamed_quantized_expert_b200 import build as libbuild
+    from streamed_quantized_expert_b200 import ops, synth
+    from streamed_quantized_expert_b200.runtime import PASS_EXPERTS, LayerSpec, Streamer, quantize_bank_gpu
+
+    libbuild.build()
+    ops.lib()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    n_layers, E, k, H, I, g, bits, T, desc_txt = PREFILL[args.config]
+    if args.layers:
+        n_layers = args.layers
+        desc_txt += f" [layers overridden to {n_layers}]"
+    seed = 1000 * rank
+    descs = [ops.desc(E, k, H, I, g, *bits(l)) for l in range(n_layers)]
+    banks = {}
+    for d in descs:
+        key = (d.bits_gu, d.bits_down)
+        if key not in banks:
+            banks[key] = quantize_bank_gpu(E, d, seed + 17 * d.bits_down, device)
+    specs = [LayerSpec(d, banks[(d.bits_gu, d.bits_down)], synth.bank_permutation(seed, l, E).tolist())
+             for l, d in enumerate(descs)]
+    st = Streamer(specs, E, max_tokens=T, device=device)
+    for l in range(n_layers):
+        st.place(l, list(range(E)), synth.slot_permutation(seed, l, E).tolist())
+    assert all(ops.moe_ffn_kernel_path(d, T, True) == ops.MOE_PATH_TC_PREFILL for d in descs)
+    xs = torch.from_numpy(np.stack([synth.activations(seed, l, T, H).view(np.int16) for l in range(n_layers)]))
+    lg = torch.from_numpy(np.stack([synth.router_logits(seed, l, T, E) for l in range(n_layers)]))
+    x_d, lg_d = xs.to(device), lg.to(device)
+    s = st.stream
+    y = torch.zeros((T, H), dtype=torch.float32, device=device)
+
+    # whole path (route, sort with sorted x, per pass: FFN), host-driven passes
+    def whole(i0=0):
+        for l in range(n_layers):
+            st.prefill_layer(l, x_d[l], lg_d[l], T, y)
+
+    for _ in range(args.warmup):
+        whole()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(args.steps):
+        whole()
+    e1.record(s)
+    torch.cuda.synchronize(device)
+    whole_ms = e0.elapsed_time(e1) / args.steps
+
+    # per-layer routing snapshots, then a CUDA graph of every pass of every layer
+    snaps, n_act = [], []
+    for l in range(n_layers):
+        st.route_sort(l, x_d[l], lg_d[l], T, 0.0, want_sorted_x=True)
+        torch.cuda.synchronize(device)
+        snaps.append({"ids": st.ids[:T].clone(), "w": st.w[:T].clone(), "offsets": st.offsets.clone(),
+                      "pairs": st.pairs[:T * k].clone(), "meta": st.meta.clone(),
+                      "xs": st.x_sorted[:T * k].clone()})
+        n_act.append(int(snaps[-1]["meta"][0].item()))
+    g_ = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(device)
+    with torch.cuda.graph(g_, stream=cap):
+        cs = torch.cuda.current_stream(device)
+        for l in range(n_layers):
+            sn = snaps[l]
+            y.zero_()
+            for p in range(0, n_act[l], PASS_EXPERTS):
+                ops.moe_expert_ffn(x_d[l], T, descs[l], st.pool_of(l), st.n_slots_of(l), st.table_dev[l],
+                                   sn["ids"], sn["w"], sn["offsets"], sn["pairs"], sn["meta"][2:], sn["meta"][0:1],
+                                   sn["xs"], p, PASS_EXPERTS, y, st.ws, st.ws_bytes, st.dev_err, cs)
+    for _ in range(3):
+        g_.replay()
+    torch.cuda.synchronize(device)
+    with ClockSampler(local_rank) as clk:
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(s)
+        for _ in range(args.ffn_reps):
+            g_.replay()
+        f1.record(s)
+        torch.cuda.synchronize(device)
+    ffn_ms = f0.elapsed_time(f1) / args.ffn_reps  # all layers
+    del g_
+    t = torch.tensor([ffn_ms, whole_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ffn_ms, whole_ms = float(t[0].item()), float(t[1].item())
+    err = st.check_dev_err()
+
+    # e2e: x and logits from pinned host memory, y of every layer read back
+    xh, lgh = xs.pin_memory(), lg.pin_memory()
+    yh = torch.empty((n_layers, T, H), dtype=torch.float32).pin_memory()
+    xd2 = torch.empty_like(x_d)
+    lgd2 = torch.empty_like(lg_d)
+    torch.cuda.synchronize(device)
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record(s)
+    for _ in range(args.steps):
+        with torch.cuda.stream(s):
+            xd2.copy_(xh, non_blocking=True)
+            lgd2.copy_(lgh, non_blocking=True)
+        for l in range(n_layers):
+            st.prefill_layer(l, xd2[l], lgd2[l], T, y)
+            with torch.cuda.stream(s):
+                yh[l].copy_(y, non_blocking=True)
+    h1.record(s)
+    torch.cuda.synchronize(device)
+    e2e_ms = h0.elapsed_time(h1) / args.steps
+    if rank != 0:
+        return None
+    hbm_peak, tf_peak, peak_kind = peaks()
+    flops = sum(2.0 * T * k * 3 * H * I for _ in range(n_layers))
+    slot_b = [ops.moe_slot_bytes(d) for d in descs]
+    bytes_ = sum(n_act[l] * slot_b[l] + T * H * 2 + T * H * 4 for l in range(n_layers))
+    tflops = flops / (ffn_ms * 1e-3) / 1e12
+    gbs = bytes_ / (ffn_ms * 1e-3) / 1e9
+    return {
+        "metric": METRIC,
+        "value": round(tflops, 2),
+        "unit": "TFLOP/s (prefill expert FFN, all passes of %d layers)" % n_layers,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(whole_ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 tensor-core operands (dequantised 3/4/6-bit weights), fp32 TMEM accumulate",
+        "data": "synthetic (seeded N(0,0.02) experts quantised on the GPU; N(0,1) bf16 x; log-Zipf-biased logits)",
+        "config": {"workload": desc_txt, "layers": n_layers, "experts": E, "top_k": k, "hidden": H,
+                   "intermediate": I, "group": g, "tokens": T,
+                   "bits_per_layer": sorted({tuple(bits(l)) for l in range(n_layers)}),
+                   "active_experts_per_layer": round(sum(n_act) / n_layers, 1),
+                   "l2": "inputs larger than L2: %.0f MB of expert slots per replay" % (bytes_ / 1e6),
+                   "parallelism": f"replicas x{world} (independent chunks)"},
+        "ffn": {"ms_all_layers": round(ffn_ms, 3), "us_per_layer": round(1e3 * ffn_ms / n_layers, 1),
+                "tflops": round(tflops, 2), "hbm_gbs": round(gbs, 1),
+                "tok_s_equiv": round(T / (ffn_ms * 1e-3), 1),
+                "how": "CUDA graph of every pass (moe_expert_ffn) of every layer, replayed %d times, CUDA events"
+                       % args.ffn_reps},
+        "whole_path": {"ms_per_chunk": round(whole_ms, 3), "tok_s": round(T / (whole_ms * 1e-3), 1),
+                       "how": "route + sort (sorted x) + host-driven passes of the FFN, every layer"},
+        "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": tf_peak, "unit": "TFLOP/s",
+                     "frac": round(tflops / tf_peak, 4), "traffic": None,
+                     "hbm": {"achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                             "frac": round(gbs / hbm_peak, 4)},
+                     "kernel": "pf_gemm_kernel (gate/up + SwiGLU, down) + combine, per pass",
+                     "flops_per_layer": 2.0 * T * k * 3 * H * I, "peak_kind": peak_kind},
+        "gpu_launches": sum((n_act[l] + PASS_EXPERTS - 1) // PASS_EXPERTS for l in range(n_layers)) * 3 * args.ffn_reps,
+        "dev_err": err,
+        "clocks": clk.summary(),
+        "e2e": {"value": round(T / (e2e_ms * 1e-3), 1), "unit": "tok/s",
+                "h2d_bytes_per_step": int(xs.numel() * 2 + lg.numel() * 4),
+                "d2h_bytes_per_step": int(n_layers * T * H * 4)},
+        **({} if args.no_cpu_baseline else {"cpu_baseline": cpu_baseline_prefill(PREFILL[args.config], seed)}),
+    }
 
 
 def run_ours(args, rank, world, local_rank):
@@ -360,9 +532,51 @@ def cpu_baseline(cfg, seed, samples=2, as_reference=False):
                       f"scaled to {n_layers} layers; {dt:.2f} s of CPU time"}
 
 
+def cpu_baseline_prefill(pcfg, seed, n_tok=6):
+    """The oracle as it stands, single-threaded, on a bounded sample of a
+    prefill chunk: route + sort of the whole chunk of layer 0, then the FFN of
+    `n_tok` of its tokens (the oracle computes tokens one by one); the rate is
+    the sample's FFN flops over its time."""
+    import numpy as np
+
+    import oracle as orc
+    from streamed_quantized_expert_b200 import synth
+
+    n_layers, E, k, H, I, g, bits, T, _ = pcfg
+    bg, bd = bits(0)
+    x = synth.activations(seed, 0, T, H)
+    logits = synth.router_logits(seed, 0, T, E)
+    tok = np.linspace(0, T - 1, n_tok).astype(int)
+    ids, _, _ = orc.route(logits[tok], k)
+    slots = [None] * E
+    for e in np.unique(ids):
+        slots[int(e)] = orc.build_slot(*synth.expert_weights(seed, int(e), H, I), g, bg, bd)
+    t0 = time.perf_counter()
+    ids_all, w_all, _ = orc.route(logits, k)
+    orc.sort(ids_all, E)
+    ids_s, w_s, _ = orc.route(logits[tok], k)
+    orc.expert_ffn(x[tok], H, I, g, bg, bd, ids_s, w_s, slots)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * n_tok * k * 3 * H * I
+    return {"value": round(flops / dt / 1e12, 9), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": f"layer 0: route + sort of the {T}-token chunk, FFN of {n_tok} sampled tokens "
+                      f"({dt:.2f} s of CPU time)"}
+
+
 def run_reference(args, rank):
     if rank != 0:
         return None
+    if args.config in PREFILL:
+        pcfg = PREFILL[args.config]
+        vals = [cpu_baseline_prefill(pcfg, 7 + i, n_tok=2) for i in range(args.warmup + args.steps)][args.warmup:]
+        v = statistics.mean(r["value"] for r in vals)
+        return {"metric": METRIC, "impl": "reference", "value": v, "unit": "TFLOP/s (prefill expert FFN)",
+                "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+                "data": "synthetic", "config": {"workload": pcfg[-1]},
+                "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                                 "sample": "per step: route + sort of layer 0's chunk, FFN of 2 sampled tokens"},
+                "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     cfg = CONFIGS[args.config]
     n_layers, E, k, H, I, g, bg, bd, T, S, desc_txt = cfg
     vals = []
@@ -386,7 +600,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", choices=sorted(CONFIGS), default="decode")
+    ap.add_argument("--config", choices=sorted(CONFIGS) + sorted(PREFILL), default="decode")
     ap.add_argument("--cpu-layers", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ffn-reps", type=int, default=20)
@@ -397,7 +611,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.layers:
+    if args.layers and args.config in CONFIGS:
         c = list(CONFIGS[args.config])
         c[0] = args.layers
         c[-1] = c[-1] + f" [layers overridden to {args.layers}]"
@@ -417,7 +631,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        out = run_ours(args, rank, world, local_rank)
+        out = (run_prefill if args.config in PREFILL else run_ours)(args, rank, world, local_rank)
         if out is not None:
             print(json.dumps(out), flush=True)
     finally:

@@ -392,28 +392,62 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
 }
 
 // y[t][r] += sum_j [expert of (t,j) in the pass] w[t,j] * o[t*k+j][r], j ascending.
+// One warp per token: lane j tests pair j (k <= 32) and a ballot gives the
+// token's pairs in this pass; a token with none is skipped (its y row is not
+// touched unless y is overwritten).  Columns go 4 at a time.
 __global__ void combine_kernel(const FfnArgs a) {
   pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int w0 = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), nw = (int)((gridDim.x * blockDim.x) >> 5);
   const int n_act = pass_count(a);
-  if (n_act == 0) {
-    if (a.y_overwrite)
-      for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)a.T * a.H;
-           i += (int64_t)gridDim.x * blockDim.x)
-        a.y[i] = 0.f;
-    return;
-  }
-  const int e_lo = a.active[a.pass_begin], e_hi = a.active[a.pass_begin + n_act - 1];
-  const int64_t total = (int64_t)a.T * a.H;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-    const int t = (int)(i / a.H), r = (int)(i % a.H);
-    float s = 0.f;
-    for (int j = 0; j < a.k; ++j) {
-      const int pf = t * a.k + j;
+  const int e_lo = n_act > 0 ? a.active[a.pass_begin] : 1, e_hi = n_act > 0 ? a.active[a.pass_begin + n_act - 1] : 0;
+  const bool vec = (reinterpret_cast<uintptr_t>(a.y) & 15) == 0;
+  for (int t = w0; t < a.T; t += nw) {
+    bool in = false;
+    float wj = 0.f;
+    if (lane < a.k) {
+      const int pf = t * a.k + lane;
       const int e = a.ids[pf];
-      if (e >= e_lo && e <= e_hi && slot_ok(a, a.table[e])) s += a.w[pf] * a.o[(int64_t)pf * a.H + r];
+      in = e >= e_lo && e <= e_hi && slot_ok(a, a.table[e]);
+      wj = a.w[pf];
     }
-    a.y[i] = a.y_overwrite ? s : a.y[i] + s;
+    const unsigned mask = __ballot_sync(0xffffffffu, in);
+    if (mask == 0u && !a.y_overwrite) continue;
+    float* yrow = a.y + (int64_t)t * a.H;
+    for (int c = 4 * lane; c < a.H; c += 128) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (unsigned m = mask; m; m &= m - 1) {
+        const int j = __ffs(m) - 1;
+        const float wv = __shfl_sync(0xffffffffu, wj, j);  // mask is warp-uniform
+        const float4 o = *reinterpret_cast<const float4*>(a.o + ((int64_t)t * a.k + j) * a.H + c);
+        acc.x += wv * o.x;
+        acc.y += wv * o.y;
+        acc.z += wv * o.z;
+        acc.w += wv * o.w;
+      }
+      if (vec) {
+        float4* yp = reinterpret_cast<float4*>(yrow + c);
+        if (!a.y_overwrite) {
+          const float4 y0 = *yp;
+          acc.x += y0.x;
+          acc.y += y0.y;
+          acc.z += y0.z;
+          acc.w += y0.w;
+        }
+        *yp = acc;
+      } else {
+        const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+        for (int q = 0; q < 4; ++q) yrow[c + q] = a.y_overwrite ? v[q] : yrow[c + q] + v[q];
+      }
+    }
   }
+}
+
+// Grid of the combine: one warp per token, 8 warps per block.
+int combine_grid(int T, int num_sms) {
+  int g = (T + 7) / 8;
+  if (g > num_sms * 16) g = num_sms * 16;
+  return g < 1 ? 1 : g;
 }
 
 // ---------------------------------------------------------------------------
@@ -572,10 +606,7 @@ cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, c
   else if (mode == 1) e = dn_by_bits<1>(a, d.bits_down, gs, n_rt, dn_smem, st);
   else e = dn_by_bits<2>(a, d.bits_down, gs, n_rt, dn_smem, st);
   if (e != cudaSuccess || mode < 2) return e;
-  const int64_t total = (int64_t)a.T * d.H;
-  int cgrid = (int)((total + 255) / 256);
-  if (cgrid > num_sms * 8) cgrid = num_sms * 8;
-  return launch_pdl(reinterpret_cast<const void*>(combine_kernel), cgrid, 256, 0, st, a);
+  return launch_pdl(reinterpret_cast<const void*>(combine_kernel), combine_grid(a.T, num_sms), 256, 0, st, a);
 }
 
 }  // namespace moe

@@ -11,18 +11,22 @@
 // expert GEMMs: a token count per expert of tens to hundreds fits N, which
 // steps by 16, where it would leave most of a 128-row M tile empty).
 //
-// Warp roles (320 threads):
-//   0-3  dequant: thread = weight row; unpack the packed codes of a 128-input
-//        block (landed by TMA), w = fma(scale, q, bias) in bf16x2 with one
-//        rounding, stored as the MMA's A operand in the 128-byte swizzled
-//        K-major layout;
-//   4-7  epilogue: TMEM -> registers (warp i reads TMEM lanes 32 (i % 4)..);
-//   8    producer: TMA loads of codes, (scale, bias) words and token rows;
-//   9    MMA issuer (one thread): tcgen05.mma kind::f16 (bf16 x bf16 -> fp32
-//        in TMEM), M = 128, N = tokens rounded up to 16, K = 16 per
-//        instruction; tcgen05.commit frees stages and publishes accumulators.
+// Warp roles (704 threads):
+//   0-15  dequant: warp w = (K quarter w / 4, TMEM lane quadrant w % 4), lane
+//         = weight row; unpack its row's codes of a 128-input block (landed by
+//         TMA), w = fma(scale, q, bias) in bf16x2 with one rounding, and store
+//         the quarter's 16 bf16 pairs (inputs 32 q .. 32 q + 31) to the A
+//         operand in TMEM with one tcgen05.st (lane = row, column = input / 2);
+//   16-19 epilogue: TMEM -> registers (warp i reads TMEM lanes 32 (i % 4)..);
+//   20    producer: TMA loads of codes, (scale, bias) words and token rows;
+//   21    MMA issuer (one thread): tcgen05.mma kind::f16 (bf16 x bf16 -> fp32
+//        in TMEM) with A from TMEM and B (token rows) from shared memory,
+//        M = 128, N = tokens rounded up to 16, K = 16 per instruction;
+//        tcgen05.commit frees stages and publishes accumulators.
 // Accumulators are double-buffered in TMEM (2 x 128 columns), so the epilogue
-// of one tile overlaps the MMAs of the next.
+// of one tile overlaps the MMAs of the next; the two A buffers take 2 x 64
+// more columns.  With A in TMEM, shared memory carries only the TMA traffic
+// and the MMA's B reads (the dequantised tile never goes through it).
 //
 // Every wait is bounded; a wait that runs out sets a CTA-wide abort flag and
 // MOE_DEV_ERR_TIMEOUT, the roles leave their loops, the producer waits for
@@ -42,12 +46,16 @@ namespace {
 
 constexpr int kPfBM = 128;      // weight rows per tile (MMA M)
 constexpr int kPfBN = 128;      // tokens per tile (MMA N, at most)
-constexpr int kPfStages = 3;    // load stages (codes + scale/bias + token rows)
-constexpr int kPfABufs = 2;     // dequantised A buffers
-constexpr int kPfThreads = 320;
-constexpr int kPfTmemCols = 256;  // two accumulators of kPfBN fp32 columns
+constexpr int kPfABufs = 2;     // dequantised A buffers (in TMEM)
+constexpr int kPfDqWarps = 16;  // one per 8-row group of the 128-row tile
+constexpr int kPfEpiWarp0 = kPfDqWarps, kPfProdWarp = kPfDqWarps + 4, kPfMmaWarp = kPfDqWarps + 5;
+constexpr int kPfThreads = (kPfDqWarps + 6) * 32;
+constexpr int kPfTmemCols = 512;  // two accumulators of kPfBN fp32 columns, then two A buffers
+constexpr int kPfAcol = 2 * kPfBN;  // first TMEM column of the A buffers
+constexpr int kPfAcols = 64;       // one A buffer: 128 inputs as bf16 pairs, 128 lanes = rows
 constexpr int kPfXHalf = kPfBN * 128;   // one 64-input half of a token stage: 128 rows x 128 B
-constexpr int kPfAHalf = kPfBM * 128;   // one 64-input half of an A buffer
+// load stages (codes + scale/bias + token rows) that fit the shared memory
+__host__ __device__ constexpr int pf_stages(int bits) { return bits == 6 ? 4 : 5; }
 
 struct PfEntry {
   int slot;    // slot of the expert (tiles skipped when not resident)
@@ -127,6 +135,15 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Same with A (M x 16 bf16: lane m, columns k / 2) in TMEM at a_tmem.
+__device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::
+          "r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive on `bar` once every tcgen05 operation this thread issued so far has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
@@ -147,6 +164,16 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Thread i of the warp writes v to lane (base lane + i), columns col..col+15.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ bool slot_ok_pf(int n_slots, int slot) { return slot >= 0 && slot < n_slots; }
 
@@ -164,50 +191,49 @@ __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, volatile
   }
 }
 
-// One 128-input block of weight row r (0..127 of the tile) -> bf16 A operand.
-// Codes: the tile's 16 8-row groups, each 4 units x 8 rows x B words (unit t
-// of row rr at word (8 t + sigma) B); scale/bias: per 16-row tile, GPB groups
-// of 16 words.  Input k = 16 s + 2 t + 8 h' (+1) of the block is pair 2 s + h'
-// of unit t, so the 16-byte chunk c = 2 (s % 4) + h' of 64-input half s / 4
-// holds pair (2 s + h') of units 0..3 in that order.
-template <int B, int GPB>
-__device__ __forceinline__ void pf_dequant_block(const uint32_t* cs, const uint32_t* sbs, uint8_t* abuf, int r) {
+// K quarter CQ (inputs 32 CQ .. 32 CQ + 31) of weight row r (0..127 of the
+// tile) for one 128-input block -> 16 bf16 pairs, stored at TMEM columns
+// 16 CQ .. 16 CQ + 15 of this thread's lane (ta: the warp's lanes, A buffer
+// column 0).  Codes: the tile's 16 8-row groups, each 4 units x 8 rows x B
+// words (unit t of row rr at word (8 t + sigma) B); scale/bias: per 16-row
+// tile, GPB groups of 16 words.  Pair i = 2 s + h' of unit t holds inputs
+// 16 s + 2 t + 8 h' (+1), i.e. TMEM column 8 s + 4 h' + t: the quarter's
+// pairs are i = 4 CQ + m (m = 0..3) at local column 4 m + t.
+template <int B, int GPB, int CQ>
+__device__ __forceinline__ void pf_dequant_quarter(const uint8_t* cs, const uint32_t* sbs, uint32_t ta, int r) {
   const int g8 = r >> 3, rr = r & 7;
-  uint32_t p[4][16];
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    uint32_t w[B];
-    const uint32_t* up = cs + g8 * 32 * B + (8 * t + unit_sigma<B>(t, rr)) * B;
-#pragma unroll
-    for (int i = 0; i < B; ++i) w[i] = up[i];
-    unpack_unit<B>(w, p[t]);
-  }
-  __nv_bfloat162 sc[GPB], sc8[GPB], bi[GPB];
-#pragma unroll
-  for (int gi = 0; gi < GPB; ++gi) {
-    const uint32_t word = sbs[(r >> 4) * 16 * GPB + gi * 16 + (r & 15)];
-    const uint32_t s2 = (word & 0xFFFFu) * 0x10001u, b2 = (word >> 16) * 0x10001u;
-    sc[gi] = *reinterpret_cast<const __nv_bfloat162*>(&s2);
-    bi[gi] = *reinterpret_cast<const __nv_bfloat162*>(&b2);
-    sc8[gi] = __hmul2(sc[gi], __floats2bfloat162_rn(0.125f, 0.125f));
-  }
+  constexpr int GI = (CQ * GPB) / 4;  // the quarter's (single) group within the block
+  const uint32_t word = sbs[(r >> 4) * 16 * GPB + GI * 16 + (r & 15)];
+  const uint32_t s2 = (word & 0xFFFFu) * 0x10001u, b2 = (word >> 16) * 0x10001u;
+  const __nv_bfloat162 sc = *reinterpret_cast<const __nv_bfloat162*>(&s2);
+  const __nv_bfloat162 bi = *reinterpret_cast<const __nv_bfloat162*>(&b2);
+  const __nv_bfloat162 sc8 = __hmul2(sc, __floats2bfloat162_rn(0.125f, 0.125f));
   const uint32_t m = kMagic;
   const __nv_bfloat162 m128 = *reinterpret_cast<const __nv_bfloat162*>(&m);
-  uint8_t* rowbase = abuf + (r >> 3) * 1024 + (r & 7) * 128;
+  uint32_t out[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int s = i >> 1, hp = i & 1, hf = s >> 2, c = 2 * (s & 3) + hp;
-    const int gi = (s * GPB) >> 3;
-    const __nv_bfloat162 scale = PairShift<B>::a(i) == 3 ? sc8[gi] : sc[gi];
-    uint32_t o[4];
+  for (int t = 0; t < 4; ++t) {
+    uint32_t w[B], p[16];
+    load_unit<B>(cs + (g8 * 32 + 8 * t + unit_sigma<B>(t, rr)) * 4 * B, w);
+    unpack_unit<B>(w, p);
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const __nv_bfloat162 q = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&p[t][i]), m128);
-      const __nv_bfloat162 v = __hfma2(scale, q, bi[gi]);
-      o[t] = *reinterpret_cast<const uint32_t*>(&v);
+    for (int mm = 0; mm < 4; ++mm) {
+      const int i = 4 * CQ + mm;
+      const __nv_bfloat162 scale = PairShift<B>::a(i) == 3 ? sc8 : sc;
+      const __nv_bfloat162 q = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&p[i]), m128);
+      const __nv_bfloat162 v = __hfma2(scale, q, bi);
+      out[4 * mm + t] = *reinterpret_cast<const uint32_t*>(&v);
     }
-    *reinterpret_cast<uint4*>(rowbase + hf * kPfAHalf + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
   }
+  tmem_st16(ta + 16 * CQ, out);
+}
+
+template <int B, int GPB>
+__device__ __forceinline__ void pf_dequant(int cq, const uint8_t* cs, const uint32_t* sbs, uint32_t ta, int r) {
+  if (cq == 0) pf_dequant_quarter<B, GPB, 0>(cs, sbs, ta, r);
+  else if (cq == 1) pf_dequant_quarter<B, GPB, 1>(cs, sbs, ta, r);
+  else if (cq == 2) pf_dequant_quarter<B, GPB, 2>(cs, sbs, ta, r);
+  else pf_dequant_quarter<B, GPB, 3>(cs, sbs, ta, r);
 }
 
 struct PfTile {
@@ -222,16 +248,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   extern __shared__ uint8_t pf_smem_raw[];
   constexpr int kCodesBytes = 2048 * B;   // 16 groups x 4 units x 8 rows x B words
   constexpr int kSbBytes = 512 * GPB;     // 8 tiles x 16 GPB words
+  constexpr int kPfStages = pf_stages(B);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xst = base;                                           // [stage][2 halves][128 rows][128 B]
-  uint8_t* abuf = xst + kPfStages * 2 * kPfXHalf;                // [buf][2 halves][128 rows][128 B]
-  uint8_t* cst = abuf + kPfABufs * 2 * kPfAHalf;                 // [stage] codes
+  uint8_t* cst = xst + kPfStages * 2 * kPfXHalf;                 // [stage] codes
   uint8_t* sbst = cst + kPfStages * kCodesBytes;                 // [stage] scale/bias words
   uint64_t* bars = reinterpret_cast<uint64_t*>(sbst + kPfStages * kSbBytes);
   uint64_t* full = bars;                        // producer (expect_tx) -> dequant, MMA
   uint64_t* empty = full + kPfStages;           // MMA commit -> producer
-  uint64_t* afull = empty + kPfStages;          // dequant threads (128) -> MMA
+  uint64_t* afull = empty + kPfStages;          // dequant warps (TMEM stores done) -> MMA
   uint64_t* aempty = afull + kPfABufs;          // MMA commit -> dequant
   uint64_t* accfull = aempty + kPfABufs;        // MMA commit -> epilogue
   uint64_t* accempty = accfull + 2;             // epilogue threads (128) -> MMA
@@ -247,7 +273,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < kPfABufs; ++b) {
-      mbar_init(&afull[b], 128);
+      mbar_init(&afull[b], kPfDqWarps);
       mbar_init(&aempty[b], 1);
     }
     for (int c = 0; c < 2; ++c) {
@@ -258,13 +284,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     fence_barrier_init();
     s_abort = 0;
   }
-  if (warp == 9) {  // TMEM: two accumulators of kPfBN columns
+  if (warp == kPfMmaWarp) {  // TMEM: two accumulators of kPfBN columns
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
                  "r"(kPfTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == kPfProdWarp && lane == 0) {
     tmap_prefetch(&tm_q);
     tmap_prefetch(&tm_sb);
     tmap_prefetch(&tm_b);
@@ -318,7 +344,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     return tl;
   };
 
-  if (warp == 8) {
+  if (warp == kPfProdWarp) {
     // ---------------- producer ----------------
     if (lane == 0) {
       int s = 0;
@@ -354,7 +380,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int q = 0; q < kPfStages; ++q)
         if ((issued >> q) & 1u) mbar_wait_bounded(&full[q], (last_ph >> q) & 1u);
     }
-  } else if (warp == 9) {
+  } else if (warp == kPfMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       int s = 0, ab = 0, c = 0;
@@ -374,11 +400,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t abase = smem_addr(abuf + ab * 2 * kPfAHalf), xbase = smem_addr(xst + s * 2 * kPfXHalf);
+          const uint32_t a_tm = tmem_base + (uint32_t)(kPfAcol + ab * kPfAcols);
+          const uint32_t xbase = smem_addr(xst + s * 2 * kPfXHalf);
 #pragma unroll
           for (int k16 = 0; k16 < 8; ++k16) {
-            const uint32_t off = (uint32_t)((k16 >> 2) * kPfAHalf + (k16 & 3) * 32);
-            umma_bf16(d, sw128_desc(abase + off), sw128_desc(xbase + off), idesc, (kb | k16) != 0 ? 1u : 0u);
+            const uint32_t off = (uint32_t)((k16 >> 2) * kPfXHalf + (k16 & 3) * 32);
+            umma_bf16_ta(d, a_tm + 8 * k16, sw128_desc(xbase + off), idesc, (kb | k16) != 0 ? 1u : 0u);
           }
           issued_any = true;
           umma_commit(&empty[s]);
@@ -404,8 +431,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         mbar_wait_bounded(drain, 0);
       }
     }
-  } else if (warp < 4) {
+  } else if (warp < kPfDqWarps) {
     // ---------------- dequant ----------------
+    const int q = warp & 3, cq = warp >> 2, r = 32 * q + lane;  // TMEM lane quadrant, K quarter, weight row
     int s = 0, ab = 0;
     uint32_t ph = 0, pa = 0;
     for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
@@ -415,11 +443,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           ok = false;
           break;
         }
-        pf_dequant_block<B, GPB>(reinterpret_cast<const uint32_t*>(cst + s * kCodesBytes),
-                                 reinterpret_cast<const uint32_t*>(sbst + s * kSbBytes), abuf + ab * 2 * kPfAHalf,
-                                 tid);
-        proxy_fence_smem();
-        mbar_arrive(&afull[ab]);
+        tc_fence_after();
+        pf_dequant<B, GPB>(cq, cst + s * kCodesBytes, reinterpret_cast<const uint32_t*>(sbst + s * kSbBytes),
+                           tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kPfAcol + ab * kPfAcols), r);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[ab]);
         if (++s == kPfStages) {
           s = 0;
           ph ^= 1u;
@@ -432,7 +462,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (!ok) break;
     }
   } else {
-    // ---------------- epilogue (warps 4-7: TMEM lanes 32 (warp % 4) ..) ----------------
+    // ---------------- epilogue (TMEM lanes 32 (warp % 4) ..) ----------------
     const int q = warp & 3, r = 32 * q + lane;
     int c = 0;
     uint32_t pc = 0;
@@ -441,26 +471,41 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (!pf_wait(&accfull[c], pc, &s_abort)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * kPfBN);
-      for (int n0 = 0; n0 < tl.n; n0 += 16) {
-        uint32_t v[16];
-        tmem_ld16(taddr + (uint32_t)n0, v);
-        tmem_ld_wait();
-        if (GU) {
-          // storage rows: 16-row blocks of 8 gate rows then 8 up rows
-          const bool gate = (r & 15) < 8;
-          const int j = tl.mt * (kPfBM / 2) + (r >> 4) * 8 + (r & 7);
+      // the tile's pair indices (down) in registers: lane l holds columns l, 32 + l, ...
+      int pidx[kPfBN / 32];
+      if (!GU) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float x = __uint_as_float(v[i]);
-            const float u = __shfl_xor_sync(0xffffffffu, x, 8);
-            if (gate && n0 + i < tl.n)
-              a.h[(int64_t)(tl.row0 + n0 + i) * a.I + j] = f32_to_bf16_rne(x / (1.0f + expf(-x)) * u);
+        for (int q4 = 0; q4 < kPfBN / 32; ++q4)
+          pidx[q4] = 32 * q4 + lane < tl.n ? a.pairs[tl.row0 + 32 * q4 + lane] : 0;
+      }
+      const bool gate = (r & 15) < 8;  // storage rows: 16-row blocks of 8 gate rows then 8 up rows
+      const int j = tl.mt * (kPfBM / 2) + (r >> 4) * 8 + (r & 7);
+      const int row = tl.mt * kPfBM + r;
+#pragma unroll
+      for (int nb = 0; nb < kPfBN / 32; ++nb) {
+        if (32 * nb >= tl.n) break;
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+          const int n0 = 32 * nb + 16 * hb;
+          if (n0 >= tl.n) break;
+          uint32_t v[16];
+          tmem_ld16(taddr + (uint32_t)n0, v);
+          tmem_ld_wait();
+          if (GU) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float x = __uint_as_float(v[i]);
+              const float u = __shfl_xor_sync(0xffffffffu, x, 8);
+              if (gate && n0 + i < tl.n)
+                a.h[(int64_t)(tl.row0 + n0 + i) * a.I + j] = f32_to_bf16_rne(__fdividef(x, 1.0f + __expf(-x)) * u);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int pf = __shfl_sync(0xffffffffu, pidx[nb], 16 * hb + i);
+              if (n0 + i < tl.n) a.o[(int64_t)pf * a.H + row] = __uint_as_float(v[i]);
+            }
           }
-        } else {
-          const int row = tl.mt * kPfBM + r;
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (n0 + i < tl.n) a.o[(int64_t)a.pairs[tl.row0 + n0 + i] * a.H + row] = __uint_as_float(v[i]);
         }
       }
       tc_fence_before();
@@ -476,7 +521,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 9)
+  if (warp == kPfMmaWarp)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kPfTmemCols)
                  : "memory");
 }
@@ -535,8 +580,8 @@ bool encode_rows(CUtensorMap* m, const uint16_t* base, int64_t rows, int cols) {
 }
 
 size_t pf_smem_bytes(int bits, int gpb) {
-  return 1024 + (size_t)kPfStages * 2 * kPfXHalf + (size_t)kPfABufs * 2 * kPfAHalf + (size_t)kPfStages * 2048 * bits +
-         (size_t)kPfStages * 512 * gpb + 16 * 8;
+  const size_t ns = (size_t)pf_stages(bits);
+  return 1024 + ns * 2 * kPfXHalf + ns * 2048 * bits + ns * 512 * gpb + (2 * ns + 2 * kPfABufs + 5) * 8;
 }
 
 template <int B, int GPB, bool GU>
@@ -626,10 +671,7 @@ cudaError_t launch_ffn_prefill_tc(const FfnArgs& a, const moe_layer_desc& d, int
   pa.mtiles = d.H / kPfBM;
   e = launch_pf<false>(d.bits_down, gpb, q_d, sb_d, hm, pa, grid, st);
   if (e != cudaSuccess) return e;
-  const int64_t total = (int64_t)a.T * d.H;
-  int cgrid = (int)((total + 255) / 256);
-  if (cgrid > num_sms * 8) cgrid = num_sms * 8;
-  return launch_pdl(reinterpret_cast<const void*>(combine_kernel), cgrid, 256, 0, st, a);
+  return launch_pdl(reinterpret_cast<const void*>(combine_kernel), combine_grid(a.T, num_sms), 256, 0, st, a);
 }
 
 }  // namespace moe
