@@ -30,6 +30,28 @@ sys.path.insert(0, ROOT)
 METRIC = "expert-FFN HBM GB/s & decode tok/s-equiv; prefill TFLOP/s; % of B200 roofline"
 
 
+def recorded_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the ncu capture recorded in
+    profiles/traffic.txt, or None when the kernel's sources changed since."""
+    import hashlib
+
+    try:
+        for line in open(os.path.join(ROOT, "profiles", "traffic.txt")):
+            if line.startswith("#") or not line.strip():
+                continue
+            f = dict(kv.split("=", 1) for kv in line.split())
+            if f.get("kernel") != kernel:
+                continue
+            m = hashlib.sha256()
+            for src in f["sources"].split(","):
+                with open(os.path.join(ROOT, "streamed_quantized_expert_b200", "csrc", src), "rb") as fh:
+                    m.update(fh.read())
+            return int(f["bytes"]) if m.hexdigest()[:16] == f["source_sha256"] else None
+    except Exception:
+        return None
+    return None
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
@@ -342,7 +364,9 @@ def run_prefill(args, rank, world, local_rank):
         "whole_path": {"ms_per_chunk": round(whole_ms, 3), "tok_s": round(T / (whole_ms * 1e-3), 1),
                        "how": "route + sort (sorted x) + host-driven passes of the FFN, every layer"},
         "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": tf_peak, "unit": "TFLOP/s",
-                     "frac": round(tflops / tf_peak, 4), "traffic": None,
+                     "frac": round(tflops / tf_peak, 4),
+                     "traffic": recorded_traffic("pf_gemm_kernel"),
+                     "traffic_note": "DRAM bytes of one pass's gate/up + down launches (uniform routing, 4096 tokens)",
                      "hbm": {"achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                              "frac": round(gbs / hbm_peak, 4)},
                      "kernel": "pf_gemm_kernel (gate/up + SwiGLU, down) + combine, per pass",
@@ -479,8 +503,11 @@ def run_ours(args, rank, world, local_rank):
                      "miss_rate": round(installs / max(args.steps * n_layers * T * k, 1), 4),
                      "bytes": inst_bytes},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "traffic": None,
-                     "kernel": "moe_expert_ffn (gate/up+SwiGLU kernel + down+combine kernel), per layer",
+                     "frac": round(achieved / hbm_peak, 4),
+                     "traffic": recorded_traffic("ffn_fused_kernel") if T * k <= 64 and T <= 8 else None,
+                     "kernel": ("ffn_fused_kernel (one launch per layer: gate/up + SwiGLU, grid barrier, down + "
+                                "combine)" if T <= 8 and T * k <= 64 else
+                                "moe_expert_ffn (gate/up+SwiGLU kernel + down kernel), per layer"),
                      "bytes_per_launch": int(ffn_bytes), "peak_kind": peak_kind},
         "gpu_launches": launches,
         "dev_err": err,
