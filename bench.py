@@ -70,7 +70,13 @@ CONFIGS = {
               "Coder-30B-like batched decode: 48 layers x 128 experts, top-8, H 2048, I 768, 4-bit g64, "
               "64 tokens/step, all 128 experts resident"),
     "tiny": (1, 8, 2, 64, 32, 32, 4, 4, 4, 8, "tiny MoE layer: 8 experts, top-2, H 64, I 32, 4-bit g32, 4 tokens"),
+    "decode_mixed": (48, 512, 10, 2048, 512, 64, 4, 4, 1, 128,
+                     "mixed size classes decode with cache-aware substitution: Flash-Next-like shapes, 4-bit "
+                     "gate/up, 6-bit down on layers l % 4 == 0 (2 slot size classes), 1 token/step, 128 slots/layer "
+                     "(25% resident), L = 0.15, misses installed from pinned host"),
 }
+# per-layer widths and the substitution strength of the decode configurations (default: uniform, L = 0)
+DECODE_EXTRA = {"decode_mixed": {"bits": lambda l: (4, 6) if l % 4 == 0 else (4, 4), "L": 0.15}}
 
 # Prefill chunks: every expert of every layer resident (the metric is the expert
 # FFN's tensor-core rate; installs are PCIe-bound and reported by decode).
@@ -147,7 +153,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
-def build_streamer(cfg, seed, device):
+def build_streamer(cfg, seed, device, bits=None):
     import numpy as np
     import torch
 
@@ -155,9 +161,13 @@ def build_streamer(cfg, seed, device):
     from streamed_quantized_expert_b200.runtime import LayerSpec, Streamer, quantize_bank_gpu
 
     n_layers, E, k, H, I, g, bg, bd, T, S, _ = cfg
-    d = ops.desc(E, k, H, I, g, bg, bd)
-    bank = quantize_bank_gpu(E, d, seed, device)  # one layer's worth of distinct experts, pinned
-    specs = [LayerSpec(d, bank, synth.bank_permutation(seed, l, E).tolist()) for l in range(n_layers)]
+    descs = [ops.desc(E, k, H, I, g, *(bits(l) if bits else (bg, bd))) for l in range(n_layers)]
+    banks = {}  # one layer's worth of distinct experts per size class, pinned
+    for d in descs:
+        if (d.bits_gu, d.bits_down) not in banks:
+            banks[(d.bits_gu, d.bits_down)] = quantize_bank_gpu(E, d, seed + 17 * d.bits_down, device)
+    specs = [LayerSpec(d, banks[(d.bits_gu, d.bits_down)], synth.bank_permutation(seed, l, E).tolist())
+             for l, d in enumerate(descs)]
     st = Streamer(specs, S, max_tokens=T, device=device)
     for l in range(n_layers):  # the S most popular experts start resident, on a random slot permutation
         hot = np.argsort(synth.popularity_rank(seed, l, E))[:S]
@@ -394,8 +404,10 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(device)
     cfg = CONFIGS[args.config]
     n_layers, E, k, H, I, g, bg, bd, T, S, desc_txt = cfg
+    extra = DECODE_EXTRA.get(args.config, {})
+    Lsub = extra.get("L", 0.0)
     seed = 1000 * rank
-    st = build_streamer(cfg, seed, device)
+    st = build_streamer(cfg, seed, device, extra.get("bits"))
     steps_total = args.warmup + args.steps
     # the popularity bias of the logits and the initially resident experts come from the same seed
     x, logits = make_inputs(cfg, seed, steps_total + 1, device)
@@ -403,7 +415,7 @@ def run_ours(args, rank, world, local_rank):
 
     def step(i, x_src, lg_src):
         for l in range(n_layers):
-            st.decode_layer(l, x_src[i, l], lg_src[i, l], T)
+            st.decode_layer(l, x_src[i, l], lg_src[i, l], T, Lsub)
 
     for i in range(args.warmup):
         step(i, x, logits)
@@ -427,7 +439,7 @@ def run_ours(args, rank, world, local_rank):
         # one more (untimed) step whose per-layer routing is kept for the FFN-only replay
         snaps = []
         for l in range(n_layers):
-            st.decode_layer(l, x[steps_total, l], logits[steps_total, l], T)
+            st.decode_layer(l, x[steps_total, l], logits[steps_total, l], T, Lsub)
             snaps.append({"x": x[steps_total, l], "ids": st.ids.clone(), "w": st.w.clone(),
                           "offsets": st.offsets.clone(), "pairs": st.pairs.clone(), "meta": st.meta.clone()})
         torch.cuda.synchronize(device)
@@ -438,6 +450,19 @@ def run_ours(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_max = float(t.item())
     err = st.check_dev_err()
+    miss_no_sub = None
+    if Lsub > 0:  # the same token sequence from the same initial cache, without substitution (untimed)
+        st0 = build_streamer(cfg, seed, device, extra.get("bits"))
+        base0 = 0
+        for i in range(steps_total):
+            if i == args.warmup:
+                base0 = st0.installs
+            for l in range(n_layers):
+                st0.decode_layer(l, x[i, l], logits[i, l], T, 0.0)
+        torch.cuda.synchronize(device)
+        miss_no_sub = round((st0.installs - base0) / max(args.steps * n_layers * T * k, 1), 4)
+        del st0
+        torch.cuda.empty_cache()
 
     # e2e: inputs from pinned host memory copied in, y of every layer read back, same K steps
     xh, lgh = make_inputs(cfg, seed, args.steps, device, pinned=True, step0=steps_total + 1)
@@ -454,7 +479,7 @@ def run_ours(args, rank, world, local_rank):
             xd.copy_(xh[i], non_blocking=True)
             lgd.copy_(lgh[i], non_blocking=True)
         for l in range(n_layers):
-            y = st.decode_layer(l, xd[l], lgd[l], T)
+            y = st.decode_layer(l, xd[l], lgd[l], T, Lsub)
             with torch.cuda.stream(s):
                 yh[i, l].copy_(y, non_blocking=True)
     f1.record(s)
@@ -471,8 +496,9 @@ def run_ours(args, rank, world, local_rank):
     tokens = args.steps * T * world
     from streamed_quantized_expert_b200 import ops as _ops
 
-    slot_b = _ops.moe_slot_bytes(_ops.desc(E, k, H, I, g, bg, bd))
-    ffn_bytes = n_unique * slot_b + T * H * 2 + T * H * 4
+    slot_bytes = [_ops.moe_slot_bytes(st.layers[l].desc) for l in range(n_layers)]
+    ffn_bytes = (sum(int(sn["meta"][0].item()) * slot_bytes[l] for l, sn in enumerate(snaps)) / n_layers
+                 + T * H * 2 + T * H * 4)
     achieved = ffn_bytes / (ffn_us * 1e-6) / 1e9
     flops_per_ffn = 2.0 * T * k * 3 * H * I
     out = {
@@ -501,7 +527,10 @@ def run_ours(args, rank, world, local_rank):
                        (n_layers, args.ffn_reps)},
         "installs": {"experts": installs, "per_token": round(installs / max(args.steps * T, 1), 2),
                      "miss_rate": round(installs / max(args.steps * n_layers * T * k, 1), 4),
-                     "bytes": inst_bytes},
+                     "bytes": inst_bytes, "substitution_L": Lsub,
+                     **({} if miss_no_sub is None else
+                        {"miss_rate_without_substitution": miss_no_sub,
+                         "how_compared": "same tokens and initial cache, L = 0, installs of the timed steps"})},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4),
                      "traffic": recorded_traffic("ffn_fused_kernel") if T * k <= 64 and T <= 8 else None,

@@ -11,15 +11,16 @@
 // expert GEMMs: a token count per expert of tens to hundreds fits N, which
 // steps by 16, where it would leave most of a 128-row M tile empty).
 //
-// Warp roles (704 threads):
+// Warp roles (832 threads):
 //   0-15  dequant: warp w = (K quarter w / 4, TMEM lane quadrant w % 4), lane
 //         = weight row; unpack its row's codes of a 128-input block (landed by
 //         TMA), w = fma(scale, q, bias) in bf16x2 with one rounding, and store
 //         the quarter's 16 bf16 pairs (inputs 32 q .. 32 q + 31) to the A
 //         operand in TMEM with one tcgen05.st (lane = row, column = input / 2);
-//   16-19 epilogue: TMEM -> registers (warp i reads TMEM lanes 32 (i % 4)..);
-//   20    producer: TMA loads of codes, (scale, bias) words and token rows;
-//   21    MMA issuer (one thread): tcgen05.mma kind::f16 (bf16 x bf16 -> fp32
+//   16-23 epilogue: TMEM -> registers (warp i reads TMEM lanes 32 (i % 4)..;
+//         the two warps of a quadrant take alternate 16-column chunks);
+//   24    producer: TMA loads of codes, (scale, bias) words and token rows;
+//   25    MMA issuer (one thread): tcgen05.mma kind::f16 (bf16 x bf16 -> fp32
 //        in TMEM) with A from TMEM and B (token rows) from shared memory,
 //        M = 128, N = tokens rounded up to 16, K = 16 per instruction;
 //        tcgen05.commit frees stages and publishes accumulators.
@@ -48,8 +49,9 @@ constexpr int kPfBM = 128;      // weight rows per tile (MMA M)
 constexpr int kPfBN = 128;      // tokens per tile (MMA N, at most)
 constexpr int kPfABufs = 2;     // dequantised A buffers (in TMEM)
 constexpr int kPfDqWarps = 16;  // one per 8-row group of the 128-row tile
-constexpr int kPfEpiWarp0 = kPfDqWarps, kPfProdWarp = kPfDqWarps + 4, kPfMmaWarp = kPfDqWarps + 5;
-constexpr int kPfThreads = (kPfDqWarps + 6) * 32;
+constexpr int kPfEpiWarps = 8;  // two per TMEM lane quadrant, taking alternate 16-column chunks
+constexpr int kPfEpiWarp0 = kPfDqWarps, kPfProdWarp = kPfEpiWarp0 + kPfEpiWarps, kPfMmaWarp = kPfProdWarp + 1;
+constexpr int kPfThreads = (kPfMmaWarp + 1) * 32;
 constexpr int kPfTmemCols = 512;  // two accumulators of kPfBN fp32 columns, then two A buffers
 constexpr int kPfAcol = 2 * kPfBN;  // first TMEM column of the A buffers
 constexpr int kPfAcols = 64;       // one A buffer: 128 inputs as bf16 pairs, 128 lanes = rows
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* afull = empty + kPfStages;          // dequant warps (TMEM stores done) -> MMA
   uint64_t* aempty = afull + kPfABufs;          // MMA commit -> dequant
   uint64_t* accfull = aempty + kPfABufs;        // MMA commit -> epilogue
-  uint64_t* accempty = accfull + 2;             // epilogue threads (128) -> MMA
+  uint64_t* accempty = accfull + 2;             // epilogue threads -> MMA
   uint64_t* drain = accempty + 2;               // MMA commit at exit
   __shared__ PfEntry s_ent[kMaxCtaExperts];
   __shared__ int s_nent, s_ntiles;
@@ -278,7 +280,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     for (int c = 0; c < 2; ++c) {
       mbar_init(&accfull[c], 1);
-      mbar_init(&accempty[c], 128);
+      mbar_init(&accempty[c], kPfEpiWarps * 32);
     }
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -463,7 +465,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
   } else {
     // ---------------- epilogue (TMEM lanes 32 (warp % 4) ..) ----------------
-    const int q = warp & 3, r = 32 * q + lane;
+    const int q = warp & 3, r = 32 * q + lane, eh = (warp - kPfEpiWarp0) >> 2;  // quadrant, row, chunk parity
     int c = 0;
     uint32_t pc = 0;
     for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
@@ -488,6 +490,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int hb = 0; hb < 2; ++hb) {
           const int n0 = 32 * nb + 16 * hb;
           if (n0 >= tl.n) break;
+          if (hb != eh) continue;  // the other warp of this quadrant takes this chunk
           uint32_t v[16];
           tmem_ld16(taddr + (uint32_t)n0, v);
           tmem_ld_wait();
