@@ -392,17 +392,23 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
 }
 
 // y[t][r] += sum_j [expert of (t,j) in the pass] w[t,j] * o[t*k+j][r], j ascending.
-// One warp per token: lane j tests pair j (k <= 32) and a ballot gives the
-// token's pairs in this pass; a token with none is skipped (its y row is not
-// touched unless y is overwritten).  Columns go 4 at a time.
+// One warp per (token, 256-column chunk): lane j tests pair j (k <= 32) and a
+// ballot gives the token's pairs in this pass; a token with none is skipped
+// (its y row is not touched unless y is overwritten).  Each lane sums two
+// groups of 4 columns, so a warp issues its loads together.
+constexpr int kCombineChunk = 256;
+
 __global__ void combine_kernel(const FfnArgs a) {
   pdl_wait();
   const int lane = threadIdx.x & 31;
-  const int w0 = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), nw = (int)((gridDim.x * blockDim.x) >> 5);
+  const int64_t w0 = (int64_t)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int64_t nw = (int64_t)((gridDim.x * blockDim.x) >> 5);
+  const int nch = (a.H + kCombineChunk - 1) / kCombineChunk;
   const int n_act = pass_count(a);
   const int e_lo = n_act > 0 ? a.active[a.pass_begin] : 1, e_hi = n_act > 0 ? a.active[a.pass_begin + n_act - 1] : 0;
   const bool vec = (reinterpret_cast<uintptr_t>(a.y) & 15) == 0;
-  for (int t = w0; t < a.T; t += nw) {
+  for (int64_t it = w0; it < (int64_t)a.T * nch; it += nw) {
+    const int t = (int)(it / nch), ch = (int)(it % nch);
     bool in = false;
     float wj = 0.f;
     if (lane < a.k) {
@@ -414,40 +420,52 @@ __global__ void combine_kernel(const FfnArgs a) {
     const unsigned mask = __ballot_sync(0xffffffffu, in);
     if (mask == 0u && !a.y_overwrite) continue;
     float* yrow = a.y + (int64_t)t * a.H;
-    for (int c = 4 * lane; c < a.H; c += 128) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (unsigned m = mask; m; m &= m - 1) {
-        const int j = __ffs(m) - 1;
-        const float wv = __shfl_sync(0xffffffffu, wj, j);  // mask is warp-uniform
-        const float4 o = *reinterpret_cast<const float4*>(a.o + ((int64_t)t * a.k + j) * a.H + c);
-        acc.x += wv * o.x;
-        acc.y += wv * o.y;
-        acc.z += wv * o.z;
-        acc.w += wv * o.w;
+    float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+    const int c0 = ch * kCombineChunk + 4 * lane;
+    for (unsigned m = mask; m; m &= m - 1) {
+      const int j = __ffs(m) - 1;
+      const float wv = __shfl_sync(0xffffffffu, wj, j);  // mask is warp-uniform
+      const float* orow = a.o + ((int64_t)t * a.k + j) * a.H;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c = c0 + 128 * h;
+        if (c < a.H) {
+          const float4 o = *reinterpret_cast<const float4*>(orow + c);
+          acc[h].x += wv * o.x;
+          acc[h].y += wv * o.y;
+          acc[h].z += wv * o.z;
+          acc[h].w += wv * o.w;
+        }
       }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = c0 + 128 * h;
+      if (c >= a.H) continue;
       if (vec) {
         float4* yp = reinterpret_cast<float4*>(yrow + c);
         if (!a.y_overwrite) {
           const float4 y0 = *yp;
-          acc.x += y0.x;
-          acc.y += y0.y;
-          acc.z += y0.z;
-          acc.w += y0.w;
+          acc[h].x += y0.x;
+          acc[h].y += y0.y;
+          acc[h].z += y0.z;
+          acc[h].w += y0.w;
         }
-        *yp = acc;
+        *yp = acc[h];
       } else {
-        const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+        const float v[4] = {acc[h].x, acc[h].y, acc[h].z, acc[h].w};
         for (int q = 0; q < 4; ++q) yrow[c + q] = a.y_overwrite ? v[q] : yrow[c + q] + v[q];
       }
     }
   }
 }
 
-// Grid of the combine: one warp per token, 8 warps per block.
-int combine_grid(int T, int num_sms) {
-  int g = (T + 7) / 8;
-  if (g > num_sms * 16) g = num_sms * 16;
-  return g < 1 ? 1 : g;
+// Grid of the combine: one warp per (token, column chunk), 8 warps per block.
+int combine_grid(int T, int H, int num_sms) {
+  const int64_t items = (int64_t)T * ((H + kCombineChunk - 1) / kCombineChunk);
+  int64_t g = (items + 7) / 8;
+  if (g > (int64_t)num_sms * 16) g = (int64_t)num_sms * 16;
+  return g < 1 ? 1 : (int)g;
 }
 
 // ---------------------------------------------------------------------------
@@ -606,7 +624,7 @@ cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, c
   else if (mode == 1) e = dn_by_bits<1>(a, d.bits_down, gs, n_rt, dn_smem, st);
   else e = dn_by_bits<2>(a, d.bits_down, gs, n_rt, dn_smem, st);
   if (e != cudaSuccess || mode < 2) return e;
-  return launch_pdl(reinterpret_cast<const void*>(combine_kernel), combine_grid(a.T, num_sms), 256, 0, st, a);
+  return launch_pdl(reinterpret_cast<const void*>(combine_kernel), combine_grid(a.T, d.H, num_sms), 256, 0, st, a);
 }
 
 }  // namespace moe

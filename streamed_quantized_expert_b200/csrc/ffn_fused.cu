@@ -532,12 +532,15 @@ bool ffn_fused_plan(FfnArgs& a, const moe_layer_desc& d, int num_sms, size_t& sm
                        kFuTableBytes;
   const size_t cap = 220 * 1024;
   if (fixed + a.gu_stage_bytes + a.d_stage_bytes + 64 > cap) return false;
-  // down stages: every expert of the pass if possible, else half the room
-  int nsd = max_pass;
+  // down stages: every expert of the pass if possible, else half the room; at
+  // least one per down warp group, so that a window of experts never waits on
+  // a stage it has not released
+  constexpr int kMinDn = kFuConsumers / kDnKSplit;
+  int nsd = max_pass > kMinDn ? max_pass : kMinDn;
   int nsg = (int)(items_per_cta < 1 ? 1 : items_per_cta);
   while ((size_t)nsd * a.d_stage_bytes + (size_t)nsg * a.gu_stage_bytes + fixed + 16 * (nsd + nsg) > cap) {
     if (nsg > nsd && nsg > 2) --nsg;
-    else if (nsd > 2) --nsd;
+    else if (nsd > kMinDn) --nsd;
     else if (nsg > 1) --nsg;
     else return false;
   }

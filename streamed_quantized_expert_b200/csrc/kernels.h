@@ -11,6 +11,7 @@ namespace moe {
 
 constexpr int kFusedMaxTokens = 64;  // decode down kernel combines in shared memory up to this T
 constexpr int kPrefillTcMinTokens = 256;  // from this T on, prefill runs on the tcgen05 grouped GEMM
+constexpr int kRouteBlockMaxTokens = 64;  // up to this T, routing takes a block (8 warps) per token
 
 struct FfnArgs {
   const uint16_t* x;
@@ -85,7 +86,7 @@ bool ffn_fused_plan(FfnArgs& a, const moe_layer_desc& d, int num_sms, size_t& sm
 bool ffn_prefill_tc_shape_ok(const moe_layer_desc& d);
 int ffn_kernel_path(const moe_layer_desc& d, int T, bool has_x_sorted, int num_sms);
 __global__ void combine_kernel(const FfnArgs a);
-int combine_grid(int T, int num_sms);
+int combine_grid(int T, int H, int num_sms);
 constexpr size_t kWsControlBytes = 256;  // head of the workspace: grid-barrier words
 
 }  // namespace moe

@@ -129,15 +129,8 @@ __device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
-          d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// Same with A (M x 16 bf16: lane m, columns k / 2) in TMEM at a_tmem.
+// D (TMEM, fp32) (+)= A . B^T, M x N x 16: A (M x 16 bf16: lane m, columns k / 2) in TMEM at a_tmem,
+// B (N x 16 bf16, K-major, 128-byte swizzled) in shared memory; kind::f16.
 __device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                              uint32_t accumulate) {
   asm volatile(
@@ -153,7 +146,6 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void proxy_fence_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // 32 TMEM lanes x 16 consecutive 32-bit columns: thread i of the warp gets
 // lane (base lane + i), columns col..col+15.
@@ -674,7 +666,7 @@ cudaError_t launch_ffn_prefill_tc(const FfnArgs& a, const moe_layer_desc& d, int
   pa.mtiles = d.H / kPfBM;
   e = launch_pf<false>(d.bits_down, gpb, q_d, sb_d, hm, pa, grid, st);
   if (e != cudaSuccess) return e;
-  return launch_pdl(reinterpret_cast<const void*>(combine_kernel), combine_grid(a.T, num_sms), 256, 0, st, a);
+  return launch_pdl(reinterpret_cast<const void*>(combine_kernel), combine_grid(a.T, d.H, num_sms), 256, 0, st, a);
 }
 
 }  // namespace moe

@@ -136,6 +136,162 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
   }
 }
 
+// One block (8 warps) per token, for decode-sized T: thread i owns experts
+// e = i + 256 m.  Each warp takes the top-k of its experts by the same key,
+// then warp 0 takes the top-k of the 8 k candidates: every expert of the
+// token's top-k is in its own warp's top-k, so the ids, their order and the
+// weights equal those of route_kernel.
+template <int NPT>
+__global__ void __launch_bounds__(256) route_block_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                          float L, const int32_t* __restrict__ table,
+                                                          int32_t* __restrict__ ids, float* __restrict__ wout) {
+  __shared__ float s_red[8];
+  __shared__ float s_cu[8 * 32], s_cl[8 * 32], s_cw[8 * 32];
+  __shared__ int s_ce[8 * 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t = blockIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
+  if (t >= T) return;
+  const float* l = logits + (size_t)t * E;
+  float lv[NPT], u[NPT], up[NPT];
+  float lmax = -FLT_MAX;
+#pragma unroll
+  for (int m = 0; m < NPT; ++m) {
+    const int e = tid + 256 * m;
+    lv[m] = e < E ? l[e] : -FLT_MAX;
+    lmax = fmaxf(lmax, lv[m]);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+  if (lane == 0) s_red[warp] = lmax;
+  __syncthreads();
+  lmax = s_red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) lmax = fmaxf(lmax, s_red[w]);
+#pragma unroll
+  for (int m = 0; m < NPT; ++m) {
+    const int e = tid + 256 * m;
+    u[m] = e < E ? route_exp(__fsub_rn(lv[m], lmax)) : -1.0f;
+    up[m] = u[m];
+  }
+  if (L > 0.0f && table != nullptr) {
+    float umin = FLT_MAX;
+#pragma unroll
+    for (int m = 0; m < NPT; ++m)
+      if (tid + 256 * m < E) umin = fminf(umin, u[m]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) umin = fminf(umin, __shfl_xor_sync(0xffffffffu, umin, o));
+    __syncthreads();  // every warp has read s_red
+    if (lane == 0) s_red[warp] = umin;
+    __syncthreads();
+    umin = s_red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) umin = fminf(umin, s_red[w]);
+    const float boost = __fmul_rn(L, __fsub_rn(1.0f, umin));
+#pragma unroll
+    for (int m = 0; m < NPT; ++m) {
+      const int e = tid + 256 * m;
+      if (e < E && table[e] >= 0) up[m] = __fadd_rn(u[m], boost);
+    }
+  }
+  // this warp's top-k -> candidates [warp][j]
+  uint32_t taken = 0;
+  for (int j = 0; j < k; ++j) {
+    float bu = -FLT_MAX, bl = -FLT_MAX, bw = 0.0f;
+    int be = INT_MAX;
+#pragma unroll
+    for (int m = 0; m < NPT; ++m) {
+      const int e = tid + 256 * m;
+      if (e < E && !((taken >> m) & 1u) && key_better(up[m], lv[m], e, bu, bl, be)) {
+        bu = up[m];
+        bl = lv[m];
+        be = e;
+        bw = u[m];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float ou = __shfl_xor_sync(0xffffffffu, bu, o);
+      const float ol = __shfl_xor_sync(0xffffffffu, bl, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      const float ow = __shfl_xor_sync(0xffffffffu, bw, o);
+      if (key_better(ou, ol, oe, bu, bl, be)) {
+        bu = ou;
+        bl = ol;
+        be = oe;
+        bw = ow;
+      }
+    }
+    if (be != INT_MAX && (be & 255) == tid) taken |= 1u << (be >> 8);
+    if (lane == 0) {
+      s_cu[warp * 32 + j] = bu;
+      s_cl[warp * 32 + j] = bl;
+      s_ce[warp * 32 + j] = be;
+      s_cw[warp * 32 + j] = bw;
+    }
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  // top-k of the 8 k candidates; lane holds candidates c = lane + 32 q
+  constexpr int kQ = 8;  // 8 warps x at most 32 candidates / 32 lanes
+  float cu[kQ], cl[kQ], cw[kQ];
+  int ce[kQ];
+#pragma unroll
+  for (int q = 0; q < kQ; ++q) {
+    const int c = lane + 32 * q, w = c / 32, j = c % 32;  // candidate j of warp w (c = 32 w + j)
+    const bool ok = j < k;
+    cu[q] = ok ? s_cu[w * 32 + j] : -FLT_MAX;
+    cl[q] = ok ? s_cl[w * 32 + j] : -FLT_MAX;
+    ce[q] = ok ? s_ce[w * 32 + j] : INT_MAX;
+    cw[q] = ok ? s_cw[w * 32 + j] : 0.0f;
+  }
+  uint32_t tk = 0;
+  int my_e = 0;
+  float my_u = 0.0f;
+  for (int j = 0; j < k; ++j) {
+    float bu = -FLT_MAX, bl = -FLT_MAX, bw = 0.0f;
+    int be = INT_MAX, bq = -1;
+#pragma unroll
+    for (int q = 0; q < kQ; ++q)
+      if (!((tk >> q) & 1u) && ce[q] != INT_MAX && key_better(cu[q], cl[q], ce[q], bu, bl, be)) {
+        bu = cu[q];
+        bl = cl[q];
+        be = ce[q];
+        bw = cw[q];
+        bq = q;
+      }
+    int bsrc = bq >= 0 ? 32 * bq + lane : -1;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float ou = __shfl_xor_sync(0xffffffffu, bu, o);
+      const float ol = __shfl_xor_sync(0xffffffffu, bl, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      const float ow = __shfl_xor_sync(0xffffffffu, bw, o);
+      const int os = __shfl_xor_sync(0xffffffffu, bsrc, o);
+      if (key_better(ou, ol, oe, bu, bl, be)) {
+        bu = ou;
+        bl = ol;
+        be = oe;
+        bw = ow;
+        bsrc = os;
+      }
+    }
+    if (bsrc >= 0 && (bsrc & 31) == lane) tk |= 1u << (bsrc >> 5);
+    if (lane == j) {
+      my_e = be;
+      my_u = bw;
+    }
+  }
+  float s = lane < k ? my_u : 0.0f;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
+  if (lane < k) {
+    ids[(size_t)t * k + lane] = my_e;
+    wout[(size_t)t * k + lane] = __fdiv_rn(my_u, s);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // moe_sort
 // ---------------------------------------------------------------------------
@@ -315,6 +471,12 @@ __global__ void __launch_bounds__(1024) lookup_kernel(const int32_t* __restrict_
 // ---------------------------------------------------------------------------
 cudaError_t launch_route(const float* logits, int T, int E, int k, float L, const int32_t* table, int32_t* ids,
                          float* w, cudaStream_t st) {
+  if (T <= kRouteBlockMaxTokens && E <= 1024) {  // decode sizes: a block per token
+    const void* kb = E <= 256 ? reinterpret_cast<const void*>(route_block_kernel<1>)
+                     : E <= 512 ? reinterpret_cast<const void*>(route_block_kernel<2>)
+                                : reinterpret_cast<const void*>(route_block_kernel<4>);
+    return launch_pdl(kb, T, 256, 0, st, logits, T, E, k, L, table, ids, w);
+  }
   const int blocks = (T + 7) / 8;
   const void* kern = E <= 32    ? reinterpret_cast<const void*>(route_kernel<1>)
                      : E <= 128 ? reinterpret_cast<const void*>(route_kernel<4>)
