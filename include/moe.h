@@ -354,7 +354,14 @@ typedef struct {
  *   moe_slot_lookup, copy n_active/active to meta_host, synchronise `stream`,
  *   moe_cache_step, moe_install_slots on `side`, upload the table, record
  *   `installed` on `side` and make `stream` wait on it -> one pass of
- *   moe_expert_ffn over every active expert, writing y.
+ *   moe_expert_ffn over every active expert, writing y.  When experts are
+ *   installed, the pass is split: the active list is rewritten as [experts
+ *   that were resident..., installed experts...] into b->slots (the LRU step
+ *   never evicts an expert of the step, so the resident ones keep their
+ *   slots), moe_expert_ffn over the resident ones writes y on `stream` while
+ *   the copies run on `side`, and after the wait on `installed` a second
+ *   call adds the installed experts' outputs (summation order: resident
+ *   experts, then installed, each in expert order; deterministic).
  * y: device fp32 [T, H] (overwritten).  *n_installed (host, may be NULL): the
  * number of experts installed.  Errors as the calls it makes. */
 moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc, const moe_step_buffers* b,

@@ -3,7 +3,9 @@
 // fully resident) one small device->host copy and its synchronisation.
 //
 //   route -> sort -> [lookup -> misses to host -> LRU step -> pinned installs on
-//   the side stream + table upload -> compute stream waits] -> FFN (writes y)
+//   the side stream + table upload -> FFN of the resident experts (writes y),
+//   overlapping the copies -> compute stream waits] -> FFN (of the installed
+//   experts, adding to y; or of every expert, writing y)
 //
 // RFC "How the prototype works": each layer copies its routing to the host
 // once; misses become one host-to-device copy per expert; when every expert
@@ -67,8 +69,36 @@ extern "C" moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const mo
                           side) != cudaSuccess)
         return MOE_ERR_CUDA;
       if (cudaEventRecord(installed, side) != cudaSuccess) return MOE_ERR_CUDA;
-      if (cudaStreamWaitEvent(stream, installed, 0) != cudaSuccess) return MOE_ERR_CUDA;
       if (n_installed) *n_installed = n;
+      // The experts that were resident keep their slots (the LRU step never
+      // evicts an expert of the step), so their FFN runs while the copies land:
+      // the pass is reordered as [resident..., installed...] (both ascending)
+      // in the host copy's miss region, which has been read, and goes to the
+      // device slots buffer, which the lookup no longer needs.
+      int32_t* order = b->meta_host + 2 + E;
+      const int32_t* act = b->meta_host + 2;
+      int32_t nr = 0;
+      for (int32_t i = 0, m = 0; i < na; ++i) {
+        if (m < n && out_e[m] == act[i]) {
+          ++m;
+          continue;
+        }
+        order[nr++] = act[i];
+      }
+      for (int32_t i = 0; i < n; ++i) order[nr + i] = out_e[i];
+      if (cudaMemcpyAsync(b->slots, order, sizeof(int32_t) * (size_t)na, cudaMemcpyHostToDevice, stream) !=
+          cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (nr > 0) {
+        s = moe_internal_expert_ffn(x, T, d, lc->pool, lc->n_slots, lc->table_dev, b->ids, b->w, b->offsets,
+                                    b->pairs, b->slots, n_active, nullptr, 0, nr, y, b->ws, b->ws_bytes, b->dev_err,
+                                    stream, 1);
+        if (s != MOE_OK) return s;
+      }
+      if (cudaStreamWaitEvent(stream, installed, 0) != cudaSuccess) return MOE_ERR_CUDA;
+      return moe_internal_expert_ffn(x, T, d, lc->pool, lc->n_slots, lc->table_dev, b->ids, b->w, b->offsets,
+                                     b->pairs, b->slots, n_active, nullptr, nr, n, y, b->ws, b->ws_bytes,
+                                     b->dev_err, stream, nr > 0 ? 0 : 1);
     }
   }
   // one pass over every active expert, writing y (no separate zeroing)
