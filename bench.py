@@ -212,8 +212,8 @@ def ffn_graph_time(st, cfg, snaps, reps, device):
         for l in range(n_layers):
             sn = snaps[l]
             ops.moe_expert_ffn(sn["x"], T, st.layers[l].desc, st.pool_of(l), st.n_slots_of(l), st.table_dev[l],
-                               sn["ids"], sn["w"], sn["offsets"], sn["pairs"], sn["meta"][2:], sn["meta"][0:1], None,
-                               0, E, y, st.ws, st.ws_bytes, st.dev_err, cs)
+                               sn["ids"], sn["w"], sn["offsets"], sn["pairs"], sn["meta"][2:], sn["meta"][0:1],
+                               sn.get("xs"), 0, E, y, st.ws, st.ws_bytes, st.dev_err, cs)
     for _ in range(3):
         g_.replay()
     torch.cuda.synchronize(device)
@@ -441,7 +441,8 @@ def run_ours(args, rank, world, local_rank):
         for l in range(n_layers):
             st.decode_layer(l, x[steps_total, l], logits[steps_total, l], T, Lsub)
             snaps.append({"x": x[steps_total, l], "ids": st.ids.clone(), "w": st.w.clone(),
-                          "offsets": st.offsets.clone(), "pairs": st.pairs.clone(), "meta": st.meta.clone()})
+                          "offsets": st.offsets.clone(), "pairs": st.pairs.clone(), "meta": st.meta.clone(),
+                          **({"xs": st.x_sorted[:T * k].clone()} if T >= 32 else {})})
         torch.cuda.synchronize(device)
         n_unique = sum(int(sn["meta"][0].item()) for sn in snaps) / n_layers
         ffn_us = ffn_graph_time(st, cfg, snaps, args.ffn_reps, device)
@@ -536,6 +537,8 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": recorded_traffic("ffn_fused_kernel") if T * k <= 64 and T <= 8 else None,
                      "kernel": ("ffn_fused_kernel (one launch per layer: gate/up + SwiGLU, grid barrier, down + "
                                 "combine)" if T <= 8 and T * k <= 64 else
+                                "pf_gemm_kernel (tcgen05 grouped GEMM: gate/up + SwiGLU, down) + combine, per layer"
+                                if T >= 32 else
                                 "moe_expert_ffn (gate/up+SwiGLU kernel + down kernel), per layer"),
                      "bytes_per_launch": int(ffn_bytes), "peak_kind": peak_kind},
         "gpu_launches": launches,

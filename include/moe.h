@@ -198,8 +198,8 @@ moe_status moe_install_slots(void* pool, size_t slot_bytes, int32_t n_slots, con
  *   n_slots    slots in the pool
  *   slot_table device int32 [E]
  *   ids, w     from moe_route; offsets, pairs, active, n_active from moe_sort
- *   x_sorted   from moe_sort, or NULL (needed by the tensor-core prefill path
- *              when T >= 256; else unused)
+ *   x_sorted   from moe_sort, or NULL (needed by the tensor-core grouped GEMM,
+ *              which runs from 32 tokens when it is given; else unused)
  *   pass_begin, pass_len  which active experts this call runs
  *   y_accum    device fp32 [T, H]; the pass's expert outputs are ADDED:
  *              y_t += sum over the pass's pairs (t, j) of w[t,j] * o_{t,j}.
@@ -223,8 +223,11 @@ moe_status moe_expert_ffn(const uint16_t* x, int32_t T, const moe_layer_desc* d,
  * The scratch is one fixed device array of moe_noalloc_scratch_bytes() bytes
  * (1 MiB) inside the library, held by every GPU that loads it until the
  * process exits.  Same arguments and results as moe_expert_ffn, except:
- *   - T must be <= 64 and moe_workspace_bytes(d, T) <= 1 MiB, else
- *     MOE_ERR_CAPACITY is returned and nothing is launched;
+ *   - T must be <= 64 and the workspace of a call without x_sorted must fit
+ *     1 MiB (that is moe_workspace_bytes(d, T) below 32 tokens; from 32 on,
+ *     moe_workspace_bytes also counts the tensor-core path's per-pair output
+ *     buffer, which this call never uses), else MOE_ERR_CAPACITY is returned
+ *     and nothing is launched;
  *   - x_sorted is not taken (the decode kernels do not use it);
  *   - the first call on a device looks up the array's device address (with
  *     that device current); make that first call outside any stream capture;
@@ -273,8 +276,9 @@ const char* moe_status_string(moe_status s);
  *                          combine (T <= 8, T*k <= 64, H/16 <= SM count)
  *   MOE_PATH_GEMV          gate/up + SwiGLU kernel, down kernel (+ combine
  *                          kernel for T > 64): tensor-core GEMV (mma.sync)
- *   MOE_PATH_TC_PREFILL    tcgen05/TMEM grouped GEMM fed by TMA (T >= 256,
- *                          x_sorted given, H and I multiples of 128)
+ *   MOE_PATH_TC_PREFILL    tcgen05/TMEM grouped GEMM fed by TMA (T >= 32,
+ *                          x_sorted given, H and I multiples of 128): prefill
+ *                          chunks and batched decode
  * or -1 if d is invalid or T < 1.  Host only; no device work. */
 enum { MOE_PATH_FUSED_DECODE = 0, MOE_PATH_GEMV = 1, MOE_PATH_TC_PREFILL = 2 };
 int32_t moe_ffn_kernel_path(const moe_layer_desc* d, int32_t T, int32_t has_x_sorted);
@@ -334,6 +338,8 @@ typedef struct {
   void* ws;            /* device workspace */
   size_t ws_bytes;     /* >= moe_workspace_bytes(desc, max_tokens) */
   int32_t max_tokens;
+  uint16_t* x_sorted;  /* device bf16 [max_tokens*k, H], or NULL: from 32 tokens the layer
+                          sorts x into it and its FFN runs on the tensor-core grouped GEMM */
 } moe_step_buffers;
 
 /* One layer's slot pool and tables. */
@@ -350,7 +356,8 @@ typedef struct {
 /* One decode layer, T <= 64 tokens (RFC "How the prototype works": each layer
  * copies its routing to the host once; misses cost one host-to-device copy
  * per expert; a fully resident layer never synchronises with the host):
- *   moe_route (L) -> moe_sort -> if the layer is not fully resident in `cache`:
+ *   moe_route (L) -> moe_sort (sorting x into b->x_sorted when T >= 32 and
+ *   b->x_sorted is given) -> if the layer is not fully resident in `cache`:
  *   moe_slot_lookup, copy n_active/active to meta_host, synchronise `stream`,
  *   moe_cache_step, moe_install_slots on `side`, upload the table, record
  *   `installed` on `side` and make `stream` wait on it -> one pass of

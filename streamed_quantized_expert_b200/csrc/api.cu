@@ -53,14 +53,17 @@ struct WsCarve {
   size_t sort, hb, h, o, total;
 };
 
-WsCarve carve(const moe_layer_desc& d, int T) {
+// tc: the call may run the tensor-core path (x_sorted given), whose per-pair
+// outputs need o from kTcMinTokens tokens; without it o is needed above 64.
+WsCarve carve(const moe_layer_desc& d, int T, bool tc = true) {
   WsCarve c{};
   const int64_t np = (int64_t)T * d.k;
   c.sort = (size_t)round_up((int64_t)sort_ws_bytes((int)np, d.E), 256);
   // h (bf16, rows padded to 128-blocks) and its per-8-column partial sums
   c.hb = (size_t)round_up(np * padded_k(d.I) * 2, 256);
   c.h = c.hb + (size_t)round_up(np * padded_k(d.I), 256);
-  c.o = T > kFusedMaxTokens ? (size_t)round_up(np * d.H * 4, 256) : 0;
+  // o: per-pair outputs of the tensor-core path (T >= kTcMinTokens) and of the GEMV path for T > 64
+  c.o = ((tc && T >= kTcMinTokens) || T > kFusedMaxTokens) ? (size_t)round_up(np * d.H * 4, 256) : 0;
   const size_t ffn = c.h + c.o;
   c.total = kWsControlBytes + (c.sort > ffn ? c.sort : ffn);
   return c;
@@ -111,6 +114,13 @@ moe_status moe_slot_layout(const moe_layer_desc* d, moe_slot_layout_t* out) {
 size_t moe_workspace_bytes(const moe_layer_desc* d, int32_t max_tokens) {
   if (check_desc(d) != MOE_OK || max_tokens < 0) return 0;
   return carve(*d, max_tokens).total;
+}
+
+// Workspace bytes of a call that passes no x_sorted (the GEMV / fused kernels).
+__attribute__((visibility("hidden"))) size_t moe_internal_workspace_bytes_no_tc(const moe_layer_desc* d,
+                                                                               int32_t max_tokens) {
+  if (check_desc(d) != MOE_OK || max_tokens < 0) return 0;
+  return carve(*d, max_tokens, false).total;
 }
 
 moe_status moe_route(const float* logits, int32_t T, const moe_layer_desc* d, float L, const int32_t* slot_table,
@@ -181,7 +191,7 @@ __attribute__((visibility("hidden"))) moe_status moe_internal_expert_ffn(
   if (!aligned(pool, 256) || !aligned(x, 16) || !aligned(ws, 256)) return MOE_ERR_INVALID;
   if ((int64_t)T * d->k > (1 << 24)) return MOE_ERR_UNSUPPORTED;
   if (!ffn_decode_supported(*d)) return MOE_ERR_UNSUPPORTED;
-  const WsCarve c = carve(*d, T);
+  const WsCarve c = carve(*d, T, x_sorted != nullptr);
   if (!ws || ws_bytes < c.total) return MOE_ERR_CAPACITY;
   FfnArgs a{};
   a.x = x;

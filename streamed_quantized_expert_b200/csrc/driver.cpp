@@ -40,7 +40,10 @@ extern "C" moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const mo
   int32_t* miss = b->meta + 2 + E;
   moe_status s = moe_route(logits, T, d, L, lc->table_dev, b->ids, b->w, stream);
   if (s != MOE_OK) return s;
-  s = moe_sort(b->ids, nullptr, T, d, b->offsets, b->pairs, active, n_active, nullptr, b->ws, b->ws_bytes, stream);
+  // from 32 tokens the FFN runs on the tensor-core grouped GEMM, which reads x sorted by expert
+  uint16_t* xs = (T >= 32 && b->x_sorted) ? b->x_sorted : nullptr;
+  s = moe_sort(b->ids, xs ? x : nullptr, T, d, b->offsets, b->pairs, active, n_active, xs, b->ws, b->ws_bytes,
+               stream);
   if (s != MOE_OK) return s;
   if (moe_cache_resident(cache, layer) < E) {
     s = moe_slot_lookup(lc->table_dev, active, n_active, 0, E, lc->n_slots, b->slots, miss, n_miss, b->dev_err,
@@ -91,17 +94,17 @@ extern "C" moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const mo
         return MOE_ERR_CUDA;
       if (nr > 0) {
         s = moe_internal_expert_ffn(x, T, d, lc->pool, lc->n_slots, lc->table_dev, b->ids, b->w, b->offsets,
-                                    b->pairs, b->slots, n_active, nullptr, 0, nr, y, b->ws, b->ws_bytes, b->dev_err,
+                                    b->pairs, b->slots, n_active, xs, 0, nr, y, b->ws, b->ws_bytes, b->dev_err,
                                     stream, 1);
         if (s != MOE_OK) return s;
       }
       if (cudaStreamWaitEvent(stream, installed, 0) != cudaSuccess) return MOE_ERR_CUDA;
       return moe_internal_expert_ffn(x, T, d, lc->pool, lc->n_slots, lc->table_dev, b->ids, b->w, b->offsets,
-                                     b->pairs, b->slots, n_active, nullptr, nr, n, y, b->ws, b->ws_bytes,
+                                     b->pairs, b->slots, n_active, xs, nr, n, y, b->ws, b->ws_bytes,
                                      b->dev_err, stream, nr > 0 ? 0 : 1);
     }
   }
   // one pass over every active expert, writing y (no separate zeroing)
   return moe_internal_expert_ffn(x, T, d, lc->pool, lc->n_slots, lc->table_dev, b->ids, b->w, b->offsets, b->pairs,
-                                 active, n_active, nullptr, 0, E, y, b->ws, b->ws_bytes, b->dev_err, stream, 1);
+                                 active, n_active, xs, 0, E, y, b->ws, b->ws_bytes, b->dev_err, stream, 1);
 }

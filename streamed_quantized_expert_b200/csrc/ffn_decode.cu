@@ -543,7 +543,7 @@ int ffn_kernel_path(const moe_layer_desc& d, int T, bool has_x_sorted, int num_s
   a.ctl = &ctl_stub;  // the plan only checks that a control block exists
   size_t smem = 0;
   if (ffn_fused_plan(a, d, num_sms, smem)) return 0;
-  if (T >= kPrefillTcMinTokens && has_x_sorted && ffn_prefill_tc_shape_ok(d)) return 2;
+  if (T >= kTcMinTokens && has_x_sorted && ffn_prefill_tc_shape_ok(d)) return 2;
   return 1;
 }
 
@@ -574,7 +574,7 @@ cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, c
   a.ng_d = L.ng_d;
   a.nblk_gu = L.nblk_gu;
   a.nblk_d = L.nblk_d;
-  if (a.T >= kPrefillTcMinTokens) {  // tensor-core grouped GEMM (needs x_sorted)
+  if (a.T >= kTcMinTokens) {  // tensor-core grouped GEMM (needs x_sorted)
     const cudaError_t e = launch_ffn_prefill_tc(a, d, num_sms, st);
     if (e != cudaErrorNotSupported) return e;
   }

@@ -10,7 +10,7 @@
 namespace moe {
 
 constexpr int kFusedMaxTokens = 64;  // decode down kernel combines in shared memory up to this T
-constexpr int kPrefillTcMinTokens = 256;  // from this T on, prefill runs on the tcgen05 grouped GEMM
+constexpr int kTcMinTokens = 32;  // from this T on (with x_sorted) the FFN runs on the tcgen05 grouped GEMM
 constexpr int kRouteBlockMaxTokens = 64;  // up to this T, routing takes a block (8 warps) per token
 
 struct FfnArgs {

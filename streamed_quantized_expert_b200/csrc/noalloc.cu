@@ -37,6 +37,8 @@ moe_status scratch_of_current_device(void** out) {
 
 }  // namespace
 
+extern "C" size_t moe_internal_workspace_bytes_no_tc(const moe_layer_desc* d, int32_t max_tokens);
+
 extern "C" size_t moe_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 extern "C" moe_status moe_expert_ffn_noalloc(const uint16_t* x, int32_t T, const moe_layer_desc* d,
@@ -45,7 +47,7 @@ extern "C" moe_status moe_expert_ffn_noalloc(const uint16_t* x, int32_t T, const
                                              const int32_t* pairs, const int32_t* active, const int32_t* n_active,
                                              int32_t pass_begin, int32_t pass_len, float* y_accum,
                                              int32_t* dev_err, cudaStream_t stream) {
-  const size_t need = moe_workspace_bytes(d, T);
+  const size_t need = moe_internal_workspace_bytes_no_tc(d, T);  // no x_sorted is passed below
   if (need == 0 || T < 0) return MOE_ERR_INVALID;
   if (T > moe::kFusedMaxTokens || need > kNoAllocScratchBytes) return MOE_ERR_CAPACITY;
   void* scratch = nullptr;

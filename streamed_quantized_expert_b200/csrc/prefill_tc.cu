@@ -656,16 +656,24 @@ cudaError_t launch_ffn_prefill_tc(const FfnArgs& a, const moe_layer_desc& d, int
   pa.o = a.o;
   pa.dev_err = a.dev_err;
   const int grid = num_sms;
-  pa.K = d.H;
-  pa.nkb = L.nblk_gu;
-  pa.mtiles = 2 * d.I / kPfBM;
-  cudaError_t e = launch_pf<true>(d.bits_gu, gpb, q_gu, sb_gu, xm, pa, grid, st);
-  if (e != cudaSuccess) return e;
-  pa.K = d.I;
-  pa.nkb = L.nblk_d;
-  pa.mtiles = d.H / kPfBM;
-  e = launch_pf<false>(d.bits_down, gpb, q_d, sb_d, hm, pa, grid, st);
-  if (e != cudaSuccess) return e;
+  // a CTA's tile table holds kMaxCtaExperts experts: longer passes run as
+  // several gate/up + down launches over consecutive sub-ranges (sub-ranges
+  // past the active list find no experts), then one combine over the pass
+  const int pass_end = a.pass_len < d.E - a.pass_begin ? a.pass_begin + a.pass_len : d.E;
+  for (int pb = a.pass_begin; pb < pass_end; pb += kMaxCtaExperts) {
+    pa.pass_begin = pb;
+    pa.pass_len = pass_end - pb < kMaxCtaExperts ? pass_end - pb : kMaxCtaExperts;
+    pa.K = d.H;
+    pa.nkb = L.nblk_gu;
+    pa.mtiles = 2 * d.I / kPfBM;
+    cudaError_t e = launch_pf<true>(d.bits_gu, gpb, q_gu, sb_gu, xm, pa, grid, st);
+    if (e != cudaSuccess) return e;
+    pa.K = d.I;
+    pa.nkb = L.nblk_d;
+    pa.mtiles = d.H / kPfBM;
+    e = launch_pf<false>(d.bits_down, gpb, q_d, sb_d, hm, pa, grid, st);
+    if (e != cudaSuccess) return e;
+  }
   return launch_pdl(reinterpret_cast<const void*>(combine_kernel), combine_grid(a.T, d.H, num_sms), 256, 0, st, a);
 }
 

@@ -47,7 +47,8 @@ class LayerDesc(C.Structure):
 class StepBuffers(C.Structure):
     _fields_ = [("ids", C.c_void_p), ("w", C.c_void_p), ("offsets", C.c_void_p), ("pairs", C.c_void_p),
                 ("meta", C.c_void_p), ("meta_host", C.c_void_p), ("slots", C.c_void_p), ("dev_err", C.c_void_p),
-                ("ws", C.c_void_p), ("ws_bytes", C.c_size_t), ("max_tokens", C.c_int32)]
+                ("ws", C.c_void_p), ("ws_bytes", C.c_size_t), ("max_tokens", C.c_int32),
+                ("x_sorted", C.c_void_p)]
 
 
 class LayerCtx(C.Structure):

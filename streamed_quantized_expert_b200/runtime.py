@@ -103,10 +103,13 @@ class Streamer:
         self.launches = 0          # libmoe kernel launches issued (for reporting)
         # native per-layer driver state
         self.installed.record(self.side)  # materialise the event
+        if max_tokens >= 32:  # batched decode sorts x for the tensor-core grouped GEMM
+            self.x_sorted = torch.empty((max_tokens * self.k, self.H), dtype=torch.uint16, device=self.device)
         self._bufs = ops.StepBuffers(self.ids.data_ptr(), self.w.data_ptr(), self.offsets.data_ptr(),
                                      self.pairs.data_ptr(), self.meta.data_ptr(), self.meta_pin.data_ptr(),
                                      self.slots.data_ptr(), self.dev_err.data_ptr(), self.ws.data_ptr(),
-                                     self.ws_bytes, max_tokens)
+                                     self.ws_bytes, max_tokens,
+                                     self.x_sorted.data_ptr() if self.x_sorted is not None else None)
         self._ctx = []
         self._rows = []
         for l, spec in enumerate(layers):
@@ -205,7 +208,7 @@ class Streamer:
         self.launches += 2 if T <= 64 else 3
         ops.moe_expert_ffn(x, T, d, self.pool_of(layer), self.n_slots_of(layer), self.table_dev[layer], self.ids,
                            self.w, self.offsets, self.pairs, self._active(), self._n_active(),
-                           self.x_sorted if T >= 256 else None, pass_begin, pass_len, y, self.ws, self.ws_bytes,
+                           self.x_sorted if T >= 32 else None, pass_begin, pass_len, y, self.ws, self.ws_bytes,
                            self.dev_err, self.stream)
         if ev is not None:
             ev[1].record(self.stream)
@@ -250,7 +253,7 @@ class Streamer:
         """One prefill chunk: passes of <= 64 active experts; returns y."""
         y = self.y[:T] if y is None else y
         s = self.stream
-        self.route_sort(layer, x, logits, T, 0.0, want_sorted_x=T >= 256)
+        self.route_sort(layer, x, logits, T, 0.0, want_sorted_x=T >= 32)
         with torch.cuda.stream(s):
             y.zero_()
             self.meta_pin.copy_(self.meta, non_blocking=True)

@@ -1,5 +1,5 @@
-"""GPU vs oracle for the prefill expert FFN on the tcgen05 grouped GEMM
-(T >= 256 tokens with sorted activations): dequantised weight tiles in the
+"""GPU vs oracle for the expert FFN on the tcgen05 grouped GEMM (prefill
+chunks and batched decode, from 32 tokens with sorted activations): dequantised weight tiles in the
 128-byte swizzled layout, token tiles by TMA, fp32 accumulators in TMEM.
 Within 2e-2 of max(|ref|, row rms) elementwise on sampled token rows (the
 oracle computes them one by one), and equal to the GEMV path within the
@@ -82,3 +82,12 @@ def test_non_resident_expert_flagged_on_tc_path(orc):
     # the expert is skipped: token rows that never routed to it are unaffected
     keep = np.array([t for t in range(320) if gone not in ids[t]][:4])
     assert_close(y[keep], s.oracle(orc, x, ids, w, keep), TOL)
+
+
+@pytest.mark.parametrize("T", [32, 64])
+def test_coder_batched_decode_on_tensor_cores(orc, T):
+    # batched decode (Coder-like: 128 experts, top-8, H 2048, I 768, 4-bit g64) with sorted x
+    # takes the tensor-core path from 32 tokens, one call over every expert (split into
+    # launches of 64 experts inside the library)
+    s, x, ids, w = _case(orc, 128, 8, 2048, 768, 64, 4, 4, T, R=6, seed=16 + T)
+    _check(orc, s, x, ids, w, T, passes=[(0, 128)], ntok=4)
