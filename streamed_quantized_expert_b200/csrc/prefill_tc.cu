@@ -1,8 +1,10 @@
-// Prefill expert FFN on the 5th-generation tensor cores (tcgen05 + TMEM),
-// fed by TMA: the grouped GEMM of a pass's experts over their sorted tokens.
+// Expert FFN on the 5th-generation tensor cores (tcgen05 + TMEM), fed by TMA:
+// the grouped GEMM of a pass's experts over their sorted tokens, for prefill
+// chunks and batched decode (from 32 tokens, when x sorted by expert is given).
 //
-// Two launches per pass, one persistent CTA per SM, each looping over tiles
-// of (expert, 128 weight rows, up to 128 tokens):
+// Two launches per pass of at most 64 experts (a longer pass runs as several),
+// one persistent CTA per SM, each looping over tiles of (expert, 128 weight
+// rows, up to 128 tokens):
 //   gate/up: GU[rows, tokens] = deq(W_gu[e])[rows, H] . X_sorted[tokens, H]^T,
 //            then h[token][j] = silu(gate_j) * up_j (bf16), j = intermediate;
 //   down:    O[rows, tokens]  = deq(W_d[e])[rows, I] . h[tokens, I]^T,
