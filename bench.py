@@ -30,6 +30,18 @@ sys.path.insert(0, ROOT)
 METRIC = "expert-FFN HBM GB/s & decode tok/s-equiv; prefill TFLOP/s; % of B200 roofline"
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of `values` over the default process group (the
+    values themselves without one): every rank gets the slowest rank's times."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def recorded_traffic(kernel):
     """DRAM bytes per launch of `kernel` from the ncu capture recorded in
     profiles/traffic.txt, or None when the kernel's sources changed since."""
@@ -318,10 +330,7 @@ def run_prefill(args, rank, world, local_rank):
         torch.cuda.synchronize(device)
     ffn_ms = f0.elapsed_time(f1) / args.ffn_reps  # all layers
     del g_
-    t = torch.tensor([ffn_ms, whole_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ffn_ms, whole_ms = float(t[0].item()), float(t[1].item())
+    ffn_ms, whole_ms = max_over_ranks([ffn_ms, whole_ms], device)
     err = st.check_dev_err()
 
     # e2e: x and logits from pinned host memory, y of every layer read back
@@ -446,10 +455,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(device)
         n_unique = sum(int(sn["meta"][0].item()) for sn in snaps) / n_layers
         ffn_us = ffn_graph_time(st, cfg, snaps, args.ffn_reps, device)
-    t = torch.tensor([ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks([ms], device)[0]
     err = st.check_dev_err()
     miss_no_sub = None
     if Lsub > 0:  # the same token sequence from the same initial cache, without substitution (untimed)
@@ -486,10 +492,7 @@ def run_ours(args, rank, world, local_rank):
     f1.record(s)
     torch.cuda.synchronize(device)
     e2e_ms = f0.elapsed_time(f1)
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms_max = float(t.item())
+    e2e_ms_max = max_over_ranks([e2e_ms], device)[0]
 
     if rank != 0:
         return None

@@ -94,3 +94,19 @@ def test_slot_cache_capacity(lib):
     c = ops.SlotCache(10, 1, 2)
     st, inst = c.step(0, [1, 2, 3])
     assert st == ops.MOE_ERR_CAPACITY and inst[-1] == (3, -1)
+
+
+def test_kernel_path_choice_and_workspace_growth(lib):
+    # host-only decisions: the fused single-launch decode up to T*k <= 64 (T <= 8), the GEMV kernels
+    # without sorted x, -1 for an invalid shape; the workspace counts the per-pair output buffer of the
+    # tensor-core path from 32 tokens on
+    d = ops.desc(512, 10, 2048, 512, 64, 3, 3)
+    assert ops.moe_ffn_kernel_path(d, 1, False) == ops.MOE_PATH_FUSED_DECODE
+    assert ops.moe_ffn_kernel_path(d, 6, False) == ops.MOE_PATH_FUSED_DECODE
+    assert ops.moe_ffn_kernel_path(d, 7, False) == ops.MOE_PATH_GEMV  # 70 pairs > 64
+    assert ops.moe_ffn_kernel_path(d, 300, False) == ops.MOE_PATH_GEMV
+    assert ops.moe_ffn_kernel_path(d, 0, False) == -1
+    assert ops.moe_ffn_kernel_path(ops.desc(8, 2, 64, 32, 48, 4, 4), 4, False) == -1  # group 48
+    per_pair_o = 10 * 2048 * 4
+    w31, w32 = ops.moe_workspace_bytes(d, 31), ops.moe_workspace_bytes(d, 32)
+    assert w32 - w31 >= 32 * per_pair_o
