@@ -87,6 +87,8 @@ CONFIGS = {
                      "gate/up, 6-bit down on layers l % 4 == 0 (2 slot size classes), 1 token/step, 128 slots/layer "
                      "(25% resident), L = 0.15, misses installed from pinned host"),
 }
+# token counts of a configuration's batch sweep (besides its own T), FFN-only
+SWEEP = {"coder": (1, 8, 32)}
 # per-layer widths and the substitution strength of the decode configurations (default: uniform, L = 0)
 DECODE_EXTRA = {"decode_mixed": {"bits": lambda l: (4, 6) if l % 4 == 0 else (4, 4), "L": 0.15}}
 
@@ -206,15 +208,16 @@ def make_inputs(cfg, seed, n_steps, device, pinned=False, step0=0):
     return x.to(device), logits.to(device)
 
 
-def ffn_graph_time(st, cfg, snaps, reps, device):
+def ffn_graph_time(st, cfg, snaps, reps, device, T=None):
     """Time the FFN alone: a CUDA graph of the 48 layers' moe_expert_ffn calls
-    (each with its layer's routing from one decode step), replayed `reps`
-    times; returns microseconds per layer."""
+    (each with its layer's routing from one decode step of T tokens, default
+    the configuration's), replayed `reps` times; returns microseconds per layer."""
     import torch
 
     from streamed_quantized_expert_b200 import ops
 
-    n_layers, E, k, H, I, g, bg, bd, T, S, _ = cfg
+    n_layers, E, k, H, I, g, bg, bd, T0, S, _ = cfg
+    T = T0 if T is None else T
     y = torch.zeros((T, H), dtype=torch.float32, device=device)
     g_ = torch.cuda.CUDAGraph()
     cap = torch.cuda.Stream(device)
@@ -455,6 +458,18 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(device)
         n_unique = sum(int(sn["meta"][0].item()) for sn in snaps) / n_layers
         ffn_us = ffn_graph_time(st, cfg, snaps, args.ffn_reps, device)
+        # batch sweep (configurations that name one): the same step's first T2 tokens through every layer
+        sweep = []
+        for T2 in SWEEP.get(args.config, ()):
+            sn2 = []
+            for l in range(n_layers):
+                st.decode_layer(l, x[steps_total, l, :T2], logits[steps_total, l, :T2], T2, Lsub)
+                sn2.append({"x": x[steps_total, l, :T2], "ids": st.ids.clone(), "w": st.w.clone(),
+                            "offsets": st.offsets.clone(), "pairs": st.pairs.clone(), "meta": st.meta.clone(),
+                            **({"xs": st.x_sorted[:T2 * k].clone()} if T2 >= 32 else {})})
+            torch.cuda.synchronize(device)
+            us2 = ffn_graph_time(st, cfg, sn2, args.ffn_reps, device, T=T2)
+            sweep.append((T2, us2, sn2))
     ms_max = max_over_ranks([ms], device)[0]
     err = st.check_dev_err()
     miss_no_sub = None
@@ -544,6 +559,17 @@ def run_ours(args, rank, world, local_rank):
                                 if T >= 32 else
                                 "moe_expert_ffn (gate/up+SwiGLU kernel + down kernel), per layer"),
                      "bytes_per_launch": int(ffn_bytes), "peak_kind": peak_kind},
+        **({"batch_sweep": [
+            {"tokens": T2, "us_per_layer": round(us2, 2),
+             "hbm_gbs": round(b2 / (us2 * 1e-6) / 1e9, 1), "frac": round(b2 / (us2 * 1e-6) / 1e9 / hbm_peak, 4),
+             "unique_experts_per_layer": round(nu2, 1),
+             "kernel_path": ["fused decode", "GEMV", "tcgen05 grouped GEMM"][
+                 _ops.moe_ffn_kernel_path(st.layers[0].desc, T2, T2 >= 32)]}
+            for T2, us2, nu2, b2 in [
+                (T2, us2, sum(int(sn["meta"][0].item()) for sn in sn2) / n_layers,
+                 sum(int(sn["meta"][0].item()) * slot_bytes[l] for l, sn in enumerate(sn2)) / n_layers
+                 + T2 * H * 6)
+                for T2, us2, sn2 in sweep + [(T, ffn_us, snaps)]]]} if sweep else {}),
         "gpu_launches": launches,
         "dev_err": err,
         "clocks": clk.summary(),
