@@ -233,14 +233,16 @@ __global__ void __launch_bounds__(256) route_block_kernel(const float* __restric
   }
   __syncthreads();
   if (warp != 0) return;
-  // top-k of the 8 k candidates; lane holds candidates c = lane + 32 q
+  // top-k of the 8 k candidates, packed: candidate c = k w + j (j-th of warp w) sits at lane c % 32,
+  // register c / 32 (at most 8 k / 32 registers hold candidates)
   constexpr int kQ = 8;  // 8 warps x at most 32 candidates / 32 lanes
+  const int nq = (8 * k + 31) / 32;
   float cu[kQ], cl[kQ], cw[kQ];
   int ce[kQ];
 #pragma unroll
   for (int q = 0; q < kQ; ++q) {
-    const int c = lane + 32 * q, w = c / 32, j = c % 32;  // candidate j of warp w (c = 32 w + j)
-    const bool ok = j < k;
+    const int c = lane + 32 * q, w = c / k, j = c - w * k;
+    const bool ok = c < 8 * k;
     cu[q] = ok ? s_cu[w * 32 + j] : -FLT_MAX;
     cl[q] = ok ? s_cl[w * 32 + j] : -FLT_MAX;
     ce[q] = ok ? s_ce[w * 32 + j] : INT_MAX;
@@ -254,7 +256,7 @@ __global__ void __launch_bounds__(256) route_block_kernel(const float* __restric
     int be = INT_MAX, bq = -1;
 #pragma unroll
     for (int q = 0; q < kQ; ++q)
-      if (!((tk >> q) & 1u) && ce[q] != INT_MAX && key_better(cu[q], cl[q], ce[q], bu, bl, be)) {
+      if (q < nq && !((tk >> q) & 1u) && ce[q] != INT_MAX && key_better(cu[q], cl[q], ce[q], bu, bl, be)) {
         bu = cu[q];
         bl = cl[q];
         be = ce[q];
