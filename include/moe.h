@@ -131,12 +131,14 @@ moe_status moe_slot_layout(const moe_layer_desc* d, moe_slot_layout_t* out);
 
 /* Device workspace needed by moe_sort and moe_expert_ffn for up to
  * max_tokens tokens (0 if d is invalid).  One buffer of this size may be
- * shared by the two calls when they run in stream order.  Its first 256
- * bytes are a control block (the grid barrier of the single-launch decode
- * FFN, an arrival counter that every launch advances by its grid size): zero
- * them once after allocating the workspace (e.g. cudaMemset), and again after
- * a call that reported MOE_DEV_ERR_TIMEOUT.  The rest needs no
- * initialisation. */
+ * shared by the two calls when they run in stream order.  Its first 512
+ * bytes are a control block (the single-launch decode FFN's per-expert
+ * readiness counters and its down CTAs' departure count): zero them once
+ * after allocating the workspace (e.g. cudaMemset).  Every launch leaves them
+ * at zero again, also one whose waits ran out; only a launch cut short on the
+ * device (its context lost) can leave them otherwise, and a later call then
+ * reports MOE_DEV_ERR_TIMEOUT instead of using them -- zero them after a
+ * reported timeout.  The rest needs no initialisation. */
 size_t moe_workspace_bytes(const moe_layer_desc* d, int32_t max_tokens);
 
 /* Stage 1.  Cache-aware top-k (BigMoeOnEdge note: every expert already in
@@ -231,9 +233,11 @@ moe_status moe_expert_ffn(const uint16_t* x, int32_t T, const moe_layer_desc* d,
  *   - x_sorted is not taken (the decode kernels do not use it);
  *   - the first call on a device looks up the array's device address (with
  *     that device current); make that first call outside any stream capture;
- *   - every call shares the one array and leaves its contents behind; nothing
- *     in it has to start at zero, but calls whose kernels overlap on the GPU
- *     (e.g. on two streams at once) race on it.
+ *   - every call shares the one array and leaves its contents behind; the
+ *     array's first 512 bytes (the control block that moe_workspace_bytes
+ *     describes) are cleared on `stream` (cudaMemsetAsync) before each call's
+ *     kernels, the rest needs no initialisation; calls whose kernels overlap
+ *     on the GPU (e.g. on two streams at once) race on the array.
  * Allocates nothing. */
 moe_status moe_expert_ffn_noalloc(const uint16_t* x, int32_t T, const moe_layer_desc* d, const void* pool,
                                   int32_t n_slots, const int32_t* slot_table, const int32_t* ids, const float* w,
@@ -272,8 +276,9 @@ const char* moe_status_string(moe_status s);
 /* Which kernels moe_expert_ffn runs on the current device for a call over
  * all E experts of a layer of shape d with T tokens, with (has_x_sorted != 0)
  * or without x_sorted:
- *   MOE_PATH_FUSED_DECODE  one launch: gate/up + SwiGLU, grid barrier, down +
- *                          combine (T <= 8, T*k <= 64, H/16 <= SM count)
+ *   MOE_PATH_FUSED_DECODE  one launch: gate/up + SwiGLU CTAs and down +
+ *                          combine CTAs linked by per-expert readiness
+ *                          counters (T <= 8, T*k <= 64)
  *   MOE_PATH_GEMV          gate/up + SwiGLU kernel, down kernel (+ combine
  *                          kernel for T > 64): tensor-core GEMV (mma.sync)
  *   MOE_PATH_TC_PREFILL    tcgen05/TMEM grouped GEMM fed by TMA (T >= 32,
@@ -282,6 +287,15 @@ const char* moe_status_string(moe_status s);
  * or -1 if d is invalid or T < 1.  Host only; no device work. */
 enum { MOE_PATH_FUSED_DECODE = 0, MOE_PATH_GEMV = 1, MOE_PATH_TC_PREFILL = 2 };
 int32_t moe_ffn_kernel_path(const moe_layer_desc* d, int32_t T, int32_t has_x_sorted);
+
+/* Test/inspection: the limit, in SM clock cycles, of every bounded device
+ * wait (a bulk copy that should land, a pipeline stage that should free up,
+ * the single-launch decode FFN's readiness counters) in kernels launched afterwards
+ * by this process; cycles <= 0 restores the default of 4e9 (about 2 s at the
+ * top clock).  A wait that runs out sets MOE_DEV_ERR_TIMEOUT in dev_err and
+ * the kernel returns; tests lower the limit to make such a wait run out
+ * quickly.  Host only; process-wide. */
+void moe_set_wait_limit_cycles(int64_t cycles);
 
 /* Name of the last CUDA error that made a call of this thread return
  * MOE_ERR_CUDA ("no error" if none). */

@@ -1,5 +1,9 @@
 """Build libmoe.so (sm_100a) in-tree with nvcc.
 
+Every source is compiled to its own object in parallel (one nvcc per file;
+there is no device code shared across files), then linked into one shared
+library next to this file.
+
 python -m streamed_quantized_expert_b200.build   # or build() from Python
 """
 from __future__ import annotations
@@ -7,34 +11,63 @@ from __future__ import annotations
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 SO = os.path.join(HERE, "libmoe.so")
-SOURCES = ["api.cu", "route_sort.cu", "quant.cu", "ffn_decode.cu", "ffn_fused.cu", "prefill_tc.cu", "noalloc.cu", "slot_cache.cpp", "driver.cpp"]
+OBJ_DIR = os.path.join(HERE, "_build")
+SOURCES = ["api.cu", "route_sort.cu", "quant.cu", "ffn_decode.cu", "ffn_fused.cu", "prefill_tc.cu", "noalloc.cu",
+           "slot_cache.cpp", "driver.cpp"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "--extended-lambda",
-    "-Xcompiler", "-fPIC", "-shared", "-Xptxas", "-warn-spills",
+    "-Xcompiler", "-fPIC", "-Xptxas", "-warn-spills",
 ]
 
 
-def _stale() -> bool:
-    if not os.path.exists(SO):
+def _headers() -> list[str]:
+    hs = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
+    return hs + [os.path.join(INCLUDE, "moe.h"), __file__]
+
+
+def _obj(src: str) -> str:
+    return os.path.join(OBJ_DIR, src + ".o")
+
+
+def _stale(target: str, deps: list[str]) -> bool:
+    if not os.path.exists(target):
         return True
-    t = os.path.getmtime(SO)
-    deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(INCLUDE, "moe.h"), __file__]
+    t = os.path.getmtime(target)
     return any(os.path.getmtime(p) > t for p in deps)
 
 
+def _compile(src: str, verbose: bool) -> str:
+    out = _obj(src)
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = [NVCC, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", os.path.join(CSRC, src), "-o", tmp]
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    subprocess.check_call(cmd)
+    os.replace(tmp, out)
+    return out
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    hdrs = _headers()
+    todo = [s for s in SOURCES if force or _stale(_obj(s), [os.path.join(CSRC, s)] + hdrs)]
+    if todo:
+        with ThreadPoolExecutor(max_workers=max(1, min(len(todo), os.cpu_count() or 1))) as ex:
+            list(ex.map(lambda s: _compile(s, verbose), todo))
+    objs = [_obj(s) for s in SOURCES]
+    if not force and not todo and not _stale(SO, objs):
         return SO
     tmp = SO + f".tmp{os.getpid()}"
-    cmd = [NVCC, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *[os.path.join(CSRC, s) for s in SOURCES],
+    cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs,
            "-lcudart"]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)

@@ -1,6 +1,7 @@
 // libmoe C ABI: argument checks, workspace carving and launches.  Every
 // entry point validates before launching anything and returns a moe_status;
 // see include/moe.h for the contract of each call.
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -27,6 +28,8 @@ moe_status check_desc(const moe_layer_desc* d) {
 }
 
 thread_local const char* g_last_cuda_error = "no error";
+
+std::atomic<long long> g_wait_limit{kDefaultWaitCycles};
 
 moe_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return MOE_OK;
@@ -71,7 +74,13 @@ WsCarve carve(const moe_layer_desc& d, int T, bool tc = true) {
 
 }  // namespace
 
+long long moe::wait_limit_cycles() { return g_wait_limit.load(std::memory_order_relaxed); }
+
 extern "C" {
+
+void moe_set_wait_limit_cycles(int64_t cycles) {
+  g_wait_limit.store(cycles > 0 ? (long long)cycles : kDefaultWaitCycles, std::memory_order_relaxed);
+}
 
 const char* moe_last_cuda_error(void) { return g_last_cuda_error; }
 
@@ -222,6 +231,7 @@ __attribute__((visibility("hidden"))) moe_status moe_internal_expert_ffn(
   a.o = c.o ? reinterpret_cast<float*>(static_cast<char*>(ws) + kWsControlBytes + c.h) : nullptr;
   a.dev_err = dev_err;
   a.y_overwrite = overwrite ? 1 : 0;
+  a.wait_limit = wait_limit_cycles();
   return cuda_status(launch_ffn_decode(a, *d, device_sms(), stream));
 }
 

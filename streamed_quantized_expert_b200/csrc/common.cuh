@@ -242,7 +242,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, ui
 // a copy that never lands cannot keep the GPU busy; the caller records
 // MOE_DEV_ERR_TIMEOUT and returns.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  long long limit_cycles = 4000000000ll) {
+                                                  long long limit_cycles) {
   if (mbar_test(bar, parity)) return true;  // non-blocking test: the common already-complete case
   const long long t0 = clock64();
   while (true) {

@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) 
       int cur_ai = -1, slot = -1;
       for (int r = 0; r < my_items; ++r) {
         const int s = r % NST;
-        if (r >= NST && !mbar_wait_bounded(&empty[s], (uint32_t)(((r / NST) - 1) & 1))) {
+        if (r >= NST && !mbar_wait_bounded(&empty[s], (uint32_t)(((r / NST) - 1) & 1), a.wait_limit)) {
           if (a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
           break;  // the consumers time out on full[s]; nothing more is issued
         }
@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(kGuThreads, 1) ffn_gu_kernel(const FfnArgs a) 
     if (!ok && tid == 0 && jt == 0) flag_slot(a, em.slot);
     // a wait that runs out marks the warp; it keeps walking the items (no
     // waits, no math) so that every consumer reaches the same batch barriers
-    if (!timed_out && !mbar_wait_bounded(&full[s], (uint32_t)((r / NST) & 1))) timed_out = true;
+    if (!timed_out && !mbar_wait_bounded(&full[s], (uint32_t)((r / NST) & 1), a.wait_limit)) timed_out = true;
     const uint8_t* st = smem + (size_t)s * SB;
     const uint32_t* sbs = reinterpret_cast<const uint32_t*>(st + 2 * GRP);
     const int n_tiles = !ok ? 0 : DENSE ? 1 : (em.cnt + 7) / 8;
@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
       const uint32_t tb = (uint32_t)a.tile_d;
       for (int r = 0; r < n_act; ++r) {
         const int s = r % NST;
-        if (r >= NST && !mbar_wait_bounded(&empty[s], (uint32_t)(((r / NST) - 1) & 1))) {
+        if (r >= NST && !mbar_wait_bounded(&empty[s], (uint32_t)(((r / NST) - 1) & 1), a.wait_limit)) {
           if (a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
           break;
         }
@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(kDnThreads, 1) ffn_down_kernel(const FfnArgs a
     const bool ok = slot_ok(a, em.slot);
     // every warp waits on every stage before releasing it, which keeps the
     // phases of the empty barriers in order
-    if (!timed_out && !mbar_wait_bounded(&full[s], (uint32_t)((r / NST) & 1))) timed_out = true;
+    if (!timed_out && !mbar_wait_bounded(&full[s], (uint32_t)((r / NST) & 1), a.wait_limit)) timed_out = true;
     const uint8_t* st = smem + (size_t)s * SB;
     const uint32_t* sbs = reinterpret_cast<const uint32_t*>(st + 2 * GRP);
     const bool mine = (r % egrp) == my_grp;

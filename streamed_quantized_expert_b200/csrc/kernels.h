@@ -35,14 +35,16 @@ struct FfnArgs {
   float* hpart;   // workspace (fused kernel): [T*k][padded I / 8] (sum h, sum 128 h 2^-a) pairs
   float* o;     // workspace: [T*k][H] fp32, by flat pair index (T > kFusedMaxTokens)
   int32_t* dev_err;
-  unsigned* ctl;    // workspace control block (grid barrier of the fused kernel); zero between calls
+  unsigned* ctl;    // workspace control block (readiness counters of the fused kernel)
   int y_overwrite;  // 1: y = result (single pass over all experts); 0: y += result
   Layout L;
   // filled by the launcher
   int64_t q_gu, q_d, tile_gu, tile_d, rb_gu, rb_d;
   int ng_gu, ng_d, nblk_gu, nblk_d;
   int gu_stage_bytes, d_stage_bytes, gu_nstage, d_nstage;
-  int xh_stage_bytes;  // fused kernel: shared region for x (gate/up phase), then h (down phase)
+  int xh_stage_bytes;  // fused kernel: shared region for x (gate/up CTAs) or h (down CTAs)
+  int fu_n_dn, fu_rt_per_dn, fu_stage_area;  // fused kernel: down CTAs, their 16-row tiles, stage bytes
+  long long wait_limit;  // clock-cycle limit of every bounded device wait (wait_limit_cycles())
 };
 
 // Launch with programmatic stream serialization, so the kernel's CTAs can be
@@ -87,6 +89,10 @@ bool ffn_prefill_tc_shape_ok(const moe_layer_desc& d);
 int ffn_kernel_path(const moe_layer_desc& d, int T, bool has_x_sorted, int num_sms);
 __global__ void combine_kernel(const FfnArgs a);
 int combine_grid(int T, int H, int num_sms);
-constexpr size_t kWsControlBytes = 256;  // head of the workspace: grid-barrier words
+constexpr size_t kWsControlBytes = 512;  // head of the workspace: the fused kernel's readiness counters
+constexpr long long kDefaultWaitCycles = 4000000000ll;  // about 2 s at the top SM clock
+// Limit of the bounded device waits of kernels launched from now on
+// (moe_set_wait_limit_cycles; kDefaultWaitCycles unless a test lowered it).
+long long wait_limit_cycles();
 
 }  // namespace moe

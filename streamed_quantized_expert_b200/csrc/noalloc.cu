@@ -53,6 +53,11 @@ extern "C" moe_status moe_expert_ffn_noalloc(const uint16_t* x, int32_t T, const
   void* scratch = nullptr;
   const moe_status s = scratch_of_current_device(&scratch);
   if (s != MOE_OK) return s;
+  // The array keeps whatever the previous call (on any stream) left in it.
+  // Its head is the control block (the fused kernel's readiness counters),
+  // which must start every call at zero: clear it in stream order, so that
+  // even a call that was cut short before cannot leave a later one wrong.
+  if (cudaMemsetAsync(scratch, 0, moe::kWsControlBytes, stream) != cudaSuccess) return MOE_ERR_CUDA;
   return moe_expert_ffn(x, T, d, pool, n_slots, slot_table, ids, w, offsets, pairs, active, n_active, nullptr,
                         pass_begin, pass_len, y_accum, scratch, kNoAllocScratchBytes, dev_err, stream);
 }

@@ -83,6 +83,7 @@ struct PfArgs {
   uint16_t* h;      // [T*k][I] bf16 by sorted position (gate/up writes, down reads through its map)
   float* o;         // [T*k][H] fp32 by flat pair (down writes)
   int32_t* dev_err;
+  long long wait_limit;  // clock-cycle limit of every bounded wait
 };
 
 // ---------------------------------------------------------------------------
@@ -174,13 +175,14 @@ __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.
 __device__ __forceinline__ bool slot_ok_pf(int n_slots, int slot) { return slot >= 0 && slot < n_slots; }
 
 // Bounded wait that also gives up once another role of the CTA has aborted.
-__device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                        long long limit_cycles) {
   if (mbar_test(bar, parity)) return true;
   const long long t0 = clock64();
   for (;;) {
     if (mbar_try_wait(bar, parity, 20000u)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > 4000000000ll) {
+    if (clock64() - t0 > limit_cycles) {
       *abort_flag = 1;
       return false;
     }
@@ -351,7 +353,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const uint32_t bytes = kCodesBytes + kSbBytes + (uint32_t)nbox * 2 * 32 * 128;
         bool ok = true;
         for (int kb = 0; kb < a.nkb; ++kb) {
-          if (!pf_wait(&empty[s], ph ^ 1u, &s_abort)) {
+          if (!pf_wait(&empty[s], ph ^ 1u, &s_abort, a.wait_limit)) {
             ok = false;
             break;
           }
@@ -374,7 +376,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       // every copy issued lands before the CTA can exit
       for (int q = 0; q < kPfStages; ++q)
-        if ((issued >> q) & 1u) mbar_wait_bounded(&full[q], (last_ph >> q) & 1u);
+        if ((issued >> q) & 1u) mbar_wait_bounded(&full[q], (last_ph >> q) & 1u, a.wait_limit);
     }
   } else if (warp == kPfMmaWarp) {
     // ---------------- MMA issuer ----------------
@@ -386,12 +388,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const PfTile tl = tile_at(t);
         const int npad = (tl.n + 15) & ~15;
         const uint32_t idesc = idesc_bf16(kPfBM, npad);
-        if (!pf_wait(&accempty[c], pc ^ 1u, &s_abort)) break;
+        if (!pf_wait(&accempty[c], pc ^ 1u, &s_abort, a.wait_limit)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(c * kPfBN);
         bool ok = true;
         for (int kb = 0; kb < a.nkb; ++kb) {
-          if (!pf_wait(&full[s], ph, &s_abort) || !pf_wait(&afull[ab], pa, &s_abort)) {
+          if (!pf_wait(&full[s], ph, &s_abort, a.wait_limit) || !pf_wait(&afull[ab], pa, &s_abort, a.wait_limit)) {
             ok = false;
             break;
           }
@@ -424,7 +426,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       if (issued_any) {  // every MMA issued completes before TMEM is freed
         umma_commit(drain);
-        mbar_wait_bounded(drain, 0);
+        mbar_wait_bounded(drain, 0, a.wait_limit);
       }
     }
   } else if (warp < kPfDqWarps) {
@@ -435,7 +437,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
       bool ok = true;
       for (int kb = 0; kb < a.nkb; ++kb) {
-        if (!pf_wait(&full[s], ph, &s_abort) || !pf_wait(&aempty[ab], pa ^ 1u, &s_abort)) {
+        if (!pf_wait(&full[s], ph, &s_abort, a.wait_limit) || !pf_wait(&aempty[ab], pa ^ 1u, &s_abort, a.wait_limit)) {
           ok = false;
           break;
         }
@@ -464,7 +466,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     uint32_t pc = 0;
     for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
       const PfTile tl = tile_at(t);
-      if (!pf_wait(&accfull[c], pc, &s_abort)) break;
+      if (!pf_wait(&accfull[c], pc, &s_abort, a.wait_limit)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * kPfBN);
       // the tile's pair indices (down) in registers: lane l holds columns l, 32 + l, ...
@@ -657,6 +659,7 @@ cudaError_t launch_ffn_prefill_tc(const FfnArgs& a, const moe_layer_desc& d, int
   pa.h = a.h;
   pa.o = a.o;
   pa.dev_err = a.dev_err;
+  pa.wait_limit = a.wait_limit;
   const int grid = num_sms;
   // a CTA's tile table holds kMaxCtaExperts experts: longer passes run as
   // several gate/up + down launches over consecutive sub-ranges (sub-ranges

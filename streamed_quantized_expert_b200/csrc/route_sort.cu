@@ -137,49 +137,78 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 }
 
 // One block (8 warps) per token, for decode-sized T: thread i owns experts
-// e = i + 256 m.  Each warp takes the top-k of its experts by the same key,
-// then warp 0 takes the top-k of the 8 k candidates: every expert of the
-// token's top-k is in its own warp's top-k, so the ids, their order and the
-// weights equal those of route_kernel.
+// e = i + 256 m.  The top-k is a radix select on a 64-bit key whose order is
+// the selection order: high word = bits of u' (non-negative floats order as
+// their bit patterns), low word = l mapped to an order-preserving unsigned
+// (-0 taken as +0, so that equal logits compare equal), ties on the whole key
+// broken by the lower expert id.  Eight-bit digits from the top: each pass
+// histograms the digit of the experts still tied with the selection boundary,
+// finds the digit value that holds the k-th best, takes every expert above
+// it and keeps the tied ones; a pass whose boundary bucket is exactly the
+// number still to take ends the select (usually after two or three passes).
+// The chosen experts are then put in key order by counting, for each, the
+// chosen ones with a better key.  Same ids, order and weights as route_kernel.
+__device__ __forceinline__ uint32_t ordered_logit(float l) {
+  uint32_t b = __float_as_uint(l);
+  if (b == 0x80000000u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ uint32_t key_digit(uint32_t k1, uint32_t k2, int d) {
+  return d < 4 ? (k1 >> (24 - 8 * d)) & 0xFFu : (k2 >> (56 - 8 * d)) & 0xFFu;
+}
+
+__device__ __forceinline__ bool key_before(uint32_t a1, uint32_t a2, int ae, uint32_t b1, uint32_t b2, int be) {
+  return a1 > b1 || (a1 == b1 && (a2 > b2 || (a2 == b2 && ae < be)));
+}
+
 template <int NPT>
-__global__ void __launch_bounds__(256) route_block_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                                          float L, const int32_t* __restrict__ table,
-                                                          int32_t* __restrict__ ids, float* __restrict__ wout) {
+__global__ void __launch_bounds__(256) route_select_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                           float L, const int32_t* __restrict__ table,
+                                                           int32_t* __restrict__ ids, float* __restrict__ wout) {
   __shared__ float s_red[8];
-  __shared__ float s_cu[8 * 32], s_cl[8 * 32], s_cw[8 * 32];
-  __shared__ int s_ce[8 * 32];
+  __shared__ uint32_t s_hist[256];
+  __shared__ int s_ctl[3];  // boundary digit, experts still to take, boundary bucket size
+  __shared__ int s_warp[8];
+  __shared__ int s_nsel;
+  __shared__ uint32_t s_k1[32], s_k2[32];
+  __shared__ int s_e[32];
+  __shared__ float s_u[32];
+  __shared__ int s_oe[32];
+  __shared__ float s_ou[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t = blockIdx.x;
   pdl_wait();
   pdl_launch_dependents();
   if (t >= T) return;
   const float* l = logits + (size_t)t * E;
-  float lv[NPT], u[NPT], up[NPT];
+  float lv[NPT], u[NPT];
+  bool res[NPT];
   float lmax = -FLT_MAX;
 #pragma unroll
   for (int m = 0; m < NPT; ++m) {
     const int e = tid + 256 * m;
     lv[m] = e < E ? l[e] : -FLT_MAX;
+    res[m] = (L > 0.0f && table != nullptr && e < E) ? table[e] >= 0 : false;
     lmax = fmaxf(lmax, lv[m]);
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
   if (lane == 0) s_red[warp] = lmax;
+  if (tid == 0) s_nsel = 0;
   __syncthreads();
   lmax = s_red[0];
 #pragma unroll
   for (int w = 1; w < 8; ++w) lmax = fmaxf(lmax, s_red[w]);
+  float umin = FLT_MAX;
 #pragma unroll
   for (int m = 0; m < NPT; ++m) {
     const int e = tid + 256 * m;
-    u[m] = e < E ? route_exp(__fsub_rn(lv[m], lmax)) : -1.0f;
-    up[m] = u[m];
+    u[m] = e < E ? route_exp(__fsub_rn(lv[m], lmax)) : 0.0f;
+    if (e < E) umin = fminf(umin, u[m]);
   }
+  float boost = 0.0f;
   if (L > 0.0f && table != nullptr) {
-    float umin = FLT_MAX;
-#pragma unroll
-    for (int m = 0; m < NPT; ++m)
-      if (tid + 256 * m < E) umin = fminf(umin, u[m]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) umin = fminf(umin, __shfl_xor_sync(0xffffffffu, umin, o));
     __syncthreads();  // every warp has read s_red
@@ -188,109 +217,122 @@ __global__ void __launch_bounds__(256) route_block_kernel(const float* __restric
     umin = s_red[0];
 #pragma unroll
     for (int w = 1; w < 8; ++w) umin = fminf(umin, s_red[w]);
-    const float boost = __fmul_rn(L, __fsub_rn(1.0f, umin));
+    boost = __fmul_rn(L, __fsub_rn(1.0f, umin));
+  }
+  uint32_t k1[NPT], k2[NPT];
+  bool cand[NPT], sel[NPT];
+#pragma unroll
+  for (int m = 0; m < NPT; ++m) {
+    const int e = tid + 256 * m;
+    k1[m] = __float_as_uint(res[m] ? __fadd_rn(u[m], boost) : u[m]);
+    k2[m] = ordered_logit(lv[m]);
+    cand[m] = e < E;
+    sel[m] = false;
+  }
+  int need = k;  // experts still to take among the candidates
+  bool done = false;
+  for (int d = 0; d < 8 && !done; ++d) {
+    s_hist[tid] = 0u;
+    __syncthreads();
 #pragma unroll
     for (int m = 0; m < NPT; ++m) {
-      const int e = tid + 256 * m;
-      if (e < E && table[e] >= 0) up[m] = __fadd_rn(u[m], boost);
+      const uint32_t dig = cand[m] ? key_digit(k1[m], k2[m], d) : 0x100u;
+      const uint32_t peers = __match_any_sync(0xffffffffu, dig);
+      if (cand[m] && lane == __ffs(peers) - 1) atomicAdd(&s_hist[dig], (uint32_t)__popc(peers));
     }
-  }
-  // this warp's top-k -> candidates [warp][j]
-  uint32_t taken = 0;
-  for (int j = 0; j < k; ++j) {
-    float bu = -FLT_MAX, bl = -FLT_MAX, bw = 0.0f;
-    int be = INT_MAX;
+    __syncthreads();
+    if (warp == 0) {  // lane i covers bins 255 - 8 i down to 248 - 8 i
+      uint32_t c[8], tot = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        c[i] = s_hist[255 - 8 * lane - i];
+        tot += c[i];
+      }
+      uint32_t incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      uint32_t above = incl - tot;
+      if (above < (uint32_t)need && (uint32_t)need <= incl) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (above + c[i] >= (uint32_t)need) {
+            s_ctl[0] = 255 - 8 * lane - i;
+            s_ctl[1] = need - (int)above;
+            s_ctl[2] = (int)c[i];
+            break;
+          }
+          above += c[i];
+        }
+      }
+    }
+    __syncthreads();
+    const uint32_t bd = (uint32_t)s_ctl[0];
+    need = s_ctl[1];
+    done = s_ctl[2] == need;  // the whole boundary bucket is taken
 #pragma unroll
     for (int m = 0; m < NPT; ++m) {
-      const int e = tid + 256 * m;
-      if (e < E && !((taken >> m) & 1u) && key_better(up[m], lv[m], e, bu, bl, be)) {
-        bu = up[m];
-        bl = lv[m];
-        be = e;
-        bw = u[m];
+      if (!cand[m]) continue;
+      const uint32_t dig = key_digit(k1[m], k2[m], d);
+      if (dig > bd || (done && dig == bd)) {
+        sel[m] = true;
+        cand[m] = false;
+      } else if (dig < bd) {
+        cand[m] = false;
       }
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      const float ou = __shfl_xor_sync(0xffffffffu, bu, o);
-      const float ol = __shfl_xor_sync(0xffffffffu, bl, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      const float ow = __shfl_xor_sync(0xffffffffu, bw, o);
-      if (key_better(ou, ol, oe, bu, bl, be)) {
-        bu = ou;
-        bl = ol;
-        be = oe;
-        bw = ow;
-      }
-    }
-    if (be != INT_MAX && (be & 255) == tid) taken |= 1u << (be >> 8);
-    if (lane == 0) {
-      s_cu[warp * 32 + j] = bu;
-      s_cl[warp * 32 + j] = bl;
-      s_ce[warp * 32 + j] = be;
-      s_cw[warp * 32 + j] = bw;
     }
   }
+  if (!done) {  // the candidates left share the whole key: take the `need` lowest expert ids
+    int base = 0;
+#pragma unroll
+    for (int m = 0; m < NPT; ++m) {
+      const uint32_t bal = __ballot_sync(0xffffffffu, cand[m]);
+      __syncthreads();  // s_warp free
+      if (lane == 0) s_warp[warp] = __popc(bal);
+      __syncthreads();
+      int before = 0, total = 0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        before += w < warp ? s_warp[w] : 0;
+        total += s_warp[w];
+      }
+      const int rank = base + before + __popc(bal & ((1u << lane) - 1u));
+      if (cand[m] && rank < need) sel[m] = true;
+      base += total;
+    }
+  }
+  // the k chosen experts, then each one's position in key order
+#pragma unroll
+  for (int m = 0; m < NPT; ++m)
+    if (sel[m]) {
+      const int i = atomicAdd(&s_nsel, 1);
+      s_k1[i] = k1[m];
+      s_k2[i] = k2[m];
+      s_e[i] = tid + 256 * m;
+      s_u[i] = u[m];
+    }
   __syncthreads();
-  if (warp != 0) return;
-  // top-k of the 8 k candidates, packed: candidate c = k w + j (j-th of warp w) sits at lane c % 32,
-  // register c / 32 (at most 8 k / 32 registers hold candidates)
-  constexpr int kQ = 8;  // 8 warps x at most 32 candidates / 32 lanes
-  const int nq = (8 * k + 31) / 32;
-  float cu[kQ], cl[kQ], cw[kQ];
-  int ce[kQ];
-#pragma unroll
-  for (int q = 0; q < kQ; ++q) {
-    const int c = lane + 32 * q, w = c / k, j = c - w * k;
-    const bool ok = c < 8 * k;
-    cu[q] = ok ? s_cu[w * 32 + j] : -FLT_MAX;
-    cl[q] = ok ? s_cl[w * 32 + j] : -FLT_MAX;
-    ce[q] = ok ? s_ce[w * 32 + j] : INT_MAX;
-    cw[q] = ok ? s_cw[w * 32 + j] : 0.0f;
-  }
-  uint32_t tk = 0;
-  int my_e = 0;
-  float my_u = 0.0f;
-  for (int j = 0; j < k; ++j) {
-    float bu = -FLT_MAX, bl = -FLT_MAX, bw = 0.0f;
-    int be = INT_MAX, bq = -1;
-#pragma unroll
-    for (int q = 0; q < kQ; ++q)
-      if (q < nq && !((tk >> q) & 1u) && ce[q] != INT_MAX && key_better(cu[q], cl[q], ce[q], bu, bl, be)) {
-        bu = cu[q];
-        bl = cl[q];
-        be = ce[q];
-        bw = cw[q];
-        bq = q;
-      }
-    int bsrc = bq >= 0 ? 32 * bq + lane : -1;
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      const float ou = __shfl_xor_sync(0xffffffffu, bu, o);
-      const float ol = __shfl_xor_sync(0xffffffffu, bl, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      const float ow = __shfl_xor_sync(0xffffffffu, bw, o);
-      const int os = __shfl_xor_sync(0xffffffffu, bsrc, o);
-      if (key_better(ou, ol, oe, bu, bl, be)) {
-        bu = ou;
-        bl = ol;
-        be = oe;
-        bw = ow;
-        bsrc = os;
-      }
+  if (warp == 0) {
+    int pos = 0;
+    const bool mine = lane < k;
+    const uint32_t a1 = mine ? s_k1[lane] : 0u, a2 = mine ? s_k2[lane] : 0u;
+    const int ae = mine ? s_e[lane] : 0;
+    for (int i = 0; i < k; ++i) pos += key_before(s_k1[i], s_k2[i], s_e[i], a1, a2, ae) ? 1 : 0;
+    if (mine) {
+      s_oe[pos] = ae;
+      s_ou[pos] = s_u[lane];
     }
-    if (bsrc >= 0 && (bsrc & 31) == lane) tk |= 1u << (bsrc >> 5);
-    if (lane == j) {
-      my_e = be;
-      my_u = bw;
-    }
-  }
-  float s = lane < k ? my_u : 0.0f;
+    __syncwarp();
+    const float my_u = mine ? s_ou[lane] : 0.0f;
+    float sum = my_u;
 #pragma unroll
-  for (int o = 16; o; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
-  if (lane < k) {
-    ids[(size_t)t * k + lane] = my_e;
-    wout[(size_t)t * k + lane] = __fdiv_rn(my_u, s);
+    for (int o = 16; o; o >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, o));
+    if (mine) {
+      ids[(size_t)t * k + lane] = s_oe[lane];
+      wout[(size_t)t * k + lane] = __fdiv_rn(my_u, sum);
+    }
   }
 }
 
@@ -474,9 +516,9 @@ __global__ void __launch_bounds__(1024) lookup_kernel(const int32_t* __restrict_
 cudaError_t launch_route(const float* logits, int T, int E, int k, float L, const int32_t* table, int32_t* ids,
                          float* w, cudaStream_t st) {
   if (T <= kRouteBlockMaxTokens && E <= 1024) {  // decode sizes: a block per token
-    const void* kb = E <= 256 ? reinterpret_cast<const void*>(route_block_kernel<1>)
-                     : E <= 512 ? reinterpret_cast<const void*>(route_block_kernel<2>)
-                                : reinterpret_cast<const void*>(route_block_kernel<4>);
+    const void* kb = E <= 256 ? reinterpret_cast<const void*>(route_select_kernel<1>)
+                     : E <= 512 ? reinterpret_cast<const void*>(route_select_kernel<2>)
+                                : reinterpret_cast<const void*>(route_select_kernel<4>);
     return launch_pdl(kb, T, 256, 0, st, logits, T, E, k, L, table, ids, w);
   }
   const int blocks = (T + 7) / 8;

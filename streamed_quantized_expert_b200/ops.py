@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe.so")
 MOE_OK, MOE_ERR_INVALID, MOE_ERR_CUDA, MOE_ERR_UNSUPPORTED, MOE_ERR_NOT_RESIDENT, MOE_ERR_CAPACITY, \
     MOE_ERR_TIMEOUT = range(7)
 DEV_ERR_NOT_RESIDENT, DEV_ERR_SLOT_RANGE, DEV_ERR_TIMEOUT, DEV_ERR_BAD_EXPERT = 1, 2, 4, 8
+WS_CONTROL_BYTES = 512  # head of the workspace: the control block (include/moe.h, moe_workspace_bytes)
 
 # every entry point declared in include/moe.h
 ABI_SYMBOLS = [
@@ -24,7 +25,7 @@ ABI_SYMBOLS = [
     "moe_status_string", "moe_cache_create", "moe_cache_destroy", "moe_cache_table", "moe_cache_layer_base",
     "moe_cache_class_slots", "moe_cache_place", "moe_cache_step", "moe_cache_stats",
     "moe_expert_ffn_noalloc", "moe_noalloc_scratch_bytes", "moe_cache_resident", "moe_decode_layer",
-    "moe_last_cuda_error", "moe_ffn_kernel_path",
+    "moe_last_cuda_error", "moe_ffn_kernel_path", "moe_set_wait_limit_cycles",
 ]
 
 
@@ -90,6 +91,7 @@ def lib():
             "moe_status_string": (C.c_char_p, [C.c_int]),
             "moe_last_cuda_error": (C.c_char_p, []),
             "moe_ffn_kernel_path": (i32, [D, i32, i32]),
+            "moe_set_wait_limit_cycles": (None, [i64]),
             "moe_cache_create": (C.c_int, [i32, i32, P, i32, C.POINTER(P)]),
             "moe_cache_destroy": (None, [P]),
             "moe_cache_table": (C.POINTER(i32), [P, i32]),
@@ -116,6 +118,12 @@ MOE_PATH_FUSED_DECODE, MOE_PATH_GEMV, MOE_PATH_TC_PREFILL = 0, 1, 2
 def moe_ffn_kernel_path(d: LayerDesc, T: int, has_x_sorted: bool) -> int:
     """Kernels moe_expert_ffn runs for this layer shape and token count."""
     return int(lib().moe_ffn_kernel_path(C.byref(d), int(T), 1 if has_x_sorted else 0))
+
+
+def moe_set_wait_limit_cycles(cycles: int) -> None:
+    """Clock-cycle limit of every bounded device wait in kernels launched
+    from now on (process-wide); 0 restores the default (4e9 cycles)."""
+    lib().moe_set_wait_limit_cycles(int(cycles))
 
 
 def status_string(s: int) -> str:

@@ -275,5 +275,10 @@ class Streamer:
         return y
 
     def check_dev_err(self) -> int:
+        """The device error word (MOE_DEV_ERR_* bits).  After a wait that ran
+        out, the workspace's control block (the single-launch decode kernel's
+        readiness counters) is zeroed again before any later call."""
         v = int(self.dev_err.item())
+        if v & ops.DEV_ERR_TIMEOUT:
+            self.ws[:ops.WS_CONTROL_BYTES].zero_()
         return v

@@ -17,10 +17,13 @@ def dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
-def test_noalloc_matches_workspace_entry_point():
+@pytest.mark.parametrize("T", [6, 16])
+def test_noalloc_matches_workspace_entry_point(T):
+    # T = 6: the single-launch decode kernel; T = 16: the gate/up + down GEMV kernels
     build.build()
-    E, k, H, I, g, b, T = 64, 4, 512, 256, 64, 4, 6
+    E, k, H, I, g, b = 64, 4, 512, 256, 64, 4
     d = ops.desc(E, k, H, I, g, b, b)
+    assert ops.moe_ffn_kernel_path(d, T, False) == (ops.MOE_PATH_FUSED_DECODE if T <= 8 else ops.MOE_PATH_GEMV)
     sb = ops.moe_slot_bytes(d)
     lay = ops.moe_slot_layout(d)
     pool = torch.zeros((E, sb), dtype=torch.uint8, device="cuda")
