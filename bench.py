@@ -167,7 +167,20 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
-def build_streamer(cfg, seed, device, bits=None):
+# The mixed-class configuration as one sequence: a prefill chunk through the
+# 25%-resident two-class cache (passes of 64 active experts, installs between
+# passes), then decode steps with cache-aware substitution from the cache the
+# prefill left.
+# name: (layers, E, k, H, I, g, bits(layer), prefill T, decode steps, slots per layer, L, description)
+SEQUENCE = {
+    "mixed_sequence": (48, 512, 10, 2048, 512, 64, lambda l: (4, 6) if l % 4 == 0 else (4, 4), 4096, 256, 128, 0.15,
+                       "mixed size classes as one sequence: Flash-Next-like shapes, 4-bit gate/up, 6-bit down on "
+                       "layers l % 4 == 0, 128 of 512 slots per layer (25%), 4096-token prefill chunk (passes of 64 "
+                       "active experts, installs between passes), then 256 decode steps with L = 0.15"),
+}
+
+
+def build_streamer(cfg, seed, device, bits=None, max_tokens=None):
     import numpy as np
     import torch
 
@@ -182,7 +195,7 @@ def build_streamer(cfg, seed, device, bits=None):
             banks[(d.bits_gu, d.bits_down)] = quantize_bank_gpu(E, d, seed + 17 * d.bits_down, device)
     specs = [LayerSpec(d, banks[(d.bits_gu, d.bits_down)], synth.bank_permutation(seed, l, E).tolist())
              for l, d in enumerate(descs)]
-    st = Streamer(specs, S, max_tokens=T, device=device)
+    st = Streamer(specs, S, max_tokens=max_tokens or T, device=device)
     for l in range(n_layers):  # the S most popular experts start resident, on a random slot permutation
         hot = np.argsort(synth.popularity_rank(seed, l, E))[:S]
         st.place(l, hot.tolist(), synth.slot_permutation(seed, l, S).tolist())
@@ -470,6 +483,96 @@ def run_prefill(args, rank, world, local_rank, name=None, layers=0, embedded=Fal
                 "h2d_bytes_per_step": int(xs.numel() * 2 + lg.numel() * 4),
                 "d2h_bytes_per_step": int(n_layers * T * H * 4)},
         **({} if args.no_cpu_baseline else {"cpu_baseline": cpu_baseline_prefill(PREFILL[args.config], seed)}),
+    }
+
+
+def run_sequence(args, rank, world, local_rank):
+    """Prefill chunk, then decode steps, on one cache (see SEQUENCE).  `value`
+    is the decode tok/s of the whole path after the prefill; the prefill
+    chunk's time (with its installs) and both phases' miss rates are reported,
+    and the same sequence is replayed from the same initial cache with L = 0
+    (untimed) for the miss rate without substitution."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from streamed_quantized_expert_b200 import build as libbuild
+    from streamed_quantized_expert_b200 import ops, synth
+
+    libbuild.build()
+    ops.lib()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    n_layers, E, k, H, I, g, bits, Tp, n_dec, S, Lsub, desc_txt = SEQUENCE[args.config]
+    if args.layers:
+        n_layers = args.layers
+        desc_txt += f" [{n_layers} of the layers]"
+    n_dec = args.decode_steps or n_dec
+    seed = 1000 * rank
+    cfg = (n_layers, E, k, H, I, g, 4, 4, 1, S, desc_txt)
+    # prefill inputs (x of four distinct layers reused: the FFN's work does not depend on it), decode inputs
+    xs_p = [torch.from_numpy(synth.activations(seed, l, Tp, H).view(np.int16)).to(device) for l in range(4)]
+    lg_p = [torch.from_numpy(synth.router_logits(seed, l, Tp, E)).to(device) for l in range(n_layers)]
+    x_d, lg_d = make_inputs(cfg, seed, n_dec, device, step0=1)
+    y = torch.zeros((Tp, H), dtype=torch.float32, device=device)
+
+    def sequence(st, L):
+        s = st.stream
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        i0 = st.installs
+        ev[0].record(s)
+        for l in range(n_layers):
+            st.prefill_layer(l, xs_p[l % 4], lg_p[l], Tp, y)
+        ev[1].record(s)
+        i1 = st.installs
+        ev[2].record(s)
+        for i in range(n_dec):
+            for l in range(n_layers):
+                st.decode_layer(l, x_d[i, l], lg_d[i, l], 1, L)
+        ev[3].record(s)
+        torch.cuda.synchronize(device)
+        return (ev[0].elapsed_time(ev[1]), ev[2].elapsed_time(ev[3]), i1 - i0, st.installs - i1,
+                st.installed_bytes)
+
+    st = build_streamer(cfg, seed, device, bits, max_tokens=Tp)
+    if world > 1:
+        dist.barrier()
+    with ClockSampler(local_rank) as clk:
+        pf_ms, dec_ms, pf_inst, dec_inst, inst_bytes = sequence(st, Lsub)
+    pf_ms, dec_ms = max_over_ranks([pf_ms, dec_ms], device)
+    err = st.check_dev_err()
+    del st
+    torch.cuda.empty_cache()
+    st0 = build_streamer(cfg, seed, device, bits, max_tokens=Tp)
+    _, _, pf_inst0, dec_inst0, _ = sequence(st0, 0.0)
+    del st0
+    torch.cuda.empty_cache()
+    if rank != 0:
+        return None
+    flops = 2.0 * Tp * k * 3 * H * I * n_layers
+    pairs_pf = Tp * k * n_layers
+    pairs_dec = n_dec * k * n_layers
+    return {
+        "metric": METRIC, "value": round(n_dec * world / (dec_ms * 1e-3), 3), "unit": "tok/s",
+        "value_is": "decode tok/s of the whole path (route+sort+lookup+installs+FFN+combine, %d layers) after the "
+                    "prefill chunk, from the cache it left" % n_layers,
+        "n_gpus": world, "steps": n_dec, "warmup": 0, "ms_per_step": round(dec_ms / n_dec, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 (4/6-bit codes, bf16 tensor-core operands, fp32 accumulate)",
+        "data": "synthetic (seeded N(0,0.02) experts quantised on the GPU; N(0,1) bf16 x; log-Zipf-biased logits)",
+        "config": {"workload": desc_txt, "layers": n_layers, "experts": E, "top_k": k, "hidden": H, "intermediate": I,
+                   "group": g, "prefill_tokens": Tp, "decode_steps": n_dec, "slots_per_layer": S,
+                   "substitution_L": Lsub, "parallelism": f"replicas x{world}"},
+        "prefill": {"ms_per_chunk": round(pf_ms, 3), "tok_s": round(Tp / (pf_ms * 1e-3), 1),
+                    "tflops_with_installs": round(flops / (pf_ms * 1e-3) / 1e12, 2),
+                    "installs": pf_inst, "miss_rate": round(pf_inst / pairs_pf, 5),
+                    "how": "route + sort + per pass of 64 active experts: lookup, host LRU step, pinned installs, "
+                           "FFN (host-driven passes), every layer, CUDA events"},
+        "decode": {"ms_per_token": round(dec_ms / n_dec, 4), "installs": dec_inst,
+                   "miss_rate": round(dec_inst / pairs_dec, 4),
+                   "miss_rate_without_substitution": round(dec_inst0 / pairs_dec, 4),
+                   "prefill_installs_without_substitution": pf_inst0},
+        "dev_err": err, "clocks": clk.summary(),
     }
 
 
@@ -867,11 +970,12 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", choices=sorted(CONFIGS) + sorted(PREFILL), default="decode")
+    ap.add_argument("--config", choices=sorted(CONFIGS) + sorted(PREFILL) + sorted(SEQUENCE), default="decode")
     ap.add_argument("--cpu-layers", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ffn-reps", type=int, default=20)
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (small profiling runs)")
+    ap.add_argument("--decode-steps", type=int, default=0, help="mixed_sequence: decode steps (default 256)")
     ap.add_argument("--prefill-layers", type=int, default=8,
                     help="decode line: layers of the Flash-Next-like prefill chunk timed into its `prefill` object "
                          "(0: none)")
@@ -901,7 +1005,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        out = (run_prefill if args.config in PREFILL else run_ours)(args, rank, world, local_rank)
+        run = run_prefill if args.config in PREFILL else run_sequence if args.config in SEQUENCE else run_ours
+        out = run(args, rank, world, local_rank)
         if out is not None:
             print(json.dumps(out), flush=True)
     finally:

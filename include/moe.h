@@ -164,7 +164,9 @@ moe_status moe_route(const float* logits, int32_t T, const moe_layer_desc* d, fl
  *   pairs    device int32 [T*k]: flat index t*k+j, by expert then flat index
  *   active   device int32 [E]: experts with >= 1 pair, ascending
  *   n_active device int32 [1]
- *   x_sorted device bf16 [T*k, H]: x_sorted[i] = x[pairs[i] / k] (if x)
+ *   x_sorted device fp16 [T*k, H]: x_sorted[i] = x[pairs[i] / k] converted
+ *            to fp16 (round to nearest even, saturating at +-65504), the
+ *            operand type of the tensor-core grouped GEMM (if x)
  *   ws       device workspace of ws_bytes >= moe_workspace_bytes(d, T)
  * Prefill pass p covers active[64p .. 64p+64). */
 moe_status moe_sort(const int32_t* ids, const uint16_t* x, int32_t T, const moe_layer_desc* d,
@@ -352,7 +354,7 @@ typedef struct {
   void* ws;            /* device workspace */
   size_t ws_bytes;     /* >= moe_workspace_bytes(desc, max_tokens) */
   int32_t max_tokens;
-  uint16_t* x_sorted;  /* device bf16 [max_tokens*k, H], or NULL: from 32 tokens the layer
+  uint16_t* x_sorted;  /* device fp16 [max_tokens*k, H], or NULL: from 32 tokens the layer
                           sorts x into it and its FFN runs on the tensor-core grouped GEMM */
 } moe_step_buffers;
 

@@ -6,6 +6,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "moe.h"
@@ -58,6 +59,9 @@ inline Layout make_layout(const moe_layer_desc& d) {
 // bits of bf16 128.0 (0x4300), at bit offset a(i) (0 or 3).  Consumers either
 // subtract the offset per group (tensor-core GEMV) or convert to the exact q.
 constexpr uint32_t kMagic = 0x43004300u;
+// The same codes under the fp16 magic 1024.0 (0x6400): 1024 + q * 2^a in each
+// half (q * 2^a < 1024 for every width), for fp16 tensor-core operands.
+constexpr uint32_t kMagic16 = 0x64006400u;
 
 // (a & mask) | c  in one LOP3 (truth table 0xEA = (A & B) | C).
 template <uint32_t MASK>
@@ -83,11 +87,17 @@ struct PairShift<6> {
   static __host__ __device__ constexpr int a(int) { return 0; }
 };
 
-template <int B>
-__device__ __forceinline__ void unpack_unit(const uint32_t (&w)[B], uint32_t (&p)[16]);
+template <int B, uint32_t M = kMagic>
+struct Unpack;
 
-template <>
-__device__ __forceinline__ void unpack_unit<4>(const uint32_t (&w)[4], uint32_t (&p)[16]) {
+template <int B, uint32_t M = kMagic>
+__device__ __forceinline__ void unpack_unit(const uint32_t (&w)[B], uint32_t (&p)[16]) {
+  Unpack<B, M>::run(w, p);
+}
+
+template <uint32_t kMagic>
+struct Unpack<4, kMagic> {
+static __device__ __forceinline__ void run(const uint32_t (&w)[4], uint32_t (&p)[16]) {
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const uint32_t v = w[k];
@@ -98,9 +108,11 @@ __device__ __forceinline__ void unpack_unit<4>(const uint32_t (&w)[4], uint32_t 
     p[4 * k + 3] = andor<0x00780078u>(v8 >> 1, kMagic); // bits 12..15 -> 3..6, a = 3
   }
 }
+};
 
-template <>
-__device__ __forceinline__ void unpack_unit<3>(const uint32_t (&w)[3], uint32_t (&p)[16]) {
+template <uint32_t kMagic>
+struct Unpack<3, kMagic> {
+static __device__ __forceinline__ void run(const uint32_t (&w)[3], uint32_t (&p)[16]) {
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
     const uint32_t v = w[k];
@@ -116,9 +128,11 @@ __device__ __forceinline__ void unpack_unit<3>(const uint32_t (&w)[3], uint32_t 
   t = andor<0x00020002u>(w[1] >> 14, t);
   p[15] = andor<0x00040004u>(w[2] >> 13, t);
 }
+};
 
-template <>
-__device__ __forceinline__ void unpack_unit<6>(const uint32_t (&w)[6], uint32_t (&p)[16]) {
+template <uint32_t kMagic>
+struct Unpack<6, kMagic> {
+static __device__ __forceinline__ void run(const uint32_t (&w)[6], uint32_t (&p)[16]) {
 #pragma unroll
   for (int k = 0; k < 6; ++k) {
     p[2 * k + 0] = andor<0x003F003Fu>(w[k], kMagic);       // bits 0..5
@@ -131,6 +145,7 @@ __device__ __forceinline__ void unpack_unit<6>(const uint32_t (&w)[6], uint32_t 
     p[12 + m] = andor<0x00300030u>(w[4 + m / 2] >> (8 + 2 * (m % 2)), t);
   }
 }
+};
 
 // bf16x2 (128 + q*2^a) -> exact q of the low / high half as float.
 __device__ __forceinline__ float pair_lo_q(uint32_t p, int a) {
@@ -180,6 +195,13 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
   if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu)) return (uint16_t)((u >> 16) | 0x40u);
   u += 0x7fffu + ((u >> 16) & 1u);
   return (uint16_t)(u >> 16);
+}
+
+// fp32 -> fp16 bits, round to nearest even, saturating at +-65504 (the
+// tensor-core path's operands: sorted activations and h).
+__device__ __forceinline__ uint16_t f32_to_f16_sat(float f) {
+  f = fminf(fmaxf(f, -65504.0f), 65504.0f);
+  return __half_as_ushort(__float2half_rn(f));
 }
 
 // ---------------------------------------------------------------------------

@@ -13,7 +13,7 @@ constexpr int kDenseMaxTokens = 8;    // T <= 8: every token gets its own MMA co
 constexpr int kMaxCtaExperts = 64;    // per-CTA expert metadata table
 constexpr int kHStageMax = 24 * 1024; // h staged in shared memory up to this many bytes
 constexpr int kDnKSplit = 4;          // down: warps split K four ways, the rest take experts in turn
-constexpr int kFuConsumers = 8;       // fused kernel consumer warps
+constexpr int kFuConsumers = 16;      // fused kernel consumer warps
 
 struct RedMeta {
   int ei;    // CTA-local expert index

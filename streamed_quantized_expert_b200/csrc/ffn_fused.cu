@@ -1,25 +1,31 @@
 // Decode FFN in one launch (T <= 8 tokens, every routed pair in the per-CTA
 // tables): gate/up + SwiGLU -> h, then down + weighted combine -> y.
 //
-// One CTA per SM, all co-resident (cooperative launch), in two roles:
-//   * gate/up CTAs (blockIdx.x >= n_dn) take the pass's gate/up items -- a
-//     16-row tile (8 gate + 8 up rows) of one expert -- in rounds: item
-//     i = r * n_gu + c.  Items run expert-major, so each round finishes the
-//     next experts of the pass.  After every pair of items a CTA writes their
-//     h columns and adds the item count to each expert's readiness counter
-//     (release);
-//   * down CTAs (blockIdx.x < n_dn) own rt_per_dn 16-row tiles of the down
-//     projection: at kernel start they copy those rows of every active
-//     expert (one contiguous bulk copy per expert), then take the experts as
-//     their counters report complete (acquire), several at once, and
-//     accumulate w * (W_d h) for every token in registers; y is written once.
-// The role split is chosen on the host so that every SM streams about the
-// same number of bytes.  There is no grid-wide barrier: the down work of the
-// first experts overlaps the gate/up work of the last, and a layer costs one
-// launch and one metadata round trip.  The producer warp of every CTA reads
-// the pass's active experts and the whole expert -> slot table in one round
-// of independent loads, then its 32 lanes issue the CTA's bulk copies in
-// parallel.
+// One CTA per SM, all co-resident (cooperative launch); a producer warp and
+// 16 consumer warps per CTA.  Every CTA first takes a contiguous range of the
+// pass's gate/up items (a 16-row tile: 8 gate + 8 up rows of one expert;
+// items run expert-major), then -- if it owns one -- a 16-row tile of the
+// down projection for every active expert.  The ranges are weighted so that
+// each SM streams about the same number of bytes (CTAs without a down tile
+// take more gate/up items).  There is no grid-wide barrier: after every pair
+// of items a CTA writes their h columns and adds the item count to each
+// expert's readiness counter (release); a CTA's down work takes the experts
+// in order as their counters report every item written (acquire), so the
+// down work of the first experts overlaps the gate/up work of the last.
+//
+// Before the dependency wait (programmatic dependent launch) every CTA asks
+// L2 for the pass's tables, x and the expert -> slot table, so that the
+// metadata round after the wait hits L2.  The producer warp then reads the
+// active experts and the whole slot table in one round of independent loads
+// and its 32 lanes issue, in parallel, one bulk copy per gate/up item and one
+// per expert for the down tile, so the down weights stream in while gate/up
+// computes.  The consumer warps form four groups of four; group g takes the
+// CTA's items g, g + 4, ... and splits K over its warps, so four items are in
+// flight at once and every barrier of the gate/up phase is group-local.  A
+// group reduces its four warps' partial sums with shuffles, writes the item's
+// h columns, and hands the item to the producer warp, which makes the writes
+// visible (release) and adds to the expert's readiness counter, so no
+// consumer waits on that fence.
 //
 // Control block (head of the workspace): one readiness counter per pass
 // entry and the down CTAs' departure count.  Every launch starts with them at
@@ -36,9 +42,11 @@
 namespace moe {
 
 constexpr int kFuThreads = (kFuConsumers + 1) * 32;
-constexpr int kFuRtMax = 4;  // 16-row down tiles per down CTA
-constexpr int kFuRedFloats = kRedBatch * kFuConsumers * 32 * 4;
-static_assert(kFuConsumers * kFuRtMax * 32 * 4 <= kFuRedFloats, "down partial sums fit the reduction buffer");
+constexpr int kFuDnGroups = kFuConsumers / kDnKSplit;  // warp groups taking down experts in turn
+constexpr int kGuGroups = 4;                            // gate/up warp groups (one item each at a time)
+constexpr int kGuGroupWarps = kFuConsumers / kGuGroups;
+constexpr int kGuPubRing = 32;                          // items a group can hand over before they are published
+constexpr int kFuRedFloats = kFuConsumers * 32 * 4;     // one item per group: [warp][lane][4]
 // control block words
 constexpr int kCtlReady = 0;                // uint32 [kMaxCtaExperts]
 constexpr int kCtlDepart = kMaxCtaExperts;  // uint32
@@ -56,57 +64,97 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 
 // Named barrier 2 over all threads of the CTA: the producer warp arrives once
 // the pass tables are in shared memory, the consumer warps wait on it.
 __device__ __forceinline__ void tables_arrive() { asm volatile("bar.arrive 2, %0;" ::"n"(kFuThreads) : "memory"); }
 __device__ __forceinline__ void tables_sync() { asm volatile("bar.sync 2, %0;" ::"n"(kFuThreads) : "memory"); }
+// Named barriers 3 .. 6: one per gate/up warp group.
+__device__ __forceinline__ void group_sync(int g) {
+  asm volatile("bar.sync %0, %1;" ::"r"(3 + g), "n"(kGuGroupWarps * 32) : "memory");
+}
+__device__ __forceinline__ int ld_volatile_shared(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
+
+// First gate/up item of CTA c (c = grid: the item count): every CTA's quota
+// is the pass's bytes / grid, less the bytes of its down tile for the CTAs
+// that own one, in gate/up items (closed form of the prefix sum).
+__device__ __forceinline__ int fu_item_bound(int c, int n_items, int n_act, const FfnArgs& a) {
+  const int64_t G = gridDim.x, nd = a.H / 16;
+  const int64_t dn = (int64_t)n_act * a.tile_d;                // bytes of one down tile over the pass
+  const int64_t tot = (int64_t)n_items * a.tile_gu + nd * dn;  // bytes of the pass
+  int64_t f = (int64_t)c * tot - (c < nd ? c : nd) * G * dn;   // prefix * G, in bytes
+  if (f < 0) f = 0;
+  const int64_t v = f / (G * a.tile_gu);
+  return v > n_items ? n_items : (int)v;
+}
 
 template <int BG, int BD, int BPW, int GS>
 __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, t4 = lane & 3, g8 = lane >> 2;
-  const bool dn_role = (int)blockIdx.x < a.fu_n_dn;
-  const int NS = dn_role ? a.d_nstage : a.gu_nstage;
-  const int SB = dn_role ? a.d_stage_bytes : a.gu_stage_bytes;
-  uint8_t* stg = smem;                                         // stages of the CTA's role
-  uint8_t* xh = stg + (size_t)a.fu_stage_area;                 // gate/up: x [T][H]; down: h rows + sums
-  float* red = reinterpret_cast<float*>(xh + a.xh_stage_bytes);                 // partial sums
-  RedMeta* rmeta = reinterpret_cast<RedMeta*>(red + kFuRedFloats);              // [kRedBatch]
-  int* s_act = reinterpret_cast<int*>(rmeta + kRedBatch);      // pass entry -> expert id
-  int* s_slot = s_act + kMaxCtaExperts;                        // pass entry -> slot
-  int* s_ids = s_slot + kMaxCtaExperts;                        // flat pair -> expert id
+  const int NSG = a.gu_nstage, SBG = a.gu_stage_bytes, NSD = a.d_nstage, SBD = a.d_stage_bytes;
+  uint8_t* gst = smem;                                            // gate/up stages
+  uint8_t* dst_ = gst + (size_t)NSG * SBG;                        // down stages
+  uint8_t* xh = dst_ + (size_t)NSD * SBD;                         // x [T][H], then h rows + sums
+  float* red = reinterpret_cast<float*>(xh + a.xh_stage_bytes);   // partial sums [warps][32][4]
+  int* s_act = reinterpret_cast<int*>(red + kFuRedFloats);        // pass entry -> expert id
+  int* s_slot = s_act + kMaxCtaExperts;                           // pass entry -> slot
+  int* s_ids = s_slot + kMaxCtaExperts;                           // flat pair -> expert id
   float* s_w = reinterpret_cast<float*>(s_ids + kMaxCtaExperts);  // flat pair -> routing weight
   int* s_tok = reinterpret_cast<int*>(s_w + kMaxCtaExperts);      // [entry][token] -> flat pair or -1
-  uint64_t* full = reinterpret_cast<uint64_t*>(s_tok + kMaxCtaExperts * kDenseMaxTokens);
-  uint64_t* empty = full + NS;
-  int* s_table = reinterpret_cast<int*>(empty + NS);           // expert -> slot, [E]
-  __shared__ int s_nact;
+  uint64_t* gfull = reinterpret_cast<uint64_t*>(s_tok + kMaxCtaExperts * kDenseMaxTokens);
+  uint64_t* gempty = gfull + NSG;
+  uint64_t* dfull = gempty + NSG;
+  uint64_t* dempty = dfull + NSD;
+  int* s_table = reinterpret_cast<int*>(dempty + NSD);  // expert -> slot, [E]
+  __shared__ int s_nact, s_i0, s_i1;
   __shared__ unsigned long long s_ready;
   __shared__ int s_timeout, s_npl;
   __shared__ int s_plist[kMaxCtaExperts];
+  __shared__ int s_pub_e[kGuGroups][kGuPubRing];  // per group: entries of its written items, in order
+  __shared__ int s_pub_cnt[kGuGroups];             // items a group has handed over
   unsigned* ready = a.ctl + kCtlReady;
+  const int np = a.T * a.k;  // <= kMaxCtaExperts (dense mode)
 
+  // ask L2 for what the metadata round reads; nothing is read into the SM
+  // before the dependency wait (the previous kernel may still write it)
+  if (warp == kFuConsumers) {
+    for (int e = 32 * lane; e < a.E; e += 32 * 32) prefetch_l2(a.table + e);
+    if (lane == 0) prefetch_l2(a.n_active);
+    if (lane < 2) prefetch_l2(a.active + a.pass_begin + 32 * lane);
+    if (lane == 2) prefetch_l2(a.ids);
+    if (lane == 3) prefetch_l2(a.w);
+  } else {
+    const int nx = a.T * a.H * 2;  // bytes of x
+    for (int b = 128 * tid; b < nx; b += 128 * kFuConsumers * 32)
+      prefetch_l2(reinterpret_cast<const uint8_t*>(a.x) + b);
+  }
   if (tid == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kFuConsumers);
+    for (int s = 0; s < NSG; ++s) {
+      mbar_init(&gfull[s], 1);
+      mbar_init(&gempty[s], kGuGroupWarps);
+    }
+    for (int s = 0; s < NSD; ++s) {
+      mbar_init(&dfull[s], 1);
+      mbar_init(&dempty[s], kFuConsumers);
     }
     fence_barrier_init();
     s_timeout = 0;
+    for (int g = 0; g < kGuGroups; ++g) s_pub_cnt[g] = 0;
   }
   __syncthreads();
   pdl_wait();
-  const int np = a.T * a.k;  // <= kMaxCtaExperts (dense mode)
   int cap = a.E - a.pass_begin;
   if (cap > a.pass_len) cap = a.pass_len;
   if (cap > kMaxCtaExperts) cap = kMaxCtaExperts;
   if (cap < 0) cap = 0;
   const int jt_n = a.I / 8;
-  const int n_gu = (int)gridDim.x - a.fu_n_dn;
   const int n_rt = a.H / 16;
-  const int rt0 = (int)blockIdx.x * a.fu_rt_per_dn;
-  const int nrt = dn_role ? (n_rt - rt0 < a.fu_rt_per_dn ? n_rt - rt0 : a.fu_rt_per_dn) : 0;
+  const int rt = blockIdx.x;  // the CTA's down tile, if rt < n_rt
+  const bool has_rt = rt < n_rt;
   const int Ip = a.nblk_d * 128;  // h row stride: the intermediate size padded to whole 128-blocks
 
   if (warp == kFuConsumers) {
@@ -144,54 +192,75 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
         s_slot[i] = (e >= 0 && e < a.E) ? s_table[e] : -1;
       }
     }
-    if (lane == 0) s_nact = n_act;
+    const int n_items = n_act * jt_n;
+    const int i0 = fu_item_bound(blockIdx.x, n_items, n_act, a);
+    const int i1 = fu_item_bound(blockIdx.x + 1, n_items, n_act, a);
+    if (lane == 0) {
+      s_nact = n_act;
+      s_i0 = i0;
+      s_i1 = i1;
+    }
     __syncwarp();
     tables_arrive();
-    const int64_t sbytes = a.slot_bytes;
+    const int my_items = i1 - i0, n_dn = has_rt ? n_act : 0;
+    const uint32_t tbg = (uint32_t)a.tile_gu, tbd = (uint32_t)a.tile_d;
+    auto issue_gu = [&](int r) -> bool {
+      const int s = r % NSG;
+      if (r >= NSG && !mbar_wait_bounded(&gempty[s], (uint32_t)(((r / NSG) - 1) & 1), a.wait_limit)) return false;
+      const int item = i0 + r;
+      const int slot = s_slot[item / jt_n];
+      if (!slot_ok(a, slot)) {
+        mbar_arrive_expect_tx(&gfull[s], 0);
+        return true;
+      }
+      mbar_arrive_expect_tx(&gfull[s], tbg);
+      bulk_g2s(gst + (size_t)s * SBG, a.pool + (int64_t)slot * a.slot_bytes + a.q_gu + (int64_t)(item % jt_n) * tbg,
+               tbg, &gfull[s]);
+      return true;
+    };
+    auto issue_dn = [&](int i) -> bool {
+      const int s = i % NSD;
+      if (i >= NSD && !mbar_wait_bounded(&dempty[s], (uint32_t)(((i / NSD) - 1) & 1), a.wait_limit)) return false;
+      const int slot = s_slot[i];
+      if (!slot_ok(a, slot)) {
+        mbar_arrive_expect_tx(&dfull[s], 0);
+        return true;
+      }
+      mbar_arrive_expect_tx(&dfull[s], tbd);
+      bulk_g2s(dst_ + (size_t)s * SBD, a.pool + (int64_t)slot * a.slot_bytes + a.q_d + (int64_t)rt * tbd, tbd,
+               &dfull[s]);
+      return true;
+    };
+    // everything that fits goes out at once, one copy per lane; the rest
+    // (lane 0) as stages free up
+    const int ng0 = my_items < NSG ? my_items : NSG, nd0 = n_dn < NSD ? n_dn : NSD;
+    for (int r = lane; r < ng0; r += 32) issue_gu(r);
+    for (int i = lane; i < nd0; i += 32) issue_dn(i);
     bool ok = true;
-    if (dn_role) {
-      // entry i: rows rt0*16 .. (rt0+nrt)*16 of its down projection, one copy
-      const uint32_t bytes = (uint32_t)(nrt * a.tile_d);
-      auto issue = [&](int i) -> bool {
-        const int s = i % NS;
-        if (i >= NS && !mbar_wait_bounded(&empty[s], (uint32_t)(((i / NS) - 1) & 1), a.wait_limit)) return false;
-        const int slot = s_slot[i];
-        if (!slot_ok(a, slot) || nrt <= 0) {
-          mbar_arrive_expect_tx(&full[s], 0);
-          return true;
+    if (lane == 0) {
+      for (int r = ng0; ok && r < my_items; ++r) ok = issue_gu(r);
+      for (int i = nd0; ok && i < n_dn; ++i) ok = issue_dn(i);
+    }
+    // publish service: lane 1 + g makes gate/up group g's h writes visible
+    // (fence) and adds each written item to its expert's readiness counter
+    // (lane 0 may still be refilling stages, which waits on the consumers)
+    if (lane >= 1 && lane <= kGuGroups) {
+      const int g = lane - 1;
+      const int n_g = my_items > g ? (my_items - g + kGuGroups - 1) / kGuGroups : 0;
+      int done = 0;
+      const long long t0 = clock64();
+      while (ok && done < n_g) {
+        const int c = ld_volatile_shared(&s_pub_cnt[g]);
+        if (c == done) {
+          if (clock64() - t0 > a.wait_limit) ok = false;
+          continue;
         }
-        mbar_arrive_expect_tx(&full[s], bytes);
-        bulk_g2s(stg + (size_t)s * SB, a.pool + (int64_t)slot * sbytes + a.q_d + (int64_t)rt0 * a.tile_d, bytes,
-                 &full[s]);
-        return true;
-      };
-      const int n0 = n_act < NS ? n_act : NS;
-      for (int i = lane; i < n0; i += 32) issue(i);
-      if (lane == 0)
-        for (int i = n0; ok && i < n_act; ++i) ok = issue(i);
-    } else {
-      const int gi = (int)blockIdx.x - a.fu_n_dn;
-      const int n_items = n_act * jt_n;
-      const int my_items = gi < n_items ? (n_items - gi + n_gu - 1) / n_gu : 0;
-      const uint32_t bytes = (uint32_t)a.tile_gu;
-      auto issue = [&](int q) -> bool {
-        const int s = q % NS;
-        if (q >= NS && !mbar_wait_bounded(&empty[s], (uint32_t)(((q / NS) - 1) & 1), a.wait_limit)) return false;
-        const int item = gi + q * n_gu;
-        const int slot = s_slot[item / jt_n];
-        if (!slot_ok(a, slot)) {
-          mbar_arrive_expect_tx(&full[s], 0);
-          return true;
+        __threadfence();
+        for (; done < c; ++done) {
+          const int e = s_pub_e[g][done % kGuPubRing];
+          if (e >= 0) atomicAdd(ready + e, 1u);
         }
-        mbar_arrive_expect_tx(&full[s], bytes);
-        bulk_g2s(stg + (size_t)s * SB, a.pool + (int64_t)slot * sbytes + a.q_gu + (int64_t)(item % jt_n) * bytes,
-                 bytes, &full[s]);
-        return true;
-      };
-      const int n0 = my_items < NS ? my_items : NS;
-      for (int q = lane; q < n0; q += 32) issue(q);
-      if (lane == 0)
-        for (int q = n0; ok && q < my_items; ++q) ok = issue(q);
+      }
     }
     if (!ok && a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
     return;
@@ -202,22 +271,44 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
     s_ids[p] = a.ids[p];
     s_w[p] = a.w[p];
   }
-  if (!dn_role) {  // x -> shared memory, in the producer's round (H a multiple of 32: whole 16-byte words)
-    const int nx = a.T * a.H / 8;
+  {
+    // x' = x 2^-a (exact: a power of two; a by input position within its
+    // 128-block) -> shared memory, with the per-(group, token) sums
+    // sum x and 128 sum x' that the group epilogues apply
+    const int nx = a.T * a.H / 8;  // 16-byte words of x (H a multiple of 32)
+    const int wpg = a.g / 8;       // words per group: consecutive lanes, aligned
     uint4* xd = reinterpret_cast<uint4*>(xh);
-    for (int b0 = tid; b0 < nx; b0 += 4 * kFuConsumers * 32) {
-      uint4 v[4];
+    float* xsum = reinterpret_cast<float*>(xh + (size_t)a.T * a.H * 2);
+    for (int base = warp * 32; base < nx; base += kFuConsumers * 32) {
+      const int idx = base + lane;
+      const bool act = idx < nx;
+      uint4 v = act ? __ldg(reinterpret_cast<const uint4*>(a.x) + idx) : make_uint4(0u, 0u, 0u, 0u);
+      const int t = idx / (a.H / 8), k = (idx % (a.H / 8)) * 8, kk = k & 127;
+      const bool eighth = PairShift<BG>::a(2 * (kk >> 4) + ((kk & 15) >> 3)) == 3;
+      uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      float sx = 0.f, so = 0.f;
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (b0 + u * kFuConsumers * 32 < nx)
-          v[u] = __ldg(reinterpret_cast<const uint4*>(a.x) + b0 + u * kFuConsumers * 32);
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (b0 + u * kFuConsumers * 32 < nx) xd[b0 + u * kFuConsumers * 32] = v[u];
+      for (int u = 0; u < 4; ++u) {
+        sx += bf16_lo(w4[u]) + bf16_hi(w4[u]);
+        if (eighth) w4[u] = bf2_scale_eighth(w4[u]);
+        so += bf16_lo(w4[u]) + bf16_hi(w4[u]);
+      }
+      for (int o = 1; o < wpg; o <<= 1) {
+        sx += __shfl_xor_sync(0xffffffffu, sx, o);
+        so += __shfl_xor_sync(0xffffffffu, so, o);
+      }
+      if (act) {
+        xd[idx] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        if ((idx % wpg) == 0) {
+          const int G = k / a.g;
+          xsum[(G * a.T + t) * 2] = sx;
+          xsum[(G * a.T + t) * 2 + 1] = 128.0f * so;
+        }
+      }
     }
   }
   tables_sync();  // the producer's pass tables
-  const int n_act = s_nact;
+  const int n_act = s_nact, i0 = s_i0, i1 = s_i1;
   // (entry, token) -> flat pair from the routed ids (a token routes to an expert at most once)
   for (int i = tid; i < n_act * kDenseMaxTokens; i += kFuConsumers * 32) {
     const int r = i / kDenseMaxTokens, t = i % kDenseMaxTokens;
@@ -232,154 +323,125 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
   if (blockIdx.x == 0)
     for (int i = tid; i < n_act; i += kFuConsumers * 32)
       if (!slot_ok(a, s_slot[i])) flag_slot(a, s_slot[i]);
-  consumers_sync(kFuConsumers * 32);
-  pdl_launch_dependents();
+  consumers_sync(kFuConsumers * 32);  // x in shared memory, pair map written
   bool timed_out = false;
 
-  if (!dn_role) {
-    // ---------------- gate/up + SwiGLU -> h, item pairs ----------------
-    const int gi = (int)blockIdx.x - a.fu_n_dn;
-    const int n_items = n_act * jt_n;
-    const int my_items = gi < n_items ? (n_items - gi + n_gu - 1) / n_gu : 0;
-    uint32_t xbf[BPW][8][2];
-    float xs[BPW][8 / GS][2], xo[BPW][8 / GS][2];
-    {
-      const uint16_t* xrow = g8 < a.T ? reinterpret_cast<const uint16_t*>(xh) + g8 * a.H : nullptr;
-#pragma unroll
-      for (int bi = 0; bi < BPW; ++bi) load_b_block<BG, GS>(xrow, warp * BPW + bi, a.H, t4, xbf[bi], xs[bi], xo[bi]);
-    }
+  // ---------------- gate/up + SwiGLU -> h, one item per warp group ----------------
+  {
+    const int gg = warp / kGuGroupWarps, wg = warp % kGuGroupWarps;  // group, warp within the group
+    const uint16_t* xrow = g8 < a.T ? reinterpret_cast<const uint16_t*>(xh) + g8 * a.H : nullptr;
+    const float* xsum = reinterpret_cast<const float*>(xh + (size_t)a.T * a.H * 2);
     const int GRP = 8 * (int)a.rb_gu;
     const int uoff = thread_unit_off<BG>(t4, g8);
-    const bool all_blocks = (warp + 1) * BPW <= a.nblk_gu;
-    auto item_mma = [&](const uint8_t* st, float (&acc)[4]) {
-      const uint32_t* sbs = reinterpret_cast<const uint32_t*>(st + 2 * GRP);
-#pragma unroll
-      for (int bi = 0; bi < BPW; ++bi)
-        if (all_blocks || warp * BPW + bi < a.nblk_gu)
-          block_mma<BG, GS>(st, st + GRP, sbs + g8, sbs + 8 + g8, warp * BPW + bi, uoff, xbf[bi], xs[bi], xo[bi],
-                            acc);
-    };
-    const int nflush = a.T * 8;  // (token, column) pairs of one entry
-    for (int q = 0; q < my_items; q += 2) {
-      const bool two = q + 1 < my_items;
-      const int it0 = gi + q * n_gu, it1 = it0 + n_gu;
-      const int e0 = it0 / jt_n, e1 = two ? it1 / jt_n : 0;
-      const bool ok0 = slot_ok(a, s_slot[e0]), ok1 = two && slot_ok(a, s_slot[e1]);
-      const int s0 = q % NS, s1 = (q + 1) % NS;
-      if (!timed_out && !mbar_wait_bounded(&full[s0], (uint32_t)((q / NS) & 1), a.wait_limit)) timed_out = true;
-      if (two && !timed_out && !mbar_wait_bounded(&full[s1], (uint32_t)(((q + 1) / NS) & 1), a.wait_limit))
-        timed_out = true;
-      float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+    const int n0 = 2 * t4 < a.T ? 2 * t4 : 0, n1 = 2 * t4 + 1 < a.T ? 2 * t4 + 1 : 0;  // C fragment columns
+    const int my_items = i1 - i0;
+    int handed = 0;
+    for (int q = gg; q < my_items; q += kGuGroups) {
+      const int it = i0 + q, e = it / jt_n, jt = it % jt_n;
+      const int s = q % NSG;
+      const bool ok = slot_ok(a, s_slot[e]);
+      if (!timed_out && !mbar_wait_bounded(&gfull[s], (uint32_t)((q / NSG) & 1), a.wait_limit)) timed_out = true;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
       if (!timed_out) {
-        if (ok0 && ok1) {  // the two items' load / unpack / MMA chains interleave
-          const uint8_t* st0 = stg + (size_t)s0 * SB;
-          const uint8_t* st1 = stg + (size_t)s1 * SB;
-          const uint32_t* sb0 = reinterpret_cast<const uint32_t*>(st0 + 2 * GRP);
-          const uint32_t* sb1 = reinterpret_cast<const uint32_t*>(st1 + 2 * GRP);
+        const uint8_t* st = gst + (size_t)s * SBG;
+        const uint32_t* sbs = reinterpret_cast<const uint32_t*>(st + 2 * GRP);
+        for (int kb = wg; kb < a.nblk_gu; kb += kGuGroupWarps) {
+          uint32_t bf[8][2];
+          float xs[8 / GS][2], xo[8 / GS][2];
+          const uint16_t* row = xrow ? xrow + kb * 128 + 2 * t4 : nullptr;
 #pragma unroll
-          for (int bi = 0; bi < BPW; ++bi)
-            if (all_blocks || warp * BPW + bi < a.nblk_gu) {
-              block_mma<BG, GS>(st0, st0 + GRP, sb0 + g8, sb0 + 8 + g8, warp * BPW + bi, uoff, xbf[bi], xs[bi],
-                                xo[bi], acc0);
-              block_mma<BG, GS>(st1, st1 + GRP, sb1 + g8, sb1 + 8 + g8, warp * BPW + bi, uoff, xbf[bi], xs[bi],
-                                xo[bi], acc1);
-            }
-        } else {
-          if (ok0) item_mma(stg + (size_t)s0 * SB, acc0);
-          if (ok1) item_mma(stg + (size_t)s1 * SB, acc1);
+          for (int u = 0; u < 8; ++u) {
+            bf[u][0] = row ? ld_pair(row + 16 * u) : 0u;
+            bf[u][1] = row ? ld_pair(row + 16 * u + 8) : 0u;
+          }
+#pragma unroll
+          for (int G = 0; G < 8 / GS; ++G) {
+            const int gi = kb * (8 / GS) + G;
+            xs[G][0] = xsum[(gi * a.T + n0) * 2];
+            xo[G][0] = xsum[(gi * a.T + n0) * 2 + 1];
+            xs[G][1] = xsum[(gi * a.T + n1) * 2];
+            xo[G][1] = xsum[(gi * a.T + n1) * 2 + 1];
+          }
+          block_mma<BG, GS>(st, st + GRP, sbs + g8, sbs + 8 + g8, kb, uoff, bf, xs, xo, acc);
         }
       }
-      int nent = 0;
-      if (ok0) {
-        *reinterpret_cast<float4*>(&red[((size_t)warp * 32 + lane) * 4]) =
-            make_float4(acc0[0], acc0[1], acc0[2], acc0[3]);
-        if (tid == 0) rmeta[0] = RedMeta{e0, 0, a.T, it0 % jt_n};
-        nent = 1;
-      }
-      if (ok1) {
-        *reinterpret_cast<float4*>(&red[(((size_t)nent * kFuConsumers + warp) * 32 + lane) * 4]) =
-            make_float4(acc1[0], acc1[1], acc1[2], acc1[3]);
-        if (tid == 0) rmeta[nent] = RedMeta{e1, 0, a.T, it1 % jt_n};
-        ++nent;
-      }
+      *reinterpret_cast<float4*>(&red[((size_t)warp * 32 + lane) * 4]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&empty[s0]);
-        if (two) mbar_arrive(&empty[s1]);
-      }
-      if (nent == 0) continue;
-      consumers_sync(kFuConsumers * 32);
-      // eight consecutive lanes hold the eight columns of one (entry, token);
-      // h is stored scaled by 2^-a of its down pair slot (exact: a power of
-      // two), with the partial sums (sum h, sum 128 h 2^-a) of the eight
-      for (int base = warp * 32; base < nent * nflush; base += kFuConsumers * 32) {
-        const int idx = base + lane;
-        const bool act = idx < nent * nflush;
-        const int en = act ? idx / nflush : 0, n = act ? (idx % nflush) >> 3 : 0, j = idx & 7;
-        const RedMeta m = rmeta[en];
-        const int pos = act ? s_tok[m.ei * kDenseMaxTokens + n] : -1;  // -1 for absent tokens
-        const int src = 4 * j + (n >> 1), c = n & 1;
-        const float* rp = red + (size_t)en * kFuConsumers * 32 * 4;
-        float gate = 0.f, up = 0.f;
-#pragma unroll
-        for (int w = 0; w < kFuConsumers; ++w) {
-          gate += rp[(w * 32 + src) * 4 + c];
-          up += rp[(w * 32 + src) * 4 + 2 + c];
-        }
+      if (lane == 0) mbar_arrive(&gempty[s]);
+      group_sync(gg);
+      // warp wg takes tokens wg, wg + 4, ...: lane 4 j + w holds column j's
+      // gate/up partial of the group's warp w; shuffles sum the four warps,
+      // then (sum h, sum 128 h 2^-a) over the eight columns
+      for (int n = wg; n < a.T; n += kGuGroupWarps) {
+        const int j = lane >> 2, w = lane & 3;
+        const float* rp = red + ((size_t)(gg * kGuGroupWarps + w) * 32 + 4 * j + (n >> 1)) * 4;
+        float gate = rp[n & 1], up = rp[2 + (n & 1)];
+        gate += __shfl_xor_sync(0xffffffffu, gate, 1);
+        up += __shfl_xor_sync(0xffffffffu, up, 1);
+        gate += __shfl_xor_sync(0xffffffffu, gate, 2);
+        up += __shfl_xor_sync(0xffffffffu, up, 2);
         const float hv = gate / (1.0f + expf(-gate)) * up;
-        const int kcol = m.jt * 8 + j, kk = kcol & 127;
+        const int kcol = jt * 8 + j, kk = kcol & 127;
         const bool eighth = PairShift<BD>::a(2 * (kk >> 4) + ((kk & 15) >> 3)) == 3;
         const uint16_t hb = f32_to_bf16_rne(eighth ? hv * 0.125f : hv);
         const float hsv = __uint_as_float((uint32_t)hb << 16);
         float sx = eighth ? 8.0f * hsv : hsv, so = 128.0f * hsv;
 #pragma unroll
-        for (int o = 1; o < 8; o <<= 1) {
+        for (int o = 4; o < 32; o <<= 1) {
           sx += __shfl_xor_sync(0xffffffffu, sx, o);
           so += __shfl_xor_sync(0xffffffffu, so, o);
         }
-        if (pos >= 0) {
-          a.h[(int64_t)pos * Ip + kcol] = hb;
-          if (j == 0) *reinterpret_cast<float2*>(a.hpart + 2 * ((int64_t)pos * (Ip / 8) + m.jt)) = make_float2(sx, so);
+        const int pos = s_tok[e * kDenseMaxTokens + n];  // -1: the token does not route here
+        if (ok && !timed_out && pos >= 0) {
+          if (w == 0) a.h[(int64_t)pos * Ip + kcol] = hb;
+          if (lane == 0) *reinterpret_cast<float2*>(a.hpart + 2 * ((int64_t)pos * (Ip / 8) + jt)) = make_float2(sx, so);
         }
       }
-      consumers_sync(kFuConsumers * 32);
-      // publish: the items' h columns are written (CTA barrier, then a release add per item)
-      if (tid == 0)
-        for (int en = 0; en < nent; ++en) red_release_add(ready + rmeta[en].ei, 1u);
+      group_sync(gg);  // the item's h columns are written; red is free again
+      if (wg == 0 && lane == 0) {  // hand the item to the producer warp's publish service
+        s_pub_e[gg][handed % kGuPubRing] = ok && !timed_out ? e : -1;
+        __threadfence_block();
+        *reinterpret_cast<volatile int*>(&s_pub_cnt[gg]) = handed + 1;
+      }
+      ++handed;
     }
-  } else if (nrt > 0) {
-    // ---------------- down + combine -> y, experts as they complete ----------------
+  }
+  consumers_sync(kFuConsumers * 32);  // every group is done with x' and red
+
+  // ---------------- down + combine -> y, experts in order as they complete ----------------
+  if (has_rt) {
     const int ngd = Ip / a.g;
     uint16_t* hs = reinterpret_cast<uint16_t*>(xh);
     float2* hsum = reinterpret_cast<float2*>(xh + (size_t)np * Ip * 2);
     const int GRP = 8 * (int)a.rb_d;
     const int uoff = thread_unit_off<BD>(t4, g8);
-    const int kq = warp % kDnKSplit, grp = warp / kDnKSplit, ngrp = kFuConsumers / kDnKSplit;
-    float yacc[kFuRtMax][4];
-#pragma unroll
-    for (int r = 0; r < kFuRtMax; ++r) yacc[r][0] = yacc[r][1] = yacc[r][2] = yacc[r][3] = 0.f;
-    // entries still to take (all of the pass: an entry whose slot is not
-    // valid is taken at once and skipped, so that its stage is released)
+    const int kq = warp % kDnKSplit, grp = warp / kDnKSplit;
+    float yacc[4] = {0.f, 0.f, 0.f, 0.f};
     unsigned long long pending = n_act >= 64 ? ~0ull : ((1ull << n_act) - 1ull);
-    int low = 0;  // lowest entry not yet taken (the stages hold entries low .. low + NS - 1)
+    int low = 0;  // lowest entry not yet taken (the stages hold entries low .. low + NSD - 1)
     const long long t0 = clock64();
     const int cpr = Ip / 8, cpg = a.g / 8, jt_i = a.I / 8;
     while (pending != 0ull) {
-      // which entries of the window have every gate/up item published
+      // the run of entries from the lowest pending one whose every gate/up
+      // item is published (an entry whose slot is not valid counts as done);
+      // taking entries in order keeps each warp's sum order fixed
       if (warp == 0) {
         unsigned long long m = 0ull;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int i = lane + 32 * q;
           bool r = false;
-          if (i < n_act && i < low + NS && ((pending >> i) & 1ull))
+          if (i < n_act && i < low + NSD && ((pending >> i) & 1ull))
             r = !slot_ok(a, s_slot[i]) || ld_acquire_u32(ready + i) == (unsigned)jt_n;
           m |= (unsigned long long)__ballot_sync(0xffffffffu, r) << (32 * q);
         }
+        const unsigned long long run = ~(m >> low);
+        const int len = run == 0ull ? 64 - low : __ffsll((long long)run) - 1;
+        const unsigned long long take = len >= 64 ? ~0ull : (((1ull << len) - 1ull) << low);
         if (lane == 0) {
-          s_ready = m;
+          s_ready = take;
           s_npl = 0;
-          if (m == 0ull && clock64() - t0 > a.wait_limit) s_timeout = 1;
+          if (take == 0ull && clock64() - t0 > a.wait_limit) s_timeout = 1;
         }
       }
       consumers_sync(kFuConsumers * 32);
@@ -389,7 +451,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
         break;
       }
       if (now == 0ull) {
-        __nanosleep(64);
+        __nanosleep(32);
         continue;
       }
       // the flat pairs of the newly complete experts
@@ -403,23 +465,23 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
       // their h rows (already scaled by 2^-a; padding columns zeroed) and the
       // per-(pair, group) epilogue sums from the per-8-column partials, all
       // loads of a thread in flight together
-      for (int b0 = tid; b0 < npl * cpr; b0 += 4 * kFuConsumers * 32) {
-        uint4 v[4];
-        int dst[4];
+      for (int b0 = tid; b0 < npl * cpr; b0 += 2 * kFuConsumers * 32) {
+        uint4 v[2];
+        int dsti[2];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 2; ++u) {
           const int idx = b0 + u * kFuConsumers * 32;
-          dst[u] = -1;
+          dsti[u] = -1;
           v[u] = make_uint4(0u, 0u, 0u, 0u);
           if (idx < npl * cpr) {
             const int p = s_plist[idx / cpr], c = idx % cpr;
-            dst[u] = p * cpr + c;
+            dsti[u] = p * cpr + c;
             if (8 * c < a.I) v[u] = __ldcg(reinterpret_cast<const uint4*>(a.h + (int64_t)p * Ip) + c);
           }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (dst[u] >= 0) reinterpret_cast<uint4*>(hs)[dst[u]] = v[u];
+        for (int u = 0; u < 2; ++u)
+          if (dsti[u] >= 0) reinterpret_cast<uint4*>(hs)[dsti[u]] = v[u];
       }
       for (int task = tid; task < npl * ngd; task += kFuConsumers * 32) {
         const int p = s_plist[task / ngd], G = task % ngd;
@@ -437,24 +499,18 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
         hsum[p * ngd + G] = make_float2(sx, so);
       }
       consumers_sync(kFuConsumers * 32);
-      // warps w and w + kDnKSplit split K the same way; the groups take the
-      // ready experts in turn, each over all of the CTA's row tiles
-      int nth = 0;
+      // warps w, w + kDnKSplit, ... split K the same way; entry i belongs to
+      // warp group i % kFuDnGroups
       for (int i = low; i < n_act; ++i) {
         if (!((now >> i) & 1ull)) continue;
-        const bool valid = slot_ok(a, s_slot[i]);
-        const bool mine = valid && (nth % ngrp) == grp;
-        nth += valid ? 1 : 0;
-        const int s = i % NS;
-        if (!timed_out && !mbar_wait_bounded(&full[s], (uint32_t)((i / NS) & 1), a.wait_limit)) timed_out = true;
-        if (mine && !timed_out) {
-          const uint8_t* st = stg + (size_t)s * SB;
+        const int s = i % NSD;
+        if (!timed_out && !mbar_wait_bounded(&dfull[s], (uint32_t)((i / NSD) & 1), a.wait_limit)) timed_out = true;
+        if (!timed_out && slot_ok(a, s_slot[i]) && (i % kFuDnGroups) == grp) {
+          const uint8_t* st = dst_ + (size_t)s * SBD;
+          const uint32_t* sbs = reinterpret_cast<const uint32_t*>(st + 2 * GRP);
           const int pb = s_tok[i * kDenseMaxTokens + g8];
           const int p0 = s_tok[i * kDenseMaxTokens + 2 * t4], p1 = s_tok[i * kDenseMaxTokens + 2 * t4 + 1];
-          const float w0 = p0 >= 0 ? s_w[p0] : 0.f, w1 = p1 >= 0 ? s_w[p1] : 0.f;
-          float acc[kFuRtMax][4];
-#pragma unroll
-          for (int r = 0; r < kFuRtMax; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
           for (int kb = kq; kb < a.nblk_d; kb += kDnKSplit) {
             uint32_t bf[8][2];
             float xs1[8 / GS][2], xo1[8 / GS][2];
@@ -474,55 +530,40 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
               xs1[G][1] = v1.x;
               xo1[G][1] = v1.y;
             }
-#pragma unroll
-            for (int r = 0; r < kFuRtMax; ++r)
-              if (r < nrt) {
-                const uint8_t* tile = st + (size_t)r * a.tile_d;
-                const uint32_t* sbs = reinterpret_cast<const uint32_t*>(tile + 2 * GRP);
-                block_mma<BD, GS>(tile, tile + GRP, sbs + g8, sbs + 8 + g8, kb, uoff, bf, xs1, xo1, acc[r]);
-              }
+            block_mma<BD, GS>(st, st + GRP, sbs + g8, sbs + 8 + g8, kb, uoff, bf, xs1, xo1, acc);
           }
-#pragma unroll
-          for (int r = 0; r < kFuRtMax; ++r) {
-            yacc[r][0] += w0 * acc[r][0];
-            yacc[r][1] += w1 * acc[r][1];
-            yacc[r][2] += w0 * acc[r][2];
-            yacc[r][3] += w1 * acc[r][3];
-          }
+          const float w0 = p0 >= 0 ? s_w[p0] : 0.f, w1 = p1 >= 0 ? s_w[p1] : 0.f;
+          yacc[0] += w0 * acc[0];
+          yacc[1] += w1 * acc[1];
+          yacc[2] += w0 * acc[2];
+          yacc[3] += w1 * acc[3];
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+        if (lane == 0) mbar_arrive(&dempty[s]);
       }
       pending &= ~now;
       while (low < n_act && !((pending >> low) & 1ull)) ++low;
       consumers_sync(kFuConsumers * 32);  // s_ready, s_plist and the h rows are read
     }
-    // y rows of the CTA's tiles: the sum over the warps (fixed order)
-#pragma unroll
-    for (int r = 0; r < kFuRtMax; ++r)
-      if (r < nrt)
-        *reinterpret_cast<float4*>(&red[(((size_t)r * kFuConsumers + warp) * 32 + lane) * 4]) =
-            make_float4(yacc[r][0], yacc[r][1], yacc[r][2], yacc[r][3]);
+    // y rows of the CTA's tile: the sum over the warps (fixed order)
+    *reinterpret_cast<float4*>(&red[((size_t)warp * 32 + lane) * 4]) = make_float4(yacc[0], yacc[1], yacc[2], yacc[3]);
     consumers_sync(kFuConsumers * 32);
-    for (int i = tid; i < nrt * a.T * 16; i += kFuConsumers * 32) {
-      const int r = i / (a.T * 16), rem = i % (a.T * 16), tok = rem >> 4, row = rem & 15;
+    for (int i = tid; i < a.T * 16; i += kFuConsumers * 32) {
+      const int tok = i >> 4, row = i & 15;
       const int src = 4 * (row & 7) + (tok >> 1), c = (row >> 3) * 2 + (tok & 1);
-      const float* rp = red + (size_t)r * kFuConsumers * 32 * 4;
       float sum = 0.f;
 #pragma unroll
-      for (int w = 0; w < kFuConsumers; ++w) sum += rp[(w * 32 + src) * 4 + c];
-      float* yp = a.y + (int64_t)tok * a.H + (rt0 + r) * 16 + row;
+      for (int w = 0; w < kFuConsumers; ++w) sum += red[(w * 32 + src) * 4 + c];
+      float* yp = a.y + (int64_t)tok * a.H + rt * 16 + row;
       *yp = a.y_overwrite ? sum : *yp + sum;
     }
-  }
-  if (dn_role) {
-    // the last down CTA to leave zeroes the control block for the next launch
+    // the last CTA with a down tile to leave zeroes the control block for the next launch
     consumers_sync(kFuConsumers * 32);
     if (tid == 0) {
       unsigned* depart = a.ctl + kCtlDepart;
       __threadfence();
       const unsigned old = atomicAdd(depart, 1u);
-      if (old == (unsigned)a.fu_n_dn - 1u) {
+      if (old == (unsigned)n_rt - 1u) {
         for (int i = 0; i < kMaxCtaExperts; ++i) ready[i] = 0u;
         *depart = 0u;
         __threadfence();
@@ -551,10 +592,10 @@ static cudaError_t launch_fused_t(const FfnArgs& a, int grid, size_t smem, cudaS
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   void* argv[] = {const_cast<void*>(static_cast<const void*>(&a))};
-  // co-residency of every CTA is required (the down CTAs wait for the gate/up
-  // CTAs): always cooperative; early launch behind the previous kernel as
-  // well where the driver accepts the combination (remembered after the
-  // first refusal)
+  // co-residency of every CTA is required (down work waits for other CTAs'
+  // gate/up items): always cooperative; early launch behind the previous
+  // kernel as well where the driver accepts the combination (remembered after
+  // the first refusal)
   static int pdl_refused = 0;
   if (!__atomic_load_n(&pdl_refused, __ATOMIC_RELAXED)) {
     cfg.numAttrs = 2;
@@ -587,56 +628,51 @@ static cudaError_t fused_bd(const FfnArgs& a, int bd, int bpw, int gs, int grid,
   return fused_bpw<BG, 6>(a, bpw, gs, grid, smem, st);
 }
 
-// Role split, stage counts and shared memory of the fused kernel for this
-// call (into a); false when the fused path does not apply (the caller then
+// Stage sizes and counts of the fused kernel for this call (into a), its
+// shared memory; false when the fused path does not apply (the caller then
 // uses the two-kernel path).
 bool ffn_fused_plan(FfnArgs& a, const moe_layer_desc& d, int num_sms, size_t& smem) {
   if (!(a.T <= kDenseMaxTokens && a.T * d.k <= kMaxCtaExperts) || a.ctl == nullptr) return false;
   if (a.L.nblk_gu > 2 * kFuConsumers || d.E > 1024 || d.I % 8) return false;
+  if (d.H / 16 > num_sms) return false;
   const int grid = num_sms;
-  const int n_rt = d.H / 16, jt_n = d.I / 8;
   int max_pass = a.pass_len < d.E ? a.pass_len : d.E;
   if (a.T * d.k < max_pass) max_pass = a.T * d.k;
   if (max_pass < 1) max_pass = 1;
-  // down CTAs in proportion to the down projection's share of the bytes
-  const double gu_b = (double)jt_n * a.L.tile_gu, dn_b = (double)n_rt * a.L.tile_d;
-  int want = (int)(grid * dn_b / (gu_b + dn_b) + 0.5);
-  if (want < 1) want = 1;
-  int rpd = (n_rt + want - 1) / want;
-  if (rpd > kFuRtMax) return false;
-  const int n_dn = (n_rt + rpd - 1) / rpd;
-  if (n_dn >= grid) return false;
-  const int n_gu = grid - n_dn;
-  a.fu_n_dn = n_dn;
-  a.fu_rt_per_dn = rpd;
   a.gu_stage_bytes = (int)round_up(a.L.tile_gu, 128);
-  a.d_stage_bytes = (int)round_up((int64_t)rpd * a.L.tile_d, 128);
+  a.d_stage_bytes = (int)round_up(a.L.tile_d, 128);
   {
-    // x in the gate/up CTAs; h (scaled, rows padded to 128-blocks) and the
-    // per-(pair, group) sums in the down CTAs
+    // x' and its per-(group, token) sums in the gate/up phase; h (scaled,
+    // rows padded to 128-blocks) and the per-(pair, group) sums in the down phase
     const size_t np = (size_t)a.T * d.k, Ip = (size_t)a.L.nblk_d * 128;
-    const size_t xb = (size_t)a.T * d.H * 2, hb = np * Ip * 2 + np * (Ip / d.group) * 8;
+    const size_t xb = (size_t)a.T * d.H * 2 + (size_t)(d.H / d.group) * a.T * 8;
+    const size_t hb = np * Ip * 2 + np * (Ip / d.group) * 8;
     a.xh_stage_bytes = (int)round_up((int64_t)(xb > hb ? xb : hb), 128);
   }
-  const size_t fixed = (size_t)a.xh_stage_bytes + (size_t)kFuRedFloats * 4 + kRedBatch * sizeof(RedMeta) +
-                       kFuTableBytes + (size_t)d.E * 4 + 16;
+  // the most gate/up items a CTA can get: a CTA without a down tile takes the
+  // whole quota of (gate/up + down bytes) / grid
+  const int n_rt = d.H / 16, jt_n = d.I / 8;
+  const double tot = (double)max_pass * jt_n * a.L.tile_gu + (double)n_rt * max_pass * a.L.tile_d;
+  const int64_t items_max = (int64_t)(tot / grid / a.L.tile_gu) + 2;
+  if ((items_max + kGuGroups - 1) / kGuGroups > kGuPubRing) return false;
+  const size_t fixed = (size_t)a.xh_stage_bytes + (size_t)kFuRedFloats * 4 + kFuTableBytes + (size_t)d.E * 4 + 16;
   const size_t cap = 220 * 1024;
-  if (fixed + (size_t)2 * a.gu_stage_bytes + 32 > cap) return false;
-  const size_t area = cap - fixed;
-  const int64_t items_per_cta = ((int64_t)max_pass * jt_n + n_gu - 1) / n_gu;
-  int nsg = (int)(area / (a.gu_stage_bytes + 16));
-  if (nsg > items_per_cta) nsg = (int)items_per_cta;
-  if (nsg < 2) nsg = 2;
-  int nsd = (int)(area / (a.d_stage_bytes + 16));
-  if (nsd > max_pass) nsd = max_pass;
-  if (nsd < 1) return false;
+  constexpr int kMinDn = kFuDnGroups;
+  if (fixed + 2 * (size_t)a.gu_stage_bytes + kMinDn * (size_t)a.d_stage_bytes + 64 > cap) return false;
+  // down stages: every expert of the pass if possible; gate/up stages: every
+  // item of the CTA if possible, at least two (a pair is computed at once)
+  int nsd = max_pass > kMinDn ? max_pass : kMinDn;
+  int nsg = (int)(items_max < 2 ? 2 : items_max);
+  while ((size_t)nsd * a.d_stage_bytes + (size_t)nsg * a.gu_stage_bytes + fixed + 16 * (nsd + nsg) > cap) {
+    if (nsg > nsd && nsg > 2) --nsg;
+    else if (nsd > kMinDn) --nsd;
+    else if (nsg > 2) --nsg;
+    else return false;
+  }
   a.gu_nstage = nsg;
   a.d_nstage = nsd;
-  const size_t sg = (size_t)nsg * a.gu_stage_bytes, sd = (size_t)nsd * a.d_stage_bytes;
-  a.fu_stage_area = (int)round_up((int64_t)(sg > sd ? sg : sd), 128);
-  const int nbar = nsg > nsd ? nsg : nsd;
-  smem = (size_t)a.fu_stage_area + fixed + 16 * (size_t)nbar;
-  return smem <= cap + 16 * (size_t)nbar;
+  smem = (size_t)nsg * a.gu_stage_bytes + (size_t)nsd * a.d_stage_bytes + fixed + 16 * (nsd + nsg);
+  return true;
 }
 
 cudaError_t launch_ffn_fused(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st) {

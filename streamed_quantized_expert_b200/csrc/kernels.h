@@ -43,7 +43,6 @@ struct FfnArgs {
   int ng_gu, ng_d, nblk_gu, nblk_d;
   int gu_stage_bytes, d_stage_bytes, gu_nstage, d_nstage;
   int xh_stage_bytes;  // fused kernel: shared region for x (gate/up CTAs) or h (down CTAs)
-  int fu_n_dn, fu_rt_per_dn, fu_stage_area;  // fused kernel: down CTAs, their 16-row tiles, stage bytes
   long long wait_limit;  // clock-cycle limit of every bounded device wait (wait_limit_cycles())
 };
 

@@ -16,16 +16,19 @@
 // Warp roles (832 threads):
 //   0-15  dequant: warp w = (K quarter w / 4, TMEM lane quadrant w % 4), lane
 //         = weight row; unpack its row's codes of a 128-input block (landed by
-//         TMA), w = fma(scale, q, bias) in bf16x2 with one rounding, and store
-//         the quarter's 16 bf16 pairs (inputs 32 q .. 32 q + 31) to the A
+//         TMA), w = fma(scale, q, bias) in fp16x2 with one rounding, and store
+//         the quarter's 16 fp16 pairs (inputs 32 q .. 32 q + 31) to the A
 //         operand in TMEM with one tcgen05.st (lane = row, column = input / 2);
 //   16-23 epilogue: TMEM -> registers (warp i reads TMEM lanes 32 (i % 4)..;
 //         the two warps of a quadrant take alternate 16-column chunks);
 //   24    producer: TMA loads of codes, (scale, bias) words and token rows;
-//   25    MMA issuer (one thread): tcgen05.mma kind::f16 (bf16 x bf16 -> fp32
+//   25    MMA issuer (one thread): tcgen05.mma kind::f16 (fp16 x fp16 -> fp32
 //        in TMEM) with A from TMEM and B (token rows) from shared memory,
 //        M = 128, N = tokens rounded up to 16, K = 16 per instruction;
 //        tcgen05.commit frees stages and publishes accumulators.
+// The operands are fp16 (11 significant bits): the token rows come sorted and
+// converted by moe_sort, h is written in fp16 by the gate/up epilogue, and the
+// weights are dequantised to fp16, so each rounding is 4x finer than bf16's.
 // Accumulators are double-buffered in TMEM (2 x 128 columns), so the epilogue
 // of one tile overlaps the MMAs of the next; the two A buffers take 2 x 64
 // more columns.  With A in TMEM, shared memory carries only the TMA traffic
@@ -36,6 +39,7 @@
 // the copies it issued, the MMA thread waits for its MMAs, and TMEM is freed.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -126,14 +130,14 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulator (bits 4-5 = 1), A and
-// B bf16 (bits 7-9 = 1, bits 10-12 = 1), both K-major (bits 15, 16 = 0),
+// B fp16 (bits 7-9 = 0, bits 10-12 = 0), both K-major (bits 15, 16 = 0),
 // N >> 3 in bits 17-22, M >> 4 in bits 24-28.
-__device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+__device__ __forceinline__ uint32_t idesc_f16(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// D (TMEM, fp32) (+)= A . B^T, M x N x 16: A (M x 16 bf16: lane m, columns k / 2) in TMEM at a_tmem,
-// B (N x 16 bf16, K-major, 128-byte swizzled) in shared memory; kind::f16.
+// D (TMEM, fp32) (+)= A . B^T, M x N x 16: A (M x 16 fp16: lane m, columns k / 2) in TMEM at a_tmem,
+// B (N x 16 fp16, K-major, 128-byte swizzled) in shared memory; kind::f16.
 __device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                              uint32_t accumulate) {
   asm volatile(
@@ -190,7 +194,7 @@ __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, volatile
 }
 
 // K quarter CQ (inputs 32 CQ .. 32 CQ + 31) of weight row r (0..127 of the
-// tile) for one 128-input block -> 16 bf16 pairs, stored at TMEM columns
+// tile) for one 128-input block -> 16 fp16 pairs, stored at TMEM columns
 // 16 CQ .. 16 CQ + 15 of this thread's lane (ta: the warp's lanes, A buffer
 // column 0).  Codes: the tile's 16 8-row groups, each 4 units x 8 rows x B
 // words (unit t of row rr at word (8 t + sigma) B); scale/bias: per 16-row
@@ -202,24 +206,27 @@ __device__ __forceinline__ void pf_dequant_quarter(const uint8_t* cs, const uint
   const int g8 = r >> 3, rr = r & 7;
   constexpr int GI = (CQ * GPB) / 4;  // the quarter's (single) group within the block
   const uint32_t word = sbs[(r >> 4) * 16 * GPB + GI * 16 + (r & 15)];
-  const uint32_t s2 = (word & 0xFFFFu) * 0x10001u, b2 = (word >> 16) * 0x10001u;
-  const __nv_bfloat162 sc = *reinterpret_cast<const __nv_bfloat162*>(&s2);
-  const __nv_bfloat162 bi = *reinterpret_cast<const __nv_bfloat162*>(&b2);
-  const __nv_bfloat162 sc8 = __hmul2(sc, __floats2bfloat162_rn(0.125f, 0.125f));
-  const uint32_t m = kMagic;
-  const __nv_bfloat162 m128 = *reinterpret_cast<const __nv_bfloat162*>(&m);
+  // bf16 scale and bias -> fp16 (exact for normal fp16 magnitudes); codes
+  // unpacked onto the fp16 magic 1024: q = p - 1024 exactly, then one fp16
+  // rounding of s * q + b
+  const float sf = bf16_lo(word), bf = bf16_hi(word);
+  const __half2 sc = __half2half2(__float2half_rn(sf));
+  const __half2 sc8 = __half2half2(__float2half_rn(sf * 0.125f));
+  const __half2 bi = __half2half2(__float2half_rn(bf));
+  const uint32_t m = kMagic16;
+  const __half2 m1024 = *reinterpret_cast<const __half2*>(&m);
   uint32_t out[16];
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
     uint32_t w[B], p[16];
     load_unit<B>(cs + (g8 * 32 + 8 * t + unit_sigma<B>(t, rr)) * 4 * B, w);
-    unpack_unit<B>(w, p);
+    unpack_unit<B, kMagic16>(w, p);
 #pragma unroll
     for (int mm = 0; mm < 4; ++mm) {
       const int i = 4 * CQ + mm;
-      const __nv_bfloat162 scale = PairShift<B>::a(i) == 3 ? sc8 : sc;
-      const __nv_bfloat162 q = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&p[i]), m128);
-      const __nv_bfloat162 v = __hfma2(scale, q, bi);
+      const __half2 scale = PairShift<B>::a(i) == 3 ? sc8 : sc;
+      const __half2 q = __hsub2(*reinterpret_cast<const __half2*>(&p[i]), m1024);
+      const __half2 v = __hfma2(scale, q, bi);
       out[4 * mm + t] = *reinterpret_cast<const uint32_t*>(&v);
     }
   }
@@ -387,7 +394,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
         const PfTile tl = tile_at(t);
         const int npad = (tl.n + 15) & ~15;
-        const uint32_t idesc = idesc_bf16(kPfBM, npad);
+        const uint32_t idesc = idesc_f16(kPfBM, npad);
         if (!pf_wait(&accempty[c], pc ^ 1u, &s_abort, a.wait_limit)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(c * kPfBN);
@@ -496,7 +503,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               const float x = __uint_as_float(v[i]);
               const float u = __shfl_xor_sync(0xffffffffu, x, 8);
               if (gate && n0 + i < tl.n)
-                a.h[(int64_t)(tl.row0 + n0 + i) * a.I + j] = f32_to_bf16_rne(__fdividef(x, 1.0f + __expf(-x)) * u);
+                a.h[(int64_t)(tl.row0 + n0 + i) * a.I + j] = f32_to_f16_sat(__fdividef(x, 1.0f + __expf(-x)) * u);
             }
           } else {
 #pragma unroll
@@ -569,13 +576,13 @@ bool encode_proj(CUtensorMap* q, CUtensorMap* sb, const uint8_t* proj, int64_t r
   return encode(sb, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, proj + 16 * rb, sd, ss, sbx, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-// Token rows (bf16 [rows][cols], row-major) for the MMA's B operand: boxes of
+// Token rows (fp16 [rows][cols], row-major) for the MMA's B operand: boxes of
 // 64 columns (128 bytes, 128-byte swizzle) x 32 rows.
 bool encode_rows(CUtensorMap* m, const uint16_t* base, int64_t rows, int cols) {
   const cuuint64_t d[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t s[1] = {(cuuint64_t)cols * 2};
   const cuuint32_t b[2] = {64, 32};
-  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, d, s, b, CU_TENSOR_MAP_SWIZZLE_128B);
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, d, s, b, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 size_t pf_smem_bytes(int bits, int gpb) {

@@ -468,7 +468,13 @@ __global__ void __launch_bounds__(1024) sort_scatter_kernel(const int32_t* __res
   }
 }
 
-// x_sorted[i] = x[pairs[i] / k]: one warp per row, 16-byte copies.
+// x_sorted[i] = fp16(x[pairs[i] / k]) (the tensor-core path's operand type):
+// one warp per row, 16-byte loads and stores, bf16 -> fp16 round to nearest
+// even, saturating at +-65504.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  return (uint32_t)f32_to_f16_sat(bf16_lo(v)) | ((uint32_t)f32_to_f16_sat(bf16_hi(v)) << 16);
+}
+
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ pairs, int n, int k,
                                    int H, uint16_t* __restrict__ xs) {
   const int lane = threadIdx.x & 31;
@@ -476,7 +482,10 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t
   if (row >= n) return;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(pairs[row] / k) * H);
   uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)row * H);
-  for (int c = lane; c < H / 8; c += 32) dst[c] = src[c];
+  for (int c = lane; c < H / 8; c += 32) {
+    const uint4 v = src[c];
+    dst[c] = make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
+  }
 }
 
 // ---------------------------------------------------------------------------

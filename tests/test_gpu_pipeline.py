@@ -1,7 +1,8 @@
 """All five stages with installs, through the runtime over the C ABI, against
 the oracle: decode with LRU misses installed from pinned host rows, decode
-with cache-aware substitution over two size classes, and a prefill chunk in
-passes of 64 experts with installs between passes."""
+with cache-aware substitution over two size classes, a prefill chunk in
+passes of 64 experts with installs between passes, and the mixed-class
+prefill-then-decode sequence."""
 import numpy as np
 import pytest
 import torch
@@ -110,4 +111,46 @@ def test_prefill_passes_with_installs(orc):
     assert st.installs > 0
     tok = np.array([0, 7, 100, T - 1])
     assert_close(y.cpu().numpy()[tok], orc.expert_ffn(x, H, I, g, 3, 3, ids, w, host_slots[0], tok), TOL)
+    assert st.check_dev_err() == 0
+
+
+def test_prefill_then_decode_sequence_two_classes(orc):
+    # the mixed-class sequence at reduced size: a prefill chunk through a 25%-resident two-class cache
+    # (passes of 64 experts, installs between passes), then decode steps with cache-aware substitution
+    # (L = 0.15) from the cache the prefill left; every layer's y, routing and slot table against the oracle
+    E, k, H, I, g, S, T, L = 256, 4, 256, 128, 64, 64, 96, 0.15  # a pass of 64 experts needs 64 slots
+    bits = [(4, 6), (4, 4)]
+    specs, host_slots = make(orc, 2, E, k, H, I, g, bits, S, R=7, seed=13)
+    st = Streamer(specs, S, max_tokens=T)
+    placed = initial_fill(st, 13, S)
+    models = []
+    for l in range(2):
+        m = orc.LruModel(E, S, slot_base=st.cache.layer_base(l))
+        m.place(*placed[l])
+        models.append(m)
+    for l in range(2):
+        x = synth.activations(13, l, T, H)
+        logits = synth.router_logits(13, l, T, E)
+        y = st.prefill_layer(l, dev(x.view(np.int16)), dev(logits), T)
+        ids, w, _ = orc.route(logits, k)
+        assert np.array_equal(st.ids[:T].cpu().numpy(), ids)
+        active = np.unique(ids).astype(np.int32)
+        assert active.size > 64  # at least two passes
+        for p in range(0, active.size, 64):
+            models[l].step(active[p:p + 64])
+        assert np.array_equal(st.table_dev[l].cpu().numpy(), models[l].table)
+        assert_close(y.cpu().numpy(), orc.expert_ffn(x, H, I, g, *bits[l], ids, w, host_slots[l]), TOL)
+    inst_prefill = st.installs
+    assert inst_prefill > 0
+    for step in range(6):
+        for l in range(2):
+            x = synth.activations(13, l, 1, H, step=step + 1)
+            logits = synth.router_logits(13, l, 1, E, step=step + 1)
+            table_before = st.table_dev[l].cpu().numpy()
+            assert np.array_equal(table_before, models[l].table)
+            y = st.decode_layer(l, dev(x.view(np.int16)), dev(logits), 1, L=L)
+            ids, w, _ = orc.route(logits, k, L, table_before)
+            assert np.array_equal(st.ids[:1].cpu().numpy(), ids)
+            models[l].step(np.sort(ids[0]).astype(np.int32))
+            assert_close(y.cpu().numpy(), orc.expert_ffn(x, H, I, g, *bits[l], ids, w, host_slots[l]), TOL)
     assert st.check_dev_err() == 0
