@@ -739,8 +739,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4),
                      "traffic": recorded_traffic("ffn_fused_kernel") if T * k <= 64 and T <= 8 else None,
-                     "kernel": ("ffn_fused_kernel (one launch per layer: gate/up + SwiGLU CTAs and down + combine "
-                                "CTAs linked by per-expert readiness counters)" if T <= 8 and T * k <= 64 else
+                     "kernel": ("ffn_fused_kernel (one launch per layer: every CTA gate/up + SwiGLU items, then the "
+                                "first H/16 CTAs a down + combine tile, over launch-tagged h words)" if T <= 8 and T * k <= 64 else
                                 "pf_gemm_kernel (tcgen05 grouped GEMM: gate/up + SwiGLU, down) + combine, per layer"
                                 if T >= 32 else
                                 "moe_expert_ffn (gate/up+SwiGLU kernel + down kernel), per layer"),

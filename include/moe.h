@@ -131,14 +131,16 @@ moe_status moe_slot_layout(const moe_layer_desc* d, moe_slot_layout_t* out);
 
 /* Device workspace needed by moe_sort and moe_expert_ffn for up to
  * max_tokens tokens (0 if d is invalid).  One buffer of this size may be
- * shared by the two calls when they run in stream order.  Its first 512
- * bytes are a control block (the single-launch decode FFN's per-expert
- * readiness counters and its down CTAs' departure count): zero them once
- * after allocating the workspace (e.g. cudaMemset).  Every launch leaves them
- * at zero again, also one whose waits ran out; only a launch cut short on the
- * device (its context lost) can leave them otherwise, and a later call then
- * reports MOE_DEV_ERR_TIMEOUT instead of using them -- zero them after a
- * reported timeout.  The rest needs no initialisation. */
+ * shared by the two calls when they run in stream order.  Zero the whole
+ * buffer once after allocating it (e.g. cudaMemset).  Its head -- a 512-byte
+ * control block (the single-launch decode FFN's launch epoch and arrival
+ * count) and that kernel's h words, each tagged with its launch -- carries
+ * over from call to call; every launch leaves the head consistent, also one
+ * whose waits ran out.  Only a launch cut short on the device (its context
+ * lost) or foreign writes can leave it otherwise; a later call then reports
+ * MOE_DEV_ERR_TIMEOUT instead of using stale values -- zero the whole buffer
+ * after a reported timeout.  Calls with different layer descriptions may
+ * share the buffer if it is large enough for each. */
 size_t moe_workspace_bytes(const moe_layer_desc* d, int32_t max_tokens);
 
 /* Stage 1.  Cache-aware top-k (BigMoeOnEdge note: every expert already in
@@ -236,10 +238,11 @@ moe_status moe_expert_ffn(const uint16_t* x, int32_t T, const moe_layer_desc* d,
  *   - the first call on a device looks up the array's device address (with
  *     that device current); make that first call outside any stream capture;
  *   - every call shares the one array and leaves its contents behind; the
- *     array's first 512 bytes (the control block that moe_workspace_bytes
- *     describes) are cleared on `stream` (cudaMemsetAsync) before each call's
- *     kernels, the rest needs no initialisation; calls whose kernels overlap
- *     on the GPU (e.g. on two streams at once) race on the array.
+ *     head that moe_workspace_bytes describes as carried over (control block
+ *     and tagged h words) is cleared on `stream` (cudaMemsetAsync) before
+ *     each call's kernels, the rest needs no initialisation; calls whose
+ *     kernels overlap on the GPU (e.g. on two streams at once) race on the
+ *     array.
  * Allocates nothing. */
 moe_status moe_expert_ffn_noalloc(const uint16_t* x, int32_t T, const moe_layer_desc* d, const void* pool,
                                   int32_t n_slots, const int32_t* slot_table, const int32_t* ids, const float* w,
@@ -278,9 +281,11 @@ const char* moe_status_string(moe_status s);
 /* Which kernels moe_expert_ffn runs on the current device for a call over
  * all E experts of a layer of shape d with T tokens, with (has_x_sorted != 0)
  * or without x_sorted:
- *   MOE_PATH_FUSED_DECODE  one launch: gate/up + SwiGLU CTAs and down +
- *                          combine CTAs linked by per-expert readiness
- *                          counters (T <= 8, T*k <= 64)
+ *   MOE_PATH_FUSED_DECODE  one launch: every CTA runs its share of the
+ *                          gate/up + SwiGLU tiles, then (the first H/16
+ *                          CTAs) a down + combine tile over every expert,
+ *                          reading h words tagged with the launch
+ *                          (T <= 8, T*k <= 64)
  *   MOE_PATH_GEMV          gate/up + SwiGLU kernel, down kernel (+ combine
  *                          kernel for T > 64): tensor-core GEMV (mma.sync)
  *   MOE_PATH_TC_PREFILL    tcgen05/TMEM grouped GEMM fed by TMA (T >= 32,
@@ -292,7 +297,7 @@ int32_t moe_ffn_kernel_path(const moe_layer_desc* d, int32_t T, int32_t has_x_so
 
 /* Test/inspection: the limit, in SM clock cycles, of every bounded device
  * wait (a bulk copy that should land, a pipeline stage that should free up,
- * the single-launch decode FFN's readiness counters) in kernels launched afterwards
+ * the single-launch decode FFN's reads of other CTAs' h) in kernels launched afterwards
  * by this process; cycles <= 0 restores the default of 4e9 (about 2 s at the
  * top clock).  A wait that runs out sets MOE_DEV_ERR_TIMEOUT in dev_err and
  * the kernel returns; tests lower the limit to make such a wait run out

@@ -48,12 +48,15 @@ int device_sms() {
   return sms;
 }
 
-// Workspace: [control block (kWsControlBytes)][sort scratch | FFN scratch].
-// The control block must be zero before the first call with a workspace
-// (every fused launch then advances its arrival counter by its grid size);
-// the sort and FFN scratch overlap (different calls, stream-ordered).
+// Workspace: [control block (kWsControlBytes)][tagged h words][sort scratch |
+// FFN scratch].  The control block (the single-launch decode kernel's epoch
+// and arrival count) and the tagged h words (that kernel's h, each word
+// carrying its launch's tag) persist from call to call and are zeroed
+// together, once, before the first call; they sit at the same place for
+// every T.  The sort and FFN scratch overlap (different calls,
+// stream-ordered).
 struct WsCarve {
-  size_t sort, hb, h, o, total;
+  size_t sort, hb, h, o, tag, total;
 };
 
 // tc: the call may run the tensor-core path (x_sorted given), whose per-pair
@@ -61,6 +64,10 @@ struct WsCarve {
 WsCarve carve(const moe_layer_desc& d, int T, bool tc = true) {
   WsCarve c{};
   const int64_t np = (int64_t)T * d.k;
+  // the single-launch decode kernel's tagged h words, for its largest call
+  // (T * k <= 64): at the same place for every T, written by nothing else
+  const int64_t np_tag = 8 * (int64_t)d.k < 64 ? 8 * (int64_t)d.k : 64;
+  c.tag = (size_t)round_up(np_tag * padded_k(d.I) * 8, 256);
   c.sort = (size_t)round_up((int64_t)sort_ws_bytes((int)np, d.E), 256);
   // h (bf16, rows padded to 128-blocks) and its per-8-column partial sums
   c.hb = (size_t)round_up(np * padded_k(d.I) * 2, 256);
@@ -68,7 +75,7 @@ WsCarve carve(const moe_layer_desc& d, int T, bool tc = true) {
   // o: per-pair outputs of the tensor-core path (T >= kTcMinTokens) and of the GEMV path for T > 64
   c.o = ((tc && T >= kTcMinTokens) || T > kFusedMaxTokens) ? (size_t)round_up(np * d.H * 4, 256) : 0;
   const size_t ffn = c.h + c.o;
-  c.total = kWsControlBytes + (c.sort > ffn ? c.sort : ffn);
+  c.total = kWsControlBytes + c.tag + (c.sort > ffn ? c.sort : ffn);
   return c;
 }
 
@@ -126,6 +133,13 @@ size_t moe_workspace_bytes(const moe_layer_desc* d, int32_t max_tokens) {
 }
 
 // Workspace bytes of a call that passes no x_sorted (the GEMV / fused kernels).
+// Head of the workspace that persists from call to call (control block and
+// tagged h words): the bytes moe_expert_ffn_noalloc clears before each call.
+__attribute__((visibility("hidden"))) size_t moe_internal_workspace_persistent_bytes(const moe_layer_desc* d) {
+  if (check_desc(d) != MOE_OK) return 0;
+  return kWsControlBytes + carve(*d, 1).tag;
+}
+
 __attribute__((visibility("hidden"))) size_t moe_internal_workspace_bytes_no_tc(const moe_layer_desc* d,
                                                                                int32_t max_tokens) {
   if (check_desc(d) != MOE_OK || max_tokens < 0) return 0;
@@ -154,7 +168,7 @@ moe_status moe_sort(const int32_t* ids, const uint16_t* x, int32_t T, const moe_
   if (x && (!x_sorted || !aligned(x, 16) || !aligned(x_sorted, 16) || d->H % 8)) return MOE_ERR_INVALID;
   const WsCarve c = carve(*d, T);
   if (c.sort > 0 && (!ws || ws_bytes < c.total)) return MOE_ERR_CAPACITY;
-  void* scratch = c.sort > 0 ? static_cast<char*>(ws) + kWsControlBytes : nullptr;
+  void* scratch = c.sort > 0 ? static_cast<char*>(ws) + kWsControlBytes + c.tag : nullptr;
   return cuda_status(launch_sort(ids, x, T, d->k, d->E, d->H, offsets, pairs, active, n_active, x_sorted, scratch,
                                  stream));
 }
@@ -226,9 +240,11 @@ __attribute__((visibility("hidden"))) moe_status moe_internal_expert_ffn(
   a.pass_len = pass_len;
   a.y = y_accum;
   a.ctl = static_cast<unsigned*>(ws);
-  a.h = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + kWsControlBytes);
-  a.hpart = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsControlBytes + c.hb);
-  a.o = c.o ? reinterpret_cast<float*>(static_cast<char*>(ws) + kWsControlBytes + c.h) : nullptr;
+  char* const scr = static_cast<char*>(ws) + kWsControlBytes + c.tag;  // sort | FFN scratch
+  a.h = reinterpret_cast<uint16_t*>(scr);
+  a.hpart = reinterpret_cast<float*>(scr + c.hb);
+  a.o = c.o ? reinterpret_cast<float*>(scr + c.h) : nullptr;
+  a.htag = static_cast<char*>(ws) + kWsControlBytes;
   a.dev_err = dev_err;
   a.y_overwrite = overwrite ? 1 : 0;
   a.wait_limit = wait_limit_cycles();

@@ -540,7 +540,8 @@ int ffn_kernel_path(const moe_layer_desc& d, int T, bool has_x_sorted, int num_s
   a.pass_len = d.E;
   a.L = make_layout(d);
   unsigned ctl_stub = 0;
-  a.ctl = &ctl_stub;  // the plan only checks that a control block exists
+  a.ctl = &ctl_stub;  // the plan only checks that a control block and the tagged h region exist
+  a.htag = &ctl_stub;
   size_t smem = 0;
   if (ffn_fused_plan(a, d, num_sms, smem)) return 0;
   if (T >= kTcMinTokens && has_x_sorted && ffn_prefill_tc_shape_ok(d)) return 2;

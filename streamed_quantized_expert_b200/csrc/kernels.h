@@ -32,17 +32,19 @@ struct FfnArgs {
   float* y;
   uint16_t* h;    // workspace: [T*k][I] bf16 by sorted position (two-kernel path); the fused kernel
                   // uses [T*k][padded I] by flat pair, scaled by 2^-a of the down pair slot
-  float* hpart;   // workspace (fused kernel): [T*k][padded I / 8] (sum h, sum 128 h 2^-a) pairs
+  float* hpart;   // workspace: [T*k][padded I / 8] float pairs (unused by the fused kernel)
+  void* htag;     // workspace (fused kernel): [T*k][padded I] 64-bit words (bf16 h, launch tag)
   float* o;     // workspace: [T*k][H] fp32, by flat pair index (T > kFusedMaxTokens)
   int32_t* dev_err;
-  unsigned* ctl;    // workspace control block (readiness counters of the fused kernel)
+  unsigned* ctl;    // workspace control block (the fused kernel's 64-bit launch ticket counter)
   int y_overwrite;  // 1: y = result (single pass over all experts); 0: y += result
   Layout L;
   // filled by the launcher
   int64_t q_gu, q_d, tile_gu, tile_d, rb_gu, rb_d;
   int ng_gu, ng_d, nblk_gu, nblk_d;
   int gu_stage_bytes, d_stage_bytes, gu_nstage, d_nstage;
-  int xh_stage_bytes;  // fused kernel: shared region for x (gate/up CTAs) or h (down CTAs)
+  int xh_stage_bytes;  // fused kernel: shared region for x' and its sums, then (at h_stage_off) h
+  int h_stage_off;
   long long wait_limit;  // clock-cycle limit of every bounded device wait (wait_limit_cycles())
 };
 
@@ -88,7 +90,7 @@ bool ffn_prefill_tc_shape_ok(const moe_layer_desc& d);
 int ffn_kernel_path(const moe_layer_desc& d, int T, bool has_x_sorted, int num_sms);
 __global__ void combine_kernel(const FfnArgs a);
 int combine_grid(int T, int H, int num_sms);
-constexpr size_t kWsControlBytes = 512;  // head of the workspace: the fused kernel's readiness counters
+constexpr size_t kWsControlBytes = 512;  // head of the workspace: the fused kernel's launch ticket counter
 constexpr long long kDefaultWaitCycles = 4000000000ll;  // about 2 s at the top SM clock
 // Limit of the bounded device waits of kernels launched from now on
 // (moe_set_wait_limit_cycles; kDefaultWaitCycles unless a test lowered it).

@@ -53,14 +53,15 @@ namespace {
 
 constexpr int kPfBM = 128;      // weight rows per tile (MMA M)
 constexpr int kPfBN = 128;      // tokens per tile (MMA N, at most)
-constexpr int kPfABufs = 2;     // dequantised A buffers (in TMEM)
+constexpr int kPfABufs = 4;     // dequantised A buffers (in TMEM)
 constexpr int kPfDqWarps = 16;  // one per 8-row group of the 128-row tile
 constexpr int kPfEpiWarps = 8;  // two per TMEM lane quadrant, taking alternate 16-column chunks
 constexpr int kPfEpiWarp0 = kPfDqWarps, kPfProdWarp = kPfEpiWarp0 + kPfEpiWarps, kPfMmaWarp = kPfProdWarp + 1;
 constexpr int kPfThreads = (kPfMmaWarp + 1) * 32;
-constexpr int kPfTmemCols = 512;  // two accumulators of kPfBN fp32 columns, then two A buffers
+constexpr int kPfTmemCols = 512;  // two accumulators of kPfBN fp32 columns, then the A buffers
 constexpr int kPfAcol = 2 * kPfBN;  // first TMEM column of the A buffers
-constexpr int kPfAcols = 64;       // one A buffer: 128 inputs as bf16 pairs, 128 lanes = rows
+constexpr int kPfAcols = 64;       // one A buffer: 128 inputs as fp16 pairs, 128 lanes = rows
+static_assert(kPfAcol + kPfABufs * kPfAcols <= kPfTmemCols, "TMEM columns");
 constexpr int kPfXHalf = kPfBN * 128;   // one 64-input half of a token stage: 128 rows x 128 B
 // load stages (codes + scale/bias + token rows) that fit the shared memory
 __host__ __device__ constexpr int pf_stages(int bits) { return bits == 6 ? 4 : 5; }
@@ -249,7 +250,8 @@ struct PfTile {
 template <int B, int GPB, bool GU>
 __global__ void __launch_bounds__(kPfThreads, 1)
     pf_gemm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_sb,
-                   const __grid_constant__ CUtensorMap tm_b, const PfArgs a) {
+                   const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_b64,
+                   const __grid_constant__ CUtensorMap tm_b128, const PfArgs a) {
   extern __shared__ uint8_t pf_smem_raw[];
   constexpr int kCodesBytes = 2048 * B;   // 16 groups x 4 units x 8 rows x B words
   constexpr int kSbBytes = 512 * GPB;     // 8 tiles x 16 GPB words
@@ -299,6 +301,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     tmap_prefetch(&tm_q);
     tmap_prefetch(&tm_sb);
     tmap_prefetch(&tm_b);
+    tmap_prefetch(&tm_b64);
+    tmap_prefetch(&tm_b128);
   }
   pdl_wait();
   // the pass's experts and their tiles (token tiles x row tiles, row tile fastest)
@@ -356,8 +360,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       uint32_t ph = 0, issued = 0, last_ph = 0;  // per-stage bit masks for the exit drain
       for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
         const PfTile tl = tile_at(t);
-        const int nbox = (tl.n + 31) >> 5;
-        const uint32_t bytes = kCodesBytes + kSbBytes + (uint32_t)nbox * 2 * 32 * 128;
+        // the tile's token rows: one box of 32, 64 or 128 rows per 64-column half
+        // (rows past the expert's tokens are loaded and never read by the MMA)
+        const int brows = tl.n <= 32 ? 32 : tl.n <= 64 ? 64 : 128;
+        const CUtensorMap* tmb = brows == 32 ? &tm_b : brows == 64 ? &tm_b64 : &tm_b128;
+        const uint32_t bytes = kCodesBytes + kSbBytes + (uint32_t)brows * 2 * 128;
         bool ok = true;
         for (int kb = 0; kb < a.nkb; ++kb) {
           if (!pf_wait(&empty[s], ph ^ 1u, &s_abort, a.wait_limit)) {
@@ -367,11 +374,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           mbar_arrive_expect_tx(&full[s], bytes);
           tma_load_4d(cst + s * kCodesBytes, &tm_q, kb * 32 * B, 0, tl.mt * 8, tl.slot, &full[s]);
           tma_load_3d(sbst + s * kSbBytes, &tm_sb, kb * 16 * GPB, tl.mt * 8, tl.slot, &full[s]);
-          for (int j = 0; j < nbox; ++j)
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf)
-              tma_load_2d(xst + (s * 2 + hf) * kPfXHalf + j * 4096, &tm_b, kb * 128 + hf * 64, tl.row0 + 32 * j,
-                          &full[s]);
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_2d(xst + (s * 2 + hf) * kPfXHalf, tmb, kb * 128 + hf * 64, tl.row0, &full[s]);
           issued |= 1u << s;
           last_ph = (last_ph & ~(1u << s)) | (ph << s);
           if (++s == kPfStages) {
@@ -577,11 +582,11 @@ bool encode_proj(CUtensorMap* q, CUtensorMap* sb, const uint8_t* proj, int64_t r
 }
 
 // Token rows (fp16 [rows][cols], row-major) for the MMA's B operand: boxes of
-// 64 columns (128 bytes, 128-byte swizzle) x 32 rows.
-bool encode_rows(CUtensorMap* m, const uint16_t* base, int64_t rows, int cols) {
+// 64 columns (128 bytes, 128-byte swizzle) x box_rows rows.
+bool encode_rows(CUtensorMap* m, const uint16_t* base, int64_t rows, int cols, int box_rows) {
   const cuuint64_t d[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t s[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t b[2] = {64, 32};
+  const cuuint32_t b[2] = {64, (cuuint32_t)box_rows};
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, d, s, b, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
@@ -591,7 +596,7 @@ size_t pf_smem_bytes(int bits, int gpb) {
 }
 
 template <int B, int GPB, bool GU>
-cudaError_t launch_pf_t(const CUtensorMap& q, const CUtensorMap& sb, const CUtensorMap& bm, const PfArgs& pa,
+cudaError_t launch_pf_t(const CUtensorMap& q, const CUtensorMap& sb, const CUtensorMap (&bm)[3], const PfArgs& pa,
                         int grid, cudaStream_t st) {
   static int done[4] = {0, 0, 0, 0};
   const void* kern = reinterpret_cast<const void*>(pf_gemm_kernel<B, GPB, GU>);
@@ -604,11 +609,11 @@ cudaError_t launch_pf_t(const CUtensorMap& q, const CUtensorMap& sb, const CUten
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&done[dev >> 5], 1 << (dev & 31), __ATOMIC_RELAXED);
   }
-  return launch_pdl(kern, grid, kPfThreads, smem, st, q, sb, bm, pa);
+  return launch_pdl(kern, grid, kPfThreads, smem, st, q, sb, bm[0], bm[1], bm[2], pa);
 }
 
 template <int B, bool GU>
-cudaError_t launch_pf_gpb(int gpb, const CUtensorMap& q, const CUtensorMap& sb, const CUtensorMap& bm,
+cudaError_t launch_pf_gpb(int gpb, const CUtensorMap& q, const CUtensorMap& sb, const CUtensorMap (&bm)[3],
                           const PfArgs& pa, int grid, cudaStream_t st) {
   if (gpb == 1) return launch_pf_t<B, 1, GU>(q, sb, bm, pa, grid, st);
   if (gpb == 2) return launch_pf_t<B, 2, GU>(q, sb, bm, pa, grid, st);
@@ -616,7 +621,7 @@ cudaError_t launch_pf_gpb(int gpb, const CUtensorMap& q, const CUtensorMap& sb, 
 }
 
 template <bool GU>
-cudaError_t launch_pf(int bits, int gpb, const CUtensorMap& q, const CUtensorMap& sb, const CUtensorMap& bm,
+cudaError_t launch_pf(int bits, int gpb, const CUtensorMap& q, const CUtensorMap& sb, const CUtensorMap (&bm)[3],
                       const PfArgs& pa, int grid, cudaStream_t st) {
   if (bits == 3) return launch_pf_gpb<3, GU>(gpb, q, sb, bm, pa, grid, st);
   if (bits == 4) return launch_pf_gpb<4, GU>(gpb, q, sb, bm, pa, grid, st);
@@ -641,12 +646,14 @@ cudaError_t launch_ffn_prefill_tc(const FfnArgs& a, const moe_layer_desc& d, int
   const Layout& L = a.L;
   const int gpb = 128 / d.group;
   const int64_t np = (int64_t)a.T * d.k;
-  CUtensorMap q_gu, sb_gu, q_d, sb_d, xm, hm;
+  CUtensorMap q_gu, sb_gu, q_d, sb_d, xm[3], hm[3];
   if (!encode_proj(&q_gu, &sb_gu, a.pool + L.gu, L.rb_gu, L.tile_gu, L.ng_gu, 2 * d.I, d.bits_gu, gpb, L.slot_bytes,
                    a.n_slots) ||
       !encode_proj(&q_d, &sb_d, a.pool + L.d, L.rb_d, L.tile_d, L.ng_d, d.H, d.bits_down, gpb, L.slot_bytes,
                    a.n_slots) ||
-      !encode_rows(&xm, a.x_sorted, np, d.H) || !encode_rows(&hm, a.h, np, d.I))
+      !encode_rows(&xm[0], a.x_sorted, np, d.H, 32) || !encode_rows(&xm[1], a.x_sorted, np, d.H, 64) ||
+      !encode_rows(&xm[2], a.x_sorted, np, d.H, 128) || !encode_rows(&hm[0], a.h, np, d.I, 32) ||
+      !encode_rows(&hm[1], a.h, np, d.I, 64) || !encode_rows(&hm[2], a.h, np, d.I, 128))
     return cudaErrorInvalidValue;
   PfArgs pa{};
   pa.T = a.T;

@@ -276,9 +276,9 @@ class Streamer:
 
     def check_dev_err(self) -> int:
         """The device error word (MOE_DEV_ERR_* bits).  After a wait that ran
-        out, the workspace's control block (the single-launch decode kernel's
-        readiness counters) is zeroed again before any later call."""
+        out, the whole workspace (its control block and the tagged h words
+        that carry over between calls) is zeroed before any later call."""
         v = int(self.dev_err.item())
         if v & ops.DEV_ERR_TIMEOUT:
-            self.ws[:ops.WS_CONTROL_BYTES].zero_()
+            self.ws.zero_()
         return v
