@@ -38,6 +38,7 @@ moe_status scratch_of_current_device(void** out) {
 }  // namespace
 
 extern "C" size_t moe_internal_workspace_bytes_no_tc(const moe_layer_desc* d, int32_t max_tokens);
+extern "C" size_t moe_internal_workspace_persistent_bytes(const moe_layer_desc* d);
 
 extern "C" size_t moe_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
@@ -53,11 +54,14 @@ extern "C" moe_status moe_expert_ffn_noalloc(const uint16_t* x, int32_t T, const
   void* scratch = nullptr;
   const moe_status s = scratch_of_current_device(&scratch);
   if (s != MOE_OK) return s;
-  // The array keeps whatever the previous call (on any stream) left in it.
-  // Its head is the control block (the fused kernel's readiness counters),
-  // which must start every call at zero: clear it in stream order, so that
-  // even a call that was cut short before cannot leave a later one wrong.
-  if (cudaMemsetAsync(scratch, 0, moe::kWsControlBytes, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  // The array keeps whatever the previous call (on any stream, with any
+  // layer description) left in it.  Its head -- the control block and the
+  // tagged h words, which a workspace keeps from call to call -- is cleared
+  // in stream order, so that every call starts from a zeroed workspace and
+  // depends on no earlier one.
+  const size_t head = moe_internal_workspace_persistent_bytes(d);
+  if (head == 0 || head > need) return MOE_ERR_INVALID;
+  if (cudaMemsetAsync(scratch, 0, head, stream) != cudaSuccess) return MOE_ERR_CUDA;
   return moe_expert_ffn(x, T, d, pool, n_slots, slot_table, ids, w, offsets, pairs, active, n_active, nullptr,
                         pass_begin, pass_len, y_accum, scratch, kNoAllocScratchBytes, dev_err, stream);
 }
