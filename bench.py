@@ -82,6 +82,10 @@ CONFIGS = {
               "Coder-30B-like batched decode: 48 layers x 128 experts, top-8, H 2048, I 768, 4-bit g64, "
               "64 tokens/step, all 128 experts resident"),
     "tiny": (1, 8, 2, 64, 32, 32, 4, 4, 4, 8, "tiny MoE layer: 8 experts, top-2, H 64, I 32, 4-bit g32, 4 tokens"),
+    "decode_shared": (48, 512, 10, 2048, 512, 64, 3, 3, 1, 192,
+                      "Flash-Next-like decode with one always-on shared expert per layer (same shape, pinned slot, "
+                      "run in the routed experts' FFN launch): 48 layers x 512 routed experts, top-10, H 2048, I 512, "
+                      "3-bit g64, 1 token/step, 192 slots/layer, misses installed from pinned host"),
     "decode_mixed": (48, 512, 10, 2048, 512, 64, 4, 4, 1, 128,
                      "mixed size classes decode with cache-aware substitution: Flash-Next-like shapes, 4-bit "
                      "gate/up, 6-bit down on layers l % 4 == 0 (2 slot size classes), 1 token/step, 128 slots/layer "
@@ -90,7 +94,8 @@ CONFIGS = {
 # token counts of a configuration's batch sweep (besides its own T), FFN-only
 SWEEP = {"coder": (1, 8, 32)}
 # per-layer widths and the substitution strength of the decode configurations (default: uniform, L = 0)
-DECODE_EXTRA = {"decode_mixed": {"bits": lambda l: (4, 6) if l % 4 == 0 else (4, 4), "L": 0.15}}
+DECODE_EXTRA = {"decode_mixed": {"bits": lambda l: (4, 6) if l % 4 == 0 else (4, 4), "L": 0.15},
+                "decode_shared": {"n_shared": 1}}
 
 # Prefill chunks: every expert of every layer resident (the metric is the expert
 # FFN's tensor-core rate; installs are PCIe-bound and reported by decode).
@@ -180,7 +185,7 @@ SEQUENCE = {
 }
 
 
-def build_streamer(cfg, seed, device, bits=None, max_tokens=None):
+def build_streamer(cfg, seed, device, bits=None, max_tokens=None, n_shared=0):
     import numpy as np
     import torch
 
@@ -193,9 +198,13 @@ def build_streamer(cfg, seed, device, bits=None, max_tokens=None):
     for d in descs:
         if (d.bits_gu, d.bits_down) not in banks:
             banks[(d.bits_gu, d.bits_down)] = quantize_bank_gpu(E, d, seed + 17 * d.bits_down, device)
-    specs = [LayerSpec(d, banks[(d.bits_gu, d.bits_down)], synth.bank_permutation(seed, l, E).tolist())
+    # shared experts: the bank's last n_shared rows (distinct weights from a seed of their own)
+    shared = {c: quantize_bank_gpu(n_shared, descs[0] if c is None else c, seed + 7919, device)
+              for c in ([None] if n_shared else [])}
+    specs = [LayerSpec(d, banks[(d.bits_gu, d.bits_down)], synth.bank_permutation(seed, l, E).tolist(),
+                       shared[None] if n_shared else None)
              for l, d in enumerate(descs)]
-    st = Streamer(specs, S, max_tokens=max_tokens or T, device=device)
+    st = Streamer(specs, S, max_tokens=max_tokens or T, device=device, n_shared=n_shared)
     for l in range(n_layers):  # the S most popular experts start resident, on a random slot permutation
         hot = np.argsort(synth.popularity_rank(seed, l, E))[:S]
         st.place(l, hot.tolist(), synth.slot_permutation(seed, l, S).tolist())
@@ -239,9 +248,9 @@ def ffn_graph_time(st, cfg, snaps, reps, device, T=None):
         cs = torch.cuda.current_stream(device)
         for l in range(n_layers):
             sn = snaps[l]
-            ops.moe_expert_ffn(sn["x"], T, st.layers[l].desc, st.pool_of(l), st.n_slots_of(l), st.table_dev[l],
+            ops.moe_expert_ffn(sn["x"], T, st.wdesc[l], st.pool_of(l), st.n_slots_of(l), st.table_dev[l],
                                sn["ids"], sn["w"], sn["offsets"], sn["pairs"], sn["meta"][2:], sn["meta"][0:1],
-                               sn.get("xs"), 0, E, y, st.ws, st.ws_bytes, st.dev_err, cs)
+                               sn.get("xs"), 0, st.Ew, y, st.ws, st.ws_bytes, st.dev_err, cs)
     for _ in range(3):
         g_.replay()
     torch.cuda.synchronize(device)
@@ -265,7 +274,8 @@ def stage_graph_times(st, cfg, snaps, logits, Lsub, reps, device):
 
     from streamed_quantized_expert_b200 import ops
 
-    n_layers, E, k, H, I, g, bg, bd, T, S, _ = cfg
+    n_layers, _, _, H, I, g, bg, bd, T, S, _ = cfg
+    E, k = st.Ew, st.kw  # the widened layer (shared experts after the routed ones)
     ids = torch.empty((T, k), dtype=torch.int32, device=device)
     w = torch.empty((T, k), dtype=torch.float32, device=device)
     offsets = torch.empty(E + 1, dtype=torch.int32, device=device)
@@ -274,11 +284,14 @@ def stage_graph_times(st, cfg, snaps, logits, Lsub, reps, device):
     slots = torch.empty(E, dtype=torch.int32, device=device)
 
     def route(l, cs):
-        ops.moe_route(logits[l], T, st.layers[l].desc, Lsub, st.table_dev[l], ids, w, cs)
+        if st.ns:
+            ops.moe_route_shared(logits[l], T, st.layers[l].desc, Lsub, st.table_dev[l], st.ns, None, ids, w, cs)
+        else:
+            ops.moe_route(logits[l], T, st.layers[l].desc, Lsub, st.table_dev[l], ids, w, cs)
 
     def sort(l, cs):
         sn = snaps[l]
-        ops.moe_sort(sn["ids"], None, T, st.layers[l].desc, offsets, pairs, meta[2:2 + E], meta[0:1], None, st.ws,
+        ops.moe_sort(sn["ids"], None, T, st.wdesc[l], offsets, pairs, meta[2:2 + E], meta[0:1], None, st.ws,
                      st.ws_bytes, cs)
 
     def lookup(l, cs):
@@ -592,7 +605,7 @@ def run_ours(args, rank, world, local_rank):
     extra = DECODE_EXTRA.get(args.config, {})
     Lsub = extra.get("L", 0.0)
     seed = 1000 * rank
-    st = build_streamer(cfg, seed, device, extra.get("bits"))
+    st = build_streamer(cfg, seed, device, extra.get("bits"), n_shared=extra.get("n_shared", 0))
     steps_total = args.warmup + args.steps
     # the popularity bias of the logits and the initially resident experts come from the same seed
     x, logits = make_inputs(cfg, seed, steps_total + 1, device)
@@ -627,7 +640,7 @@ def run_ours(args, rank, world, local_rank):
             st.decode_layer(l, x[steps_total, l], logits[steps_total, l], T, Lsub)
             snaps.append({"x": x[steps_total, l], "ids": st.ids.clone(), "w": st.w.clone(),
                           "offsets": st.offsets.clone(), "pairs": st.pairs.clone(), "meta": st.meta.clone(),
-                          **({"xs": st.x_sorted[:T * k].clone()} if T >= 32 else {})})
+                          **({"xs": st.x_sorted[:T * st.kw].clone()} if T >= 32 else {})})
         torch.cuda.synchronize(device)
         n_unique = sum(int(sn["meta"][0].item()) for sn in snaps) / n_layers
         ffn_us = ffn_graph_time(st, cfg, snaps, args.ffn_reps, device)
@@ -640,7 +653,7 @@ def run_ours(args, rank, world, local_rank):
                 st.decode_layer(l, x[steps_total, l, :T2], logits[steps_total, l, :T2], T2, Lsub)
                 sn2.append({"x": x[steps_total, l, :T2], "ids": st.ids.clone(), "w": st.w.clone(),
                             "offsets": st.offsets.clone(), "pairs": st.pairs.clone(), "meta": st.meta.clone(),
-                            **({"xs": st.x_sorted[:T2 * k].clone()} if T2 >= 32 else {})})
+                            **({"xs": st.x_sorted[:T2 * st.kw].clone()} if T2 >= 32 else {})})
             torch.cuda.synchronize(device)
             us2 = ffn_graph_time(st, cfg, sn2, args.ffn_reps, device, T=T2)
             sweep.append((T2, us2, sn2))
@@ -717,7 +730,8 @@ def run_ours(args, rank, world, local_rank):
                    "intermediate": I, "group": g, "bits": [bg, bd], "tokens_per_step": T, "slots_per_layer": S,
                    "l2": "inputs larger than L2: each step reads ~%.0f MB of distinct expert slots" %
                          (n_layers * ffn_bytes / 1e6),
-                   "parallelism": f"replicas x{world} (independent token streams)"},
+                   "parallelism": f"replicas x{world} (independent token streams)",
+                   **({"shared_experts": st.ns} if st.ns else {})},
         "ffn": {"tok_s_equiv": round(T / (n_layers * ffn_us * 1e-6), 1),
                 "us_per_layer": round(ffn_us, 3),
                 "hbm_gbs": round(achieved, 1),

@@ -159,6 +159,25 @@ size_t moe_workspace_bytes(const moe_layer_desc* d, int32_t max_tokens);
 moe_status moe_route(const float* logits, int32_t T, const moe_layer_desc* d, float L,
                      const int32_t* slot_table, int32_t* ids, float* w, cudaStream_t stream);
 
+/* Stage 1 for a layer with always-on shared experts (BigMoeOnEdge
+ * docs/limitations.md, "Limitations", bullet "Shared experts stay resident":
+ * the routed experts stream, the shared expert stays resident).  The top-k
+ * of moe_route, then n_shared (0..8) shared experts appended to every token:
+ *   ids  device int32 [T, k + n_shared]: the top-k in rank order, then the
+ *        expert ids E, E+1, ..., E+n_shared-1
+ *   w    device fp32 [T, k + n_shared]: the top-k weights (normalised over
+ *        the top-k only), then shared_w[t] for each shared expert, or 1 when
+ *        shared_w is NULL (device fp32 [T], e.g. a per-token gate)
+ * The layer's other calls then take the widened description (E + n_shared
+ * experts, k + n_shared per token) and a slot table of E + n_shared entries
+ * whose last n_shared entries hold the shared experts' slots, so the shared
+ * experts run in the same moe_expert_ffn launch as the routed ones.  Keeping
+ * those slots resident is the caller's (moe_cache manages routed experts
+ * only).  n_shared outside 0..8 returns MOE_ERR_INVALID. */
+moe_status moe_route_shared(const float* logits, int32_t T, const moe_layer_desc* d, float L,
+                            const int32_t* slot_table, int32_t n_shared, const float* shared_w, int32_t* ids,
+                            float* w, cudaStream_t stream);
+
 /* Stage 2.  Stable counting sort of the T*k (token, rank) pairs by expert.
  *   ids      device int32 [T, k]
  *   x        device bf16 [T, H] or NULL; when given, x_sorted is written
@@ -346,7 +365,9 @@ int32_t moe_cache_resident(const moe_cache* c, int32_t layer);
  * Native driver of one decode layer (the sequence of the calls above).
  * ---------------------------------------------------------------------- */
 
-/* Per-call device buffers, caller-owned, sized for max_tokens tokens. */
+/* Per-call device buffers, caller-owned, sized for max_tokens tokens (with
+ * shared experts, E and k below are those of the widened layer: E + n_shared,
+ * k + n_shared). */
 typedef struct {
   int32_t* ids;        /* device int32 [max_tokens, k] */
   float* w;            /* device fp32 [max_tokens, k] */
@@ -372,6 +393,11 @@ typedef struct {
   int32_t* table_dev;           /* device int32 [E]: this layer's expert -> slot */
   int32_t* table_stage;         /* pinned host int32 [E]: staging for table uploads */
   const void* const* bank_rows; /* host [E]: pinned host address of each expert's slot bytes */
+  int32_t n_shared;             /* always-on shared experts (moe_route_shared), 0..8: their slots
+                                   are table_dev[E .. E+n_shared), kept resident by the caller;
+                                   table_dev then has E + n_shared entries and the step buffers
+                                   are sized for E + n_shared experts, k + n_shared per token */
+  const float* shared_w;        /* device fp32 [T] per-token weight of the shared experts, or NULL (1) */
 } moe_layer_ctx;
 
 /* One decode layer, T <= 64 tokens (RFC "How the prototype works": each layer

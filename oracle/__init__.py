@@ -116,6 +116,25 @@ def route(logits: np.ndarray, k: int, L: float = 0.0, slot_table: np.ndarray | N
     return ids, w, u
 
 
+def route_shared(logits: np.ndarray, k: int, n_shared: int, shared_w=None, L: float = 0.0,
+                 slot_table: np.ndarray | None = None):
+    """route(), then every token's always-on shared experts (BigMoeOnEdge
+    docs/limitations.md, "Limitations", "Shared experts stay resident": the
+    shared expert runs for every token).  Shared expert s of a layer with E
+    routed experts has id E + s and weight shared_w[t] (1 when None) for
+    every token; the top-k weights stay normalised over the top-k alone.
+    Returns (ids int32 [T, k + n_shared], w float64 [T, k + n_shared], u)."""
+    ids, w, u = route(logits, k, L, slot_table)
+    T, E = np.asarray(logits).shape
+    sid = np.broadcast_to(np.arange(E, E + n_shared, dtype=np.int32), (T, n_shared))
+    if shared_w is None:
+        sw = np.ones((T, n_shared), np.float64)
+    else:
+        sw = np.repeat(np.asarray(shared_w, np.float32).astype(np.float64)[:, None], n_shared, axis=1)
+    return (np.ascontiguousarray(np.concatenate([ids, sid], axis=1), dtype=np.int32),
+            np.ascontiguousarray(np.concatenate([w, sw], axis=1)), u)
+
+
 def sort(ids: np.ndarray, E: int):
     """Returns (offsets [E+1], pairs [T*k], active [n_active])."""
     ids = np.ascontiguousarray(ids, dtype=np.int32)

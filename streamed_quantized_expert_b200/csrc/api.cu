@@ -154,7 +154,19 @@ moe_status moe_route(const float* logits, int32_t T, const moe_layer_desc* d, fl
   if (T == 0) return MOE_OK;
   if (!logits || !ids || !w) return MOE_ERR_INVALID;
   if (L > 0.0f && !slot_table) return MOE_ERR_INVALID;
-  return cuda_status(launch_route(logits, T, d->E, d->k, L, slot_table, ids, w, stream));
+  return cuda_status(launch_route(logits, T, d->E, d->k, L, slot_table, ids, w, 0, nullptr, stream));
+}
+
+moe_status moe_route_shared(const float* logits, int32_t T, const moe_layer_desc* d, float L,
+                            const int32_t* slot_table, int32_t n_shared, const float* shared_w, int32_t* ids,
+                            float* w, cudaStream_t stream) {
+  moe_status s = check_desc(d);
+  if (s != MOE_OK) return s;
+  if (T < 0 || !(L >= 0.0f) || L > 1e30f || n_shared < 0 || n_shared > kMaxShared) return MOE_ERR_INVALID;
+  if (T == 0) return MOE_OK;
+  if (!logits || !ids || !w) return MOE_ERR_INVALID;
+  if (L > 0.0f && !slot_table) return MOE_ERR_INVALID;
+  return cuda_status(launch_route(logits, T, d->E, d->k, L, slot_table, ids, w, n_shared, shared_w, stream));
 }
 
 moe_status moe_sort(const int32_t* ids, const uint16_t* x, int32_t T, const moe_layer_desc* d, int32_t* offsets,

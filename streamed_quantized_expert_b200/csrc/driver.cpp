@@ -30,22 +30,30 @@ extern "C" moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const mo
                                        int32_t T, float L, float* y, cudaStream_t stream, cudaStream_t side,
                                        cudaEvent_t installed, int32_t* n_installed) {
   if (!cache || !lc || !b || !lc->desc || !y || !x || !logits) return MOE_ERR_INVALID;
-  const moe_layer_desc* d = lc->desc;
+  const moe_layer_desc* d0 = lc->desc;  // the routed experts
+  const int32_t ns = lc->n_shared;
+  if (ns < 0 || ns > 8) return MOE_ERR_INVALID;
+  // the widened layer: shared experts E0 .. E0 + ns - 1 after the routed ones
+  moe_layer_desc dw = *d0;
+  dw.E += ns;
+  dw.k += ns;
+  const moe_layer_desc* d = &dw;
   if (T < 1 || T > b->max_tokens || T > 64) return MOE_ERR_INVALID;
-  const int32_t E = d->E;
+  const int32_t E = d->E, E0 = d0->E;
   if (n_installed) *n_installed = 0;
   int32_t* n_active = b->meta;
   int32_t* n_miss = b->meta + 1;
   int32_t* active = b->meta + 2;
   int32_t* miss = b->meta + 2 + E;
-  moe_status s = moe_route(logits, T, d, L, lc->table_dev, b->ids, b->w, stream);
+  moe_status s = ns ? moe_route_shared(logits, T, d0, L, lc->table_dev, ns, lc->shared_w, b->ids, b->w, stream)
+                    : moe_route(logits, T, d0, L, lc->table_dev, b->ids, b->w, stream);
   if (s != MOE_OK) return s;
   // from 32 tokens the FFN runs on the tensor-core grouped GEMM, which reads x sorted by expert
   uint16_t* xs = (T >= 32 && b->x_sorted) ? b->x_sorted : nullptr;
   s = moe_sort(b->ids, xs ? x : nullptr, T, d, b->offsets, b->pairs, active, n_active, xs, b->ws, b->ws_bytes,
                stream);
   if (s != MOE_OK) return s;
-  if (moe_cache_resident(cache, layer) < E) {
+  if (moe_cache_resident(cache, layer) < E0) {
     s = moe_slot_lookup(lc->table_dev, active, n_active, 0, E, lc->n_slots, b->slots, miss, n_miss, b->dev_err,
                         stream);
     if (s != MOE_OK) return s;
@@ -54,21 +62,23 @@ extern "C" moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const mo
       return MOE_ERR_CUDA;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
     const int32_t na = b->meta_host[0];
-    if (na < 0 || na > E) return MOE_ERR_INVALID;
+    if (na < ns || na > E) return MOE_ERR_INVALID;
     thread_local std::vector<int32_t> out_e, out_s;
     thread_local std::vector<const void*> rows;
     out_e.resize(E);
     out_s.resize(E);
     int32_t n = 0;
-    s = moe_cache_step(cache, layer, b->meta_host + 2, na, out_e.data(), out_s.data(), &n);
+    // the active list is ascending: every token's shared experts are its last
+    // ns entries, and the cache manages the routed ones only
+    s = moe_cache_step(cache, layer, b->meta_host + 2, na - ns, out_e.data(), out_s.data(), &n);
     if (s != MOE_OK) return s;
     if (n > 0) {
       rows.resize(n);
       for (int32_t i = 0; i < n; ++i) rows[i] = lc->bank_rows[out_e[i]];
       s = moe_install_slots(lc->pool, lc->slot_bytes, lc->n_slots, rows.data(), out_s.data(), n, side, nullptr);
       if (s != MOE_OK) return s;
-      std::memcpy(lc->table_stage, moe_cache_table(cache, layer), sizeof(int32_t) * (size_t)E);
-      if (cudaMemcpyAsync(lc->table_dev, lc->table_stage, sizeof(int32_t) * (size_t)E, cudaMemcpyHostToDevice,
+      std::memcpy(lc->table_stage, moe_cache_table(cache, layer), sizeof(int32_t) * (size_t)E0);
+      if (cudaMemcpyAsync(lc->table_dev, lc->table_stage, sizeof(int32_t) * (size_t)E0, cudaMemcpyHostToDevice,
                           side) != cudaSuccess)
         return MOE_ERR_CUDA;
       if (cudaEventRecord(installed, side) != cudaSuccess) return MOE_ERR_CUDA;

@@ -11,6 +11,7 @@ namespace moe {
 
 constexpr int kFusedMaxTokens = 64;  // decode down kernel combines in shared memory up to this T
 constexpr int kTcMinTokens = 32;  // from this T on (with x_sorted) the FFN runs on the tcgen05 grouped GEMM
+constexpr int kMaxShared = 8;  // shared experts per layer (moe_route_shared)
 constexpr int kRouteBlockMaxTokens = 64;  // up to this T, routing takes a block (8 warps) per token
 
 struct FfnArgs {
@@ -69,7 +70,7 @@ inline cudaError_t launch_pdl(const void* func, int grid, int block, size_t smem
 }
 
 cudaError_t launch_route(const float* logits, int T, int E, int k, float L, const int32_t* table, int32_t* ids,
-                         float* w, cudaStream_t st);
+                         float* w, int n_shared, const float* shared_w, cudaStream_t st);
 size_t sort_ws_bytes(int n, int E);
 cudaError_t launch_sort(const int32_t* ids, const uint16_t* x, int T, int k, int E, int H, int32_t* offsets,
                         int32_t* pairs, int32_t* active, int32_t* n_active, uint16_t* x_sorted, void* ws,

@@ -55,7 +55,7 @@ __device__ __forceinline__ bool key_better(float au, float al, int ae, float bu,
 template <int NPL>
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int k, float L,
                                                     const int32_t* __restrict__ table, int32_t* __restrict__ ids,
-                                                    float* __restrict__ wout) {
+                                                    float* __restrict__ wout, int ns, const float* __restrict__ sw) {
   const int lane = threadIdx.x & 31;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   pdl_wait();
@@ -130,9 +130,14 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
   float s = lane < k ? my_u : 0.0f;
 #pragma unroll
   for (int o = 16; o; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
+  const int ks = k + ns;  // output row: the top-k, then the shared experts
   if (lane < k) {
-    ids[(size_t)t * k + lane] = my_e;
-    wout[(size_t)t * k + lane] = __fdiv_rn(my_u, s);
+    ids[(size_t)t * ks + lane] = my_e;
+    wout[(size_t)t * ks + lane] = __fdiv_rn(my_u, s);
+  }
+  if (lane < ns) {
+    ids[(size_t)t * ks + k + lane] = E + lane;
+    wout[(size_t)t * ks + k + lane] = sw ? sw[t] : 1.0f;
   }
 }
 
@@ -165,7 +170,8 @@ __device__ __forceinline__ bool key_before(uint32_t a1, uint32_t a2, int ae, uin
 template <int NPT>
 __global__ void __launch_bounds__(256) route_select_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                            float L, const int32_t* __restrict__ table,
-                                                           int32_t* __restrict__ ids, float* __restrict__ wout) {
+                                                           int32_t* __restrict__ ids, float* __restrict__ wout, int ns,
+                                                           const float* __restrict__ sw) {
   __shared__ float s_red[8];
   __shared__ uint32_t s_hist[256];
   __shared__ int s_ctl[3];  // boundary digit, experts still to take, boundary bucket size
@@ -329,9 +335,14 @@ __global__ void __launch_bounds__(256) route_select_kernel(const float* __restri
     float sum = my_u;
 #pragma unroll
     for (int o = 16; o; o >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, o));
+    const int ks = k + ns;  // output row: the top-k, then the shared experts
     if (mine) {
-      ids[(size_t)t * k + lane] = s_oe[lane];
-      wout[(size_t)t * k + lane] = __fdiv_rn(my_u, sum);
+      ids[(size_t)t * ks + lane] = s_oe[lane];
+      wout[(size_t)t * ks + lane] = __fdiv_rn(my_u, sum);
+    }
+    if (lane < ns) {
+      ids[(size_t)t * ks + k + lane] = E + lane;
+      wout[(size_t)t * ks + k + lane] = sw ? sw[t] : 1.0f;
     }
   }
 }
@@ -523,19 +534,19 @@ __global__ void __launch_bounds__(1024) lookup_kernel(const int32_t* __restrict_
 // launchers
 // ---------------------------------------------------------------------------
 cudaError_t launch_route(const float* logits, int T, int E, int k, float L, const int32_t* table, int32_t* ids,
-                         float* w, cudaStream_t st) {
+                         float* w, int n_shared, const float* shared_w, cudaStream_t st) {
   if (T <= kRouteBlockMaxTokens && E <= 1024) {  // decode sizes: a block per token
     const void* kb = E <= 256 ? reinterpret_cast<const void*>(route_select_kernel<1>)
                      : E <= 512 ? reinterpret_cast<const void*>(route_select_kernel<2>)
                                 : reinterpret_cast<const void*>(route_select_kernel<4>);
-    return launch_pdl(kb, T, 256, 0, st, logits, T, E, k, L, table, ids, w);
+    return launch_pdl(kb, T, 256, 0, st, logits, T, E, k, L, table, ids, w, n_shared, shared_w);
   }
   const int blocks = (T + 7) / 8;
   const void* kern = E <= 32    ? reinterpret_cast<const void*>(route_kernel<1>)
                      : E <= 128 ? reinterpret_cast<const void*>(route_kernel<4>)
                      : E <= 512 ? reinterpret_cast<const void*>(route_kernel<16>)
                                 : reinterpret_cast<const void*>(route_kernel<32>);
-  return launch_pdl(kern, blocks, 256, 0, st, logits, T, E, k, L, table, ids, w);
+  return launch_pdl(kern, blocks, 256, 0, st, logits, T, E, k, L, table, ids, w, n_shared, shared_w);
 }
 
 size_t sort_ws_bytes(int n, int E) { return n <= 1024 ? 0 : (size_t)((n + 1023) / 1024) * E * sizeof(int32_t); }

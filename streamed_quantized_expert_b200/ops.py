@@ -25,7 +25,7 @@ ABI_SYMBOLS = [
     "moe_status_string", "moe_cache_create", "moe_cache_destroy", "moe_cache_table", "moe_cache_layer_base",
     "moe_cache_class_slots", "moe_cache_place", "moe_cache_step", "moe_cache_stats",
     "moe_expert_ffn_noalloc", "moe_noalloc_scratch_bytes", "moe_cache_resident", "moe_decode_layer",
-    "moe_last_cuda_error", "moe_ffn_kernel_path", "moe_set_wait_limit_cycles",
+    "moe_last_cuda_error", "moe_ffn_kernel_path", "moe_set_wait_limit_cycles", "moe_route_shared",
 ]
 
 
@@ -55,7 +55,7 @@ class StepBuffers(C.Structure):
 class LayerCtx(C.Structure):
     _fields_ = [("desc", C.POINTER(LayerDesc)), ("pool", C.c_void_p), ("n_slots", C.c_int32),
                 ("slot_bytes", C.c_size_t), ("table_dev", C.c_void_p), ("table_stage", C.c_void_p),
-                ("bank_rows", C.POINTER(C.c_void_p))]
+                ("bank_rows", C.POINTER(C.c_void_p)), ("n_shared", C.c_int32), ("shared_w", C.c_void_p)]
 
 
 class SlotLayout(C.Structure):
@@ -79,6 +79,7 @@ def lib():
             "moe_slot_layout": (C.c_int, [D, C.POINTER(SlotLayout)]),
             "moe_workspace_bytes": (sz, [D, i32]),
             "moe_route": (C.c_int, [P, i32, D, f32, P, P, P, P]),
+            "moe_route_shared": (C.c_int, [P, i32, D, f32, P, i32, P, P, P, P]),
             "moe_sort": (C.c_int, [P, P, i32, D, P, P, P, P, P, P, sz, P]),
             "moe_slot_lookup": (C.c_int, [P, P, P, i32, i32, i32, P, P, P, P, P]),
             "moe_install_slots": (C.c_int, [P, sz, i32, P, P, i32, P, P]),
@@ -179,6 +180,17 @@ def moe_workspace_bytes(d: LayerDesc, max_tokens: int) -> int:
 def moe_route(logits, T, d, L, slot_table, ids, w, stream=None) -> None:
     _ck(lib().moe_route(_ptr(logits), int(T), C.byref(d), float(L), _ptr(slot_table), _ptr(ids), _ptr(w),
                         _stream(stream)), "moe_route")
+
+
+def moe_route_shared(logits, T, d, L, slot_table, n_shared, shared_w, ids, w, stream=None) -> None:
+    _ck(lib().moe_route_shared(_ptr(logits), int(T), C.byref(d), float(L), _ptr(slot_table), int(n_shared),
+                               _ptr(shared_w), _ptr(ids), _ptr(w), _stream(stream)), "moe_route_shared")
+
+
+def widened(d: LayerDesc, n_shared: int) -> LayerDesc:
+    """The description the calls after moe_route_shared take: E + n_shared
+    experts, k + n_shared per token."""
+    return desc(d.E + n_shared, d.k + n_shared, d.H, d.I, d.group, d.bits_gu, d.bits_down)
 
 
 def moe_sort(ids, x, T, d, offsets, pairs, active, n_active, x_sorted, ws, ws_bytes, stream=None) -> None:

@@ -10,6 +10,9 @@ When every expert of a layer is resident the layer never synchronises with
 the host (RFC: "When every expert is resident, layers never synchronize with
 the host").  Layers are grouped into size classes by slot byte size, one
 device pool and one LRU range per (class, layer) (1bit-MONSTER PR #137).
+Always-on shared experts (BigMoeOnEdge docs/limitations.md, "Shared experts
+stay resident") get pinned slots after the class's LRU ranges and run in the
+same FFN launch as the routed experts (moe_route_shared widens the layer).
 """
 from __future__ import annotations
 
@@ -28,6 +31,7 @@ class LayerSpec:
     desc: ops.LayerDesc
     bank: torch.Tensor            # pinned uint8 [rows, slot_bytes] of this layer's class
     bank_row: list                # expert e -> row of `bank`
+    shared: torch.Tensor | None = None  # uint8 [n_shared, slot_bytes]: the layer's shared experts
 
 
 def quantize_bank_gpu(E: int, desc: ops.LayerDesc, seed: int, device="cuda", std: float = 0.02) -> torch.Tensor:
@@ -51,7 +55,7 @@ def quantize_bank_gpu(E: int, desc: ops.LayerDesc, seed: int, device="cuda", std
 
 class Streamer:
     def __init__(self, layers: list[LayerSpec], slots_per_layer: int, max_tokens: int, device="cuda",
-                 stream: torch.cuda.Stream | None = None):
+                 stream: torch.cuda.Stream | None = None, n_shared: int = 0):
         self.layers = layers
         self.n_layers = len(layers)
         self.device = torch.device(device)
@@ -59,6 +63,10 @@ class Streamer:
         self.k = layers[0].desc.k
         self.H = layers[0].desc.H
         assert all(l.desc.E == self.E and l.desc.H == self.H for l in layers)
+        self.ns = n_shared
+        assert n_shared == 0 or all(l.shared is not None and l.shared.shape[0] == n_shared for l in layers)
+        self.Ew, self.kw = self.E + n_shared, self.k + n_shared  # the widened layer
+        self.wdesc = [ops.widened(l.desc, n_shared) for l in layers]
         self.S = slots_per_layer
         self.max_tokens = max_tokens
         self.stream = stream or torch.cuda.current_stream(self.device)
@@ -74,16 +82,26 @@ class Streamer:
             self.layer_class.append(sizes.index(sb))
         self.class_bytes = sizes
         self.cache = ops.SlotCache(self.E, self.n_layers, self.S, self.layer_class)
+        # per class: the LRU's slots, then n_shared pinned slots per layer of the class
         self.pools = []
+        self.class_n_slots = []
         for c, sb in enumerate(sizes):
-            n = self.cache.class_slots(c)
+            n = self.cache.class_slots(c) + n_shared * self.layer_class.count(c)
             self.pools.append(torch.empty(n * sb, dtype=torch.uint8, device=self.device))
-        self.class_n_slots = [self.cache.class_slots(c) for c in range(len(sizes))]
-        # device tables + pinned mirrors
-        self.table_dev = torch.full((self.n_layers, self.E), -1, dtype=torch.int32, device=self.device)
-        self.table_pin = torch.full((self.n_layers, self.E), -1, dtype=torch.int32).pin_memory()
-        # per-call buffers
-        T, E, k = max_tokens, self.E, self.k
+            self.class_n_slots.append(n)
+        # device tables + pinned mirrors (routed experts, then the shared ones)
+        self.table_dev = torch.full((self.n_layers, self.Ew), -1, dtype=torch.int32, device=self.device)
+        self.table_pin = torch.full((self.n_layers, self.Ew), -1, dtype=torch.int32).pin_memory()
+        for l in range(self.n_layers) if n_shared else ():
+            c = self.layer_class[l]
+            first = self.cache.class_slots(c) + n_shared * self.layer_class[:l].count(c)
+            sb = self.class_bytes[c]
+            for s_ in range(n_shared):
+                self.pools[c][(first + s_) * sb: (first + s_ + 1) * sb].copy_(layers[l].shared[s_])
+                self.table_pin[l, self.E + s_] = first + s_
+        self.table_dev.copy_(self.table_pin)
+        # per-call buffers (widened layer)
+        T, E, k = max_tokens, self.Ew, self.kw
         self.ids = torch.empty((T, k), dtype=torch.int32, device=self.device)
         self.w = torch.empty((T, k), dtype=torch.float32, device=self.device)
         self.offsets = torch.empty(E + 1, dtype=torch.int32, device=self.device)
@@ -93,7 +111,7 @@ class Streamer:
         self.meta_pin = torch.zeros(2 + 2 * E, dtype=torch.int32).pin_memory()
         self.slots = torch.empty(E, dtype=torch.int32, device=self.device)
         self.dev_err = torch.zeros(1, dtype=torch.int32, device=self.device)
-        ws = max(ops.moe_workspace_bytes(l.desc, T) for l in layers)
+        ws = max(ops.moe_workspace_bytes(d, T) for d in self.wdesc)
         self.ws_bytes = ws
         self.ws = torch.zeros(ws, dtype=torch.uint8, device=self.device)
         self.x_sorted = None
@@ -104,7 +122,7 @@ class Streamer:
         # native per-layer driver state
         self.installed.record(self.side)  # materialise the event
         if max_tokens >= 32:  # batched decode sorts x for the tensor-core grouped GEMM
-            self.x_sorted = torch.empty((max_tokens * self.k, self.H), dtype=torch.uint16, device=self.device)
+            self.x_sorted = torch.empty((max_tokens * self.kw, self.H), dtype=torch.uint16, device=self.device)
         self._bufs = ops.StepBuffers(self.ids.data_ptr(), self.w.data_ptr(), self.offsets.data_ptr(),
                                      self.pairs.data_ptr(), self.meta.data_ptr(), self.meta_pin.data_ptr(),
                                      self.slots.data_ptr(), self.dev_err.data_ptr(), self.ws.data_ptr(),
@@ -118,7 +136,7 @@ class Streamer:
             self._ctx.append(ops.LayerCtx(C.pointer(spec.desc), self.pools[self.layer_class[l]].data_ptr(),
                                           self.class_n_slots[self.layer_class[l]],
                                           self.class_bytes[self.layer_class[l]], self.table_dev[l].data_ptr(),
-                                          self.table_pin[l].data_ptr(), rows))
+                                          self.table_pin[l].data_ptr(), rows, n_shared, None))
         self.ffn_events = None     # list to collect (start, end) CUDA events around FFN calls
 
     # -- views into meta --------------------------------------------------
@@ -129,10 +147,10 @@ class Streamer:
         return self.meta[1:2]
 
     def _active(self):
-        return self.meta[2: 2 + self.E]
+        return self.meta[2: 2 + self.Ew]
 
     def _miss(self):
-        return self.meta[2 + self.E: 2 + 2 * self.E]
+        return self.meta[2 + self.Ew: 2 + 2 * self.Ew]
 
     # -- residency ----------------------------------------------------------
     def pool_of(self, layer: int) -> torch.Tensor:
@@ -169,6 +187,7 @@ class Streamer:
         return self.cache.resident(layer) >= self.E
 
     def _install_pass(self, layer: int, pass_experts) -> int:
+        pass_experts = [e for e in pass_experts if e < self.E]  # shared experts stay where they are
         st, inst = self.cache.step(layer, pass_experts)
         if st != ops.MOE_OK:
             raise ops.MoeError(st, f"slot cache step (layer {layer})")
@@ -185,22 +204,25 @@ class Streamer:
 
     # -- stages -------------------------------------------------------------
     def route_sort(self, layer: int, x, logits, T: int, L: float = 0.0, want_sorted_x: bool = False):
-        d = self.layers[layer].desc
+        d, dw = self.layers[layer].desc, self.wdesc[layer]
         s = self.stream
-        ops.moe_route(logits, T, d, L, self.table_dev[layer], self.ids, self.w, s)
+        if self.ns:
+            ops.moe_route_shared(logits, T, d, L, self.table_dev[layer], self.ns, None, self.ids, self.w, s)
+        else:
+            ops.moe_route(logits, T, d, L, self.table_dev[layer], self.ids, self.w, s)
         self.launches += 1
         xs = None
         if want_sorted_x:
-            if self.x_sorted is None or self.x_sorted.numel() < T * self.k * self.H:
-                self.x_sorted = torch.empty((self.max_tokens * self.k, self.H), dtype=torch.uint16,
+            if self.x_sorted is None or self.x_sorted.numel() < T * self.kw * self.H:
+                self.x_sorted = torch.empty((self.max_tokens * self.kw, self.H), dtype=torch.uint16,
                                             device=self.device)
             xs = self.x_sorted
-        ops.moe_sort(self.ids, x if want_sorted_x else None, T, d, self.offsets, self.pairs, self._active(),
+        ops.moe_sort(self.ids, x if want_sorted_x else None, T, dw, self.offsets, self.pairs, self._active(),
                      self._n_active(), xs, self.ws, self.ws_bytes, s)
-        self.launches += (1 if T * self.k <= 1024 else 3) + (1 if want_sorted_x else 0)
+        self.launches += (1 if T * self.kw <= 1024 else 3) + (1 if want_sorted_x else 0)
 
     def ffn(self, layer: int, x, T: int, pass_begin: int, pass_len: int, y) -> None:
-        d = self.layers[layer].desc
+        d = self.wdesc[layer]
         ev = None
         if self.ffn_events is not None:
             ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -224,7 +246,7 @@ class Streamer:
         if n:
             self.installs += n
             self.installed_bytes += n * self.class_bytes[self.layer_class[layer]]
-        self.launches += 4 + (0 if full else 1) + (0 if T * self.k <= 1024 else 2)
+        self.launches += 4 + (0 if full else 1) + (0 if T * self.kw <= 1024 else 2)
         return y
 
     def decode_layer_steps(self, layer: int, x, logits, T: int, L: float = 0.0, y=None):
@@ -234,7 +256,7 @@ class Streamer:
         self.route_sort(layer, x, logits, T, L)
         if not self.fully_resident(layer):
             d = self.layers[layer].desc
-            ops.moe_slot_lookup(self.table_dev[layer], self._active(), self._n_active(), 0, self.E,
+            ops.moe_slot_lookup(self.table_dev[layer], self._active(), self._n_active(), 0, self.Ew,
                                 self.n_slots_of(layer), self.slots, self._miss(), self._n_miss(), self.dev_err, s)
             self.launches += 1
             with torch.cuda.stream(s):
@@ -246,7 +268,7 @@ class Streamer:
             del d
         with torch.cuda.stream(s):
             y.zero_()
-        self.ffn(layer, x, T, 0, self.E, y)
+        self.ffn(layer, x, T, 0, self.Ew, y)
         return y
 
     def prefill_layer(self, layer: int, x, logits, T: int, y=None):

@@ -73,6 +73,30 @@ def test_single_expert_is_plain_mlp(orc):
         assert np.allclose(y[t], ref, rtol=1e-12, atol=1e-15)
 
 
+@pytest.mark.parametrize("n_shared,gated", [(1, False), (2, True)])
+def test_shared_experts_vs_textbook_moe(orc, n_shared, gated):
+    # textbook MoE with always-on shared experts: y_t = sum_j w_tj E_j(x_t) +
+    # sum_s g_t S_s(x_t), every expert a dense SwiGLU MLP from the numpy decoder
+    E, k, H, I, g, T = 8, 2, 64, 32, 32, 5
+    slots, dense = _bank(orc, E + n_shared, H, I, g, 4, 4, seed=3)
+    x = synth.activations(4, 0, T, H)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    logits = synth.router_logits(4, 0, T, E, beta=0.0)
+    gate = synth.rng(9, T).uniform(0.2, 1.0, T).astype(np.float32) if gated else None
+    ids, w, _ = orc.route_shared(logits, k, n_shared, gate)
+    r_ids, r_w, _ = orc.route(logits, k)
+    assert np.array_equal(ids[:, :k], r_ids) and np.array_equal(w[:, :k], r_w)
+    assert np.all(ids[:, k:] == np.arange(E, E + n_shared))
+    y = orc.expert_ffn(x, H, I, g, 4, 4, ids, w, slots)
+    ref = _dense_moe(xf, dense[:E], r_ids, r_w, I)
+    for s in range(n_shared):
+        Wgu, Wd = dense[E + s]
+        for t in range(T):
+            a, u = Wgu[:I] @ xf[t], Wgu[I:] @ xf[t]
+            ref[t] += (float(gate[t]) if gated else 1.0) * (Wd @ (a * u / (1.0 + np.exp(-a))))
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-15)
+
+
 def test_zero_input_gives_zero_output(orc):
     slots, _ = _bank(orc, 2, 64, 32, 32, 3, 3)
     x = np.zeros((2, 64), np.uint16)
