@@ -784,6 +784,126 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
+# Guessed prefetch: hidden states as a residual stream, per-layer routers on
+# the GPU (moe_router_logits), the next two layers' routers evaluated on each
+# layer's state, their guessed misses read ahead (moe_decode_layer_ahead).
+# name: (layers, E, k, H, I, g, bits_gu, bits_down, T, slots per layer, description)
+AHEAD = {
+    "decode_ahead": (48, 512, 10, 2048, 512, 64, 3, 3, 1, 192,
+                     "Flash-Next-like decode with guessed prefetch: 48 layers x 512 experts, top-10, H 2048, I 512, "
+                     "3-bit g64, 1 token/step, 192 slots/layer, misses installed from pinned host; hidden states a "
+                     "residual stream (consecutive layers at correlation 0.89), logits = router(x) on the GPU, the "
+                     "next two layers' routers run on each layer's state and their guessed misses read ahead"),
+}
+
+
+def run_decode_ahead(args, rank, world, local_rank):
+    """The same token sequence twice from the same initial cache: plain
+    decode layers, then decode layers with guessed prefetch; both time the
+    whole path including the routers."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from streamed_quantized_expert_b200 import build as libbuild
+    from streamed_quantized_expert_b200 import ops, synth
+
+    libbuild.build()
+    ops.lib()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    cfg = AHEAD[args.config]
+    n_layers, E, k, H, I, g, bg, bd, T, S, desc_txt = cfg
+    seed = 1000 * rank
+    steps_total = args.warmup + args.steps
+    xs = torch.from_numpy(np.stack([synth.hidden_stream(seed, n_layers, T, H, step=i)
+                                    for i in range(steps_total)]).view(np.int16)).to(device)
+    Wr = torch.from_numpy(np.stack([synth.router_weights(seed, l, E, H) for l in range(n_layers)]).view(np.int16)
+                          ).to(device)
+    br = torch.from_numpy(np.stack([synth.router_bias(seed, l, E) for l in range(n_layers)])).to(device)
+    scale = 1.0 / float(np.sqrt(H))
+    logits = torch.empty((n_layers, T, E), dtype=torch.float32, device=device)
+    glog = torch.empty((n_layers, 2, T, E), dtype=torch.float32, device=device)
+    results = {}
+    for mode in ("plain", "ahead"):
+        st = build_streamer(cfg, seed, device)
+        s = st.stream
+
+        def step(i):
+            for l in range(n_layers):
+                ops.moe_router_logits(xs[i, l], T, Wr[l], br[l], scale, E, H, logits[l], s)
+                if mode == "plain":
+                    st.decode_layer(l, xs[i, l], logits[l], T, 0.0)
+                    continue
+                guesses = []
+                for d in range(1, args.ahead_layers + 1):
+                    if l + d < n_layers:
+                        ops.moe_router_logits(xs[i, l], T, Wr[l + d], br[l + d], scale, E, H, glog[l, d - 1], s)
+                        guesses.append((l + d, glog[l, d - 1], args.ahead_top))
+                st.decode_layer_ahead(l, xs[i, l], logits[l], T, 0.0, guesses)
+
+        for i in range(args.warmup):
+            step(i)
+        torch.cuda.synchronize(device)
+        if world > 1:
+            dist.barrier()
+        inst0, bytes0, pf0 = st.installs, st.installed_bytes, st.prefetch.stats()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local_rank) as clk:
+            torch.cuda.synchronize(device)
+            e0.record(s)
+            for i in range(args.warmup, steps_total):
+                step(i)
+            e1.record(s)
+            torch.cuda.synchronize(device)
+        st.ahead.synchronize()
+        ms = max_over_ranks([e0.elapsed_time(e1)], device)[0]
+        pf = {key: v - pf0[key] for key, v in st.prefetch.stats().items()}
+        results[mode] = {"ms": ms, "installs": st.installs - inst0, "bytes": st.installed_bytes - bytes0, "pf": pf,
+                         "clocks": clk.summary(), "dev_err": st.check_dev_err(), "launches": st.launches}
+        del st
+        torch.cuda.empty_cache()
+    if rank != 0:
+        return None
+    r0, r1 = results["plain"], results["ahead"]
+    tokens = args.steps * T * world
+    sb = ops.moe_slot_bytes(ops.desc(E, k, H, I, g, bg, bd))
+    pf = r1["pf"]
+    per_tok = lambda v: round(v / max(args.steps * T, 1), 2)
+    return {
+        "metric": METRIC,
+        "value": round(tokens / (r1["ms"] / 1e3), 3),
+        "unit": "tok/s",
+        "value_is": "decode tok/s of the whole path with guessed prefetch (routers + route+sort+lookup+installs+FFN"
+                    "+combine, %d layers)" % n_layers,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(r1["ms"] / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 (3-bit codes, bf16 tensor-core operands, fp32 accumulate)",
+        "data": "synthetic (seeded N(0,0.02) experts quantised on the GPU; residual-stream bf16 hidden states; "
+                "N(0,1) bf16 routers with a log-Zipf popularity bias)",
+        "config": {"workload": desc_txt, "layers": n_layers, "experts": E, "top_k": k, "hidden": H,
+                   "intermediate": I, "group": g, "bits": [bg, bd], "tokens_per_step": T, "slots_per_layer": S,
+                   "guessed_layers_ahead": args.ahead_layers, "guesses_read_per_token": args.ahead_top or k,
+                   "parallelism": f"replicas x{world} (independent token streams)"},
+        "without_prefetch": {"value": round(tokens / (r0["ms"] / 1e3), 3), "unit": "tok/s",
+                             "ms_per_step": round(r0["ms"] / args.steps, 4),
+                             "installs_per_token": per_tok(r0["installs"])},
+        "installs": {"per_token": per_tok(r1["installs"]),
+                     "guessed_per_token": per_tok(pf["guessed"]),
+                     "guessed_copies_per_token": per_tok(pf["started"]),
+                     "guesses_entered_per_token": per_tok(pf["entered"]),
+                     "guesses_wasted_per_token": per_tok(pf["wasted"]),
+                     "skipped_in_flight_per_token": per_tok(pf["skipped_in_flight"]),
+                     "bytes_per_token": round((r1["bytes"] + pf["started"] * sb) / max(args.steps * T, 1)),
+                     "how": "installs: the layers' own misses; guessed: distinct experts of the two guessed "
+                            "layers' top-k per layer; copies: guesses absent from the cache; entered: copies "
+                            "that landed before their layer ran and found their expert still absent"},
+        "dev_err": r0["dev_err"] | r1["dev_err"],
+        "clocks": r1["clocks"],
+    }
+
+
 def install_copy_rate(st, device, n=32, reps=3):
     """GB/s of moe_install_slots copying n experts' slot bytes from the pinned
     bank into a scratch pool (best of `reps`), CUDA events on the side stream."""
@@ -984,8 +1104,11 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", choices=sorted(CONFIGS) + sorted(PREFILL) + sorted(SEQUENCE), default="decode")
+    ap.add_argument("--config", choices=sorted(CONFIGS) + sorted(PREFILL) + sorted(SEQUENCE) + sorted(AHEAD),
+                    default="decode")
     ap.add_argument("--cpu-layers", type=int, default=8)
+    ap.add_argument("--ahead-layers", type=int, default=2, help="decode_ahead: layers guessed ahead (0..2)")
+    ap.add_argument("--ahead-top", type=int, default=0, help="decode_ahead: best guesses read per token (0 = k)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ffn-reps", type=int, default=20)
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (small profiling runs)")
@@ -1019,7 +1142,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run = run_prefill if args.config in PREFILL else run_sequence if args.config in SEQUENCE else run_ours
+        run = (run_prefill if args.config in PREFILL else run_sequence if args.config in SEQUENCE else
+               run_decode_ahead if args.config in AHEAD else run_ours)
         out = run(args, rank, world, local_rank)
         if out is not None:
             print(json.dumps(out), flush=True)

@@ -292,6 +292,18 @@ moe_status moe_dequant_slot(const void* pool, int32_t slot, const moe_layer_desc
 moe_status moe_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t group, int32_t bits,
                              int32_t gate_up_I, uint8_t* proj, cudaStream_t stream);
 
+/* Router projection (the guess input of moe_decode_layer_ahead: a layer's
+ * router evaluated on an earlier layer's hidden state; RFC "How the
+ * prototype works", item "Reads"):
+ *   logits[t][e] = scale * sum_h x[t][h] * W[e][h] + (bias ? bias[e] : 0)
+ *   x      device bf16 [T, H], 16-byte aligned; H a multiple of 8
+ *   W      device bf16 [E, H] (row e = expert e's router weights), aligned
+ *   bias   device fp32 [E] or NULL
+ *   logits device fp32 [T, E]
+ * fp32 accumulation in a fixed order (deterministic). */
+moe_status moe_router_logits(const uint16_t* x, int32_t T, const uint16_t* W, const float* bias, float scale,
+                             int32_t E, int32_t H, float* logits, cudaStream_t stream);
+
 /* Test: the fp32 exp used by moe_route, elementwise on n device floats. */
 moe_status moe_exp_portable(const float* x, int64_t n, float* out, cudaStream_t stream);
 
@@ -361,6 +373,22 @@ void moe_cache_stats(const moe_cache* c, int64_t* hits, int64_t* misses, int64_t
 /* Experts of `layer` that currently have a slot (E means fully resident). */
 int32_t moe_cache_resident(const moe_cache* c, int32_t layer);
 
+/* Guessed prefetch (RFC "How the prototype works", item "Reads": the next two
+ * layers' experts are guessed and read in the background).  For each of the
+ * n experts (host) that is neither resident nor already reserved, take the
+ * least recently used slot of the layer that has no copy in flight (empty
+ * slots first), evict its owner and reserve the slot for the expert, which
+ * stays out of the table until moe_cache_commit.  Writes the n_out reserved
+ * (expert, slot) pairs; stops early when every slot has a copy in flight.
+ * moe_cache_step never takes a reserved slot. */
+moe_status moe_cache_reserve(moe_cache* c, int32_t layer, const int32_t* experts, int32_t n, int32_t* out_experts,
+                             int32_t* out_slots, int32_t* n_out);
+/* The copy into reserved `slot` has landed: its expert enters the table as
+ * the most recent (*entered = 1), or, if the expert was installed elsewhere
+ * meanwhile, the slot becomes empty (*entered = 0).  MOE_ERR_INVALID if the
+ * slot holds no reservation. */
+moe_status moe_cache_commit(moe_cache* c, int32_t layer, int32_t slot, int32_t* entered);
+
 /* ------------------------------------------------------------------------
  * Native driver of one decode layer (the sequence of the calls above).
  * ---------------------------------------------------------------------- */
@@ -421,6 +449,55 @@ typedef struct {
 moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc, const moe_step_buffers* b,
                             const uint16_t* x, const float* logits, int32_t T, float L, float* y,
                             cudaStream_t stream, cudaStream_t side, cudaEvent_t installed, int32_t* n_installed);
+
+/* Guessed prefetch state: per layer, the batches of guessed copies in flight. */
+typedef struct moe_prefetch moe_prefetch;
+moe_status moe_prefetch_create(int32_t n_layers, moe_prefetch** out);
+void moe_prefetch_destroy(moe_prefetch* p);
+/* Counters: guessed experts (distinct per guess), copies started, guesses
+ * entered into a table, copies wasted (the expert was installed normally
+ * first), and reservations found still in flight when their layer ran. */
+void moe_prefetch_stats(const moe_prefetch* p, int64_t* guessed, int64_t* started, int64_t* entered,
+                        int64_t* wasted, int64_t* skipped);
+
+/* One guessed layer: its router evaluated on the current layer's hidden state. */
+typedef struct {
+  int32_t layer;           /* the guessed layer (not the current one) */
+  const moe_layer_ctx* lc; /* its pool and tables */
+  const float* logits;     /* device fp32 [T, E] */
+  int32_t top;             /* read ahead each token's `top` best guesses (rank order); 0 = all k */
+} moe_guess;
+/* Buffers of the guessed top-k, caller-owned. */
+typedef struct {
+  int32_t* ids;      /* device int32 [2 * stride] */
+  float* w;          /* device fp32 [2 * stride] */
+  int32_t* ids_host; /* pinned host int32 [2 * stride] */
+  int32_t stride;    /* >= max_tokens * k of the guessed layers */
+} moe_guess_buffers;
+
+/* moe_decode_layer with guessed prefetch (RFC "How the prototype works",
+ * item "Reads": the next two layers' experts are guessed by running their
+ * routers on the current hidden states and read in the background;
+ * PR #50717, commit note: install_ahead skips guessed reads still in flight
+ * instead of waiting for them):
+ *   1. the guessed copies of `layer` that have landed (event query, no wait)
+ *      enter its table, which is uploaded on `stream` if it changed; copies
+ *      still in flight are skipped: their experts count as absent now;
+ *   2. moe_decode_layer's sequence, with the n_guesses (0..2) guessed
+ *      layers' top-k (moe_route, L = 0) launched next to the layer's own
+ *      stages and read back on the same synchronisation (one more if the
+ *      layer itself is fully resident);
+ *   3. after the layer's own misses have their slots, each guessed layer's
+ *      absent guesses get reserved slots (moe_cache_reserve) and their
+ *      copies start on `ahead` (a stream of their own, so the layer's own
+ *      installs never queue behind them), one event per batch.
+ * The results (y) are those of moe_decode_layer: the guesses only move
+ * installs earlier. */
+moe_status moe_decode_layer_ahead(moe_cache* cache, moe_prefetch* pf, int32_t layer, const moe_layer_ctx* lc,
+                                  const moe_step_buffers* b, const uint16_t* x, const float* logits, int32_t T,
+                                  float L, float* y, cudaStream_t stream, cudaStream_t side, cudaEvent_t installed,
+                                  int32_t* n_installed, const moe_guess* guesses, int32_t n_guesses,
+                                  const moe_guess_buffers* gb, cudaStream_t ahead);
 
 #ifdef __cplusplus
 }

@@ -116,6 +116,19 @@ def route(logits: np.ndarray, k: int, L: float = 0.0, slot_table: np.ndarray | N
     return ids, w, u
 
 
+def router_logits(x_bf16: np.ndarray, W_bf16: np.ndarray, bias, scale: float) -> np.ndarray:
+    """logits[t][e] = scale * sum_h x[t][h] W[e][h] + bias[e], in double from
+    the bf16 inputs: a layer's router evaluated on a hidden state (RFC "How
+    the prototype works", item "Reads": the next layers' routers run on the
+    current hidden states to guess their experts)."""
+    x = (np.ascontiguousarray(x_bf16, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    W = (np.ascontiguousarray(W_bf16, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    out = float(scale) * (x @ W.T)
+    if bias is not None:
+        out += np.asarray(bias, np.float32).astype(np.float64)[None, :]
+    return out
+
+
 def route_shared(logits: np.ndarray, k: int, n_shared: int, shared_w=None, L: float = 0.0,
                  slot_table: np.ndarray | None = None):
     """route(), then every token's always-on shared experts (BigMoeOnEdge

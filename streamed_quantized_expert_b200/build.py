@@ -19,7 +19,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 SO = os.path.join(HERE, "libmoe.so")
 OBJ_DIR = os.path.join(HERE, "_build")
-SOURCES = ["api.cu", "route_sort.cu", "quant.cu", "ffn_decode.cu", "ffn_fused.cu", "prefill_tc.cu", "noalloc.cu",
+SOURCES = ["api.cu", "route_sort.cu", "router.cu", "quant.cu", "ffn_decode.cu", "ffn_fused.cu", "prefill_tc.cu", "noalloc.cu",
            "slot_cache.cpp", "driver.cpp"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

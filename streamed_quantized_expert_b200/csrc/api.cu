@@ -294,6 +294,15 @@ moe_status moe_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t gr
   return cuda_status(launch_quantize(w, rows, K, group, bits, gate_up_I, proj, stream));
 }
 
+moe_status moe_router_logits(const uint16_t* x, int32_t T, const uint16_t* W, const float* bias, float scale,
+                             int32_t E, int32_t H, float* logits, cudaStream_t stream) {
+  if (T < 0 || E < 1 || H < 8 || H % 8 || !(scale == scale)) return MOE_ERR_INVALID;
+  if (T == 0) return MOE_OK;
+  if (!x || !W || !logits || !aligned(x, 16) || !aligned(W, 16)) return MOE_ERR_INVALID;
+  if (T > 65535) return MOE_ERR_UNSUPPORTED;
+  return cuda_status(launch_router(x, W, bias, scale, T, E, H, logits, stream));
+}
+
 moe_status moe_exp_portable(const float* x, int64_t n, float* out, cudaStream_t stream) {
   if (n < 0 || (n > 0 && (!x || !out))) return MOE_ERR_INVALID;
   return cuda_status(launch_exp(x, n, out, stream));

@@ -10,6 +10,18 @@
 // RFC "How the prototype works": each layer copies its routing to the host
 // once; misses become one host-to-device copy per expert; when every expert
 // is resident the layer never synchronises with the host.
+//
+// Guessed prefetch (same page, item "Reads": the next two layers' experts are
+// guessed by running their routers on the current hidden states and read in
+// the background; PR #50717 commit note: install_ahead skips guessed reads
+// still in flight instead of waiting for them).  moe_decode_layer_ahead routes
+// the guessed layers' logits (top-k, L = 0) next to the layer's own stages, so
+// their ids come back with the layer's one synchronisation; the guessed
+// misses get slots reserved in the cache and their copies start on an `ahead`
+// stream of their own, one event per batch.  At the start of a layer its
+// landed batches are entered into the table (an event query, never a wait);
+// batches still in flight are skipped and stay reserved.
+#include <algorithm>
 #include <cstring>
 #include <vector>
 
@@ -25,10 +37,103 @@ extern "C" moe_status moe_internal_expert_ffn(const uint16_t* x, int32_t T, cons
                                               float* y_accum, void* ws, size_t ws_bytes, int32_t* dev_err,
                                               cudaStream_t stream, int overwrite);
 
-extern "C" moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc,
-                                       const moe_step_buffers* b, const uint16_t* x, const float* logits,
-                                       int32_t T, float L, float* y, cudaStream_t stream, cudaStream_t side,
-                                       cudaEvent_t installed, int32_t* n_installed) {
+struct moe_prefetch {
+  struct Batch {
+    cudaEvent_t ev;
+    std::vector<int32_t> slots;
+  };
+  std::vector<std::vector<Batch>> q;  // [layer]: guessed copies in flight, oldest first
+  std::vector<cudaEvent_t> spare;     // recycled events
+  std::vector<uint8_t> dirty;         // [layer]: host table changed by reservations since the last upload
+  int64_t guessed = 0, started = 0, entered = 0, wasted = 0, skipped = 0;
+};
+
+namespace {
+
+struct Guess {
+  moe_prefetch* pf;
+  const moe_guess* g;
+  int32_t n;
+  const moe_guess_buffers* gb;
+  cudaStream_t ahead;
+};
+
+// Enter the landed guessed copies of `layer` into the table; upload it on
+// `stream` if reservations or entries changed it.
+moe_status retire(moe_prefetch* pf, moe_cache* cache, int32_t layer, const moe_layer_ctx* lc, cudaStream_t stream) {
+  auto& q = pf->q[layer];
+  size_t done = 0;
+  for (; done < q.size(); ++done) {
+    const cudaError_t e = cudaEventQuery(q[done].ev);
+    if (e == cudaErrorNotReady) break;  // this batch and the later ones are still in flight: skipped
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    for (int32_t slot : q[done].slots) {
+      int32_t in = 0;
+      if (moe_cache_commit(cache, layer, slot, &in) != MOE_OK) return MOE_ERR_INVALID;
+      pf->entered += in;
+      pf->wasted += 1 - in;
+    }
+    pf->spare.push_back(q[done].ev);
+    pf->dirty[layer] = 1;
+  }
+  for (size_t i = done; i < q.size(); ++i) pf->skipped += (int64_t)q[i].slots.size();
+  q.erase(q.begin(), q.begin() + (ptrdiff_t)done);
+  if (pf->dirty[layer]) {
+    const int32_t E0 = lc->desc->E;
+    std::memcpy(lc->table_stage, moe_cache_table(cache, layer), sizeof(int32_t) * (size_t)E0);
+    if (cudaMemcpyAsync(lc->table_dev, lc->table_stage, sizeof(int32_t) * (size_t)E0, cudaMemcpyHostToDevice,
+                        stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    pf->dirty[layer] = 0;
+  }
+  return MOE_OK;
+}
+
+// The guessed layers' experts (ids back on the host): reserve slots for the
+// misses and start their copies on the ahead stream.
+moe_status start_guesses(const Guess& G, moe_cache* cache, int32_t T) {
+  thread_local std::vector<int32_t> want, out_e, out_s;
+  thread_local std::vector<const void*> rows;
+  for (int32_t gi = 0; gi < G.n; ++gi) {
+    const moe_guess& g = G.g[gi];
+    const int32_t k = g.lc->desc->k, E0 = g.lc->desc->E;
+    const int32_t* ids = G.gb->ids_host + (size_t)gi * G.gb->stride;
+    const int32_t top = g.top > 0 && g.top < k ? g.top : k;  // ids are in rank order per token
+    want.clear();
+    for (int32_t t = 0; t < T; ++t) want.insert(want.end(), ids + (size_t)t * k, ids + (size_t)t * k + top);
+    std::sort(want.begin(), want.end());
+    want.erase(std::unique(want.begin(), want.end()), want.end());
+    while (!want.empty() && (want.back() >= E0 || want.back() < 0)) want.pop_back();
+    G.pf->guessed += (int64_t)want.size();
+    out_e.resize(want.size());
+    out_s.resize(want.size());
+    int32_t n = 0;
+    moe_status s = moe_cache_reserve(cache, g.layer, want.data(), (int32_t)want.size(), out_e.data(), out_s.data(), &n);
+    if (s != MOE_OK) return s;
+    if (n == 0) continue;
+    rows.resize(n);
+    for (int32_t i = 0; i < n; ++i) rows[i] = g.lc->bank_rows[out_e[i]];
+    s = moe_install_slots(g.lc->pool, g.lc->slot_bytes, g.lc->n_slots, rows.data(), out_s.data(), n, G.ahead,
+                          nullptr);
+    if (s != MOE_OK) return s;
+    cudaEvent_t ev;
+    if (!G.pf->spare.empty()) {
+      ev = G.pf->spare.back();
+      G.pf->spare.pop_back();
+    } else if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) {
+      return MOE_ERR_CUDA;
+    }
+    if (cudaEventRecord(ev, G.ahead) != cudaSuccess) return MOE_ERR_CUDA;
+    G.pf->q[g.layer].push_back({ev, std::vector<int32_t>(out_s.begin(), out_s.begin() + n)});
+    G.pf->dirty[g.layer] = 1;  // victims left the table
+    G.pf->started += n;
+  }
+  return MOE_OK;
+}
+
+moe_status decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc, const moe_step_buffers* b,
+                        const uint16_t* x, const float* logits, int32_t T, float L, float* y, cudaStream_t stream,
+                        cudaStream_t side, cudaEvent_t installed, int32_t* n_installed, const Guess* G) {
   if (!cache || !lc || !b || !lc->desc || !y || !x || !logits) return MOE_ERR_INVALID;
   const moe_layer_desc* d0 = lc->desc;  // the routed experts
   const int32_t ns = lc->n_shared;
@@ -53,7 +158,26 @@ extern "C" moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const mo
   s = moe_sort(b->ids, xs ? x : nullptr, T, d, b->offsets, b->pairs, active, n_active, xs, b->ws, b->ws_bytes,
                stream);
   if (s != MOE_OK) return s;
-  if (moe_cache_resident(cache, layer) < E0) {
+  // the guessed layers' top-k, on the same synchronisation as the layer's own lookup
+  const bool guessing = G && G->n > 0;
+  if (guessing) {
+    for (int32_t gi = 0; gi < G->n; ++gi) {
+      const moe_guess& g = G->g[gi];
+      int32_t* gids = G->gb->ids + (size_t)gi * G->gb->stride;
+      s = moe_route(g.logits, T, g.lc->desc, 0.0f, nullptr, gids, G->gb->w + (size_t)gi * G->gb->stride, stream);
+      if (s != MOE_OK) return s;
+      if (cudaMemcpyAsync(G->gb->ids_host + (size_t)gi * G->gb->stride, gids,
+                          sizeof(int32_t) * (size_t)T * g.lc->desc->k, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+  }
+  const bool resident = moe_cache_resident(cache, layer) >= E0;
+  if (resident && guessing) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+    s = start_guesses(*G, cache, T);
+    if (s != MOE_OK) return s;
+  }
+  if (!resident) {
     s = moe_slot_lookup(lc->table_dev, active, n_active, 0, E, lc->n_slots, b->slots, miss, n_miss, b->dev_err,
                         stream);
     if (s != MOE_OK) return s;
@@ -72,6 +196,10 @@ extern "C" moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const mo
     // ns entries, and the cache manages the routed ones only
     s = moe_cache_step(cache, layer, b->meta_host + 2, na - ns, out_e.data(), out_s.data(), &n);
     if (s != MOE_OK) return s;
+    if (guessing) {  // after this layer's own misses have their slots
+      s = start_guesses(*G, cache, T);
+      if (s != MOE_OK) return s;
+    }
     if (n > 0) {
       rows.resize(n);
       for (int32_t i = 0; i < n; ++i) rows[i] = lc->bank_rows[out_e[i]];
@@ -118,3 +246,61 @@ extern "C" moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const mo
   return moe_internal_expert_ffn(x, T, d, lc->pool, lc->n_slots, lc->table_dev, b->ids, b->w, b->offsets, b->pairs,
                                  active, n_active, xs, 0, E, y, b->ws, b->ws_bytes, b->dev_err, stream, 1);
 }
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc, const moe_step_buffers* b,
+                            const uint16_t* x, const float* logits, int32_t T, float L, float* y,
+                            cudaStream_t stream, cudaStream_t side, cudaEvent_t installed, int32_t* n_installed) {
+  return decode_layer(cache, layer, lc, b, x, logits, T, L, y, stream, side, installed, n_installed, nullptr);
+}
+
+moe_status moe_prefetch_create(int32_t n_layers, moe_prefetch** out) {
+  if (!out || n_layers < 1) return MOE_ERR_INVALID;
+  moe_prefetch* p = new moe_prefetch();
+  p->q.resize(n_layers);
+  p->dirty.assign(n_layers, 0);
+  *out = p;
+  return MOE_OK;
+}
+
+void moe_prefetch_destroy(moe_prefetch* p) {
+  if (!p) return;
+  for (auto& q : p->q)
+    for (auto& b : q) cudaEventDestroy(b.ev);
+  for (cudaEvent_t e : p->spare) cudaEventDestroy(e);
+  delete p;
+}
+
+void moe_prefetch_stats(const moe_prefetch* p, int64_t* guessed, int64_t* started, int64_t* entered,
+                        int64_t* wasted, int64_t* skipped) {
+  if (!p) return;
+  if (guessed) *guessed = p->guessed;
+  if (started) *started = p->started;
+  if (entered) *entered = p->entered;
+  if (wasted) *wasted = p->wasted;
+  if (skipped) *skipped = p->skipped;
+}
+
+moe_status moe_decode_layer_ahead(moe_cache* cache, moe_prefetch* pf, int32_t layer, const moe_layer_ctx* lc,
+                                  const moe_step_buffers* b, const uint16_t* x, const float* logits, int32_t T,
+                                  float L, float* y, cudaStream_t stream, cudaStream_t side, cudaEvent_t installed,
+                                  int32_t* n_installed, const moe_guess* guesses, int32_t n_guesses,
+                                  const moe_guess_buffers* gb, cudaStream_t ahead) {
+  if (!cache || !pf || layer < 0 || layer >= (int32_t)pf->q.size() || !lc || !lc->desc) return MOE_ERR_INVALID;
+  if (n_guesses < 0 || n_guesses > 2 || (n_guesses > 0 && (!guesses || !gb))) return MOE_ERR_INVALID;
+  for (int32_t i = 0; i < n_guesses; ++i) {
+    const moe_guess& g = guesses[i];
+    if (!g.lc || !g.lc->desc || !g.logits || g.layer < 0 || g.layer >= (int32_t)pf->q.size() || g.layer == layer)
+      return MOE_ERR_INVALID;
+    if ((int64_t)T * g.lc->desc->k > gb->stride) return MOE_ERR_CAPACITY;
+  }
+  moe_status s = retire(pf, cache, layer, lc, stream);
+  if (s != MOE_OK) return s;
+  const Guess G{pf, guesses, n_guesses, gb, ahead};
+  return decode_layer(cache, layer, lc, b, x, logits, T, L, y, stream, side, installed, n_installed, &G);
+}
+
+}  // extern "C"

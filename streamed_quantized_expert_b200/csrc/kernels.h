@@ -69,6 +69,8 @@ inline cudaError_t launch_pdl(const void* func, int grid, int block, size_t smem
   return cudaLaunchKernelExC(&cfg, func, argv);
 }
 
+cudaError_t launch_router(const uint16_t* x, const uint16_t* W, const float* bias, float scale, int T, int E, int H,
+                          float* logits, cudaStream_t st);
 cudaError_t launch_route(const float* logits, int T, int E, int k, float L, const int32_t* table, int32_t* ids,
                          float* w, int n_shared, const float* shared_w, cudaStream_t st);
 size_t sort_ws_bytes(int n, int E);

@@ -26,6 +26,8 @@ ABI_SYMBOLS = [
     "moe_cache_class_slots", "moe_cache_place", "moe_cache_step", "moe_cache_stats",
     "moe_expert_ffn_noalloc", "moe_noalloc_scratch_bytes", "moe_cache_resident", "moe_decode_layer",
     "moe_last_cuda_error", "moe_ffn_kernel_path", "moe_set_wait_limit_cycles", "moe_route_shared",
+    "moe_router_logits", "moe_cache_reserve", "moe_cache_commit", "moe_prefetch_create", "moe_prefetch_destroy",
+    "moe_prefetch_stats", "moe_decode_layer_ahead",
 ]
 
 
@@ -56,6 +58,14 @@ class LayerCtx(C.Structure):
     _fields_ = [("desc", C.POINTER(LayerDesc)), ("pool", C.c_void_p), ("n_slots", C.c_int32),
                 ("slot_bytes", C.c_size_t), ("table_dev", C.c_void_p), ("table_stage", C.c_void_p),
                 ("bank_rows", C.POINTER(C.c_void_p)), ("n_shared", C.c_int32), ("shared_w", C.c_void_p)]
+
+
+class Guess(C.Structure):
+    _fields_ = [("layer", C.c_int32), ("lc", C.POINTER(LayerCtx)), ("logits", C.c_void_p), ("top", C.c_int32)]
+
+
+class GuessBuffers(C.Structure):
+    _fields_ = [("ids", C.c_void_p), ("w", C.c_void_p), ("ids_host", C.c_void_p), ("stride", C.c_int32)]
 
 
 class SlotLayout(C.Structure):
@@ -104,6 +114,15 @@ def lib():
             "moe_cache_resident": (i32, [P, i32]),
             "moe_decode_layer": (C.c_int, [P, i32, C.POINTER(LayerCtx), C.POINTER(StepBuffers), P, P, i32, f32, P,
                                            P, P, P, C.POINTER(i32)]),
+            "moe_router_logits": (C.c_int, [P, i32, P, P, f32, i32, i32, P, P]),
+            "moe_cache_reserve": (C.c_int, [P, i32, P, i32, P, P, P]),
+            "moe_cache_commit": (C.c_int, [P, i32, i32, P]),
+            "moe_prefetch_create": (C.c_int, [i32, C.POINTER(P)]),
+            "moe_prefetch_destroy": (None, [P]),
+            "moe_prefetch_stats": (None, [P, P, P, P, P, P]),
+            "moe_decode_layer_ahead": (C.c_int, [P, P, i32, C.POINTER(LayerCtx), C.POINTER(StepBuffers), P, P, i32,
+                                                 f32, P, P, P, P, C.POINTER(i32), C.POINTER(Guess), i32,
+                                                 C.POINTER(GuessBuffers), P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -306,10 +325,65 @@ class SlotCache:
     def resident(self, layer: int) -> int:
         return int(lib().moe_cache_resident(self._h, layer))
 
+    def reserve(self, layer: int, experts):
+        """Returns [(expert, slot), ...] reserved for guessed copies."""
+        n = len(experts)
+        ea = (C.c_int32 * max(n, 1))(*[int(e) for e in experts])
+        nout = C.c_int32(0)
+        _ck(lib().moe_cache_reserve(self._h, layer, ea, n, self._out_e, self._out_s, C.byref(nout)),
+            "moe_cache_reserve")
+        return [(self._out_e[i], self._out_s[i]) for i in range(nout.value)]
+
+    def commit(self, layer: int, slot: int) -> bool:
+        """The guessed copy into `slot` landed; True if its expert entered the table."""
+        ent = C.c_int32(0)
+        _ck(lib().moe_cache_commit(self._h, layer, int(slot), C.byref(ent)), "moe_cache_commit")
+        return bool(ent.value)
+
     def stats(self):
         h, m, e = C.c_int64(), C.c_int64(), C.c_int64()
         lib().moe_cache_stats(self._h, C.byref(h), C.byref(m), C.byref(e))
         return h.value, m.value, e.value
+
+
+def moe_router_logits(x, T, W, bias, scale, E, H, logits, stream=None) -> None:
+    _ck(lib().moe_router_logits(_ptr(x), int(T), _ptr(W), _ptr(bias), float(scale), int(E), int(H), _ptr(logits),
+                                _stream(stream)), "moe_router_logits")
+
+
+class Prefetch:
+    """moe_prefetch_*: the guessed copies in flight, per layer."""
+
+    def __init__(self, n_layers: int):
+        h = C.c_void_p()
+        _ck(lib().moe_prefetch_create(n_layers, C.byref(h)), "moe_prefetch_create")
+        self._h = h
+
+    def close(self):
+        if self._h:
+            lib().moe_prefetch_destroy(self._h)
+            self._h = None
+
+    __del__ = close
+
+    def stats(self) -> dict:
+        v = [C.c_int64() for _ in range(5)]
+        lib().moe_prefetch_stats(self._h, *[C.byref(x) for x in v])
+        return dict(zip(("guessed", "started", "entered", "wasted", "skipped_in_flight"), [x.value for x in v]))
+
+
+def moe_decode_layer_ahead(cache: "SlotCache", pf: Prefetch, layer: int, ctx: LayerCtx, bufs: StepBuffers, x,
+                           logits, T: int, L: float, y, stream, side, installed, guesses, gbufs: GuessBuffers,
+                           ahead) -> int:
+    """moe_decode_layer with guessed prefetch; guesses: [(layer, LayerCtx, logits tensor, top), ...] (0..2)."""
+    n = C.c_int32(0)
+    ev = installed if isinstance(installed, int) else installed.cuda_event
+    ga = (Guess * max(len(guesses), 1))(*[Guess(int(gl), C.pointer(gc), _ptr(glog), int(top))
+                                          for gl, gc, glog, top in guesses])
+    _ck(lib().moe_decode_layer_ahead(cache._h, pf._h, int(layer), C.byref(ctx), C.byref(bufs), _ptr(x), _ptr(logits),
+                                     int(T), float(L), _ptr(y), _stream(stream), _stream(side), ev, C.byref(n), ga,
+                                     len(guesses), C.byref(gbufs), _stream(ahead)), "moe_decode_layer_ahead")
+    return n.value
 
 
 def moe_decode_layer(cache: "SlotCache", layer: int, ctx: LayerCtx, bufs: StepBuffers, x, logits, T: int, L: float,

@@ -138,6 +138,14 @@ class Streamer:
                                           self.class_bytes[self.layer_class[l]], self.table_dev[l].data_ptr(),
                                           self.table_pin[l].data_ptr(), rows, n_shared, None))
         self.ffn_events = None     # list to collect (start, end) CUDA events around FFN calls
+        # guessed prefetch (moe_decode_layer_ahead): its own copy stream, state and buffers
+        self.prefetch = ops.Prefetch(self.n_layers)
+        self.ahead = torch.cuda.Stream(self.device)
+        stride = max(max_tokens * self.k, 1)
+        self.g_ids = torch.empty(2 * stride, dtype=torch.int32, device=self.device)
+        self.g_w = torch.empty(2 * stride, dtype=torch.float32, device=self.device)
+        self.g_ids_pin = torch.empty(2 * stride, dtype=torch.int32).pin_memory()
+        self._gbufs = ops.GuessBuffers(self.g_ids.data_ptr(), self.g_w.data_ptr(), self.g_ids_pin.data_ptr(), stride)
 
     # -- views into meta --------------------------------------------------
     def _n_active(self):
@@ -247,6 +255,22 @@ class Streamer:
             self.installs += n
             self.installed_bytes += n * self.class_bytes[self.layer_class[layer]]
         self.launches += 4 + (0 if full else 1) + (0 if T * self.kw <= 1024 else 2)
+        return y
+
+    def decode_layer_ahead(self, layer: int, x, logits, T: int, L: float = 0.0, guesses=(), y=None):
+        """decode_layer with guessed prefetch (moe_decode_layer_ahead).
+        guesses: up to two (later layer, logits [T, E] device[, top]) tuples,
+        each that layer's router evaluated on this layer's hidden state; top =
+        how many of each token's best guesses to read ahead (default all k)."""
+        y = self.y[:T] if y is None else y
+        full = self.cache.resident(layer) >= self.E
+        g = [(gu[0], self._ctx[gu[0]], gu[1], gu[2] if len(gu) > 2 else 0) for gu in guesses]
+        n = ops.moe_decode_layer_ahead(self.cache, self.prefetch, layer, self._ctx[layer], self._bufs, x, logits, T,
+                                       L, y, self.stream, self.side, self.installed, g, self._gbufs, self.ahead)
+        if n:
+            self.installs += n
+            self.installed_bytes += n * self.class_bytes[self.layer_class[layer]]
+        self.launches += 4 + len(g) + (0 if full else 1) + (0 if T * self.kw <= 1024 else 2)
         return y
 
     def decode_layer_steps(self, layer: int, x, logits, T: int, L: float = 0.0, y=None):

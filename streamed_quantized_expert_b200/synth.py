@@ -10,13 +10,19 @@ Recipe (same shapes and distributions as the pages' workloads, synthetic):
   * expert weights: N(0, 0.02) fp32, per (bank row) sub-stream;
   * router logits: N(0, 1) + beta * (-s * ln rank_e), rank a per-layer seeded
     permutation of 1..E (a log-Zipf(s) popularity bias), beta = 0.55, s = 1.1;
+  * guessed-prefetch workload: a unit-variance residual stream of hidden
+    states, x_{l+1} = (x_l + sigma n_l) / sqrt(1 + sigma^2) with n_l ~ N(0, 1)
+    and sigma = 0.5 (consecutive layers' states at correlation 0.89), and per
+    layer router weights W ~ N(0, 1) [E, H] in bf16, so that
+    x W^T / sqrt(H) + bias is N(0, 1) + the same popularity bias as above;
   * every stream is keyed by (seed, tensor kind, layer/row, ...).
 """
 from __future__ import annotations
 
 import numpy as np
 
-KIND_X, KIND_LOGITS, KIND_RANK, KIND_WEIGHTS, KIND_BANKPERM, KIND_SLOTPERM, KIND_IDS = range(1, 8)
+KIND_X, KIND_LOGITS, KIND_RANK, KIND_WEIGHTS, KIND_BANKPERM, KIND_SLOTPERM, KIND_IDS, KIND_ROUTER, KIND_STREAM = \
+    range(1, 10)
 
 
 def rng(seed: int, *stream) -> np.random.Generator:
@@ -53,6 +59,29 @@ def router_logits(seed: int, layer: int, T: int, E: int, beta: float = 0.55, s: 
         return base
     bias = (beta * (-s * np.log(popularity_rank(seed, layer, E).astype(np.float64)))).astype(np.float32)
     return (base + bias[None, :]).astype(np.float32)
+
+
+def router_bias(seed: int, layer: int, E: int, beta: float = 0.55, s: float = 1.1) -> np.ndarray:
+    """fp32 [E]: the popularity bias of router_logits, beta * (-s * ln rank_e)."""
+    return (beta * (-s * np.log(popularity_rank(seed, layer, E).astype(np.float64)))).astype(np.float32)
+
+
+def router_weights(seed: int, layer: int, E: int, H: int) -> np.ndarray:
+    """bf16 bits [E, H] of N(0, 1): a layer's router rows."""
+    return to_bf16_bits(rng(seed, KIND_ROUTER, layer).standard_normal((E, H), dtype=np.float32))
+
+
+def hidden_stream(seed: int, n_layers: int, T: int, H: int, sigma: float = 0.5, step: int = 0) -> np.ndarray:
+    """bf16 bits [n_layers, T, H]: a unit-variance residual stream, each
+    layer's state the previous one plus sigma * N(0, 1), rescaled."""
+    r = rng(seed, KIND_STREAM, step)
+    x = r.standard_normal((T, H), dtype=np.float32)
+    out = np.empty((n_layers, T, H), np.uint16)
+    c = np.float32(1.0 / np.sqrt(1.0 + sigma * sigma))
+    for l in range(n_layers):
+        out[l] = to_bf16_bits(x)
+        x = ((x + np.float32(sigma) * r.standard_normal((T, H), dtype=np.float32)) * c).astype(np.float32)
+    return out
 
 
 def expert_weights(seed: int, bank_row: int, H: int, I: int, std: float = 0.02):
