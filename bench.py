@@ -433,7 +433,8 @@ def run_prefill(args, rank, world, local_rank, name=None, layers=0, embedded=Fal
     roof = {"bound": "tensor", "achieved": round(tflops, 2), "peak": tf_peak, "unit": "TFLOP/s",
             "frac": round(tflops / tf_peak, 4),
             "traffic": recorded_traffic("pf_gemm_kernel"),
-            "traffic_note": "DRAM bytes of one pass's gate/up + down launches (uniform routing, 4096 tokens)",
+            "traffic_note": "DRAM bytes of one 64-expert pass's gate/up + down launches of the 1024-token "
+                            "Flash-Next-like chunk (profiles/traffic.txt)",
             "hbm": {"achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4)},
             "kernel": "pf_gemm_kernel (gate/up + SwiGLU, down) + combine, per pass",
             "flops_per_layer": 2.0 * T * k * 3 * H * I, "peak_kind": peak_kind}
