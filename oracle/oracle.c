@@ -280,14 +280,22 @@ void orc_slot_lookup(const int32_t* table, const int32_t* active, int32_t n_acti
  */
 static int64_t orc_round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
-int orc_bits_supported(int32_t b) { return b == 3 || b == 4 || b == 6; }
+/* b = 16: unquantized BF16 experts (RFC "stream MoE experts from disk in
+ * from_pretrained", "How the prototype works", item "Cache": BF16 experts run
+ * through the grouped experts kernel).  Reading: a BF16 projection is its
+ * rows of K bf16 values, row-major, each row padded to a multiple of 128
+ * inputs with zeros, rows in the same storage order as the quantized formats,
+ * no scale/bias words. */
+int orc_bits_supported(int32_t b) { return b == 3 || b == 4 || b == 6 || b == 16; }
 
 int64_t orc_row_bytes(int32_t K, int32_t b) { return orc_round_up(K, 128) * b / 8; }
 
 int64_t orc_row_groups(int32_t K, int32_t g) { return orc_round_up(K, 128) / g; }
 
 /* Bytes of one 16-row tile of a projection with K inputs per row. */
-int64_t orc_tile_bytes(int32_t K, int32_t g, int32_t b) { return 16 * orc_row_bytes(K, b) + 16 * orc_row_groups(K, g) * 4; }
+int64_t orc_tile_bytes(int32_t K, int32_t g, int32_t b) {
+  return 16 * orc_row_bytes(K, b) + (b == 16 ? 0 : 16 * orc_row_groups(K, g) * 4);
+}
 
 /* off[0] = gate_up projection, off[1] = down projection, off[2] = gate_up
  * tile bytes, off[3] = down tile bytes, off[4] = slot bytes. */
@@ -364,9 +372,14 @@ static void orc_code_bit(int32_t row, int64_t row_bytes, int64_t tile_bytes, int
   *bit = bi + (odd ? 16 : 0);
 }
 
-/* Code of input k of row `row` in a projection of K inputs per row. */
+/* Code of input k of row `row` in a projection of K inputs per row (b = 16:
+ * the bf16 bits of the weight, little-endian at row * row_bytes + 2 k). */
 int32_t orc_get_code(const uint8_t* proj, int32_t K, int32_t g, int32_t row, int32_t k, int32_t b) {
   int64_t rb = orc_row_bytes(K, b), tb = orc_tile_bytes(K, g, b);
+  if (b == 16) {
+    const uint8_t* e = proj + (int64_t)row * rb + 2 * (int64_t)k;
+    return (int32_t)((uint32_t)e[0] | ((uint32_t)e[1] << 8));
+  }
   int32_t q = 0;
   for (int32_t j = 0; j < b; ++j) {
     int64_t wb;
@@ -379,6 +392,12 @@ int32_t orc_get_code(const uint8_t* proj, int32_t K, int32_t g, int32_t row, int
 
 void orc_set_code(uint8_t* proj, int32_t K, int32_t g, int32_t row, int32_t k, int32_t b, int32_t q) {
   int64_t rb = orc_row_bytes(K, b), tb = orc_tile_bytes(K, g, b);
+  if (b == 16) {
+    uint8_t* e = proj + (int64_t)row * rb + 2 * (int64_t)k;
+    e[0] = (uint8_t)q;
+    e[1] = (uint8_t)(q >> 8);
+    return;
+  }
   for (int32_t j = 0; j < b; ++j) {
     int64_t wb;
     int32_t bit;
@@ -424,6 +443,11 @@ void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32
   int64_t ng = orc_row_groups(K, g);
   int32_t qmax = (1 << b) - 1;
   memset(proj, 0, (size_t)((rows / 16) * orc_tile_bytes(K, g, b)));
+  if (b == 16) {  /* BF16 experts: the weights rounded to bf16 (nearest even) */
+    for (int32_t r = 0; r < rows; ++r)
+      for (int32_t k = 0; k < K; ++k) orc_set_code(proj, K, g, r, k, 16, orc_f32_to_bf16(w[(int64_t)r * K + k]));
+    return;
+  }
   for (int32_t r = 0; r < rows; ++r) {
     const float* wr = w + (int64_t)r * K;
     for (int64_t gi = 0; gi < ng; ++gi) {
@@ -463,6 +487,10 @@ void orc_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t g, int32
 void orc_dequant_rows(const uint8_t* proj, int32_t rows, int32_t K, int32_t g, int32_t b, float* out) {
   for (int32_t r = 0; r < rows; ++r) {
     for (int32_t k = 0; k < K; ++k) {
+      if (b == 16) {  /* BF16 experts: the stored value itself */
+        out[(int64_t)r * K + k] = orc_bf16_to_f32((uint16_t)orc_get_code(proj, K, g, r, k, 16));
+        continue;
+      }
       uint32_t sbw = orc_get_sb(proj, r, k / g, K, g, b);
       float s = orc_bf16_to_f32((uint16_t)(sbw & 0xffffu));
       float bb = orc_bf16_to_f32((uint16_t)(sbw >> 16));

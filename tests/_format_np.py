@@ -58,10 +58,11 @@ def _bit_positions(K, b):
 
 
 def geometry(K, g, b):
-    """(row bytes of codes, groups per row, tile bytes)."""
+    """(row bytes of codes, groups per row, tile bytes); b = 16 (BF16 experts)
+    has no scale/bias words."""
     rb = ceil128(K) * b // 8
     ng = ceil128(K) // g
-    return rb, ng, 16 * rb + 16 * ng * 4
+    return rb, ng, 16 * rb + (0 if b == 16 else 16 * ng * 4)
 
 
 def decode_rows(proj, rows, K, g, b):
@@ -90,7 +91,11 @@ def sb_rows(proj, rows, K, g, b):
 
 def dequant_rows(proj, rows, K, g, b):
     """Closed form of fma(scale, q, bias) in fp32: the exact product-sum in
-    float64 (exact for bf16 scale/bias and q < 64), rounded once to fp32."""
+    float64 (exact for bf16 scale/bias and q < 64), rounded once to fp32.
+    b = 16: the rows are bf16 values, row-major, each row padded to Kp."""
+    if b == 16:
+        v = np.ascontiguousarray(proj, dtype=np.uint8).reshape(-1).view("<u2").reshape(rows, ceil128(K))
+        return (v[:, :K].astype(np.uint32) << 16).view(np.float32)
     codes = decode_rows(proj, rows, K, g, b).astype(np.float64)
     sb = sb_rows(proj, rows, K, g, b)
     s = ((sb & 0xFFFF).astype(np.uint32) << 16).view(np.float32).astype(np.float64)

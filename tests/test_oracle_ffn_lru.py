@@ -47,7 +47,7 @@ def _dense_moe(x, dense, ids, w, I):
     return np.einsum("te,teh->th", M, o)
 
 
-@pytest.mark.parametrize("b_gu,b_d", [(4, 4), (3, 3), (4, 6)])
+@pytest.mark.parametrize("b_gu,b_d", [(4, 4), (3, 3), (4, 6), (16, 16), (16, 4)])
 def test_ffn_vs_dense_moe(orc, b_gu, b_d):
     E, k, H, I, g, T = 8, 2, 64, 32, 32, 4
     slots, dense = _bank(orc, E, H, I, g, b_gu, b_d)

@@ -6,6 +6,7 @@ expert; 1bit-MONSTER PR #137 keys size classes by the bytes one expert needs.
 import numpy as np
 import pytest
 
+from streamed_quantized_expert_b200 import synth
 from tests import _format_np as F
 
 
@@ -123,3 +124,23 @@ def test_slot_sections_roundtrip(orc):
     assert np.max(np.abs(gu - w_gu)) < 0.02
     pd = slot[off[1]: off[1] + H // 16 * off[3]]
     assert np.array_equal(dn, F.dequant_rows(pd, H, I, g, 6))
+
+
+def test_bf16_experts_format(orc):
+    # BF16 experts (RFC "How the prototype works", item "Cache"): a projection
+    # is its rows of bf16 values, row-major, rows padded to 128 inputs, no
+    # scale/bias words; the "quantizer" rounds to bf16 (nearest even)
+    H, I = 208, 96  # neither a multiple of 128
+    w_gu, w_d = synth.expert_weights(4, 1, H, I)
+    slot = orc.build_slot(w_gu, w_d, 32, 16, 16)
+    off, nbytes = orc.slot_layout(H, I, 32, 16, 16)
+    assert off[2] == 16 * 256 * 2 and off[3] == 16 * 128 * 2  # tile = 16 padded rows, 2 bytes per input
+    assert off[1] == 2 * I * 256 * 2 and nbytes == off[1] + H * 128 * 2
+    gu, dn = orc.dequant_slot(slot, H, I, 32, 16, 16)
+    assert np.array_equal(gu, synth.bf16_bits_to_f32(synth.to_bf16_bits(w_gu)))
+    assert np.array_equal(dn, synth.bf16_bits_to_f32(synth.to_bf16_bits(w_d)))
+    # the padding is zero and the storage rows are the gate/up interleave
+    pg = slot[:off[1]].view("<u2").reshape(2 * I, 256)
+    assert not pg[:, H:].any()
+    R = 100  # up row 100 - 96 = 4 -> storage row 16 * 0 + 8 + 4
+    assert np.array_equal(pg[12, :H], synth.to_bf16_bits(w_gu[R]))
