@@ -104,6 +104,9 @@ PREFILL = {
     "prefill": (48, 512, 10, 2048, 512, 64, lambda l: (3, 3), 1024,
                 "Flash-Next-like prefill: 48 layers x 512 experts, top-10, H 2048, I 512, SwiGLU, 3-bit g64, "
                 "1024-token chunk, passes of 64 active experts, tcgen05 grouped GEMM"),
+    "prefill_bf16": (48, 128, 8, 2048, 768, 64, lambda l: (16, 16), 1024,
+                     "Coder-30B-like prefill with unquantized BF16 experts: 48 layers x 128 experts, top-8, H 2048, "
+                     "I 768, SwiGLU, bf16 weights (16-bit slots), 1024-token chunk, tcgen05 grouped GEMM"),
     "prefill_mixed": (48, 512, 10, 2048, 512, 64, lambda l: (4, 6) if l % 4 == 0 else (4, 4), 4096,
                       "mixed size classes prefill: Flash-Next-like shapes, 4-bit gate/up, 6-bit down on layers "
                       "l % 4 == 0 (2 slot size classes), 4096-token chunk, passes of 64 active experts"),
@@ -477,7 +480,8 @@ def run_prefill(args, rank, world, local_rank, name=None, layers=0, embedded=Fal
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(whole_ms, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16 tensor-core operands (dequantised 3/4/6-bit weights), fp32 TMEM accumulate",
+        "dtype": "fp16 tensor-core operands (weights dequantised from 3/4/6-bit codes, or bf16 weights converted; "
+                 "x and h in fp16), fp32 TMEM accumulate",
         "data": "synthetic (seeded N(0,0.02) experts quantised on the GPU; N(0,1) bf16 x; log-Zipf-biased logits)",
         "config": {"workload": desc_txt, "layers": n_layers, "experts": E, "top_k": k, "hidden": H,
                    "intermediate": I, "group": g, "tokens": T,

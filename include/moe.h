@@ -74,6 +74,10 @@
  *     down    [H rows]
  *   slot_bytes = end of the down projection rounded to 256.  Dequantised weight
  *   = fmaf(scale, q, bias) in fp32 (one rounding).
+ * BF16 experts (b = 16; RFC "How the prototype works", item "Cache": BF16
+ * experts run through the grouped experts kernel): a projection is its rows
+ * of bf16 values, row-major (row r at r * Kp * 2 bytes), zero-padded to Kp,
+ * in the same storage row order, with no scale/bias words; a tile is 16 rows.
  */
 #ifndef MOE_H
 #define MOE_H
@@ -104,15 +108,19 @@ typedef enum {
 #define MOE_DEV_ERR_BAD_EXPERT 8   /* an expert id outside [0, E) */
 
 /* Shapes of one MoE layer.  Limits: 1 <= k <= E <= 1024; H and I multiples of
- * group; group in {32, 64, 128}; bits in {3, 4, 6}. */
+ * group; group in {32, 64, 128}; bits in {3, 4, 6}, or 16 for a BF16
+ * projection (unquantized; group then only checks H and I).  A layer with a
+ * 16-bit projection runs on the tensor-core grouped GEMM only: its
+ * moe_expert_ffn calls need x_sorted at every T and H, I multiples of 128
+ * (else MOE_ERR_UNSUPPORTED). */
 typedef struct {
   int32_t E;         /* experts in the layer */
   int32_t k;         /* experts per token (top-k) */
   int32_t H;         /* hidden size: input of gate/up, output of down */
   int32_t I;         /* expert intermediate size */
   int32_t group;     /* inputs per (scale, bias) group */
-  int32_t bits_gu;   /* code width of the gate/up projection */
-  int32_t bits_down; /* code width of the down projection */
+  int32_t bits_gu;   /* code width of the gate/up projection (16: bf16 values) */
+  int32_t bits_down; /* code width of the down projection (16: bf16 values) */
 } moe_layer_desc;
 
 /* Byte offsets of the two projections in a slot, their 16-row tile sizes, and
@@ -282,7 +290,8 @@ moe_status moe_dequant_slot(const void* pool, int32_t slot, const moe_layer_desc
 /* Input preparation (the RFC's one-time quantize_experts, on the GPU):
  * quantise rows of fp32 weights w [rows, K] into the slot format:
  * per group scale = bf16((max-min)/(2^b-1)), bias = bf16(min),
- * q = clamp(rint((w - bias)/scale), 0, 2^b-1) (q = 0 if scale = 0).
+ * q = clamp(rint((w - bias)/scale), 0, 2^b-1) (q = 0 if scale = 0); bits = 16
+ * writes the weights rounded to bf16 (nearest even).
  *   rows       a multiple of 16
  *   gate_up_I  0: row r of w is storage row r; I > 0: w is a gate/up matrix
  *              [2I, K] (gate rows then up rows) and its rows go to their
@@ -321,8 +330,10 @@ const char* moe_status_string(moe_status s);
  *                          kernel for T > 64): tensor-core GEMV (mma.sync)
  *   MOE_PATH_TC_PREFILL    tcgen05/TMEM grouped GEMM fed by TMA (T >= 32,
  *                          x_sorted given, H and I multiples of 128): prefill
- *                          chunks and batched decode
- * or -1 if d is invalid or T < 1.  Host only; no device work. */
+ *                          chunks and batched decode; a layer with a 16-bit
+ *                          (BF16) projection at every T
+ * or -1 if d is invalid, T < 1, or a BF16 layer has no path (no x_sorted).
+ * Host only; no device work. */
 enum { MOE_PATH_FUSED_DECODE = 0, MOE_PATH_GEMV = 1, MOE_PATH_TC_PREFILL = 2 };
 int32_t moe_ffn_kernel_path(const moe_layer_desc* d, int32_t T, int32_t has_x_sorted);
 

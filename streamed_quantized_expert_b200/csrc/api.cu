@@ -19,7 +19,7 @@ moe_status check_desc(const moe_layer_desc* d) {
   if (!d) return MOE_ERR_INVALID;
   if (d->E < 1 || d->k < 1 || d->k > d->E || d->H < 1 || d->I < 1) return MOE_ERR_INVALID;
   if (d->group != 32 && d->group != 64 && d->group != 128) return MOE_ERR_UNSUPPORTED;
-  auto bits_ok = [](int b) { return b == 3 || b == 4 || b == 6; };
+  auto bits_ok = [](int b) { return b == 3 || b == 4 || b == 6 || b == 16; };  // 16: BF16 experts
   if (!bits_ok(d->bits_gu) || !bits_ok(d->bits_down)) return MOE_ERR_UNSUPPORTED;
   if (d->H % d->group || d->I % d->group) return MOE_ERR_INVALID;
   if (d->E > 1024 || d->k > 32) return MOE_ERR_UNSUPPORTED;
@@ -73,7 +73,8 @@ WsCarve carve(const moe_layer_desc& d, int T, bool tc = true) {
   c.hb = (size_t)round_up(np * padded_k(d.I) * 2, 256);
   c.h = c.hb + (size_t)round_up(np * padded_k(d.I), 256);
   // o: per-pair outputs of the tensor-core path (T >= kTcMinTokens) and of the GEMV path for T > 64
-  c.o = ((tc && T >= kTcMinTokens) || T > kFusedMaxTokens) ? (size_t)round_up(np * d.H * 4, 256) : 0;
+  c.o = ((tc && (T >= kTcMinTokens || bf16_experts(d))) || T > kFusedMaxTokens) ? (size_t)round_up(np * d.H * 4, 256)
+                                                                                  : 0;
   const size_t ffn = c.h + c.o;
   c.total = kWsControlBytes + c.tag + (c.sort > ffn ? c.sort : ffn);
   return c;
@@ -226,6 +227,7 @@ __attribute__((visibility("hidden"))) moe_status moe_internal_expert_ffn(
   if (!aligned(pool, 256) || !aligned(x, 16) || !aligned(ws, 256)) return MOE_ERR_INVALID;
   if ((int64_t)T * d->k > (1 << 24)) return MOE_ERR_UNSUPPORTED;
   if (!ffn_decode_supported(*d)) return MOE_ERR_UNSUPPORTED;
+  if (bf16_experts(*d) && (!x_sorted || !ffn_prefill_tc_shape_ok(*d))) return MOE_ERR_UNSUPPORTED;
   const WsCarve c = carve(*d, T, x_sorted != nullptr);
   if (!ws || ws_bytes < c.total) return MOE_ERR_CAPACITY;
   FfnArgs a{};
@@ -287,7 +289,7 @@ moe_status moe_quantize_rows(const float* w, int32_t rows, int32_t K, int32_t gr
   if (rows < 0 || K < 1 || rows % 16) return MOE_ERR_INVALID;
   if (gate_up_I < 0 || (gate_up_I > 0 && (rows != 2 * gate_up_I || gate_up_I % 8))) return MOE_ERR_INVALID;
   if (group != 32 && group != 64 && group != 128) return MOE_ERR_UNSUPPORTED;
-  if (bits != 3 && bits != 4 && bits != 6) return MOE_ERR_UNSUPPORTED;
+  if (bits != 3 && bits != 4 && bits != 6 && bits != 16) return MOE_ERR_UNSUPPORTED;
   if (K % group) return MOE_ERR_INVALID;
   if (rows == 0) return MOE_OK;
   if (!w || !proj || !aligned(proj, 16)) return MOE_ERR_INVALID;

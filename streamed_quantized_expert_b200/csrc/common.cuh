@@ -30,8 +30,10 @@ struct Layout {
   int64_t slot_bytes;
 };
 
+// bits = 16: unquantized BF16 experts, rows of bf16 values (row-major, padded
+// to whole 128-input blocks with zeros), no (scale, bias) words.
 __host__ __device__ constexpr int64_t tile_bytes(int64_t K, int g, int bits) {
-  return 16 * row_bytes(K, bits) + 16 * row_groups(K, g) * 4;
+  return 16 * row_bytes(K, bits) + (bits == 16 ? 0 : 16 * row_groups(K, g) * 4);
 }
 
 inline Layout make_layout(const moe_layer_desc& d) {

@@ -153,8 +153,9 @@ moe_status decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc
   moe_status s = ns ? moe_route_shared(logits, T, d0, L, lc->table_dev, ns, lc->shared_w, b->ids, b->w, stream)
                     : moe_route(logits, T, d0, L, lc->table_dev, b->ids, b->w, stream);
   if (s != MOE_OK) return s;
-  // from 32 tokens the FFN runs on the tensor-core grouped GEMM, which reads x sorted by expert
-  uint16_t* xs = (T >= 32 && b->x_sorted) ? b->x_sorted : nullptr;
+  // from 32 tokens (BF16 experts: always) the FFN runs on the tensor-core grouped GEMM, which reads x
+  // sorted by expert
+  uint16_t* xs = ((T >= 32 || d0->bits_gu == 16 || d0->bits_down == 16) && b->x_sorted) ? b->x_sorted : nullptr;
   s = moe_sort(b->ids, xs ? x : nullptr, T, d, b->offsets, b->pairs, active, n_active, xs, b->ws, b->ws_bytes,
                stream);
   if (s != MOE_OK) return s;

@@ -535,6 +535,8 @@ constexpr size_t kDnSmemCap = 72 * 1024;
 // 2: tcgen05 grouped GEMM (prefill) -- the choice launch_ffn_decode makes
 // for a call covering every expert of the layer.
 int ffn_kernel_path(const moe_layer_desc& d, int T, bool has_x_sorted, int num_sms) {
+  // BF16 experts run on the tensor-core grouped GEMM only, at any T
+  if (bf16_experts(d)) return has_x_sorted && ffn_prefill_tc_shape_ok(d) ? 2 : -1;
   FfnArgs a{};
   a.T = T;
   a.pass_len = d.E;
@@ -550,6 +552,11 @@ int ffn_kernel_path(const moe_layer_desc& d, int T, bool has_x_sorted, int num_s
 
 cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st) {
   const Layout& L = a.L;
+  if (bf16_experts(d)) {
+    a.q_gu = L.gu;
+    a.q_d = L.d;
+    return launch_ffn_prefill_tc(a, d, num_sms, st);
+  }
   {
     FfnArgs f = a;
     f.q_gu = L.gu;

@@ -29,6 +29,10 @@
 // The operands are fp16 (11 significant bits): the token rows come sorted and
 // converted by moe_sort, h is written in fp16 by the gate/up epilogue, and the
 // weights are dequantised to fp16, so each rounding is 4x finer than bf16's.
+// BF16 experts (16-bit slots: rows of bf16 values) take the same path: TMA
+// brings 128 rows x 128 inputs with the 128-byte swizzle and the "dequant"
+// warps convert each row's quarter to fp16 on its way into TMEM (exact for
+// normal fp16 magnitudes).
 // Accumulators are double-buffered in TMEM (2 x 128 columns), so the epilogue
 // of one tile overlaps the MMAs of the next; the two A buffers take 2 x 64
 // more columns.  With A in TMEM, shared memory carries only the TMA traffic
@@ -64,7 +68,7 @@ constexpr int kPfAcols = 64;       // one A buffer: 128 inputs as fp16 pairs, 12
 static_assert(kPfAcol + kPfABufs * kPfAcols <= kPfTmemCols, "TMEM columns");
 constexpr int kPfXHalf = kPfBN * 128;   // one 64-input half of a token stage: 128 rows x 128 B
 // load stages (codes + scale/bias + token rows) that fit the shared memory
-__host__ __device__ constexpr int pf_stages(int bits) { return bits == 6 ? 4 : 5; }
+__host__ __device__ constexpr int pf_stages(int bits) { return bits == 16 ? 3 : bits == 6 ? 4 : 5; }
 
 struct PfEntry {
   int slot;    // slot of the expert (tiles skipped when not resident)
@@ -234,6 +238,24 @@ __device__ __forceinline__ void pf_dequant_quarter(const uint8_t* cs, const uint
   tmem_st16(ta + 16 * CQ, out);
 }
 
+// BF16 experts: K quarter cq of row r from the stage's two 64-input halves
+// (128 rows x 128 bytes each, 128-byte swizzle: 16-byte chunk c of row r sits
+// at chunk c ^ (r % 8)), converted to fp16 pairs (pair index = TMEM column).
+__device__ __forceinline__ void pf_bf16_quarter(int cq, const uint8_t* cs, uint32_t ta, int r) {
+  const uint8_t* row = cs + (cq >> 1) * (128 * 128) + r * 128;
+  uint32_t out[16];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int c = (cq & 1) * 4 + j;
+    const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * (c ^ (r & 7)));
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      out[4 * j + u] = (uint32_t)f32_to_f16_sat(bf16_lo(w4[u])) | ((uint32_t)f32_to_f16_sat(bf16_hi(w4[u])) << 16);
+  }
+  tmem_st16(ta + 16 * cq, out);
+}
+
 template <int B, int GPB>
 __device__ __forceinline__ void pf_dequant(int cq, const uint8_t* cs, const uint32_t* sbs, uint32_t ta, int r) {
   if (cq == 0) pf_dequant_quarter<B, GPB, 0>(cs, sbs, ta, r);
@@ -253,8 +275,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                    const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_b64,
                    const __grid_constant__ CUtensorMap tm_b128, const PfArgs a) {
   extern __shared__ uint8_t pf_smem_raw[];
-  constexpr int kCodesBytes = 2048 * B;   // 16 groups x 4 units x 8 rows x B words
-  constexpr int kSbBytes = 512 * GPB;     // 8 tiles x 16 GPB words
+  constexpr int kCodesBytes = 2048 * B;   // 16 groups x 4 units x 8 rows x B words (B = 16: 128 x 128 bf16)
+  constexpr int kSbBytes = B == 16 ? 0 : 512 * GPB;  // 8 tiles x 16 GPB words
   constexpr int kPfStages = pf_stages(B);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -372,8 +394,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[s], bytes);
-          tma_load_4d(cst + s * kCodesBytes, &tm_q, kb * 32 * B, 0, tl.mt * 8, tl.slot, &full[s]);
-          tma_load_3d(sbst + s * kSbBytes, &tm_sb, kb * 16 * GPB, tl.mt * 8, tl.slot, &full[s]);
+          if constexpr (B == 16) {  // (input, row, slot) boxes of 64 x 128 x 1
+            tma_load_3d(cst + s * kCodesBytes, &tm_q, kb * 128, tl.mt * kPfBM, tl.slot, &full[s]);
+            tma_load_3d(cst + s * kCodesBytes + 128 * 128, &tm_q, kb * 128 + 64, tl.mt * kPfBM, tl.slot, &full[s]);
+          } else {
+            tma_load_4d(cst + s * kCodesBytes, &tm_q, kb * 32 * B, 0, tl.mt * 8, tl.slot, &full[s]);
+            tma_load_3d(sbst + s * kSbBytes, &tm_sb, kb * 16 * GPB, tl.mt * 8, tl.slot, &full[s]);
+          }
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf)
             tma_load_2d(xst + (s * 2 + hf) * kPfXHalf, tmb, kb * 128 + hf * 64, tl.row0, &full[s]);
@@ -454,8 +481,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           break;
         }
         tc_fence_after();
-        pf_dequant<B, GPB>(cq, cst + s * kCodesBytes, reinterpret_cast<const uint32_t*>(sbst + s * kSbBytes),
-                           tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kPfAcol + ab * kPfAcols), r);
+        const uint32_t ta = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kPfAcol + ab * kPfAcols);
+        if constexpr (B == 16)
+          pf_bf16_quarter(cq, cst + s * kCodesBytes, ta, r);
+        else
+          pf_dequant<B, GPB>(cq, cst + s * kCodesBytes, reinterpret_cast<const uint32_t*>(sbst + s * kSbBytes), ta,
+                             r);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -581,6 +612,15 @@ bool encode_proj(CUtensorMap* q, CUtensorMap* sb, const uint8_t* proj, int64_t r
   return encode(sb, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, proj + 16 * rb, sd, ss, sbx, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+// BF16 experts: a projection's rows of bf16 values as (input, row, slot),
+// boxes of 64 inputs (128 bytes, 128-byte swizzle) x 128 rows x 1 slot.
+bool encode_proj_bf16(CUtensorMap* q, const uint8_t* proj, int64_t kp, int rows, int64_t slot_bytes, int n_slots) {
+  const cuuint64_t d[3] = {(cuuint64_t)kp, (cuuint64_t)rows, (cuuint64_t)n_slots};
+  const cuuint64_t st[2] = {(cuuint64_t)kp * 2, (cuuint64_t)slot_bytes};
+  const cuuint32_t b[3] = {64, (cuuint32_t)kPfBM, 1};
+  return encode(q, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, proj, d, st, b, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 // Token rows (fp16 [rows][cols], row-major) for the MMA's B operand: boxes of
 // 64 columns (128 bytes, 128-byte swizzle) x box_rows rows.
 bool encode_rows(CUtensorMap* m, const uint16_t* base, int64_t rows, int cols, int box_rows) {
@@ -592,7 +632,8 @@ bool encode_rows(CUtensorMap* m, const uint16_t* base, int64_t rows, int cols, i
 
 size_t pf_smem_bytes(int bits, int gpb) {
   const size_t ns = (size_t)pf_stages(bits);
-  return 1024 + ns * 2 * kPfXHalf + ns * 2048 * bits + ns * 512 * gpb + (2 * ns + 2 * kPfABufs + 5) * 8;
+  return 1024 + ns * 2 * kPfXHalf + ns * 2048 * bits + (bits == 16 ? 0 : ns * 512 * gpb) +
+         (2 * ns + 2 * kPfABufs + 5) * 8;
 }
 
 template <int B, int GPB, bool GU>
@@ -625,6 +666,7 @@ cudaError_t launch_pf(int bits, int gpb, const CUtensorMap& q, const CUtensorMap
                       const PfArgs& pa, int grid, cudaStream_t st) {
   if (bits == 3) return launch_pf_gpb<3, GU>(gpb, q, sb, bm, pa, grid, st);
   if (bits == 4) return launch_pf_gpb<4, GU>(gpb, q, sb, bm, pa, grid, st);
+  if (bits == 16) return launch_pf_t<16, 1, GU>(q, sb, bm, pa, grid, st);
   return launch_pf_gpb<6, GU>(gpb, q, sb, bm, pa, grid, st);
 }
 
@@ -647,10 +689,16 @@ cudaError_t launch_ffn_prefill_tc(const FfnArgs& a, const moe_layer_desc& d, int
   const int gpb = 128 / d.group;
   const int64_t np = (int64_t)a.T * d.k;
   CUtensorMap q_gu, sb_gu, q_d, sb_d, xm[3], hm[3];
-  if (!encode_proj(&q_gu, &sb_gu, a.pool + L.gu, L.rb_gu, L.tile_gu, L.ng_gu, 2 * d.I, d.bits_gu, gpb, L.slot_bytes,
-                   a.n_slots) ||
-      !encode_proj(&q_d, &sb_d, a.pool + L.d, L.rb_d, L.tile_d, L.ng_d, d.H, d.bits_down, gpb, L.slot_bytes,
-                   a.n_slots) ||
+  auto proj_maps = [&](CUtensorMap* q, CUtensorMap* sb, int64_t off, int64_t rb, int64_t tile, int ng, int rows,
+                       int bits, int64_t K) {
+    if (bits == 16) {
+      *sb = CUtensorMap{};  // no scale/bias words
+      return encode_proj_bf16(q, a.pool + off, padded_k(K), rows, L.slot_bytes, a.n_slots);
+    }
+    return encode_proj(q, sb, a.pool + off, rb, tile, ng, rows, bits, gpb, L.slot_bytes, a.n_slots);
+  };
+  if (!proj_maps(&q_gu, &sb_gu, L.gu, L.rb_gu, L.tile_gu, L.ng_gu, 2 * d.I, d.bits_gu, d.H) ||
+      !proj_maps(&q_d, &sb_d, L.d, L.rb_d, L.tile_d, L.ng_d, d.H, d.bits_down, d.I) ||
       !encode_rows(&xm[0], a.x_sorted, np, d.H, 32) || !encode_rows(&xm[1], a.x_sorted, np, d.H, 64) ||
       !encode_rows(&xm[2], a.x_sorted, np, d.H, 128) || !encode_rows(&hm[0], a.h, np, d.I, 32) ||
       !encode_rows(&hm[1], a.h, np, d.I, 64) || !encode_rows(&hm[2], a.h, np, d.I, 128))

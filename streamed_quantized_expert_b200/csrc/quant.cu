@@ -1,6 +1,7 @@
 // Quantization into the slot row format (input preparation: the RFC's
-// one-time quantize_experts, which writes experts in MLX's affine format) and
-// the test-only dequantisation of a slot through the FFN's code unpackers.
+// one-time quantize_experts, which writes experts in MLX's affine format; and
+// the rounding of BF16 experts to their bf16 rows) and the test-only
+// dequantisation of a slot through the FFN's code unpackers.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -107,6 +108,33 @@ __global__ void __launch_bounds__(256) quantize_kernel(const float* __restrict__
   }
 }
 
+// BF16 experts: the rows rounded to bf16 (nearest even), row-major in storage
+// row order, each row padded with zeros to whole 128-input blocks.  One thread
+// per (row, pair of inputs).
+__global__ void __launch_bounds__(256) bf16_rows_kernel(const float* __restrict__ w, int rows, int K, int gu_I,
+                                                        uint8_t* __restrict__ q) {
+  const int Kp = (int)padded_k(K);
+  const int64_t task = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (task >= (int64_t)rows * (Kp / 2)) return;
+  const int r = (int)(task / (Kp / 2)), k = 2 * (int)(task % (Kp / 2));
+  const float v0 = k < K ? w[(int64_t)r * K + k] : 0.0f, v1 = k + 1 < K ? w[(int64_t)r * K + k + 1] : 0.0f;
+  const int srow = gu_I > 0 ? gate_up_row(r, gu_I) : r;
+  reinterpret_cast<uint32_t*>(q + (int64_t)srow * Kp * 2)[k / 2] =
+      (uint32_t)f32_to_bf16_rne(v0) | ((uint32_t)f32_to_bf16_rne(v1) << 16);
+}
+
+// BF16 experts (test): the stored values, logical row order.
+__global__ void bf16_dequant_kernel(const uint8_t* __restrict__ qbase, int rows, int K, int gu_I,
+                                    float* __restrict__ out32, uint16_t* __restrict__ out16) {
+  const int64_t task = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (task >= (int64_t)rows * K) return;
+  const int lr = (int)(task / K), k = (int)(task % K);
+  const int r = gu_I > 0 ? gate_up_row(lr, gu_I) : lr;
+  const uint16_t v = reinterpret_cast<const uint16_t*>(qbase + (int64_t)r * padded_k(K) * 2)[k];
+  if (out32) out32[task] = __uint_as_float((uint32_t)v << 16);
+  if (out16) out16[task] = v;
+}
+
 // Dequantise rows of one projection: one thread per (storage row, unit),
 // through the same unpack_unit<B> the FFN kernels use.  out[r][k] = fmaf(s,
 // q, b), r the logical row (gu_I > 0: gate/up row order).
@@ -157,7 +185,11 @@ static void dq_dispatch(int b, const uint8_t* q, int rows, int K, int g, int gu_
                         cudaStream_t st) {
   if (b == 3) launch_dq<3>(q, rows, K, g, gu_I, o32, o16, st);
   else if (b == 4) launch_dq<4>(q, rows, K, g, gu_I, o32, o16, st);
-  else launch_dq<6>(q, rows, K, g, gu_I, o32, o16, st);
+  else if (b == 6) launch_dq<6>(q, rows, K, g, gu_I, o32, o16, st);
+  else {
+    const int64_t n = (int64_t)rows * K;
+    bf16_dequant_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(q, rows, K, gu_I, o32, o16);
+  }
 }
 
 cudaError_t launch_dequant_slot(const uint8_t* slot, const moe_layer_desc& d, const Layout& L, float* out32,
@@ -170,6 +202,12 @@ cudaError_t launch_dequant_slot(const uint8_t* slot, const moe_layer_desc& d, co
 }
 
 cudaError_t launch_quantize(const float* w, int rows, int K, int g, int b, int gu_I, uint8_t* q, cudaStream_t st) {
+  if (b == 16) {
+    const int64_t n = (int64_t)rows * (padded_k(K) / 2);
+    if (n == 0) return cudaSuccess;
+    bf16_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(w, rows, K, gu_I, q);
+    return cudaGetLastError();
+  }
   const int64_t tasks = (int64_t)rows * (padded_k(K) / 128);
   if (tasks == 0) return cudaSuccess;
   quantize_kernel<<<(unsigned)((tasks + 7) / 8), 256, 0, st>>>(w, rows, K, g, b, gu_I, q);

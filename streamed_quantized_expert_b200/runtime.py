@@ -121,7 +121,8 @@ class Streamer:
         self.launches = 0          # libmoe kernel launches issued (for reporting)
         # native per-layer driver state
         self.installed.record(self.side)  # materialise the event
-        if max_tokens >= 32:  # batched decode sorts x for the tensor-core grouped GEMM
+        bf16 = any(l.desc.bits_gu == 16 or l.desc.bits_down == 16 for l in layers)
+        if max_tokens >= 32 or bf16:  # the tensor-core grouped GEMM (batched decode, BF16 experts) reads sorted x
             self.x_sorted = torch.empty((max_tokens * self.kw, self.H), dtype=torch.uint16, device=self.device)
         self._bufs = ops.StepBuffers(self.ids.data_ptr(), self.w.data_ptr(), self.offsets.data_ptr(),
                                      self.pairs.data_ptr(), self.meta.data_ptr(), self.meta_pin.data_ptr(),
@@ -236,9 +237,10 @@ class Streamer:
             ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             ev[0].record(self.stream)
         self.launches += 2 if T <= 64 else 3
+        tc = T >= 32 or d.bits_gu == 16 or d.bits_down == 16
         ops.moe_expert_ffn(x, T, d, self.pool_of(layer), self.n_slots_of(layer), self.table_dev[layer], self.ids,
                            self.w, self.offsets, self.pairs, self._active(), self._n_active(),
-                           self.x_sorted if T >= 32 else None, pass_begin, pass_len, y, self.ws, self.ws_bytes,
+                           self.x_sorted if tc else None, pass_begin, pass_len, y, self.ws, self.ws_bytes,
                            self.dev_err, self.stream)
         if ev is not None:
             ev[1].record(self.stream)
@@ -277,7 +279,8 @@ class Streamer:
         """Same as decode_layer, one ABI call at a time from Python."""
         y = self.y[:T] if y is None else y
         s = self.stream
-        self.route_sort(layer, x, logits, T, L)
+        d0 = self.layers[layer].desc
+        self.route_sort(layer, x, logits, T, L, want_sorted_x=T >= 32 or d0.bits_gu == 16 or d0.bits_down == 16)
         if not self.fully_resident(layer):
             d = self.layers[layer].desc
             ops.moe_slot_lookup(self.table_dev[layer], self._active(), self._n_active(), 0, self.Ew,
@@ -299,7 +302,8 @@ class Streamer:
         """One prefill chunk: passes of <= 64 active experts; returns y."""
         y = self.y[:T] if y is None else y
         s = self.stream
-        self.route_sort(layer, x, logits, T, 0.0, want_sorted_x=T >= 32)
+        d0 = self.layers[layer].desc
+        self.route_sort(layer, x, logits, T, 0.0, want_sorted_x=T >= 32 or d0.bits_gu == 16 or d0.bits_down == 16)
         with torch.cuda.stream(s):
             y.zero_()
             self.meta_pin.copy_(self.meta, non_blocking=True)

@@ -42,7 +42,7 @@ def test_exp_bit_exact_on_every_float_in_domain(orc):
 
 
 @pytest.mark.parametrize("rows,K,g,b", [(16, 64, 32, 4), (48, 2048, 64, 3), (16, 512, 64, 6), (16, 768, 128, 4),
-                                        (16, 32, 32, 3), (64, 2048, 64, 4)])
+                                        (16, 32, 32, 3), (64, 2048, 64, 4), (32, 768, 64, 16), (16, 96, 32, 16)])
 def test_quantize_bit_exact(orc, rows, K, g, b):
     w = (synth.rng(rows, K, g, b).standard_normal((rows, K), dtype=np.float32) * np.float32(0.02))
     w[0, :g] = np.float32(0.5)  # constant group
@@ -54,9 +54,10 @@ def test_quantize_bit_exact(orc, rows, K, g, b):
     assert np.array_equal(proj.cpu().numpy(), ref)
 
 
-def test_quantize_gate_up_order_bit_exact(orc):
+@pytest.mark.parametrize("bg,bd", [(3, 4), (16, 16), (16, 6)])
+def test_quantize_gate_up_order_bit_exact(orc, bg, bd):
     # a whole expert through moe_quantize_rows (gate/up row order) vs the oracle's slot builder
-    H, I, g, bg, bd = 256, 64, 64, 3, 4
+    H, I, g = 256, 64, 64
     w_gu, w_d = synth.expert_weights(4, 0, H, I)
     ref = orc.build_slot(w_gu, w_d, g, bg, bd)
     d = ops.desc(8, 2, H, I, g, bg, bd)
@@ -70,7 +71,8 @@ def test_quantize_gate_up_order_bit_exact(orc):
 
 
 @pytest.mark.parametrize("H,I,g,bg,bd", [(64, 32, 32, 4, 4), (2048, 512, 64, 3, 3), (256, 128, 64, 4, 6),
-                                         (2048, 768, 64, 4, 4), (384, 256, 128, 6, 3)])
+                                         (2048, 768, 64, 4, 4), (384, 256, 128, 6, 3), (256, 96, 32, 16, 16),
+                                         (512, 256, 64, 16, 4)])
 def test_dequant_slot_bit_exact(orc, H, I, g, bg, bd):
     bank = oracle_bank(orc, 3, H, I, g, bg, bd, seed=H + I)
     d = ops.desc(8, 2, H, I, g, bg, bd)
