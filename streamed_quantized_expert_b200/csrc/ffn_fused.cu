@@ -67,7 +67,8 @@ namespace moe {
 constexpr int kFuThreads = (kFuConsumers + 1) * 32;
 constexpr int kFuPairs = kFuConsumers / 2;              // gate/up warp pairs
 constexpr int kFuRedFloats = kFuConsumers * 32 * 4;     // [warp][lane][4]: pair partials, then y partials
-constexpr int kFuScratchPerTok = 128 * 2 + 8 * 8;       // per warp and token: an h block (bf16) + group sums
+constexpr int kFuScratchRowWords = 64 + 4;              // one token's 128-column h block, fragment order, padded
+constexpr int kFuScratchPerTok = kFuScratchRowWords * 4 + 8 * 8;  // bytes per warp and token: h block + group sums
 static_assert(8 <= (int)kWsControlBytes, "control block size");
 constexpr unsigned long long kEpochOne = 1ull << 32;
 // per-pass tables in shared memory: active ids, slots, routed ids, routed
@@ -91,6 +92,30 @@ __device__ __forceinline__ void st_u64(uint64_t* p, uint64_t v) {
 // value and tag always come from the same store.
 __device__ __forceinline__ void ld_volatile_2w(const uint64_t* p, uint64_t& w0, uint64_t& w1) {
   asm volatile("ld.volatile.global.v2.u64 {%0, %1}, [%2];" : "=l"(w0), "=l"(w1) : "l"(p) : "memory");
+}
+
+// MMA fragment order of a bf16 row vector in shared memory: the pair
+// (k, k + 1), k even, of 128-input block kb is 32-bit word
+// ((kb * 4 + t4) * 8 + s) * 2 + half, s = k's 16-input step in the block,
+// half = which 8 of the step, t4 = the pair within those 8.  So the 16 words
+// lane t4 takes as B fragments for a block are contiguous (four 16-byte
+// loads instead of sixteen 4-byte ones: the shared-memory instruction queue,
+// not the tensor pipe, bounds this loop).  Rows are Kp + 8 elements apart, so
+// consecutive rows start on different banks.
+__device__ __forceinline__ int frag_word(int k) {
+  const int kb = k >> 7, kk = k & 127;
+  return ((kb * 4 + ((kk >> 1) & 3)) * 8 + (kk >> 4)) * 2 + ((kk >> 3) & 1);
+}
+__host__ __device__ constexpr int frag_rows_bytes(int rows, int Kp) { return rows * (Kp + 8) * 2; }
+__device__ __forceinline__ void load_frag(const uint4* row, int kb, int t4, uint32_t (&bf)[8][2]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 v = row ? row[(kb * 4 + t4) * 4 + j] : make_uint4(0u, 0u, 0u, 0u);
+    bf[2 * j][0] = v.x;
+    bf[2 * j][1] = v.y;
+    bf[2 * j + 1][0] = v.z;
+    bf[2 * j + 1][1] = v.w;
+  }
 }
 
 // Named barrier 2 over all threads of the CTA: the producer warp arrives once
@@ -328,12 +353,14 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
   }
   {
     // x' = x 2^-a (exact: a power of two; a by input position within its
-    // 128-block) -> shared memory, with the per-(group, token) sums
-    // sum x and 128 sum x' that the group epilogues apply
+    // 128-block) -> shared memory in MMA fragment order (frag_word), with
+    // the per-(group, token) sums sum x and 128 sum x' that the group
+    // epilogues apply; columns past H, tokens past T and groups past H are 0
     const int nx = a.T * a.H / 8;  // 16-byte words of x (H a multiple of 32)
     const int wpg = a.g / 8;       // words per group: consecutive lanes, aligned
-    uint4* xd = reinterpret_cast<uint4*>(xh);
-    float* xsum = reinterpret_cast<float*>(xh + (size_t)a.T * a.H * 2);
+    const int Kp = a.nblk_gu * 128, rw = (Kp + 8) / 2;  // padded row, row stride in words
+    uint32_t* xw = reinterpret_cast<uint32_t*>(xh);
+    float* xq = reinterpret_cast<float*>(xh + frag_rows_bytes(a.T, Kp));
     for (int base = warp * 32; base < nx; base += kFuConsumers * 32) {
       const int idx = base + lane;
       const bool act = idx < nx;
@@ -353,14 +380,21 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
         so += __shfl_xor_sync(0xffffffffu, so, o);
       }
       if (act) {
-        xd[idx] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        uint32_t* dst = xw + t * rw + frag_word(k);  // the four pairs are four t4 lanes apart
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dst[16 * u] = w4[u];
         if ((idx % wpg) == 0) {
           const int G = k / a.g;
-          xsum[(G * a.T + t) * 2] = sx;
-          xsum[(G * a.T + t) * 2 + 1] = 128.0f * so;
+          xq[(G * 8 + t) * 2] = sx;
+          xq[(G * 8 + t) * 2 + 1] = 128.0f * so;
         }
       }
     }
+    const int npad = (Kp - a.H) / 2;  // pair words past H, per row
+    for (int i = tid; i < a.T * npad; i += kFuConsumers * 32)
+      xw[(i / npad) * rw + frag_word(a.H + 2 * (i % npad))] = 0u;
+    for (int i = tid; i < (Kp / a.g) * 8; i += kFuConsumers * 32)
+      if (i % 8 >= a.T || i / 8 >= a.H / a.g) xq[2 * i] = xq[2 * i + 1] = 0.f;
   }
   tables_sync();  // the producer's pass tables
   const int n_act = s_nact, i0 = s_i0, i1 = s_i1;
@@ -385,11 +419,11 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
   // ---------------- gate/up + SwiGLU -> h: one item per warp pair ----------------
   {
     const int m = warp >> 1, hw = warp & 1;  // pair, half of K
-    const uint16_t* xrow = g8 < a.T ? reinterpret_cast<const uint16_t*>(xh) + g8 * a.H : nullptr;
-    const float* xsum = reinterpret_cast<const float*>(xh + (size_t)a.T * a.H * 2);
+    const int Kp = a.nblk_gu * 128;
+    const uint4* xrow = g8 < a.T ? reinterpret_cast<const uint4*>(xh) + g8 * ((Kp + 8) / 8) : nullptr;
+    const float4* xq4 = reinterpret_cast<const float4*>(xh + frag_rows_bytes(a.T, Kp));
     const int GRP = 8 * (int)a.rb_gu;
     const int uoff = thread_unit_off<BG>(t4, g8);
-    const int n0 = 2 * t4 < a.T ? 2 * t4 : 0, n1 = 2 * t4 + 1 < a.T ? 2 * t4 + 1 : 0;  // C fragment columns
     const int my_items = i1 - i0;
     int pass = 0;
     for (int q = m; q < my_items; q += kFuPairs, ++pass) {
@@ -409,19 +443,14 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
         for (int kb = hw; kb < a.nblk_gu; kb += 2) {
           uint32_t bf[8][2];
           float xs[8 / GS][2], xo[8 / GS][2];
-          const uint16_t* row = xrow ? xrow + kb * 128 + 2 * t4 : nullptr;
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            bf[u][0] = row ? ld_pair(row + 16 * u) : 0u;
-            bf[u][1] = row ? ld_pair(row + 16 * u + 8) : 0u;
-          }
+          load_frag(xrow, kb, t4, bf);
 #pragma unroll
           for (int G = 0; G < 8 / GS; ++G) {
-            const int gi = kb * (8 / GS) + G;
-            xs[G][0] = xsum[(gi * a.T + n0) * 2];
-            xo[G][0] = xsum[(gi * a.T + n0) * 2 + 1];
-            xs[G][1] = xsum[(gi * a.T + n1) * 2];
-            xo[G][1] = xsum[(gi * a.T + n1) * 2 + 1];
+            const float4 q = xq4[(kb * (8 / GS) + G) * 4 + t4];  // tokens 2 t4, 2 t4 + 1
+            xs[G][0] = q.x;
+            xo[G][0] = q.y;
+            xs[G][1] = q.z;
+            xo[G][1] = q.w;
           }
           block_mma<BG, GS>(st, st + GRP, sbs + g8, sbs + 8 + g8, kb, uoff, bf, xs, xo, acc);
         }
@@ -466,8 +495,8 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
     const int uoff = thread_unit_off<BD>(t4, g8);
     const int nb = a.nblk_d;
     constexpr int GPB = 8 / GS;  // groups per 128-block
-    uint16_t* hsc = reinterpret_cast<uint16_t*>(xh + a.h_stage_off + (size_t)warp * a.T * kFuScratchPerTok);
-    float2* gsum = reinterpret_cast<float2*>(hsc + a.T * 128);  // [token][group of the block]
+    uint32_t* hsc = reinterpret_cast<uint32_t*>(xh + a.h_stage_off + (size_t)warp * a.T * kFuScratchPerTok);
+    float2* gsum = reinterpret_cast<float2*>(hsc + a.T * kFuScratchRowWords);  // [token][group of the block]
     float yacc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int task = warp; task < n_act * nb; task += kFuConsumers) {
       const int i = task / nb, kb = task % nb;
@@ -502,7 +531,9 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
           const uint32_t h1 = c0 + 1 < a.I ? (uint32_t)(w[1] & 0xFFFFu) : 0u;
           const uint32_t h2 = c0 + 2 < a.I ? (uint32_t)(w[2] & 0xFFFFu) : 0u;
           const uint32_t h3 = c0 + 3 < a.I ? (uint32_t)(w[3] & 0xFFFFu) : 0u;
-          *reinterpret_cast<uint2*>(hsc + t * 128 + 4 * lane) = make_uint2(h0 | (h1 << 16), h2 | (h3 << 16));
+          uint32_t* dst = hsc + t * kFuScratchRowWords + frag_word(4 * lane);  // pairs one t4 apart
+          dst[0] = h0 | (h1 << 16);
+          dst[16] = h2 | (h3 << 16);
           // per-group sums: the four columns share a pair slot, so one scale
           const int kk = (4 * lane) & 127;
           const bool eighth = PairShift<BD>::a(2 * (kk >> 4) + ((kk & 15) >> 3)) == 3;
@@ -529,12 +560,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
         const int p0 = s_tok[i * kDenseMaxTokens + 2 * t4], p1 = s_tok[i * kDenseMaxTokens + 2 * t4 + 1];
         uint32_t bf[8][2];
         float xs1[GPB][2], xo1[GPB][2];
-        const uint16_t* row = pb < 0 ? nullptr : hsc + g8 * 128 + 2 * t4;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          bf[u][0] = row ? ld_pair(row + 16 * u) : 0u;
-          bf[u][1] = row ? ld_pair(row + 16 * u + 8) : 0u;
-        }
+        load_frag(pb < 0 ? nullptr : reinterpret_cast<const uint4*>(hsc + g8 * kFuScratchRowWords), 0, t4, bf);
 #pragma unroll
         for (int G = 0; G < GPB; ++G) {
           const float2 v0 = p0 < 0 ? make_float2(0.f, 0.f) : gsum[(2 * t4) * GPB + G];
@@ -634,8 +660,10 @@ bool ffn_fused_plan(FfnArgs& a, const moe_layer_desc& d, int num_sms, size_t& sm
   if (max_pass < 1) max_pass = 1;
   a.gu_stage_bytes = (int)round_up(a.L.tile_gu, 128);
   a.d_stage_bytes = (int)round_up(a.L.tile_d, 128);
-  // x' and its per-(group, token) sums; then each warp's h block scratch
-  const size_t xb = (size_t)round_up((int64_t)a.T * d.H * 2 + (int64_t)(d.H / d.group) * a.T * 8, 128);
+  // x' (fragment order) and its per-(group, token) sums, tokens padded to 8;
+  // then each warp's h block scratch
+  const int Kx = (int)padded_k(d.H);
+  const size_t xb = (size_t)round_up((int64_t)frag_rows_bytes(a.T, Kx) + (int64_t)(Kx / d.group) * 8 * 8, 128);
   a.h_stage_off = (int)xb;
   a.xh_stage_bytes = (int)round_up((int64_t)xb + (int64_t)kFuConsumers * a.T * kFuScratchPerTok, 128);
   // the most gate/up items a CTA can get: a CTA without a down tile takes the
