@@ -30,6 +30,9 @@
 // stages it in the warp's shared scratch with its per-group sums, and runs
 // the CTA's 16-row tile over that block.  The warps' partial sums of y meet
 // once, in a fixed order, at the end (deterministic).
+// With one token and every entry's down tile resident at once, a warp's
+// tasks (at most three) read their h blocks together -- one round of global
+// reads instead of one per task -- then compute back to back.
 //
 // Stage rings (when a CTA's items or entries outnumber its stages): several
 // warps consume the uses of one stage, so a consumer could reach use u of a
@@ -68,7 +71,8 @@ constexpr int kFuThreads = (kFuConsumers + 1) * 32;
 constexpr int kFuPairs = kFuConsumers / 2;              // gate/up warp pairs
 constexpr int kFuRedFloats = kFuConsumers * 32 * 4;     // [warp][lane][4]: pair partials, then y partials
 constexpr int kFuScratchRowWords = 64 + 4;              // one token's 128-column h block, fragment order, padded
-constexpr int kFuScratchPerTok = kFuScratchRowWords * 4 + 8 * 8;  // bytes per warp and token: h block + group sums
+constexpr int kFuScratchPerTok = kFuScratchRowWords * 4 + 8 * 8;  // bytes per warp and row: h block + group sums
+constexpr int kFuFastTasks = 3;  // one-token down: tasks per warp read together
 static_assert(8 <= (int)kWsControlBytes, "control block size");
 constexpr unsigned long long kEpochOne = 1ull << 32;
 // per-pass tables in shared memory: active ids, slots, routed ids, routed
@@ -495,10 +499,121 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
     const int uoff = thread_unit_off<BD>(t4, g8);
     const int nb = a.nblk_d;
     constexpr int GPB = 8 / GS;  // groups per 128-block
-    uint32_t* hsc = reinterpret_cast<uint32_t*>(xh + a.h_stage_off + (size_t)warp * a.T * kFuScratchPerTok);
-    float2* gsum = reinterpret_cast<float2*>(hsc + a.T * kFuScratchRowWords);  // [token][group of the block]
+    const int srows = a.T > kFuFastTasks ? a.T : kFuFastTasks;  // scratch rows per warp
+    uint32_t* hsc = reinterpret_cast<uint32_t*>(xh + a.h_stage_off + (size_t)warp * srows * kFuScratchPerTok);
+    float2* gsum = reinterpret_cast<float2*>(hsc + srows * kFuScratchRowWords);  // [row][group of the block]
     float yacc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int task = warp; task < n_act * nb; task += kFuConsumers) {
+    const int ntask = n_act * nb;
+    // One token whose down tiles are all resident at once (every entry has its
+    // own stage, each used once): a warp's tasks (at most kFuFastTasks) read
+    // their h blocks together -- one round of global reads instead of one
+    // per task -- then wait for their tiles and compute back to back.
+    const bool fast = a.T == 1 && n_act <= NSD && ntask <= kFuConsumers * kFuFastTasks;
+    if (fast && !timed_out) {
+      uint64_t fw[kFuFastTasks][4];
+      int fi[kFuFastTasks], fkb[kFuFastTasks];
+      bool fv[kFuFastTasks];
+#pragma unroll
+      for (int j = 0; j < kFuFastTasks; ++j) {
+        const int task = warp + kFuConsumers * j;
+        fi[j] = task < ntask ? task / nb : 0;
+        fkb[j] = task < ntask ? task % nb : 0;
+        const int p = task < ntask ? s_tok[fi[j] * kDenseMaxTokens] : -1;
+        fv[j] = task < ntask && slot_ok(a, s_slot[fi[j]]) && p >= 0;
+        fw[j][0] = fw[j][1] = fw[j][2] = fw[j][3] = 0ull;
+        if (fv[j]) {
+          const uint64_t* src = htag + (int64_t)p * Ip + fkb[j] * 128 + 4 * lane;
+          ld_volatile_2w(src, fw[j][0], fw[j][1]);
+          ld_volatile_2w(src + 2, fw[j][2], fw[j][3]);
+        }
+      }
+      const long long t0 = clock64();
+      for (;;) {
+        bool fresh[kFuFastTasks];
+        bool all = true;
+#pragma unroll
+        for (int j = 0; j < kFuFastTasks; ++j) {
+          fresh[j] = true;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            fresh[j] &= !fv[j] || fkb[j] * 128 + 4 * lane + q >= a.I || (unsigned)(fw[j][q] >> 32) == tag;
+          all &= fresh[j];
+        }
+        if (__all_sync(0xffffffffu, all)) break;
+        if (clock64() - t0 > a.wait_limit) {
+          timed_out = true;
+          break;
+        }
+        __nanosleep(32);
+#pragma unroll
+        for (int j = 0; j < kFuFastTasks; ++j)
+          if (!fresh[j]) {
+            const uint64_t* src = htag + (int64_t)s_tok[fi[j] * kDenseMaxTokens] * Ip + fkb[j] * 128 + 4 * lane;
+            ld_volatile_2w(src, fw[j][0], fw[j][1]);
+            ld_volatile_2w(src + 2, fw[j][2], fw[j][3]);
+          }
+      }
+      // stage each task's block (its own scratch row) and its per-group sums
+      const int kk = (4 * lane) & 127;
+      const bool eighth = PairShift<BD>::a(2 * (kk >> 4) + ((kk & 15) >> 3)) == 3;
+      const int lpg = a.g / 4;  // lanes per group (8, 16 or 32)
+#pragma unroll
+      for (int j = 0; j < kFuFastTasks; ++j) {
+        if (!fv[j]) continue;  // warp-uniform
+        const int c0 = fkb[j] * 128 + 4 * lane;
+        const uint32_t h0 = c0 < a.I ? (uint32_t)(fw[j][0] & 0xFFFFu) : 0u;
+        const uint32_t h1 = c0 + 1 < a.I ? (uint32_t)(fw[j][1] & 0xFFFFu) : 0u;
+        const uint32_t h2 = c0 + 2 < a.I ? (uint32_t)(fw[j][2] & 0xFFFFu) : 0u;
+        const uint32_t h3 = c0 + 3 < a.I ? (uint32_t)(fw[j][3] & 0xFFFFu) : 0u;
+        uint32_t* dst = hsc + j * kFuScratchRowWords + frag_word(4 * lane);  // pairs one t4 apart
+        dst[0] = h0 | (h1 << 16);
+        dst[16] = h2 | (h3 << 16);
+        const float v = __uint_as_float(h0 << 16) + __uint_as_float(h1 << 16) + __uint_as_float(h2 << 16) +
+                        __uint_as_float(h3 << 16);
+        float sx = eighth ? 8.0f * v : v, so = 128.0f * v;
+        for (int o = 1; o < lpg; o <<= 1) {
+          sx += __shfl_xor_sync(0xffffffffu, sx, o);
+          so += __shfl_xor_sync(0xffffffffu, so, o);
+        }
+        if ((lane % lpg) == 0) gsum[j * GPB + lane / lpg] = make_float2(sx, so);
+      }
+      __syncwarp();
+      // the tasks' down tiles: entry i on stage i, its first and only use
+#pragma unroll
+      for (int j = 0; j < kFuFastTasks; ++j) {
+        if (!fv[j] || timed_out) continue;
+        if (!issued(NSG + fi[j], 0) || !mbar_wait_bounded(&dfull[fi[j]], 0u, a.wait_limit)) timed_out = true;
+      }
+      if (timed_out) *abort_flag = 1;
+#pragma unroll
+      for (int j = 0; j < kFuFastTasks; ++j) {
+        if (!fv[j] || timed_out) continue;
+        const int i = fi[j];
+        const uint8_t* st = dst_ + (size_t)i * SBD;
+        const uint32_t* sbs = reinterpret_cast<const uint32_t*>(st + 2 * GRP);
+        const int pb = s_tok[i * kDenseMaxTokens + g8];
+        const int p0 = s_tok[i * kDenseMaxTokens + 2 * t4], p1 = s_tok[i * kDenseMaxTokens + 2 * t4 + 1];
+        uint32_t bf[8][2];
+        float xs1[GPB][2], xo1[GPB][2];
+        load_frag(pb < 0 ? nullptr : reinterpret_cast<const uint4*>(hsc + j * kFuScratchRowWords), 0, t4, bf);
+#pragma unroll
+        for (int G = 0; G < GPB; ++G) {
+          const float2 v0 = p0 < 0 ? make_float2(0.f, 0.f) : gsum[j * GPB + G];
+          xs1[G][0] = v0.x;
+          xo1[G][0] = v0.y;
+          xs1[G][1] = 0.f;  // token 1 does not exist
+          xo1[G][1] = 0.f;
+        }
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        block_mma<BD, GS>(st, st + GRP, sbs + g8, sbs + 8 + g8, fkb[j], uoff, bf, xs1, xo1, acc);
+        const float w0 = p0 >= 0 ? s_w[p0] : 0.f, w1 = p1 >= 0 ? s_w[p1] : 0.f;
+        yacc[0] += w0 * acc[0];
+        yacc[1] += w1 * acc[1];
+        yacc[2] += w0 * acc[2];
+        yacc[3] += w1 * acc[3];
+      }
+    }
+    for (int task = fast ? ntask : warp; task < ntask; task += kFuConsumers) {
       const int i = task / nb, kb = task % nb;
       const int s = i % NSD;
       const bool ok = slot_ok(a, s_slot[i]);
@@ -665,7 +780,8 @@ bool ffn_fused_plan(FfnArgs& a, const moe_layer_desc& d, int num_sms, size_t& sm
   const int Kx = (int)padded_k(d.H);
   const size_t xb = (size_t)round_up((int64_t)frag_rows_bytes(a.T, Kx) + (int64_t)(Kx / d.group) * 8 * 8, 128);
   a.h_stage_off = (int)xb;
-  a.xh_stage_bytes = (int)round_up((int64_t)xb + (int64_t)kFuConsumers * a.T * kFuScratchPerTok, 128);
+  const int srows = a.T > kFuFastTasks ? a.T : kFuFastTasks;  // each warp's scratch rows
+  a.xh_stage_bytes = (int)round_up((int64_t)xb + (int64_t)kFuConsumers * srows * kFuScratchPerTok, 128);
   // the most gate/up items a CTA can get: a CTA without a down tile takes the
   // whole quota of (gate/up + down bytes) / grid, or the items / (CTAs
   // without a down tile) where a down tile is more than the quota (which case
