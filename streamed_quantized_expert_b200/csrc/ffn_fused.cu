@@ -16,6 +16,8 @@
 // and its 32 lanes issue, in parallel, one bulk copy per gate/up item and one
 // per expert for the down tile, so the down weights stream in while gate/up
 // computes.
+// The CTA's arrival on the launch's control word is taken by a consumer
+// lane, off the producer's path to its first copy.
 //
 // Gate/up: warp pair m takes the CTA's items m, m + 8, ...; each warp of the
 // pair runs half of K, one adds the other's partial sums (a pair barrier), so
@@ -227,12 +229,6 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
   if (warp == kFuConsumers) {
     // ---------------- producer: pass tables, then the CTA's bulk copies ----------------
     const int na_raw = *a.n_active;
-    unsigned long long cw = 0ull;  // control word before this CTA's arrival
-    if (lane == 0) {
-      unsigned long long* ctr = reinterpret_cast<unsigned long long*>(a.ctl);
-      cw = atomicAdd(ctr, 1ull);
-      if ((unsigned)cw == gridDim.x - 1u) atomicAdd(ctr, kEpochOne - gridDim.x);  // the next launch's epoch
-    }
     int act_v[2];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -255,11 +251,6 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
     int n_act = na_raw - a.pass_begin;
     if (n_act > cap) n_act = cap;
     if (n_act < 0) n_act = 0;
-    cw = __shfl_sync(0xffffffffu, cw, 0);
-    if ((unsigned)cw >= gridDim.x) {  // not a count this launch can complete: no work, no valid tag
-      n_act = 0;
-      if (lane == 0 && a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
-    }
     __syncwarp();
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -277,8 +268,6 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
       s_nact = n_act;
       s_i0 = i0;
       s_i1 = i1;
-      const unsigned t = (unsigned)(cw >> 32) + 1u;
-      s_tag = fmix32(t == 0u ? 1u : t);  // fmix32 maps only 0 to 0
     }
     __syncwarp();
     tables_arrive();
@@ -351,6 +340,14 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
   }
 
   // ---------------- consumers ----------------
+  // this CTA's arrival on the launch's control word (its result is needed only
+  // when the tag is published, before the table barrier)
+  unsigned long long cw = 0ull;
+  if (warp == 0 && lane == 0) {
+    unsigned long long* ctr = reinterpret_cast<unsigned long long*>(a.ctl);
+    cw = atomicAdd(ctr, 1ull);
+    if ((unsigned)cw == gridDim.x - 1u) atomicAdd(ctr, kEpochOne - gridDim.x);  // the next launch's epoch
+  }
   for (int p = tid; p < np; p += kFuConsumers * 32) {
     s_ids[p] = a.ids[p];
     s_w[p] = a.w[p];
@@ -400,7 +397,18 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
     for (int i = tid; i < (Kp / a.g) * 8; i += kFuConsumers * 32)
       if (i % 8 >= a.T || i / 8 >= a.H / a.g) xq[2 * i] = xq[2 * i + 1] = 0.f;
   }
-  tables_sync();  // the producer's pass tables
+  if (warp == 0 && lane == 0) {
+    unsigned tg = 0u;  // 0: a count this launch cannot complete -- no valid tag, no work
+    if ((unsigned)cw < gridDim.x) {
+      const unsigned t = (unsigned)(cw >> 32) + 1u;
+      tg = fmix32(t == 0u ? 1u : t);  // fmix32 maps only 0 to 0
+    } else {
+      *abort_flag = 1;
+      if (a.dev_err) atomicOr(a.dev_err, MOE_DEV_ERR_TIMEOUT);
+    }
+    s_tag = tg;
+  }
+  tables_sync();  // the producer's pass tables (and the tag)
   const int n_act = s_nact, i0 = s_i0, i1 = s_i1;
   const unsigned tag = s_tag;
   // (entry, token) -> flat pair from the routed ids (a token routes to an expert at most once)
@@ -418,7 +426,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
     for (int i = tid; i < n_act; i += kFuConsumers * 32)
       if (!slot_ok(a, s_slot[i])) flag_slot(a, s_slot[i]);
   consumers_sync(kFuConsumers * 32);  // x' in shared memory, pair map written
-  bool timed_out = false;
+  bool timed_out = tag == 0u;
 
   // ---------------- gate/up + SwiGLU -> h: one item per warp pair ----------------
   {
