@@ -327,32 +327,56 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     tmap_prefetch(&tm_b128);
   }
   pdl_wait();
-  // the pass's experts and their tiles (token tiles x row tiles, row tile fastest)
+  // the pass's experts and their tiles (token tiles x row tiles, row tile
+  // fastest): the active list is read next to its length (one round), then
+  // the experts' slots and token ranges (a second), and the tile offsets are a
+  // warp scan
   if (warp == 0) {
-    int n = *a.n_active - a.pass_begin;
-    if (n > a.pass_len) n = a.pass_len;
-    if (n > kMaxCtaExperts) n = kMaxCtaExperts;
+    int cap = a.E - a.pass_begin;
+    if (cap > a.pass_len) cap = a.pass_len;
+    if (cap > kMaxCtaExperts) cap = kMaxCtaExperts;
+    if (cap < 0) cap = 0;
+    const int na = *a.n_active;
+    int ev[2];
+#pragma unroll
+    for (int qq = 0; qq < 2; ++qq) ev[qq] = lane + 32 * qq < cap ? a.active[a.pass_begin + lane + 32 * qq] : -1;
+    int n = na - a.pass_begin;
+    if (n > cap) n = cap;
     if (n < 0) n = 0;
-    for (int i = lane; i < n; i += 32) {
-      const int e = a.active[a.pass_begin + i];
+    int tiles[2];
+#pragma unroll
+    for (int qq = 0; qq < 2; ++qq) {
+      const int i = lane + 32 * qq, e = ev[qq];
+      const bool in = i < n && e >= 0 && e < a.E;
       PfEntry en;
-      en.slot = (e >= 0 && e < a.E) ? a.table[e] : -1;
-      en.pos0 = (e >= 0 && e < a.E) ? a.offsets[e] : 0;
-      en.cnt = (e >= 0 && e < a.E) ? a.offsets[e + 1] - en.pos0 : 0;
-      en.tile0 = 0;
-      s_ent[i] = en;
-      if (blockIdx.x == 0 && !slot_ok_pf(a.n_slots, en.slot) && a.dev_err)
-        atomicOr(a.dev_err, en.slot < 0 ? MOE_DEV_ERR_NOT_RESIDENT : MOE_DEV_ERR_SLOT_RANGE);
-    }
-    __syncwarp();
-    if (lane == 0) {
-      int acc = 0;
-      for (int i = 0; i < n; ++i) {
-        s_ent[i].tile0 = acc;
-        if (slot_ok_pf(a.n_slots, s_ent[i].slot)) acc += ((s_ent[i].cnt + kPfBN - 1) / kPfBN) * a.mtiles;
+      en.slot = in ? a.table[e] : -1;
+      en.pos0 = in ? a.offsets[e] : 0;
+      en.cnt = in ? a.offsets[e + 1] - en.pos0 : 0;
+      tiles[qq] = slot_ok_pf(a.n_slots, en.slot) ? ((en.cnt + kPfBN - 1) / kPfBN) * a.mtiles : 0;
+      if (i < n) {
+        en.slot = (e >= 0 && e < a.E) ? en.slot : -1;
+        s_ent[i] = en;
+        if (blockIdx.x == 0 && !slot_ok_pf(a.n_slots, en.slot) && a.dev_err)
+          atomicOr(a.dev_err, en.slot < 0 ? MOE_DEV_ERR_NOT_RESIDENT : MOE_DEV_ERR_SLOT_RANGE);
       }
+    }
+    // exclusive prefix of the tile counts over entries 0..63 (entry i = lane + 32 qq)
+    int incl0 = tiles[0], incl1 = tiles[1];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u0 = __shfl_up_sync(0xffffffffu, incl0, o), u1 = __shfl_up_sync(0xffffffffu, incl1, o);
+      if (lane >= o) {
+        incl0 += u0;
+        incl1 += u1;
+      }
+    }
+    const int tot0 = __shfl_sync(0xffffffffu, incl0, 31);
+    if (lane < n) s_ent[lane].tile0 = incl0 - tiles[0];
+    if (lane + 32 < n) s_ent[lane + 32].tile0 = tot0 + incl1 - tiles[1];
+    const int total = tot0 + __shfl_sync(0xffffffffu, incl1, 31);
+    if (lane == 0) {
       s_nent = n;
-      s_ntiles = acc;
+      s_ntiles = total;
     }
   }
   tc_fence_before();
