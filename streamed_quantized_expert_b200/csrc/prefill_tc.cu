@@ -56,19 +56,22 @@ namespace moe {
 namespace {
 
 constexpr int kPfBM = 128;      // weight rows per tile (MMA M)
-constexpr int kPfBN = 128;      // tokens per tile (MMA N, at most)
+constexpr int kPfBN = 128;      // tokens per tile (MMA N), at most; a launch takes 64 or 128
 constexpr int kPfABufs = 4;     // dequantised A buffers (in TMEM)
 constexpr int kPfDqWarps = 16;  // one per 8-row group of the 128-row tile
 constexpr int kPfEpiWarps = 8;  // two per TMEM lane quadrant, taking alternate 16-column chunks
 constexpr int kPfEpiWarp0 = kPfDqWarps, kPfProdWarp = kPfEpiWarp0 + kPfEpiWarps, kPfMmaWarp = kPfProdWarp + 1;
 constexpr int kPfThreads = (kPfMmaWarp + 1) * 32;
-constexpr int kPfTmemCols = 512;  // two accumulators of kPfBN fp32 columns, then the A buffers
-constexpr int kPfAcol = 2 * kPfBN;  // first TMEM column of the A buffers
+constexpr int kPfTmemCols = 512;  // two accumulators of NB fp32 columns, then the A buffers
 constexpr int kPfAcols = 64;       // one A buffer: 128 inputs as fp16 pairs, 128 lanes = rows
-static_assert(kPfAcol + kPfABufs * kPfAcols <= kPfTmemCols, "TMEM columns");
-constexpr int kPfXHalf = kPfBN * 128;   // one 64-input half of a token stage: 128 rows x 128 B
-// load stages (codes + scale/bias + token rows) that fit the shared memory
-__host__ __device__ constexpr int pf_stages(int bits) { return bits == 16 ? 3 : bits == 6 ? 4 : 5; }
+static_assert(2 * kPfBN + kPfABufs * kPfAcols <= kPfTmemCols, "TMEM columns");
+// load stages (codes + scale/bias + token rows of NB rows) that fit the
+// shared memory: a tile of at most 64 tokens has half the token bytes per
+// stage, so its ring is deeper (the ring, not the arithmetic, paces the
+// stages when the tokens per expert are few)
+__host__ __device__ constexpr int pf_stages(int bits, int nb) {
+  return nb == 64 ? (bits == 16 ? 4 : bits == 6 ? 7 : 8) : (bits == 16 ? 3 : bits == 6 ? 4 : 5);
+}
 
 struct PfEntry {
   int slot;    // slot of the expert (tiles skipped when not resident)
@@ -269,7 +272,7 @@ struct PfTile {
   int slot, row0;      // slot; first sorted position of the tile's tokens
 };
 
-template <int B, int GPB, bool GU>
+template <int B, int GPB, bool GU, int NB>
 __global__ void __launch_bounds__(kPfThreads, 1)
     pf_gemm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_sb,
                    const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_b64,
@@ -277,11 +280,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   extern __shared__ uint8_t pf_smem_raw[];
   constexpr int kCodesBytes = 2048 * B;   // 16 groups x 4 units x 8 rows x B words (B = 16: 128 x 128 bf16)
   constexpr int kSbBytes = B == 16 ? 0 : 512 * GPB;  // 8 tiles x 16 GPB words
-  constexpr int kPfStages = pf_stages(B);
+  constexpr int kPfStages = pf_stages(B, NB);
+  constexpr int kXHalf = NB * 128;  // one 64-input half of a token stage: NB rows x 128 B
+  constexpr int kAcol = 2 * NB;     // first TMEM column of the A buffers
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xst = base;                                           // [stage][2 halves][128 rows][128 B]
-  uint8_t* cst = xst + kPfStages * 2 * kPfXHalf;                 // [stage] codes
+  uint8_t* cst = xst + kPfStages * 2 * kXHalf;                 // [stage] codes
   uint8_t* sbst = cst + kPfStages * kCodesBytes;                 // [stage] scale/bias words
   uint64_t* bars = reinterpret_cast<uint64_t*>(sbst + kPfStages * kSbBytes);
   uint64_t* full = bars;                        // producer (expect_tx) -> dequant, MMA
@@ -313,7 +318,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     fence_barrier_init();
     s_abort = 0;
   }
-  if (warp == kPfMmaWarp) {  // TMEM: two accumulators of kPfBN columns
+  if (warp == kPfMmaWarp) {  // TMEM: two accumulators of NB columns
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem)),
                  "r"(kPfTmemCols)
                  : "memory");
@@ -352,7 +357,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       en.slot = in ? a.table[e] : -1;
       en.pos0 = in ? a.offsets[e] : 0;
       en.cnt = in ? a.offsets[e + 1] - en.pos0 : 0;
-      tiles[qq] = slot_ok_pf(a.n_slots, en.slot) ? ((en.cnt + kPfBN - 1) / kPfBN) * a.mtiles : 0;
+      tiles[qq] = slot_ok_pf(a.n_slots, en.slot) ? ((en.cnt + NB - 1) / NB) * a.mtiles : 0;
       if (i < n) {
         en.slot = (e >= 0 && e < a.E) ? en.slot : -1;
         s_ent[i] = en;
@@ -384,28 +389,31 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = s_tmem;
   const int nent = s_nent, ntiles = s_ntiles;
-  auto tile_at = [&](int t) -> PfTile {
-    int i = 0;
+  // tile t's entry: each role visits its tiles in increasing order, so the
+  // scan resumes from the entry of the role's previous tile (hint)
+  auto tile_at = [&](int t, int& hint) -> PfTile {
+    int i = hint;
     while (i + 1 < nent && s_ent[i + 1].tile0 <= t) ++i;
+    hint = i;
     const PfEntry en = s_ent[i];
     const int local = t - en.tile0;
     PfTile tl;
     tl.ent = i;
     tl.nt = local / a.mtiles;
     tl.mt = local - tl.nt * a.mtiles;
-    tl.n = en.cnt - tl.nt * kPfBN < kPfBN ? en.cnt - tl.nt * kPfBN : kPfBN;
+    tl.n = en.cnt - tl.nt * NB < NB ? en.cnt - tl.nt * NB : NB;
     tl.slot = en.slot;
-    tl.row0 = en.pos0 + tl.nt * kPfBN;
+    tl.row0 = en.pos0 + tl.nt * NB;
     return tl;
   };
 
   if (warp == kPfProdWarp) {
     // ---------------- producer ----------------
     if (lane == 0) {
-      int s = 0;
+      int s = 0, ent_hint = 0;
       uint32_t ph = 0, issued = 0, last_ph = 0;  // per-stage bit masks for the exit drain
       for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
-        const PfTile tl = tile_at(t);
+        const PfTile tl = tile_at(t, ent_hint);
         // the tile's token rows: one box of 32, 64 or 128 rows per 64-column half
         // (rows past the expert's tokens are loaded and never read by the MMA)
         const int brows = tl.n <= 32 ? 32 : tl.n <= 64 ? 64 : 128;
@@ -427,7 +435,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf)
-            tma_load_2d(xst + (s * 2 + hf) * kPfXHalf, tmb, kb * 128 + hf * 64, tl.row0, &full[s]);
+            tma_load_2d(xst + (s * 2 + hf) * kXHalf, tmb, kb * 128 + hf * 64, tl.row0, &full[s]);
           issued |= 1u << s;
           last_ph = (last_ph & ~(1u << s)) | (ph << s);
           if (++s == kPfStages) {
@@ -444,30 +452,33 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   } else if (warp == kPfMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      int s = 0, ab = 0, c = 0;
+      int s = 0, ab = 0, c = 0, ent_hint = 0;
       uint32_t ph = 0, pa = 0, pc = 0;
       bool issued_any = false;
       for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
-        const PfTile tl = tile_at(t);
+        const PfTile tl = tile_at(t, ent_hint);
         const int npad = (tl.n + 15) & ~15;
         const uint32_t idesc = idesc_f16(kPfBM, npad);
         if (!pf_wait(&accempty[c], pc ^ 1u, &s_abort, a.wait_limit)) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + (uint32_t)(c * kPfBN);
+        const uint32_t d = tmem_base + (uint32_t)(c * NB);
         bool ok = true;
         for (int kb = 0; kb < a.nkb; ++kb) {
+          // operands of the block's 8 MMAs, formed before the waits so that
+          // the issue loop is the MMAs alone (the thread shares its
+          // sub-partition's issue slots with the dequant warps)
+          const uint32_t a_tm = tmem_base + (uint32_t)(kAcol + ab * kPfAcols);
+          const uint64_t bd0 = sw128_desc(smem_addr(xst + s * 2 * kXHalf));  // + (offset >> 4): no carry (< 2^18 B)
+          const uint32_t acc0 = kb != 0 ? 1u : 0u;
           if (!pf_wait(&full[s], ph, &s_abort, a.wait_limit) || !pf_wait(&afull[ab], pa, &s_abort, a.wait_limit)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_tm = tmem_base + (uint32_t)(kPfAcol + ab * kPfAcols);
-          const uint32_t xbase = smem_addr(xst + s * 2 * kPfXHalf);
 #pragma unroll
-          for (int k16 = 0; k16 < 8; ++k16) {
-            const uint32_t off = (uint32_t)((k16 >> 2) * kPfXHalf + (k16 & 3) * 32);
-            umma_bf16_ta(d, a_tm + 8 * k16, sw128_desc(xbase + off), idesc, (kb | k16) != 0 ? 1u : 0u);
-          }
+          for (int k16 = 0; k16 < 8; ++k16)
+            umma_bf16_ta(d, a_tm + 8 * k16, bd0 + (uint64_t)(((k16 >> 2) * kXHalf + (k16 & 3) * 32) >> 4), idesc,
+                         k16 != 0 ? 1u : acc0);
           issued_any = true;
           umma_commit(&empty[s]);
           umma_commit(&aempty[ab]);
@@ -505,7 +516,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t ta = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kPfAcol + ab * kPfAcols);
+        const uint32_t ta = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAcol + ab * kPfAcols);
         if constexpr (B == 16)
           pf_bf16_quarter(cq, cst + s * kCodesBytes, ta, r);
         else
@@ -529,25 +540,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   } else {
     // ---------------- epilogue (TMEM lanes 32 (warp % 4) ..) ----------------
     const int q = warp & 3, r = 32 * q + lane, eh = (warp - kPfEpiWarp0) >> 2;  // quadrant, row, chunk parity
-    int c = 0;
+    int c = 0, ent_hint = 0;
     uint32_t pc = 0;
     for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
-      const PfTile tl = tile_at(t);
+      const PfTile tl = tile_at(t, ent_hint);
       if (!pf_wait(&accfull[c], pc, &s_abort, a.wait_limit)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * kPfBN);
+      const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * NB);
       // the tile's pair indices (down) in registers: lane l holds columns l, 32 + l, ...
-      int pidx[kPfBN / 32];
+      int pidx[NB / 32];
       if (!GU) {
 #pragma unroll
-        for (int q4 = 0; q4 < kPfBN / 32; ++q4)
+        for (int q4 = 0; q4 < NB / 32; ++q4)
           pidx[q4] = 32 * q4 + lane < tl.n ? a.pairs[tl.row0 + 32 * q4 + lane] : 0;
       }
       const bool gate = (r & 15) < 8;  // storage rows: 16-row blocks of 8 gate rows then 8 up rows
       const int j = tl.mt * (kPfBM / 2) + (r >> 4) * 8 + (r & 7);
       const int row = tl.mt * kPfBM + r;
 #pragma unroll
-      for (int nb = 0; nb < kPfBN / 32; ++nb) {
+      for (int nb = 0; nb < NB / 32; ++nb) {
         if (32 * nb >= tl.n) break;
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
@@ -654,18 +665,18 @@ bool encode_rows(CUtensorMap* m, const uint16_t* base, int64_t rows, int cols, i
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, d, s, b, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-size_t pf_smem_bytes(int bits, int gpb) {
-  const size_t ns = (size_t)pf_stages(bits);
-  return 1024 + ns * 2 * kPfXHalf + ns * 2048 * bits + (bits == 16 ? 0 : ns * 512 * gpb) +
+size_t pf_smem_bytes(int bits, int gpb, int nb) {
+  const size_t ns = (size_t)pf_stages(bits, nb);
+  return 1024 + ns * 2 * (size_t)nb * 128 + ns * 2048 * bits + (bits == 16 ? 0 : ns * 512 * gpb) +
          (2 * ns + 2 * kPfABufs + 5) * 8;
 }
 
-template <int B, int GPB, bool GU>
+template <int B, int GPB, bool GU, int NB>
 cudaError_t launch_pf_t(const CUtensorMap& q, const CUtensorMap& sb, const CUtensorMap (&bm)[3], const PfArgs& pa,
                         int grid, cudaStream_t st) {
   static int done[4] = {0, 0, 0, 0};
-  const void* kern = reinterpret_cast<const void*>(pf_gemm_kernel<B, GPB, GU>);
-  const size_t smem = pf_smem_bytes(B, GPB);
+  const void* kern = reinterpret_cast<const void*>(pf_gemm_kernel<B, GPB, GU, NB>);
+  const size_t smem = pf_smem_bytes(B, GPB, NB);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   if (dev >= 128) return cudaErrorNotSupported;
@@ -677,21 +688,28 @@ cudaError_t launch_pf_t(const CUtensorMap& q, const CUtensorMap& sb, const CUten
   return launch_pdl(kern, grid, kPfThreads, smem, st, q, sb, bm[0], bm[1], bm[2], pa);
 }
 
-template <int B, bool GU>
+template <int B, bool GU, int NB>
 cudaError_t launch_pf_gpb(int gpb, const CUtensorMap& q, const CUtensorMap& sb, const CUtensorMap (&bm)[3],
                           const PfArgs& pa, int grid, cudaStream_t st) {
-  if (gpb == 1) return launch_pf_t<B, 1, GU>(q, sb, bm, pa, grid, st);
-  if (gpb == 2) return launch_pf_t<B, 2, GU>(q, sb, bm, pa, grid, st);
-  return launch_pf_t<B, 4, GU>(q, sb, bm, pa, grid, st);
+  if (gpb == 1) return launch_pf_t<B, 1, GU, NB>(q, sb, bm, pa, grid, st);
+  if (gpb == 2) return launch_pf_t<B, 2, GU, NB>(q, sb, bm, pa, grid, st);
+  return launch_pf_t<B, 4, GU, NB>(q, sb, bm, pa, grid, st);
+}
+
+template <bool GU, int NB>
+cudaError_t launch_pf_nb(int bits, int gpb, const CUtensorMap& q, const CUtensorMap& sb, const CUtensorMap (&bm)[3],
+                         const PfArgs& pa, int grid, cudaStream_t st) {
+  if (bits == 3) return launch_pf_gpb<3, GU, NB>(gpb, q, sb, bm, pa, grid, st);
+  if (bits == 4) return launch_pf_gpb<4, GU, NB>(gpb, q, sb, bm, pa, grid, st);
+  if (bits == 16) return launch_pf_t<16, 1, GU, NB>(q, sb, bm, pa, grid, st);
+  return launch_pf_gpb<6, GU, NB>(gpb, q, sb, bm, pa, grid, st);
 }
 
 template <bool GU>
-cudaError_t launch_pf(int bits, int gpb, const CUtensorMap& q, const CUtensorMap& sb, const CUtensorMap (&bm)[3],
-                      const PfArgs& pa, int grid, cudaStream_t st) {
-  if (bits == 3) return launch_pf_gpb<3, GU>(gpb, q, sb, bm, pa, grid, st);
-  if (bits == 4) return launch_pf_gpb<4, GU>(gpb, q, sb, bm, pa, grid, st);
-  if (bits == 16) return launch_pf_t<16, 1, GU>(q, sb, bm, pa, grid, st);
-  return launch_pf_gpb<6, GU>(gpb, q, sb, bm, pa, grid, st);
+cudaError_t launch_pf(int bits, int gpb, int nb, const CUtensorMap& q, const CUtensorMap& sb,
+                      const CUtensorMap (&bm)[3], const PfArgs& pa, int grid, cudaStream_t st) {
+  return nb == 64 ? launch_pf_nb<GU, 64>(bits, gpb, q, sb, bm, pa, grid, st)
+                  : launch_pf_nb<GU, 128>(bits, gpb, q, sb, bm, pa, grid, st);
 }
 
 }  // namespace
@@ -747,6 +765,10 @@ cudaError_t launch_ffn_prefill_tc(const FfnArgs& a, const moe_layer_desc& d, int
   pa.dev_err = a.dev_err;
   pa.wait_limit = a.wait_limit;
   const int grid = num_sms;
+  // tokens per tile: 64 when an expert averages at most 48 of the chunk's
+  // pairs (the deeper load ring pays more than the second token tile of a
+  // crowded expert costs), else 128
+  const int nb = np <= 48LL * d.E ? 64 : 128;
   // a CTA's tile table holds kMaxCtaExperts experts: longer passes run as
   // several gate/up + down launches over consecutive sub-ranges (sub-ranges
   // past the active list find no experts), then one combine over the pass
@@ -757,12 +779,12 @@ cudaError_t launch_ffn_prefill_tc(const FfnArgs& a, const moe_layer_desc& d, int
     pa.K = d.H;
     pa.nkb = L.nblk_gu;
     pa.mtiles = 2 * d.I / kPfBM;
-    cudaError_t e = launch_pf<true>(d.bits_gu, gpb, q_gu, sb_gu, xm, pa, grid, st);
+    cudaError_t e = launch_pf<true>(d.bits_gu, gpb, nb, q_gu, sb_gu, xm, pa, grid, st);
     if (e != cudaSuccess) return e;
     pa.K = d.I;
     pa.nkb = L.nblk_d;
     pa.mtiles = d.H / kPfBM;
-    e = launch_pf<false>(d.bits_down, gpb, q_d, sb_d, hm, pa, grid, st);
+    e = launch_pf<false>(d.bits_down, gpb, nb, q_d, sb_d, hm, pa, grid, st);
     if (e != cudaSuccess) return e;
   }
   return launch_pdl(reinterpret_cast<const void*>(combine_kernel), combine_grid(a.T, d.H, num_sms), 256, 0, st, a);
