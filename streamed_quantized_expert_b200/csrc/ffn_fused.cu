@@ -346,6 +346,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
   if (warp == 0 && lane == 0) {
     unsigned long long* ctr = reinterpret_cast<unsigned long long*>(a.ctl);
     cw = atomicAdd(ctr, 1ull);
+    if ((unsigned)cw == gridDim.x - 1u) atomicAdd(ctr, kEpochOne - gridDim.x);  // the next launch's epoch
   }
   for (int p = tid; p < np; p += kFuConsumers * 32) {
     s_ids[p] = a.ids[p];
@@ -398,10 +399,6 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
   }
   if (warp == 0 && lane == 0) {
     unsigned tg = 0u;  // 0: a count this launch cannot complete -- no valid tag, no work
-    // the last arrival moves the word to the next launch's epoch (taken here,
-    // where the count is needed anyway, so the warp never waits on it earlier)
-    if ((unsigned)cw == gridDim.x - 1u)
-      atomicAdd(reinterpret_cast<unsigned long long*>(a.ctl), kEpochOne - gridDim.x);
     if ((unsigned)cw < gridDim.x) {
       const unsigned t = (unsigned)(cw >> 32) + 1u;
       tg = fmix32(t == 0u ? 1u : t);  // fmix32 maps only 0 to 0
@@ -522,29 +519,21 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
     const bool fast = a.T == 1 && n_act <= NSD && ntask <= kFuConsumers * kFuFastTasks;
     if (fast && !timed_out) {
       uint64_t fw[kFuFastTasks][4];
-      int fi[kFuFastTasks], fkb[kFuFastTasks], fp[kFuFastTasks], fsl[kFuFastTasks];
+      int fi[kFuFastTasks], fkb[kFuFastTasks];
       bool fv[kFuFastTasks];
-      const uint64_t* fsrc[kFuFastTasks];
 #pragma unroll
       for (int j = 0; j < kFuFastTasks; ++j) {
         const int task = warp + kFuConsumers * j;
         fi[j] = task < ntask ? task / nb : 0;
         fkb[j] = task < ntask ? task % nb : 0;
-      }
-#pragma unroll
-      for (int j = 0; j < kFuFastTasks; ++j) {
-        fp[j] = s_tok[fi[j] * kDenseMaxTokens];
-        fsl[j] = s_slot[fi[j]];
-      }
-      // every task reads at once, without branches; a task without h (none,
-      // or its expert has no slot) reads row 0 of the tag region (in bounds:
-      // one token has k >= 1 rows) and ignores it
-#pragma unroll
-      for (int j = 0; j < kFuFastTasks; ++j) {
-        fv[j] = warp + kFuConsumers * j < ntask && slot_ok(a, fsl[j]) && fp[j] >= 0;
-        fsrc[j] = htag + (int64_t)(fv[j] ? fp[j] : 0) * Ip + fkb[j] * 128 + 4 * lane;
-        ld_volatile_2w(fsrc[j], fw[j][0], fw[j][1]);
-        ld_volatile_2w(fsrc[j] + 2, fw[j][2], fw[j][3]);
+        const int p = task < ntask ? s_tok[fi[j] * kDenseMaxTokens] : -1;
+        fv[j] = task < ntask && slot_ok(a, s_slot[fi[j]]) && p >= 0;
+        fw[j][0] = fw[j][1] = fw[j][2] = fw[j][3] = 0ull;
+        if (fv[j]) {
+          const uint64_t* src = htag + (int64_t)p * Ip + fkb[j] * 128 + 4 * lane;
+          ld_volatile_2w(src, fw[j][0], fw[j][1]);
+          ld_volatile_2w(src + 2, fw[j][2], fw[j][3]);
+        }
       }
       const long long t0 = clock64();
       for (;;) {
@@ -567,60 +556,41 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
 #pragma unroll
         for (int j = 0; j < kFuFastTasks; ++j)
           if (!fresh[j]) {
-            ld_volatile_2w(fsrc[j], fw[j][0], fw[j][1]);
-            ld_volatile_2w(fsrc[j] + 2, fw[j][2], fw[j][3]);
+            const uint64_t* src = htag + (int64_t)s_tok[fi[j] * kDenseMaxTokens] * Ip + fkb[j] * 128 + 4 * lane;
+            ld_volatile_2w(src, fw[j][0], fw[j][1]);
+            ld_volatile_2w(src + 2, fw[j][2], fw[j][3]);
           }
       }
-      // stage each task's block (its own scratch row) and its per-group sums,
-      // the tasks side by side (no branches, so their shuffles interleave)
+      // stage each task's block (its own scratch row) and its per-group sums
       const int kk = (4 * lane) & 127;
       const bool eighth = PairShift<BD>::a(2 * (kk >> 4) + ((kk & 15) >> 3)) == 3;
       const int lpg = a.g / 4;  // lanes per group (8, 16 or 32)
-      float fsx[kFuFastTasks], fso[kFuFastTasks];
 #pragma unroll
       for (int j = 0; j < kFuFastTasks; ++j) {
+        if (!fv[j]) continue;  // warp-uniform
         const int c0 = fkb[j] * 128 + 4 * lane;
-        const uint32_t h0 = fv[j] && c0 < a.I ? (uint32_t)(fw[j][0] & 0xFFFFu) : 0u;
-        const uint32_t h1 = fv[j] && c0 + 1 < a.I ? (uint32_t)(fw[j][1] & 0xFFFFu) : 0u;
-        const uint32_t h2 = fv[j] && c0 + 2 < a.I ? (uint32_t)(fw[j][2] & 0xFFFFu) : 0u;
-        const uint32_t h3 = fv[j] && c0 + 3 < a.I ? (uint32_t)(fw[j][3] & 0xFFFFu) : 0u;
+        const uint32_t h0 = c0 < a.I ? (uint32_t)(fw[j][0] & 0xFFFFu) : 0u;
+        const uint32_t h1 = c0 + 1 < a.I ? (uint32_t)(fw[j][1] & 0xFFFFu) : 0u;
+        const uint32_t h2 = c0 + 2 < a.I ? (uint32_t)(fw[j][2] & 0xFFFFu) : 0u;
+        const uint32_t h3 = c0 + 3 < a.I ? (uint32_t)(fw[j][3] & 0xFFFFu) : 0u;
         uint32_t* dst = hsc + j * kFuScratchRowWords + frag_word(4 * lane);  // pairs one t4 apart
         dst[0] = h0 | (h1 << 16);
         dst[16] = h2 | (h3 << 16);
         const float v = __uint_as_float(h0 << 16) + __uint_as_float(h1 << 16) + __uint_as_float(h2 << 16) +
                         __uint_as_float(h3 << 16);
-        fsx[j] = eighth ? 8.0f * v : v;
-        fso[j] = 128.0f * v;
-      }
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-#pragma unroll
-        for (int j = 0; j < kFuFastTasks; ++j) {
-          const float tx = __shfl_xor_sync(0xffffffffu, fsx[j], o);
-          const float to = __shfl_xor_sync(0xffffffffu, fso[j], o);
-          if (o < lpg) {
-            fsx[j] += tx;
-            fso[j] += to;
-          }
+        float sx = eighth ? 8.0f * v : v, so = 128.0f * v;
+        for (int o = 1; o < lpg; o <<= 1) {
+          sx += __shfl_xor_sync(0xffffffffu, sx, o);
+          so += __shfl_xor_sync(0xffffffffu, so, o);
         }
-      }
-      if ((lane % lpg) == 0) {
-#pragma unroll
-        for (int j = 0; j < kFuFastTasks; ++j) gsum[j * GPB + lane / lpg] = make_float2(fsx[j], fso[j]);
+        if ((lane % lpg) == 0) gsum[j * GPB + lane / lpg] = make_float2(sx, so);
       }
       __syncwarp();
-      // the tasks' down tiles: entry i on stage i, its first and only use (one
-      // test of all of them, as they have usually landed; else wait in turn)
-      bool landed = true;
+      // the tasks' down tiles: entry i on stage i, its first and only use
 #pragma unroll
-      for (int j = 0; j < kFuFastTasks; ++j)
-        landed &= !fv[j] || (reinterpret_cast<volatile int*>(s_iss)[NSG + fi[j]] > 0 && mbar_test(&dfull[fi[j]], 0u));
-      if (!landed) {
-#pragma unroll
-        for (int j = 0; j < kFuFastTasks; ++j) {
-          if (!fv[j] || timed_out) continue;
-          if (!issued(NSG + fi[j], 0) || !mbar_wait_bounded(&dfull[fi[j]], 0u, a.wait_limit)) timed_out = true;
-        }
+      for (int j = 0; j < kFuFastTasks; ++j) {
+        if (!fv[j] || timed_out) continue;
+        if (!issued(NSG + fi[j], 0) || !mbar_wait_bounded(&dfull[fi[j]], 0u, a.wait_limit)) timed_out = true;
       }
       if (timed_out) *abort_flag = 1;
 #pragma unroll
