@@ -435,9 +435,10 @@ def run_prefill(args, rank, world, local_rank, name=None, layers=0, embedded=Fal
                       % args.ffn_reps}
     roof = {"bound": "tensor", "achieved": round(tflops, 2), "peak": tf_peak, "unit": "TFLOP/s",
             "frac": round(tflops / tf_peak, 4),
-            "traffic": recorded_traffic("pf_gemm_kernel"),
+            # the capture covers the 1024-token Flash-Next-like chunk only
+            "traffic": recorded_traffic("pf_gemm_kernel") if (name or args.config) == "prefill" else None,
             "traffic_note": "DRAM bytes of one 64-expert pass's gate/up + down launches of the 1024-token "
-                            "Flash-Next-like chunk (profiles/traffic.txt)",
+                            "Flash-Next-like chunk (profiles/traffic.txt); null for other workloads",
             "hbm": {"achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4)},
             "kernel": "pf_gemm_kernel (gate/up + SwiGLU, down) + combine, per pass",
             "flops_per_layer": 2.0 * T * k * 3 * H * I, "peak_kind": peak_kind}
@@ -757,7 +758,8 @@ def run_ours(args, rank, world, local_rank):
                          "how_compared": "same tokens and initial cache, L = 0, installs of the timed steps"})},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4),
-                     "traffic": recorded_traffic("ffn_fused_kernel") if T * k <= 64 and T <= 8 else None,
+                     # the capture covers the default decode workload only
+                     "traffic": recorded_traffic("ffn_fused_kernel") if args.config == "decode" else None,
                      "kernel": ("ffn_fused_kernel (one launch per layer: every CTA gate/up + SwiGLU items, then the "
                                 "first H/16 CTAs a down + combine tile, over launch-tagged h words)" if T <= 8 and T * k <= 64 else
                                 "pf_gemm_kernel (tcgen05 grouped GEMM: gate/up + SwiGLU, down) + combine, per layer"
