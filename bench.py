@@ -86,6 +86,10 @@ CONFIGS = {
                       "Flash-Next-like decode with one always-on shared expert per layer (same shape, pinned slot, "
                       "run in the routed experts' FFN launch): 48 layers x 512 routed experts, top-10, H 2048, I 512, "
                       "3-bit g64, 1 token/step, 192 slots/layer, misses installed from pinned host"),
+    "decode_resident": (48, 512, 10, 2048, 512, 64, 3, 3, 1, 512,
+                        "Flash-Next-like decode with every expert resident: 48 layers x 512 experts, top-10, H 2048, "
+                        "I 512, 3-bit g64, 1 token/step, 512 slots/layer (34 GB of slots); no layer synchronises "
+                        "with the host, so each step is one CUDA graph of the 48 layers' moe_decode_layer calls"),
     "decode_mixed": (48, 512, 10, 2048, 512, 64, 4, 4, 1, 128,
                      "mixed size classes decode with cache-aware substitution: Flash-Next-like shapes, 4-bit "
                      "gate/up, 6-bit down on layers l % 4 == 0 (2 slot size classes), 1 token/step, 128 slots/layer "
@@ -95,7 +99,8 @@ CONFIGS = {
 SWEEP = {"coder": (1, 8, 32)}
 # per-layer widths and the substitution strength of the decode configurations (default: uniform, L = 0)
 DECODE_EXTRA = {"decode_mixed": {"bits": lambda l: (4, 6) if l % 4 == 0 else (4, 4), "L": 0.15},
-                "decode_shared": {"n_shared": 1}}
+                "decode_shared": {"n_shared": 1},
+                "decode_resident": {"graph_step": True}}
 
 # Prefill chunks: every expert of every layer resident (the metric is the expert
 # FFN's tensor-core rate; installs are PCIe-bound and reported by decode).
@@ -188,7 +193,7 @@ SEQUENCE = {
 }
 
 
-def build_streamer(cfg, seed, device, bits=None, max_tokens=None, n_shared=0):
+def build_streamer(cfg, seed, device, bits=None, max_tokens=None, n_shared=0, stream=None):
     import numpy as np
     import torch
 
@@ -207,7 +212,7 @@ def build_streamer(cfg, seed, device, bits=None, max_tokens=None, n_shared=0):
     specs = [LayerSpec(d, banks[(d.bits_gu, d.bits_down)], synth.bank_permutation(seed, l, E).tolist(),
                        shared[None] if n_shared else None)
              for l, d in enumerate(descs)]
-    st = Streamer(specs, S, max_tokens=max_tokens or T, device=device, n_shared=n_shared)
+    st = Streamer(specs, S, max_tokens=max_tokens or T, device=device, n_shared=n_shared, stream=stream)
     for l in range(n_layers):  # the S most popular experts start resident, on a random slot permutation
         hot = np.argsort(synth.popularity_rank(seed, l, E))[:S]
         st.place(l, hot.tolist(), synth.slot_permutation(seed, l, S).tolist())
@@ -611,7 +616,9 @@ def run_ours(args, rank, world, local_rank):
     extra = DECODE_EXTRA.get(args.config, {})
     Lsub = extra.get("L", 0.0)
     seed = 1000 * rank
-    st = build_streamer(cfg, seed, device, extra.get("bits"), n_shared=extra.get("n_shared", 0))
+    # a step captured as a CUDA graph runs on a stream of its own (capture needs a non-default stream)
+    st = build_streamer(cfg, seed, device, extra.get("bits"), n_shared=extra.get("n_shared", 0),
+                        stream=torch.cuda.Stream(device) if extra.get("graph_step") else None)
     steps_total = args.warmup + args.steps
     # the popularity bias of the logits and the initially resident experts come from the same seed
     x, logits = make_inputs(cfg, seed, steps_total + 1, device)
@@ -624,6 +631,20 @@ def run_ours(args, rank, world, local_rank):
     for i in range(args.warmup):
         step(i, x, logits)
     torch.cuda.synchronize(device)
+    graphs = []
+    if extra.get("graph_step"):
+        # every layer fully resident: the driver never waits on the host, so each
+        # timed step (its own inputs) is captured once and replayed in the timed region
+        if any(st.cache.resident(l) < E for l in range(n_layers)):
+            raise RuntimeError("graph_step needs every expert of every layer resident")
+        l_cap = st.launches
+        for i in range(args.warmup, steps_total):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=s):
+                step(i, x, logits)
+            graphs.append(gr)
+        torch.cuda.synchronize(device)
+        graph_launches = (st.launches - l_cap) // max(len(graphs), 1)
     if world > 1:
         dist.barrier()
 
@@ -633,12 +654,17 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(device)
         e0.record(s)
         for i in range(args.warmup, steps_total):
-            step(i, x, logits)
+            if graphs:
+                with torch.cuda.stream(s):  # replayed on the stream the events are recorded on
+                    graphs[i - args.warmup].replay()
+            else:
+                step(i, x, logits)
         e1.record(s)
         torch.cuda.synchronize(device)
         ms = e0.elapsed_time(e1)
-        launches = st.launches - l0
+        launches = st.launches - l0 if not graphs else graph_launches * len(graphs)
         installs, inst_bytes = st.installs - inst0, st.installed_bytes - bytes0
+        del graphs
 
         # one more (untimed) step whose per-layer routing is kept for the FFN-only replay
         snaps = []
@@ -722,7 +748,9 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC,
         "value": round(tokens / (ms_max / 1e3), 3),
         "unit": "tok/s",
-        "value_is": "decode tok/s of the whole path (route+sort+lookup+installs+FFN+combine, %d layers)" % n_layers,
+        "value_is": ("decode tok/s of the whole path (route+sort+FFN+combine, %d layers, every expert resident: one "
+                     "CUDA graph per step, replayed)" if extra.get("graph_step") else
+                     "decode tok/s of the whole path (route+sort+lookup+installs+FFN+combine, %d layers)") % n_layers,
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,

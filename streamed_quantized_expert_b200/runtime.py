@@ -119,6 +119,7 @@ class Streamer:
         self.installed_bytes = 0
         self.installs = 0
         self.launches = 0          # libmoe kernel launches issued (for reporting)
+        self._paths = {}           # (layer, T, sorted x) -> moe_ffn_kernel_path
         # native per-layer driver state
         self.installed.record(self.side)  # materialise the event
         bf16 = any(l.desc.bits_gu == 16 or l.desc.bits_down == 16 for l in layers)
@@ -246,6 +247,28 @@ class Streamer:
             ev[1].record(self.stream)
             self.ffn_events.append(ev)
 
+    def _ffn_launches(self, layer: int, T: int, pass_len: int) -> int:
+        """Kernels one moe_expert_ffn call over pass_len experts launches."""
+        d = self.wdesc[layer]
+        tc = T >= 32 or d.bits_gu == 16 or d.bits_down == 16
+        key = (layer, T, tc)
+        path = self._paths.get(key)
+        if path is None:
+            path = self._paths[key] = ops.moe_ffn_kernel_path(d, T, tc)
+        if path == 0:
+            return 1  # the fused decode kernel
+        if path == 2:  # gate/up + down per sub-range of 64 experts, then the combine
+            return 2 * -(-min(pass_len, self.Ew) // 64) + 1
+        return 3
+
+    def _decode_launches(self, layer: int, T: int, full: bool, n_installed: int) -> int:
+        d = self.layers[layer].desc
+        tc = T >= 32 or d.bits_gu == 16 or d.bits_down == 16
+        n = 1 + (1 if T * self.kw <= 1024 else 3) + (1 if tc else 0) + (0 if full else 1)  # route, sort, lookup
+        if n_installed:  # resident experts, then the installed ones
+            return n + self._ffn_launches(layer, T, self.kw * T) + self._ffn_launches(layer, T, n_installed)
+        return n + self._ffn_launches(layer, T, self.Ew)
+
     def decode_layer(self, layer: int, x, logits, T: int, L: float = 0.0, y=None):
         """One decode layer (T <= 64 tokens) through the native driver
         (moe_decode_layer); returns y fp32 [T, H] (device)."""
@@ -256,7 +279,7 @@ class Streamer:
         if n:
             self.installs += n
             self.installed_bytes += n * self.class_bytes[self.layer_class[layer]]
-        self.launches += 4 + (0 if full else 1) + (0 if T * self.kw <= 1024 else 2)
+        self.launches += self._decode_launches(layer, T, full, n)
         return y
 
     def decode_layer_ahead(self, layer: int, x, logits, T: int, L: float = 0.0, guesses=(), y=None):
@@ -272,7 +295,7 @@ class Streamer:
         if n:
             self.installs += n
             self.installed_bytes += n * self.class_bytes[self.layer_class[layer]]
-        self.launches += 4 + len(g) + (0 if full else 1) + (0 if T * self.kw <= 1024 else 2)
+        self.launches += self._decode_launches(layer, T, full, n) + len(g)
         return y
 
     def decode_layer_steps(self, layer: int, x, logits, T: int, L: float = 0.0, y=None):
