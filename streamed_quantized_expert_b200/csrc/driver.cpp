@@ -150,15 +150,24 @@ moe_status decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc
   int32_t* n_miss = b->meta + 1;
   int32_t* active = b->meta + 2;
   int32_t* miss = b->meta + 2 + E;
-  moe_status s = ns ? moe_route_shared(logits, T, d0, L, lc->table_dev, ns, lc->shared_w, b->ids, b->w, stream)
-                    : moe_route(logits, T, d0, L, lc->table_dev, b->ids, b->w, stream);
-  if (s != MOE_OK) return s;
   // from 32 tokens (BF16 experts: always) the FFN runs on the tensor-core grouped GEMM, which reads x
   // sorted by expert
   uint16_t* xs = ((T >= 32 || d0->bits_gu == 16 || d0->bits_down == 16) && b->x_sorted) ? b->x_sorted : nullptr;
-  s = moe_sort(b->ids, xs ? x : nullptr, T, d, b->offsets, b->pairs, active, n_active, xs, b->ws, b->ws_bytes,
-               stream);
-  if (s != MOE_OK) return s;
+  // one token without shared experts or sorted x: routing, sort and lookup in one launch
+  const bool one = T == 1 && ns == 0 && !xs;
+  moe_status s = MOE_OK;
+  if (one) {
+    s = moe_route_sort_lookup(logits, T, d0, L, lc->table_dev, lc->n_slots, b->ids, b->w, b->offsets, b->pairs,
+                              active, n_active, b->slots, miss, n_miss, b->dev_err, stream);
+    if (s != MOE_OK) return s;
+  } else {
+    s = ns ? moe_route_shared(logits, T, d0, L, lc->table_dev, ns, lc->shared_w, b->ids, b->w, stream)
+           : moe_route(logits, T, d0, L, lc->table_dev, b->ids, b->w, stream);
+    if (s != MOE_OK) return s;
+    s = moe_sort(b->ids, xs ? x : nullptr, T, d, b->offsets, b->pairs, active, n_active, xs, b->ws, b->ws_bytes,
+                 stream);
+    if (s != MOE_OK) return s;
+  }
   // the guessed layers' top-k, on the same synchronisation as the layer's own lookup
   const bool guessing = G && G->n > 0;
   if (guessing) {
@@ -179,9 +188,11 @@ moe_status decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc
     if (s != MOE_OK) return s;
   }
   if (!resident) {
-    s = moe_slot_lookup(lc->table_dev, active, n_active, 0, E, lc->n_slots, b->slots, miss, n_miss, b->dev_err,
-                        stream);
-    if (s != MOE_OK) return s;
+    if (!one) {
+      s = moe_slot_lookup(lc->table_dev, active, n_active, 0, E, lc->n_slots, b->slots, miss, n_miss, b->dev_err,
+                          stream);
+      if (s != MOE_OK) return s;
+    }
     if (cudaMemcpyAsync(b->meta_host, b->meta, sizeof(int32_t) * (size_t)(2 + E), cudaMemcpyDeviceToHost,
                         stream) != cudaSuccess)
       return MOE_ERR_CUDA;

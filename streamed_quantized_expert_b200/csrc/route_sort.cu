@@ -167,11 +167,13 @@ __device__ __forceinline__ bool key_before(uint32_t a1, uint32_t a2, int ae, uin
   return a1 > b1 || (a1 == b1 && (a2 > b2 || (a2 == b2 && ae < be)));
 }
 
+// The 256 threads of the block route the token of logits row `l`: ids_row /
+// w_row receive its k experts in key order and their weights, then the ns
+// shared experts (ids E.., weight sw_t).
 template <int NPT>
-__global__ void __launch_bounds__(256) route_select_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                                           float L, const int32_t* __restrict__ table,
-                                                           int32_t* __restrict__ ids, float* __restrict__ wout, int ns,
-                                                           const float* __restrict__ sw) {
+__device__ __forceinline__ void route_select_token(const float* __restrict__ l, int E, int k, float L,
+                                                   const int32_t* __restrict__ table, int32_t* __restrict__ ids_row,
+                                                   float* __restrict__ w_row, int ns, float sw_t) {
   __shared__ float s_red[8];
   __shared__ uint32_t s_hist[256];
   __shared__ int s_ctl[3];  // boundary digit, experts still to take, boundary bucket size
@@ -183,11 +185,6 @@ __global__ void __launch_bounds__(256) route_select_kernel(const float* __restri
   __shared__ int s_oe[32];
   __shared__ float s_ou[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t = blockIdx.x;
-  pdl_wait();
-  pdl_launch_dependents();
-  if (t >= T) return;
-  const float* l = logits + (size_t)t * E;
   float lv[NPT], u[NPT];
   bool res[NPT];
   float lmax = -FLT_MAX;
@@ -335,14 +332,76 @@ __global__ void __launch_bounds__(256) route_select_kernel(const float* __restri
     float sum = my_u;
 #pragma unroll
     for (int o = 16; o; o >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, o));
-    const int ks = k + ns;  // output row: the top-k, then the shared experts
-    if (mine) {
-      ids[(size_t)t * ks + lane] = s_oe[lane];
-      wout[(size_t)t * ks + lane] = __fdiv_rn(my_u, sum);
+    if (mine) {  // the row: the top-k, then the shared experts
+      ids_row[lane] = s_oe[lane];
+      w_row[lane] = __fdiv_rn(my_u, sum);
     }
     if (lane < ns) {
-      ids[(size_t)t * ks + k + lane] = E + lane;
-      wout[(size_t)t * ks + k + lane] = sw ? sw[t] : 1.0f;
+      ids_row[k + lane] = E + lane;
+      w_row[k + lane] = sw_t;
+    }
+  }
+}
+
+template <int NPT>
+__global__ void __launch_bounds__(256) route_select_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                           float L, const int32_t* __restrict__ table,
+                                                           int32_t* __restrict__ ids, float* __restrict__ wout, int ns,
+                                                           const float* __restrict__ sw) {
+  const int t = blockIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
+  if (t >= T) return;
+  const int ks = k + ns;  // output row: the top-k, then the shared experts
+  route_select_token<NPT>(logits + (size_t)t * E, E, k, L, table, ids + (size_t)t * ks, wout + (size_t)t * ks, ns,
+                          (ns > 0 && sw) ? sw[t] : 1.0f);
+}
+
+// One decode token's stages 1-3 in one block: route (as route_select_kernel),
+// then the sort of its k pairs (distinct experts: the active list is the
+// routed experts ascending, pair j of rank r at position r) and the slot
+// lookup over the whole active list (as sort_small_kernel and lookup_kernel
+// write them for T = 1).
+template <int NPT>
+__global__ void __launch_bounds__(256) route_sort_lookup_kernel(
+    const float* __restrict__ logits, int E, int k, float L, const int32_t* __restrict__ table, int n_slots,
+    int32_t* __restrict__ ids, float* __restrict__ w, int32_t* __restrict__ offsets, int32_t* __restrict__ pairs,
+    int32_t* __restrict__ active, int32_t* __restrict__ n_active, int32_t* __restrict__ slots,
+    int32_t* __restrict__ miss, int32_t* __restrict__ n_miss, int32_t* __restrict__ dev_err) {
+  __shared__ int s_sel[32];  // the routed experts, rank order
+  __shared__ int s_act[32];  // ascending
+  const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_launch_dependents();
+  route_select_token<NPT>(logits, E, k, L, table, ids, w, 0, 1.0f);
+  __syncthreads();  // the block's own global writes of ids are visible to it
+  if (tid < k) s_sel[tid] = ids[tid];
+  __syncthreads();
+  if (tid < k) {
+    const int e = s_sel[tid];
+    int r = 0;
+    for (int j = 0; j < k; ++j) r += s_sel[j] < e;
+    s_act[r] = e;
+    active[r] = e;
+    pairs[r] = tid;
+  }
+  for (int e = tid; e <= E; e += 256) {
+    int c = 0;
+    for (int j = 0; j < k; ++j) c += s_sel[j] < e;
+    offsets[e] = c;
+  }
+  __syncthreads();
+  if (tid < 32) {  // lookup: one lane per active expert (k <= 32)
+    const bool in = tid < k;
+    const int e = in ? s_act[tid] : -1;
+    const int sl = in ? table[e] : 0;
+    if (in) slots[tid] = sl;
+    if (in && sl >= n_slots && dev_err) atomicOr(dev_err, MOE_DEV_ERR_SLOT_RANGE);
+    const unsigned bal = __ballot_sync(0xffffffffu, in && sl < 0);
+    if (in && sl < 0) miss[__popc(bal & ((1u << tid) - 1u))] = e;
+    if (tid == 0) {
+      *n_active = k;
+      *n_miss = __popc(bal);
     }
   }
 }
@@ -547,6 +606,17 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, float L, cons
                      : E <= 512 ? reinterpret_cast<const void*>(route_kernel<16>)
                                 : reinterpret_cast<const void*>(route_kernel<32>);
   return launch_pdl(kern, blocks, 256, 0, st, logits, T, E, k, L, table, ids, w, n_shared, shared_w);
+}
+
+cudaError_t launch_route_sort_lookup(const float* logits, int E, int k, float L, const int32_t* table, int n_slots,
+                                     int32_t* ids, float* w, int32_t* offsets, int32_t* pairs, int32_t* active,
+                                     int32_t* n_active, int32_t* slots, int32_t* miss, int32_t* n_miss,
+                                     int32_t* dev_err, cudaStream_t st) {
+  const void* kb = E <= 256 ? reinterpret_cast<const void*>(route_sort_lookup_kernel<1>)
+                   : E <= 512 ? reinterpret_cast<const void*>(route_sort_lookup_kernel<2>)
+                              : reinterpret_cast<const void*>(route_sort_lookup_kernel<4>);
+  return launch_pdl(kb, 1, 256, 0, st, logits, E, k, L, table, n_slots, ids, w, offsets, pairs, active, n_active,
+                    slots, miss, n_miss, dev_err);
 }
 
 size_t sort_ws_bytes(int n, int E) { return n <= 1024 ? 0 : (size_t)((n + 1023) / 1024) * E * sizeof(int32_t); }

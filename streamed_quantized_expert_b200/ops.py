@@ -27,7 +27,7 @@ ABI_SYMBOLS = [
     "moe_expert_ffn_noalloc", "moe_noalloc_scratch_bytes", "moe_cache_resident", "moe_decode_layer",
     "moe_last_cuda_error", "moe_ffn_kernel_path", "moe_set_wait_limit_cycles", "moe_route_shared",
     "moe_router_logits", "moe_cache_reserve", "moe_cache_commit", "moe_prefetch_create", "moe_prefetch_destroy",
-    "moe_prefetch_stats", "moe_decode_layer_ahead",
+    "moe_prefetch_stats", "moe_decode_layer_ahead", "moe_route_sort_lookup",
 ]
 
 
@@ -92,6 +92,7 @@ def lib():
             "moe_route_shared": (C.c_int, [P, i32, D, f32, P, i32, P, P, P, P]),
             "moe_sort": (C.c_int, [P, P, i32, D, P, P, P, P, P, P, sz, P]),
             "moe_slot_lookup": (C.c_int, [P, P, P, i32, i32, i32, P, P, P, P, P]),
+            "moe_route_sort_lookup": (C.c_int, [P, i32, D, f32, P, i32, P, P, P, P, P, P, P, P, P, P, P]),
             "moe_install_slots": (C.c_int, [P, sz, i32, P, P, i32, P, P]),
             "moe_expert_ffn": (C.c_int, [P, i32, D, P, i32, P, P, P, P, P, P, P, P, i32, i32, P, P, sz, P, P]),
             "moe_expert_ffn_noalloc": (C.c_int, [P, i32, D, P, i32, P, P, P, P, P, P, P, i32, i32, P, P, P]),
@@ -215,6 +216,16 @@ def widened(d: LayerDesc, n_shared: int) -> LayerDesc:
 def moe_sort(ids, x, T, d, offsets, pairs, active, n_active, x_sorted, ws, ws_bytes, stream=None) -> None:
     _ck(lib().moe_sort(_ptr(ids), _ptr(x), int(T), C.byref(d), _ptr(offsets), _ptr(pairs), _ptr(active),
                        _ptr(n_active), _ptr(x_sorted), _ptr(ws), int(ws_bytes), _stream(stream)), "moe_sort")
+
+
+def moe_route_sort_lookup(logits, T, d, L, slot_table, n_slots, ids, w, offsets, pairs, active, n_active, slots,
+                          miss, n_miss, dev_err, stream=None) -> None:
+    """moe_route + moe_sort (no x_sorted) + moe_slot_lookup over the whole
+    active list for one token, in one launch (T must be 1)."""
+    _ck(lib().moe_route_sort_lookup(_ptr(logits), int(T), C.byref(d), float(L), _ptr(slot_table), int(n_slots),
+                                    _ptr(ids), _ptr(w), _ptr(offsets), _ptr(pairs), _ptr(active), _ptr(n_active),
+                                    _ptr(slots), _ptr(miss), _ptr(n_miss), _ptr(dev_err), _stream(stream)),
+        "moe_route_sort_lookup")
 
 
 def moe_slot_lookup(slot_table, active, n_active, pass_begin, pass_len, n_slots, slots, miss, n_miss, dev_err,

@@ -264,7 +264,10 @@ class Streamer:
     def _decode_launches(self, layer: int, T: int, full: bool, n_installed: int) -> int:
         d = self.layers[layer].desc
         tc = T >= 32 or d.bits_gu == 16 or d.bits_down == 16
-        n = 1 + (1 if T * self.kw <= 1024 else 3) + (1 if tc else 0) + (0 if full else 1)  # route, sort, lookup
+        if T == 1 and not self.ns and not tc:
+            n = 1  # moe_route_sort_lookup
+        else:
+            n = 1 + (1 if T * self.kw <= 1024 else 3) + (1 if tc else 0) + (0 if full else 1)  # route, sort, lookup
         if n_installed:  # resident experts, then the installed ones
             return n + self._ffn_launches(layer, T, self.kw * T) + self._ffn_launches(layer, T, n_installed)
         return n + self._ffn_launches(layer, T, self.Ew)
