@@ -262,6 +262,29 @@ moe_status moe_expert_ffn(const uint16_t* x, int32_t T, const moe_layer_desc* d,
                           int32_t pass_len, float* y_accum, void* ws, size_t ws_bytes, int32_t* dev_err,
                           cudaStream_t stream);
 
+/* Stages 1-5 of one decode token in one launch, for a layer whose routed
+ * experts are resident (RFC "How the prototype works", item "Cache": a fully
+ * resident layer never synchronises with the host, so its routing need not
+ * leave the device before its FFN).  The fused decode kernel routes the token
+ * itself -- the routing of moe_route with strength L over slot_table's
+ * residency, bit for bit -- and runs every routed expert, as
+ * moe_route_sort_lookup followed by moe_expert_ffn over one pass would.
+ *   x        device bf16 [1, H];  logits  device fp32 [1, E]
+ *   T        must be 1; E <= 1024; quantized experts only (else
+ *            MOE_ERR_UNSUPPORTED: use moe_route_sort_lookup and
+ *            moe_expert_ffn)
+ *   ids, w, offsets, pairs, active, n_active, slots, miss, n_miss: device
+ *            outputs, the values moe_route_sort_lookup writes
+ *   y        device fp32 [1, H], OVERWRITTEN with the layer's output
+ *   ws       device workspace, ws_bytes >= moe_workspace_bytes(d, 1)
+ *   dev_err  as moe_expert_ffn: a routed expert without a slot is flagged
+ *            MOE_DEV_ERR_NOT_RESIDENT (and listed in miss) and skipped */
+moe_status moe_route_expert_ffn(const uint16_t* x, const float* logits, int32_t T, const moe_layer_desc* d, float L,
+                                const void* pool, int32_t n_slots, const int32_t* slot_table, int32_t* ids, float* w,
+                                int32_t* offsets, int32_t* pairs, int32_t* active, int32_t* n_active, int32_t* slots,
+                                int32_t* miss, int32_t* n_miss, float* y, void* ws, size_t ws_bytes, int32_t* dev_err,
+                                cudaStream_t stream);
+
 /* moe_expert_ffn without a caller-supplied workspace.  (The pages have no
  * counterpart; this is an interface convenience.)  For callers that cannot
  * allocate device memory themselves -- e.g. a plugin whose host process owns

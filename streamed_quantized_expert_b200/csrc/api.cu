@@ -291,6 +291,61 @@ moe_status moe_expert_ffn(const uint16_t* x, int32_t T, const moe_layer_desc* d,
                                  x_sorted, pass_begin, pass_len, y_accum, ws, ws_bytes, dev_err, stream, 0);
 }
 
+moe_status moe_route_expert_ffn(const uint16_t* x, const float* logits, int32_t T, const moe_layer_desc* d, float L,
+                                const void* pool, int32_t n_slots, const int32_t* slot_table, int32_t* ids, float* w,
+                                int32_t* offsets, int32_t* pairs, int32_t* active, int32_t* n_active, int32_t* slots,
+                                int32_t* miss, int32_t* n_miss, float* y, void* ws, size_t ws_bytes, int32_t* dev_err,
+                                cudaStream_t stream) {
+  moe_status s = check_desc(d);
+  if (s != MOE_OK) return s;
+  if (T < 1 || n_slots < 0 || !(L >= 0.0f) || L > 1e30f) return MOE_ERR_INVALID;
+  if (!x || !logits || !pool || !slot_table || !ids || !w || !offsets || !pairs || !active || !n_active || !slots ||
+      !miss || !n_miss || !y)
+    return MOE_ERR_INVALID;
+  if (!aligned(pool, 256) || !aligned(x, 16) || !aligned(ws, 256)) return MOE_ERR_INVALID;
+  if (T != 1 || d->E > kRouteMaxExperts || bf16_experts(*d) || !ffn_decode_supported(*d)) return MOE_ERR_UNSUPPORTED;
+  const WsCarve c = carve(*d, T, false);
+  if (!ws || ws_bytes < c.total) return MOE_ERR_CAPACITY;
+  FfnArgs a{};
+  a.x = x;
+  a.T = T;
+  a.E = d->E;
+  a.k = d->k;
+  a.H = d->H;
+  a.I = d->I;
+  a.g = d->group;
+  a.pool = static_cast<const uint8_t*>(pool);
+  a.L = make_layout(*d);
+  a.slot_bytes = a.L.slot_bytes;
+  a.n_slots = n_slots;
+  a.table = slot_table;
+  a.pass_begin = 0;
+  a.pass_len = d->E;
+  a.y = y;
+  a.ctl = static_cast<unsigned*>(ws);
+  char* const scr = static_cast<char*>(ws) + kWsControlBytes + c.tag;
+  a.h = reinterpret_cast<uint16_t*>(scr);
+  a.hpart = reinterpret_cast<float*>(scr + c.hb);
+  a.htag = static_cast<char*>(ws) + kWsControlBytes;
+  a.dev_err = dev_err;
+  a.y_overwrite = 1;
+  a.wait_limit = wait_limit_cycles();
+  a.logits = logits;
+  a.route_L = L;
+  a.r_ids = ids;
+  a.r_w = w;
+  a.r_offsets = offsets;
+  a.r_pairs = pairs;
+  a.r_active = active;
+  a.r_n_active = n_active;
+  a.r_slots = slots;
+  a.r_miss = miss;
+  a.r_n_miss = n_miss;
+  const cudaError_t e = launch_ffn_route_fused(a, *d, device_sms(), stream);
+  if (e == cudaErrorNotSupported) return MOE_ERR_UNSUPPORTED;
+  return cuda_status(e);
+}
+
 moe_status moe_dequant_slot(const void* pool, int32_t slot, const moe_layer_desc* d, float* out_fp32,
                             uint16_t* out_bf16, cudaStream_t stream) {
   moe_status s = check_desc(d);

@@ -155,6 +155,13 @@ moe_status decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc
   uint16_t* xs = ((T >= 32 || d0->bits_gu == 16 || d0->bits_down == 16) && b->x_sorted) ? b->x_sorted : nullptr;
   // one token without shared experts or sorted x: routing, sort and lookup in one launch
   const bool one = T == 1 && ns == 0 && !xs;
+  if (one && !(G && G->n > 0) && moe_cache_resident(cache, layer) >= E0) {
+    // a fully resident layer: the FFN launch routes the token itself (the host needs none of it)
+    const moe_status r = moe_route_expert_ffn(x, logits, T, d0, L, lc->pool, lc->n_slots, lc->table_dev, b->ids,
+                                              b->w, b->offsets, b->pairs, active, n_active, b->slots, miss, n_miss,
+                                              y, b->ws, b->ws_bytes, b->dev_err, stream);
+    if (r != MOE_ERR_UNSUPPORTED) return r;
+  }
   moe_status s = MOE_OK;
   if (one) {
     s = moe_route_sort_lookup(logits, T, d0, L, lc->table_dev, lc->n_slots, b->ids, b->w, b->offsets, b->pairs,

@@ -550,6 +550,22 @@ int ffn_kernel_path(const moe_layer_desc& d, int T, bool has_x_sorted, int num_s
   return 1;
 }
 
+// The fused decode kernel in route mode only (a.logits set): no other path routes.
+cudaError_t launch_ffn_route_fused(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st) {
+  const Layout& L = a.L;
+  a.q_gu = L.gu;
+  a.q_d = L.d;
+  a.tile_gu = L.tile_gu;
+  a.tile_d = L.tile_d;
+  a.rb_gu = L.rb_gu;
+  a.rb_d = L.rb_d;
+  a.ng_gu = L.ng_gu;
+  a.ng_d = L.ng_d;
+  a.nblk_gu = L.nblk_gu;
+  a.nblk_d = L.nblk_d;
+  return launch_ffn_fused(a, d, num_sms, st);
+}
+
 cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st) {
   const Layout& L = a.L;
   if (bf16_experts(d)) {

@@ -65,6 +65,7 @@
 
 #include "common.cuh"
 #include "ffn_common.cuh"
+#include "route_block.cuh"
 #include "kernels.h"
 
 namespace moe {
@@ -128,6 +129,16 @@ __device__ __forceinline__ void load_frag(const uint4* row, int kb, int t4, uint
 // the pass tables are in shared memory, the consumer warps wait on it.
 __device__ __forceinline__ void tables_arrive() { asm volatile("bar.arrive 2, %0;" ::"n"(kFuThreads) : "memory"); }
 __device__ __forceinline__ void tables_sync() { asm volatile("bar.sync 2, %0;" ::"n"(kFuThreads) : "memory"); }
+// Route mode: named barrier 12 is the routing threads' own (warps 0-7, the
+// block routing function's barrier); on named barrier 11 they arrive once the
+// token's ids and weights are in shared memory and the producer waits.
+constexpr int kRouteWarps = 8;
+__device__ __forceinline__ void routed_arrive() {
+  asm volatile("bar.arrive 11, %0;" ::"n"(32 * (kRouteWarps + 1)) : "memory");
+}
+__device__ __forceinline__ void routed_sync() {
+  asm volatile("bar.sync 11, %0;" ::"n"(32 * (kRouteWarps + 1)) : "memory");
+}
 // Named barriers 3 .. 10: one per gate/up warp pair.
 __device__ __forceinline__ void pair_sync(int m) { asm volatile("bar.sync %0, 64;" ::"r"(3 + m) : "memory"); }
 
@@ -151,7 +162,11 @@ __device__ __forceinline__ int fu_item_bound(int c, int n_items, int n_act, cons
   return v > n_items ? n_items : (int)v;
 }
 
-template <int BG, int BD, int BPW, int GS>
+// RT: route mode (moe_route_expert_ffn, one token): consumer warps 0-7 route
+// it with the routing kernels' block function (same ids, order and weights),
+// the producer forms the active list from the routed ids, and CTA 0 writes
+// the routing, the sort and the lookup for the caller.
+template <int BG, int BD, int BPW, int GS, bool RT>
 __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, t4 = lane & 3, g8 = lane >> 2;
@@ -174,6 +189,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
   __shared__ int s_nact, s_i0, s_i1;
   __shared__ unsigned s_tag;
   __shared__ int s_abort;  // a wait of this CTA ran out
+  __shared__ unsigned s_mask[kRouteMaxExperts / 32];  // route mode: the routed experts, as bits
   const int np = a.T * a.k;  // <= kMaxCtaExperts (dense mode)
   uint64_t* htag = reinterpret_cast<uint64_t*>(a.htag);  // [T*k][padded I] tagged h words
 
@@ -181,10 +197,14 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
   // before the dependency wait (the previous kernel may still write it)
   if (warp == kFuConsumers) {
     for (int e = 32 * lane; e < a.E; e += 32 * 32) prefetch_l2(a.table + e);
-    if (lane == 0) prefetch_l2(a.n_active);
-    if (lane < 2) prefetch_l2(a.active + a.pass_begin + 32 * lane);
-    if (lane == 2) prefetch_l2(a.ids);
-    if (lane == 3) prefetch_l2(a.w);
+    if (RT) {  // the token's logits (the routing's input) instead of the routing
+      for (int b = 128 * lane; b < a.E * 4; b += 128 * 32) prefetch_l2(reinterpret_cast<const uint8_t*>(a.logits) + b);
+    } else {
+      if (lane == 0) prefetch_l2(a.n_active);
+      if (lane < 2) prefetch_l2(a.active + a.pass_begin + 32 * lane);
+      if (lane == 2) prefetch_l2(a.ids);
+      if (lane == 3) prefetch_l2(a.w);
+    }
   } else {
     const int nx = a.T * a.H * 2;  // bytes of x
     for (int b = 128 * tid; b < nx; b += 128 * kFuConsumers * 32)
@@ -228,12 +248,17 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
 
   if (warp == kFuConsumers) {
     // ---------------- producer: pass tables, then the CTA's bulk copies ----------------
-    const int na_raw = *a.n_active;
-    int act_v[2];
+    int na_raw = 0;
+    int act_v[2] = {-1, -1};
+    if (!RT) {
+      na_raw = *a.n_active;
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int i = lane + 32 * q;
-      act_v[q] = i < cap ? a.active[a.pass_begin + i] : -1;
+      for (int q = 0; q < 2; ++q) {
+        const int i = lane + 32 * q;
+        act_v[q] = i < cap ? a.active[a.pass_begin + i] : -1;
+      }
+    } else {
+      s_mask[lane] = 0u;
     }
     for (int e0 = 0; e0 < a.E; e0 += 512) {  // the table in one round (two for E > 512)
       int v[16];
@@ -246,6 +271,28 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
       for (int u = 0; u < 16; ++u) {
         const int e = e0 + lane + 32 * u;
         if (e < a.E) s_table[e] = v[u];
+      }
+    }
+    if (RT) {
+      // the routed experts ascending (k distinct of E <= 1024): a bit each, then a warp scan
+      routed_sync();
+      if (lane < np) atomicOr(&s_mask[s_ids[lane] >> 5], 1u << (s_ids[lane] & 31));
+      __syncwarp();
+      const unsigned m = s_mask[lane];
+      int incl = __popc(m);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int pos = incl - __popc(m);
+      for (unsigned b = m; b; b &= b - 1) s_act[pos++] = 32 * lane + __ffs(b) - 1;
+      na_raw = __shfl_sync(0xffffffffu, incl, 31);
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int i = lane + 32 * q;
+        act_v[q] = i < na_raw ? s_act[i] : -1;
       }
     }
     int n_act = na_raw - a.pass_begin;
@@ -348,9 +395,15 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
     cw = atomicAdd(ctr, 1ull);
     if ((unsigned)cw == gridDim.x - 1u) atomicAdd(ctr, kEpochOne - gridDim.x);  // the next launch's epoch
   }
-  for (int p = tid; p < np; p += kFuConsumers * 32) {
-    s_ids[p] = a.ids[p];
-    s_w[p] = a.w[p];
+  if (!RT) {
+    for (int p = tid; p < np; p += kFuConsumers * 32) {
+      s_ids[p] = a.ids[p];
+      s_w[p] = a.w[p];
+    }
+  } else if (warp < kRouteWarps) {
+    // route the token: every CTA the same, bit for bit
+    route_select_token<kRouteMaxExperts / 256, 12>(a.logits, a.E, a.k, a.route_L, a.table, s_ids, s_w, 0, 1.0f);
+    routed_arrive();
   }
   {
     // x' = x 2^-a (exact: a power of two; a by input position within its
@@ -411,6 +464,39 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
   tables_sync();  // the producer's pass tables (and the tag)
   const int n_act = s_nact, i0 = s_i0, i1 = s_i1;
   const unsigned tag = s_tag;
+  if (RT && blockIdx.x == 0) {
+    // the caller's copy of the routing, the sort and the lookup (as
+    // moe_route_sort_lookup writes them): one token, so its k experts are
+    // distinct and pair j of rank r in expert order sits at position r
+    if (tid < np) {
+      const int e = s_ids[tid];
+      int r = 0;
+      for (int q = 0; q < np; ++q) r += s_ids[q] < e;
+      a.r_ids[tid] = e;
+      a.r_w[tid] = s_w[tid];
+      a.r_pairs[r] = tid;
+    }
+    for (int e = tid; e <= a.E; e += kFuConsumers * 32) {
+      int r = 0;
+      for (int q = 0; q < np; ++q) r += s_ids[q] < e;
+      a.r_offsets[e] = r;
+    }
+    if (warp == 1) {
+      const bool in = lane < n_act;
+      const int e = in ? s_act[lane] : -1;
+      const int sl = in ? s_slot[lane] : 0;
+      if (in) {
+        a.r_active[lane] = e;
+        a.r_slots[lane] = sl;
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, in && sl < 0);
+      if (in && sl < 0) a.r_miss[__popc(bal & ((1u << lane) - 1u))] = e;
+      if (lane == 0) {
+        *a.r_n_active = n_act;
+        *a.r_n_miss = __popc(bal);
+      }
+    }
+  }
   // (entry, token) -> flat pair from the routed ids (a token routes to an expert at most once)
   for (int i = tid; i < n_act * kDenseMaxTokens; i += kFuConsumers * 32) {
     const int r = i / kDenseMaxTokens, t = i % kDenseMaxTokens;
@@ -722,10 +808,10 @@ __global__ void __launch_bounds__(kFuThreads, 1) ffn_fused_kernel(const FfnArgs 
 }
 
 // ---------------------------------------------------------------------------
-template <int BG, int BD, int BPW, int GS>
+template <int BG, int BD, int BPW, int GS, bool RT>
 static cudaError_t launch_fused_t(const FfnArgs& a, int grid, size_t smem, cudaStream_t st) {
   static int done[4] = {0, 0, 0, 0};
-  const void* kern = reinterpret_cast<const void*>(ffn_fused_kernel<BG, BD, BPW, GS>);
+  const void* kern = reinterpret_cast<const void*>(ffn_fused_kernel<BG, BD, BPW, GS, RT>);
   cudaError_t e = ensure_smem_attr(kern, done);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -758,9 +844,13 @@ static cudaError_t launch_fused_t(const FfnArgs& a, int grid, size_t smem, cudaS
 
 template <int BG, int BD, int BPW>
 static cudaError_t fused_gs(const FfnArgs& a, int gs, int grid, size_t smem, cudaStream_t st) {
-  if (gs == 2) return launch_fused_t<BG, BD, BPW, 2>(a, grid, smem, st);
-  if (gs == 4) return launch_fused_t<BG, BD, BPW, 4>(a, grid, smem, st);
-  return launch_fused_t<BG, BD, BPW, 8>(a, grid, smem, st);
+  const bool rt = a.logits != nullptr;
+  if (gs == 2) return rt ? launch_fused_t<BG, BD, BPW, 2, true>(a, grid, smem, st)
+                         : launch_fused_t<BG, BD, BPW, 2, false>(a, grid, smem, st);
+  if (gs == 4) return rt ? launch_fused_t<BG, BD, BPW, 4, true>(a, grid, smem, st)
+                         : launch_fused_t<BG, BD, BPW, 4, false>(a, grid, smem, st);
+  return rt ? launch_fused_t<BG, BD, BPW, 8, true>(a, grid, smem, st)
+            : launch_fused_t<BG, BD, BPW, 8, false>(a, grid, smem, st);
 }
 
 template <int BG>
@@ -821,6 +911,12 @@ bool ffn_fused_plan(FfnArgs& a, const moe_layer_desc& d, int num_sms, size_t& sm
 cudaError_t launch_ffn_fused(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st) {
   size_t smem = 0;
   if (!ffn_fused_plan(a, d, num_sms, smem)) return cudaErrorNotSupported;
+  // route mode: one token, one pass over every expert
+  if (a.logits != nullptr &&
+      (a.T != 1 || d.E > kRouteMaxExperts || d.k > 32 || a.pass_begin != 0 || a.pass_len < d.E || !a.r_ids ||
+       !a.r_w || !a.r_offsets || !a.r_pairs || !a.r_active || !a.r_n_active || !a.r_slots || !a.r_miss ||
+       !a.r_n_miss))
+    return cudaErrorNotSupported;
   const int grid = num_sms;
   const int gs = d.group / 16;
   if (d.bits_gu == 3) return fused_bd<3>(a, d.bits_down, gs, grid, smem, st);

@@ -49,7 +49,24 @@ struct FfnArgs {
   int xh_stage_bytes;  // fused kernel: shared region for x' and its sums, then (at h_stage_off) h
   int h_stage_off;
   long long wait_limit;  // clock-cycle limit of every bounded device wait (wait_limit_cycles())
+  // route mode of the fused decode kernel (moe_route_expert_ffn, one token):
+  // the kernel routes it from logits [E] itself (ids / w / offsets / pairs /
+  // active / n_active above are then unused) and its CTA 0 writes the
+  // routing, the sort and the slot lookup to the r_ buffers
+  const float* logits;
+  float route_L;
+  int32_t* r_ids;
+  float* r_w;
+  int32_t* r_offsets;
+  int32_t* r_pairs;
+  int32_t* r_active;
+  int32_t* r_n_active;
+  int32_t* r_slots;
+  int32_t* r_miss;
+  int32_t* r_n_miss;
 };
+// experts a layer may have for the fused decode kernel to route its token itself
+constexpr int kRouteMaxExperts = 1024;
 
 // Launch with programmatic stream serialization, so the kernel's CTAs can be
 // scheduled while the previous kernel in the stream drains; every kernel
@@ -92,6 +109,7 @@ cudaError_t launch_dequant_slot(const uint8_t* slot, const moe_layer_desc& d, co
                                 uint16_t* out16, cudaStream_t st);
 bool ffn_decode_supported(const moe_layer_desc& d);
 cudaError_t launch_ffn_decode(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st);
+cudaError_t launch_ffn_route_fused(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st);
 cudaError_t launch_ffn_fused(FfnArgs a, const moe_layer_desc& d, int num_sms, cudaStream_t st);
 cudaError_t launch_ffn_prefill_tc(const FfnArgs& a, const moe_layer_desc& d, int num_sms, cudaStream_t st);
 bool ffn_fused_plan(FfnArgs& a, const moe_layer_desc& d, int num_sms, size_t& smem);

@@ -27,7 +27,7 @@ ABI_SYMBOLS = [
     "moe_expert_ffn_noalloc", "moe_noalloc_scratch_bytes", "moe_cache_resident", "moe_decode_layer",
     "moe_last_cuda_error", "moe_ffn_kernel_path", "moe_set_wait_limit_cycles", "moe_route_shared",
     "moe_router_logits", "moe_cache_reserve", "moe_cache_commit", "moe_prefetch_create", "moe_prefetch_destroy",
-    "moe_prefetch_stats", "moe_decode_layer_ahead", "moe_route_sort_lookup",
+    "moe_prefetch_stats", "moe_decode_layer_ahead", "moe_route_sort_lookup", "moe_route_expert_ffn",
 ]
 
 
@@ -93,6 +93,8 @@ def lib():
             "moe_sort": (C.c_int, [P, P, i32, D, P, P, P, P, P, P, sz, P]),
             "moe_slot_lookup": (C.c_int, [P, P, P, i32, i32, i32, P, P, P, P, P]),
             "moe_route_sort_lookup": (C.c_int, [P, i32, D, f32, P, i32, P, P, P, P, P, P, P, P, P, P, P]),
+            "moe_route_expert_ffn": (C.c_int, [P, P, i32, D, f32, P, i32, P, P, P, P, P, P, P, P, P, P, P, P, sz, P,
+                                               P]),
             "moe_install_slots": (C.c_int, [P, sz, i32, P, P, i32, P, P]),
             "moe_expert_ffn": (C.c_int, [P, i32, D, P, i32, P, P, P, P, P, P, P, P, i32, i32, P, P, sz, P, P]),
             "moe_expert_ffn_noalloc": (C.c_int, [P, i32, D, P, i32, P, P, P, P, P, P, P, i32, i32, P, P, P]),
@@ -226,6 +228,18 @@ def moe_route_sort_lookup(logits, T, d, L, slot_table, n_slots, ids, w, offsets,
                                     _ptr(ids), _ptr(w), _ptr(offsets), _ptr(pairs), _ptr(active), _ptr(n_active),
                                     _ptr(slots), _ptr(miss), _ptr(n_miss), _ptr(dev_err), _stream(stream)),
         "moe_route_sort_lookup")
+
+
+def moe_route_expert_ffn(x, logits, T, d, L, pool, n_slots, slot_table, ids, w, offsets, pairs, active, n_active,
+                         slots, miss, n_miss, y, ws, ws_bytes, dev_err, stream=None) -> None:
+    """Routing, sort, lookup and FFN of one token of a resident layer in one
+    launch (T must be 1): the stage outputs as moe_route_sort_lookup writes
+    them, and y (overwritten)."""
+    _ck(lib().moe_route_expert_ffn(_ptr(x), _ptr(logits), int(T), C.byref(d), float(L), _ptr(pool), int(n_slots),
+                                   _ptr(slot_table), _ptr(ids), _ptr(w), _ptr(offsets), _ptr(pairs), _ptr(active),
+                                   _ptr(n_active), _ptr(slots), _ptr(miss), _ptr(n_miss), _ptr(y), _ptr(ws),
+                                   int(ws_bytes), _ptr(dev_err), _stream(stream)),
+        "moe_route_expert_ffn")
 
 
 def moe_slot_lookup(slot_table, active, n_active, pass_begin, pass_len, n_slots, slots, miss, n_miss, dev_err,

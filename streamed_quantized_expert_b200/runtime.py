@@ -261,10 +261,12 @@ class Streamer:
             return 2 * -(-min(pass_len, self.Ew) // 64) + 1
         return 3
 
-    def _decode_launches(self, layer: int, T: int, full: bool, n_installed: int) -> int:
+    def _decode_launches(self, layer: int, T: int, full: bool, n_installed: int, guessing: bool = False) -> int:
         d = self.layers[layer].desc
         tc = T >= 32 or d.bits_gu == 16 or d.bits_down == 16
         if T == 1 and not self.ns and not tc:
+            if full and not guessing and d.E <= 1024 and self._ffn_launches(layer, T, self.Ew) == 1:
+                return 1  # moe_route_expert_ffn: every stage in the FFN launch
             n = 1  # moe_route_sort_lookup
         else:
             n = 1 + (1 if T * self.kw <= 1024 else 3) + (1 if tc else 0) + (0 if full else 1)  # route, sort, lookup
@@ -298,7 +300,7 @@ class Streamer:
         if n:
             self.installs += n
             self.installed_bytes += n * self.class_bytes[self.layer_class[layer]]
-        self.launches += self._decode_launches(layer, T, full, n) + len(g)
+        self.launches += self._decode_launches(layer, T, full, n, guessing=bool(g)) + len(g)
         return y
 
     def decode_layer_steps(self, layer: int, x, logits, T: int, L: float = 0.0, y=None):
