@@ -307,8 +307,16 @@ def stage_graph_times(st, cfg, snaps, logits, Lsub, reps, device):
         ops.moe_slot_lookup(st.table_dev[l], sn["meta"][2:2 + E], sn["meta"][0:1], 0, E, st.n_slots_of(l), slots,
                             meta[2 + E:], meta[1:2], st.dev_err, cs)
 
+    def route_sort_lookup(l, cs):  # the three in one launch (one token, no shared experts)
+        ops.moe_route_sort_lookup(logits[l], T, st.layers[l].desc, Lsub, st.table_dev[l], st.n_slots_of(l), ids, w,
+                                  offsets, pairs, meta[2:2 + E], meta[0:1], slots, meta[2 + E:], meta[1:2],
+                                  st.dev_err, cs)
+
     out = {}
-    for name, fn in (("route", route), ("sort", sort), ("lookup", lookup)):
+    stages = [("route", route), ("sort", sort), ("lookup", lookup)]
+    if T == 1 and not st.ns:
+        stages.append(("route_sort_lookup", route_sort_lookup))
+    for name, fn in stages:
         g_ = torch.cuda.CUDAGraph()
         cap = torch.cuda.Stream(device)
         torch.cuda.synchronize(device)
@@ -329,7 +337,8 @@ def stage_graph_times(st, cfg, snaps, logits, Lsub, reps, device):
         out[name + "_us"] = round(1e3 * e0.elapsed_time(e1) / (reps * n_layers), 2)
         del g_
     out["how"] = ("per stage, a CUDA graph of the %d layers' calls (one decode step's inputs), replayed %d times, "
-                  "CUDA events" % (n_layers, reps))
+                  "CUDA events; route_sort_lookup: the three stages of one token in one launch, as the decode "
+                  "driver runs them" % (n_layers, reps))
     return out
 
 
