@@ -96,7 +96,7 @@ CONFIGS = {
                      "(25% resident), L = 0.15, misses installed from pinned host"),
 }
 # token counts of a configuration's batch sweep (besides its own T), FFN-only
-SWEEP = {"coder": (1, 8, 32)}
+SWEEP = {"coder": (1, 8, 16, 32)}
 # per-layer widths and the substitution strength of the decode configurations (default: uniform, L = 0)
 DECODE_EXTRA = {"decode_mixed": {"bits": lambda l: (4, 6) if l % 4 == 0 else (4, 4), "L": 0.15},
                 "decode_shared": {"n_shared": 1},
@@ -681,7 +681,7 @@ def run_ours(args, rank, world, local_rank):
             st.decode_layer(l, x[steps_total, l], logits[steps_total, l], T, Lsub)
             snaps.append({"x": x[steps_total, l], "ids": st.ids.clone(), "w": st.w.clone(),
                           "offsets": st.offsets.clone(), "pairs": st.pairs.clone(), "meta": st.meta.clone(),
-                          **({"xs": st.x_sorted[:T * st.kw].clone()} if T >= 32 else {})})
+                          **({"xs": st.x_sorted[:T * st.kw].clone()} if st.uses_tc(l, T) else {})})
         torch.cuda.synchronize(device)
         n_unique = sum(int(sn["meta"][0].item()) for sn in snaps) / n_layers
         ffn_us = ffn_graph_time(st, cfg, snaps, args.ffn_reps, device)
@@ -694,7 +694,7 @@ def run_ours(args, rank, world, local_rank):
                 st.decode_layer(l, x[steps_total, l, :T2], logits[steps_total, l, :T2], T2, Lsub)
                 sn2.append({"x": x[steps_total, l, :T2], "ids": st.ids.clone(), "w": st.w.clone(),
                             "offsets": st.offsets.clone(), "pairs": st.pairs.clone(), "meta": st.meta.clone(),
-                            **({"xs": st.x_sorted[:T2 * st.kw].clone()} if T2 >= 32 else {})})
+                            **({"xs": st.x_sorted[:T2 * st.kw].clone()} if st.uses_tc(l, T2) else {})})
             torch.cuda.synchronize(device)
             us2 = ffn_graph_time(st, cfg, sn2, args.ffn_reps, device, T=T2)
             sweep.append((T2, us2, sn2))
@@ -800,7 +800,7 @@ def run_ours(args, rank, world, local_rank):
                      "kernel": ("ffn_fused_kernel (one launch per layer: every CTA gate/up + SwiGLU items, then the "
                                 "first H/16 CTAs a down + combine tile, over launch-tagged h words)" if T <= 8 and T * k <= 64 else
                                 "pf_gemm_kernel (tcgen05 grouped GEMM: gate/up + SwiGLU, down) + combine, per layer"
-                                if T >= 32 else
+                                if st.uses_tc(0, T) else
                                 "moe_expert_ffn (gate/up+SwiGLU kernel + down kernel), per layer"),
                      "bytes_per_launch": int(ffn_bytes), "peak_kind": peak_kind},
         **({"batch_sweep": [
@@ -808,7 +808,7 @@ def run_ours(args, rank, world, local_rank):
              "hbm_gbs": round(b2 / (us2 * 1e-6) / 1e9, 1), "frac": round(b2 / (us2 * 1e-6) / 1e9 / hbm_peak, 4),
              "unique_experts_per_layer": round(nu2, 1),
              "kernel_path": ["fused decode", "GEMV", "tcgen05 grouped GEMM"][
-                 _ops.moe_ffn_kernel_path(st.layers[0].desc, T2, T2 >= 32)]}
+                 _ops.moe_ffn_kernel_path(st.layers[0].desc, T2, st.uses_tc(0, T2))]}
             for T2, us2, nu2, b2 in [
                 (T2, us2, sum(int(sn["meta"][0].item()) for sn in sn2) / n_layers,
                  sum(int(sn["meta"][0].item()) * slot_bytes[l] for l, sn in enumerate(sn2)) / n_layers

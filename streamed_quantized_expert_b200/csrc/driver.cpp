@@ -150,9 +150,10 @@ moe_status decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc
   int32_t* n_miss = b->meta + 1;
   int32_t* active = b->meta + 2;
   int32_t* miss = b->meta + 2 + E;
-  // from 32 tokens (BF16 experts: always) the FFN runs on the tensor-core grouped GEMM, which reads x
-  // sorted by expert
-  uint16_t* xs = ((T >= 32 || d0->bits_gu == 16 || d0->bits_down == 16) && b->x_sorted) ? b->x_sorted : nullptr;
+  // where the FFN runs on the tensor-core grouped GEMM (above the fused decode kernel's range; BF16
+  // experts always), it reads x sorted by expert
+  uint16_t* xs =
+      (b->x_sorted && moe_ffn_kernel_path(d, T, 1) == MOE_PATH_TC_PREFILL) ? b->x_sorted : nullptr;
   // one token without shared experts or sorted x: routing, sort and lookup in one launch
   const bool one = T == 1 && ns == 0 && !xs;
   if (one && !(G && G->n > 0) && moe_cache_resident(cache, layer) >= E0) {

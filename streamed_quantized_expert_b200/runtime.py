@@ -238,7 +238,7 @@ class Streamer:
             ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             ev[0].record(self.stream)
         self.launches += 2 if T <= 64 else 3
-        tc = T >= 32 or d.bits_gu == 16 or d.bits_down == 16
+        tc = self.uses_tc(layer, T)
         ops.moe_expert_ffn(x, T, d, self.pool_of(layer), self.n_slots_of(layer), self.table_dev[layer], self.ids,
                            self.w, self.offsets, self.pairs, self._active(), self._n_active(),
                            self.x_sorted if tc else None, pass_begin, pass_len, y, self.ws, self.ws_bytes,
@@ -247,10 +247,19 @@ class Streamer:
             ev[1].record(self.stream)
             self.ffn_events.append(ev)
 
+    def uses_tc(self, layer: int, T: int) -> bool:
+        """Whether the layer's FFN over T tokens runs on the tensor-core grouped
+        GEMM (which reads x sorted by expert) when given sorted x."""
+        key = (layer, T, "tc")
+        v = self._paths.get(key)
+        if v is None:
+            v = self._paths[key] = ops.moe_ffn_kernel_path(self.wdesc[layer], T, True) == ops.MOE_PATH_TC_PREFILL
+        return v
+
     def _ffn_launches(self, layer: int, T: int, pass_len: int) -> int:
         """Kernels one moe_expert_ffn call over pass_len experts launches."""
         d = self.wdesc[layer]
-        tc = T >= 32 or d.bits_gu == 16 or d.bits_down == 16
+        tc = self.uses_tc(layer, T)
         key = (layer, T, tc)
         path = self._paths.get(key)
         if path is None:
@@ -263,7 +272,7 @@ class Streamer:
 
     def _decode_launches(self, layer: int, T: int, full: bool, n_installed: int, guessing: bool = False) -> int:
         d = self.layers[layer].desc
-        tc = T >= 32 or d.bits_gu == 16 or d.bits_down == 16
+        tc = self.uses_tc(layer, T)
         if T == 1 and not self.ns and not tc:
             if full and not guessing and d.E <= 1024 and self._ffn_launches(layer, T, self.Ew) == 1:
                 return 1  # moe_route_expert_ffn: every stage in the FFN launch
@@ -308,7 +317,7 @@ class Streamer:
         y = self.y[:T] if y is None else y
         s = self.stream
         d0 = self.layers[layer].desc
-        self.route_sort(layer, x, logits, T, L, want_sorted_x=T >= 32 or d0.bits_gu == 16 or d0.bits_down == 16)
+        self.route_sort(layer, x, logits, T, L, want_sorted_x=self.uses_tc(layer, T))
         if not self.fully_resident(layer):
             d = self.layers[layer].desc
             ops.moe_slot_lookup(self.table_dev[layer], self._active(), self._n_active(), 0, self.Ew,
@@ -331,7 +340,7 @@ class Streamer:
         y = self.y[:T] if y is None else y
         s = self.stream
         d0 = self.layers[layer].desc
-        self.route_sort(layer, x, logits, T, 0.0, want_sorted_x=T >= 32 or d0.bits_gu == 16 or d0.bits_down == 16)
+        self.route_sort(layer, x, logits, T, 0.0, want_sorted_x=self.uses_tc(layer, T))
         with torch.cuda.stream(s):
             y.zero_()
             self.meta_pin.copy_(self.meta, non_blocking=True)

@@ -69,7 +69,7 @@ def test_mixed_class_prefill_chunk_every_row(orc, bd, layer):
     assert_close(y, oracle_rows_parallel(orc, x, s.geom, ids, w, s.slots_np), TOL, what=f"prefill T=4096 4/{bd}")
 
 
-@pytest.mark.parametrize("T", [32, 64])
+@pytest.mark.parametrize("T", [12, 32, 64])
 @pytest.mark.parametrize("sorted_x", [True, False])
 def test_coder_batched_decode_every_row(orc, T, sorted_x):
     E, k, H, I, g = 128, 8, 2048, 768, 64
