@@ -246,7 +246,8 @@ moe_status moe_route_sort_lookup(const float* logits, int32_t T, const moe_layer
  *   slot_table device int32 [E]
  *   ids, w     from moe_route; offsets, pairs, active, n_active from moe_sort
  *   x_sorted   from moe_sort, or NULL (needed by the tensor-core grouped GEMM,
- *              which runs from 9 tokens when it is given; else unused)
+ *              which runs wherever the fused decode kernel does not
+ *              apply when it is given; else unused)
  *   pass_begin, pass_len  which active experts this call runs
  *   y_accum    device fp32 [T, H]; the pass's expert outputs are ADDED:
  *              y_t += sum over the pass's pairs (t, j) of w[t,j] * o_{t,j}.
@@ -294,9 +295,9 @@ moe_status moe_route_expert_ffn(const uint16_t* x, const float* logits, int32_t 
  * (1 MiB) inside the library, held by every GPU that loads it until the
  * process exits.  Same arguments and results as moe_expert_ffn, except:
  *   - T must be <= 64 and the workspace of a call without x_sorted must fit
- *     1 MiB (that is moe_workspace_bytes(d, T) below 9 tokens; from 9 on,
- *     moe_workspace_bytes also counts the tensor-core path's per-pair output
- *     buffer, which this call never uses), else MOE_ERR_CAPACITY is returned
+ *     1 MiB (moe_workspace_bytes(d, T) less the tensor-core path's per-pair
+ *     output buffer, which this call never uses), else MOE_ERR_CAPACITY is
+ *     returned
  *     and nothing is launched;
  *   - x_sorted is not taken (the decode kernels do not use it);
  *   - the first call on a device looks up the array's device address (with
@@ -365,8 +366,9 @@ const char* moe_status_string(moe_status s);
  *                          (T <= 8, T*k <= 64)
  *   MOE_PATH_GEMV          gate/up + SwiGLU kernel, down kernel (+ combine
  *                          kernel for T > 64): tensor-core GEMV (mma.sync)
- *   MOE_PATH_TC_PREFILL    tcgen05/TMEM grouped GEMM fed by TMA (T >= 9,
- *                          x_sorted given, H and I multiples of 128): prefill
+ *   MOE_PATH_TC_PREFILL    tcgen05/TMEM grouped GEMM fed by TMA (beyond the
+ *                          fused decode kernel's range, x_sorted given, H and
+ *                          I multiples of 128): prefill
  *                          chunks and batched decode; a layer with a 16-bit
  *                          (BF16) projection at every T
  * or -1 if d is invalid, T < 1, or a BF16 layer has no path (no x_sorted).
@@ -456,7 +458,7 @@ typedef struct {
   void* ws;            /* device workspace */
   size_t ws_bytes;     /* >= moe_workspace_bytes(desc, max_tokens) */
   int32_t max_tokens;
-  uint16_t* x_sorted;  /* device fp16 [max_tokens*k, H], or NULL: from 9 tokens the layer
+  uint16_t* x_sorted;  /* device fp16 [max_tokens*k, H], or NULL: beyond the fused range the layer
                           sorts x into it and its FFN runs on the tensor-core grouped GEMM */
 } moe_step_buffers;
 
@@ -479,7 +481,7 @@ typedef struct {
 /* One decode layer, T <= 64 tokens (RFC "How the prototype works": each layer
  * copies its routing to the host once; misses cost one host-to-device copy
  * per expert; a fully resident layer never synchronises with the host):
- *   moe_route (L) -> moe_sort (sorting x into b->x_sorted when T >= 9 and
+ *   moe_route (L) -> moe_sort (sorting x into b->x_sorted beyond the fused range and
  *   b->x_sorted is given) -> if the layer is not fully resident in `cache`:
  *   moe_slot_lookup, copy n_active/active to meta_host, synchronise `stream`,
  *   moe_cache_step, moe_install_slots on `side`, upload the table, record

@@ -10,9 +10,9 @@
 namespace moe {
 
 constexpr int kFusedMaxTokens = 64;  // decode down kernel combines in shared memory up to this T
-constexpr int kTcMinTokens = 9;  // from this T on (with x_sorted) the FFN runs on the tcgen05 grouped GEMM:
-                                 // every T above the fused decode kernel's range (it beats the GEMV kernels
-                                 // from 9 tokens on, measured at the Coder-like shapes)
+constexpr int kTcMinTokens = 1;  // with x_sorted the FFN runs on the tcgen05 grouped GEMM wherever the fused
+                                 // decode kernel does not apply (it matches or beats the GEMV kernels at every
+                                 // such T measured: 7 to 32 tokens, Flash- and Coder-like shapes)
 constexpr int kMaxShared = 8;  // shared experts per layer (moe_route_shared)
 // BF16 experts (a 16-bit projection): only the tensor-core grouped GEMM runs them
 inline bool bf16_experts(const moe_layer_desc& d) { return d.bits_gu == 16 || d.bits_down == 16; }

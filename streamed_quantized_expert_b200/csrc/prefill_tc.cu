@@ -1,6 +1,7 @@
 // Expert FFN on the 5th-generation tensor cores (tcgen05 + TMEM), fed by TMA:
 // the grouped GEMM of a pass's experts over their sorted tokens, for prefill
-// chunks and batched decode (from 9 tokens, when x sorted by expert is given).
+// chunks and batched decode (above the fused decode kernel's range, when x sorted
+// by expert is given).
 //
 // Two launches per pass of at most 64 experts (a longer pass runs as several),
 // one persistent CTA per SM, each looping over tiles of (expert, 128 weight

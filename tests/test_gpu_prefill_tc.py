@@ -1,5 +1,6 @@
 """GPU vs oracle for the expert FFN on the tcgen05 grouped GEMM (prefill
-chunks and batched decode, from 32 tokens with sorted activations): dequantised weight tiles in the
+chunks and batched decode, wherever the fused decode kernel does not apply, with sorted activations):
+dequantised weight tiles in the
 128-byte swizzled layout, token tiles by TMA, fp32 accumulators in TMEM.
 Within 2e-2 of max(|ref|, row rms) elementwise on sampled token rows (the
 oracle computes them one by one), and equal to the GEMV path within the
@@ -54,6 +55,17 @@ def test_coder_shape_prefill(orc):
     # 128 experts, top-8, H 2048, I 768, 4-bit g64 (I = 6 blocks of 128)
     s, x, ids, w = _case(orc, 128, 8, 2048, 768, 64, 4, 4, 512, R=6, seed=13)
     _check(orc, s, x, ids, w, 512, [(0, 64), (64, 64)])
+
+
+@pytest.mark.parametrize("T", [7, 8, 9])
+def test_few_tokens_past_the_fused_range(orc, T):
+    # top-10 at 7 and 8 tokens (70 and 80 pairs) is past the fused decode kernel: every row, and the
+    # same values as the GEMV kernels within the tolerance
+    s, x, ids, w = _case(orc, 64, 10, 256, 128, 64, 3, 3, T, R=5, seed=30 + T)
+    y = _check(orc, s, x, ids, w, T, ntok=T)
+    y2, err = s.gpu(x, ids, w, T, sorted_x=False)
+    assert err == 0
+    assert_close(y, y2, TOL)
 
 
 @pytest.mark.parametrize("g,bg,bd", [(32, 3, 4), (128, 6, 3), (64, 4, 4)])
