@@ -15,11 +15,13 @@
 // steps by 16, where it would leave most of a 128-row M tile empty).
 //
 // Warp roles (832 threads):
-//   0-15  dequant: warp w = (K quarter w / 4, TMEM lane quadrant w % 4), lane
-//         = weight row; unpack its row's codes of a 128-input block (landed by
-//         TMA), w = fma(scale, q, bias) in fp16x2 with one rounding, and store
-//         the quarter's 16 fp16 pairs (inputs 32 q .. 32 q + 31) to the A
-//         operand in TMEM with one tcgen05.st (lane = row, column = input / 2);
+//   0-15  dequant: warp w = (group w / 4, TMEM lane quadrant w % 4), lane =
+//         weight row; for quantized codes the four warps of a group take whole
+//         rows of every fourth 128-input block (landed by TMA): unpack the
+//         row's codes once, w = fma(scale, q, bias) in fp16x2 with one
+//         rounding, and store its 64 fp16 pairs to the A operand in TMEM with
+//         four tcgen05.st (lane = row, column = input / 2); BF16 rows: warp w
+//         converts K quarter w / 4 of its rows of every block;
 //   16-23 epilogue: TMEM -> registers (warp i reads TMEM lanes 32 (i % 4)..;
 //         the two warps of a quadrant take alternate 16-column chunks);
 //   24    producer: TMA loads of codes, (scale, bias) words and token rows;
@@ -66,6 +68,7 @@ constexpr int kPfThreads = (kPfMmaWarp + 1) * 32;
 constexpr int kPfTmemCols = 512;  // two accumulators of NB fp32 columns, then the A buffers
 constexpr int kPfAcols = 64;       // one A buffer: 128 inputs as fp16 pairs, 128 lanes = rows
 static_assert(2 * kPfBN + kPfABufs * kPfAcols <= kPfTmemCols, "TMEM columns");
+static_assert(kPfABufs == 4 && kPfDqWarps == 16, "dequant warps: one group of four (one per TMEM lane quadrant) per A buffer");
 // load stages (codes + scale/bias + token rows of NB rows) that fit the
 // shared memory: a tile of at most 64 tokens has half the token bytes per
 // stage, so its ring is deeper (the ring, not the arithmetic, paces the
@@ -202,46 +205,6 @@ __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, volatile
   }
 }
 
-// K quarter CQ (inputs 32 CQ .. 32 CQ + 31) of weight row r (0..127 of the
-// tile) for one 128-input block -> 16 fp16 pairs, stored at TMEM columns
-// 16 CQ .. 16 CQ + 15 of this thread's lane (ta: the warp's lanes, A buffer
-// column 0).  Codes: the tile's 16 8-row groups, each 4 units x 8 rows x B
-// words (unit t of row rr at word (8 t + sigma) B); scale/bias: per 16-row
-// tile, GPB groups of 16 words.  Pair i = 2 s + h' of unit t holds inputs
-// 16 s + 2 t + 8 h' (+1), i.e. TMEM column 8 s + 4 h' + t: the quarter's
-// pairs are i = 4 CQ + m (m = 0..3) at local column 4 m + t.
-template <int B, int GPB, int CQ>
-__device__ __forceinline__ void pf_dequant_quarter(const uint8_t* cs, const uint32_t* sbs, uint32_t ta, int r) {
-  const int g8 = r >> 3, rr = r & 7;
-  constexpr int GI = (CQ * GPB) / 4;  // the quarter's (single) group within the block
-  const uint32_t word = sbs[(r >> 4) * 16 * GPB + GI * 16 + (r & 15)];
-  // bf16 scale and bias -> fp16 (exact for normal fp16 magnitudes); codes
-  // unpacked onto the fp16 magic 1024: q = p - 1024 exactly, then one fp16
-  // rounding of s * q + b
-  const float sf = bf16_lo(word), bf = bf16_hi(word);
-  const __half2 sc = __half2half2(__float2half_rn(sf));
-  const __half2 sc8 = __half2half2(__float2half_rn(sf * 0.125f));
-  const __half2 bi = __half2half2(__float2half_rn(bf));
-  const uint32_t m = kMagic16;
-  const __half2 m1024 = *reinterpret_cast<const __half2*>(&m);
-  uint32_t out[16];
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    uint32_t w[B], p[16];
-    load_unit<B>(cs + (g8 * 32 + 8 * t + unit_sigma<B>(t, rr)) * 4 * B, w);
-    unpack_unit<B, kMagic16>(w, p);
-#pragma unroll
-    for (int mm = 0; mm < 4; ++mm) {
-      const int i = 4 * CQ + mm;
-      const __half2 scale = PairShift<B>::a(i) == 3 ? sc8 : sc;
-      const __half2 q = __hsub2(*reinterpret_cast<const __half2*>(&p[i]), m1024);
-      const __half2 v = __hfma2(scale, q, bi);
-      out[4 * mm + t] = *reinterpret_cast<const uint32_t*>(&v);
-    }
-  }
-  tmem_st16(ta + 16 * CQ, out);
-}
-
 // BF16 experts: K quarter cq of row r from the stage's two 64-input halves
 // (128 rows x 128 bytes each, 128-byte swizzle: 16-byte chunk c of row r sits
 // at chunk c ^ (r % 8)), converted to fp16 pairs (pair index = TMEM column).
@@ -260,12 +223,49 @@ __device__ __forceinline__ void pf_bf16_quarter(int cq, const uint8_t* cs, uint3
   tmem_st16(ta + 16 * cq, out);
 }
 
+// The whole 128-input block of weight row r (0..127 of the tile) -> 64 fp16
+// pairs at TMEM columns 0..63 of this thread's lane (ta: the warp's lanes, A
+// buffer column 0).  Codes: the tile's 16 8-row groups, each 4 units x 8 rows
+// x B words (unit t of row rr at word (8 t + sigma) B), loaded once;
+// scale/bias: per 16-row tile, GPB groups of 16 words.  Pair i = 2 s + h' of
+// unit t holds inputs 16 s + 2 t + 8 h' (+1), i.e. TMEM column 8 s + 4 h' + t:
+// K quarter cq (inputs 32 cq .. 32 cq + 31, a single group) is pairs
+// i = 4 cq + m of every unit, at columns 16 cq + 4 m + t.  Each weight is
+// scale * q + bias in fp16 with one rounding: bf16 scale and bias -> fp16
+// (exact for normal fp16 magnitudes), codes unpacked onto the fp16 magic 1024
+// so that q = p - 1024 exactly.
 template <int B, int GPB>
-__device__ __forceinline__ void pf_dequant(int cq, const uint8_t* cs, const uint32_t* sbs, uint32_t ta, int r) {
-  if (cq == 0) pf_dequant_quarter<B, GPB, 0>(cs, sbs, ta, r);
-  else if (cq == 1) pf_dequant_quarter<B, GPB, 1>(cs, sbs, ta, r);
-  else if (cq == 2) pf_dequant_quarter<B, GPB, 2>(cs, sbs, ta, r);
-  else pf_dequant_quarter<B, GPB, 3>(cs, sbs, ta, r);
+__device__ __forceinline__ void pf_dequant_row(const uint8_t* cs, const uint32_t* sbs, uint32_t ta, int r) {
+  const int g8 = r >> 3, rr = r & 7;
+  uint32_t w[4][B];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) load_unit<B>(cs + (g8 * 32 + 8 * t + unit_sigma<B>(t, rr)) * 4 * B, w[t]);
+  const uint32_t m = kMagic16;
+  const __half2 m1024 = *reinterpret_cast<const __half2*>(&m);
+#pragma unroll
+  for (int cq = 0; cq < 4; ++cq) {
+    const int gi = (cq * GPB) / 4;  // the quarter's (single) group within the block
+    const uint32_t word = sbs[(r >> 4) * 16 * GPB + gi * 16 + (r & 15)];
+    const float sf = bf16_lo(word), bf = bf16_hi(word);
+    const __half2 sc = __half2half2(__float2half_rn(sf));
+    const __half2 sc8 = __half2half2(__float2half_rn(sf * 0.125f));
+    const __half2 bi = __half2half2(__float2half_rn(bf));
+    uint32_t out[16];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      uint32_t p[16];
+      unpack_unit<B, kMagic16>(w[t], p);
+#pragma unroll
+      for (int mm = 0; mm < 4; ++mm) {
+        const int i = 4 * cq + mm;
+        const __half2 scale = PairShift<B>::a(i) == 3 ? sc8 : sc;
+        const __half2 q = __hsub2(*reinterpret_cast<const __half2*>(&p[i]), m1024);
+        const __half2 v = __hfma2(scale, q, bi);
+        out[4 * mm + t] = *reinterpret_cast<const uint32_t*>(&v);
+      }
+    }
+    tmem_st16(ta + 16 * cq, out);
+  }
 }
 
 struct PfTile {
@@ -308,7 +308,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < kPfABufs; ++b) {
-      mbar_init(&afull[b], kPfDqWarps);
+      // quantized codes: the four warps of the buffer's block group; BF16 rows: all sixteen
+      mbar_init(&afull[b], B == 16 ? kPfDqWarps : kPfDqWarps / kPfABufs);
       mbar_init(&aempty[b], 1);
     }
     for (int c = 0; c < 2; ++c) {
@@ -506,12 +507,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
   } else if (warp < kPfDqWarps) {
     // ---------------- dequant ----------------
-    const int q = warp & 3, cq = warp >> 2, r = 32 * q + lane;  // TMEM lane quadrant, K quarter, weight row
-    int s = 0, ab = 0;
-    uint32_t ph = 0, pa = 0;
+    // Quantized codes: warp = (block group sel, TMEM lane quadrant q), lane =
+    // weight row; the four warps of group sel dequantise whole rows of every
+    // fourth block of the CTA's block sequence (block b when b % 4 == sel)
+    // into A buffer sel, so a row's code words are loaded once and four blocks
+    // are in flight.  BF16 rows (nothing to unpack, nothing loaded twice):
+    // every warp takes K quarter sel of its quadrant's rows of every block.
+    constexpr bool kRowGroups = B != 16;
+    const int q = warp & 3, sel = warp >> 2, r = 32 * q + lane;
+    int b = 0;  // position in the CTA's block sequence
     for (int t = blockIdx.x; t < ntiles && !s_abort; t += gridDim.x) {
       bool ok = true;
-      for (int kb = 0; kb < a.nkb; ++kb) {
+      for (int kb = 0; kb < a.nkb; ++kb, ++b) {
+        if (kRowGroups && (b & (kPfABufs - 1)) != sel) continue;
+        const int s = b % kPfStages, ab = b & (kPfABufs - 1);
+        const uint32_t ph = (uint32_t)((b / kPfStages) & 1), pa = (uint32_t)((b / kPfABufs) & 1);
         if (!pf_wait(&full[s], ph, &s_abort, a.wait_limit) || !pf_wait(&aempty[ab], pa ^ 1u, &s_abort, a.wait_limit)) {
           ok = false;
           break;
@@ -519,22 +529,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc_fence_after();
         const uint32_t ta = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAcol + ab * kPfAcols);
         if constexpr (B == 16)
-          pf_bf16_quarter(cq, cst + s * kCodesBytes, ta, r);
+          pf_bf16_quarter(sel, cst + s * kCodesBytes, ta, r);
         else
-          pf_dequant<B, GPB>(cq, cst + s * kCodesBytes, reinterpret_cast<const uint32_t*>(sbst + s * kSbBytes), ta,
-                             r);
+          pf_dequant_row<B, GPB>(cst + s * kCodesBytes, reinterpret_cast<const uint32_t*>(sbst + s * kSbBytes), ta, r);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&afull[ab]);
-        if (++s == kPfStages) {
-          s = 0;
-          ph ^= 1u;
-        }
-        if (++ab == kPfABufs) {
-          ab = 0;
-          pa ^= 1u;
-        }
       }
       if (!ok) break;
     }
