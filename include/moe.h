@@ -226,18 +226,26 @@ moe_status moe_install_slots(void* pool, size_t slot_bytes, int32_t n_slots, con
                              const int32_t* slots, int32_t n, cudaStream_t side, cudaEvent_t done);
 
 /* Stages 1 + 2 + 3 of one decode token in one launch (the calls above would
- * take three): the routing of moe_route (strength L), the sort of moe_sort
- * without x_sorted, and moe_slot_lookup over the whole active list
- * (pass_begin 0, pass_len E) -- the same values in the same buffers, bit for
- * bit.  T must be 1 (else MOE_ERR_UNSUPPORTED: use the three calls).
- *   slot_table device int32 [E] (read for substitution and lookup); n_slots
- *   as moe_slot_lookup; ids, w, offsets, pairs, active, n_active as moe_route
- *   and moe_sort; slots, miss, n_miss, dev_err as moe_slot_lookup. */
+ * take three): the routing of moe_route_shared (strength L, n_shared 0..8
+ * shared experts of weight shared_w[0], or 1 when shared_w is NULL; with
+ * n_shared 0 that is moe_route), the sort of moe_sort without x_sorted, and
+ * moe_slot_lookup over the whole active list (pass_begin 0, pass_len
+ * E + n_shared) -- the same values in the same buffers, bit for bit.  d is
+ * the routed experts' description, as for moe_route_shared; the sort and
+ * lookup outputs are those of the widened layer (E + n_shared experts,
+ * k + n_shared per token).  T must be 1 (else MOE_ERR_UNSUPPORTED: use the
+ * three calls); n_shared outside 0..8 returns MOE_ERR_INVALID, and
+ * k + n_shared above 32 MOE_ERR_UNSUPPORTED (as moe_sort on that layer).
+ *   slot_table device int32 [E + n_shared] (the first E entries read for
+ *   substitution, every active entry for the lookup); n_slots as
+ *   moe_slot_lookup; ids, w, offsets, pairs, active, n_active as
+ *   moe_route_shared and moe_sort; slots, miss, n_miss, dev_err as
+ *   moe_slot_lookup. */
 moe_status moe_route_sort_lookup(const float* logits, int32_t T, const moe_layer_desc* d, float L,
-                                 const int32_t* slot_table, int32_t n_slots, int32_t* ids, float* w,
-                                 int32_t* offsets, int32_t* pairs, int32_t* active, int32_t* n_active,
-                                 int32_t* slots, int32_t* miss, int32_t* n_miss, int32_t* dev_err,
-                                 cudaStream_t stream);
+                                 const int32_t* slot_table, int32_t n_shared, const float* shared_w,
+                                 int32_t n_slots, int32_t* ids, float* w, int32_t* offsets, int32_t* pairs,
+                                 int32_t* active, int32_t* n_active, int32_t* slots, int32_t* miss,
+                                 int32_t* n_miss, int32_t* dev_err, cudaStream_t stream);
 
 /* Stages 4 + 5 for one pass.
  *   x          device bf16 [T, H]

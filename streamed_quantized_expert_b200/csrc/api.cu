@@ -187,20 +187,22 @@ moe_status moe_sort(const int32_t* ids, const uint16_t* x, int32_t T, const moe_
 }
 
 moe_status moe_route_sort_lookup(const float* logits, int32_t T, const moe_layer_desc* d, float L,
-                                 const int32_t* slot_table, int32_t n_slots, int32_t* ids, float* w,
-                                 int32_t* offsets, int32_t* pairs, int32_t* active, int32_t* n_active,
-                                 int32_t* slots, int32_t* miss, int32_t* n_miss, int32_t* dev_err,
-                                 cudaStream_t stream) {
+                                 const int32_t* slot_table, int32_t n_shared, const float* shared_w,
+                                 int32_t n_slots, int32_t* ids, float* w, int32_t* offsets, int32_t* pairs,
+                                 int32_t* active, int32_t* n_active, int32_t* slots, int32_t* miss,
+                                 int32_t* n_miss, int32_t* dev_err, cudaStream_t stream) {
   moe_status s = check_desc(d);
   if (s != MOE_OK) return s;
-  if (T < 0 || !(L >= 0.0f) || L > 1e30f || n_slots < 0) return MOE_ERR_INVALID;
+  if (T < 0 || !(L >= 0.0f) || L > 1e30f || n_slots < 0 || n_shared < 0 || n_shared > kMaxShared)
+    return MOE_ERR_INVALID;
   if (T == 0) return MOE_OK;
-  if (T != 1) return MOE_ERR_UNSUPPORTED;
+  if (T != 1 || d->k + n_shared > 32) return MOE_ERR_UNSUPPORTED;  // the widened layer, as moe_sort takes it
   if (!logits || !slot_table || !ids || !w || !offsets || !pairs || !active || !n_active || !slots || !miss ||
       !n_miss)
     return MOE_ERR_INVALID;
-  return cuda_status(launch_route_sort_lookup(logits, d->E, d->k, L, slot_table, n_slots, ids, w, offsets, pairs,
-                                              active, n_active, slots, miss, n_miss, dev_err, stream));
+  return cuda_status(launch_route_sort_lookup(logits, d->E, d->k, L, slot_table, n_shared, shared_w, n_slots, ids, w,
+                                              offsets, pairs, active, n_active, slots, miss, n_miss, dev_err,
+                                              stream));
 }
 
 moe_status moe_slot_lookup(const int32_t* slot_table, const int32_t* active, const int32_t* n_active,

@@ -154,9 +154,9 @@ moe_status decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc
   // experts always), it reads x sorted by expert
   uint16_t* xs =
       (b->x_sorted && moe_ffn_kernel_path(d, T, 1) == MOE_PATH_TC_PREFILL) ? b->x_sorted : nullptr;
-  // one token without shared experts or sorted x: routing, sort and lookup in one launch
-  const bool one = T == 1 && ns == 0 && !xs;
-  if (one && !(G && G->n > 0) && moe_cache_resident(cache, layer) >= E0) {
+  // one token without sorted x: routing, sort and lookup in one launch
+  const bool one = T == 1 && !xs;
+  if (one && ns == 0 && !(G && G->n > 0) && moe_cache_resident(cache, layer) >= E0) {
     // a fully resident layer: the FFN launch routes the token itself (the host needs none of it)
     const moe_status r = moe_route_expert_ffn(x, logits, T, d0, L, lc->pool, lc->n_slots, lc->table_dev, b->ids,
                                               b->w, b->offsets, b->pairs, active, n_active, b->slots, miss, n_miss,
@@ -165,8 +165,8 @@ moe_status decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc
   }
   moe_status s = MOE_OK;
   if (one) {
-    s = moe_route_sort_lookup(logits, T, d0, L, lc->table_dev, lc->n_slots, b->ids, b->w, b->offsets, b->pairs,
-                              active, n_active, b->slots, miss, n_miss, b->dev_err, stream);
+    s = moe_route_sort_lookup(logits, T, d0, L, lc->table_dev, ns, lc->shared_w, lc->n_slots, b->ids, b->w,
+                              b->offsets, b->pairs, active, n_active, b->slots, miss, n_miss, b->dev_err, stream);
     if (s != MOE_OK) return s;
   } else {
     s = ns ? moe_route_shared(logits, T, d0, L, lc->table_dev, ns, lc->shared_w, b->ids, b->w, stream)

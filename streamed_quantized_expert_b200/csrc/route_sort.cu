@@ -124,42 +124,44 @@ __global__ void __launch_bounds__(256) route_select_kernel(const float* __restri
                           (ns > 0 && sw) ? sw[t] : 1.0f);
 }
 
-// One decode token's stages 1-3 in one block: route (as route_select_kernel),
-// then the sort of its k pairs (distinct experts: the active list is the
-// routed experts ascending, pair j of rank r at position r) and the slot
-// lookup over the whole active list (as sort_small_kernel and lookup_kernel
-// write them for T = 1).
+// One decode token's stages 1-3 in one block: route (as route_select_kernel,
+// with ns shared experts E .. E + ns - 1 of weight sw after the top k), then
+// the sort of its k + ns pairs (distinct experts: the active list is the
+// routed experts ascending, then the shared ones; pair j of rank r sits at
+// position r) and the slot lookup over the whole active list (as
+// sort_small_kernel and lookup_kernel write them for T = 1).
 template <int NPT>
 __global__ void __launch_bounds__(256) route_sort_lookup_kernel(
-    const float* __restrict__ logits, int E, int k, float L, const int32_t* __restrict__ table, int n_slots,
-    int32_t* __restrict__ ids, float* __restrict__ w, int32_t* __restrict__ offsets, int32_t* __restrict__ pairs,
-    int32_t* __restrict__ active, int32_t* __restrict__ n_active, int32_t* __restrict__ slots,
-    int32_t* __restrict__ miss, int32_t* __restrict__ n_miss, int32_t* __restrict__ dev_err) {
-  __shared__ int s_sel[32];  // the routed experts, rank order
+    const float* __restrict__ logits, int E, int k, float L, const int32_t* __restrict__ table, int ns,
+    const float* __restrict__ sw, int n_slots, int32_t* __restrict__ ids, float* __restrict__ w,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ pairs, int32_t* __restrict__ active,
+    int32_t* __restrict__ n_active, int32_t* __restrict__ slots, int32_t* __restrict__ miss,
+    int32_t* __restrict__ n_miss, int32_t* __restrict__ dev_err) {
+  __shared__ int s_sel[32];  // the token's experts, rank order (k + ns <= 32)
   __shared__ int s_act[32];  // ascending
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, n = k + ns, Ew = E + ns;
   pdl_wait();
   pdl_launch_dependents();
-  route_select_token<NPT>(logits, E, k, L, table, ids, w, 0, 1.0f);
+  route_select_token<NPT>(logits, E, k, L, table, ids, w, ns, (ns > 0 && sw) ? sw[0] : 1.0f);
   __syncthreads();  // the block's own global writes of ids are visible to it
-  if (tid < k) s_sel[tid] = ids[tid];
+  if (tid < n) s_sel[tid] = ids[tid];
   __syncthreads();
-  if (tid < k) {
+  if (tid < n) {
     const int e = s_sel[tid];
     int r = 0;
-    for (int j = 0; j < k; ++j) r += s_sel[j] < e;
+    for (int j = 0; j < n; ++j) r += s_sel[j] < e;
     s_act[r] = e;
     active[r] = e;
     pairs[r] = tid;
   }
-  for (int e = tid; e <= E; e += 256) {
+  for (int e = tid; e <= Ew; e += 256) {
     int c = 0;
-    for (int j = 0; j < k; ++j) c += s_sel[j] < e;
+    for (int j = 0; j < n; ++j) c += s_sel[j] < e;
     offsets[e] = c;
   }
   __syncthreads();
-  if (tid < 32) {  // lookup: one lane per active expert (k <= 32)
-    const bool in = tid < k;
+  if (tid < 32) {  // lookup: one lane per active expert (k + ns <= 32)
+    const bool in = tid < n;
     const int e = in ? s_act[tid] : -1;
     const int sl = in ? table[e] : 0;
     if (in) slots[tid] = sl;
@@ -167,7 +169,7 @@ __global__ void __launch_bounds__(256) route_sort_lookup_kernel(
     const unsigned bal = __ballot_sync(0xffffffffu, in && sl < 0);
     if (in && sl < 0) miss[__popc(bal & ((1u << tid) - 1u))] = e;
     if (tid == 0) {
-      *n_active = k;
+      *n_active = n;
       *n_miss = __popc(bal);
     }
   }
@@ -375,15 +377,15 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, float L, cons
   return launch_pdl(kern, blocks, 256, 0, st, logits, T, E, k, L, table, ids, w, n_shared, shared_w);
 }
 
-cudaError_t launch_route_sort_lookup(const float* logits, int E, int k, float L, const int32_t* table, int n_slots,
-                                     int32_t* ids, float* w, int32_t* offsets, int32_t* pairs, int32_t* active,
-                                     int32_t* n_active, int32_t* slots, int32_t* miss, int32_t* n_miss,
-                                     int32_t* dev_err, cudaStream_t st) {
+cudaError_t launch_route_sort_lookup(const float* logits, int E, int k, float L, const int32_t* table, int ns,
+                                     const float* sw, int n_slots, int32_t* ids, float* w, int32_t* offsets,
+                                     int32_t* pairs, int32_t* active, int32_t* n_active, int32_t* slots,
+                                     int32_t* miss, int32_t* n_miss, int32_t* dev_err, cudaStream_t st) {
   const void* kb = E <= 256 ? reinterpret_cast<const void*>(route_sort_lookup_kernel<1>)
                    : E <= 512 ? reinterpret_cast<const void*>(route_sort_lookup_kernel<2>)
                               : reinterpret_cast<const void*>(route_sort_lookup_kernel<4>);
-  return launch_pdl(kb, 1, 256, 0, st, logits, E, k, L, table, n_slots, ids, w, offsets, pairs, active, n_active,
-                    slots, miss, n_miss, dev_err);
+  return launch_pdl(kb, 1, 256, 0, st, logits, E, k, L, table, ns, sw, n_slots, ids, w, offsets, pairs, active,
+                    n_active, slots, miss, n_miss, dev_err);
 }
 
 size_t sort_ws_bytes(int n, int E) { return n <= 1024 ? 0 : (size_t)((n + 1023) / 1024) * E * sizeof(int32_t); }

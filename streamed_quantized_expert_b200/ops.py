@@ -92,7 +92,7 @@ def lib():
             "moe_route_shared": (C.c_int, [P, i32, D, f32, P, i32, P, P, P, P]),
             "moe_sort": (C.c_int, [P, P, i32, D, P, P, P, P, P, P, sz, P]),
             "moe_slot_lookup": (C.c_int, [P, P, P, i32, i32, i32, P, P, P, P, P]),
-            "moe_route_sort_lookup": (C.c_int, [P, i32, D, f32, P, i32, P, P, P, P, P, P, P, P, P, P, P]),
+            "moe_route_sort_lookup": (C.c_int, [P, i32, D, f32, P, i32, P, i32, P, P, P, P, P, P, P, P, P, P, P]),
             "moe_route_expert_ffn": (C.c_int, [P, P, i32, D, f32, P, i32, P, P, P, P, P, P, P, P, P, P, P, P, sz, P,
                                                P]),
             "moe_install_slots": (C.c_int, [P, sz, i32, P, P, i32, P, P]),
@@ -221,12 +221,14 @@ def moe_sort(ids, x, T, d, offsets, pairs, active, n_active, x_sorted, ws, ws_by
 
 
 def moe_route_sort_lookup(logits, T, d, L, slot_table, n_slots, ids, w, offsets, pairs, active, n_active, slots,
-                          miss, n_miss, dev_err, stream=None) -> None:
-    """moe_route + moe_sort (no x_sorted) + moe_slot_lookup over the whole
-    active list for one token, in one launch (T must be 1)."""
-    _ck(lib().moe_route_sort_lookup(_ptr(logits), int(T), C.byref(d), float(L), _ptr(slot_table), int(n_slots),
-                                    _ptr(ids), _ptr(w), _ptr(offsets), _ptr(pairs), _ptr(active), _ptr(n_active),
-                                    _ptr(slots), _ptr(miss), _ptr(n_miss), _ptr(dev_err), _stream(stream)),
+                          miss, n_miss, dev_err, stream=None, n_shared=0, shared_w=None) -> None:
+    """moe_route_shared (moe_route when n_shared is 0) + moe_sort (no
+    x_sorted) + moe_slot_lookup over the whole active list for one token, in
+    one launch (T must be 1; d the routed experts' description)."""
+    _ck(lib().moe_route_sort_lookup(_ptr(logits), int(T), C.byref(d), float(L), _ptr(slot_table), int(n_shared),
+                                    _ptr(shared_w), int(n_slots), _ptr(ids), _ptr(w), _ptr(offsets), _ptr(pairs),
+                                    _ptr(active), _ptr(n_active), _ptr(slots), _ptr(miss), _ptr(n_miss),
+                                    _ptr(dev_err), _stream(stream)),
         "moe_route_sort_lookup")
 
 

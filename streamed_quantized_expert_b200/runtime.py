@@ -273,8 +273,8 @@ class Streamer:
     def _decode_launches(self, layer: int, T: int, full: bool, n_installed: int, guessing: bool = False) -> int:
         d = self.layers[layer].desc
         tc = self.uses_tc(layer, T)
-        if T == 1 and not self.ns and not tc:
-            if full and not guessing and d.E <= 1024 and self._ffn_launches(layer, T, self.Ew) == 1:
+        if T == 1 and not tc:
+            if not self.ns and full and not guessing and d.E <= 1024 and self._ffn_launches(layer, T, self.Ew) == 1:
                 return 1  # moe_route_expert_ffn: every stage in the FFN launch
             n = 1  # moe_route_sort_lookup
         else:
