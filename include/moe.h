@@ -460,7 +460,7 @@ typedef struct {
   int32_t* offsets;    /* device int32 [E+1] */
   int32_t* pairs;      /* device int32 [max_tokens*k] */
   int32_t* meta;       /* device int32 [2+2E]: n_active, n_miss, active[E], miss[E] */
-  int32_t* meta_host;  /* pinned host int32 [2+2E] */
+  int32_t* meta_host;  /* pinned host int32 [2+2E] (written by the device when it maps it) */
   int32_t* slots;      /* device int32 [E] */
   int32_t* dev_err;    /* device int32 [1] */
   void* ws;            /* device workspace */
@@ -491,7 +491,12 @@ typedef struct {
  * per expert; a fully resident layer never synchronises with the host):
  *   moe_route (L) -> moe_sort (sorting x into b->x_sorted beyond the fused range and
  *   b->x_sorted is given) -> if the layer is not fully resident in `cache`:
- *   moe_slot_lookup, copy n_active/active to meta_host, synchronise `stream`,
+ *   moe_slot_lookup, copy n_active/active to meta_host, synchronise `stream`
+ *   (for one token without guesses, when the device addresses meta_host at
+ *   the same pointer -- page-locked memory from cudaHostAlloc/cudaMallocHost
+ *   -- the one-launch routing kernel writes them there itself, then a
+ *   sequence word to meta_host[1], and the host waits for that word: bounded,
+ *   MOE_ERR_TIMEOUT after 5 s, no copy back and no stream synchronisation),
  *   moe_cache_step, moe_install_slots on `side`, upload the table, record
  *   `installed` on `side` and make `stream` wait on it -> one pass of
  *   moe_expert_ffn over every active expert, writing y.  When experts are

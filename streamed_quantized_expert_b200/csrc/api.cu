@@ -186,11 +186,15 @@ moe_status moe_sort(const int32_t* ids, const uint16_t* x, int32_t T, const moe_
                                  stream));
 }
 
-moe_status moe_route_sort_lookup(const float* logits, int32_t T, const moe_layer_desc* d, float L,
-                                 const int32_t* slot_table, int32_t n_shared, const float* shared_w,
-                                 int32_t n_slots, int32_t* ids, float* w, int32_t* offsets, int32_t* pairs,
-                                 int32_t* active, int32_t* n_active, int32_t* slots, int32_t* miss,
-                                 int32_t* n_miss, int32_t* dev_err, cudaStream_t stream) {
+// moe_route_sort_lookup that also publishes n_active and the active list to
+// host_meta (page-locked host memory the device addresses at the same
+// pointer; NULL: not at all) and then seq to host_meta[1] (used by the
+// decode driver in place of a copy back and a stream synchronisation).
+__attribute__((visibility("hidden"))) moe_status moe_internal_route_sort_lookup(
+    const float* logits, int32_t T, const moe_layer_desc* d, float L, const int32_t* slot_table, int32_t n_shared,
+    const float* shared_w, int32_t n_slots, int32_t* ids, float* w, int32_t* offsets, int32_t* pairs,
+    int32_t* active, int32_t* n_active, int32_t* slots, int32_t* miss, int32_t* n_miss, int32_t* dev_err,
+    cudaStream_t stream, int32_t* host_meta, int32_t seq) {
   moe_status s = check_desc(d);
   if (s != MOE_OK) return s;
   if (T < 0 || !(L >= 0.0f) || L > 1e30f || n_slots < 0 || n_shared < 0 || n_shared > kMaxShared)
@@ -202,7 +206,16 @@ moe_status moe_route_sort_lookup(const float* logits, int32_t T, const moe_layer
     return MOE_ERR_INVALID;
   return cuda_status(launch_route_sort_lookup(logits, d->E, d->k, L, slot_table, n_shared, shared_w, n_slots, ids, w,
                                               offsets, pairs, active, n_active, slots, miss, n_miss, dev_err,
-                                              stream));
+                                              stream, host_meta, seq));
+}
+
+moe_status moe_route_sort_lookup(const float* logits, int32_t T, const moe_layer_desc* d, float L,
+                                 const int32_t* slot_table, int32_t n_shared, const float* shared_w,
+                                 int32_t n_slots, int32_t* ids, float* w, int32_t* offsets, int32_t* pairs,
+                                 int32_t* active, int32_t* n_active, int32_t* slots, int32_t* miss,
+                                 int32_t* n_miss, int32_t* dev_err, cudaStream_t stream) {
+  return moe_internal_route_sort_lookup(logits, T, d, L, slot_table, n_shared, shared_w, n_slots, ids, w, offsets,
+                                        pairs, active, n_active, slots, miss, n_miss, dev_err, stream, nullptr, 0);
 }
 
 moe_status moe_slot_lookup(const int32_t* slot_table, const int32_t* active, const int32_t* n_active,

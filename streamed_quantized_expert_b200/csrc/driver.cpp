@@ -1,6 +1,8 @@
 // Host driver of one decode layer: the whole five-stage sequence in native
 // code, so the per-layer host cost is the launches and (when the layer is not
-// fully resident) one small device->host copy and its synchronisation.
+// fully resident) one small device->host copy and its synchronisation -- or,
+// for one token, a wait on a word the routing kernel writes to host memory
+// after the active list itself.
 //
 //   route -> sort -> [lookup -> misses to host -> LRU step -> pinned installs on
 //   the side stream + table upload -> FFN of the resident experts (writes y),
@@ -22,6 +24,8 @@
 // landed batches are entered into the table (an event query, never a wait);
 // batches still in flight are skipped and stay reserved.
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <cstring>
 #include <vector>
 
@@ -36,6 +40,11 @@ extern "C" moe_status moe_internal_expert_ffn(const uint16_t* x, int32_t T, cons
                                               const uint16_t* x_sorted, int32_t pass_begin, int32_t pass_len,
                                               float* y_accum, void* ws, size_t ws_bytes, int32_t* dev_err,
                                               cudaStream_t stream, int overwrite);
+extern "C" moe_status moe_internal_route_sort_lookup(
+    const float* logits, int32_t T, const moe_layer_desc* d, float L, const int32_t* slot_table, int32_t n_shared,
+    const float* shared_w, int32_t n_slots, int32_t* ids, float* w, int32_t* offsets, int32_t* pairs,
+    int32_t* active, int32_t* n_active, int32_t* slots, int32_t* miss, int32_t* n_miss, int32_t* dev_err,
+    cudaStream_t stream, int32_t* host_meta, int32_t seq);
 
 struct moe_prefetch {
   struct Batch {
@@ -49,6 +58,52 @@ struct moe_prefetch {
 };
 
 namespace {
+
+// Whether the device addresses host memory p at the same pointer (page-locked
+// memory from cudaHostAlloc / cudaMallocHost under unified addressing).
+// Checked on every call: a cached answer could outlive the allocation.
+bool device_maps_host(const void* p) {
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost && a.devicePointer == p;
+}
+
+// Sequence words of the one-token routing kernel's host writes: distinct
+// from every count the copy-back path leaves in the same word (<= 1032).
+int32_t next_host_seq() {
+  static std::atomic<uint32_t> n{0};
+  return (int32_t)(0x40000000u | (n.fetch_add(1, std::memory_order_relaxed) & 0x3fffffffu));
+}
+
+// Wait until the routing kernel has published the active list to host
+// memory (host_meta[1] == seq).  Bounded: the stream's state is polled every
+// 1024 reads, and a stream that has failed or finished without the word, or
+// a wait past kHostWaitSeconds, ends it with an error.
+constexpr double kHostWaitSeconds = 5.0;
+moe_status wait_host_seq(const int32_t* host_meta, int32_t seq, cudaStream_t stream) {
+  const volatile int32_t* word = host_meta + 1;
+  const auto t0 = std::chrono::steady_clock::now();
+  for (uint32_t i = 1; *word != seq; ++i) {
+    if ((i & 1023u) == 0) {
+      const cudaError_t e = cudaStreamQuery(stream);
+      if (e == cudaSuccess) {
+        if (*word == seq) break;
+        return MOE_ERR_CUDA;  // the stream drained, the word never came
+      }
+      if (e != cudaErrorNotReady) return MOE_ERR_CUDA;
+      if (std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count() > kHostWaitSeconds)
+        return MOE_ERR_TIMEOUT;
+    }
+#if defined(__x86_64__)
+    __builtin_ia32_pause();
+#endif
+  }
+  std::atomic_thread_fence(std::memory_order_acquire);
+  return MOE_OK;
+}
 
 struct Guess {
   moe_prefetch* pf;
@@ -164,9 +219,20 @@ moe_status decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc
     if (r != MOE_ERR_UNSUPPORTED) return r;
   }
   moe_status s = MOE_OK;
+  const bool guessing = G && G->n > 0;
+  const bool resident = moe_cache_resident(cache, layer) >= E0;
+  // the host needs the active list: for one token the routing kernel writes it
+  // straight to host memory, with no copy back or stream synchronisation
+  int32_t* host_meta = nullptr;
+  int32_t seq = 0;
+  if (one && !resident && !guessing && device_maps_host(b->meta_host)) {
+    host_meta = b->meta_host;
+    seq = next_host_seq();
+  }
   if (one) {
-    s = moe_route_sort_lookup(logits, T, d0, L, lc->table_dev, ns, lc->shared_w, lc->n_slots, b->ids, b->w,
-                              b->offsets, b->pairs, active, n_active, b->slots, miss, n_miss, b->dev_err, stream);
+    s = moe_internal_route_sort_lookup(logits, T, d0, L, lc->table_dev, ns, lc->shared_w, lc->n_slots, b->ids,
+                                       b->w, b->offsets, b->pairs, active, n_active, b->slots, miss, n_miss,
+                                       b->dev_err, stream, host_meta, seq);
     if (s != MOE_OK) return s;
   } else {
     s = ns ? moe_route_shared(logits, T, d0, L, lc->table_dev, ns, lc->shared_w, b->ids, b->w, stream)
@@ -177,7 +243,6 @@ moe_status decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc
     if (s != MOE_OK) return s;
   }
   // the guessed layers' top-k, on the same synchronisation as the layer's own lookup
-  const bool guessing = G && G->n > 0;
   if (guessing) {
     for (int32_t gi = 0; gi < G->n; ++gi) {
       const moe_guess& g = G->g[gi];
@@ -189,7 +254,6 @@ moe_status decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc
         return MOE_ERR_CUDA;
     }
   }
-  const bool resident = moe_cache_resident(cache, layer) >= E0;
   if (resident && guessing) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
     s = start_guesses(*G, cache, T);
@@ -201,10 +265,15 @@ moe_status decode_layer(moe_cache* cache, int32_t layer, const moe_layer_ctx* lc
                           stream);
       if (s != MOE_OK) return s;
     }
-    if (cudaMemcpyAsync(b->meta_host, b->meta, sizeof(int32_t) * (size_t)(2 + E), cudaMemcpyDeviceToHost,
-                        stream) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+    if (host_meta) {
+      s = wait_host_seq(host_meta, seq, stream);
+      if (s != MOE_OK) return s;
+    } else {
+      if (cudaMemcpyAsync(b->meta_host, b->meta, sizeof(int32_t) * (size_t)(2 + E), cudaMemcpyDeviceToHost,
+                          stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+    }
     const int32_t na = b->meta_host[0];
     if (na < ns || na > E) return MOE_ERR_INVALID;
     thread_local std::vector<int32_t> out_e, out_s;

@@ -104,7 +104,8 @@ cudaError_t launch_lookup(const int32_t* table, const int32_t* active, const int
 cudaError_t launch_route_sort_lookup(const float* logits, int E, int k, float L, const int32_t* table, int ns,
                                      const float* sw, int n_slots, int32_t* ids, float* w, int32_t* offsets,
                                      int32_t* pairs, int32_t* active, int32_t* n_active, int32_t* slots,
-                                     int32_t* miss, int32_t* n_miss, int32_t* dev_err, cudaStream_t st);
+                                     int32_t* miss, int32_t* n_miss, int32_t* dev_err, cudaStream_t st,
+                                     int32_t* host_meta = nullptr, int32_t seq = 0);
 cudaError_t launch_exp(const float* x, int64_t n, float* out, cudaStream_t st);
 cudaError_t launch_quantize(const float* w, int rows, int K, int g, int b, int gu_I, uint8_t* q, cudaStream_t st);
 cudaError_t launch_dequant_slot(const uint8_t* slot, const moe_layer_desc& d, const Layout& L, float* out32,

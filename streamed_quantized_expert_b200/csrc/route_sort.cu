@@ -129,14 +129,18 @@ __global__ void __launch_bounds__(256) route_select_kernel(const float* __restri
 // the sort of its k + ns pairs (distinct experts: the active list is the
 // routed experts ascending, then the shared ones; pair j of rank r sits at
 // position r) and the slot lookup over the whole active list (as
-// sort_small_kernel and lookup_kernel write them for T = 1).
+// sort_small_kernel and lookup_kernel write them for T = 1).  With host_meta
+// (page-locked host memory the device can address), warp 1 also writes
+// n_active to host_meta[0] and the active list to host_meta[2 ..], then, once
+// those writes are visible system-wide, seq to host_meta[1]: the host waits
+// for seq there instead of copying the list back and synchronising.
 template <int NPT>
 __global__ void __launch_bounds__(256) route_sort_lookup_kernel(
     const float* __restrict__ logits, int E, int k, float L, const int32_t* __restrict__ table, int ns,
     const float* __restrict__ sw, int n_slots, int32_t* __restrict__ ids, float* __restrict__ w,
     int32_t* __restrict__ offsets, int32_t* __restrict__ pairs, int32_t* __restrict__ active,
     int32_t* __restrict__ n_active, int32_t* __restrict__ slots, int32_t* __restrict__ miss,
-    int32_t* __restrict__ n_miss, int32_t* __restrict__ dev_err) {
+    int32_t* __restrict__ n_miss, int32_t* __restrict__ dev_err, int32_t* host_meta, int32_t seq) {
   __shared__ int s_sel[32];  // the token's experts, rank order (k + ns <= 32)
   __shared__ int s_act[32];  // ascending
   const int tid = threadIdx.x, n = k + ns, Ew = E + ns;
@@ -172,6 +176,13 @@ __global__ void __launch_bounds__(256) route_sort_lookup_kernel(
       *n_active = n;
       *n_miss = __popc(bal);
     }
+  } else if (tid < 64 && host_meta) {
+    const int lane = tid - 32;
+    if (lane < n) host_meta[2 + lane] = s_act[lane];
+    if (lane == 0) host_meta[0] = n;
+    __threadfence_system();
+    __syncwarp();
+    if (lane == 0) *reinterpret_cast<volatile int32_t*>(host_meta + 1) = seq;
   }
 }
 
@@ -380,12 +391,13 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, float L, cons
 cudaError_t launch_route_sort_lookup(const float* logits, int E, int k, float L, const int32_t* table, int ns,
                                      const float* sw, int n_slots, int32_t* ids, float* w, int32_t* offsets,
                                      int32_t* pairs, int32_t* active, int32_t* n_active, int32_t* slots,
-                                     int32_t* miss, int32_t* n_miss, int32_t* dev_err, cudaStream_t st) {
+                                     int32_t* miss, int32_t* n_miss, int32_t* dev_err, cudaStream_t st,
+                                     int32_t* host_meta, int32_t seq) {
   const void* kb = E <= 256 ? reinterpret_cast<const void*>(route_sort_lookup_kernel<1>)
                    : E <= 512 ? reinterpret_cast<const void*>(route_sort_lookup_kernel<2>)
                               : reinterpret_cast<const void*>(route_sort_lookup_kernel<4>);
   return launch_pdl(kb, 1, 256, 0, st, logits, E, k, L, table, ns, sw, n_slots, ids, w, offsets, pairs, active,
-                    n_active, slots, miss, n_miss, dev_err);
+                    n_active, slots, miss, n_miss, dev_err, host_meta, seq);
 }
 
 size_t sort_ws_bytes(int n, int E) { return n <= 1024 ? 0 : (size_t)((n + 1023) / 1024) * E * sizeof(int32_t); }

@@ -50,10 +50,18 @@ def initial_fill(st, seed, S):
     return placed
 
 
-def test_decode_with_installs(orc):
+@pytest.mark.parametrize("meta_host", ["pinned", "pageable"])
+def test_decode_with_installs(orc, meta_host):
+    """pinned: the one-token routing kernel writes the active list to the
+    host buffer and the driver waits for its sequence word; pageable (memory
+    the device cannot address): the driver copies the list back and
+    synchronises instead."""
     E, k, H, I, g, S = 512, 10, 2048, 512, 64, 192
     specs, host_slots = make(orc, 2, E, k, H, I, g, [(3, 3), (3, 3)], S, R=12)
     st = Streamer(specs, S, max_tokens=1)
+    if meta_host == "pageable":
+        st.meta_pin = torch.zeros(st.meta_pin.numel(), dtype=torch.int32)
+        st._bufs.meta_host = st.meta_pin.data_ptr()
     placed = initial_fill(st, 0, S)
     models = []
     for l in range(2):
