@@ -64,6 +64,17 @@ def test_argument_checks(lib):
         ops.moe_expert_ffn(1 << 20, 4, d, 1 << 24, 8, 1 << 21, 1 << 21, 1 << 21, 1 << 21, 1 << 21, 1 << 21,
                            1 << 21, None, 0, 8, 1 << 21, 1 << 24, 16, None)
     assert ei.value.status == ops.MOE_ERR_CAPACITY
+    p = 1 << 21  # checked before any launch: no device memory is touched
+    one = (p, p, p, p, p, p, p, p, p, p)
+    with pytest.raises(ops.MoeError) as ei:  # at most 8 shared experts
+        ops.moe_route_sort_lookup(p, 1, d, 0.0, p, 8, *one, n_shared=9)
+    assert ei.value.status == ops.MOE_ERR_INVALID
+    with pytest.raises(ops.MoeError) as ei:  # k + n_shared above 32
+        ops.moe_route_sort_lookup(p, 1, ops.desc(64, 30, 64, 32, 32, 4), 0.0, p, 64, *one, n_shared=3)
+    assert ei.value.status == ops.MOE_ERR_UNSUPPORTED
+    with pytest.raises(ops.MoeError) as ei:  # one token only
+        ops.moe_route_sort_lookup(p, 2, d, 0.0, p, 8, *one)
+    assert ei.value.status == ops.MOE_ERR_UNSUPPORTED
     assert ops.status_string(ops.MOE_ERR_TIMEOUT) == "device wait timed out"
 
 
